@@ -1,0 +1,276 @@
+"""Plain, slow float64 CPU oracle of CLHA calibration (collect -> aggregate -> GPTQ).
+
+TEST INFRASTRUCTURE ONLY: the tests, the package smoke check and the bench's CPU-baseline and
+reference legs call this module; the CUDA library never does, and it shares no code with it.
+
+Sources. "CLHA page" below is the technical summary "CLHA – Cross-Layer Hessian Aggregation voor
+het kwantiseren van Weight-Shared Mixture-of-Experts Transformers" (gist.science, rs-10133806),
+whose section 2 defines the method:
+  §2.1   the shared-weight loss L(Wq) = sum_i alpha_i tr[(Wq - W) H_i (Wq - W)^T], alpha_i the share of
+         tokens of layer i, and Proposition 1: minimising it is GPTQ with H_comb = sum_i alpha_i H_i;
+  §2.2   the three phases: (1) collection of per-layer Hessians and token counts per active expert,
+         (2) aggregation with alpha = n_a/(n_a+n_b) ("rt") or alpha = 0.5 ("eq"),
+         (3) standard GPTQ column-sequential updates with H_comb;
+  §2.3   CLHA-MP: b+1 bits for always-active shared experts;
+  §2.4   layer-aware collection (one accumulator per (layer, expert), never mixed).
+GPTQ itself is the published algorithm of Frantar, Ashkboos, Hoefler and Alistarh (2022), "GPTQ:
+Accurate Post-Training Quantization for Generative Pre-trained Transformers", Algorithm 1; it is
+restated here from its mathematics (damped Hessian, upper Cholesky factor of H^-1, column-by-column
+rounding with the error fed forward along that factor's row).
+
+Readings where the pages are silent (each also listed in the design notes):
+  * H_l = (2/n_l) sum x x^T over the tokens routed to the expert in layer l; tokens are not weighted
+    by their gate probability.
+  * top-k ties go to the lower expert index; an expert's token list is in ascending token order.
+  * the down-projection input is h = SiLU(x Wg^T) * (x Wu^T) of the full-precision weights, rounded
+    to bfloat16 (round to nearest, ties to even) because that is the dtype h is stored in.
+  * damping lambda = damp_frac * mean(diag H_comb) of the undamped aggregate; H_d = H_comb + lambda I.
+  * the grid of a group is min-max asymmetric over the group's current (error-updated) values with 0
+    included; an all-zero group uses [-1, 1].
+  * the grid and the integer code are decided in binary32 (float32), the precision the kernel decides
+    them in, so both sides take each rounding decision in the same precision; the error propagation
+    around those decisions stays float64.
+  * columns are quantized in natural order (no activation reordering).
+  * a layer with no tokens contributes a zero Hessian; an expert with no tokens in any layer is an
+    error (there is nothing to calibrate on).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "route_topk", "expert_tokens", "gram", "hessian", "bf16_round", "silu", "ffn_act",
+    "aggregate", "factor", "grid_fp32", "quantize_fp32", "gptq", "loss",
+    "calibrate_dense", "calibrate_moe_group",
+]
+
+
+# ----------------------------------------------------------------------------------- phase 1
+def route_topk(logits, k: int):
+    """Top-k routing of each token (CLHA page §2.2 (1): tokens reach their active experts).
+
+    Returns ids [n, k] int32 (experts in descending logit order; ties -> lower expert index) and
+    counts [E] int64 (tokens each expert receives).
+    """
+    lg = np.asarray(logits, dtype=np.float64)
+    n, E = lg.shape
+    if not (0 < k <= E):
+        raise ValueError("k must be in 1..E")
+    order = np.argsort(-lg, axis=1, kind="stable")
+    ids = order[:, :k].astype(np.int32)
+    counts = np.bincount(ids.ravel(), minlength=E).astype(np.int64)
+    return ids, counts
+
+
+def expert_tokens(ids, E: int):
+    """Per expert, the ascending list of token indices routed to it."""
+    ids = np.asarray(ids)
+    return [np.nonzero((ids == e).any(axis=1))[0] for e in range(E)]
+
+
+def gram(X):
+    """S = sum over tokens of x x^T, in float64 from the exact stored values (CLHA page §2.2 (1))."""
+    X = np.asarray(X, dtype=np.float64)
+    return X.T @ X
+
+
+def hessian(S, n: int):
+    """H = (2/n) S; a layer without tokens contributes a zero Hessian."""
+    S = np.asarray(S, dtype=np.float64)
+    if n == 0:
+        return np.zeros_like(S)
+    return (2.0 / n) * S
+
+
+def bf16_round(v):
+    """Round float64 values to the nearest bfloat16 value (8 significant bits), ties to even."""
+    v = np.asarray(v, dtype=np.float64)
+    _, ex = np.frexp(v)
+    ulp_exp = np.maximum(ex - 8, -133)           # bfloat16 spacing; never finer than its subnormals
+    r = np.ldexp(np.rint(np.ldexp(v, -ulp_exp)), ulp_exp)
+    big = np.abs(r) >= 2.0 ** 128
+    if np.any(big):
+        r = np.where(big, np.copysign(np.inf, v), r)
+    return r
+
+
+def silu(a):
+    """SiLU(a) = a * sigmoid(a), evaluated without overflow."""
+    a = np.asarray(a, dtype=np.float64)
+    out = np.empty_like(a)
+    pos = a >= 0
+    out[pos] = a[pos] / (1.0 + np.exp(-a[pos]))
+    ea = np.exp(a[~pos])
+    out[~pos] = a[~pos] * ea / (1.0 + ea)
+    return out
+
+
+def ffn_act(Xe, Wg, Wu):
+    """Input of an expert's down projection, h = SiLU(x Wg^T) * (x Wu^T), rounded to bfloat16."""
+    Xe = np.asarray(Xe, dtype=np.float64)
+    a = Xe @ np.asarray(Wg, dtype=np.float64).T
+    b = Xe @ np.asarray(Wu, dtype=np.float64).T
+    return bf16_round(silu(a) * b)
+
+
+# ----------------------------------------------------------------------------------- phase 2
+def aggregate(S_list, n_list, mode: str = "rt", alpha=None, damp_frac: float = 0.01):
+    """Cross-layer aggregation (CLHA page §2.1 Proposition 1, §2.2 (2)) and damping.
+
+    mode "rt": alpha_i = n_i / sum_j n_j; "eq": alpha_i = 1/L (0.5 for a pair);
+    "explicit": alpha given (e.g. (1, 0) for per-layer calibration on the first layer only).
+    Returns dict(alpha, H_comb, lam, H_d) with H_comb = sum_i alpha_i (2/n_i) S_i,
+    lam = damp_frac * mean(diag H_comb), H_d = H_comb + lam I.
+    """
+    L = len(S_list)
+    n = np.asarray(n_list, dtype=np.int64)
+    if n.sum() == 0:
+        raise ValueError("no tokens in any layer")
+    if mode == "rt":
+        a = n / n.sum()
+    elif mode == "eq":
+        a = np.full(L, 1.0 / L)
+    elif mode == "explicit":
+        a = np.asarray(alpha, dtype=np.float64)
+        if a.shape != (L,):
+            raise ValueError("alpha must have one entry per layer")
+    else:
+        raise ValueError(mode)
+    H_comb = np.zeros_like(np.asarray(S_list[0], dtype=np.float64))
+    for ai, Si, ni in zip(a, S_list, n):
+        H_comb += ai * hessian(Si, int(ni))
+    lam = damp_frac * float(np.mean(np.diag(H_comb)))
+    H_d = H_comb + lam * np.eye(H_comb.shape[0])
+    return {"alpha": a, "H_comb": H_comb, "lam": lam, "H_d": H_d}
+
+
+# ----------------------------------------------------------------------------------- phase 3
+def factor(H_d):
+    """U: the upper-triangular Cholesky factor of H_d^-1 (H_d^-1 = U^T U), by the plain route:
+    H_d = L L^T, H_d^-1 = L^-T L^-1, then the Cholesky factorisation of that inverse."""
+    H_d = np.asarray(H_d, dtype=np.float64)
+    L = np.linalg.cholesky(H_d)
+    Linv = np.linalg.inv(L)
+    Hinv = Linv.T @ Linv
+    Hinv = 0.5 * (Hinv + Hinv.T)
+    return np.linalg.cholesky(Hinv).T
+
+
+def grid_fp32(wgrp, bits: int):
+    """Asymmetric min-max grid of each row of a group, decided in binary32.
+
+    wgrp: [rows, g] current values. Returns (s, z) float32 [rows]: step s = (xmax - xmin)/(2^b - 1)
+    and integer zero point z = round(-xmin / s), with xmin <= 0 <= xmax (0 always on the grid) and
+    [-1, 1] for an all-zero group.
+    """
+    w = np.asarray(wgrp, dtype=np.float64).astype(np.float32)
+    maxq = np.float32(2 ** bits - 1)
+    xmin = np.minimum(np.float32(0), w.min(axis=1))
+    xmax = np.maximum(np.float32(0), w.max(axis=1))
+    dead = (xmin == 0) & (xmax == 0)
+    xmin = np.where(dead, np.float32(-1), xmin).astype(np.float32)
+    xmax = np.where(dead, np.float32(1), xmax).astype(np.float32)
+    s = ((xmax - xmin).astype(np.float32) / maxq).astype(np.float32)
+    z = np.rint((-xmin).astype(np.float32) / s).astype(np.float32)
+    return s, z
+
+
+def quantize_fp32(w, s, z, bits: int):
+    """Code q = clamp(round(w/s) + z, 0, 2^b - 1) and value s (q - z), both in binary32."""
+    w32 = np.asarray(w, dtype=np.float64).astype(np.float32)
+    maxq = np.float32(2 ** bits - 1)
+    q = np.clip(np.rint((w32 / s).astype(np.float32)) + z, np.float32(0), maxq).astype(np.float32)
+    wq = (s * (q - z).astype(np.float32)).astype(np.float32)
+    return q, wq
+
+
+def gptq(W, U, bits: int, group: int):
+    """GPTQ column-sequential quantization of W [d_out, d_in] with U = chol_upper(H_d^-1).
+
+    Unblocked form (lazy blocks change only the order of the same float64 updates). For each column
+    j in natural order: at a group start, fix each row's grid from the current values of that group;
+    quantize the current value; e = (w_j - what_j) / U_jj; subtract e * U[j, k] from every later
+    column k of the row. Rows are independent and are processed together.
+    Returns codes uint8 [d_out, d_in], scales float32 and zeros uint8 [d_out, d_in/group],
+    W_hat float32 [d_out, d_in].
+    """
+    Wc = np.array(W, dtype=np.float64, copy=True)
+    U = np.asarray(U, dtype=np.float64)
+    d_out, d_in = Wc.shape
+    if d_in % group:
+        raise ValueError("d_in must be a multiple of the group size")
+    codes = np.zeros((d_out, d_in), np.uint8)
+    scales = np.zeros((d_out, d_in // group), np.float32)
+    zeros = np.zeros((d_out, d_in // group), np.uint8)
+    W_hat = np.zeros((d_out, d_in), np.float32)
+    s = z = None
+    for j in range(d_in):
+        if j % group == 0:
+            s, z = grid_fp32(Wc[:, j:j + group], bits)
+            scales[:, j // group] = s
+            zeros[:, j // group] = z.astype(np.uint8)
+        q, wq = quantize_fp32(Wc[:, j], s, z, bits)
+        codes[:, j] = q.astype(np.uint8)
+        W_hat[:, j] = wq
+        err = (Wc[:, j] - wq.astype(np.float64)) / U[j, j]
+        Wc[:, j + 1:] -= np.outer(err, U[j, j + 1:])
+    return codes, scales, zeros, W_hat
+
+
+def loss(W, W_hat, H):
+    """tr[(W_hat - W) H (W_hat - W)^T] (CLHA page §2.1, one term of the shared-weight loss)."""
+    D = np.asarray(W_hat, dtype=np.float64) - np.asarray(W, dtype=np.float64)
+    return float(np.sum((D @ np.asarray(H, dtype=np.float64)) * D))
+
+
+# ----------------------------------------------------------------------------------- pipelines
+def calibrate_dense(W, X_list, bits: int, group: int = 128, mode: str = "rt", alpha=None,
+                    damp_frac: float = 0.01):
+    """CLHA for one weight W [d_out, d_in] shared by the layers whose inputs are X_list."""
+    S = [gram(X) for X in X_list]
+    n = [int(np.asarray(X).shape[0]) for X in X_list]
+    agg = aggregate(S, n, mode, alpha, damp_frac)
+    U = factor(agg["H_d"])
+    codes, scales, zeros, W_hat = gptq(W, U, bits, group)
+    return {"S": S, "n": n, **agg, "U": U, "codes": codes, "scales": scales, "zeros": zeros,
+            "W_hat": W_hat, "loss": loss(W, W_hat, agg["H_comb"]),
+            "layer_loss": [loss(W, W_hat, hessian(Si, ni)) for Si, ni in zip(S, n)]}
+
+
+def calibrate_moe_group(X_list, logits_list, k: int, routed, shared=(), experts=None,
+                        bits_routed: int = 2, bits_shared: int = 3, group: int = 128,
+                        mode: str = "rt", damp_frac: float = 0.01):
+    """CLHA on one group of layers sharing routed experts `routed` [(Wg, Wu, Wd)] and always-active
+    experts `shared` (CLHA page §2.2 phases 1-3, §2.3 mixed precision, §2.4 per-layer accumulators).
+
+    experts: which routed experts to calibrate (default all); shared ones are always calibrated.
+    Returns per-layer routing and, per expert key ("r", e) / ("s", e), counts, alphas and the GPTQ
+    results of gate/up (input Hessian over x) and down (input Hessian over h).
+    """
+    E = len(routed)
+    if experts is None:
+        experts = range(E)
+    routes = [route_topk(lg, k) for lg in logits_list]
+    toks = [expert_tokens(ids, E) for ids, _ in routes]
+    out = {"routes": routes, "experts": {}}
+    jobs = [(("r", e), routed[e], [t[e] for t in toks], bits_routed) for e in experts]
+    jobs += [(("s", i), w, [np.arange(np.asarray(X).shape[0]) for X in X_list], bits_shared)
+             for i, w in enumerate(shared)]
+    for key, (Wg, Wu, Wd), tok_l, bits in jobs:
+        Xe = [np.asarray(X, dtype=np.float64)[t] for X, t in zip(X_list, tok_l)]
+        he = [ffn_act(x, Wg, Wu) for x in Xe]
+        n = [len(t) for t in tok_l]
+        res = {"n": n}
+        for kind, inputs, mats in (("in", Xe, (("gate", Wg), ("up", Wu))), ("down", he, (("down", Wd),))):
+            S = [gram(x) for x in inputs]
+            agg = aggregate(S, n, mode, None, damp_frac)
+            U = factor(agg["H_d"])
+            res[kind] = {"S": S, **agg, "U": U}
+            for name, Wm in mats:
+                codes, scales, zeros, W_hat = gptq(Wm, U, bits, group)
+                res[name] = {"codes": codes, "scales": scales, "zeros": zeros, "W_hat": W_hat,
+                             "loss": loss(Wm, W_hat, agg["H_comb"])}
+        res["loss"] = res["gate"]["loss"] + res["up"]["loss"] + res["down"]["loss"]
+        res["h"] = he
+        out["experts"][key] = res
+    return out
