@@ -1,0 +1,380 @@
+"""Throughput of CLHA calibration on B200: expert weight columns quantized per second, end to end.
+
+One step = the whole hot path on one weight-sharing MoE layer pair (E=16 routed experts, top-2,
+d_model 1024, d_ff 512, 8192 tokens per layer, 3-bit): for both layers route -> gather -> Hessians of
+the expert inputs -> expert activation -> Hessians of the down-projection inputs; then for both
+weightings (routing-frequency and equal) aggregate -> factor -> GPTQ of gate, up and down -> loss.
+Inputs are synthetic (seeded), resident in HBM; L2 is flushed (512 MB write) before every timed step.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one process per GPU) every rank calibrates its own independent layer pair:
+weak scaling, no data-path collective; the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+N_SMS = 148
+METRIC = "expert weight columns quantized/sec (CLHA-GPTQ end to end)"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def alu_peaks(peaks):
+    """Nominal SIMT peaks at the maximum SM clock: 128 FP32 and 64 FP64 FMA lanes per SM."""
+    mhz = peaks.get("sm_max_mhz", 1965.0)
+    return {"fp32_tflops": N_SMS * 128 * 2 * mhz * 1e6 / 1e12, "fp64_tflops": N_SMS * 64 * 2 * mhz * 1e6 / 1e12}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    mhz.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------------------------------ workload
+def make_inputs(rank: int):
+    from synth import workload
+    wl = workload(2, "cpu", seed=1235 + 7919 * rank)
+    s = wl.spec
+    X = [wl.x(l) for l in range(2)]
+    lg = [wl.logits(l) for l in range(2)]
+    routed = [wl.expert_weights(0, e) for e in range(s.E)]
+    return wl, X, lg, routed
+
+
+def oracle_sample(X, lg, routed, spec, expert: int):
+    """The float64 oracle on a bounded sample of the workload: one expert's full path, both weightings
+    (routing of both layers is computed in full)."""
+    import oracle as O
+    X64 = [x.double().numpy() for x in X]
+    L64 = [l.numpy() for l in lg]
+    W64 = [tuple(t.double().numpy() for t in routed[expert])]
+    cols = 0
+    for mode in ("rt", "eq"):
+        O.calibrate_moe_group(X64, L64, spec.k, [W64[0] if e == expert else None for e in range(spec.E)], (),
+                              [expert], spec.bits_routed, spec.bits_shared, spec.group, mode, spec.damp_frac)
+        cols += 2 * spec.d_model + spec.d_ff
+    return cols
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    wl, X, lg, routed = make_inputs(0)
+    s = wl.spec
+    for i in range(args.warmup):
+        oracle_sample(X, lg, routed, s, i % s.E)
+    times, cols = [], 0
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        cols = oracle_sample(X, lg, routed, s, (args.warmup + i) % s.E)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * statistics.mean(times)
+    value = cols / (ms / 1e3)
+    sample = "one routed expert per step (gate, up, down) through route, gather, Hessians, aggregate, factor, GPTQ and loss, both weightings"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "columns/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": s.name, "columns_per_step": cols, "l2": "n/a (host)"},
+            "cpu_baseline": {"value": value, "unit": "columns/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "columns/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+    from post_quantization_expert_b200 import clha as L
+    from post_quantization_expert_b200.pipeline import MoECalibration, PhaseTimer, stack_weights
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl, X, lg, routed = make_inputs(rank)
+    s = wl.spec
+    ctx = L.Context(local)
+    timer = PhaseTimer(ctx.stream)
+    w = stack_weights((routed, []), dev)
+    Xd = [x.to(dev) for x in X]
+    Ld = [l.to(dev) for l in lg]
+    cal = MoECalibration(ctx, 2, max(s.tokens), s.E, s.k, s.d_model, s.d_ff, 0, 0, s.bits_routed, s.bits_shared,
+                         s.damp_frac, timer=timer)
+    modes = s.alpha_modes
+    cols_per_step = cal.columns() * len(modes)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        cal.reset()
+        for l in range(2):
+            cal.collect(l, Xd[l], Ld[l], w)
+        for m in modes:
+            cal.quantize(w, m)
+
+    timer.enabled = False
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    timer.enabled = True
+    timer.reset()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    launches0 = L.clha_kernel_launches(ctx)
+    ev = []
+    stream = ctx.stream
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    launches = L.clha_kernel_launches(ctx) - launches0
+    barrier(world)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    timer.collect()
+    ms = max_over_ranks(statistics.mean(step_ms), world)
+    value = world * cols_per_step / (ms / 1e3)
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
+    pin = lambda t: t.pin_memory()
+    hX, hL = [pin(x) for x in X], [pin(l) for l in lg]
+    hW = [pin(w.Wg.cpu()), pin(w.Wu.cpu()), pin(w.Wd.cpu())]
+    outs = [cal.qg, cal.qu, cal.qd]
+    hout = {m: [(pin(torch.empty_like(q.codes, device="cpu")), pin(torch.empty_like(q.scales, device="cpu")),
+                 pin(torch.empty_like(q.zeros, device="cpu"))) for q in outs] for m in modes}
+    h2d = sum(t.numel() * t.element_size() for t in hX + hL + hW)
+    d2h = sum(t.numel() * t.element_size() for m in modes for trip in hout[m] for t in trip)
+    timer.enabled = False
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for d_, h_ in zip(Xd + Ld + [w.Wg, w.Wu, w.Wd], hX + hL + hW):
+                d_.copy_(h_, non_blocking=True)
+            cal.reset()
+            for l in range(2):
+                cal.collect(l, Xd[l], Ld[l], w)
+            for m in modes:
+                cal.quantize(w, m)
+                for q, (hc, hs, hz) in zip(outs, hout[m]):
+                    hc.copy_(q.codes, non_blocking=True)
+                    hs.copy_(q.scales, non_blocking=True)
+                    hz.copy_(q.zeros, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ev = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        e2e_ev.append((a, b))
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e2e_ev), world)
+
+    # ---- per-phase timing and the roofline of the dominant kernel
+    K = args.steps
+    phase_ms = {k: v / K for k, v in timer.totals.items()}
+    counts = [cal.counts[l].cpu().numpy().astype(np.int64) for l in range(2)]
+    dm, dff, E = s.d_model, s.d_ff, s.E
+    hess_flops = sum(int(c.sum()) * (dm * (dm + 1) + dff * (dff + 1)) for c in counts)
+    mats = [(dff, dm)] * (2 * E) + [(dm, dff)] * E          # gate, up, down per weighting
+    gptq_flops = len(modes) * sum(o * i * i for o, i in mats)
+    loss_flops = len(modes) * sum(2 * o * i * i for o, i in mats)
+    factor_flops = len(modes) * E * (2 * dm ** 3 // 3 + 2 * dff ** 3 // 3)
+    act_flops = sum(int(c.sum()) * 4 * dm * dff for c in counts)
+    agg_bytes = len(modes) * E * sum(2 * (d * (d + 32) // 2) * 4 + 2 * d * d * 4 for d in (dm, dff))
+    peaks, src = load_peaks()
+    alu = alu_peaks(peaks)
+    sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    kernels = {
+        "hessian": ("tensor", hess_flops / 1e12, sustained, "TFLOP/s", "syrk_bf16_tc (tcgen05 kind::f16)"),
+        "gptq": ("alu", gptq_flops / 1e12, alu["fp32_tflops"], "TFLOP/s", "gptq_simt (fp32 FMA)"),
+        "factor": ("alu", factor_flops / 1e12, alu["fp64_tflops"], "TFLOP/s", "fac_* (fp64 FMA)"),
+        "loss": ("alu", loss_flops / 1e12, alu["fp32_tflops"], "TFLOP/s", "loss_simt (fp32 FMA)"),
+        "act": ("alu", act_flops / 1e12, alu["fp32_tflops"], "TFLOP/s", "expert_act_simt (fp32 FMA)"),
+        "aggregate": ("hbm", agg_bytes / 1e9, peaks["hbm_gbs"], "GB/s", "agg_combine"),
+    }
+    dom = max((k for k in phase_ms if k in kernels), key=lambda k: phase_ms[k])
+    bound, work, peak, unit, kname = kernels[dom]
+    achieved = work / (phase_ms[dom] / 1e3)
+    phases = {k: {"ms": round(v, 4)} for k, v in sorted(phase_ms.items(), key=lambda kv: -kv[1])}
+    for k, v in phases.items():
+        if k in kernels:
+            b_, wk, pk, un, _ = kernels[k]
+            v["achieved"] = round(wk / (phase_ms[k] / 1e3), 3)
+            v["unit"] = un
+            v["frac"] = round(v["achieved"] / pk, 4)
+    hess_tflops = hess_flops / 1e12 / (phase_ms["hessian"] / 1e3)
+
+    # ---- the oracle on the host cores, bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t0 = time.perf_counter()
+        c = oracle_sample(X, lg, routed, s, 0)
+        dt = time.perf_counter() - t0
+        cpu = {"value": c / dt, "unit": "columns/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"expert 0 of layer pair (gate, up, down; both weightings; {c} columns) in {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "columns/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": s.name, "global_batch": world * sum(s.tokens), "tokens_per_layer": s.tokens[0],
+                       "E": E, "top_k": s.k, "d_model": dm, "d_ff": dff, "bits": s.bits_routed,
+                       "weightings": list(modes), "columns_per_step_per_gpu": cols_per_step,
+                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "flushed (512 MB write) before every timed step"},
+            "hessian_tflops": hess_tflops,
+            "hessian_frac_of_bf16_peak": hess_tflops / sustained,
+            "roofline": {"kernel": kname, "phase": dom, "bound": bound, "achieved": achieved, "peak": peak,
+                         "unit": unit, "frac": achieved / peak, "traffic": None,
+                         "peak_source": src if bound in ("tensor", "hbm") else "derived (SM count x lanes x max clock)"},
+            "phases_ms_per_step": phases,
+            "e2e": {"value": world * cols_per_step / (e2e_ms / 1e3), "unit": "columns/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line))
+    ctx.close()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            return run_reference(args, world, rank)
+        return run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,189 @@
+/*
+ * clha.h — C ABI of the CLHA calibration library (libclha.so, CUDA, sm_100a).
+ *
+ * CLHA (Cross-Layer Hessian Aggregation) quantizes weights that several layers of a weight-shared
+ * Mixture-of-Experts transformer reuse. Source: the technical summary "CLHA – Cross-Layer Hessian
+ * Aggregation voor het kwantiseren van Weight-Shared Mixture-of-Experts Transformers" (below: the
+ * CLHA page). Its section 2.2 gives three phases, which the calls below follow:
+ *   (1) collection  — per layer and per active expert, a Hessian and a token count
+ *                     (clha_route_topk, clha_gather, clha_expert_act, clha_collect);
+ *   (2) aggregation — H_comb = sum_i alpha_i H_i with routing-frequency or equal weights (clha_aggregate);
+ *   (3) quantization — standard GPTQ column-sequential updates with H_comb (clha_factor, clha_quantize),
+ *                     scored by the loss of section 2.1 (clha_loss).
+ * GPTQ is the algorithm of Frantar et al. (2022), "GPTQ: Accurate Post-Training Quantization for
+ * Generative Pre-trained Transformers", Algorithm 1.
+ *
+ * Conventions for every call:
+ *   - Array arguments are DEVICE pointers owned by the caller unless the comment says "host".
+ *     The library owns only clha_ctx, clha_accum and its internal workspace.
+ *   - Work is queued on the context's stream, in call order. Calls that return host values
+ *     (alpha_out, lambda_out, loss_out, clha_accum_export, clha_check) synchronise that stream.
+ *   - Row-major layouts. X is [tokens, d] (a token's d values contiguous). A weight W is
+ *     [d_out, d_in] with y = W x. Hessians and factors are [d, d] float32.
+ *   - Shapes: every d, d_in and d_out must be a multiple of 128, else CLHA_ERR_UNSUPPORTED_SHAPE.
+ *     Token counts may be any value >= 0.
+ *   - Errors are returned, never raised: no call aborts or traps. Argument errors are detected on
+ *     the host before any work is queued. Errors found by a kernel (a non-finite input, a
+ *     non-positive pivot) are recorded on the device and returned by the next synchronising call
+ *     on the context; clha_last_error() then names the call and, for a pivot, the column.
+ */
+#ifndef CLHA_H
+#define CLHA_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CLHA_API __attribute__((visibility("default")))
+#else
+#define CLHA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CLHA_OK = 0,
+    CLHA_ERR_INVALID_ARG = 1,       /* null pointer, negative size, k > E, bits outside 2..8, ... */
+    CLHA_ERR_UNSUPPORTED_SHAPE = 2, /* d / d_in / d_out not a multiple of 128, group not 128, ... */
+    CLHA_ERR_NOT_PD = 3,            /* damped Hessian has a non-positive pivot (index in last_error) */
+    CLHA_ERR_NONFINITE = 4,         /* NaN or Inf in logits, activations or a Hessian */
+    CLHA_ERR_EMPTY = 5,             /* aggregation over slots with no tokens in any layer */
+    CLHA_ERR_OOM = 6,               /* workspace allocation failed */
+    CLHA_ERR_CUDA = 7,              /* a CUDA runtime call failed (message in last_error) */
+    CLHA_ERR_TIMEOUT = 8            /* reserved: a bounded device-side wait ran out */
+} clha_status;
+
+typedef enum { CLHA_BF16 = 0, CLHA_F32 = 1 } clha_dtype;
+
+typedef enum {
+    CLHA_ALPHA_ROUTING = 0,   /* alpha_i = n_i / sum_j n_j           (CLHA page §2.2 (2), "rt") */
+    CLHA_ALPHA_EQUAL = 1,     /* alpha_i = 1 / n_layers              (CLHA page §2.2 (2), "eq") */
+    CLHA_ALPHA_EXPLICIT = 2   /* alpha from the caller; (1, 0) is per-layer calibration on layer 0 */
+} clha_alpha_mode;
+
+/* GPTQ parameters: bits in 2..8, group = 128 (grid per 128 input columns), block = 128 (lazy-update
+ * block), damp_frac > 0 (lambda = damp_frac * mean(diag H_comb)). */
+typedef struct { int bits; int group; int block; float damp_frac; } clha_quant_params;
+
+typedef struct clha_ctx clha_ctx;
+typedef struct clha_accum clha_accum;
+
+/* ------------------------------------------------------------------------------------------ context */
+
+/* Create a context on CUDA `device` that queues work on `cuda_stream` (a cudaStream_t; NULL = the
+ * legacy default stream). The stream is borrowed, not owned. */
+CLHA_API clha_status clha_create(int device, void* cuda_stream, clha_ctx** out);
+/* Release the context and its workspace (synchronises its stream first). NULL is ignored. */
+CLHA_API void clha_destroy(clha_ctx* ctx);
+/* Message of the last failed call on this context ("" if none). Valid until the next call. */
+CLHA_API const char* clha_last_error(const clha_ctx* ctx);
+/* Synchronise the stream and return (and clear) any error a kernel recorded. */
+CLHA_API clha_status clha_check(clha_ctx* ctx);
+/* Library ABI version (major*100 + minor). */
+CLHA_API int clha_version(void);
+/* Number of kernels this context has launched so far (a tracing counter; 0 for NULL). */
+CLHA_API int64_t clha_kernel_launches(const clha_ctx* ctx);
+
+/* ------------------------------------------------------------------------------- phase 1: collection */
+
+/* Top-k routing (the CLHA page §2.2 (1) accumulates statistics "for each active expert"; §2.3 names
+ * the K-of-E routing). For each of n tokens, the k largest of its E router logits [n, E] float32:
+ * ids [n, k] int32 in descending logit order, ties to the lower expert index; counts [E] int32 is
+ * OVERWRITTEN with the number of tokens each expert receives. 1 <= k <= E <= 1024.
+ * A NaN or Inf logit is recorded as CLHA_ERR_NONFINITE. */
+CLHA_API clha_status clha_route_topk(clha_ctx* ctx, const float* logits, int64_t n, int E, int k,
+                            int32_t* ids, int32_t* counts);
+
+/* Upper bound of the rows clha_gather writes for (n, k, E): n*k + 128*E. */
+CLHA_API int64_t clha_packed_rows(int64_t n, int k, int E);
+
+/* Group the routed tokens by expert. X [n, d] (bf16 or f32) -> X_packed [packed_rows, d], same dtype,
+ * in which expert e owns rows [seg[e], seg[e] + seg[E + 1 + e]) in ascending token order, every
+ * segment starts at a multiple of 128 and the rows between segments are zero.
+ * seg is int64 [2E + 1]: seg[0..E] segment starts (seg[E] = total padded rows), seg[E+1 .. 2E]
+ * token counts. packed_rows must be >= clha_packed_rows(n, k, E). perm (optional, int32
+ * [packed_rows]) receives each packed row's token index (-1 for padding rows). */
+CLHA_API clha_status clha_gather(clha_ctx* ctx, const void* X, clha_dtype dtype, int64_t n, int d,
+                        const int32_t* ids, int k, int E, void* X_packed, int64_t packed_rows,
+                        int64_t* seg, int32_t* perm);
+
+/* Expert FFN activation feeding the down projection: h = SiLU(x Wg^T) * (x Wu^T) per token of
+ * each expert, accumulated in float32 and stored as bf16 (round to nearest even). The pages do not
+ * spell this out: the down projection's Hessian needs its input, and that input is this product.
+ * X is bf16 [rows, d_model]; Wg, Wu are bf16 [E, d_ff, d_model] (experts stacked); h is bf16
+ * [rows, d_ff]. With seg (from clha_gather) rows follow its segments and padding rows of h are
+ * written as zero; with seg == NULL, E must be 1 and all `rows` rows belong to that expert. */
+CLHA_API clha_status clha_expert_act(clha_ctx* ctx, const void* X, int64_t rows, int d_model,
+                            const int64_t* seg, int E, const void* Wg, const void* Wu, int d_ff,
+                            void* h);
+
+/* Accumulator of per-(layer, slot) Gram matrices S = sum x x^T (float32 [d, d], upper triangle
+ * authoritative, lower triangle may hold partial values) and token counts (int64). A slot is one
+ * expert (or one dense weight). Layer-aware by construction (CLHA page §2.4): every collect names
+ * its layer, and layers never share an accumulator. Created zeroed. */
+CLHA_API clha_status clha_accum_create(clha_ctx* ctx, int d, int n_layers, int n_slots, clha_accum** out);
+CLHA_API clha_status clha_accum_destroy(clha_accum* acc);
+CLHA_API clha_status clha_accum_zero(clha_ctx* ctx, clha_accum* acc);
+/* Device views: S[((layer * n_slots) + slot) * d * d ...], counts[layer * n_slots + slot]. */
+CLHA_API clha_status clha_accum_buffers(const clha_accum* acc, float** S, int64_t** counts);
+/* Checkpoint / resume: copy all of S and counts to or from host buffers of
+ * n_layers*n_slots*d*d floats and n_layers*n_slots int64. */
+CLHA_API clha_status clha_accum_export(clha_ctx* ctx, const clha_accum* acc, float* host_S, int64_t* host_counts);
+CLHA_API clha_status clha_accum_import(clha_ctx* ctx, clha_accum* acc, const float* host_S, const int64_t* host_counts);
+
+/* Phase 1 accumulation for one layer (CLHA page §2.2 (1)): S[layer][slot] += X_e^T X_e and
+ * counts[layer][slot] += n_e. With seg == NULL, all `rows` rows of X go to slot `slot0` (a dense
+ * weight, or an always-active shared expert); with seg (clha_gather's layout), expert e goes to
+ * slot slot0 + e for e < E. X is [rows, d] bf16 (tensor cores, fp32 accumulation) or f32 (fp32 FMA).
+ * A NaN or Inf entry of X is recorded as CLHA_ERR_NONFINITE. */
+CLHA_API clha_status clha_collect(clha_ctx* ctx, clha_accum* acc, int layer, const void* X, clha_dtype dtype,
+                         int64_t rows, int d, const int64_t* seg, int E, int slot0);
+
+/* ------------------------------------------------------------------------------ phase 2: aggregation */
+
+/* For each slot s in [slot0, slot0 + n_slots): alpha_i from `mode` over the accumulator's layers
+ * (CLHA page §2.2 (2); alpha_in is a host [n_layers] array for CLHA_ALPHA_EXPLICIT, else ignored),
+ * H_comb = sum_i alpha_i (2 / n_i) S_i (layers with n_i = 0 contribute nothing; §2.1 Proposition 1),
+ * lambda = damp_frac * mean(diag H_comb) and H_damped = H_comb + lambda I.
+ * H_comb and H_damped are float32 [n_slots, d, d], full symmetric. H_comb may be NULL.
+ * alpha_out (host double [n_slots * n_layers]) and lambda_out (host double [n_slots]) are optional;
+ * passing either synchronises. A slot with no tokens in any layer gives CLHA_ERR_EMPTY. */
+CLHA_API clha_status clha_aggregate(clha_ctx* ctx, const clha_accum* acc, int slot0, int n_slots,
+                           clha_alpha_mode mode, const double* alpha_in, float damp_frac,
+                           float* H_comb, float* H_damped, double* alpha_out, double* lambda_out);
+
+/* ------------------------------------------------------------------------------ phase 3: quantization */
+
+/* GPTQ's factor of the damped Hessian: U upper triangular with H_damped^-1 = U^T U (the upper
+ * Cholesky factor of the inverse), for `batch` problems [batch, d, d] float32. Computed as
+ * H_damped = R R^T with R upper (Cholesky in reversed index order) and U = R^-1, in float64.
+ * The strict lower triangle of U is written as zero. A non-positive pivot is recorded as
+ * CLHA_ERR_NOT_PD with the problem and column. */
+CLHA_API clha_status clha_factor(clha_ctx* ctx, const float* H_damped, int batch, int d, float* U);
+
+/* GPTQ (CLHA page §2.2 (3)): column-sequential quantization of `batch` weights W [batch, d_out, d_in]
+ * (bf16 or f32) in natural column order, with lazy updates over 128-column blocks. Problem b uses
+ * U + (b / w_per_u) * d_in * d_in (w_per_u >= 1 lets, e.g., gate and up share one factor).
+ * At the start of each group of 128 columns a row's grid is fixed from its current values:
+ * xmin = min(0, min w), xmax = max(0, max w) ([-1, 1] if both are 0), s = (xmax - xmin)/(2^b - 1),
+ * z = round(-xmin/s); each column then takes q = clamp(round(w/s) + z, 0, 2^b - 1), w_hat = s (q - z),
+ * and its error (w - w_hat)/U_jj is subtracted along row j of U from the later columns. The grid and
+ * the code are decided in IEEE float32 (round to nearest even); the updates accumulate in float32.
+ * Outputs: codes uint8 [batch, d_out, d_in], scales float32 and zeros uint8 [batch, d_out, d_in/128],
+ * W_hat float32 [batch, d_out, d_in] (may be NULL). */
+CLHA_API clha_status clha_quantize(clha_ctx* ctx, const float* U, int w_per_u, const void* W, clha_dtype dtype,
+                          int batch, int d_out, int d_in, const clha_quant_params* params,
+                          uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat);
+
+/* Loss of the CLHA page §2.1, one term: loss_out[b] = tr[(W_hat - W) H (W_hat - W)^T] for `batch`
+ * problems; problem b uses H + (b / w_per_h) * d_in * d_in. Accumulated in float64.
+ * loss_out is a host double [batch] array (synchronises). */
+CLHA_API clha_status clha_loss(clha_ctx* ctx, const void* W, clha_dtype dtype, const float* W_hat,
+                      const float* H, int w_per_h, int batch, int d_out, int d_in, double* loss_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CLHA_H */

@@ -239,11 +239,11 @@ def calibrate_dense(W, X_list, bits: int, group: int = 128, mode: str = "rt", al
 
 def calibrate_moe_group(X_list, logits_list, k: int, routed, shared=(), experts=None,
                         bits_routed: int = 2, bits_shared: int = 3, group: int = 128,
-                        mode: str = "rt", damp_frac: float = 0.01):
+                        mode: str = "rt", damp_frac: float = 0.01, shared_experts=None):
     """CLHA on one group of layers sharing routed experts `routed` [(Wg, Wu, Wd)] and always-active
     experts `shared` (CLHA page §2.2 phases 1-3, §2.3 mixed precision, §2.4 per-layer accumulators).
 
-    experts: which routed experts to calibrate (default all); shared ones are always calibrated.
+    experts / shared_experts: which routed / always-active experts to calibrate (default: all).
     Returns per-layer routing and, per expert key ("r", e) / ("s", e), counts, alphas and the GPTQ
     results of gate/up (input Hessian over x) and down (input Hessian over h).
     """
@@ -254,8 +254,10 @@ def calibrate_moe_group(X_list, logits_list, k: int, routed, shared=(), experts=
     toks = [expert_tokens(ids, E) for ids, _ in routes]
     out = {"routes": routes, "experts": {}}
     jobs = [(("r", e), routed[e], [t[e] for t in toks], bits_routed) for e in experts]
-    jobs += [(("s", i), w, [np.arange(np.asarray(X).shape[0]) for X in X_list], bits_shared)
-             for i, w in enumerate(shared)]
+    if shared_experts is None:
+        shared_experts = range(len(shared))
+    jobs += [(("s", i), shared[i], [np.arange(np.asarray(X).shape[0]) for X in X_list], bits_shared)
+             for i in shared_experts]
     for key, (Wg, Wu, Wd), tok_l, bits in jobs:
         Xe = [np.asarray(X, dtype=np.float64)[t] for X, t in zip(X_list, tok_l)]
         he = [ffn_act(x, Wg, Wu) for x in Xe]

@@ -1,0 +1,131 @@
+// Phase 2 of CLHA (the CLHA page, §2.1 Proposition 1 and §2.2 (2)): H_comb = sum_i alpha_i H_i with
+// H_i = (2 / n_i) S_i, routing-frequency (alpha_i = n_i / sum n), equal (1/L) or explicit weights,
+// then GPTQ damping H_d = H_comb + lambda I, lambda = damp_frac * mean(diag H_comb).
+//
+// Two kernels per call, both HBM-bound:
+//   agg_scalars  one block per slot: alpha (float64), lambda from the diagonals (float64 reduction),
+//                empty-slot and non-finite checks;
+//   agg_combine  one block per 32x32 upper tile pair: reads each layer's upper tile of S once and
+//                writes both the tile and its mirror image (through shared memory, coalesced).
+#include "clha_internal.h"
+
+namespace {
+
+__device__ __forceinline__ double layer_coef(const double* alpha, const int64_t* cnt, int l) {
+    int64_t n = cnt[l];
+    return n > 0 ? alpha[l] * 2.0 / (double)n : 0.0;
+}
+
+__global__ void __launch_bounds__(256) agg_scalars(const float* __restrict__ S, const int64_t* __restrict__ counts,
+                                                   int d, int L, int n_slots_total, int slot0, clha_alpha_args a,
+                                                   float damp_frac, double* __restrict__ d_alpha,
+                                                   double* __restrict__ d_lambda, int* err) {
+    const int sl = blockIdx.x;
+    const int slot = slot0 + sl;
+    __shared__ double alpha[16];
+    __shared__ int64_t cnt[16];
+    __shared__ double red[256];
+    if (threadIdx.x == 0) {
+        int64_t tot = 0;
+        for (int l = 0; l < L; ++l) {
+            cnt[l] = counts[(size_t)l * n_slots_total + slot];
+            tot += cnt[l];
+        }
+        for (int l = 0; l < L; ++l) {
+            double al;
+            if (a.mode == CLHA_ALPHA_ROUTING) al = tot > 0 ? (double)cnt[l] / (double)tot : 0.0;
+            else if (a.mode == CLHA_ALPHA_EQUAL) al = 1.0 / L;
+            else al = a.alpha[l];
+            alpha[l] = al;
+            d_alpha[(size_t)sl * L + l] = al;
+        }
+        if (tot == 0) clha_record_error(err, CLHA_ERR_EMPTY, slot, 0, KID_AGGREGATE);
+    }
+    __syncthreads();
+    double acc = 0.0;
+    for (int i = threadIdx.x; i < d; i += blockDim.x) {
+        double v = 0.0;
+        for (int l = 0; l < L; ++l) {
+            double c = layer_coef(alpha, cnt, l);
+            if (c != 0.0) v += c * (double)S[(((size_t)l * n_slots_total + slot) * d + i) * d + i];
+        }
+        acc += v;
+    }
+    red[threadIdx.x] = acc;
+    __syncthreads();
+    for (int off = 128; off > 0; off >>= 1) {
+        if (threadIdx.x < off) red[threadIdx.x] += red[threadIdx.x + off];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        double lam = (double)damp_frac * red[0] / d;
+        d_lambda[sl] = lam;
+        if (!isfinite(red[0])) clha_record_error(err, CLHA_ERR_NONFINITE, slot, -1, KID_AGGREGATE);
+    }
+}
+
+__global__ void __launch_bounds__(256) agg_combine(const float* __restrict__ S, const int64_t* __restrict__ counts,
+                                                   int d, int L, int n_slots_total, int slot0,
+                                                   const double* __restrict__ d_alpha,
+                                                   const double* __restrict__ d_lambda, float* __restrict__ H_comb,
+                                                   float* __restrict__ H_d, int* err) {
+    const int sl = blockIdx.y;
+    const int slot = slot0 + sl;
+    const int nt = d / 32;
+    int t = blockIdx.x, bi = 0;
+    while (t >= nt - bi) { t -= nt - bi; ++bi; }
+    const int bj = bi + t;  // bi <= bj
+    __shared__ float tile[32][33];
+    __shared__ float coef[16];
+    if (threadIdx.x < L) {
+        int64_t n = counts[(size_t)threadIdx.x * n_slots_total + slot];
+        coef[threadIdx.x] = n > 0 ? (float)(d_alpha[(size_t)sl * L + threadIdx.x] * 2.0 / (double)n) : 0.f;
+    }
+    __syncthreads();
+    const float lam = (float)d_lambda[sl];
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+    bool bad = false;
+    for (int r = ty; r < 32; r += 8) {
+        const int i = bi * 32 + r, j = bj * 32 + tx;
+        float v = 0.f;
+        for (int l = 0; l < L; ++l) {
+            float c = coef[l];
+            if (c != 0.f) v = fmaf(c, S[(((size_t)l * n_slots_total + slot) * d + i) * d + j], v);
+        }
+        if (!isfinite(v)) bad = true;
+        tile[r][tx] = v;
+    }
+    if (bad) clha_record_error(err, CLHA_ERR_NONFINITE, slot, bi * 32, KID_AGGREGATE);
+    __syncthreads();
+    float* Hc = H_comb ? H_comb + (size_t)sl * d * d : nullptr;
+    float* Hd = H_d + (size_t)sl * d * d;
+    for (int r = ty; r < 32; r += 8) {
+        // upper tile (bi, bj): entry (r, tx); inside a diagonal tile take the upper value for r > tx
+        const int i = bi * 32 + r, j = bj * 32 + tx;
+        float v = (bi == bj && r > tx) ? tile[tx][r] : tile[r][tx];
+        if (Hc) Hc[(size_t)i * d + j] = v;
+        Hd[(size_t)i * d + j] = v + (i == j ? lam : 0.f);
+        if (bi != bj) {  // mirror tile (bj, bi): entry (r, tx) = upper (tx, r)
+            const int i2 = bj * 32 + r, j2 = bi * 32 + tx;
+            float m = tile[tx][r];
+            if (Hc) Hc[(size_t)i2 * d + j2] = m;
+            Hd[(size_t)i2 * d + j2] = m;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_aggregate(cudaStream_t s, const float* S, const int64_t* counts, int d, int n_layers,
+                             int n_slots_total, int slot0, int n_slots, clha_alpha_args a, float damp_frac,
+                             float* H_comb, float* H_d, double* d_alpha, double* d_lambda, int* err) {
+    agg_scalars<<<n_slots, 256, 0, s>>>(S, counts, d, n_layers, n_slots_total, slot0, a, damp_frac, d_alpha, d_lambda,
+                                        err);
+    clha_note_launches(1);
+    int nt = d / 32;
+    dim3 grid(nt * (nt + 1) / 2, n_slots);
+    agg_combine<<<grid, 256, 0, s>>>(S, counts, d, n_layers, n_slots_total, slot0, d_alpha, d_lambda, H_comb, H_d,
+                                     err);
+    clha_note_launches(1);
+    return cudaGetLastError();
+}

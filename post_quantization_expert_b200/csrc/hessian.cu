@@ -1,0 +1,305 @@
+// Phase 1 of CLHA (the CLHA page, §2.2 (1)): per (layer, expert) Gram matrices S += X_e^T X_e of the
+// tokens routed to the expert, plus their token counts; H = (2/n) S is formed at aggregation.
+//
+// bf16 inputs: a persistent, warp-specialised tcgen05 kernel (one CTA per SM).
+//   warp 0     TMA producer: for an output tile (rows i0..i0+127, cols j0..j0+255) streams the
+//              token blocks X[t0:t0+64, i0:i0+128] and X[t0:t0+64, j0:j0+256] into a 4-stage ring
+//              (128-byte swizzle; both operands are "M/N-major": one token row = 64 contiguous
+//              channels, which is how X is laid out, so no transpose is ever materialised).
+//   warp 1     MMA issuer: tcgen05.mma kind::f16 M=128 N=256 K=16, four per 64-token block,
+//              accumulating in TMEM; two accumulators (512 TMEM columns) so the epilogue of one
+//              tile overlaps the MMAs of the next.
+//   warps 2-5  epilogue: tcgen05.ld of the fp32 tile, read-modify-write into S (float4).
+// Only tiles that touch the upper triangle are computed (rows tile r <= 2c+1 for column tile c);
+// entries below the diagonal inside those tiles are correct values but the upper triangle is the
+// authoritative one. Segments from the gather are 128-row aligned with zero padding, so a token
+// block never mixes experts and padding adds nothing.
+// float32 inputs: a plain shared-memory tiled FMA kernel (used by the small fp32 workload).
+#include "clha_internal.h"
+#include "tc_ptx.h"
+#include "tmap.h"
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int kThreads = 192;
+constexpr uint32_t IDESC = tc::idesc_f32acc(1 /*bf16*/, 1 /*A MN-major*/, 1 /*B MN-major*/, BM, BN);
+
+struct SyrkParams {
+    int d;
+    int64_t rows;
+    const int64_t* seg;
+    int E;
+    float* S;
+    int tiles_per_slot;
+    int nr, nc;
+    int total_tiles;
+    int* err;
+};
+
+__device__ __forceinline__ void decode_tile(int t, int nr, int nc, int& r, int& c) {
+    r = 0;
+    for (c = 0; c < nc; ++c) {
+        int m = min(nr, 2 * c + 2);
+        if (t < m) { r = t; return; }
+        t -= m;
+    }
+}
+
+__device__ __forceinline__ void slot_range(const SyrkParams& p, int e, int64_t& t0, int64_t& cnt) {
+    if (p.seg) { t0 = p.seg[e]; cnt = p.seg[p.E + 1 + e]; }
+    else { t0 = 0; cnt = p.rows; }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) syrk_bf16_tc(const __grid_constant__ CUtensorMap tmX, SyrkParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    const uint32_t full0 = tc::smem_u32(bars);
+    const uint32_t empty0 = full0 + 8 * STAGES;
+    const uint32_t tfull0 = full0 + 16 * STAGES;
+    const uint32_t tempty0 = tfull0 + 16;
+    const uint32_t drain = tfull0 + 32;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(full0 + 8 * s, 1);
+            tc::mbar_init(empty0 + 8 * s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            tc::mbar_init(tfull0 + 8 * a, 1);
+            tc::mbar_init(tempty0 + 8 * a, 128);
+        }
+        tc::mbar_init(drain, 1);
+        *abort_flag = 0;
+        tc::fence_barrier_init();
+        tc::prefetch_tmap(&tmX);
+    }
+    if (warp == 1) tc::tmem_alloc(tc::smem_u32(tmem_slot), 512);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int it = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < p.total_tiles && ok; w += gridDim.x) {
+                const int e = w / p.tiles_per_slot;
+                int r, c;
+                decode_tile(w % p.tiles_per_slot, p.nr, p.nc, r, c);
+                int64_t t0, cnt;
+                slot_range(p, e, t0, cnt);
+                const int nk = (int)((cnt + BK - 1) / BK);
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!tc::mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag)) { ok = false; break; }
+                    const uint32_t fb = full0 + 8 * s;
+                    tc::mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    const uint32_t a_dst = tc::smem_u32(smem + s * STAGE_BYTES);
+                    const uint32_t b_dst = a_dst + A_BYTES;
+                    const int y = (int)(t0 + (int64_t)kb * BK);
+#pragma unroll
+                    for (int h = 0; h < BM / 64; ++h) tc::tma_load_2d(a_dst + h * 8192, &tmX, fb, r * BM + h * 64, y);
+#pragma unroll
+                    for (int h = 0; h < BN / 64; ++h) tc::tma_load_2d(b_dst + h * 8192, &tmX, fb, c * BN + h * 64, y);
+                }
+            }
+            if (!ok) {  // let the copies already issued land before the CTA can exit
+                for (int j = it - 1; j >= 0 && j >= it - STAGES; --j)
+                    tc::mbar_wait_bounded(full0 + 8 * (j % STAGES), (j / STAGES) & 1, abort_flag, 100000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int it = 0, tcount = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < p.total_tiles && ok; w += gridDim.x) {
+                const int e = w / p.tiles_per_slot;
+                int64_t t0, cnt;
+                slot_range(p, e, t0, cnt);
+                const int nk = (int)((cnt + BK - 1) / BK);
+                if (nk == 0) continue;
+                const int acc = tcount & 1;
+                const uint32_t aph = (tcount >> 1) & 1;
+                if (!tc::mbar_wait_bounded(tempty0 + 8 * acc, aph ^ 1, abort_flag)) break;
+                tc::fence_after_sync();
+                const uint32_t d_tmem = tmem + acc * BN;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!tc::mbar_wait_bounded(full0 + 8 * s, ph, abort_flag)) { ok = false; break; }
+                    tc::fence_after_sync();
+                    const uint32_t a_base = tc::smem_u32(smem + s * STAGE_BYTES);
+                    const uint32_t b_base = a_base + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t ad = tc::sw128_desc(a_base + kk * 2048, 8192, 1024);
+                        const uint64_t bd = tc::sw128_desc(b_base + kk * 2048, 8192, 1024);
+                        tc::mma_f16(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
+                    }
+                    tc::mma_commit(empty0 + 8 * s);
+                }
+                if (!ok) break;
+                tc::mma_commit(tfull0 + 8 * acc);
+                ++tcount;
+            }
+        }
+        __syncwarp();
+    } else {
+        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        int tcount = 0;
+        for (int w = blockIdx.x; w < p.total_tiles; w += gridDim.x) {
+            const int e = w / p.tiles_per_slot;
+            int r, c;
+            decode_tile(w % p.tiles_per_slot, p.nr, p.nc, r, c);
+            int64_t t0, cnt;
+            slot_range(p, e, t0, cnt);
+            if (cnt == 0) continue;
+            const int acc = tcount & 1;
+            const uint32_t aph = (tcount >> 1) & 1;
+            if (!tc::mbar_wait_bounded(tfull0 + 8 * acc, aph, abort_flag)) break;
+            tc::fence_after_sync();
+            const int row = r * BM + q * 32 + lane;
+            float* Srow = p.S + (size_t)e * p.d * p.d + (size_t)row * p.d;
+            const int warp_row_min = r * BM + q * 32;
+#pragma unroll 1
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                const int col0 = c * BN + ch * 32;
+                if (col0 >= p.d) break;
+                if (col0 + 31 < warp_row_min) continue;  // whole chunk strictly below the diagonal
+                uint32_t v[32];
+                tc::tmem_ld_32x32b_x32(tmem + acc * BN + ch * 32 + ((uint32_t)(q * 32) << 16), v);
+                tc::tmem_wait_ld();
+                float4* dst = reinterpret_cast<float4*>(Srow + col0);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float4 o = dst[j];
+                    o.x += __uint_as_float(v[4 * j + 0]);
+                    o.y += __uint_as_float(v[4 * j + 1]);
+                    o.z += __uint_as_float(v[4 * j + 2]);
+                    o.w += __uint_as_float(v[4 * j + 3]);
+                    dst[j] = o;
+                }
+            }
+            tc::fence_before_sync();
+            tc::mbar_arrive(tempty0 + 8 * acc);
+            ++tcount;
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        if (lane == 0) {
+            tc::mma_commit(drain);
+            tc::mbar_wait_bounded(drain, 0, abort_flag, 100000000ull);
+        }
+        __syncwarp();
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+    if (threadIdx.x == 0 && *abort_flag) clha_record_error(p.err, CLHA_ERR_TIMEOUT, blockIdx.x, 0, KID_COLLECT);
+}
+
+__global__ void add_counts(int64_t* counts, const int64_t* seg, int E, int64_t rows) {
+    int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e < E) counts[e] += seg ? seg[E + 1 + e] : rows;
+}
+
+// ------------------------------------------------------------------------------ float32 inputs
+constexpr int FT = 64, FK = 32;
+
+__global__ void __launch_bounds__(256) syrk_f32_simt(const float* __restrict__ X, int64_t rows, int d,
+                                                     const int64_t* __restrict__ seg, int E, float* __restrict__ S) {
+    // blockIdx.x: upper tile index (r <= c) in row-major order over the tile grid; blockIdx.y: slot
+    const int nt = d / FT;
+    int t = blockIdx.x, r = 0;
+    while (t >= nt - r) { t -= nt - r; ++r; }
+    const int c = r + t;
+    const int e = blockIdx.y;
+    int64_t t0 = 0, cnt = rows;
+    if (seg) { t0 = seg[e]; cnt = seg[E + 1 + e]; }
+    __shared__ float As[FK][FT + 4];
+    __shared__ float Bs[FK][FT + 4];
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    float acc[4][4] = {};
+    for (int64_t k0 = 0; k0 < cnt; k0 += FK) {
+        for (int i = threadIdx.x; i < FK * FT; i += 256) {
+            int kk = i / FT, m = i % FT;
+            bool in = k0 + kk < cnt;
+            const float* xr = X + (t0 + k0 + kk) * (int64_t)d;
+            As[kk][m] = in ? xr[r * FT + m] : 0.f;
+            Bs[kk][m] = in ? xr[c * FT + m] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < FK; ++kk) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { a[i] = As[kk][ty * 4 + i]; b[i] = Bs[kk][tx * 4 + i]; }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+    float* Se = S + (size_t)e * d * d;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) Se[(size_t)(r * FT + ty * 4 + i) * d + c * FT + tx * 4 + j] += acc[i][j];
+}
+
+}  // namespace
+
+cudaError_t launch_collect_bf16(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t rows, int d,
+                                const int64_t* seg, int E, float* S_base, int64_t* counts_base, int* err) {
+    CUtensorMap tm;
+    cudaError_t e = make_tmap_2d(&tm, X, (uint64_t)rows, (uint64_t)d, 2, 64, 64);
+    if (e != cudaSuccess) return e;
+    static bool attr_set = false;
+    if (!attr_set) {
+        e = cudaFuncSetAttribute(syrk_bf16_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    SyrkParams p;
+    p.d = d;
+    p.rows = rows;
+    p.seg = seg;
+    p.E = E;
+    p.S = S_base;
+    p.nr = d / BM;
+    p.nc = (d + BN - 1) / BN;
+    p.tiles_per_slot = 0;
+    for (int c = 0; c < p.nc; ++c) p.tiles_per_slot += (p.nr < 2 * c + 2) ? p.nr : 2 * c + 2;
+    p.total_tiles = p.tiles_per_slot * E;
+    p.err = err;
+    int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
+    syrk_bf16_tc<<<grid, kThreads, SMEM_BYTES, s>>>(tm, p);
+    clha_note_launches(1);
+    add_counts<<<(E + 255) / 256, 256, 0, s>>>(counts_base, seg, E, rows);
+    clha_note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_collect_f32(cudaStream_t s, const float* X, int64_t rows, int d, const int64_t* seg, int E,
+                               float* S_base, int64_t* counts_base) {
+    int nt = d / FT;
+    dim3 grid(nt * (nt + 1) / 2, E);
+    syrk_f32_simt<<<grid, 256, 0, s>>>(X, rows, d, seg, E, S_base);
+    clha_note_launches(1);
+    add_counts<<<(E + 255) / 256, 256, 0, s>>>(counts_base, seg, E, rows);
+    clha_note_launches(1);
+    return cudaGetLastError();
+}

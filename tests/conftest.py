@@ -16,3 +16,15 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+@pytest.fixture(scope="session")
+def ctx():
+    """A library context on cuda:0 (GPU tests only)."""
+    import torch
+    from post_quantization_expert_b200 import clha
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    c = clha.Context(0)
+    yield c
+    torch.cuda.synchronize()
+    c.close()

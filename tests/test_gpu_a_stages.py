@@ -1,0 +1,349 @@
+"""Stage-wise parity of each CUDA step against the float64 oracle, each stage fed the same inputs as
+the oracle so its own error is isolated. Sizes span several tiles and end on ragged tails."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from helpers import code_agreement, rel_fro, sym_from_upper, to64
+from post_quantization_expert_b200 import clha as L
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _gen(seed):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return g
+
+
+# ------------------------------------------------------------------------------------ routing
+@pytest.mark.parametrize("n,E,k", [(1000, 16, 2), (4099, 64, 6), (37, 5, 5), (1, 1024, 8), (777, 33, 1)])
+def test_route_bit_exact(ctx, n, E, k):
+    g = _gen(n + E)
+    lg = torch.randn((n, E), generator=g)
+    lg[::7, 3 % E] = lg[::7, 0]                                  # ties between experts
+    lg[::11] = torch.round(lg[::11] * 2) / 2                     # many exact ties
+    lg = lg.to(DEV)
+    ids = torch.empty((n, k), dtype=torch.int32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    L.clha_route_topk(ctx, lg, n, E, k, ids, counts)
+    want_ids, want_counts = O.route_topk(lg.cpu().numpy(), k)
+    np.testing.assert_array_equal(ids.cpu().numpy(), want_ids)
+    np.testing.assert_array_equal(counts.cpu().numpy(), want_counts)
+
+
+def test_route_empty_input(ctx):
+    counts = torch.full((8,), 7, dtype=torch.int32, device=DEV)
+    L.clha_route_topk(ctx, None, 0, 8, 2, None, counts)
+    assert counts.sum().item() == 0
+
+
+# ------------------------------------------------------------------------------------ gather
+@pytest.mark.parametrize("n,E,k,d", [(1000, 16, 2, 256), (3001, 64, 6, 128), (5, 8, 2, 384)])
+def test_gather_segments(ctx, n, E, k, d):
+    g = _gen(n)
+    lg = torch.randn((n, E), generator=g).to(DEV)
+    X = torch.randn((n, d), generator=g).to(torch.bfloat16).to(DEV)
+    ids = torch.empty((n, k), dtype=torch.int32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    L.clha_route_topk(ctx, lg, n, E, k, ids, counts)
+    P = L.clha_packed_rows(n, k, E)
+    Xp = torch.full((P, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    seg = torch.empty(2 * E + 1, dtype=torch.int64, device=DEV)
+    perm = torch.empty(P, dtype=torch.int32, device=DEV)
+    L.clha_gather(ctx, X, n, d, ids, k, E, Xp, P, seg, perm)
+    seg, perm, Xp = seg.cpu().numpy(), perm.cpu().numpy(), Xp.cpu()
+    want_ids, want_counts = O.route_topk(lg.cpu().numpy(), k)
+    lists = O.expert_tokens(want_ids, E)
+    np.testing.assert_array_equal(seg[E + 1:], want_counts)
+    start = 0
+    for e in range(E):
+        assert seg[e] == start and seg[e] % 128 == 0
+        np.testing.assert_array_equal(perm[seg[e]:seg[e] + want_counts[e]], lists[e])
+        assert np.all(perm[seg[e] + want_counts[e]:seg[e] + (want_counts[e] + 127) // 128 * 128] == -1)
+        rows = Xp[seg[e]:seg[e] + want_counts[e]]
+        assert torch.equal(rows, X.cpu()[torch.from_numpy(lists[e]).long()])
+        pad = Xp[seg[e] + want_counts[e]:seg[e] + (want_counts[e] + 127) // 128 * 128]
+        assert torch.all(pad == 0)
+        start += (want_counts[e] + 127) // 128 * 128
+    assert seg[E] == start
+
+
+# ------------------------------------------------------------------------------------ collection
+@pytest.mark.parametrize("n,d", [(1000, 512), (129, 1408), (1, 256), (4096, 1024), (777, 2048)])
+def test_collect_dense_bf16(ctx, n, d):
+    g = _gen(n * d)
+    X = (torch.randn((n, d), generator=g) * (1 + torch.rand(d, generator=g))).to(torch.bfloat16).to(DEV)
+    acc = L.Accum(ctx, d, 2, 1)
+    L.clha_collect(ctx, acc, 1, X, n, d)
+    S, cnt = acc.buffers()
+    torch.cuda.synchronize()
+    want = O.gram(to64(X))
+    got = sym_from_upper(S[1, 0].double().cpu().numpy())
+    assert rel_fro(got, want) < 1e-4
+    assert cnt[1, 0].item() == n and cnt[0, 0].item() == 0
+    assert torch.all(S[0] == 0)
+
+
+def test_collect_routed_bf16_and_accumulates(ctx):
+    n, E, k, d = 3000, 16, 2, 1024
+    g = _gen(7)
+    lg = torch.randn((n, E), generator=g).to(DEV)
+    X = torch.randn((n, d), generator=g).to(torch.bfloat16).to(DEV)
+    ids = torch.empty((n, k), dtype=torch.int32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    L.clha_route_topk(ctx, lg, n, E, k, ids, counts)
+    P = L.clha_packed_rows(n, k, E)
+    Xp = torch.empty((P, d), dtype=torch.bfloat16, device=DEV)
+    seg = torch.empty(2 * E + 1, dtype=torch.int64, device=DEV)
+    L.clha_gather(ctx, X, n, d, ids, k, E, Xp, P, seg)
+    acc = L.Accum(ctx, d, 1, E + 2)
+    L.clha_collect(ctx, acc, 0, Xp, P, d, seg, E, 2)     # slots 2..E+1
+    L.clha_collect(ctx, acc, 0, Xp, P, d, seg, E, 2)     # a second batch accumulates
+    S, cnt = acc.buffers()
+    torch.cuda.synchronize()
+    want_ids, want_counts = O.route_topk(lg.cpu().numpy(), k)
+    lists = O.expert_tokens(want_ids, E)
+    X64 = to64(X)
+    np.testing.assert_array_equal(cnt[0, 2:].cpu().numpy(), 2 * want_counts)
+    assert cnt[0, :2].sum().item() == 0
+    for e in range(E):
+        want = 2 * O.gram(X64[lists[e]])
+        assert rel_fro(sym_from_upper(S[0, 2 + e].double().cpu().numpy()), want) < 1e-4
+
+
+@pytest.mark.parametrize("n,d", [(1000, 512), (1024, 512), (33, 128)])
+def test_collect_dense_f32(ctx, n, d):
+    g = _gen(n + 3)
+    X = torch.randn((n, d), generator=g).to(DEV)
+    acc = L.Accum(ctx, d, 1, 1)
+    L.clha_collect(ctx, acc, 0, X, n, d)
+    S, _ = acc.buffers()
+    torch.cuda.synchronize()
+    assert rel_fro(sym_from_upper(S[0, 0].double().cpu().numpy()), O.gram(to64(X))) < 1e-4
+
+
+def test_layer_tagged_collection_is_order_independent(ctx):
+    """Layer-aware accumulators (CLHA page §2.4): interleaving the layers' calls in any order gives
+    each layer exactly its own tokens' Gram matrix."""
+    d = 256
+    g = _gen(11)
+    Xa1, Xa2, Xb = (torch.randn((n, d), generator=g).to(torch.bfloat16).to(DEV) for n in (300, 200, 500))
+    acc1, acc2 = L.Accum(ctx, d, 2, 1), L.Accum(ctx, d, 2, 1)
+    for layer, X in ((0, Xa1), (1, Xb), (0, Xa2)):
+        L.clha_collect(ctx, acc1, layer, X, X.shape[0], d)
+    for layer, X in ((1, Xb), (0, Xa2), (0, Xa1)):
+        L.clha_collect(ctx, acc2, layer, X, X.shape[0], d)
+    S1, c1 = acc1.buffers()
+    S2, c2 = acc2.buffers()
+    torch.cuda.synchronize()
+    want_a = O.gram(np.vstack([to64(Xa1), to64(Xa2)]))
+    want_b = O.gram(to64(Xb))
+    for S in (S1, S2):
+        assert rel_fro(sym_from_upper(S[0, 0].double().cpu().numpy()), want_a) < 1e-4
+        assert rel_fro(sym_from_upper(S[1, 0].double().cpu().numpy()), want_b) < 1e-4
+    assert c1.tolist() == c2.tolist() == [[500], [500]]
+
+
+def test_accumulator_checkpoint_roundtrip(ctx):
+    d = 128
+    X = torch.randn((70, d), generator=_gen(5)).to(torch.bfloat16).to(DEV)
+    acc = L.Accum(ctx, d, 2, 3)
+    L.clha_collect(ctx, acc, 1, X, 70, d, None, 1, 2)
+    S, cnt = L.clha_accum_export(ctx, acc)
+    acc2 = L.Accum(ctx, d, 2, 3)
+    L.clha_accum_import(ctx, acc2, S, cnt)
+    L.clha_collect(ctx, acc2, 1, X, 70, d, None, 1, 2)     # resume: one more batch
+    S2, cnt2 = L.clha_accum_export(ctx, acc2)
+    np.testing.assert_array_equal(cnt2[1, 2], 140)
+    np.testing.assert_allclose(np.triu(S2[1, 2]), 2 * np.triu(S[1, 2]), rtol=1e-6)
+
+
+# ------------------------------------------------------------------------------------ FFN act
+@pytest.mark.parametrize("rows,dm,dff", [(300, 256, 384), (1000, 1024, 512)])
+def test_expert_act_dense(ctx, rows, dm, dff):
+    g = _gen(rows)
+    X = torch.randn((rows, dm), generator=g).to(torch.bfloat16).to(DEV)
+    Wg = (0.05 * torch.randn((1, dff, dm), generator=g)).to(torch.bfloat16).to(DEV)
+    Wu = (0.05 * torch.randn((1, dff, dm), generator=g)).to(torch.bfloat16).to(DEV)
+    h = torch.empty((rows, dff), dtype=torch.bfloat16, device=DEV)
+    L.clha_expert_act(ctx, X, rows, dm, None, 1, Wg, Wu, dff, h)
+    want = O.ffn_act(to64(X), to64(Wg[0]), to64(Wu[0]))
+    got = to64(h)
+    exact = np.mean(got == want)
+    assert exact > 0.995
+    np.testing.assert_allclose(got, want, rtol=2 ** -7, atol=1e-6)
+
+
+def test_expert_act_segments_zero_padding(ctx):
+    n, E, k, dm, dff = 600, 8, 2, 256, 128
+    g = _gen(9)
+    lg = torch.randn((n, E), generator=g).to(DEV)
+    X = torch.randn((n, dm), generator=g).to(torch.bfloat16).to(DEV)
+    Wg = (0.05 * torch.randn((E, dff, dm), generator=g)).to(torch.bfloat16).to(DEV)
+    Wu = (0.05 * torch.randn((E, dff, dm), generator=g)).to(torch.bfloat16).to(DEV)
+    ids = torch.empty((n, k), dtype=torch.int32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    L.clha_route_topk(ctx, lg, n, E, k, ids, counts)
+    P = L.clha_packed_rows(n, k, E)
+    Xp = torch.empty((P, dm), dtype=torch.bfloat16, device=DEV)
+    seg = torch.empty(2 * E + 1, dtype=torch.int64, device=DEV)
+    L.clha_gather(ctx, X, n, dm, ids, k, E, Xp, P, seg)
+    h = torch.full((P, dff), 3.0, dtype=torch.bfloat16, device=DEV)
+    L.clha_expert_act(ctx, Xp, P, dm, seg, E, Wg, Wu, dff, h)
+    seg = seg.cpu().numpy()
+    lists = O.expert_tokens(O.route_topk(lg.cpu().numpy(), k)[0], E)
+    X64 = to64(X)
+    hh = to64(h)
+    for e in range(E):
+        c = len(lists[e])
+        want = O.ffn_act(X64[lists[e]], to64(Wg[e]), to64(Wu[e]))
+        np.testing.assert_allclose(hh[seg[e]:seg[e] + c], want, rtol=2 ** -7, atol=1e-6)
+        assert np.all(hh[seg[e] + c:seg[e] + (c + 127) // 128 * 128] == 0)
+
+
+# ------------------------------------------------------------------------------------ aggregation
+@pytest.mark.parametrize("mode", ["rt", "eq", "explicit"])
+def test_aggregate_matches_oracle(ctx, mode):
+    d, Lyr, slots = 384, 3, 2
+    g = _gen(21)
+    Xs = [[torch.randn((n, d), generator=g).double().numpy() for n in (50 + 10 * s, 0 if s else 80, 120)]
+          for s in range(slots)]
+    S = np.zeros((Lyr, slots, d, d), np.float32)
+    cnt = np.zeros((Lyr, slots), np.int64)
+    for s in range(slots):
+        for l in range(Lyr):
+            S[l, s] = O.gram(Xs[s][l]).astype(np.float32)
+            cnt[l, s] = Xs[s][l].shape[0]
+    acc = L.Accum(ctx, d, Lyr, slots)
+    L.clha_accum_import(ctx, acc, S, cnt)
+    Hc = torch.empty((slots, d, d), device=DEV)
+    Hd = torch.empty_like(Hc)
+    alpha = [0.7, 0.2, 0.1] if mode == "explicit" else None
+    a_out, l_out = L.clha_aggregate(ctx, acc, 0, slots, {"rt": 0, "eq": 1, "explicit": 2}[mode], alpha, 0.01, Hc, Hd,
+                                    want_host=True)
+    for s in range(slots):
+        want = O.aggregate([S[l, s].astype(np.float64) for l in range(Lyr)], list(cnt[:, s]), mode, alpha, 0.01)
+        np.testing.assert_allclose(a_out[s], want["alpha"], rtol=1e-15)
+        np.testing.assert_allclose(l_out[s], want["lam"], rtol=1e-10)
+        assert rel_fro(Hc[s].double().cpu().numpy(), want["H_comb"]) < 1e-6
+        assert rel_fro(Hd[s].double().cpu().numpy(), want["H_d"]) < 1e-6
+        assert torch.equal(Hd[s], Hd[s].T)
+
+
+# ------------------------------------------------------------------------------------ factor
+@pytest.mark.parametrize("d,batch", [(128, 1), (512, 3), (1408, 1)])
+def test_factor_matches_oracle(ctx, d, batch):
+    g = _gen(d)
+    Hs = []
+    for b in range(batch):
+        A = torch.randn((d, d // 4), generator=g).double()
+        H = (A @ A.T / (d // 4) + 0.05 * torch.eye(d, dtype=torch.float64)).float()
+        Hs.append(H)
+    Hd = torch.stack(Hs).to(DEV)
+    U = torch.full_like(Hd, float("nan"))
+    L.clha_factor(ctx, Hd, batch, d, U)
+    L.clha_check(ctx)
+    for b in range(batch):
+        want = O.factor(Hs[b].double().numpy())
+        got = U[b].double().cpu().numpy()
+        assert np.all(np.tril(got, -1) == 0)
+        assert rel_fro(got, want) < 1e-6
+
+
+def test_factor_non_pd_reports_column(ctx):
+    d = 256
+    H = torch.eye(d)
+    H[200, 200] = -1.0
+    Hd = H[None].to(DEV).contiguous()
+    U = torch.empty_like(Hd)
+    L.clha_factor(ctx, Hd, 1, d, U)
+    with pytest.raises(L.ClhaError) as ei:
+        L.clha_check(ctx)
+    assert ei.value.status == L.ERR_NOT_PD
+    assert "index 200" in str(ei.value)
+    L.clha_check(ctx)   # the error is cleared
+
+
+# ------------------------------------------------------------------------------------ GPTQ
+def _H(d, seed, rank=None, damp=0.01):
+    g = _gen(seed)
+    A = torch.randn((d, rank or d // 2), generator=g).double()
+    H = A @ A.T / A.shape[1] + torch.diag(torch.rand(d, generator=g).double() + 0.5)
+    return H.numpy()
+
+
+@pytest.mark.parametrize("d_out,d_in,bits,wdt", [(256, 512, 2, torch.float32), (384, 1024, 3, torch.bfloat16),
+                                                   (128, 128, 4, torch.bfloat16), (256, 256, 8, torch.float32)])
+def test_quantize_matches_oracle_on_same_factor(ctx, d_out, d_in, bits, wdt):
+    H = _H(d_in, d_in + bits)
+    agg = O.aggregate([H], [2], "rt")
+    U32 = O.factor(agg["H_d"]).astype(np.float32)
+    W = (0.02 * torch.randn((d_out, d_in), generator=_gen(bits))).to(wdt)
+    Ud = torch.from_numpy(U32)[None].to(DEV)
+    Wd = W[None].to(DEV).contiguous()
+    codes = torch.empty((1, d_out, d_in), dtype=torch.uint8, device=DEV)
+    scales = torch.empty((1, d_out, d_in // 128), device=DEV)
+    zeros = torch.empty((1, d_out, d_in // 128), dtype=torch.uint8, device=DEV)
+    W_hat = torch.empty((1, d_out, d_in), device=DEV)
+    L.clha_quantize(ctx, Ud, 1, Wd, 1, d_out, d_in, bits, codes, scales, zeros, W_hat)
+    wc, ws, wz, wh = O.gptq(to64(W), U32.astype(np.float64), bits, 128)
+    assert code_agreement(codes[0].cpu().numpy(), wc) >= 0.999
+    # first group of every row: identical inputs, so the grid is bit-identical
+    np.testing.assert_array_equal(scales[0, :, 0].cpu().numpy(), ws[:, 0])
+    np.testing.assert_array_equal(zeros[0, :, 0].cpu().numpy(), wz[:, 0])
+    got_loss = O.loss(to64(W), to64(W_hat[0]), agg["H_comb"])
+    want_loss = O.loss(to64(W), wh, agg["H_comb"])
+    assert abs(got_loss - want_loss) <= 1e-3 * want_loss
+    # W_hat is the dequantised code
+    q = codes[0].float()
+    s = scales[0].repeat_interleave(128, 1)
+    z = zeros[0].float().repeat_interleave(128, 1)
+    assert torch.equal(W_hat[0], s * (q - z))
+
+
+def test_quantize_diagonal_hessian_is_rtn_bit_exact(ctx):
+    d_out, d_in = 256, 384
+    W = (0.02 * torch.randn((d_out, d_in), generator=_gen(3))).to(torch.bfloat16)
+    H = np.diag(np.linspace(0.5, 2.0, d_in))
+    U = O.factor(O.aggregate([H], [2], "rt")["H_d"])
+    Ud = torch.from_numpy(U.astype(np.float32))[None].to(DEV)
+    codes = torch.empty((1, d_out, d_in), dtype=torch.uint8, device=DEV)
+    scales = torch.empty((1, d_out, d_in // 128), device=DEV)
+    zeros = torch.empty((1, d_out, d_in // 128), dtype=torch.uint8, device=DEV)
+    L.clha_quantize(ctx, Ud, 1, W[None].to(DEV).contiguous(), 1, d_out, d_in, 3, codes, scales, zeros, None)
+    wc, ws, wz, _ = O.gptq(to64(W), U.astype(np.float32).astype(np.float64), 3, 128)
+    np.testing.assert_array_equal(codes[0].cpu().numpy(), wc)
+    np.testing.assert_array_equal(scales[0].cpu().numpy(), ws)
+    np.testing.assert_array_equal(zeros[0].cpu().numpy(), wz)
+
+
+def test_quantize_batched_shared_factor(ctx):
+    """w_per_u = 2: problems 0,1 use factor 0 and problems 2,3 factor 1 (gate and up share one)."""
+    d_out, d_in, bits = 128, 256, 3
+    Us = [O.factor(O.aggregate([_H(d_in, s)], [2], "rt")["H_d"]).astype(np.float32) for s in (1, 2)]
+    W = (0.02 * torch.randn((4, d_out, d_in), generator=_gen(4))).to(torch.bfloat16)
+    Ud = torch.from_numpy(np.stack(Us)).to(DEV)
+    codes = torch.empty((4, d_out, d_in), dtype=torch.uint8, device=DEV)
+    scales = torch.empty((4, d_out, d_in // 128), device=DEV)
+    zeros = torch.empty((4, d_out, d_in // 128), dtype=torch.uint8, device=DEV)
+    L.clha_quantize(ctx, Ud, 2, W.to(DEV), 4, d_out, d_in, bits, codes, scales, zeros, None)
+    for b in range(4):
+        wc, *_ = O.gptq(to64(W[b]), Us[b // 2].astype(np.float64), bits, 128)
+        assert code_agreement(codes[b].cpu().numpy(), wc) >= 0.999
+
+
+# ------------------------------------------------------------------------------------ loss
+def test_loss_matches_oracle(ctx):
+    d_out, d_in, batch = 256, 384, 3
+    g = _gen(31)
+    W = (0.02 * torch.randn((batch, d_out, d_in), generator=g)).to(torch.bfloat16)
+    W_hat = (W.float() + 0.003 * torch.randn((batch, d_out, d_in), generator=g))
+    Hs = [_H(d_in, s) for s in (5, 6)]
+    H = torch.from_numpy(np.stack(Hs).astype(np.float32))
+    got = L.clha_loss(ctx, W.to(DEV), W_hat.to(DEV), H.to(DEV), 2, batch, d_out, d_in)
+    for b in range(batch):
+        want = O.loss(to64(W[b]), to64(W_hat[b]), H[b // 2].double().numpy())
+        assert abs(got[b] - want) <= 1e-5 * want

@@ -1,0 +1,113 @@
+"""End-to-end parity of the GPU calibration path with the float64 oracle on the seeded workloads:
+routing counts bit-exact, Hessians within 1e-4 relative Frobenius error, codes agreeing on >= 99.9%
+of entries, per-expert reconstruction loss within 1e-3 relative. Where the oracle cannot afford a
+whole workload, it checks every Hessian and a sample of experts' GPTQ end to end."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from helpers import code_agreement, rel_fro, sym_from_upper, to64
+from post_quantization_expert_b200 import clha as L
+from post_quantization_expert_b200.pipeline import DenseCalibration, MoECalibration, stack_weights
+from synth import workload
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _dense_case(ctx, cfg, **over):
+    wl = workload(cfg, "cpu", **over)
+    s = wl.spec
+    W = wl.dense_weight()
+    Xs = [wl.x(l) for l in range(s.n_layers)]
+    cal = DenseCalibration(ctx, s.d_out, s.d_model, s.n_layers, s.bits_routed, s.damp_frac)
+    for l, X in enumerate(Xs):
+        cal.collect(l, X.to(DEV))
+    alpha, lam = cal.quantize(W.to(DEV), "rt", want_host=True)
+    torch.cuda.synchronize()
+    want = O.calibrate_dense(to64(W), [to64(X) for X in Xs], s.bits_routed, s.group, "rt", None, s.damp_frac)
+    return cal, want, alpha, lam, W
+
+
+def test_dense_two_layer_fp32_workload(ctx):
+    """The dense fp32 workload: W 256x512 shared by two layers of 1000 and 1024 tokens, 2-bit."""
+    cal, want, alpha, lam, W = _dense_case(ctx, 1)
+    S, cnt = cal.acc.buffers()
+    assert cnt[:, 0].tolist() == [1000, 1024]
+    for l in range(2):
+        assert rel_fro(sym_from_upper(S[l, 0].double().cpu().numpy()), want["S"][l]) < 1e-4
+    np.testing.assert_allclose(alpha[0], [1000 / 2024, 1024 / 2024], rtol=1e-15)
+    np.testing.assert_allclose(lam[0], want["lam"], rtol=1e-5)
+    assert rel_fro(cal.H_comb[0].double().cpu().numpy(), want["H_comb"]) < 1e-4
+    assert rel_fro(cal.U[0].double().cpu().numpy(), want["U"]) < 1e-4
+    assert code_agreement(cal.q.codes[0].cpu().numpy(), want["codes"]) >= 0.999
+    assert abs(cal.q.loss[0] - want["loss"]) <= 1e-3 * want["loss"]
+
+
+def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, **over):
+    wl = workload(cfg, "cpu", **over)
+    s = wl.spec
+    Xs = [wl.x(l) for l in range(2)]
+    lgs = [wl.logits(l) for l in range(2)]
+    routed = [wl.expert_weights(0, e) for e in range(s.E)]
+    shared = [wl.expert_weights(0, i, shared=True) for i in range(s.n_shared)]
+    w = stack_weights((routed, shared), DEV)
+    cal = MoECalibration(ctx, 2, max(s.tokens), s.E, s.k, s.d_model, s.d_ff, s.n_shared, s.shared_dff,
+                         s.bits_routed, s.bits_shared, s.damp_frac)
+    for l in range(2):
+        cal.collect(l, Xs[l].to(DEV), lgs[l].to(DEV), w)
+    torch.cuda.synchronize()
+    X64 = [to64(X) for X in Xs]
+    # routing counts: bit-exact
+    routes = [O.route_topk(lg.numpy(), s.k) for lg in lgs]
+    for l in range(2):
+        np.testing.assert_array_equal(cal.counts[l].cpu().numpy(), routes[l][1])
+    # every routed expert's input Hessian, both layers
+    S_in, n_in = cal.acc_in.buffers()
+    S_dn, _ = cal.acc_dn.buffers()
+    toks = [O.expert_tokens(r[0], s.E) for r in routes]
+    for l in range(2):
+        for e in range(s.E):
+            assert n_in[l, e].item() == len(toks[l][e])
+            got = sym_from_upper(S_in[l, e].double().cpu().numpy())
+            assert rel_fro(got, O.gram(X64[l][toks[l][e]])) < 1e-4
+    if s.n_shared:
+        for l in range(2):
+            assert rel_fro(sym_from_upper(S_in[l, s.E].double().cpu().numpy()), O.gram(X64[l])) < 1e-4
+    # sampled experts: down-projection Hessians and the whole GPTQ path, per weighting
+    ref = {}
+    for mode in modes:
+        cal.quantize(w, mode)
+        torch.cuda.synchronize()
+        res = O.calibrate_moe_group(X64, [lg.numpy() for lg in lgs], s.k, [tuple(to64(t) for t in r) for r in routed],
+                                    [tuple(to64(t) for t in sh) for sh in shared], experts_checked,
+                                    s.bits_routed, s.bits_shared, s.group, mode, s.damp_frac, shared_checked)
+        for key, r in res["experts"].items():
+            kind, e = key
+            if kind == "r":
+                for l in range(2):
+                    got = sym_from_upper(S_dn[l, e].double().cpu().numpy())
+                    assert rel_fro(got, r["down"]["S"][l]) < 1e-4, (mode, key, l)
+                qs = {"gate": cal.qg, "up": cal.qu, "down": cal.qd}
+            else:
+                qs = {"gate": cal.sg, "up": cal.su, "down": cal.sd}
+            for name, q in qs.items():
+                agree = code_agreement(q.codes[e].cpu().numpy(), r[name]["codes"])
+                assert agree >= 0.999, (mode, key, name, agree)
+            got_loss = sum(qs[n].loss[e] for n in ("gate", "up", "down"))
+            assert abs(got_loss - r["loss"]) <= 1e-3 * r["loss"], (mode, key, got_loss, r["loss"])
+        ref[mode] = res
+    return cal, ref
+
+
+def test_moe_pair_E16_top2_full_size(ctx):
+    """The E=16, top-2, d_model 1024, d_ff 512 layer pair at 8192 tokens per layer, 3-bit, both
+    weightings: all Hessians and routing checked; GPTQ end to end on experts 0, 7 and 15."""
+    _moe_pair(ctx, 2, [0, 7, 15], ("rt", "eq"))
+
+
+def test_moe_pair_E64_top6_shared_reduced_tokens(ctx):
+    """The E=64 top-6 shape with two always-active experts (CLHA-MP: routed 2-bit, shared 3-bit),
+    Zipf-skewed routing and outlier channels, at 4096 tokens per layer."""
+    _moe_pair(ctx, 3, [0, 63], ("rt",), shared_checked=[1], tokens=4096)
