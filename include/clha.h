@@ -150,7 +150,7 @@ CLHA_API clha_status clha_collect(clha_ctx* ctx, clha_accum* acc, int layer, con
  * alpha_out (host double [n_slots * n_layers]) and lambda_out (host double [n_slots]) are optional;
  * passing either synchronises. A slot with no tokens in any layer gives CLHA_ERR_EMPTY. */
 CLHA_API clha_status clha_aggregate(clha_ctx* ctx, const clha_accum* acc, int slot0, int n_slots,
-                           clha_alpha_mode mode, const double* alpha_in, float damp_frac,
+                           clha_alpha_mode mode, const double* alpha_in, double damp_frac,
                            float* H_comb, float* H_damped, double* alpha_out, double* lambda_out);
 
 /* ------------------------------------------------------------------------------ phase 3: quantization */

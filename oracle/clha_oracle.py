@@ -244,8 +244,9 @@ def calibrate_moe_group(X_list, logits_list, k: int, routed, shared=(), experts=
     experts `shared` (CLHA page §2.2 phases 1-3, §2.3 mixed precision, §2.4 per-layer accumulators).
 
     experts / shared_experts: which routed / always-active experts to calibrate (default: all).
-    Returns per-layer routing and, per expert key ("r", e) / ("s", e), counts, alphas and the GPTQ
-    results of gate/up (input Hessian over x) and down (input Hessian over h).
+    Returns per-layer routing and, per expert key ("r", e) / ("s", e): token counts "n", the Hessian
+    data "H_in" (gate/up inputs x) and "H_down" (down-projection inputs h), and the GPTQ results
+    "gate", "up", "down".
     """
     E = len(routed)
     if experts is None:
@@ -263,7 +264,7 @@ def calibrate_moe_group(X_list, logits_list, k: int, routed, shared=(), experts=
         he = [ffn_act(x, Wg, Wu) for x in Xe]
         n = [len(t) for t in tok_l]
         res = {"n": n}
-        for kind, inputs, mats in (("in", Xe, (("gate", Wg), ("up", Wu))), ("down", he, (("down", Wd),))):
+        for kind, inputs, mats in (("H_in", Xe, (("gate", Wg), ("up", Wu))), ("H_down", he, (("down", Wd),))):
             S = [gram(x) for x in inputs]
             agg = aggregate(S, n, mode, None, damp_frac)
             U = factor(agg["H_d"])

@@ -10,6 +10,7 @@ from __future__ import annotations
 
 import ctypes as C
 import os
+import sys
 
 import numpy as np
 import torch
@@ -74,7 +75,7 @@ def load(path: str = LIB_PATH):
         "clha_accum_export": (i32, [vp, vp, vp, vp]),
         "clha_accum_import": (i32, [vp, vp, vp, vp]),
         "clha_collect": (i32, [vp, vp, i32, vp, i32, i64, i32, vp, i32, i32]),
-        "clha_aggregate": (i32, [vp, vp, i32, i32, i32, vp, f32, vp, vp, vp, vp]),
+        "clha_aggregate": (i32, [vp, vp, i32, i32, i32, vp, f64, vp, vp, vp, vp]),
         "clha_factor": (i32, [vp, vp, i32, i32, vp]),
         "clha_quantize": (i32, [vp, vp, i32, vp, i32, i32, i32, i32, C.POINTER(QuantParams), vp, vp, vp, vp]),
         "clha_loss": (i32, [vp, vp, i32, vp, vp, i32, i32, i32, i32, vp]),
@@ -92,8 +93,12 @@ def _p(t):
     if t is None:
         return None
     if isinstance(t, torch.Tensor):
+        if not t.is_contiguous():
+            raise ValueError("libclha takes dense row-major arrays; got a non-contiguous tensor")
         return t.data_ptr()
     if isinstance(t, np.ndarray):
+        if not t.flags["C_CONTIGUOUS"]:
+            raise ValueError("libclha takes dense row-major arrays; got a non-C-contiguous ndarray")
         return t.ctypes.data
     raise TypeError(type(t))
 
@@ -128,7 +133,9 @@ class Context:
             load().clha_destroy(self.handle)
             self.handle = None
 
-    __del__ = close
+    def __del__(self):
+        if not sys.is_finalizing():
+            self.close()
 
 
 def clha_version() -> int:
@@ -181,7 +188,9 @@ class Accum:
             load().clha_accum_destroy(self.handle)
             self.handle = None
 
-    __del__ = close
+    def __del__(self):
+        if not sys.is_finalizing():
+            self.close()
 
 
 def _wrap(ptr: int, shape, dtype, device):

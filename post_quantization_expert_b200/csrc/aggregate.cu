@@ -18,7 +18,7 @@ __device__ __forceinline__ double layer_coef(const double* alpha, const int64_t*
 
 __global__ void __launch_bounds__(256) agg_scalars(const float* __restrict__ S, const int64_t* __restrict__ counts,
                                                    int d, int L, int n_slots_total, int slot0, clha_alpha_args a,
-                                                   float damp_frac, double* __restrict__ d_alpha,
+                                                   double damp_frac, double* __restrict__ d_alpha,
                                                    double* __restrict__ d_lambda, int* err) {
     const int sl = blockIdx.x;
     const int slot = slot0 + sl;
@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(256) agg_scalars(const float* __restrict__ S, 
         __syncthreads();
     }
     if (threadIdx.x == 0) {
-        double lam = (double)damp_frac * red[0] / d;
+        double lam = damp_frac * red[0] / d;
         d_lambda[sl] = lam;
         if (!isfinite(red[0])) clha_record_error(err, CLHA_ERR_NONFINITE, slot, -1, KID_AGGREGATE);
     }
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(256) agg_combine(const float* __restrict__ S, 
 }  // namespace
 
 cudaError_t launch_aggregate(cudaStream_t s, const float* S, const int64_t* counts, int d, int n_layers,
-                             int n_slots_total, int slot0, int n_slots, clha_alpha_args a, float damp_frac,
+                             int n_slots_total, int slot0, int n_slots, clha_alpha_args a, double damp_frac,
                              float* H_comb, float* H_d, double* d_alpha, double* d_lambda, int* err) {
     agg_scalars<<<n_slots, 256, 0, s>>>(S, counts, d, n_layers, n_slots_total, slot0, a, damp_frac, d_alpha, d_lambda,
                                         err);

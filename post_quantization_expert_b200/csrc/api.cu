@@ -243,7 +243,7 @@ extern "C" clha_status clha_accum_create(clha_ctx* ctx, int d, int n_layers, int
     SET_DEVICE(ctx);
     clha_accum* acc = new (std::nothrow) clha_accum();
     if (!acc) return CLHA_ERR_OOM;
-    acc->ctx = ctx;
+    acc->device = ctx->device;
     acc->d = d;
     acc->n_layers = n_layers;
     acc->n_slots = n_slots;
@@ -262,8 +262,8 @@ extern "C" clha_status clha_accum_create(clha_ctx* ctx, int d, int n_layers, int
 
 extern "C" clha_status clha_accum_destroy(clha_accum* acc) {
     if (!acc) return CLHA_OK;
-    cudaSetDevice(acc->ctx->device);
-    cudaStreamSynchronize(acc->ctx->stream);
+    cudaSetDevice(acc->device);
+    cudaDeviceSynchronize();  // work still queued on any stream may reference the buffers
     cudaFree(acc->S);
     cudaFree(acc->counts);
     delete acc;
@@ -340,7 +340,7 @@ extern "C" clha_status clha_collect(clha_ctx* ctx, clha_accum* acc, int layer, c
 
 // ------------------------------------------------------------------------------ phase 2
 extern "C" clha_status clha_aggregate(clha_ctx* ctx, const clha_accum* acc, int slot0, int n_slots,
-                                      clha_alpha_mode mode, const double* alpha_in, float damp_frac,
+                                      clha_alpha_mode mode, const double* alpha_in, double damp_frac,
                                       float* H_comb, float* H_damped, double* alpha_out, double* lambda_out) {
     CHECK_CTX(ctx);
     REQUIRE(acc && H_damped, CLHA_ERR_INVALID_ARG, "clha_aggregate: null pointer");
@@ -349,7 +349,7 @@ extern "C" clha_status clha_aggregate(clha_ctx* ctx, const clha_accum* acc, int 
     REQUIRE(mode == CLHA_ALPHA_ROUTING || mode == CLHA_ALPHA_EQUAL || mode == CLHA_ALPHA_EXPLICIT,
             CLHA_ERR_INVALID_ARG, "clha_aggregate: unknown alpha mode");
     REQUIRE(mode != CLHA_ALPHA_EXPLICIT || alpha_in, CLHA_ERR_INVALID_ARG, "clha_aggregate: explicit alpha needs alpha_in");
-    REQUIRE(damp_frac > 0.f && damp_frac == damp_frac, CLHA_ERR_INVALID_ARG, "clha_aggregate: damp_frac must be > 0");
+    REQUIRE(damp_frac > 0.0 && damp_frac == damp_frac, CLHA_ERR_INVALID_ARG, "clha_aggregate: damp_frac must be > 0");
     SET_DEVICE(ctx);
     LaunchScope launch_scope(ctx);
     clha_alpha_args a;

@@ -27,7 +27,7 @@ struct clha_ctx {
 };
 
 struct clha_accum {
-    clha_ctx* ctx = nullptr;
+    int device = 0;
     int d = 0, n_layers = 0, n_slots = 0;
     float* S = nullptr;        // [n_layers][n_slots][d][d]
     int64_t* counts = nullptr; // [n_layers][n_slots]
@@ -93,7 +93,7 @@ struct clha_alpha_args {
 };
 cudaError_t launch_aggregate(cudaStream_t s, const float* S, const int64_t* counts, int d,
                              int n_layers, int n_slots_total, int slot0, int n_slots,
-                             clha_alpha_args a, float damp_frac, float* H_comb, float* H_d,
+                             clha_alpha_args a, double damp_frac, float* H_comb, float* H_d,
                              double* d_alpha, double* d_lambda, int* err);
 size_t factor_workspace_bytes(int batch, int d);
 cudaError_t launch_factor(cudaStream_t s, const float* H_d, int batch, int d, float* U,

@@ -5,6 +5,10 @@
 //
 // Shared-memory tiled FMA kernel: a 64-row x 64-column output tile computes the gate and the up
 // tile together (two accumulators per thread), so the SiLU-times-up epilogue needs no second pass.
+// Products of bf16 values are exact in fp32; each 32-term chunk is summed in fp32 and the chunk sums
+// in fp64, which keeps the rounding of h to bf16 at the correctly rounded value far more often than
+// one long fp32 sum would (inputs with outlier channels cancel heavily); the SiLU product is
+// evaluated in fp64 and rounded once to bf16.
 #include "clha_internal.h"
 
 namespace {
@@ -40,7 +44,7 @@ __global__ void __launch_bounds__(256) expert_act_simt(const __nv_bfloat16* __re
     __shared__ float Gs[TK][TN + 4];
     __shared__ float Us[TK][TN + 4];
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    float ag[4][4] = {}, au[4][4] = {};
+    double ag[4][4] = {}, au[4][4] = {};
     for (int k0 = 0; k0 < dm; k0 += TK) {
         for (int i = threadIdx.x; i < TM * TK; i += 256) {
             int m = i / TK, kk = i % TK;
@@ -50,6 +54,7 @@ __global__ void __launch_bounds__(256) expert_act_simt(const __nv_bfloat16* __re
             Us[kk][m] = __bfloat162float(wu[(size_t)(n0 + m) * dm + k0 + kk]);
         }
         __syncthreads();
+        float pg[4][4] = {}, pu[4][4] = {};
 #pragma unroll 8
         for (int kk = 0; kk < TK; ++kk) {
             float a[4], g[4], u[4];
@@ -63,10 +68,17 @@ __global__ void __launch_bounds__(256) expert_act_simt(const __nv_bfloat16* __re
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    ag[i][j] = fmaf(a[i], g[j], ag[i][j]);
-                    au[i][j] = fmaf(a[i], u[j], au[i][j]);
+                    pg[i][j] = fmaf(a[i], g[j], pg[i][j]);
+                    pu[i][j] = fmaf(a[i], u[j], pu[i][j]);
                 }
         }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                ag[i][j] += (double)pg[i][j];
+                au[i][j] += (double)pu[i][j];
+            }
         __syncthreads();
     }
 #pragma unroll
@@ -76,9 +88,9 @@ __global__ void __launch_bounds__(256) expert_act_simt(const __nv_bfloat16* __re
         bool valid = row < valid_end;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            float g = ag[i][j];
-            float v = valid ? g / (1.f + expf(-g)) * au[i][j] : 0.f;
-            h[row * dff + n0 + tx * 4 + j] = __float2bfloat16_rn(v);
+            const double g = ag[i][j];
+            const double v = valid ? g / (1.0 + exp(-g)) * au[i][j] : 0.0;
+            h[row * dff + n0 + tx * 4 + j] = __double2bfloat16(v);
         }
     }
 }

@@ -173,7 +173,7 @@ def test_expert_act_dense(ctx, rows, dm, dff):
     want = O.ffn_act(to64(X), to64(Wg[0]), to64(Wu[0]))
     got = to64(h)
     exact = np.mean(got == want)
-    assert exact > 0.995
+    assert exact >= 0.999
     np.testing.assert_allclose(got, want, rtol=2 ** -7, atol=1e-6)
 
 
@@ -280,7 +280,7 @@ def _H(d, seed, rank=None, damp=0.01):
 def test_quantize_matches_oracle_on_same_factor(ctx, d_out, d_in, bits, wdt):
     H = _H(d_in, d_in + bits)
     agg = O.aggregate([H], [2], "rt")
-    U32 = O.factor(agg["H_d"]).astype(np.float32)
+    U32 = np.ascontiguousarray(O.factor(agg["H_d"]), np.float32)
     W = (0.02 * torch.randn((d_out, d_in), generator=_gen(bits))).to(wdt)
     Ud = torch.from_numpy(U32)[None].to(DEV)
     Wd = W[None].to(DEV).contiguous()
@@ -309,7 +309,7 @@ def test_quantize_diagonal_hessian_is_rtn_bit_exact(ctx):
     W = (0.02 * torch.randn((d_out, d_in), generator=_gen(3))).to(torch.bfloat16)
     H = np.diag(np.linspace(0.5, 2.0, d_in))
     U = O.factor(O.aggregate([H], [2], "rt")["H_d"])
-    Ud = torch.from_numpy(U.astype(np.float32))[None].to(DEV)
+    Ud = torch.from_numpy(np.ascontiguousarray(U, np.float32))[None].to(DEV)
     codes = torch.empty((1, d_out, d_in), dtype=torch.uint8, device=DEV)
     scales = torch.empty((1, d_out, d_in // 128), device=DEV)
     zeros = torch.empty((1, d_out, d_in // 128), dtype=torch.uint8, device=DEV)
@@ -323,7 +323,7 @@ def test_quantize_diagonal_hessian_is_rtn_bit_exact(ctx):
 def test_quantize_batched_shared_factor(ctx):
     """w_per_u = 2: problems 0,1 use factor 0 and problems 2,3 factor 1 (gate and up share one)."""
     d_out, d_in, bits = 128, 256, 3
-    Us = [O.factor(O.aggregate([_H(d_in, s)], [2], "rt")["H_d"]).astype(np.float32) for s in (1, 2)]
+    Us = [np.ascontiguousarray(O.factor(O.aggregate([_H(d_in, s)], [2], "rt")["H_d"]), np.float32) for s in (1, 2)]
     W = (0.02 * torch.randn((4, d_out, d_in), generator=_gen(4))).to(torch.bfloat16)
     Ud = torch.from_numpy(np.stack(Us)).to(DEV)
     codes = torch.empty((4, d_out, d_in), dtype=torch.uint8, device=DEV)

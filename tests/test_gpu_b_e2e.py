@@ -88,7 +88,7 @@ def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, **over):
             if kind == "r":
                 for l in range(2):
                     got = sym_from_upper(S_dn[l, e].double().cpu().numpy())
-                    assert rel_fro(got, r["down"]["S"][l]) < 1e-4, (mode, key, l)
+                    assert rel_fro(got, r["H_down"]["S"][l]) < 1e-4, (mode, key, l)
                 qs = {"gate": cal.qg, "up": cal.qu, "down": cal.qd}
             else:
                 qs = {"gate": cal.sg, "up": cal.su, "down": cal.sd}
