@@ -108,6 +108,22 @@ CLHA_API clha_status clha_gather(clha_ctx* ctx, const void* X, clha_dtype dtype,
                         const int32_t* ids, int k, int E, void* X_packed, int64_t packed_rows,
                         int64_t* seg, int32_t* perm);
 
+/* clha_gather without any device allocation; the paper has no counterpart (it is a service for
+ * callers, not part of the method). Same arguments, layout and results as clha_gather. It exists for
+ * callers that must not see the library allocate device memory: processes whose memory is handed
+ * out by their own allocator (a framework's caching allocator, a fixed arena), where a cudaMalloc
+ * can fail once the arena holds the memory and a cudaFree synchronises the whole device.
+ * Its scratch (block histograms and the token permutation, clha_gather's workspace) is a fixed
+ * 4 MiB array in the library's device image, which every GPU that loads the library holds until
+ * the process exits. A gather whose scratch exceeds it (roughly n*k + 128*E above ~1M rows) is
+ * rejected with CLHA_ERR_INVALID_ARG before anything is queued. The first call on a device looks up
+ * the array's device address (cudaGetSymbolAddress) with that device current, and caches it; make
+ * that first call before any stream capture. All calls share the array and it keeps the last
+ * call's contents (each call rewrites what it reads); calls that overlap on the GPU race on it. */
+CLHA_API clha_status clha_gather_noalloc(clha_ctx* ctx, const void* X, clha_dtype dtype, int64_t n, int d,
+                                         const int32_t* ids, int k, int E, void* X_packed, int64_t packed_rows,
+                                         int64_t* seg, int32_t* perm);
+
 /* Expert FFN activation feeding the down projection: h = SiLU(x Wg^T) * (x Wu^T) per token of
  * each expert, accumulated in float32 and stored as bf16 (round to nearest even). The pages do not
  * spell this out: the down projection's Hessian needs its input, and that input is this product.

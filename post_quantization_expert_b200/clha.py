@@ -26,7 +26,7 @@ ALPHA_ROUTING, ALPHA_EQUAL, ALPHA_EXPLICIT = 0, 1, 2
 # every symbol include/clha.h declares
 SYMBOLS = [
     "clha_create", "clha_destroy", "clha_last_error", "clha_check", "clha_version", "clha_kernel_launches",
-    "clha_route_topk", "clha_packed_rows", "clha_gather", "clha_expert_act",
+    "clha_route_topk", "clha_packed_rows", "clha_gather", "clha_gather_noalloc", "clha_expert_act",
     "clha_accum_create", "clha_accum_destroy", "clha_accum_zero", "clha_accum_buffers",
     "clha_accum_export", "clha_accum_import", "clha_collect",
     "clha_aggregate", "clha_factor", "clha_quantize", "clha_loss",
@@ -67,6 +67,7 @@ def load(path: str = LIB_PATH):
         "clha_route_topk": (i32, [vp, vp, i64, i32, i32, vp, vp]),
         "clha_packed_rows": (i64, [i64, i32, i32]),
         "clha_gather": (i32, [vp, vp, i32, i64, i32, vp, i32, i32, vp, i64, vp, vp]),
+        "clha_gather_noalloc": (i32, [vp, vp, i32, i64, i32, vp, i32, i32, vp, i64, vp, vp]),
         "clha_expert_act": (i32, [vp, vp, i64, i32, vp, i32, vp, vp, i32, vp]),
         "clha_accum_create": (i32, [vp, i32, i32, i32, C.POINTER(vp)]),
         "clha_accum_destroy": (i32, [vp]),
@@ -161,6 +162,13 @@ def clha_packed_rows(n: int, k: int, E: int) -> int:
 def clha_gather(ctx: Context, X, n: int, d: int, ids, k: int, E: int, X_packed, packed_rows: int, seg, perm=None):
     ctx._check(load().clha_gather(ctx.handle, _p(X), _dtype(X), n, d, _p(ids), k, E, _p(X_packed), packed_rows,
                                   _p(seg), _p(perm)))
+
+
+def clha_gather_noalloc(ctx: Context, X, n: int, d: int, ids, k: int, E: int, X_packed, packed_rows: int, seg,
+                        perm=None):
+    """clha_gather with its scratch in the library's fixed device array (no allocation)."""
+    ctx._check(load().clha_gather_noalloc(ctx.handle, _p(X), _dtype(X), n, d, _p(ids), k, E, _p(X_packed),
+                                          packed_rows, _p(seg), _p(perm)))
 
 
 def clha_expert_act(ctx: Context, X, rows: int, d_model: int, seg, E: int, Wg, Wu, d_ff: int, h):
