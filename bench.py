@@ -202,9 +202,9 @@ def run_ours(args, world, rank, local):
     w = stack_weights((routed, []), dev)
     Xd = [x.to(dev) for x in X]
     Ld = [l.to(dev) for l in lg]
-    cal = MoECalibration(ctx, 2, max(s.tokens), s.E, s.k, s.d_model, s.d_ff, 0, 0, s.bits_routed, s.bits_shared,
-                         s.damp_frac, timer=timer)
     modes = s.alpha_modes
+    cal = MoECalibration(ctx, 2, max(s.tokens), s.E, s.k, s.d_model, s.d_ff, 0, 0, s.bits_routed, s.bits_shared,
+                         s.damp_frac, timer=timer, modes=modes)
     cols_per_step = cal.columns() * len(modes)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
 
@@ -212,8 +212,7 @@ def run_ours(args, world, rank, local):
         cal.reset()
         for l in range(2):
             cal.collect(l, Xd[l], Ld[l], w)
-        for m in modes:
-            cal.quantize(w, m)
+        cal.quantize(w, modes)
 
     timer.enabled = False
     for _ in range(args.warmup):
@@ -247,24 +246,24 @@ def run_ours(args, world, rank, local):
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
     pin = lambda t: t.pin_memory()
     hX, hL = [pin(x) for x in X], [pin(l) for l in lg]
-    hW = [pin(w.Wg.cpu()), pin(w.Wu.cpu()), pin(w.Wd.cpu())]
-    outs = [cal.qg, cal.qu, cal.qd]
+    hW = [pin(w.Wgu.cpu()), pin(w.Wd.cpu())]
+    outs = {m: [cal.res[m].qgu, cal.res[m].qd] for m in modes}
     hout = {m: [(pin(torch.empty_like(q.codes, device="cpu")), pin(torch.empty_like(q.scales, device="cpu")),
-                 pin(torch.empty_like(q.zeros, device="cpu"))) for q in outs] for m in modes}
+                 pin(torch.empty_like(q.zeros, device="cpu"))) for q in outs[m]] for m in modes}
     h2d = sum(t.numel() * t.element_size() for t in hX + hL + hW)
     d2h = sum(t.numel() * t.element_size() for m in modes for trip in hout[m] for t in trip)
     timer.enabled = False
 
     def e2e_step():
         with torch.cuda.stream(stream):
-            for d_, h_ in zip(Xd + Ld + [w.Wg, w.Wu, w.Wd], hX + hL + hW):
+            for d_, h_ in zip(Xd + Ld + [w.Wgu, w.Wd], hX + hL + hW):
                 d_.copy_(h_, non_blocking=True)
             cal.reset()
             for l in range(2):
                 cal.collect(l, Xd[l], Ld[l], w)
+            cal.quantize(w, modes)
             for m in modes:
-                cal.quantize(w, m)
-                for q, (hc, hs, hz) in zip(outs, hout[m]):
+                for q, (hc, hs, hz) in zip(outs[m], hout[m]):
                     hc.copy_(q.codes, non_blocking=True)
                     hs.copy_(q.scales, non_blocking=True)
                     hz.copy_(q.zeros, non_blocking=True)

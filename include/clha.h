@@ -164,10 +164,12 @@ CLHA_API clha_status clha_collect(clha_ctx* ctx, clha_accum* acc, int layer, con
  * lambda = damp_frac * mean(diag H_comb) and H_damped = H_comb + lambda I.
  * H_comb and H_damped are float32 [n_slots, d, d], full symmetric. H_comb may be NULL.
  * alpha_out (host double [n_slots * n_layers]) and lambda_out (host double [n_slots]) are optional;
- * passing either synchronises. A slot with no tokens in any layer gives CLHA_ERR_EMPTY. */
+ * passing either synchronises. lambda_dev (device double [n_slots], optional) receives lambda without
+ * synchronising, for clha_quantize's loss. A slot with no tokens in any layer gives CLHA_ERR_EMPTY. */
 CLHA_API clha_status clha_aggregate(clha_ctx* ctx, const clha_accum* acc, int slot0, int n_slots,
                            clha_alpha_mode mode, const double* alpha_in, double damp_frac,
-                           float* H_comb, float* H_damped, double* alpha_out, double* lambda_out);
+                           float* H_comb, float* H_damped, double* alpha_out, double* lambda_out,
+                           double* lambda_dev);
 
 /* ------------------------------------------------------------------------------ phase 3: quantization */
 
@@ -179,24 +181,34 @@ CLHA_API clha_status clha_aggregate(clha_ctx* ctx, const clha_accum* acc, int sl
 CLHA_API clha_status clha_factor(clha_ctx* ctx, const float* H_damped, int batch, int d, float* U);
 
 /* GPTQ (CLHA page §2.2 (3)): column-sequential quantization of `batch` weights W [batch, d_out, d_in]
- * (bf16 or f32) in natural column order, with lazy updates over 128-column blocks. Problem b uses
- * U + (b / w_per_u) * d_in * d_in (w_per_u >= 1 lets, e.g., gate and up share one factor).
+ * (bf16 or f32) in natural column order, with lazy updates over 128-column blocks. U holds n_u
+ * factors [n_u, d_in, d_in] and problem b uses factor b % n_u (1 <= n_u <= batch; with gate and up
+ * stacked as [2E] and n_u = E they share their expert's factor).
  * At the start of each group of 128 columns a row's grid is fixed from its current values:
  * xmin = min(0, min w), xmax = max(0, max w) ([-1, 1] if both are 0), s = (xmax - xmin)/(2^b - 1),
  * z = round(-xmin/s); each column then takes q = clamp(round(w/s) + z, 0, 2^b - 1), w_hat = s (q - z),
  * and its error (w - w_hat)/U_jj is subtracted along row j of U from the later columns. The grid and
- * the code are decided in IEEE float32 (round to nearest even); the updates accumulate in float32.
+ * the code are decided in IEEE float32 (round to nearest even); the updates inside a block accumulate
+ * in float32 and the lazy block updates run on the tensor cores in three tf32 products (hi*hi +
+ * hi*lo + lo*hi), float32-class accuracy.
  * Outputs: codes uint8 [batch, d_out, d_in], scales float32 and zeros uint8 [batch, d_out, d_in/128],
- * W_hat float32 [batch, d_out, d_in] (may be NULL). */
-CLHA_API clha_status clha_quantize(clha_ctx* ctx, const float* U, int w_per_u, const void* W, clha_dtype dtype,
+ * W_hat float32 [batch, d_out, d_in] (may be NULL).
+ * Optional loss (device double [batch], overwritten), given lambda (device double [n_u], the damping of
+ * each factor, e.g. clha_aggregate's lambda_dev): the CLHA page §2.1 term tr[(W_hat - W) H_comb
+ * (W_hat - W)^T] of each problem, from GPTQ's own errors e: W - W_hat = E U and U H_d U^T = I give
+ * tr[D H_d D^T] = |E|^2, and H_comb = H_d - lambda I gives loss = |E|^2 - lambda |W_hat - W|^2
+ * (summed in float64). Pass NULL for both to skip it; clha_loss scores any other H. */
+CLHA_API clha_status clha_quantize(clha_ctx* ctx, const float* U, int n_u, const void* W, clha_dtype dtype,
                           int batch, int d_out, int d_in, const clha_quant_params* params,
-                          uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat);
+                          uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
+                          const double* lambda, double* loss);
 
 /* Loss of the CLHA page §2.1, one term: loss_out[b] = tr[(W_hat - W) H (W_hat - W)^T] for `batch`
- * problems; problem b uses H + (b / w_per_h) * d_in * d_in. Accumulated in float64.
+ * problems; H holds n_h matrices and problem b uses H[b % n_h] (1 <= n_h <= batch). Tile sums are
+ * added in float64.
  * loss_out is a host double [batch] array (synchronises). */
 CLHA_API clha_status clha_loss(clha_ctx* ctx, const void* W, clha_dtype dtype, const float* W_hat,
-                      const float* H, int w_per_h, int batch, int d_out, int d_in, double* loss_out);
+                      const float* H, int n_h, int batch, int d_out, int d_in, double* loss_out);
 
 #ifdef __cplusplus
 }

@@ -76,9 +76,10 @@ def load(path: str = LIB_PATH):
         "clha_accum_export": (i32, [vp, vp, vp, vp]),
         "clha_accum_import": (i32, [vp, vp, vp, vp]),
         "clha_collect": (i32, [vp, vp, i32, vp, i32, i64, i32, vp, i32, i32]),
-        "clha_aggregate": (i32, [vp, vp, i32, i32, i32, vp, f64, vp, vp, vp, vp]),
+        "clha_aggregate": (i32, [vp, vp, i32, i32, i32, vp, f64, vp, vp, vp, vp, vp]),
         "clha_factor": (i32, [vp, vp, i32, i32, vp]),
-        "clha_quantize": (i32, [vp, vp, i32, vp, i32, i32, i32, i32, C.POINTER(QuantParams), vp, vp, vp, vp]),
+        "clha_quantize": (i32, [vp, vp, i32, vp, i32, i32, i32, i32, C.POINTER(QuantParams), vp, vp, vp, vp, vp,
+                                vp]),
         "clha_loss": (i32, [vp, vp, i32, vp, vp, i32, i32, i32, i32, vp]),
     }
     for name, (res, args) in sig.items():
@@ -135,7 +136,7 @@ class Context:
             self.handle = None
 
     def __del__(self):
-        if not sys.is_finalizing():
+        if sys is not None and not sys.is_finalizing():
             self.close()
 
 
@@ -197,7 +198,7 @@ class Accum:
             self.handle = None
 
     def __del__(self):
-        if not sys.is_finalizing():
+        if sys is not None and not sys.is_finalizing():
             self.close()
 
 
@@ -244,13 +245,14 @@ def clha_collect(ctx: Context, acc: Accum, layer: int, X, rows: int, d: int, seg
 
 
 def clha_aggregate(ctx: Context, acc: Accum, slot0: int, n_slots: int, mode: int, alpha_in=None,
-                   damp_frac: float = 0.01, H_comb=None, H_damped=None, want_host: bool = False):
-    """Returns (alpha [n_slots, L], lambda [n_slots]) as numpy when want_host, else None."""
+                   damp_frac: float = 0.01, H_comb=None, H_damped=None, want_host: bool = False, lambda_dev=None):
+    """Returns (alpha [n_slots, L], lambda [n_slots]) as numpy when want_host, else None. lambda_dev
+    (float64 device tensor [n_slots]) receives lambda without a synchronisation."""
     a_in = None if alpha_in is None else np.ascontiguousarray(alpha_in, np.float64)
     a_out = np.empty((n_slots, acc.n_layers), np.float64) if want_host else None
     l_out = np.empty(n_slots, np.float64) if want_host else None
     ctx._check(load().clha_aggregate(ctx.handle, acc.handle, slot0, n_slots, mode, _p(a_in), damp_frac, _p(H_comb),
-                                     _p(H_damped), _p(a_out), _p(l_out)))
+                                     _p(H_damped), _p(a_out), _p(l_out), _p(lambda_dev)))
     return (a_out, l_out) if want_host else None
 
 
@@ -258,14 +260,15 @@ def clha_factor(ctx: Context, H_damped, batch: int, d: int, U):
     ctx._check(load().clha_factor(ctx.handle, _p(H_damped), batch, d, _p(U)))
 
 
-def clha_quantize(ctx: Context, U, w_per_u: int, W, batch: int, d_out: int, d_in: int, bits: int, codes, scales,
-                  zeros, W_hat=None, group: int = 128, block: int = 128, damp_frac: float = 0.01):
+def clha_quantize(ctx: Context, U, n_u: int, W, batch: int, d_out: int, d_in: int, bits: int, codes, scales,
+                  zeros, W_hat=None, group: int = 128, block: int = 128, damp_frac: float = 0.01, lam=None, loss=None):
+    """lam (float64 device [n_u]) and loss (float64 device [batch]) request the in-kernel loss."""
     qp = QuantParams(bits, group, block, damp_frac)
-    ctx._check(load().clha_quantize(ctx.handle, _p(U), w_per_u, _p(W), _dtype(W), batch, d_out, d_in, C.byref(qp),
-                                    _p(codes), _p(scales), _p(zeros), _p(W_hat)))
+    ctx._check(load().clha_quantize(ctx.handle, _p(U), n_u, _p(W), _dtype(W), batch, d_out, d_in, C.byref(qp),
+                                    _p(codes), _p(scales), _p(zeros), _p(W_hat), _p(lam), _p(loss)))
 
 
-def clha_loss(ctx: Context, W, W_hat, H, w_per_h: int, batch: int, d_out: int, d_in: int) -> np.ndarray:
+def clha_loss(ctx: Context, W, W_hat, H, n_h: int, batch: int, d_out: int, d_in: int) -> np.ndarray:
     out = np.empty(batch, np.float64)
-    ctx._check(load().clha_loss(ctx.handle, _p(W), _dtype(W), _p(W_hat), _p(H), w_per_h, batch, d_out, d_in, _p(out)))
+    ctx._check(load().clha_loss(ctx.handle, _p(W), _dtype(W), _p(W_hat), _p(H), n_h, batch, d_out, d_in, _p(out)))
     return out

@@ -341,7 +341,8 @@ extern "C" clha_status clha_collect(clha_ctx* ctx, clha_accum* acc, int layer, c
 // ------------------------------------------------------------------------------ phase 2
 extern "C" clha_status clha_aggregate(clha_ctx* ctx, const clha_accum* acc, int slot0, int n_slots,
                                       clha_alpha_mode mode, const double* alpha_in, double damp_frac,
-                                      float* H_comb, float* H_damped, double* alpha_out, double* lambda_out) {
+                                      float* H_comb, float* H_damped, double* alpha_out, double* lambda_out,
+                                      double* lambda_dev) {
     CHECK_CTX(ctx);
     REQUIRE(acc && H_damped, CLHA_ERR_INVALID_ARG, "clha_aggregate: null pointer");
     REQUIRE(n_slots >= 1 && slot0 >= 0 && slot0 + n_slots <= acc->n_slots, CLHA_ERR_INVALID_ARG,
@@ -369,6 +370,9 @@ extern "C" clha_status clha_aggregate(clha_ctx* ctx, const clha_accum* acc, int 
     CUDA_TRY(launch_aggregate(ctx->stream, acc->S, acc->counts, acc->d, acc->n_layers, acc->n_slots, slot0, n_slots,
                               a, damp_frac, H_comb, H_damped, d_alpha, d_lambda, ctx->d_err),
              "clha_aggregate");
+    if (lambda_dev)
+        CUDA_TRY(cudaMemcpyAsync(lambda_dev, d_lambda, (size_t)n_slots * sizeof(double), cudaMemcpyDeviceToDevice,
+                                 ctx->stream), "clha_aggregate lambda_dev");
     if (alpha_out || lambda_out) {
         if (alpha_out)
             CUDA_TRY(cudaMemcpyAsync(alpha_out, d_alpha, (size_t)n_slots * acc->n_layers * sizeof(double),
@@ -396,16 +400,20 @@ extern "C" clha_status clha_factor(clha_ctx* ctx, const float* H_damped, int bat
     return CLHA_OK;
 }
 
-extern "C" clha_status clha_quantize(clha_ctx* ctx, const float* U, int w_per_u, const void* W, clha_dtype dtype,
+extern "C" clha_status clha_quantize(clha_ctx* ctx, const float* U, int n_u, const void* W, clha_dtype dtype,
                                      int batch, int d_out, int d_in, const clha_quant_params* p,
-                                     uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat) {
+                                     uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
+                                     const double* lambda, double* loss) {
     CHECK_CTX(ctx);
     REQUIRE(U && W && p && codes && scales && zeros, CLHA_ERR_INVALID_ARG, "clha_quantize: null pointer");
     REQUIRE(dtype == CLHA_BF16 || dtype == CLHA_F32, CLHA_ERR_INVALID_ARG, "clha_quantize: unknown dtype");
-    REQUIRE(batch >= 1 && d_out > 0 && d_in > 0 && w_per_u >= 1, CLHA_ERR_INVALID_ARG, "clha_quantize: bad sizes");
+    REQUIRE(batch >= 1 && d_out > 0 && d_in > 0 && n_u >= 1 && n_u <= batch, CLHA_ERR_INVALID_ARG,
+            "clha_quantize: bad sizes (need batch >= 1, 1 <= n_u <= batch)");
     REQUIRE(p->bits >= 2 && p->bits <= 8, CLHA_ERR_INVALID_ARG, "clha_quantize: bits=%d outside 2..8", p->bits);
     REQUIRE(d_in % 128 == 0 && d_out % 128 == 0, CLHA_ERR_UNSUPPORTED_SHAPE,
             "clha_quantize: d_out=%d and d_in=%d must be multiples of 128", d_out, d_in);
+    REQUIRE((lambda == nullptr) == (loss == nullptr), CLHA_ERR_INVALID_ARG,
+            "clha_quantize: lambda and loss go together (both or neither)");
     REQUIRE(p->group == 128 && p->block == 128, CLHA_ERR_UNSUPPORTED_SHAPE,
             "clha_quantize: group=%d block=%d (supported: 128, 128)", p->group, p->block);
     SET_DEVICE(ctx);
@@ -413,17 +421,18 @@ extern "C" clha_status clha_quantize(clha_ctx* ctx, const float* U, int w_per_u,
     void* ws = nullptr;
     clha_status st = clha_workspace(ctx, quantize_workspace_bytes(batch, d_out, d_in), &ws);
     if (st) return st;
-    CUDA_TRY(launch_quantize(ctx->stream, U, w_per_u, W, dtype == CLHA_F32, batch, d_out, d_in, p->bits, codes,
-                             scales, zeros, W_hat, ws), "clha_quantize");
+    CUDA_TRY(launch_quantize(ctx->stream, U, n_u, W, dtype == CLHA_F32, batch, d_out, d_in, p->bits, codes,
+                             scales, zeros, W_hat, lambda, loss, ws, ctx->d_err), "clha_quantize");
     return CLHA_OK;
 }
 
 extern "C" clha_status clha_loss(clha_ctx* ctx, const void* W, clha_dtype dtype, const float* W_hat, const float* H,
-                                 int w_per_h, int batch, int d_out, int d_in, double* loss_out) {
+                                 int n_h, int batch, int d_out, int d_in, double* loss_out) {
     CHECK_CTX(ctx);
     REQUIRE(W && W_hat && H && loss_out, CLHA_ERR_INVALID_ARG, "clha_loss: null pointer");
     REQUIRE(dtype == CLHA_BF16 || dtype == CLHA_F32, CLHA_ERR_INVALID_ARG, "clha_loss: unknown dtype");
-    REQUIRE(batch >= 1 && d_out > 0 && d_in > 0 && w_per_h >= 1, CLHA_ERR_INVALID_ARG, "clha_loss: bad sizes");
+    REQUIRE(batch >= 1 && d_out > 0 && d_in > 0 && n_h >= 1 && n_h <= batch, CLHA_ERR_INVALID_ARG,
+            "clha_loss: bad sizes (need batch >= 1, 1 <= n_h <= batch)");
     REQUIRE(d_in % 128 == 0 && d_out % 128 == 0, CLHA_ERR_UNSUPPORTED_SHAPE,
             "clha_loss: d_out=%d and d_in=%d must be multiples of 128", d_out, d_in);
     SET_DEVICE(ctx);
@@ -433,7 +442,7 @@ extern "C" clha_status clha_loss(clha_ctx* ctx, const void* W, clha_dtype dtype,
     if (st) return st;
     double* d_loss = (double*)ws;
     CUDA_TRY(cudaMemsetAsync(d_loss, 0, (size_t)batch * sizeof(double), ctx->stream), "clha_loss");
-    CUDA_TRY(launch_loss(ctx->stream, W, dtype == CLHA_F32, W_hat, H, w_per_h, batch, d_out, d_in, d_loss), "clha_loss");
+    CUDA_TRY(launch_loss(ctx->stream, W, dtype == CLHA_F32, W_hat, H, n_h, batch, d_out, d_in, d_loss), "clha_loss");
     CUDA_TRY(cudaMemcpyAsync(loss_out, d_loss, (size_t)batch * sizeof(double), cudaMemcpyDeviceToHost, ctx->stream),
              "clha_loss copy");
     return clha_sync_and_check(ctx, "clha_loss");

@@ -99,8 +99,9 @@ size_t factor_workspace_bytes(int batch, int d);
 cudaError_t launch_factor(cudaStream_t s, const float* H_d, int batch, int d, float* U,
                           void* ws, int* err);
 size_t quantize_workspace_bytes(int batch, int d_out, int d_in);
-cudaError_t launch_quantize(cudaStream_t s, const float* U, int w_per_u, const void* W, int w_is_f32,
+cudaError_t launch_quantize(cudaStream_t s, const float* U, int n_u, const void* W, int w_is_f32,
                             int batch, int d_out, int d_in, int bits, uint8_t* codes, float* scales,
-                            uint8_t* zeros, float* W_hat, void* ws);
+                            uint8_t* zeros, float* W_hat, const double* lambda, double* loss, void* ws,
+                            int* err);
 cudaError_t launch_loss(cudaStream_t s, const void* W, int w_is_f32, const float* W_hat, const float* H,
-                        int w_per_h, int batch, int d_out, int d_in, double* d_loss);
+                        int n_h, int batch, int d_out, int d_in, double* d_loss);

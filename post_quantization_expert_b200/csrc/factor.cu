@@ -10,8 +10,10 @@
 //   per panel k:  fac_potrf   Cholesky of the diagonal tile in shared memory, plus its inverse
 //                 fac_trsm    panel tiles A[i][k] <- A[i][k] L_kk^-T   (a GEMM with the inverse)
 //                 fac_update  trailing lower tiles A[i][j] -= A[i][k] A[j][k]^T
-//   fac_inv_band  X = L^-1, one band of block diagonals at a time:
-//                 X[i][j] = -X[i][i] sum_{m=j}^{i-1} L[i][m] X[m][j]  (diagonal tiles come from potrf)
+//   X = L^-1, right-looking by block rows (diagonal tiles come from potrf; X starts as I):
+//     fac_inv_row   X[i][j] <- Linv_ii X[i][j]           for j < i
+//     fac_inv_upd   X[r][j] -= L[r][i] X[i][j]           for r > i, j <= i
+//   so X[i][j] = Linv_ii (I - sum_{m<i} L[i][m] X[m][j]), every launch one 64^3 product per CTA.
 //   fac_store     U = J X J as float32 (strict lower triangle zero)
 // A non-positive pivot is recorded (problem, original column) and the problem's factor is NaN.
 #include "clha_internal.h"
@@ -19,6 +21,11 @@
 namespace {
 
 constexpr int NB = 64;
+constexpr int LD = NB + 2;   // shared-memory row length (doubles): 16-byte aligned rows, few bank conflicts
+constexpr int TILE_DOUBLES = NB * LD;
+constexpr int SMEM2 = 2 * TILE_DOUBLES * sizeof(double);
+
+typedef double Tile[LD];
 
 __global__ void fac_load(const float* __restrict__ H, int d, double* __restrict__ A) {
     const int b = blockIdx.y;
@@ -29,95 +36,132 @@ __global__ void fac_load(const float* __restrict__ H, int d, double* __restrict_
     }
 }
 
+// All kernels below run 256 threads; a 64x64 tile is 16 elements per thread. The loads of a tile
+// are issued together (unrolled) so their latencies overlap.
+constexpr int PER_THREAD = NB * NB / 256;
+
+// dst[r][c] = src[r * ld + c]      (64x64 tile, rows already indexed by k)
+__device__ __forceinline__ void load_tile(Tile* dst, const double* __restrict__ src, size_t ld) {
+    double v[PER_THREAD];
+#pragma unroll
+    for (int it = 0; it < PER_THREAD; ++it) {
+        const int i = it * 256 + threadIdx.x;
+        v[it] = src[(size_t)(i >> 6) * ld + (i & 63)];
+    }
+#pragma unroll
+    for (int it = 0; it < PER_THREAD; ++it) {
+        const int i = it * 256 + threadIdx.x;
+        dst[i >> 6][i & 63] = v[it];
+    }
+}
+// dst[c][r] = src[r * ld + c]      (transpose: the tile's columns become the k index)
+__device__ __forceinline__ void load_tile_t(Tile* dst, const double* __restrict__ src, size_t ld) {
+    double v[PER_THREAD];
+#pragma unroll
+    for (int it = 0; it < PER_THREAD; ++it) {
+        const int i = it * 256 + threadIdx.x;
+        v[it] = src[(size_t)(i >> 6) * ld + (i & 63)];
+    }
+#pragma unroll
+    for (int it = 0; it < PER_THREAD; ++it) {
+        const int i = it * 256 + threadIdx.x;
+        dst[i & 63][i >> 6] = v[it];
+    }
+}
+// acc[i][j] += sum_k As[k][4ty+i] * Bs[k][4tx+j]  (k-major operands; 16-byte shared loads)
+__device__ __forceinline__ void mma_tile(const Tile* As, const Tile* Bs, double (&acc)[4][4]) {
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll 4
+    for (int k = 0; k < NB; ++k) {
+        const double2 a0 = *reinterpret_cast<const double2*>(&As[k][4 * ty]);
+        const double2 a1 = *reinterpret_cast<const double2*>(&As[k][4 * ty + 2]);
+        const double2 b0 = *reinterpret_cast<const double2*>(&Bs[k][4 * tx]);
+        const double2 b1 = *reinterpret_cast<const double2*>(&Bs[k][4 * tx + 2]);
+        const double a[4] = {a0.x, a0.y, a1.x, a1.y};
+        const double bb[4] = {b0.x, b0.y, b1.x, b1.y};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], bb[j], acc[i][j]);
+    }
+}
+
 // Cholesky of the 64x64 diagonal tile of panel k (lower), and its inverse into Dall[b][k].
 __global__ void __launch_bounds__(256) fac_potrf(double* __restrict__ A, int d, int k, double* __restrict__ Dall,
                                                  int* err) {
     const int b = blockIdx.x;
     double* Ab = A + (size_t)b * d * d;
     extern __shared__ double dsm[];
-    double (*T)[NB + 1] = reinterpret_cast<double (*)[NB + 1]>(dsm);
-    double (*X)[NB + 1] = reinterpret_cast<double (*)[NB + 1]>(dsm + NB * (NB + 1));
+    Tile* T = reinterpret_cast<Tile*>(dsm);
+    Tile* X = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
     __shared__ int bad;
     const int k0 = k * NB;
-    for (int i = threadIdx.x; i < NB * NB; i += blockDim.x) {
-        int r = i / NB, c = i % NB;
-        T[r][c] = Ab[(size_t)(k0 + r) * d + k0 + c];
-    }
+    load_tile(T, Ab + (size_t)k0 * d + k0, d);
     if (threadIdx.x == 0) bad = -1;
     __syncthreads();
     for (int c = 0; c < NB; ++c) {
-        if (threadIdx.x == 0) {
-            double p = T[c][c];
-            if (!(p > 0.0) || !isfinite(p)) {
-                if (bad < 0) bad = c;
-                p = __longlong_as_double(0x7ff8000000000000ll);  // NaN propagates to the factor
-            } else {
-                p = sqrt(p);
-            }
-            T[c][c] = p;
-        }
+        // every thread reads the pivot; a non-positive one poisons the factor with NaN
+        double p = T[c][c];
+        const bool ok = (p > 0.0) && isfinite(p);
+        p = ok ? sqrt(p) : __longlong_as_double(0x7ff8000000000000ll);
+        if (!ok && threadIdx.x == 0 && bad < 0) bad = c;
+        const double inv = 1.0 / p;
+        __syncthreads();                           // all reads of T[c][c] precede the writes below
+        if (threadIdx.x == 0) T[c][c] = p;
+        if (threadIdx.x > c && threadIdx.x < NB) T[threadIdx.x][c] *= inv;
         __syncthreads();
-        const double piv = T[c][c];
-        for (int r = c + 1 + threadIdx.x; r < NB; r += blockDim.x) T[r][c] /= piv;
-        __syncthreads();
-        // trailing update of the tile (lower part)
-        for (int i = threadIdx.x; i < NB * NB; i += blockDim.x) {
-            int r = i / NB, cc = i % NB;
-            if (cc > c && r >= cc) T[r][cc] -= T[r][c] * T[cc][c];
+        // trailing lower triangle: thread owns column cc = tid % 64 and every 4th row from c+1
+        const int cc = threadIdx.x & 63;
+        if (cc > c) {
+            const double tc_ = T[cc][c];
+            for (int r = c + 1 + (threadIdx.x >> 6); r < NB; r += 4)
+                if (r >= cc) T[r][cc] -= T[r][c] * tc_;
         }
         __syncthreads();
     }
-    if (threadIdx.x == 0 && bad >= 0)
-        clha_record_error(err, CLHA_ERR_NOT_PD, b, d - 1 - (k0 + bad), KID_FACTOR);
-    // inverse of the lower tile: column c of X solves T x = e_c (forward substitution)
-    if (threadIdx.x < NB) {
-        const int c = threadIdx.x;
-        for (int r = 0; r < NB; ++r) {
-            if (r < c) { X[r][c] = 0.0; continue; }
-            double s = (r == c) ? 1.0 : 0.0;
-            for (int m = c; m < r; ++m) s -= T[r][m] * X[m][c];
-            X[r][c] = s / T[r][r];
-        }
+    if (threadIdx.x == 0 && bad >= 0) clha_record_error(err, CLHA_ERR_NOT_PD, b, d - 1 - (k0 + bad), KID_FACTOR);
+    // inverse: row by row, X[r][c] = (delta_rc - sum_{m=c}^{r-1} T[r][m] X[m][c]) / T[r][r];
+    // 4 threads share one column's dot product (lanes 4c..4c+3 of the same warp)
+    const int col = threadIdx.x >> 2, part = threadIdx.x & 3;
+    for (int r = 0; r < NB; ++r) {
+        double sum = 0.0;
+        if (col < r)
+            for (int m = col + part; m < r; m += 4) sum = fma(T[r][m], X[m][col], sum);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        if (part == 0) X[r][col] = (col > r) ? 0.0 : (((r == col) ? 1.0 : 0.0) - sum) / T[r][r];
+        __syncthreads();
     }
-    __syncthreads();
     double* Db = Dall + ((size_t)b * (d / NB) + k) * NB * NB;
-    for (int i = threadIdx.x; i < NB * NB; i += blockDim.x) {
-        int r = i / NB, c = i % NB;
+#pragma unroll
+    for (int it = 0; it < PER_THREAD; ++it) {
+        const int i = it * 256 + threadIdx.x;
+        const int r = i >> 6, c = i & 63;
         Ab[(size_t)(k0 + r) * d + k0 + c] = (c <= r) ? T[r][c] : 0.0;
         Db[i] = X[r][c];
     }
 }
 
-// Panel tiles below the diagonal: A[i][k] <- A[i][k] * L_kk^-T, i.e. X[r][c] = sum_m B[r][m] Linv[c][m].
+// Panel tiles below the diagonal: A[i][k] <- A[i][k] L_kk^-T, i.e. out[r][c] = sum_m B[r][m] Linv[c][m].
 __global__ void __launch_bounds__(256) fac_trsm(double* __restrict__ A, int d, int k, const double* __restrict__ Dall) {
     const int b = blockIdx.y;
     const int ib = k + 1 + blockIdx.x;
     double* Ab = A + (size_t)b * d * d;
     const double* Db = Dall + ((size_t)b * (d / NB) + k) * NB * NB;
     extern __shared__ double dsm[];
-    double (*Bs)[NB + 1] = reinterpret_cast<double (*)[NB + 1]>(dsm);
-    double (*Li)[NB + 1] = reinterpret_cast<double (*)[NB + 1]>(dsm + NB * (NB + 1));
-    for (int i = threadIdx.x; i < NB * NB; i += blockDim.x) {
-        int r = i / NB, c = i % NB;
-        Bs[r][c] = Ab[(size_t)(ib * NB + r) * d + k * NB + c];
-        Li[r][c] = Db[i];
-    }
+    Tile* As = reinterpret_cast<Tile*>(dsm);
+    Tile* Bs = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
+    double* blk = Ab + (size_t)(ib * NB) * d + k * NB;
+    load_tile_t(As, blk, d);          // As[m][r] = B[r][m]
+    load_tile_t(Bs, Db, NB);          // Bs[m][c] = Linv[c][m]
     __syncthreads();
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
     double acc[4][4] = {};
-    for (int m = 0; m < NB; ++m) {
-        double a[4], l[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) { a[i] = Bs[ty * 4 + i][m]; l[i] = Li[tx * 4 + i][m]; }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], l[j], acc[i][j]);
-    }
+    mma_tile(As, Bs, acc);
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) Ab[(size_t)(ib * NB + ty * 4 + i) * d + k * NB + tx * 4 + j] = acc[i][j];
+        for (int j = 0; j < 4; ++j) blk[(size_t)(ty * 4 + i) * d + tx * 4 + j] = acc[i][j];
 }
 
 // Trailing update of the lower tiles (i >= j > k): A[i][j] -= A[i][k] A[j][k]^T.
@@ -125,34 +169,23 @@ __global__ void __launch_bounds__(256) fac_update(double* __restrict__ A, int d,
     const int b = blockIdx.y;
     int t = blockIdx.x, jj = 0;
     const int m = d / NB - k - 1;  // trailing tiles per side
-    // enumerate lower tiles column by column: column jj has m - jj tiles (rows jj..m-1)
-    while (t >= m - jj) { t -= m - jj; ++jj; }
+    while (t >= m - jj) { t -= m - jj; ++jj; }   // column jj holds m - jj tiles (rows jj..m-1)
     const int ib = k + 1 + jj + t, jb = k + 1 + jj;
     double* Ab = A + (size_t)b * d * d;
     extern __shared__ double dsm[];
-    double (*P)[NB + 1] = reinterpret_cast<double (*)[NB + 1]>(dsm);
-    double (*Q)[NB + 1] = reinterpret_cast<double (*)[NB + 1]>(dsm + NB * (NB + 1));
-    for (int i = threadIdx.x; i < NB * NB; i += blockDim.x) {
-        int r = i / NB, c = i % NB;
-        P[r][c] = Ab[(size_t)(ib * NB + r) * d + k * NB + c];
-        Q[r][c] = Ab[(size_t)(jb * NB + r) * d + k * NB + c];
-    }
+    Tile* As = reinterpret_cast<Tile*>(dsm);
+    Tile* Bs = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
+    load_tile_t(As, Ab + (size_t)(ib * NB) * d + k * NB, d);   // As[q][r] = A[ib][k][r][q]
+    load_tile_t(Bs, Ab + (size_t)(jb * NB) * d + k * NB, d);   // Bs[q][s] = A[jb][k][s][q]
     __syncthreads();
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
     double acc[4][4] = {};
-    for (int q = 0; q < NB; ++q) {
-        double a[4], c[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) { a[i] = P[ty * 4 + i][q]; c[i] = Q[tx * 4 + i][q]; }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], c[j], acc[i][j]);
-    }
+    mma_tile(As, Bs, acc);
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    double* out = Ab + (size_t)(ib * NB) * d + jb * NB;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) Ab[(size_t)(ib * NB + ty * 4 + i) * d + jb * NB + tx * 4 + j] -= acc[i][j];
+        for (int j = 0; j < 4; ++j) out[(size_t)(ty * 4 + i) * d + tx * 4 + j] -= acc[i][j];
 }
 
 // Copy the diagonal-tile inverses of all panels into X (they were produced panel by panel).
@@ -161,66 +194,52 @@ __global__ void fac_inv_diag(const double* __restrict__ Dall, int d, double* __r
     const double* Db = Dall + ((size_t)b * (d / NB) + kb) * NB * NB;
     double* Xb = X + (size_t)b * d * d;
     for (int i = threadIdx.x; i < NB * NB; i += blockDim.x) {
-        int r = i / NB, c = i % NB;
+        const int r = i >> 6, c = i & 63;
         Xb[(size_t)(kb * NB + r) * d + kb * NB + c] = Db[i];
     }
 }
 
-// Band delta of X = L^-1: tiles (ib, jb = ib - delta).
-__global__ void __launch_bounds__(256) fac_inv_band(const double* __restrict__ L, int d, int delta,
-                                                    double* __restrict__ X) {
+// X[i][j] <- Linv_ii X[i][j] for the j < i tiles of block row i (in place).
+__global__ void __launch_bounds__(256) fac_inv_row(const double* __restrict__ Dall, int d, int i,
+                                                   double* __restrict__ X) {
+    const int b = blockIdx.y, jb = blockIdx.x;
+    double* Xt = X + (size_t)b * d * d + (size_t)(i * NB) * d + jb * NB;
+    extern __shared__ double dsm[];
+    Tile* As = reinterpret_cast<Tile*>(dsm);
+    Tile* Bs = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
+    load_tile_t(As, Dall + ((size_t)b * (d / NB) + i) * NB * NB, NB);   // As[q][r] = Linv_ii[r][q]
+    load_tile(Bs, Xt, d);                                              // Bs[q][s] = X[i][jb][q][s]
+    __syncthreads();
+    double acc[4][4] = {};
+    mma_tile(As, Bs, acc);
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) Xt[(size_t)(ty * 4 + a) * d + tx * 4 + c] = acc[a][c];
+}
+
+// X[r][j] -= L[r][i] X[i][j] for r > i, j <= i.
+__global__ void __launch_bounds__(256) fac_inv_upd(const double* __restrict__ L, int d, int i,
+                                                   double* __restrict__ X) {
     const int b = blockIdx.y;
-    const int jb = blockIdx.x, ib = jb + delta;
+    const int rb = i + 1 + blockIdx.x / (i + 1), jb = blockIdx.x % (i + 1);
     const double* Lb = L + (size_t)b * d * d;
     double* Xb = X + (size_t)b * d * d;
     extern __shared__ double dsm[];
-    double (*P)[NB + 1] = reinterpret_cast<double (*)[NB + 1]>(dsm);
-    double (*Q)[NB + 1] = reinterpret_cast<double (*)[NB + 1]>(dsm + NB * (NB + 1));
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    Tile* As = reinterpret_cast<Tile*>(dsm);
+    Tile* Bs = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
+    load_tile_t(As, Lb + (size_t)(rb * NB) * d + i * NB, d);     // As[q][r] = L[rb][i][r][q]
+    load_tile(Bs, Xb + (size_t)(i * NB) * d + jb * NB, d);       // Bs[q][s] = X[i][jb][q][s]
+    __syncthreads();
     double acc[4][4] = {};
-    for (int mb = jb; mb < ib; ++mb) {  // T = sum L[ib][mb] X[mb][jb]
-        __syncthreads();
-        for (int i = threadIdx.x; i < NB * NB; i += blockDim.x) {
-            int r = i / NB, c = i % NB;
-            P[r][c] = Lb[(size_t)(ib * NB + r) * d + mb * NB + c];
-            Q[r][c] = Xb[(size_t)(mb * NB + r) * d + jb * NB + c];
-        }
-        __syncthreads();
-        for (int q = 0; q < NB; ++q) {
-            double a[4], c[4];
+    mma_tile(As, Bs, acc);
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    double* out = Xb + (size_t)(rb * NB) * d + jb * NB;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) { a[i] = P[ty * 4 + i][q]; c[i] = Q[q][tx * 4 + i]; }
+    for (int a = 0; a < 4; ++a)
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], c[j], acc[i][j]);
-        }
-    }
-    // X[ib][jb] = -X[ib][ib] * T
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) Q[ty * 4 + i][tx * 4 + j] = acc[i][j];
-    for (int i = threadIdx.x; i < NB * NB; i += blockDim.x) {
-        int r = i / NB, c = i % NB;
-        P[r][c] = Xb[(size_t)(ib * NB + r) * d + ib * NB + c];
-    }
-    __syncthreads();
-    double out[4][4] = {};
-    for (int q = 0; q < NB; ++q) {
-        double a[4], c[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) { a[i] = P[ty * 4 + i][q]; c[i] = Q[q][tx * 4 + i]; }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) out[i][j] = fma(a[i], c[j], out[i][j]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) Xb[(size_t)(ib * NB + ty * 4 + i) * d + jb * NB + tx * 4 + j] = -out[i][j];
+        for (int c = 0; c < 4; ++c) out[(size_t)(ty * 4 + a) * d + tx * 4 + c] -= acc[a][c];
 }
 
 __global__ void fac_store(const double* __restrict__ X, int d, float* __restrict__ U) {
@@ -247,12 +266,14 @@ cudaError_t launch_factor(cudaStream_t s, const float* H_d, int batch, int d, fl
     double* X = (double*)clha_carve(cur, (size_t)batch * dd * sizeof(double));
     double* Dall = (double*)clha_carve(cur, (size_t)batch * (d / NB) * NB * NB * sizeof(double));
     const int nbk = d / NB;
-    const int smem = 2 * NB * (NB + 1) * sizeof(double);
+    const int smem = SMEM2;
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(fac_potrf, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(fac_trsm, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(fac_update, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(fac_inv_band, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+    if ((e = cudaFuncSetAttribute(fac_inv_row, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(fac_inv_upd, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
         return e;
     unsigned eg = (unsigned)((dd + 255) / 256);
     if (eg > 148 * 64) eg = 148 * 64;
@@ -273,9 +294,15 @@ cudaError_t launch_factor(cudaStream_t s, const float* H_d, int batch, int d, fl
     }
     fac_inv_diag<<<dim3(nbk, batch), 256, 0, s>>>(Dall, d, X);
     clha_note_launches(1);
-    for (int delta = 1; delta < nbk; ++delta) {
-        fac_inv_band<<<dim3(nbk - delta, batch), 256, smem, s>>>(A, d, delta, X);
-        clha_note_launches(1);
+    for (int i = 0; i < nbk; ++i) {
+        if (i > 0) {
+            fac_inv_row<<<dim3(i, batch), 256, smem, s>>>(Dall, d, i, X);
+            clha_note_launches(1);
+        }
+        if (i + 1 < nbk) {
+            fac_inv_upd<<<dim3((nbk - 1 - i) * (i + 1), batch), 256, smem, s>>>(A, d, i, X);
+            clha_note_launches(1);
+        }
     }
     fac_store<<<dim3(eg, batch), 256, 0, s>>>(X, d, U);
     clha_note_launches(1);

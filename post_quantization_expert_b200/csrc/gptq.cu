@@ -1,167 +1,396 @@
 // Phase 3 of CLHA (the CLHA page, §2.2 (3)): GPTQ column-sequential quantization with the
 // aggregated Hessian's factor U (H_d^-1 = U^T U), restated from GPTQ (Frantar et al. 2022, Alg. 1).
 //
-// One CTA owns 128 rows of one weight and walks the columns in 128-column blocks; one thread owns
-// one row, so a row's whole block lives in that thread's registers and the column-by-column error
-// feedback needs no communication at all. Per block:
-//   1. lazy update, left-looking: the block's columns receive the errors of all earlier blocks at
-//      once, w[:, blk] = W[:, blk] - E[:, :cb] U[:cb, blk], from the error rows this CTA wrote
-//      earlier (shared-memory staged FMA);
-//   2. grid of the group (group = block = 128 columns): min/max over the row's current values;
-//   3. 128 sequential columns: q = clamp(round(w/s) + z), w_hat = s (q - z), e = (w - w_hat) / U_jj,
-//      later columns of the block -= e * U[j, :] (broadcast from shared memory);
-//   4. errors, codes and w_hat of the block go to memory.
+// One CTA owns 128 rows of one weight and walks the columns in 128-column blocks (the lazy-update
+// block and the quantization group coincide). Warp roles:
+//   warps 0-3  one thread per row: a row's whole block lives in its registers, so the column-by-
+//              column error feedback inside a block needs no communication. Per block: take the lazy
+//              update from TMEM, w = W[:, blk] - acc; fix the group's grid from the current values;
+//              then for 128 columns q = clamp(round(w/s) + z), w_hat = s (q - z),
+//              e = (w - w_hat) / U_jj and w[:, c > j] -= e U[j, c] (U's diagonal block in shared
+//              memory). The block's errors go to global memory split into tf32 hi + lo parts.
+//   warp 4     TMA producer: for block b+1 it streams E[:, :cb] (hi, lo) and the U panel U[:cb, blk]
+//              (hi, lo, from a transposed copy so both operands are K-major) in 32-wide k steps;
+//              the last 128 k (the errors of the block being quantized) only after the row warps
+//              signal they are written.
+//   warp 5     MMA issuer: acc = E[:, :cb] U[:cb, blk] with tcgen05.mma kind::tf32, M=128 N=128 K=8,
+//              three products per step (hi*hi + hi*lo + lo*hi: float32-class accuracy from tf32
+//              inputs), into one of two TMEM accumulators, so block b+1's update overlaps block b's
+//              sequential columns.
 // The grid and the code are decided with IEEE float32 operations (division and rounding to nearest
-// even), so a kernel decision equals the float32 decision on the same current value.
+// even), the same operations a float32 reference takes on the same current value.
 #include "clha_internal.h"
+#include "tc_ptx.h"
+#include "tmap.h"
 
 namespace {
 
-constexpr int R = 128;     // rows per CTA (one per thread)
-constexpr int BLK = 128;   // columns per block and per group
-constexpr int KC = 32;     // k-chunk of the left-looking update
-constexpr int SMEM_BYTES = (BLK * BLK + BLK + KC * BLK + KC * (R + 1)) * sizeof(float);
+constexpr int R = 128;      // rows per CTA (one per row thread)
+constexpr int BLK = 128;    // columns per lazy block and per group
+constexpr int KS = 32;      // k per pipeline stage (one 128-byte row of fp32)
+constexpr int STAGES = 2;
+constexpr int A_BYTES = R * KS * 4;                       // 16 KB: E rows (hi or lo)
+constexpr int B_BYTES = KS * BLK * 4;                     // 16 KB: U panel (hi or lo), K-major
+constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;    // 64 KB
+constexpr int UD_OFF = STAGES * STAGE_BYTES;
+constexpr int UINV_OFF = UD_OFF + BLK * BLK * 4;
+constexpr int CODES_OFF = UINV_OFF + BLK * 4;           // block codes, [column][row] bytes
+constexpr int BAR_OFF = CODES_OFF + BLK * R;
+constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;
+constexpr int kThreads = 192;
+constexpr uint32_t IDESC = tc::idesc_f32acc(2 /*tf32*/, 0 /*A K-major*/, 0 /*B K-major*/, R, BLK);
 
-__global__ void __launch_bounds__(R, 1) gptq_simt(const float* __restrict__ U, int w_per_u, const void* __restrict__ Wv,
-                                                  int w_f32, int d_out, int d_in, int bits, uint8_t* __restrict__ codes,
-                                                  float* __restrict__ scales, uint8_t* __restrict__ zeros,
-                                                  float* __restrict__ W_hat, float* __restrict__ Escr) {
-    extern __shared__ float sm[];
-    float (*Ud)[BLK] = reinterpret_cast<float (*)[BLK]>(sm);
-    float* uinv = sm + BLK * BLK;
-    float (*Us)[BLK] = reinterpret_cast<float (*)[BLK]>(uinv + BLK);
-    float (*Es)[R + 1] = reinterpret_cast<float (*)[R + 1]>(&Us[KC][0]);
+struct GptqParams {
+    const float* U;        // [n_u, d_in, d_in] (for the diagonal blocks)
+    int n_u;               // problem b uses factor b % n_u
+    const void* W;
+    int w_f32;
+    int d_out, d_in, bits;
+    uint8_t* codes;
+    float* scales;
+    uint8_t* zeros;
+    float* W_hat;
+    float* Ehi;            // [batch, d_out, d_in]
+    float* Elo;
+    const double* lambda;  // [n_u] damping of each factor, or null
+    double* loss;          // [batch] |E|^2 - lambda |W_hat - W|^2, or null
+    int* err;
+};
 
+__device__ __forceinline__ float to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
+__device__ __forceinline__ void row_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUtensorMap tmElo,
+        const __grid_constant__ CUtensorMap tmUhi, const __grid_constant__ CUtensorMap tmUlo, GptqParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float (*Ud)[BLK] = reinterpret_cast<float (*)[BLK]>(smem + UD_OFF);
+    float* uinv = reinterpret_cast<float*>(smem + UINV_OFF);
+    uint8_t (*qs)[R] = reinterpret_cast<uint8_t (*)[R]>(smem + CODES_OFF);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+    const uint32_t full0 = tc::smem_u32(bars);
+    const uint32_t empty0 = full0 + 8 * STAGES;
+    const uint32_t tfull0 = empty0 + 8 * STAGES;
+    const uint32_t tempty0 = tfull0 + 16;
+    const uint32_t eready = tempty0 + 16;
+    const uint32_t drain = eready + 8;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + BAR_OFF + 8 * (2 * STAGES + 6));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.y;
-    const int t = threadIdx.x;
-    const int row = blockIdx.x * R + t;
-    const size_t dd = (size_t)d_in * d_in;
-    const float* Ub = U + (size_t)(b / w_per_u) * dd;
-    const size_t wrow = ((size_t)b * d_out + row) * d_in;
-    float* Erow = Escr + wrow;
-    const float maxq = (float)((1 << bits) - 1);
-    const int ngroups = d_in / BLK;
+    const int r0 = blockIdx.x * R;
+    const int u = b % p.n_u;
+    const int nblk = p.d_in / BLK;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(full0 + 8 * s, 1);
+            tc::mbar_init(empty0 + 8 * s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            tc::mbar_init(tfull0 + 8 * a, 1);
+            tc::mbar_init(tempty0 + 8 * a, R);
+        }
+        tc::mbar_init(eready, R);
+        tc::mbar_init(drain, 1);
+        *abort_flag = 0;
+        tc::fence_barrier_init();
+    }
+    if (warp == 5) tc::tmem_alloc(tc::smem_u32(tmem_slot), 256);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
 
-    for (int cb = 0; cb < d_in; cb += BLK) {
-        float w[BLK];
-#pragma unroll
-        for (int c = 0; c < BLK; ++c) w[c] = 0.f;
-        // 1. lazy update from all earlier blocks
-        for (int k0 = 0; k0 < cb; k0 += KC) {
-            __syncthreads();
-            const float4* e4 = reinterpret_cast<const float4*>(Erow + k0);
-#pragma unroll
-            for (int i = 0; i < KC / 4; ++i) {
-                float4 v = e4[i];
-                Es[4 * i + 0][t] = v.x;
-                Es[4 * i + 1][t] = v.y;
-                Es[4 * i + 2][t] = v.z;
-                Es[4 * i + 3][t] = v.w;
+    if (warp == 4) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tc::prefetch_tmap(&tmEhi);
+            tc::prefetch_tmap(&tmElo);
+            tc::prefetch_tmap(&tmUhi);
+            tc::prefetch_tmap(&tmUlo);
+            int it = 0;
+            bool ok = true;
+            const int ey = b * p.d_out + r0;
+            for (int bb = 1; bb < nblk && ok; ++bb) {
+                const int cb = bb * BLK;
+                for (int ks = 0; ks < cb / KS; ++ks) {
+                    const int k0 = ks * KS;
+                    if (k0 == cb - BLK) {   // errors of the previous block: wait until they are written
+                        if (!tc::mbar_wait_bounded(eready, (bb - 1) & 1, abort_flag)) { ok = false; break; }
+                    }
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!tc::mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag)) { ok = false; break; }
+                    const uint32_t fb = full0 + 8 * s;
+                    tc::mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    const uint32_t st = tc::smem_u32(smem + s * STAGE_BYTES);
+                    tc::tma_load_2d(st, &tmEhi, fb, k0, ey);
+                    tc::tma_load_2d(st + A_BYTES, &tmElo, fb, k0, ey);
+                    const int uy = u * p.d_in + cb;           // rows n of the transposed factor
+                    tc::tma_load_2d(st + 2 * A_BYTES, &tmUhi, fb, k0, uy);
+                    tc::tma_load_2d(st + 2 * A_BYTES + B_BYTES, &tmUlo, fb, k0, uy);
+                    ++it;
+                }
             }
+            if (!ok) {
+                for (int j = it - 1; j >= 0 && j >= it - STAGES; --j)
+                    tc::mbar_wait_bounded(full0 + 8 * (j % STAGES), (j / STAGES) & 1, abort_flag, 100000000ull);
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int it = 0;
+            bool ok = true;
+            for (int bb = 1; bb < nblk && ok; ++bb) {
+                const int tcount = bb - 1;
+                const int acc = tcount & 1;
+                if (!tc::mbar_wait_bounded(tempty0 + 8 * acc, ((tcount >> 1) & 1) ^ 1, abort_flag)) break;
+                tc::fence_after_sync();
+                const uint32_t d_tmem = tmem + acc * BLK;
+                const int nks = bb * BLK / KS;
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int s = it % STAGES;
+                    if (!tc::mbar_wait_bounded(full0 + 8 * s, (it / STAGES) & 1, abort_flag)) { ok = false; break; }
+                    tc::fence_after_sync();
+                    const uint32_t ahi = tc::smem_u32(smem + s * STAGE_BYTES);
+                    const uint32_t alo = ahi + A_BYTES;
+                    const uint32_t bhi = ahi + 2 * A_BYTES;
+                    const uint32_t blo = bhi + B_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < KS / 8; ++kk) {
+                        const uint64_t dah = tc::sw128_desc(ahi + kk * 32, 16, 1024);
+                        const uint64_t dal = tc::sw128_desc(alo + kk * 32, 16, 1024);
+                        const uint64_t dbh = tc::sw128_desc(bhi + kk * 32, 16, 1024);
+                        const uint64_t dbl = tc::sw128_desc(blo + kk * 32, 16, 1024);
+                        tc::mma_tf32(d_tmem, dah, dbh, IDESC, (ks | kk) != 0);
+                        tc::mma_tf32(d_tmem, dah, dbl, IDESC, 1);
+                        tc::mma_tf32(d_tmem, dal, dbh, IDESC, 1);
+                    }
+                    tc::mma_commit(empty0 + 8 * s);
+                }
+                if (!ok) break;
+                tc::mma_commit(tfull0 + 8 * acc);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------------ row threads
+        const int t = threadIdx.x;
+        const int row = r0 + t;
+        const size_t dd = (size_t)p.d_in * p.d_in;
+        const float* Ub = p.U + (size_t)u * dd;
+        const size_t wrow = ((size_t)b * p.d_out + row) * p.d_in;
+        const float maxq = (float)((1 << p.bits) - 1);
+        const int ngroups = p.d_in / BLK;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        bool ok = true;
+        double e2 = 0.0, d2 = 0.0;   // this row's |E|^2 and |W_hat - W|^2
+        for (int bb = 0; bb < nblk; ++bb) {
+            const int cb = bb * BLK;
+            row_bar();                                   // every row thread is done with the last Ud
+            for (int i = 0; i < BLK; ++i) Ud[i][t] = Ub[(size_t)(cb + i) * p.d_in + cb + t];
+            row_bar();
+            uinv[t] = 1.0f / Ud[t][t];
+            float w[BLK];
+            if (p.w_f32) {
+                const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.W) + wrow + cb);
+#pragma unroll
+                for (int i = 0; i < BLK / 4; ++i) {
+                    const float4 v = src[i];
+                    w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+                }
+            } else {
+                const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.W) + wrow + cb);
+#pragma unroll
+                for (int i = 0; i < BLK / 8; ++i) {
+                    const uint4 v = src[i];
+                    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 f = __bfloat1622float2(h2[j]);
+                        w[8 * i + 2 * j] = f.x;
+                        w[8 * i + 2 * j + 1] = f.y;
+                    }
+                }
+            }
+            if (bb > 0 && ok) {    // lazy update of this block from all earlier blocks' errors
+                const int tcount = bb - 1;
+                const int acc = tcount & 1;
+                if (!tc::mbar_wait_bounded(tfull0 + 8 * acc, (tcount >> 1) & 1, abort_flag)) ok = false;
+                tc::fence_after_sync();
+                if (ok) {
+#pragma unroll
+                    for (int ch = 0; ch < BLK / 32; ++ch) {
+                        uint32_t v[32];
+                        tc::tmem_ld_32x32b_x32(tmem + lane_base + acc * BLK + ch * 32, v);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) w[ch * 32 + j] -= __uint_as_float(v[j]);
+                    }
+                }
+                tc::fence_before_sync();
+                tc::mbar_arrive(tempty0 + 8 * acc);
+            }
+            row_bar();                                   // uinv complete
+            // grid of the group from the current values (0 always on the grid; [-1, 1] if all zero)
+            float xmin = 0.f, xmax = 0.f;
+#pragma unroll
+            for (int c = 0; c < BLK; ++c) { xmin = fminf(xmin, w[c]); xmax = fmaxf(xmax, w[c]); }
+            if (xmin == 0.f && xmax == 0.f) { xmin = -1.f; xmax = 1.f; }
+            const float s = __fdiv_rn(__fsub_rn(xmax, xmin), maxq);
+            const float z = rintf(__fdiv_rn(-xmin, s));
+            const int g = cb / BLK;
+            p.scales[((size_t)b * p.d_out + row) * ngroups + g] = s;
+            p.zeros[((size_t)b * p.d_out + row) * ngroups + g] = (uint8_t)z;
+#pragma unroll
+            for (int j = 0; j < BLK; ++j) {
+                float q = __fadd_rn(rintf(__fdiv_rn(w[j], s)), z);
+                q = fminf(fmaxf(q, 0.f), maxq);
+                const float wh = __fmul_rn(s, __fsub_rn(q, z));
+                const float e = (w[j] - wh) * uinv[j];
+                w[j] = e;                                // a quantized column's register keeps its error
+                qs[j][t] = (uint8_t)q;
+#pragma unroll
+                for (int c = 0; c < BLK; ++c)
+                    if (c > j) w[c] = fmaf(-e, Ud[j][c], w[c]);
+            }
+            if (p.loss) {
+#pragma unroll
+                for (int c = 0; c < BLK; ++c) e2 = fma((double)w[c], (double)w[c], e2);
+            }
+            // errors for the later blocks' lazy updates, as tf32 hi + lo
+            if (bb + 1 < nblk) {
+                float4* eh = reinterpret_cast<float4*>(p.Ehi + wrow + cb);
+                float4* el = reinterpret_cast<float4*>(p.Elo + wrow + cb);
+#pragma unroll
+                for (int i = 0; i < BLK / 4; ++i) {
+                    float h[4], l[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        h[j] = to_tf32(w[4 * i + j]);
+                        l[j] = to_tf32(w[4 * i + j] - h[j]);
+                    }
+                    eh[i] = make_float4(h[0], h[1], h[2], h[3]);
+                    el[i] = make_float4(l[0], l[1], l[2], l[3]);
+                }
+                fence_proxy_async_global();
+                tc::mbar_arrive(eready);
+            }
+            uint4* co = reinterpret_cast<uint4*>(p.codes + wrow + cb);
+            float4* wo = p.W_hat ? reinterpret_cast<float4*>(p.W_hat + wrow + cb) : nullptr;
+#pragma unroll 1
+            for (int i = 0; i < BLK / 16; ++i) {
+                uint32_t word[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    word[j] = (uint32_t)qs[16 * i + 4 * j][t] | ((uint32_t)qs[16 * i + 4 * j + 1][t] << 8) |
+                              ((uint32_t)qs[16 * i + 4 * j + 2][t] << 16) | ((uint32_t)qs[16 * i + 4 * j + 3][t] << 24);
+                co[i] = make_uint4(word[0], word[1], word[2], word[3]);
+                if (wo) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        float v[4];
+#pragma unroll
+                        for (int m = 0; m < 4; ++m)
+                            v[m] = __fmul_rn(s, __fsub_rn((float)qs[16 * i + 4 * j + m][t], z));
+                        wo[4 * i + j] = make_float4(v[0], v[1], v[2], v[3]);
+                    }
+                }
+            }
+            if (p.loss) {   // |W_hat - W|^2 of this block, W re-read (its registers now hold errors)
 #pragma unroll 4
-            for (int kk = 0; kk < KC; ++kk) Us[kk][t] = Ub[(size_t)(k0 + kk) * d_in + cb + t];
-            __syncthreads();
-#pragma unroll 2
-            for (int kk = 0; kk < KC; ++kk) {
-                const float e = Es[kk][t];
-#pragma unroll
-                for (int c = 0; c < BLK; ++c) w[c] = fmaf(e, Us[kk][c], w[c]);
-            }
-        }
-        __syncthreads();
-        for (int i = 0; i < BLK; ++i) Ud[i][t] = Ub[(size_t)(cb + i) * d_in + cb + t];
-        __syncthreads();
-        uinv[t] = 1.0f / Ud[t][t];
-        // current values of this row's block
-        if (w_f32) {
-            const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(Wv) + wrow + cb);
-#pragma unroll
-            for (int i = 0; i < BLK / 4; ++i) {
-                float4 v = src[i];
-                w[4 * i + 0] = v.x - w[4 * i + 0];
-                w[4 * i + 1] = v.y - w[4 * i + 1];
-                w[4 * i + 2] = v.z - w[4 * i + 2];
-                w[4 * i + 3] = v.w - w[4 * i + 3];
-            }
-        } else {
-            const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(Wv) + wrow + cb);
-#pragma unroll
-            for (int i = 0; i < BLK / 8; ++i) {
-                uint4 v = src[i];
-                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float2 f = __bfloat1622float2(h2[j]);
-                    w[8 * i + 2 * j + 0] = f.x - w[8 * i + 2 * j + 0];
-                    w[8 * i + 2 * j + 1] = f.y - w[8 * i + 2 * j + 1];
+                for (int c = 0; c < BLK; ++c) {
+                    const float wv = p.w_f32 ? reinterpret_cast<const float*>(p.W)[wrow + cb + c]
+                                             : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.W)[wrow + cb + c]);
+                    const double dv = (double)__fmul_rn(s, __fsub_rn((float)qs[c][t], z)) - (double)wv;
+                    d2 = fma(dv, dv, d2);
                 }
             }
         }
-        __syncthreads();
-        // 2. grid of the group from the current values (0 always on the grid; [-1, 1] if all zero)
-        float xmin = 0.f, xmax = 0.f;
+        if (p.loss) {
+            double v = e2 - p.lambda[u] * d2;
 #pragma unroll
-        for (int c = 0; c < BLK; ++c) { xmin = fminf(xmin, w[c]); xmax = fmaxf(xmax, w[c]); }
-        if (xmin == 0.f && xmax == 0.f) { xmin = -1.f; xmax = 1.f; }
-        const float s = __fdiv_rn(__fsub_rn(xmax, xmin), maxq);
-        const float z = rintf(__fdiv_rn(-xmin, s));
-        const int g = cb / BLK;
-        scales[((size_t)b * d_out + row) * ngroups + g] = s;
-        zeros[((size_t)b * d_out + row) * ngroups + g] = (uint8_t)z;
-        // 3. column-sequential quantization with error feedback inside the block
-        uint32_t qp[BLK / 4];
-#pragma unroll
-        for (int i = 0; i < BLK / 4; ++i) qp[i] = 0u;
-#pragma unroll
-        for (int j = 0; j < BLK; ++j) {
-            float q = __fadd_rn(rintf(__fdiv_rn(w[j], s)), z);
-            q = fminf(fmaxf(q, 0.f), maxq);
-            const float wh = __fmul_rn(s, __fsub_rn(q, z));
-            const float err = (w[j] - wh) * uinv[j];
-            w[j] = err;  // the register of a quantized column keeps its error
-            qp[j >> 2] |= (uint32_t)q << (8 * (j & 3));
-#pragma unroll
-            for (int c = 0; c < BLK; ++c)
-                if (c > j) w[c] = fmaf(-err, Ud[j][c], w[c]);
+            for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+            if (lane == 0) atomicAdd(&p.loss[b], v);
         }
-        // 4. outputs
-        float4* e4o = reinterpret_cast<float4*>(Erow + cb);
-#pragma unroll
-        for (int i = 0; i < BLK / 4; ++i) e4o[i] = make_float4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-        uint4* co = reinterpret_cast<uint4*>(codes + wrow + cb);
-#pragma unroll
-        for (int i = 0; i < BLK / 16; ++i) co[i] = make_uint4(qp[4 * i], qp[4 * i + 1], qp[4 * i + 2], qp[4 * i + 3]);
-        if (W_hat) {
-            float4* wo = reinterpret_cast<float4*>(W_hat + wrow + cb);
-#pragma unroll
-            for (int i = 0; i < BLK / 4; ++i) {
-                float v[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int c = 4 * i + j;
-                    const float q = (float)((qp[c >> 2] >> (8 * (c & 3))) & 255u);
-                    v[j] = __fmul_rn(s, __fsub_rn(q, z));
-                }
-                wo[i] = make_float4(v[0], v[1], v[2], v[3]);
-            }
+    }
+
+    __syncthreads();
+    if (warp == 5) {
+        if (lane == 0) {
+            tc::mma_commit(drain);
+            tc::mbar_wait_bounded(drain, 0, abort_flag, 100000000ull);
         }
+        __syncwarp();
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 256);
+    }
+    if (threadIdx.x == 0 && *abort_flag) clha_record_error(p.err, CLHA_ERR_TIMEOUT, b, r0, KID_QUANTIZE);
+}
+
+// U -> transposed (hi, lo) tf32 parts: hi_t[j][i] + lo_t[j][i] ~ U[i][j], so the lazy-update
+// operand U[k][n] is read K-major (rows n, contiguous k). 32x32 tiles through shared memory.
+__global__ void __launch_bounds__(256) gptq_split_t(const float* __restrict__ U, int d, float* __restrict__ hi,
+                                                    float* __restrict__ lo) {
+    __shared__ float tile[32][33];
+    const size_t base = (size_t)blockIdx.z * d * d;
+    const int i0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    for (int r = ty; r < 32; r += 8) tile[r][tx] = U[base + (size_t)(i0 + r) * d + j0 + tx];
+    __syncthreads();
+    for (int r = ty; r < 32; r += 8) {
+        const float x = tile[tx][r];                       // U[i0 + tx][j0 + r]
+        const float h = to_tf32(x);
+        const size_t o = base + (size_t)(j0 + r) * d + i0 + tx;
+        hi[o] = h;
+        lo[o] = to_tf32(x - h);
     }
 }
 
 }  // namespace
 
 size_t quantize_workspace_bytes(int batch, int d_out, int d_in) {
-    return clha_round_up((size_t)batch * d_out * d_in * sizeof(float));
+    const size_t e = clha_round_up((size_t)batch * d_out * d_in * sizeof(float));
+    const size_t uu = clha_round_up((size_t)batch * d_in * d_in * sizeof(float));
+    return 2 * e + 2 * uu;
 }
 
-cudaError_t launch_quantize(cudaStream_t s, const float* U, int w_per_u, const void* W, int w_is_f32, int batch,
+cudaError_t launch_quantize(cudaStream_t s, const float* U, int n_u, const void* W, int w_is_f32, int batch,
                             int d_out, int d_in, int bits, uint8_t* codes, float* scales, uint8_t* zeros,
-                            float* W_hat, void* ws) {
-    cudaError_t e = cudaFuncSetAttribute(gptq_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+                            float* W_hat, const double* lambda, double* loss, void* ws, int* err) {
+    char* cur = (char*)ws;
+    float* Ehi = (float*)clha_carve(cur, (size_t)batch * d_out * d_in * sizeof(float));
+    float* Elo = (float*)clha_carve(cur, (size_t)batch * d_out * d_in * sizeof(float));
+    float* Uhi = (float*)clha_carve(cur, (size_t)batch * d_in * d_in * sizeof(float));
+    float* Ulo = (float*)clha_carve(cur, (size_t)batch * d_in * d_in * sizeof(float));
+    cudaError_t e;
+    CUtensorMap tEhi, tElo, tUhi, tUlo;
+    if ((e = make_tmap_2d(&tEhi, Ehi, (uint64_t)batch * d_out, d_in, 4, R, KS)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d(&tElo, Elo, (uint64_t)batch * d_out, d_in, 4, R, KS)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d(&tUhi, Uhi, (uint64_t)n_u * d_in, d_in, 4, BLK, KS)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d(&tUlo, Ulo, (uint64_t)n_u * d_in, d_in, 4, BLK, KS)) != cudaSuccess) return e;
+    if (d_in > BLK) {
+        gptq_split_t<<<dim3(d_in / 32, d_in / 32, n_u), 256, 0, s>>>(U, d_in, Uhi, Ulo);
+        clha_note_launches(1);
+    }
+    if ((e = cudaFuncSetAttribute(gptq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) != cudaSuccess)
+        return e;
+    if (loss && (e = cudaMemsetAsync(loss, 0, (size_t)batch * sizeof(double), s)) != cudaSuccess) return e;
+    GptqParams p{U, n_u, W, w_is_f32, d_out, d_in, bits, codes, scales, zeros, W_hat, Ehi, Elo, lambda, loss, err};
     dim3 grid(d_out / R, batch);
-    gptq_simt<<<grid, R, SMEM_BYTES, s>>>(U, w_per_u, W, w_is_f32, d_out, d_in, bits, codes, scales, zeros, W_hat,
-                                           (float*)ws);
+    gptq_tc<<<grid, kThreads, SMEM_BYTES, s>>>(tEhi, tElo, tUhi, tUlo, p);
     clha_note_launches(1);
     return cudaGetLastError();
 }

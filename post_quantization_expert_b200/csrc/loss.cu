@@ -12,12 +12,12 @@ __device__ __forceinline__ float w_at(const void* W, int f32, size_t i) {
 }
 
 __global__ void __launch_bounds__(256) loss_simt(const void* __restrict__ W, int f32, const float* __restrict__ W_hat,
-                                                 const float* __restrict__ H, int w_per_h, int d_out, int d_in,
+                                                 const float* __restrict__ H, int n_h, int d_out, int d_in,
                                                  double* __restrict__ out) {
     const int b = blockIdx.z;
     const int r0 = blockIdx.y * T, c0 = blockIdx.x * T;
     const size_t base = (size_t)b * d_out * d_in;
-    const float* Hb = H + (size_t)(b / w_per_h) * d_in * d_in;
+    const float* Hb = H + (size_t)(b % n_h) * d_in * d_in;
     __shared__ float Ds[KC][T + 4];
     __shared__ float Hs[KC][T + 4];
     __shared__ double red[256];
@@ -63,10 +63,10 @@ __global__ void __launch_bounds__(256) loss_simt(const void* __restrict__ W, int
 
 }  // namespace
 
-cudaError_t launch_loss(cudaStream_t s, const void* W, int w_is_f32, const float* W_hat, const float* H, int w_per_h,
+cudaError_t launch_loss(cudaStream_t s, const void* W, int w_is_f32, const float* W_hat, const float* H, int n_h,
                         int batch, int d_out, int d_in, double* d_loss) {
     dim3 grid(d_in / T, d_out / T, batch);
-    loss_simt<<<grid, 256, 0, s>>>(W, w_is_f32, W_hat, H, w_per_h, d_out, d_in, d_loss);
+    loss_simt<<<grid, 256, 0, s>>>(W, w_is_f32, W_hat, H, n_h, d_out, d_in, d_loss);
     clha_note_launches(1);
     return cudaGetLastError();
 }

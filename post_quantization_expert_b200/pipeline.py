@@ -91,6 +91,12 @@ def _quant_buffers(batch, d_out, d_in, device):
                     torch.empty((batch, d_out, d_in), dtype=torch.float32, device=device))
 
 
+def _halves(q: QuantOut, n: int):
+    """Views of the first and second n problems of a stacked [2n] result (gate, then up)."""
+    return (QuantOut(q.codes[:n], q.scales[:n], q.zeros[:n], q.W_hat[:n]),
+            QuantOut(q.codes[n:], q.scales[n:], q.zeros[n:], q.W_hat[n:]))
+
+
 class DenseCalibration:
     """One weight W [d_out, d_in] shared by n_layers layers (no routing)."""
 
@@ -104,6 +110,8 @@ class DenseCalibration:
         self.H_d = torch.empty_like(self.H_comb)
         self.U = torch.empty_like(self.H_comb)
         self.q = _quant_buffers(1, d_out, d_in, dev)
+        self.lam = torch.empty(1, dtype=torch.float64, device=dev)
+        self.loss_dev = torch.empty(1, dtype=torch.float64, device=dev)
 
     def reset(self):
         L.clha_accum_zero(self.ctx, self.acc)
@@ -116,15 +124,15 @@ class DenseCalibration:
         t = self.timer
         with t.span("aggregate"):
             host = L.clha_aggregate(self.ctx, self.acc, 0, 1, MODES[mode], alpha, self.damp, self.H_comb, self.H_d,
-                                    want_host=want_host)
+                                    want_host=want_host, lambda_dev=self.lam)
         with t.span("factor"):
             L.clha_factor(self.ctx, self.H_d, 1, self.d_in, self.U)
         with t.span("gptq"):
             L.clha_quantize(self.ctx, self.U, 1, W, 1, self.d_out, self.d_in, self.bits, self.q.codes, self.q.scales,
-                            self.q.zeros, self.q.W_hat)
+                            self.q.zeros, self.q.W_hat, lam=self.lam if with_loss else None,
+                            loss=self.loss_dev if with_loss else None)
         if with_loss:
-            with t.span("loss"):
-                self.q.loss = L.clha_loss(self.ctx, W, self.q.W_hat, self.H_comb, 1, 1, self.d_out, self.d_in)
+            self.q.loss = self.loss_dev.cpu().numpy()
         return host
 
     def columns(self) -> int:
@@ -133,21 +141,58 @@ class DenseCalibration:
 
 @dataclass
 class MoEWeights:
-    """Stacked expert weights of one layer group: gate/up [E, d_ff, d_model], down [E, d_model, d_ff]."""
-    Wg: torch.Tensor
-    Wu: torch.Tensor
+    """Stacked expert weights of one layer group: Wgu [2E, d_ff, d_model] holds every gate then every
+    up projection (Wg, Wu are its halves), Wd [E, d_model, d_ff]; Sgu / Sd the same for the
+    always-active experts."""
+    Wgu: torch.Tensor
     Wd: torch.Tensor
-    Sg: torch.Tensor | None = None   # always-active experts, [n_shared, shared_dff, d_model]
-    Su: torch.Tensor | None = None
+    Sgu: torch.Tensor | None = None
     Sd: torch.Tensor | None = None
+
+    @property
+    def Wg(self):
+        return self.Wgu[: self.Wgu.shape[0] // 2]
+
+    @property
+    def Wu(self):
+        return self.Wgu[self.Wgu.shape[0] // 2:]
+
+    @property
+    def Sg(self):
+        return None if self.Sgu is None else self.Sgu[: self.Sgu.shape[0] // 2]
+
+    @property
+    def Su(self):
+        return None if self.Sgu is None else self.Sgu[self.Sgu.shape[0] // 2:]
+
+
+@dataclass
+class MoEResult:
+    """GPTQ outputs of one weighting: gate and up stacked [2E] (qg, qu are views), down [E], and the
+    always-active experts' counterparts."""
+    qgu: QuantOut
+    qg: QuantOut
+    qu: QuantOut
+    qd: QuantOut
+    sgu: QuantOut | None = None
+    sg: QuantOut | None = None
+    su: QuantOut | None = None
+    sd: QuantOut | None = None
+
+    def expert_loss(self) -> np.ndarray:
+        """Per routed expert: loss(gate) + loss(up) + loss(down) under the undamped H_comb."""
+        return self.qg.loss + self.qu.loss + self.qd.loss
 
 
 class MoECalibration:
-    """Routed experts (top-k of E) plus always-active shared experts of one weight-sharing group."""
+    """Routed experts (top-k of E) plus always-active shared experts of one weight-sharing group.
+
+    quantize() takes one or several weightings; their aggregated Hessians are factored together in
+    one batched call per Hessian kind, and each weighting keeps its own results (self.res[mode])."""
 
     def __init__(self, ctx: L.Context, n_layers: int, max_tokens: int, E: int, k: int, d_model: int, d_ff: int,
                  n_shared: int = 0, shared_dff: int = 0, bits_routed: int = 2, bits_shared: int = 3,
-                 damp_frac: float = 0.01, timer=NO_TIMER):
+                 damp_frac: float = 0.01, timer=NO_TIMER, modes=("rt",)):
         self.ctx, self.n_layers, self.E, self.k = ctx, n_layers, E, k
         self.timer = timer
         self.d_model, self.d_ff, self.n_shared, self.shared_dff = d_model, d_ff, n_shared, shared_dff
@@ -165,26 +210,51 @@ class MoECalibration:
         if n_shared:
             self.hs = torch.empty((max_tokens, shared_dff), dtype=torch.bfloat16, device=dev)
             self.acc_sdn = L.Accum(ctx, shared_dff, n_layers, n_shared)
+        self.modes = tuple(modes)
+        nm = len(self.modes)
         f32 = dict(dtype=torch.float32, device=dev)
-        self.Hc_in = torch.empty((E, d_model, d_model), **f32)
+        # [weighting][expert] Hessians and factors
+        self.Hc_in = torch.empty((nm * E, d_model, d_model), **f32)
         self.Hd_in = torch.empty_like(self.Hc_in)
         self.U_in = torch.empty_like(self.Hc_in)
-        self.Hc_dn = torch.empty((E, d_ff, d_ff), **f32)
+        self.Hc_dn = torch.empty((nm * E, d_ff, d_ff), **f32)
         self.Hd_dn = torch.empty_like(self.Hc_dn)
         self.U_dn = torch.empty_like(self.Hc_dn)
-        self.qg = _quant_buffers(E, d_ff, d_model, dev)
-        self.qu = _quant_buffers(E, d_ff, d_model, dev)
-        self.qd = _quant_buffers(E, d_model, d_ff, dev)
         if n_shared:
-            self.Hc_sin = torch.empty((1, d_model, d_model), **f32)
+            self.Hc_sin = torch.empty((nm, d_model, d_model), **f32)
             self.Hd_sin = torch.empty_like(self.Hc_sin)
             self.U_sin = torch.empty_like(self.Hc_sin)
-            self.Hc_sdn = torch.empty((n_shared, shared_dff, shared_dff), **f32)
+            self.Hc_sdn = torch.empty((nm * n_shared, shared_dff, shared_dff), **f32)
             self.Hd_sdn = torch.empty_like(self.Hc_sdn)
             self.U_sdn = torch.empty_like(self.Hc_sdn)
-            self.sg = _quant_buffers(n_shared, shared_dff, d_model, dev)
-            self.su = _quant_buffers(n_shared, shared_dff, d_model, dev)
-            self.sd = _quant_buffers(n_shared, d_model, shared_dff, dev)
+        f64 = dict(dtype=torch.float64, device=dev)
+        self.lam_in = torch.empty(nm * E, **f64)
+        self.lam_dn = torch.empty(nm * E, **f64)
+        self.lam_sin = torch.empty(max(nm, 1), **f64)
+        self.lam_sdn = torch.empty(max(nm * n_shared, 1), **f64)
+        # per weighting: [gate E][up E][down E][shared gate][shared up][shared down]
+        self.nloss = 3 * E + 3 * n_shared
+        self.loss_dev = torch.empty((nm, self.nloss), **f64)
+        self.res = {}
+        for mode in self.modes:
+            qgu = _quant_buffers(2 * E, d_ff, d_model, dev)
+            r = MoEResult(qgu, *_halves(qgu, E), _quant_buffers(E, d_model, d_ff, dev))
+            if n_shared:
+                r.sgu = _quant_buffers(2 * n_shared, shared_dff, d_model, dev)
+                r.sg, r.su = _halves(r.sgu, n_shared)
+                r.sd = _quant_buffers(n_shared, d_model, shared_dff, dev)
+            self.res[mode] = r
+        self._last = self.res[self.modes[0]]
+
+    # results of the most recent weighting (convenience for single-weighting callers)
+    qgu = property(lambda self: self._last.qgu)
+    qg = property(lambda self: self._last.qg)
+    qu = property(lambda self: self._last.qu)
+    qd = property(lambda self: self._last.qd)
+    sgu = property(lambda self: self._last.sgu)
+    sg = property(lambda self: self._last.sg)
+    su = property(lambda self: self._last.su)
+    sd = property(lambda self: self._last.sd)
 
     def reset(self):
         for a in (self.acc_in, self.acc_dn) + ((self.acc_sdn,) if self.n_shared else ()):
@@ -216,55 +286,72 @@ class MoECalibration:
                     L.clha_collect(ctx, self.acc_sdn, layer, hs, n, self.shared_dff, None, 1, i)
 
     # ------------------------------------------------------------------ phases 2 and 3
-    def quantize(self, w: MoEWeights, mode: str = "rt", alpha=None, with_loss: bool = True):
+    def quantize(self, w: MoEWeights, modes=None, alpha=None, with_loss: bool = True):
+        """Aggregate, factor, GPTQ and score for each weighting in `modes` (a name or a tuple of the
+        weightings given at construction; default all of them)."""
+        if modes is None:
+            modes = self.modes
+        if isinstance(modes, str):
+            modes = (modes,)
         ctx, E, dm, dff, t = self.ctx, self.E, self.d_model, self.d_ff, self.timer
-        m = MODES[mode]
+        ns, sdff = self.n_shared, self.shared_dff
+        idx = [self.modes.index(m) for m in modes]
         with t.span("aggregate"):
-            L.clha_aggregate(ctx, self.acc_in, 0, E, m, alpha, self.damp, self.Hc_in, self.Hd_in)
+            for i, m in zip(idx, modes):
+                es, ss = slice(i * E, (i + 1) * E), slice(i * ns, (i + 1) * ns)
+                L.clha_aggregate(ctx, self.acc_in, 0, E, MODES[m], alpha, self.damp, self.Hc_in[es], self.Hd_in[es],
+                                 lambda_dev=self.lam_in[es])
+                L.clha_aggregate(ctx, self.acc_dn, 0, E, MODES[m], alpha, self.damp, self.Hc_dn[es], self.Hd_dn[es],
+                                 lambda_dev=self.lam_dn[es])
+                if ns:
+                    L.clha_aggregate(ctx, self.acc_in, E, 1, MODES[m], alpha, self.damp, self.Hc_sin[i:i + 1],
+                                     self.Hd_sin[i:i + 1], lambda_dev=self.lam_sin[i:i + 1])
+                    L.clha_aggregate(ctx, self.acc_sdn, 0, ns, MODES[m], alpha, self.damp, self.Hc_sdn[ss],
+                                     self.Hd_sdn[ss], lambda_dev=self.lam_sdn[ss])
+        # one batched factor per Hessian kind over every requested weighting (contiguous runs)
+        lo, hi = min(idx), max(idx) + 1
+        contiguous = sorted(idx) == list(range(lo, hi))
+        runs = [(lo, hi)] if contiguous else [(i, i + 1) for i in idx]
         with t.span("factor"):
-            L.clha_factor(ctx, self.Hd_in, E, dm, self.U_in)
-        with t.span("aggregate"):
-            L.clha_aggregate(ctx, self.acc_dn, 0, E, m, alpha, self.damp, self.Hc_dn, self.Hd_dn)
-        with t.span("factor"):
-            L.clha_factor(ctx, self.Hd_dn, E, dff, self.U_dn)
-        br = self.bits_routed
-        with t.span("gptq"):
-            for W, q in ((w.Wg, self.qg), (w.Wu, self.qu)):
-                L.clha_quantize(ctx, self.U_in, 1, W, E, dff, dm, br, q.codes, q.scales, q.zeros, q.W_hat)
-            L.clha_quantize(ctx, self.U_dn, 1, w.Wd, E, dm, dff, br, self.qd.codes, self.qd.scales, self.qd.zeros,
-                            self.qd.W_hat)
-        if self.n_shared:
-            ns, sdff, bs = self.n_shared, self.shared_dff, self.bits_shared
-            with t.span("aggregate"):
-                L.clha_aggregate(ctx, self.acc_in, E, 1, m, alpha, self.damp, self.Hc_sin, self.Hd_sin)
-            with t.span("factor"):
-                L.clha_factor(ctx, self.Hd_sin, 1, dm, self.U_sin)
-            with t.span("aggregate"):
-                L.clha_aggregate(ctx, self.acc_sdn, 0, ns, m, alpha, self.damp, self.Hc_sdn, self.Hd_sdn)
-            with t.span("factor"):
-                L.clha_factor(ctx, self.Hd_sdn, ns, sdff, self.U_sdn)
+            for a, b in runs:
+                L.clha_factor(ctx, self.Hd_in[a * E:b * E], (b - a) * E, dm, self.U_in[a * E:b * E])
+                L.clha_factor(ctx, self.Hd_dn[a * E:b * E], (b - a) * E, dff, self.U_dn[a * E:b * E])
+                if ns:
+                    L.clha_factor(ctx, self.Hd_sin[a:b], b - a, dm, self.U_sin[a:b])
+                    L.clha_factor(ctx, self.Hd_sdn[a * ns:b * ns], (b - a) * ns, sdff, self.U_sdn[a * ns:b * ns])
+        br, bs = self.bits_routed, self.bits_shared
+        for i, m in zip(idx, modes):
+            r = self.res[m]
+            es, ss = slice(i * E, (i + 1) * E), slice(i * ns, (i + 1) * ns)
+            lb = self.loss_dev[i]
+            opt = (lambda lam, lo: dict(lam=lam, loss=lo)) if with_loss else (lambda lam, lo: {})
             with t.span("gptq"):
-                for W, q in ((w.Sg, self.sg), (w.Su, self.su)):
-                    L.clha_quantize(ctx, self.U_sin, ns, W, ns, sdff, dm, bs, q.codes, q.scales, q.zeros, q.W_hat)
-                L.clha_quantize(ctx, self.U_sdn, 1, w.Sd, ns, dm, sdff, bs, self.sd.codes, self.sd.scales,
-                                self.sd.zeros, self.sd.W_hat)
-        if with_loss:
-            with t.span("loss"):
-                self.qg.loss = L.clha_loss(ctx, w.Wg, self.qg.W_hat, self.Hc_in, 1, E, dff, dm)
-                self.qu.loss = L.clha_loss(ctx, w.Wu, self.qu.W_hat, self.Hc_in, 1, E, dff, dm)
-                self.qd.loss = L.clha_loss(ctx, w.Wd, self.qd.W_hat, self.Hc_dn, 1, E, dm, dff)
-                if self.n_shared:
-                    ns, sdff = self.n_shared, self.shared_dff
-                    self.sg.loss = L.clha_loss(ctx, w.Sg, self.sg.W_hat, self.Hc_sin, ns, ns, sdff, dm)
-                    self.su.loss = L.clha_loss(ctx, w.Su, self.su.W_hat, self.Hc_sin, ns, ns, sdff, dm)
-                    self.sd.loss = L.clha_loss(ctx, w.Sd, self.sd.W_hat, self.Hc_sdn, 1, ns, dm, sdff)
+                q = r.qgu
+                L.clha_quantize(ctx, self.U_in[es], E, w.Wgu, 2 * E, dff, dm, br, q.codes, q.scales, q.zeros, q.W_hat,
+                                **opt(self.lam_in[es], lb[0:2 * E]))
+                L.clha_quantize(ctx, self.U_dn[es], E, w.Wd, E, dm, dff, br, r.qd.codes, r.qd.scales, r.qd.zeros,
+                                r.qd.W_hat, **opt(self.lam_dn[es], lb[2 * E:3 * E]))
+                if ns:
+                    q = r.sgu
+                    L.clha_quantize(ctx, self.U_sin[i:i + 1], 1, w.Sgu, 2 * ns, sdff, dm, bs, q.codes, q.scales,
+                                    q.zeros, q.W_hat, **opt(self.lam_sin[i:i + 1], lb[3 * E:3 * E + 2 * ns]))
+                    L.clha_quantize(ctx, self.U_sdn[ss], ns, w.Sd, ns, dm, sdff, bs, r.sd.codes, r.sd.scales,
+                                    r.sd.zeros, r.sd.W_hat, **opt(self.lam_sdn[ss], lb[3 * E + 2 * ns:]))
+            self._last = r
+        if with_loss:      # one read of every weighting's losses
+            host = self.loss_dev.cpu().numpy()
+            for i, m in zip(idx, modes):
+                r, h = self.res[m], host[i]
+                r.qg.loss, r.qu.loss, r.qd.loss = h[:E], h[E:2 * E], h[2 * E:3 * E]
+                if ns:
+                    r.sg.loss, r.su.loss, r.sd.loss = h[3 * E:3 * E + ns], h[3 * E + ns:3 * E + 2 * ns], h[3 * E + 2 * ns:]
 
     def expert_loss(self) -> np.ndarray:
-        """Per routed expert: loss(gate) + loss(up) + loss(down) under the undamped H_comb."""
-        return self.qg.loss + self.qu.loss + self.qd.loss
+        """Per routed expert loss of the most recent weighting."""
+        return self._last.expert_loss()
 
     def columns(self) -> int:
-        """Weight columns quantized per call of quantize()."""
+        """Weight columns quantized per weighting."""
         c = self.E * (2 * self.d_model + self.d_ff)
         if self.n_shared:
             c += self.n_shared * (2 * self.d_model + self.shared_dff)
@@ -274,11 +361,13 @@ class MoECalibration:
 def stack_weights(wl, device) -> MoEWeights:
     """MoEWeights from per-expert (Wg, Wu, Wd) lists (routed, and optionally shared)."""
     routed, shared = wl
-    Wg = torch.stack([w[0] for w in routed]).to(device).contiguous()
-    Wu = torch.stack([w[1] for w in routed]).to(device).contiguous()
-    Wd = torch.stack([w[2] for w in routed]).to(device).contiguous()
+
+    def gu(ws):
+        return torch.stack([w[0] for w in ws] + [w[1] for w in ws]).to(device).contiguous()
+
+    def dn(ws):
+        return torch.stack([w[2] for w in ws]).to(device).contiguous()
+
     if shared:
-        return MoEWeights(Wg, Wu, Wd, torch.stack([w[0] for w in shared]).to(device).contiguous(),
-                          torch.stack([w[1] for w in shared]).to(device).contiguous(),
-                          torch.stack([w[2] for w in shared]).to(device).contiguous())
-    return MoEWeights(Wg, Wu, Wd)
+        return MoEWeights(gu(routed), dn(routed), gu(shared), dn(shared))
+    return MoEWeights(gu(routed), dn(routed))

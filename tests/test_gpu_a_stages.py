@@ -288,7 +288,9 @@ def test_quantize_matches_oracle_on_same_factor(ctx, d_out, d_in, bits, wdt):
     scales = torch.empty((1, d_out, d_in // 128), device=DEV)
     zeros = torch.empty((1, d_out, d_in // 128), dtype=torch.uint8, device=DEV)
     W_hat = torch.empty((1, d_out, d_in), device=DEV)
-    L.clha_quantize(ctx, Ud, 1, Wd, 1, d_out, d_in, bits, codes, scales, zeros, W_hat)
+    lam = torch.tensor([agg["lam"]], dtype=torch.float64, device=DEV)
+    loss = torch.full((1,), float("nan"), dtype=torch.float64, device=DEV)
+    L.clha_quantize(ctx, Ud, 1, Wd, 1, d_out, d_in, bits, codes, scales, zeros, W_hat, lam=lam, loss=loss)
     wc, ws, wz, wh = O.gptq(to64(W), U32.astype(np.float64), bits, 128)
     assert code_agreement(codes[0].cpu().numpy(), wc) >= 0.999
     # first group of every row: identical inputs, so the grid is bit-identical
@@ -297,6 +299,8 @@ def test_quantize_matches_oracle_on_same_factor(ctx, d_out, d_in, bits, wdt):
     got_loss = O.loss(to64(W), to64(W_hat[0]), agg["H_comb"])
     want_loss = O.loss(to64(W), wh, agg["H_comb"])
     assert abs(got_loss - want_loss) <= 1e-3 * want_loss
+    # the in-kernel loss (|E|^2 - lambda |W_hat - W|^2) is the trace of the same W_hat under H_comb
+    assert abs(loss.item() - got_loss) <= 1e-5 * got_loss
     # W_hat is the dequantised code
     q = codes[0].float()
     s = scales[0].repeat_interleave(128, 1)
@@ -321,7 +325,7 @@ def test_quantize_diagonal_hessian_is_rtn_bit_exact(ctx):
 
 
 def test_quantize_batched_shared_factor(ctx):
-    """w_per_u = 2: problems 0,1 use factor 0 and problems 2,3 factor 1 (gate and up share one)."""
+    """n_u = 2: problems 0, 2 use factor 0 and problems 1, 3 factor 1 (gate and up stacked share one)."""
     d_out, d_in, bits = 128, 256, 3
     Us = [np.ascontiguousarray(O.factor(O.aggregate([_H(d_in, s)], [2], "rt")["H_d"]), np.float32) for s in (1, 2)]
     W = (0.02 * torch.randn((4, d_out, d_in), generator=_gen(4))).to(torch.bfloat16)
@@ -331,7 +335,7 @@ def test_quantize_batched_shared_factor(ctx):
     zeros = torch.empty((4, d_out, d_in // 128), dtype=torch.uint8, device=DEV)
     L.clha_quantize(ctx, Ud, 2, W.to(DEV), 4, d_out, d_in, bits, codes, scales, zeros, None)
     for b in range(4):
-        wc, *_ = O.gptq(to64(W[b]), Us[b // 2].astype(np.float64), bits, 128)
+        wc, *_ = O.gptq(to64(W[b]), Us[b % 2].astype(np.float64), bits, 128)
         assert code_agreement(codes[b].cpu().numpy(), wc) >= 0.999
 
 
@@ -345,5 +349,5 @@ def test_loss_matches_oracle(ctx):
     H = torch.from_numpy(np.stack(Hs).astype(np.float32))
     got = L.clha_loss(ctx, W.to(DEV), W_hat.to(DEV), H.to(DEV), 2, batch, d_out, d_in)
     for b in range(batch):
-        want = O.loss(to64(W[b]), to64(W_hat[b]), H[b // 2].double().numpy())
+        want = O.loss(to64(W[b]), to64(W_hat[b]), H[b % 2].double().numpy())
         assert abs(got[b] - want) <= 1e-5 * want

@@ -54,7 +54,7 @@ def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, **over):
     shared = [wl.expert_weights(0, i, shared=True) for i in range(s.n_shared)]
     w = stack_weights((routed, shared), DEV)
     cal = MoECalibration(ctx, 2, max(s.tokens), s.E, s.k, s.d_model, s.d_ff, s.n_shared, s.shared_dff,
-                         s.bits_routed, s.bits_shared, s.damp_frac)
+                         s.bits_routed, s.bits_shared, s.damp_frac, modes=modes)
     for l in range(2):
         cal.collect(l, Xs[l].to(DEV), lgs[l].to(DEV), w)
     torch.cuda.synchronize()
@@ -77,9 +77,10 @@ def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, **over):
             assert rel_fro(sym_from_upper(S_in[l, s.E].double().cpu().numpy()), O.gram(X64[l])) < 1e-4
     # sampled experts: down-projection Hessians and the whole GPTQ path, per weighting
     ref = {}
+    cal.quantize(w, modes)           # every weighting in one pass (batched factorisation)
+    torch.cuda.synchronize()
     for mode in modes:
-        cal.quantize(w, mode)
-        torch.cuda.synchronize()
+        out = cal.res[mode]
         res = O.calibrate_moe_group(X64, [lg.numpy() for lg in lgs], s.k, [tuple(to64(t) for t in r) for r in routed],
                                     [tuple(to64(t) for t in sh) for sh in shared], experts_checked,
                                     s.bits_routed, s.bits_shared, s.group, mode, s.damp_frac, shared_checked)
@@ -89,9 +90,9 @@ def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, **over):
                 for l in range(2):
                     got = sym_from_upper(S_dn[l, e].double().cpu().numpy())
                     assert rel_fro(got, r["H_down"]["S"][l]) < 1e-4, (mode, key, l)
-                qs = {"gate": cal.qg, "up": cal.qu, "down": cal.qd}
+                qs = {"gate": out.qg, "up": out.qu, "down": out.qd}
             else:
-                qs = {"gate": cal.sg, "up": cal.su, "down": cal.sd}
+                qs = {"gate": out.sg, "up": out.su, "down": out.sd}
             for name, q in qs.items():
                 agree = code_agreement(q.codes[e].cpu().numpy(), r[name]["codes"])
                 assert agree >= 0.999, (mode, key, name, agree)
