@@ -34,9 +34,13 @@ constexpr int B_BYTES = KS * BLK * 4;                     // 16 KB: U panel (hi 
 constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;    // 64 KB
 constexpr int UD_OFF = STAGES * STAGE_BYTES;
 constexpr int UINV_OFF = UD_OFF + BLK * BLK * 4;
-constexpr int CODES_OFF = UINV_OFF + BLK * 4;           // block codes, [column][row] bytes
-constexpr int BAR_OFF = CODES_OFF + BLK * R;
-constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;
+constexpr int QROW = BLK + 4;                             // bytes per row of the code buffer (padded)
+constexpr int CODES_OFF = UINV_OFF + BLK * 4;            // block codes, [row][QROW] bytes
+constexpr int QE_OFF = CODES_OFF + R * QROW;             // one quarter's errors, [column][row] floats
+constexpr int QW = 32;                                    // columns per quarter of a block
+constexpr int BAR_OFF = QE_OFF + QW * R * 4;
+constexpr int SMEM_BYTES = BAR_OFF + 128 + 1024;
+constexpr int STG = 68;                                   // staging row (floats): 64 columns + pad
 constexpr int kThreads = 192;
 constexpr uint32_t IDESC = tc::idesc_f32acc(2 /*tf32*/, 0 /*A K-major*/, 0 /*B K-major*/, R, BLK);
 
@@ -65,8 +69,54 @@ __device__ __forceinline__ float to_tf32(float x) {
 
 __device__ __forceinline__ void row_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// 16-byte asynchronous global -> shared copy (all of a thread's copies stay in flight together).
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Columns [32Q, 32Q+32) of the row's block, in order: quantize each, record its error and apply it
+// to the rest of the quarter (unrolled; every index is a compile-time constant).
+template <int Q>
+__device__ __forceinline__ void quarter_sweep(float (&w)[BLK], float s, float z, float maxq, const float* uinv,
+                                              const float (*Ud)[BLK], uint8_t (*qs)[QROW], float (*qe)[R], int t) {
+#pragma unroll
+    for (int jj = 0; jj < QW; ++jj) {
+        const int j = Q * QW + jj;
+        float q = __fadd_rn(rintf(__fdiv_rn(w[j], s)), z);
+        q = fminf(fmaxf(q, 0.f), maxq);
+        const float wh = __fmul_rn(s, __fsub_rn(q, z));
+        const float e = (w[j] - wh) * uinv[j];
+        w[j] = e;                                // a quantized column's register keeps its error
+        qs[t][j] = (uint8_t)q;
+        qe[jj][t] = e;
+#pragma unroll
+        for (int c = j + 1; c < (Q + 1) * QW; ++c) w[c] = fmaf(-e, Ud[j][c], w[c]);
+    }
+}
+
+// The quarter's 32 errors applied, column by column, to every later column of the block: a rolled
+// loop over the errors (read back from shared memory) keeps the code small.
+template <int Q>
+__device__ __forceinline__ void quarter_spill(float (&w)[BLK], const float (*Ud)[BLK], const float (*qe)[R], int t) {
+#pragma unroll 2
+    for (int jj = 0; jj < QW; ++jj) {
+        const float e = qe[jj][t];
+        const float4* u4 = reinterpret_cast<const float4*>(&Ud[Q * QW + jj][(Q + 1) * QW]);
+#pragma unroll
+        for (int c4 = 0; c4 < (BLK - (Q + 1) * QW) / 4; ++c4) {
+            const float4 u = u4[c4];
+            const int c = (Q + 1) * QW + 4 * c4;
+            w[c] = fmaf(-e, u.x, w[c]);
+            w[c + 1] = fmaf(-e, u.y, w[c + 1]);
+            w[c + 2] = fmaf(-e, u.z, w[c + 2]);
+            w[c + 3] = fmaf(-e, u.w, w[c + 3]);
+        }
+    }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -76,7 +126,8 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float (*Ud)[BLK] = reinterpret_cast<float (*)[BLK]>(smem + UD_OFF);
     float* uinv = reinterpret_cast<float*>(smem + UINV_OFF);
-    uint8_t (*qs)[R] = reinterpret_cast<uint8_t (*)[R]>(smem + CODES_OFF);
+    uint8_t (*qs)[QROW] = reinterpret_cast<uint8_t (*)[QROW]>(smem + CODES_OFF);
+    float (*qe)[R] = reinterpret_cast<float (*)[R]>(smem + QE_OFF);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
     const uint32_t full0 = tc::smem_u32(bars);
     const uint32_t empty0 = full0 + 8 * STAGES;
@@ -200,7 +251,13 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
         for (int bb = 0; bb < nblk; ++bb) {
             const int cb = bb * BLK;
             row_bar();                                   // every row thread is done with the last Ud
-            for (int i = 0; i < BLK; ++i) Ud[i][t] = Ub[(size_t)(cb + i) * p.d_in + cb + t];
+            // U's diagonal block: 128 rows x 512 B; thread t copies 16 B pieces (t % 32) of rows t/32 + 4i
+#pragma unroll 8
+            for (int i = 0; i < BLK / 4; ++i) {
+                const int r = (t >> 5) + 4 * i, c4 = (t & 31) * 4;
+                cp_async16(&Ud[r][c4], Ub + (size_t)(cb + r) * p.d_in + cb + c4);
+            }
+            cp_async_wait_all();
             row_bar();
             uinv[t] = 1.0f / Ud[t][t];
             float w[BLK];
@@ -254,68 +311,81 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
             const int g = cb / BLK;
             p.scales[((size_t)b * p.d_out + row) * ngroups + g] = s;
             p.zeros[((size_t)b * p.d_out + row) * ngroups + g] = (uint8_t)z;
-#pragma unroll
-            for (int j = 0; j < BLK; ++j) {
-                float q = __fadd_rn(rintf(__fdiv_rn(w[j], s)), z);
-                q = fminf(fmaxf(q, 0.f), maxq);
-                const float wh = __fmul_rn(s, __fsub_rn(q, z));
-                const float e = (w[j] - wh) * uinv[j];
-                w[j] = e;                                // a quantized column's register keeps its error
-                qs[j][t] = (uint8_t)q;
-#pragma unroll
-                for (int c = 0; c < BLK; ++c)
-                    if (c > j) w[c] = fmaf(-e, Ud[j][c], w[c]);
-            }
+            // 128 columns in four quarters; each column still receives the errors of all earlier
+            // columns in column order, exactly as in a single column-by-column sweep
+            quarter_sweep<0>(w, s, z, maxq, uinv, Ud, qs, qe, t);
+            quarter_spill<0>(w, Ud, qe, t);
+            quarter_sweep<1>(w, s, z, maxq, uinv, Ud, qs, qe, t);
+            quarter_spill<1>(w, Ud, qe, t);
+            quarter_sweep<2>(w, s, z, maxq, uinv, Ud, qs, qe, t);
+            quarter_spill<2>(w, Ud, qe, t);
+            quarter_sweep<3>(w, s, z, maxq, uinv, Ud, qs, qe, t);
             if (p.loss) {
 #pragma unroll
                 for (int c = 0; c < BLK; ++c) e2 = fma((double)w[c], (double)w[c], e2);
             }
-            // errors for the later blocks' lazy updates, as tf32 hi + lo
-            if (bb + 1 < nblk) {
-                float4* eh = reinterpret_cast<float4*>(p.Ehi + wrow + cb);
-                float4* el = reinterpret_cast<float4*>(p.Elo + wrow + cb);
+            // Outputs go through shared memory so that each warp writes whole rows (coalesced).
+            // The U tile is no longer needed: its space stages the errors, 64 columns at a time.
+            qe[0][t] = s;                                // the quarter-error buffer is free too:
+            qe[1][t] = z;                                // it carries each row's grid to the writers
+            float* stg = reinterpret_cast<float*>(smem + UD_OFF);
+            const bool more = bb + 1 < nblk;
 #pragma unroll
-                for (int i = 0; i < BLK / 4; ++i) {
-                    float h[4], l[4];
+            for (int h = 0; h < 2; ++h) {
+                row_bar();                               // Ud reads finished / previous half written out
+                if (more) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        h[j] = to_tf32(w[4 * i + j]);
-                        l[j] = to_tf32(w[4 * i + j] - h[j]);
-                    }
-                    eh[i] = make_float4(h[0], h[1], h[2], h[3]);
-                    el[i] = make_float4(l[0], l[1], l[2], l[3]);
+                    for (int i = 0; i < 16; ++i)
+                        *reinterpret_cast<float4*>(stg + t * STG + 4 * i) =
+                            make_float4(w[64 * h + 4 * i], w[64 * h + 4 * i + 1], w[64 * h + 4 * i + 2],
+                                        w[64 * h + 4 * i + 3]);
                 }
+                row_bar();
+                if (more) {    // errors for the later blocks' lazy updates, as tf32 hi + lo
+#pragma unroll 4
+                    for (int rr = 0; rr < 32; rr += 2) {
+                        const int r = warp * 32 + rr + (lane >> 4), c4 = (lane & 15) * 4;
+                        const float4 v = *reinterpret_cast<const float4*>(stg + r * STG + c4);
+                        const float hx = to_tf32(v.x), hy = to_tf32(v.y), hz = to_tf32(v.z), hw = to_tf32(v.w);
+                        const size_t o = ((size_t)b * p.d_out + r0 + r) * p.d_in + cb + 64 * h + c4;
+                        *reinterpret_cast<float4*>(p.Ehi + o) = make_float4(hx, hy, hz, hw);
+                        *reinterpret_cast<float4*>(p.Elo + o) =
+                            make_float4(to_tf32(v.x - hx), to_tf32(v.y - hy), to_tf32(v.z - hz), to_tf32(v.w - hw));
+                    }
+                }
+            }
+            if (more) {
                 fence_proxy_async_global();
                 tc::mbar_arrive(eready);
             }
-            uint4* co = reinterpret_cast<uint4*>(p.codes + wrow + cb);
-            float4* wo = p.W_hat ? reinterpret_cast<float4*>(p.W_hat + wrow + cb) : nullptr;
-#pragma unroll 1
-            for (int i = 0; i < BLK / 16; ++i) {
-                uint32_t word[4];
+            // codes, w_hat and |W_hat - W|^2 row by row: lane l owns columns 4l..4l+3
+#pragma unroll 2
+            for (int rr = 0; rr < 32; ++rr) {
+                const int r = warp * 32 + rr;
+                const size_t o = ((size_t)b * p.d_out + r0 + r) * p.d_in + cb + 4 * lane;
+                const uint32_t cw = *reinterpret_cast<const uint32_t*>(&qs[r][4 * lane]);
+                *reinterpret_cast<uint32_t*>(p.codes + o) = cw;
+                const float sr = qe[0][r], zr = qe[1][r];
+                float v[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    word[j] = (uint32_t)qs[16 * i + 4 * j][t] | ((uint32_t)qs[16 * i + 4 * j + 1][t] << 8) |
-                              ((uint32_t)qs[16 * i + 4 * j + 2][t] << 16) | ((uint32_t)qs[16 * i + 4 * j + 3][t] << 24);
-                co[i] = make_uint4(word[0], word[1], word[2], word[3]);
-                if (wo) {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        float v[4];
-#pragma unroll
-                        for (int m = 0; m < 4; ++m)
-                            v[m] = __fmul_rn(s, __fsub_rn((float)qs[16 * i + 4 * j + m][t], z));
-                        wo[4 * i + j] = make_float4(v[0], v[1], v[2], v[3]);
+                for (int m = 0; m < 4; ++m) v[m] = __fmul_rn(sr, __fsub_rn((float)((cw >> (8 * m)) & 255u), zr));
+                if (p.W_hat) *reinterpret_cast<float4*>(p.W_hat + o) = make_float4(v[0], v[1], v[2], v[3]);
+                if (p.loss) {
+                    float wv[4];
+                    if (p.w_f32) {
+                        const float4 f = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.W) + o);
+                        wv[0] = f.x; wv[1] = f.y; wv[2] = f.z; wv[3] = f.w;
+                    } else {
+                        const uint2 raw = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(p.W) + o);
+                        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+                        const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+                        wv[0] = f0.x; wv[1] = f0.y; wv[2] = f1.x; wv[3] = f1.y;
                     }
-                }
-            }
-            if (p.loss) {   // |W_hat - W|^2 of this block, W re-read (its registers now hold errors)
-#pragma unroll 4
-                for (int c = 0; c < BLK; ++c) {
-                    const float wv = p.w_f32 ? reinterpret_cast<const float*>(p.W)[wrow + cb + c]
-                                             : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.W)[wrow + cb + c]);
-                    const double dv = (double)__fmul_rn(s, __fsub_rn((float)qs[c][t], z)) - (double)wv;
-                    d2 = fma(dv, dv, d2);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const double dv = (double)v[m] - (double)wv[m];
+                        d2 = fma(dv, dv, d2);
+                    }
                 }
             }
         }
