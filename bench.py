@@ -8,6 +8,11 @@ Inputs are synthetic (seeded), resident in HBM; L2 is flushed (512 MB write) bef
 
   python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
 
+Kernel-level workloads (one JSON line per shape; used for the profiles and the roofline tables):
+  python bench.py --workload hessian --shape 65536x4096 ...   Gram accumulation of dense bf16 X [n, d]
+  python bench.py --workload gptq --shape 32x512x1024 ...     GPTQ of [batch, d_out, d_in] bf16 weights
+  python bench.py --workload factor --shape 32x1024 ...       inverse-Cholesky factor of [batch, d, d]
+
 With N > 1 (torchrun, one process per GPU) every rank calibrates its own independent layer pair:
 weak scaling, no data-path collective; the step time is the max over ranks.
 """
@@ -124,6 +129,33 @@ def max_over_ranks(x: float, world: int) -> float:
     t = torch.tensor([x], dtype=torch.float64, device="cuda")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+KERNEL_SOURCES = {"act": "ffn_act.cu", "gptq": "gptq.cu", "hessian": "hessian.cu", "aggregate": "aggregate.cu",
+                  "factor": "factor.cu"}
+
+
+def source_hash(phase: str) -> str:
+    import hashlib
+    path = os.path.join(ROOT, "post_quantization_expert_b200", "csrc", KERNEL_SOURCES[phase])
+    with open(path, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()[:12]
+
+
+def measured_traffic(phase: str, workload: str):
+    """DRAM bytes per launch from profiles/dram_traffic.txt, only while the kernel source is the one
+    the counters were taken on (its hash is recorded beside the figure)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    cur = source_hash(phase)
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == phase and parts[1] == workload \
+                    and parts[2] == cur:
+                return float(parts[3])
+    return None
 
 
 def blas_threads():
@@ -286,6 +318,7 @@ def run_ours(args, world, rank, local):
     # ---- per-phase timing and the roofline of the dominant kernel
     K = args.steps
     phase_ms = {k: v / K for k, v in timer.totals.items()}
+    phase_calls = {k: v // K for k, v in timer.counts.items()}
     counts = [cal.counts[l].cpu().numpy().astype(np.int64) for l in range(2)]
     dm, dff, E = s.d_model, s.d_ff, s.E
     hess_flops = sum(int(c.sum()) * (dm * (dm + 1) + dff * (dff + 1)) for c in counts)
@@ -306,9 +339,13 @@ def run_ours(args, world, rank, local):
         "act": ("alu", act_flops / 1e12, alu["fp32_tflops"], "TFLOP/s", "expert_act_simt (fp32 FMA)"),
         "aggregate": ("hbm", agg_bytes / 1e9, peaks["hbm_gbs"], "GB/s", "agg_combine"),
     }
-    dom = max((k for k in phase_ms if k in kernels), key=lambda k: phase_ms[k])
+    # the dominant single kernel: phases that are one kernel family per call (the factor is a chain
+    # of seven kernels per call and is reported in the phase table)
+    single = ("act", "gptq", "hessian", "aggregate")
+    dom = max((k for k in phase_ms if k in single), key=lambda k: phase_ms[k])
     bound, work, peak, unit, kname = kernels[dom]
     achieved = work / (phase_ms[dom] / 1e3)
+    traffic = measured_traffic(dom, "moe-E16")
     phases = {k: {"ms": round(v, 4)} for k, v in sorted(phase_ms.items(), key=lambda kv: -kv[1])}
     for k, v in phases.items():
         if k in kernels:
@@ -340,7 +377,8 @@ def run_ours(args, world, rank, local):
             "hessian_tflops": hess_tflops,
             "hessian_frac_of_bf16_peak": hess_tflops / sustained,
             "roofline": {"kernel": kname, "phase": dom, "bound": bound, "achieved": achieved, "peak": peak,
-                         "unit": unit, "frac": achieved / peak, "traffic": None,
+                         "unit": unit, "frac": achieved / peak, "traffic": traffic,
+                         "launches_per_step": phase_calls.get(dom),
                          "peak_source": src if bound in ("tensor", "hbm") else "derived (SM count x lanes x max clock)"},
             "phases_ms_per_step": phases,
             "e2e": {"value": world * cols_per_step / (e2e_ms / 1e3), "unit": "columns/s",
@@ -354,6 +392,67 @@ def run_ours(args, world, rank, local):
     return 0
 
 
+def run_kernel(args):
+    """Kernel-level timing: CUDA events around `steps` launches after `warmup`, inputs resident."""
+    import torch
+    from post_quantization_expert_b200 import clha as L
+    ctx = L.Context(0)
+    peaks, src = load_peaks()
+    alu = alu_peaks(peaks)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(0)
+    for shape in args.shape:
+        dims = [int(v) for v in shape.split("x")]
+        if args.workload == "hessian":
+            n, d = dims
+            X = torch.randn((n, d), device="cuda", generator=g).to(torch.bfloat16)
+            acc = L.Accum(ctx, d, 1, 1)
+            fn = lambda: L.clha_collect(ctx, acc, 0, X, n, d)
+            work, unit, bound, peak = n * d * (d + 1) / 1e12, "TFLOP/s", "tensor", peaks["bf16_tflops"]
+            kname = "syrk_bf16_tc"
+        else:
+            if args.workload == "gptq":
+                B, d_out, d = dims
+            else:
+                B, d = dims
+            A = torch.randn((B, d, d // 2), device="cuda", generator=g)
+            H = (A @ A.transpose(1, 2) / (d // 2) + 0.05 * torch.eye(d, device="cuda")).contiguous()
+            del A
+            U = torch.empty_like(H)
+            if args.workload == "factor":
+                fn = lambda: L.clha_factor(ctx, H, B, d, U)
+                work, unit, bound, peak = B * 2 * d ** 3 / 3 / 1e12, "TFLOP/s", "alu", alu["fp64_tflops"]
+                kname = "fac_* (fp64)"
+            else:
+                L.clha_factor(ctx, H, B, d, U)
+                W = (0.02 * torch.randn((B, d_out, d), device="cuda", generator=g)).to(torch.bfloat16)
+                codes = torch.empty((B, d_out, d), dtype=torch.uint8, device="cuda")
+                sc = torch.empty((B, d_out, d // 128), device="cuda")
+                zs = torch.empty((B, d_out, d // 128), dtype=torch.uint8, device="cuda")
+                Wh = torch.empty((B, d_out, d), device="cuda")
+                fn = lambda: L.clha_quantize(ctx, U, B, W, B, d_out, d, 3, codes, sc, zs, Wh)
+                work, unit, bound, peak = B * d_out * d * d / 1e12, "TFLOP/s", "alu", alu["fp32_tflops"]
+                kname = "gptq_tc"
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(ctx.stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(ctx.stream)
+        torch.cuda.synchronize()
+        L.clha_check(ctx)
+        ms = a.elapsed_time(b) / args.steps
+        achieved = work / (ms / 1e3)
+        print(json.dumps({"workload": args.workload, "shape": shape, "kernel": kname, "ms": ms, "achieved": achieved,
+                          "unit": unit, "bound": bound, "peak": peak, "frac": achieved / peak,
+                          "peak_source": src if bound == "tensor" else "derived (SM count x lanes x max clock)"}))
+        torch.cuda.empty_cache()
+    ctx.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -361,9 +460,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
+    ap.add_argument("--workload", choices=("moe", "hessian", "gptq", "factor"), default="moe",
+                    help="moe: the end-to-end calibration step (default); others: one kernel family")
+    ap.add_argument("--shape", nargs="+", default=[], help="kernel workload shapes, e.g. 65536x4096")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload != "moe":
+        if not args.shape:
+            ap.error("--shape is required for kernel workloads")
+        return run_kernel(args)
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":

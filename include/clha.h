@@ -125,7 +125,8 @@ CLHA_API clha_status clha_gather_noalloc(clha_ctx* ctx, const void* X, clha_dtyp
                                          int64_t* seg, int32_t* perm);
 
 /* Expert FFN activation feeding the down projection: h = SiLU(x Wg^T) * (x Wu^T) per token of
- * each expert, accumulated in float32 and stored as bf16 (round to nearest even). The pages do not
+ * each expert (bf16 products summed in fp32 over 32-term chunks, chunk sums in fp64, SiLU product in
+ * fp64), stored as bf16 (round to nearest even). The pages do not
  * spell this out: the down projection's Hessian needs its input, and that input is this product.
  * X is bf16 [rows, d_model]; Wg, Wu are bf16 [E, d_ff, d_model] (experts stacked); h is bf16
  * [rows, d_ff]. With seg (from clha_gather) rows follow its segments and padding rows of h are

@@ -228,7 +228,7 @@ extern "C" clha_status clha_expert_act(clha_ctx* ctx, const void* X, int64_t row
     SET_DEVICE(ctx);
     LaunchScope launch_scope(ctx);
     CUDA_TRY(launch_expert_act(ctx->stream, ctx->num_sms, (const __nv_bfloat16*)X, rows, d_model, seg, E,
-                               (const __nv_bfloat16*)Wg, (const __nv_bfloat16*)Wu, d_ff, (__nv_bfloat16*)h),
+                               (const __nv_bfloat16*)Wg, (const __nv_bfloat16*)Wu, d_ff, (__nv_bfloat16*)h, ctx->d_err),
              "clha_expert_act");
     return CLHA_OK;
 }
