@@ -87,57 +87,88 @@ __device__ __forceinline__ void mma_tile(const Tile* As, const Tile* Bs, double 
 }
 
 // Cholesky of the 64x64 diagonal tile of panel k (lower), and its inverse into Dall[b][k].
+// Column loop with one barrier per column: column c of L goes to a separate tile (Lt) while the
+// trailing update reads the unscaled column from T, so no thread writes what another reads in the
+// same step. The inverse is built from 16x16 blocks: four warps invert the diagonal blocks by forward
+// substitution in registers, then three bands X[i][j] = -X[i][i] (sum_m L[i][m] X[m][j]).
+constexpr int SMEM3 = 3 * TILE_DOUBLES * sizeof(double) + NB * sizeof(double);
+
 __global__ void __launch_bounds__(256) fac_potrf(double* __restrict__ A, int d, int k, double* __restrict__ Dall,
                                                  int* err) {
     const int b = blockIdx.x;
     double* Ab = A + (size_t)b * d * d;
     extern __shared__ double dsm[];
     Tile* T = reinterpret_cast<Tile*>(dsm);
-    Tile* X = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
-    __shared__ int bad;
+    Tile* Lt = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
+    Tile* X = reinterpret_cast<Tile*>(dsm + 2 * TILE_DOUBLES);
+    double* dinv = dsm + 3 * TILE_DOUBLES;           // 1 / L[c][c]
+    const int tid = threadIdx.x;
     const int k0 = k * NB;
     load_tile(T, Ab + (size_t)k0 * d + k0, d);
-    if (threadIdx.x == 0) bad = -1;
     __syncthreads();
+    int bad = -1;
     for (int c = 0; c < NB; ++c) {
-        // every thread reads the pivot; a non-positive one poisons the factor with NaN
-        double p = T[c][c];
+        const double p = T[c][c];
         const bool ok = (p > 0.0) && isfinite(p);
-        p = ok ? sqrt(p) : __longlong_as_double(0x7ff8000000000000ll);
-        if (!ok && threadIdx.x == 0 && bad < 0) bad = c;
-        const double inv = 1.0 / p;
-        __syncthreads();                           // all reads of T[c][c] precede the writes below
-        if (threadIdx.x == 0) T[c][c] = p;
-        if (threadIdx.x > c && threadIdx.x < NB) T[threadIdx.x][c] *= inv;
-        __syncthreads();
-        // trailing lower triangle: thread owns column cc = tid % 64 and every 4th row from c+1
-        const int cc = threadIdx.x & 63;
+        const double inv = ok ? rsqrt(p) : __longlong_as_double(0x7ff8000000000000ll);
+        if (!ok && bad < 0) bad = c;
+        if (tid > c && tid < NB) Lt[tid][c] = T[tid][c] * inv;
+        if (tid == 0) { Lt[c][c] = p * inv; dinv[c] = inv; }
+        const int cc = tid & 63;
         if (cc > c) {
-            const double tc_ = T[cc][c];
-            for (int r = c + 1 + (threadIdx.x >> 6); r < NB; r += 4)
-                if (r >= cc) T[r][cc] -= T[r][c] * tc_;
+            const double lcc = T[cc][c] * inv;
+            for (int r = c + 1 + (tid >> 6); r < NB; r += 4)
+                if (r >= cc) T[r][cc] -= (T[r][c] * inv) * lcc;
         }
         __syncthreads();
     }
-    if (threadIdx.x == 0 && bad >= 0) clha_record_error(err, CLHA_ERR_NOT_PD, b, d - 1 - (k0 + bad), KID_FACTOR);
-    // inverse: row by row, X[r][c] = (delta_rc - sum_{m=c}^{r-1} T[r][m] X[m][c]) / T[r][r];
-    // 4 threads share one column's dot product (lanes 4c..4c+3 of the same warp)
-    const int col = threadIdx.x >> 2, part = threadIdx.x & 3;
-    for (int r = 0; r < NB; ++r) {
-        double sum = 0.0;
-        if (col < r)
-            for (int m = col + part; m < r; m += 4) sum = fma(T[r][m], X[m][col], sum);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-        if (part == 0) X[r][col] = (col > r) ? 0.0 : (((r == col) ? 1.0 : 0.0) - sum) / T[r][r];
+    if (tid == 0 && bad >= 0) clha_record_error(err, CLHA_ERR_NOT_PD, b, d - 1 - (k0 + bad), KID_FACTOR);
+    // (1) diagonal 16x16 blocks: warp i, lane j < 16 solves column j of block i
+    const int warp = tid >> 5, lane = tid & 31;
+    if (warp < 4 && lane < 16) {
+        const int o = 16 * warp, j = lane;
+        double x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            double s = (r == j) ? 1.0 : 0.0;
+#pragma unroll
+            for (int m = 0; m < r; ++m) s -= (m >= j) ? Lt[o + r][o + m] * x[m] : 0.0;
+            x[r] = (r >= j) ? s * dinv[o + r] : 0.0;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) X[o + r][o + j] = x[r];
+    }
+    // zero the strict upper blocks of X
+    for (int i = tid; i < NB * NB; i += 256) {
+        const int r = i >> 6, c = i & 63;
+        if ((c >> 4) > (r >> 4)) X[r][c] = 0.0;
+    }
+    __syncthreads();
+    // (2) bands: T holds the partial products (T is free now)
+    for (int delta = 1; delta < 4; ++delta) {
+        const int nblk = 4 - delta;
+        for (int e = tid; e < nblk * 256; e += 256) {       // Tp = sum_{m in blocks j..i-1} L[i][m] X[m][j]
+            const int j = e >> 8, i = j + delta, r = (e >> 4) & 15, s = e & 15;
+            double acc = 0.0;
+            for (int m = 16 * j; m < 16 * i; ++m) acc = fma(Lt[16 * i + r][m], X[m][16 * j + s], acc);
+            T[16 * i + r][16 * j + s] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < nblk * 256; e += 256) {       // X[i][j] = -X[i][i] Tp
+            const int j = e >> 8, i = j + delta, r = (e >> 4) & 15, s = e & 15;
+            double acc = 0.0;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) acc = fma(X[16 * i + r][16 * i + q], T[16 * i + q][16 * j + s], acc);
+            X[16 * i + r][16 * j + s] = -acc;
+        }
         __syncthreads();
     }
     double* Db = Dall + ((size_t)b * (d / NB) + k) * NB * NB;
 #pragma unroll
     for (int it = 0; it < PER_THREAD; ++it) {
-        const int i = it * 256 + threadIdx.x;
+        const int i = it * 256 + tid;
         const int r = i >> 6, c = i & 63;
-        Ab[(size_t)(k0 + r) * d + k0 + c] = (c <= r) ? T[r][c] : 0.0;
+        Ab[(size_t)(k0 + r) * d + k0 + c] = (c <= r) ? Lt[r][c] : 0.0;
         Db[i] = X[r][c];
     }
 }
@@ -268,7 +299,8 @@ cudaError_t launch_factor(cudaStream_t s, const float* H_d, int batch, int d, fl
     const int nbk = d / NB;
     const int smem = SMEM2;
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(fac_potrf, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(fac_potrf, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM3)) != cudaSuccess)
+        return e;
     if ((e = cudaFuncSetAttribute(fac_trsm, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(fac_update, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(fac_inv_row, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
@@ -282,7 +314,7 @@ cudaError_t launch_factor(cudaStream_t s, const float* H_d, int batch, int d, fl
     e = cudaMemsetAsync(X, 0, (size_t)batch * dd * sizeof(double), s);
     if (e != cudaSuccess) return e;
     for (int k = 0; k < nbk; ++k) {
-        fac_potrf<<<batch, 256, smem, s>>>(A, d, k, Dall, err);
+        fac_potrf<<<batch, 256, SMEM3, s>>>(A, d, k, Dall, err);
         clha_note_launches(1);
         const int rem = nbk - k - 1;
         if (rem > 0) {

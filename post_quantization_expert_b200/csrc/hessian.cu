@@ -7,9 +7,15 @@
 //              (128-byte swizzle; both operands are "M/N-major": one token row = 64 contiguous
 //              channels, which is how X is laid out, so no transpose is ever materialised).
 //   warp 1     MMA issuer: tcgen05.mma kind::f16 M=128 N=256 K=16, four per 64-token block,
-//              accumulating in TMEM; two accumulators (512 TMEM columns) so the epilogue of one
-//              tile overlaps the MMAs of the next.
-//   warps 2-5  epilogue: tcgen05.ld of the fp32 tile, read-modify-write into S (float4).
+//              accumulating in TMEM one chunk of at most KCHUNK tokens at a time; two accumulators
+//              (512 TMEM columns) so the epilogue of one chunk overlaps the MMAs of the next.
+//   warps 2-5  epilogue: tcgen05.ld of the fp32 chunk sum, one 32x32 sub-tile per warp at a time
+//              written to a swizzled shared-memory buffer (two per warp) and added into S by a TMA
+//              bulk reduce (the L2 performs the fp32 adds), so the epilogue never reads S.
+// Why chunks: the tensor core's fp32 accumulation does not round to nearest, and over tens of
+// thousands of tokens the Gram diagonal (a sum of positive terms) drifts low by a few 1e-4
+// relative. Summing at most KCHUNK tokens per accumulator and adding the chunk sums into S with
+// round-to-nearest fp32 adds bounds that drift by the chunk length instead of the token count.
 // Only tiles that touch the upper triangle are computed (rows tile r <= 2c+1 for column tile c);
 // entries below the diagonal inside those tiles are correct values but the upper triangle is the
 // authoritative one. Segments from the gather are 128-row aligned with zero padding, so a token
@@ -22,10 +28,13 @@
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int KCHUNK_BLOCKS = 64;  // KCHUNK = 4096 tokens per TMEM accumulation
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int STG_OFF = STAGES * STAGE_BYTES + 1024;   // after the barriers, 1024-aligned for the swizzle
+constexpr int STG_BYTES = 4 * 2 * 32 * 32 * 4;         // 4 epilogue warps x 2 buffers x 32x32 fp32
+constexpr int SMEM_BYTES = STG_OFF + STG_BYTES + 1024;  // + alignment slack of the dynamic base
 constexpr int kThreads = 192;
 constexpr uint32_t IDESC = tc::idesc_f32acc(1 /*bf16*/, 1 /*A MN-major*/, 1 /*B MN-major*/, BM, BN);
 
@@ -55,7 +64,8 @@ __device__ __forceinline__ void slot_range(const SyrkParams& p, int e, int64_t& 
     else { t0 = 0; cnt = p.rows; }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) syrk_bf16_tc(const __grid_constant__ CUtensorMap tmX, SyrkParams p) {
+__global__ void __launch_bounds__(kThreads, 1) syrk_bf16_tc(const __grid_constant__ CUtensorMap tmX,
+                                                            const __grid_constant__ CUtensorMap tmS, SyrkParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
@@ -81,6 +91,7 @@ __global__ void __launch_bounds__(kThreads, 1) syrk_bf16_tc(const __grid_constan
         *abort_flag = 0;
         tc::fence_barrier_init();
         tc::prefetch_tmap(&tmX);
+        tc::prefetch_tmap(&tmS);
     }
     if (warp == 1) tc::tmem_alloc(tc::smem_u32(tmem_slot), 512);
     tc::fence_before_sync();
@@ -128,35 +139,39 @@ __global__ void __launch_bounds__(kThreads, 1) syrk_bf16_tc(const __grid_constan
                 int64_t t0, cnt;
                 slot_range(p, e, t0, cnt);
                 const int nk = (int)((cnt + BK - 1) / BK);
-                if (nk == 0) continue;
-                const int acc = tcount & 1;
-                const uint32_t aph = (tcount >> 1) & 1;
-                if (!tc::mbar_wait_bounded(tempty0 + 8 * acc, aph ^ 1, abort_flag)) break;
-                tc::fence_after_sync();
-                const uint32_t d_tmem = tmem + acc * BN;
-                for (int kb = 0; kb < nk; ++kb, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1;
-                    if (!tc::mbar_wait_bounded(full0 + 8 * s, ph, abort_flag)) { ok = false; break; }
+                for (int kc = 0; kc < nk && ok; kc += KCHUNK_BLOCKS) {
+                    const int kend = min(nk, kc + KCHUNK_BLOCKS);
+                    const int acc = tcount & 1;
+                    const uint32_t aph = (tcount >> 1) & 1;
+                    if (!tc::mbar_wait_bounded(tempty0 + 8 * acc, aph ^ 1, abort_flag)) { ok = false; break; }
                     tc::fence_after_sync();
-                    const uint32_t a_base = tc::smem_u32(smem + s * STAGE_BYTES);
-                    const uint32_t b_base = a_base + A_BYTES;
+                    const uint32_t d_tmem = tmem + acc * BN;
+                    for (int kb = kc; kb < kend; ++kb, ++it) {
+                        const int s = it % STAGES;
+                        const uint32_t ph = (it / STAGES) & 1;
+                        if (!tc::mbar_wait_bounded(full0 + 8 * s, ph, abort_flag)) { ok = false; break; }
+                        tc::fence_after_sync();
+                        const uint32_t a_base = tc::smem_u32(smem + s * STAGE_BYTES);
+                        const uint32_t b_base = a_base + A_BYTES;
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t ad = tc::sw128_desc(a_base + kk * 2048, 8192, 1024);
-                        const uint64_t bd = tc::sw128_desc(b_base + kk * 2048, 8192, 1024);
-                        tc::mma_f16(d_tmem, ad, bd, IDESC, (kb | kk) != 0);
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint64_t ad = tc::sw128_desc(a_base + kk * 2048, 8192, 1024);
+                            const uint64_t bd = tc::sw128_desc(b_base + kk * 2048, 8192, 1024);
+                            tc::mma_f16(d_tmem, ad, bd, IDESC, ((kb - kc) | kk) != 0);
+                        }
+                        tc::mma_commit(empty0 + 8 * s);
                     }
-                    tc::mma_commit(empty0 + 8 * s);
+                    if (!ok) break;
+                    tc::mma_commit(tfull0 + 8 * acc);
+                    ++tcount;
                 }
-                if (!ok) break;
-                tc::mma_commit(tfull0 + 8 * acc);
-                ++tcount;
             }
         }
         __syncwarp();
     } else {
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        const uint32_t stg = tc::smem_u32(smem + STG_OFF) + q * 8192;
+        int sb = 0;
         int tcount = 0;
         for (int w = blockIdx.x; w < p.total_tiles; w += gridDim.x) {
             const int e = w / p.tiles_per_slot;
@@ -164,37 +179,48 @@ __global__ void __launch_bounds__(kThreads, 1) syrk_bf16_tc(const __grid_constan
             decode_tile(w % p.tiles_per_slot, p.nr, p.nc, r, c);
             int64_t t0, cnt;
             slot_range(p, e, t0, cnt);
-            if (cnt == 0) continue;
-            const int acc = tcount & 1;
-            const uint32_t aph = (tcount >> 1) & 1;
-            if (!tc::mbar_wait_bounded(tfull0 + 8 * acc, aph, abort_flag)) break;
-            tc::fence_after_sync();
-            const int row = r * BM + q * 32 + lane;
-            float* Srow = p.S + (size_t)e * p.d * p.d + (size_t)row * p.d;
+            const int nk = (int)((cnt + BK - 1) / BK);
             const int warp_row_min = r * BM + q * 32;
+            const int srow = e * p.d + warp_row_min;  // row of this warp's sub-tiles in the [E*d, d] view
+            bool ok = true;
+            for (int kc = 0; kc < nk; kc += KCHUNK_BLOCKS) {
+                const int acc = tcount & 1;
+                const uint32_t aph = (tcount >> 1) & 1;
+                if (!tc::mbar_wait_bounded(tfull0 + 8 * acc, aph, abort_flag)) { ok = false; break; }
+                tc::fence_after_sync();
 #pragma unroll 1
-            for (int ch = 0; ch < BN / 32; ++ch) {
-                const int col0 = c * BN + ch * 32;
-                if (col0 >= p.d) break;
-                if (col0 + 31 < warp_row_min) continue;  // whole chunk strictly below the diagonal
-                uint32_t v[32];
-                tc::tmem_ld_32x32b_x32(tmem + acc * BN + ch * 32 + ((uint32_t)(q * 32) << 16), v);
-                tc::tmem_wait_ld();
-                float4* dst = reinterpret_cast<float4*>(Srow + col0);
+                for (int ch = 0; ch < BN / 32; ++ch) {
+                    const int col0 = c * BN + ch * 32;
+                    if (col0 >= p.d) break;
+                    if (col0 + 31 < warp_row_min) continue;  // whole sub-tile strictly below the diagonal
+                    uint32_t v[32];
+                    tc::tmem_ld_32x32b_x32(tmem + acc * BN + ch * 32 + ((uint32_t)(q * 32) << 16), v);
+                    tc::tmem_wait_ld();
+                    const uint32_t buf = stg + sb * 4096;
+                    if (lane == 0) tc::bulk_wait_read<1>();  // the reduce that last used buf has read it
+                    __syncwarp();
+                    // row `lane` of the box; 16-byte chunk j sits at j ^ (row % 8) (128-byte swizzle)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    float4 o = dst[j];
-                    o.x += __uint_as_float(v[4 * j + 0]);
-                    o.y += __uint_as_float(v[4 * j + 1]);
-                    o.z += __uint_as_float(v[4 * j + 2]);
-                    o.w += __uint_as_float(v[4 * j + 3]);
-                    dst[j] = o;
+                    for (int j = 0; j < 8; ++j)
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                     ::"r"(buf + lane * 128 + ((j ^ (lane & 7)) << 4)), "r"(v[4 * j]),
+                                     "r"(v[4 * j + 1]), "r"(v[4 * j + 2]), "r"(v[4 * j + 3]) : "memory");
+                    tc::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tc::tma_reduce_add_2d(&tmS, buf, col0, srow);
+                        tc::bulk_commit();
+                    }
+                    sb ^= 1;
                 }
+                tc::fence_before_sync();
+                tc::mbar_arrive(tempty0 + 8 * acc);
+                ++tcount;
             }
-            tc::fence_before_sync();
-            tc::mbar_arrive(tempty0 + 8 * acc);
-            ++tcount;
+            if (!ok) break;
         }
+        if (lane == 0) tc::bulk_wait_all();
+        __syncwarp();
     }
 
     __syncthreads();
@@ -264,8 +290,10 @@ __global__ void __launch_bounds__(256) syrk_f32_simt(const float* __restrict__ X
 
 cudaError_t launch_collect_bf16(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t rows, int d,
                                 const int64_t* seg, int E, float* S_base, int64_t* counts_base, int* err) {
-    CUtensorMap tm;
+    CUtensorMap tm, tmS;
     cudaError_t e = make_tmap_2d(&tm, X, (uint64_t)rows, (uint64_t)d, 2, 64, 64);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_2d(&tmS, S_base, (uint64_t)E * d, (uint64_t)d, 4, 32, 32);
     if (e != cudaSuccess) return e;
     static bool attr_set = false;
     if (!attr_set) {
@@ -286,7 +314,7 @@ cudaError_t launch_collect_bf16(cudaStream_t s, int num_sms, const __nv_bfloat16
     p.total_tiles = p.tiles_per_slot * E;
     p.err = err;
     int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
-    syrk_bf16_tc<<<grid, kThreads, SMEM_BYTES, s>>>(tm, p);
+    syrk_bf16_tc<<<grid, kThreads, SMEM_BYTES, s>>>(tm, tmS, p);
     clha_note_launches(1);
     add_counts<<<(E + 255) / 256, 256, 0, s>>>(counts_base, seg, E, rows);
     clha_note_launches(1);

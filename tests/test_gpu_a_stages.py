@@ -72,7 +72,8 @@ def test_gather_segments(ctx, n, E, k, d):
 
 
 # ------------------------------------------------------------------------------------ collection
-@pytest.mark.parametrize("n,d", [(1000, 512), (129, 1408), (1, 256), (4096, 1024), (777, 2048)])
+@pytest.mark.parametrize("n,d", [(1000, 512), (129, 1408), (1, 256), (4096, 1024), (777, 2048), (9000, 384),
+                                 (65536, 256)])
 def test_collect_dense_bf16(ctx, n, d):
     g = _gen(n * d)
     X = (torch.randn((n, d), generator=g) * (1 + torch.rand(d, generator=g))).to(torch.bfloat16).to(DEV)

@@ -1,0 +1,142 @@
+"""Full-size parity on the two large workloads, where the float64 oracle cannot redo everything:
+
+* the 12-pair stack (24 layers, E16 top-2 + 2 always-active experts, 131072 tokens per layer): the GPU
+  calibrates every pair with both weightings; the oracle checks every layer's routing counts and, on
+  sampled pairs (drift 0 and drift 1) and experts, the Hessians, codes and losses end to end;
+* the dense stress shape (W 8192 x 28672 bf16 shared by 4 layers of 65536 tokens, 4-bit): the oracle
+  checks a random 512-channel principal block of every layer's Gram matrix and of the aggregate;
+  factor and GPTQ are checked through properties that hold at any size (U^T U H_d = I on sampled
+  vectors; each sampled row's codes, grids and errors are consistent with the GPTQ recurrence
+  W - W_hat = E U; the in-kernel loss equals the trace computed directly).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from helpers import code_agreement, rel_fro, sym_from_upper, to64
+from post_quantization_expert_b200.pipeline import DenseCalibration, MoECalibration, stack_weights
+from synth import workload
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+DEV = "cuda:0"
+
+
+def test_stack_of_12_pairs_full_size(ctx):
+    wl = workload(4, DEV)
+    s = wl.spec
+    checked_pairs, checked_experts = (0, 3), [0, 9]
+    for gi, (la, lb) in enumerate(s.group_of_layers):
+        routed = [wl.expert_weights(gi, e) for e in range(s.E)]
+        shared = [wl.expert_weights(gi, i, shared=True) for i in range(s.n_shared)]
+        w = stack_weights((routed, shared), DEV)
+        cal = MoECalibration(ctx, 2, s.tokens[la], s.E, s.k, s.d_model, s.d_ff, s.n_shared, s.shared_dff,
+                             s.bits_routed, s.bits_shared, s.damp_frac, modes=s.alpha_modes)
+        lgs = [wl.logits(la), wl.logits(lb)]
+        for j, layer in enumerate((la, lb)):
+            cal.collect(j, wl.x(layer, cache=False), lgs[j], w)
+        cal.quantize(w, s.alpha_modes)
+        torch.cuda.synchronize()
+        routes = [O.route_topk(lg.cpu().numpy(), s.k) for lg in lgs]
+        for j in range(2):
+            np.testing.assert_array_equal(cal.counts[j].cpu().numpy(), routes[j][1])
+        for r in cal.res.values():
+            assert np.all(np.isfinite(r.expert_loss())) and np.all(r.expert_loss() > 0)
+        if gi not in checked_pairs:
+            continue
+        X64 = [to64(wl.x(la, cache=False)), to64(wl.x(lb, cache=False))]
+        S_in, _ = cal.acc_in.buffers()
+        S_dn, _ = cal.acc_dn.buffers()
+        for mode in s.alpha_modes:
+            ref = O.calibrate_moe_group(X64, [lg.cpu().numpy() for lg in lgs], s.k,
+                                        [tuple(to64(t) for t in r) for r in routed], [], checked_experts,
+                                        s.bits_routed, s.bits_shared, s.group, mode, s.damp_frac)
+            out = cal.res[mode]
+            for (kind, e), r in ref["experts"].items():
+                for j in range(2):
+                    assert rel_fro(sym_from_upper(S_in[j, e].double().cpu().numpy()), r["H_in"]["S"][j]) < 1e-4
+                    assert rel_fro(sym_from_upper(S_dn[j, e].double().cpu().numpy()), r["H_down"]["S"][j]) < 1e-4
+                qs = {"gate": out.qg, "up": out.qu, "down": out.qd}
+                for name, q in qs.items():
+                    assert code_agreement(q.codes[e].cpu().numpy(), r[name]["codes"]) >= 0.999, (gi, mode, e, name)
+                got = sum(qs[n].loss[e] for n in qs)
+                assert abs(got - r["loss"]) <= 1e-3 * r["loss"], (gi, mode, e, got, r["loss"])
+        del cal, w
+        torch.cuda.empty_cache()
+
+
+def _gptq_consistency(W, W_hat, codes, scales, zeros, U, rows, bits):
+    """Codes, grids and W_hat of sampled rows follow the GPTQ recurrence with this U: the errors
+    E = (W - W_hat) U^-1 give each column's current value w_j = W_hat_j + E_j U_jj and each group's
+    current values at its start; the float32 grid of those values and the rounding of w_j must
+    reproduce the kernel's grid (scales to 1e-4 relative) and codes (boundary cases excepted)."""
+    maxq = np.float32(2 ** bits - 1)
+    d_in = W.shape[1]
+    agree = total = grid_ok = groups = 0
+    for r in rows:
+        Wr = W[r].double()
+        D = (Wr - W_hat[r].double())[None, :]
+        E = torch.linalg.solve_triangular(U, D, upper=True, left=False)[0]           # D = E U
+        cur = (W_hat[r].double() + E * torch.diagonal(U)).cpu().numpy()
+        for g in range(d_in // 128):
+            c0 = 128 * g
+            start = (Wr[c0:c0 + 128] - E[:c0] @ U[:c0, c0:c0 + 128]).cpu().numpy().astype(np.float32)
+            xmin = min(np.float32(0), start.min())
+            xmax = max(np.float32(0), start.max())
+            sg = np.float32(np.float32(xmax - xmin) / maxq)
+            zg = np.float32(np.rint(np.float32(-xmin) / sg))
+            groups += 1
+            # the start values here come from a float64 solve, the kernel's from its own float32
+            # accumulation of the same sums: scales agree to a few ulps, zero points exactly
+            grid_ok += (abs(sg - scales[r, g].item()) <= 1e-4 * sg) and (zg == zeros[r, g].item())
+            w32 = cur[c0:c0 + 128].astype(np.float32)
+            s_k, z_k = np.float32(scales[r, g].item()), np.float32(zeros[r, g].item())
+            q = np.clip(np.rint((w32 / s_k).astype(np.float32)) + z_k, 0, maxq)
+            agree += int(np.sum(q == codes[r, c0:c0 + 128].cpu().numpy()))
+            total += 128
+    return agree / total, grid_ok / groups
+
+
+def test_dense_stress_shape_full_size(ctx):
+    wl = workload(5, DEV)
+    s = wl.spec
+    L, n, d = s.n_layers, s.tokens[0], s.d_model
+    W = wl.dense_weight()
+    cal = DenseCalibration(ctx, s.d_out, d, L, s.bits_routed, s.damp_frac)
+    g = np.random.default_rng(5)
+    J = np.sort(g.choice(d, 512, replace=False))
+    Jt = torch.from_numpy(J).to(DEV)
+    sub_ref = []
+    for l in range(L):
+        X = wl.x(l, cache=False)
+        cal.collect(l, X)
+        sub_ref.append(O.gram(to64(X[:, Jt])))
+        del X
+        torch.cuda.empty_cache()
+    alpha, lam = cal.quantize(W, "rt", want_host=True)
+    torch.cuda.synchronize()
+    S, cnt = cal.acc.buffers()
+    assert cnt[:, 0].tolist() == [n] * L
+    np.testing.assert_allclose(alpha[0], [0.25] * 4, rtol=1e-15)
+    for l in range(L):
+        blk = S[l, 0][Jt][:, Jt].double().cpu().numpy()
+        full_blk = np.where(J[:, None] <= J[None, :], blk, blk.T)          # upper triangle is authoritative
+        assert rel_fro(full_blk, sub_ref[l]) < 1e-4, l
+    agg_ref = O.aggregate(sub_ref, [n] * L, "rt")
+    assert rel_fro(cal.H_comb[0][Jt][:, Jt].double().cpu().numpy(), agg_ref["H_comb"]) < 1e-4
+    # factor: U^T U H_d v = v on random vectors (float64 products of the float32 outputs)
+    U = cal.U[0].double()
+    Hd = cal.H_d[0].double()
+    v = torch.randn((d, 4), dtype=torch.float64, device=DEV, generator=torch.Generator(DEV).manual_seed(1))
+    res = U.T @ (U @ (Hd @ v)) - v
+    assert (torch.linalg.norm(res) / torch.linalg.norm(v)).item() < 1e-2   # fp32-rounded U, cond(H_d) ~ 1e4
+    assert torch.all(torch.diagonal(U) > 0) and torch.count_nonzero(torch.tril(cal.U[0], -1)) == 0
+    # GPTQ: sampled rows consistent with the recurrence
+    rows = g.choice(s.d_out, 6, replace=False)
+    agree, grid_ok = _gptq_consistency(W, cal.q.W_hat[0], cal.q.codes[0], cal.q.scales[0], cal.q.zeros[0], U, rows,
+                                       s.bits_routed)
+    assert agree >= 0.999 and grid_ok >= 0.99, (agree, grid_ok)
+    # loss: in-kernel |E|^2 - lambda |W_hat - W|^2 equals the direct trace under H_comb
+    Dl = (cal.q.W_hat[0].double() - W.double())
+    direct = torch.sum((Dl @ cal.H_comb[0].double()) * Dl).item()
+    assert abs(cal.q.loss[0] - direct) <= 1e-3 * direct
