@@ -396,7 +396,7 @@ extern "C" clha_status clha_factor(clha_ctx* ctx, const float* H_damped, int bat
     void* ws = nullptr;
     clha_status st = clha_workspace(ctx, factor_workspace_bytes(batch, d), &ws);
     if (st) return st;
-    CUDA_TRY(launch_factor(ctx->stream, H_damped, batch, d, U, ws, ctx->d_err), "clha_factor");
+    CUDA_TRY(launch_factor(ctx->stream, ctx->num_sms, H_damped, batch, d, U, ws, ctx->d_err), "clha_factor");
     return CLHA_OK;
 }
 

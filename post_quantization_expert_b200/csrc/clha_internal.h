@@ -96,8 +96,8 @@ cudaError_t launch_aggregate(cudaStream_t s, const float* S, const int64_t* coun
                              clha_alpha_args a, double damp_frac, float* H_comb, float* H_d,
                              double* d_alpha, double* d_lambda, int* err);
 size_t factor_workspace_bytes(int batch, int d);
-cudaError_t launch_factor(cudaStream_t s, const float* H_d, int batch, int d, float* U,
-                          void* ws, int* err);
+cudaError_t launch_factor(cudaStream_t s, int num_sms, const float* H_d, int batch, int d, float* U, void* ws,
+                          int* err);
 size_t quantize_workspace_bytes(int batch, int d_out, int d_in);
 cudaError_t launch_quantize(cudaStream_t s, const float* U, int n_u, const void* W, int w_is_f32,
                             int batch, int d_out, int d_in, int bits, uint8_t* codes, float* scales,

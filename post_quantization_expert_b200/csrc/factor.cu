@@ -5,338 +5,523 @@
 // is positive, so it is THE upper Cholesky factor of H_d^-1. This needs one Cholesky and one
 // triangular inverse (no explicit inverse of H_d, no second factorisation).
 //
-// Float64 throughout, blocked with 64 x 64 tiles, batched over problems (grid.z / grid.y = problem):
-//   fac_load      A = J H_d J in float64
-//   per panel k:  fac_potrf   Cholesky of the diagonal tile in shared memory, plus its inverse
-//                 fac_trsm    panel tiles A[i][k] <- A[i][k] L_kk^-T   (a GEMM with the inverse)
-//                 fac_update  trailing lower tiles A[i][j] -= A[i][k] A[j][k]^T
-//   X = L^-1, right-looking by block rows (diagonal tiles come from potrf; X starts as I):
-//     fac_inv_row   X[i][j] <- Linv_ii X[i][j]           for j < i
-//     fac_inv_upd   X[r][j] -= L[r][i] X[i][j]           for r > i, j <= i
-//   so X[i][j] = Linv_ii (I - sum_{m<i} L[i][m] X[m][j]), every launch one 64^3 product per CTA.
-//   fac_store     U = J X J as float32 (strict lower triangle zero)
+// Float64 throughout, on 64 x 64 tiles (nt = d / 64 per side), batched over problems. Three launches:
+//   fac_load    A = J H_d J, lower tiles, tile-major float64 (each tile 32 KB contiguous)
+//   fac_dag     one persistent kernel that runs the whole blocked Cholesky and the blocked inverse
+//               as a graph of tile tasks (below)
+//   fac_store   U = J Y^T J as float32, strict lower triangle zero
+//
+// Tile tasks. The inverse is kept transposed, Y = L^-T (upper), so that every product has the form
+// C <- alpha C + beta P Q^T with row-major tiles P and Q:
+//   P(m)        L_mm = chol(A_mm), D_m = L_mm^-1, Y_mm = D_m^T                 (one CTA, in shared memory)
+//   S(i,m)      L_im = A_im D_m^T                                                i > m
+//   G(i,j,m)    A_ij -= L_im L_jm^T                                              i >= j > m
+//   Q(j,i,m)    R_ji += Y_jm L_im^T         (R_ji accumulates in Y_ji; first term m = j overwrites)
+//   F(j,m)      Y_jm = -R_jm D_m^T                                               j < m
+// since L X = I with X = L^-1 = Y^T gives X_ij = -D_i sum_{m=j}^{i-1} L_im X_mj for i > j.
+//
+// Scheduling: tasks are numbered in a topological order (stages with a one-panel lookahead, see
+// stage_counts; problems interleaved inside each class) and CTAs take numbers from a global counter. Every tile has a monotone state counter: A_ij counts the
+// updates applied (j + 1 once L_ij is final); Y_ji counts the Q terms applied (i - j + 1 once final).
+// A task waits (thread 0, acquire loads, bounded by a time limit) until its inputs have reached the
+// states it needs, runs, and publishes its output tile's new state with a release store. Any task
+// waited on has a smaller number and so is held by a CTA that is already running: the schedule
+// cannot deadlock however many CTAs are resident. Tile data moves through L2 only (cp.async.cg and
+// ld.global.cg), never through a stale L1 line.
+//
+// Products run on the FP64 tensor-core path (mma.sync m8n8k4 f64): 8 warps, each a 32 x 16 block
+// of the 64 x 64 output, operands in padded shared memory.
 // A non-positive pivot is recorded (problem, original column) and the problem's factor is NaN.
 #include "clha_internal.h"
 
 namespace {
 
 constexpr int NB = 64;
-constexpr int LD = NB + 2;   // shared-memory row length (doubles): 16-byte aligned rows, few bank conflicts
+constexpr int LD = NB + 4;   // padded shared row (doubles): conflict-free m8n8k4 fragment loads
 constexpr int TILE_DOUBLES = NB * LD;
-constexpr int SMEM2 = 2 * TILE_DOUBLES * sizeof(double);
+constexpr int TILE_ELEMS = NB * NB;
+constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;
 
 typedef double Tile[LD];
 
-__global__ void fac_load(const float* __restrict__ H, int d, double* __restrict__ A) {
+__device__ __forceinline__ uint64_t gtimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(int* p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void dmma(double& c0, double& c1, double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                 : "+d"(c0), "+d"(c1)
+                 : "d"(a), "d"(b));
+}
+
+// ------------------------------------------------------------------------------ load / store
+// A tile (i, j), i >= j: A[r][c] = H[d-1-(64i+r)][d-1-(64j+c)]. One CTA per tile.
+__global__ void __launch_bounds__(256) fac_load(const float* __restrict__ H, int d, int nt, double* __restrict__ A) {
     const int b = blockIdx.y;
-    const size_t dd = (size_t)d * d;
-    for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < dd; idx += (size_t)gridDim.x * blockDim.x) {
-        size_t i = idx / d, j = idx % d;
-        A[b * dd + idx] = (double)H[b * dd + (size_t)(d - 1 - i) * d + (d - 1 - j)];
-    }
-}
-
-// All kernels below run 256 threads; a 64x64 tile is 16 elements per thread. The loads of a tile
-// are issued together (unrolled) so their latencies overlap.
-constexpr int PER_THREAD = NB * NB / 256;
-
-// dst[r][c] = src[r * ld + c]      (64x64 tile, rows already indexed by k)
-__device__ __forceinline__ void load_tile(Tile* dst, const double* __restrict__ src, size_t ld) {
-    double v[PER_THREAD];
-#pragma unroll
-    for (int it = 0; it < PER_THREAD; ++it) {
-        const int i = it * 256 + threadIdx.x;
-        v[it] = src[(size_t)(i >> 6) * ld + (i & 63)];
-    }
-#pragma unroll
-    for (int it = 0; it < PER_THREAD; ++it) {
-        const int i = it * 256 + threadIdx.x;
-        dst[i >> 6][i & 63] = v[it];
-    }
-}
-// dst[c][r] = src[r * ld + c]      (transpose: the tile's columns become the k index)
-__device__ __forceinline__ void load_tile_t(Tile* dst, const double* __restrict__ src, size_t ld) {
-    double v[PER_THREAD];
-#pragma unroll
-    for (int it = 0; it < PER_THREAD; ++it) {
-        const int i = it * 256 + threadIdx.x;
-        v[it] = src[(size_t)(i >> 6) * ld + (i & 63)];
-    }
-#pragma unroll
-    for (int it = 0; it < PER_THREAD; ++it) {
-        const int i = it * 256 + threadIdx.x;
-        dst[i & 63][i >> 6] = v[it];
-    }
-}
-// acc[i][j] += sum_k As[k][4ty+i] * Bs[k][4tx+j]  (k-major operands; 16-byte shared loads)
-__device__ __forceinline__ void mma_tile(const Tile* As, const Tile* Bs, double (&acc)[4][4]) {
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    int t = blockIdx.x, i = 0;
+    while (t > i) { t -= i + 1; ++i; }   // lower tiles, row-major: row i holds i + 1 tiles
+    const int j = t;
+    const float* Hb = H + (size_t)b * d * d;
+    double* At = A + (((size_t)b * nt + i) * nt + j) * TILE_ELEMS;
+    const size_t r0 = (size_t)d - 1 - (size_t)NB * i, c0 = (size_t)d - 1 - (size_t)NB * j;
 #pragma unroll 4
-    for (int k = 0; k < NB; ++k) {
-        const double2 a0 = *reinterpret_cast<const double2*>(&As[k][4 * ty]);
-        const double2 a1 = *reinterpret_cast<const double2*>(&As[k][4 * ty + 2]);
-        const double2 b0 = *reinterpret_cast<const double2*>(&Bs[k][4 * tx]);
-        const double2 b1 = *reinterpret_cast<const double2*>(&Bs[k][4 * tx + 2]);
-        const double a[4] = {a0.x, a0.y, a1.x, a1.y};
-        const double bb[4] = {b0.x, b0.y, b1.x, b1.y};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], bb[j], acc[i][j]);
+    for (int e = threadIdx.x; e < TILE_ELEMS; e += 256) {
+        const int r = e >> 6, c = e & 63;
+        At[e] = (double)Hb[(r0 - r) * d + (c0 - c)];
     }
 }
 
-// Cholesky of the 64x64 diagonal tile of panel k (lower), and its inverse into Dall[b][k].
-// Column loop with one barrier per column: column c of L goes to a separate tile (Lt) while the
-// trailing update reads the unscaled column from T, so no thread writes what another reads in the
-// same step. The inverse is built from 16x16 blocks: four warps invert the diagonal blocks by forward
-// substitution in registers, then three bands X[i][j] = -X[i][i] (sum_m L[i][m] X[m][j]).
-constexpr int SMEM3 = 3 * TILE_DOUBLES * sizeof(double) + NB * sizeof(double);
-
-__global__ void __launch_bounds__(256) fac_potrf(double* __restrict__ A, int d, int k, double* __restrict__ Dall,
-                                                 int* err) {
-    const int b = blockIdx.x;
-    double* Ab = A + (size_t)b * d * d;
-    extern __shared__ double dsm[];
-    Tile* T = reinterpret_cast<Tile*>(dsm);
-    Tile* Lt = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
-    Tile* X = reinterpret_cast<Tile*>(dsm + 2 * TILE_DOUBLES);
-    double* dinv = dsm + 3 * TILE_DOUBLES;           // 1 / L[c][c]
-    const int tid = threadIdx.x;
-    const int k0 = k * NB;
-    load_tile(T, Ab + (size_t)k0 * d + k0, d);
+// U tile (ta, tc): zero below the diagonal, else U[ra][rc] = Y_{jt,it}[63-rc][63-ra] with
+// jt = nt-1-tc, it = nt-1-ta (Y upper, so jt <= it). Transposed through shared memory.
+__global__ void __launch_bounds__(256) fac_store(const double* __restrict__ Y, int d, int nt, float* __restrict__ U) {
+    __shared__ double s[NB][NB + 1];
+    const int b = blockIdx.y;
+    const int ta = blockIdx.x / nt, tc = blockIdx.x % nt;
+    float* Ub = U + (size_t)b * d * d;
+    if (ta > tc) {
+        for (int e = threadIdx.x; e < TILE_ELEMS; e += 256)
+            Ub[(size_t)(NB * ta + (e >> 6)) * d + NB * tc + (e & 63)] = 0.f;
+        return;
+    }
+    const int jt = nt - 1 - tc, it = nt - 1 - ta;
+    const double* Yt = Y + (((size_t)b * nt + jt) * nt + it) * TILE_ELEMS;
+    for (int e = threadIdx.x; e < TILE_ELEMS; e += 256) s[e >> 6][e & 63] = __ldcg(Yt + e);
     __syncthreads();
-    int bad = -1;
-    for (int c = 0; c < NB; ++c) {
-        const double p = T[c][c];
-        const bool ok = (p > 0.0) && isfinite(p);
-        const double inv = ok ? rsqrt(p) : __longlong_as_double(0x7ff8000000000000ll);
-        if (!ok && bad < 0) bad = c;
-        if (tid > c && tid < NB) Lt[tid][c] = T[tid][c] * inv;
-        if (tid == 0) { Lt[c][c] = p * inv; dinv[c] = inv; }
-        const int cc = tid & 63;
-        if (cc > c) {
-            const double lcc = T[cc][c] * inv;
-            for (int r = c + 1 + (tid >> 6); r < NB; r += 4)
-                if (r >= cc) T[r][cc] -= (T[r][c] * inv) * lcc;
+    for (int e = threadIdx.x; e < TILE_ELEMS; e += 256) {
+        const int ra = e >> 6, rc = e & 63;
+        const float v = (ta == tc && ra > rc) ? 0.f : (float)s[63 - rc][63 - ra];
+        Ub[(size_t)(NB * ta + ra) * d + NB * tc + rc] = v;
+    }
+}
+
+// ------------------------------------------------------------------------------ tile primitives
+// Contiguous 64x64 global tile -> padded shared tile (cp.async through L2).
+__device__ __forceinline__ void tile_to_smem(Tile* dst, const double* __restrict__ src) {
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+        const int q = it * 256 + threadIdx.x;   // 16-byte chunk: row q / 32, doubles 2 (q % 32) ..
+        cp_async16(&dst[q >> 5][2 * (q & 31)], src + 2 * q);
+    }
+}
+
+// C (global tile, row-major 64x64) <- (load_c ? C : 0) + sign * P Q^T; P, Q already in shared memory.
+__device__ __forceinline__ void tile_gemm_nt(const Tile* Ps, const Tile* Qs, double* C, bool load_c, bool negate) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, tq = lane & 3;
+    const int wm = warp >> 2, wn = warp & 3;   // warp block: rows 32 wm .., cols 16 wn ..
+    double c[4][2][2];
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 2; ++ni) {
+            if (load_c) {
+                const double2 v = __ldcg(reinterpret_cast<const double2*>(
+                    C + (32 * wm + 8 * mi + g) * NB + 16 * wn + 8 * ni + 2 * tq));
+                c[mi][ni][0] = v.x;
+                c[mi][ni][1] = v.y;
+            } else {
+                c[mi][ni][0] = c[mi][ni][1] = 0.0;
+            }
+        }
+#pragma unroll 4
+    for (int k0 = 0; k0 < NB; k0 += 4) {
+        double a[4], bq[2];
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi) {
+            a[mi] = Ps[32 * wm + 8 * mi + g][k0 + tq];
+            if (negate) a[mi] = -a[mi];
+        }
+#pragma unroll
+        for (int ni = 0; ni < 2; ++ni) bq[ni] = Qs[16 * wn + 8 * ni + g][k0 + tq];
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+            for (int ni = 0; ni < 2; ++ni) dmma(c[mi][ni][0], c[mi][ni][1], a[mi], bq[ni]);
+    }
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 2; ++ni)
+            *reinterpret_cast<double2*>(C + (32 * wm + 8 * mi + g) * NB + 16 * wn + 8 * ni + 2 * tq) =
+                make_double2(c[mi][ni][0], c[mi][ni][1]);
+}
+
+// Cholesky of the 64x64 tile in T (lower, in place), its inverse X = L^-1; writes L to Lg, X to Dg,
+// X^T to Yg; W is scratch. Blocked by 16 columns: for each diagonal block, warp 0 factors it in
+// registers (lane r holds row r; the pivot and the scaled column are broadcast by shuffles) and
+// inverts it by forward substitution (lane j solves column j); the CTA then forms the panel below
+// it, L_ib = A_ib L_bb^-T, and applies the rank-16 update to the trailing lower triangle. The full
+// inverse is assembled from the diagonal-block inverses by three bands
+// X[i][j] = -X[i][i] (sum_m L[i][m] X[m][j]).
+__device__ void tile_potrf_inv(Tile* T, Tile* W, Tile* X, double* dinv, double* Lg, double* Dg, double* Yg,
+                               int* err, int b, int col_base, int d) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const double qnan = __longlong_as_double(0x7ff8000000000000ll);
+    int bad = -1;   // first non-positive pivot (warp 0)
+    for (int kb = 0; kb < 4; ++kb) {
+        const int o = 16 * kb;
+        if (warp == 0) {
+            const int rr = lane & 15;   // lanes 16..31 shadow lanes 0..15 and write nothing
+            double a[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) a[c] = T[o + rr][o + c];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const double p = __shfl_sync(0xffffffffu, a[c], c);
+                const bool ok = (p > 0.0) && isfinite(p);
+                if (!ok && bad < 0) bad = o + c;
+                const double inv = ok ? rsqrt(p) : qnan;
+                const double l = (rr == c) ? p * inv : a[c] * inv;
+                a[c] = l;
+#pragma unroll
+                for (int cc = 1; cc < 16; ++cc) {   // constant trip count keeps a[] in registers
+                    if (cc > c) {
+                        const double lcc = __shfl_sync(0xffffffffu, l, cc);
+                        if (rr >= cc) a[cc] = fma(-l, lcc, a[cc]);
+                    }
+                }
+                if (lane == c) dinv[o + c] = inv;
+            }
+            if (lane < 16) {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) T[o + rr][o + c] = (c <= rr) ? a[c] : 0.0;
+            }
+            __syncwarp();
+            if (lane < 16) {   // column j = lane of the diagonal block's inverse
+                const int j = lane;
+                double x[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    double s = (r == j) ? 1.0 : 0.0;
+#pragma unroll
+                    for (int m = 0; m < r; ++m) s -= (m >= j) ? T[o + r][o + m] * x[m] : 0.0;
+                    x[r] = (r >= j) ? s * dinv[o + r] : 0.0;
+                }
+#pragma unroll
+                for (int r = 0; r < 16; ++r) X[o + r][o + j] = x[r];
+            }
         }
         __syncthreads();
-    }
-    if (tid == 0 && bad >= 0) clha_record_error(err, CLHA_ERR_NOT_PD, b, d - 1 - (k0 + bad), KID_FACTOR);
-    // (1) diagonal 16x16 blocks: warp i, lane j < 16 solves column j of block i
-    const int warp = tid >> 5, lane = tid & 31;
-    if (warp < 4 && lane < 16) {
-        const int o = 16 * warp, j = lane;
-        double x[16];
+        const int rows = 48 - o;   // rows below the diagonal block
+        if (rows > 0) {
+            double v[3];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            double s = (r == j) ? 1.0 : 0.0;
+            for (int it = 0; it < 3; ++it) {   // L[i][o+c] = sum_{k<=c} A[i][o+k] Xbb[c][k]
+                const int e = it * 256 + tid;
+                double acc = 0.0;
+                if (e < rows * 16) {
+                    const int i = o + 16 + (e >> 4), c = e & 15;
 #pragma unroll
-            for (int m = 0; m < r; ++m) s -= (m >= j) ? Lt[o + r][o + m] * x[m] : 0.0;
-            x[r] = (r >= j) ? s * dinv[o + r] : 0.0;
+                    for (int k = 0; k < 16; ++k) acc = (k <= c) ? fma(T[i][o + k], X[o + c][o + k], acc) : acc;
+                }
+                v[it] = acc;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int it = 0; it < 3; ++it) {
+                const int e = it * 256 + tid;
+                if (e < rows * 16) T[o + 16 + (e >> 4)][o + (e & 15)] = v[it];
+            }
+            __syncthreads();
+            for (int e = tid; e < rows * rows; e += 256) {   // trailing lower triangle, rank 16
+                const int i = o + 16 + e / rows, j = o + 16 + e % rows;
+                if (j <= i) {
+                    double acc = T[i][j];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) acc = fma(-T[i][o + k], T[j][o + k], acc);
+                    T[i][j] = acc;
+                }
+            }
+            __syncthreads();
         }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) X[o + r][o + j] = x[r];
     }
-    // zero the strict upper blocks of X
-    for (int i = tid; i < NB * NB; i += 256) {
+    if (tid == 0 && bad >= 0) clha_record_error(err, CLHA_ERR_NOT_PD, b, d - 1 - (col_base + bad), KID_FACTOR);
+    for (int i = tid; i < TILE_ELEMS; i += 256) {   // strict upper blocks of X are zero
         const int r = i >> 6, c = i & 63;
         if ((c >> 4) > (r >> 4)) X[r][c] = 0.0;
     }
     __syncthreads();
-    // (2) bands: T holds the partial products (T is free now)
-    for (int delta = 1; delta < 4; ++delta) {
+    for (int delta = 1; delta < 4; ++delta) {       // bands; W holds the partial products
         const int nblk = 4 - delta;
-        for (int e = tid; e < nblk * 256; e += 256) {       // Tp = sum_{m in blocks j..i-1} L[i][m] X[m][j]
+        for (int e = tid; e < nblk * 256; e += 256) {
             const int j = e >> 8, i = j + delta, r = (e >> 4) & 15, s = e & 15;
             double acc = 0.0;
-            for (int m = 16 * j; m < 16 * i; ++m) acc = fma(Lt[16 * i + r][m], X[m][16 * j + s], acc);
-            T[16 * i + r][16 * j + s] = acc;
+            for (int m = 16 * j; m < 16 * i; ++m) acc = fma(T[16 * i + r][m], X[m][16 * j + s], acc);
+            W[16 * i + r][16 * j + s] = acc;
         }
         __syncthreads();
-        for (int e = tid; e < nblk * 256; e += 256) {       // X[i][j] = -X[i][i] Tp
+        for (int e = tid; e < nblk * 256; e += 256) {
             const int j = e >> 8, i = j + delta, r = (e >> 4) & 15, s = e & 15;
             double acc = 0.0;
 #pragma unroll
-            for (int q = 0; q < 16; ++q) acc = fma(X[16 * i + r][16 * i + q], T[16 * i + q][16 * j + s], acc);
+            for (int q = 0; q < 16; ++q) acc = fma(X[16 * i + r][16 * i + q], W[16 * i + q][16 * j + s], acc);
             X[16 * i + r][16 * j + s] = -acc;
         }
         __syncthreads();
     }
-    double* Db = Dall + ((size_t)b * (d / NB) + k) * NB * NB;
-#pragma unroll
-    for (int it = 0; it < PER_THREAD; ++it) {
-        const int i = it * 256 + tid;
-        const int r = i >> 6, c = i & 63;
-        Ab[(size_t)(k0 + r) * d + k0 + c] = (c <= r) ? Lt[r][c] : 0.0;
-        Db[i] = X[r][c];
+#pragma unroll 4
+    for (int e = tid; e < TILE_ELEMS; e += 256) {
+        const int r = e >> 6, c = e & 63;
+        Lg[e] = (c <= r) ? T[r][c] : 0.0;
+        Dg[e] = X[r][c];
+        Yg[e] = X[c][r];
     }
 }
 
-// Panel tiles below the diagonal: A[i][k] <- A[i][k] L_kk^-T, i.e. out[r][c] = sum_m B[r][m] Linv[c][m].
-__global__ void __launch_bounds__(256) fac_trsm(double* __restrict__ A, int d, int k, const double* __restrict__ Dall) {
-    const int b = blockIdx.y;
-    const int ib = k + 1 + blockIdx.x;
-    double* Ab = A + (size_t)b * d * d;
-    const double* Db = Dall + ((size_t)b * (d / NB) + k) * NB * NB;
-    extern __shared__ double dsm[];
-    Tile* As = reinterpret_cast<Tile*>(dsm);
-    Tile* Bs = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
-    double* blk = Ab + (size_t)(ib * NB) * d + k * NB;
-    load_tile_t(As, blk, d);          // As[m][r] = B[r][m]
-    load_tile_t(Bs, Db, NB);          // Bs[m][c] = Linv[c][m]
-    __syncthreads();
-    double acc[4][4] = {};
-    mma_tile(As, Bs, acc);
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) blk[(size_t)(ty * 4 + i) * d + tx * 4 + j] = acc[i][j];
+// ------------------------------------------------------------------------------ the task graph
+struct Dag {
+    double* A;   // [batch][nt][nt] tiles, lower used: A, then L in place
+    double* Y;   // [batch][nt][nt] tiles, upper used: R accumulators, then Y = L^-T
+    double* D;   // [batch][nt] tiles: D_m = L_mm^-1
+    int* stA;    // [batch][nt][nt]
+    int* stY;    // [batch][nt][nt]
+    unsigned long long* ticket;
+    int* abort_flag;
+    int* err;
+    int nt, batch, d;
+    unsigned long long total;
+};
+
+__device__ __forceinline__ double* tile(double* base, const Dag& g, int b, int i, int j) {
+    return base + (((size_t)b * g.nt + i) * g.nt + j) * TILE_ELEMS;
+}
+__device__ __forceinline__ int* st(int* base, const Dag& g, int b, int i, int j) {
+    return base + ((size_t)b * g.nt + i) * g.nt + j;
 }
 
-// Trailing update of the lower tiles (i >= j > k): A[i][j] -= A[i][k] A[j][k]^T.
-__global__ void __launch_bounds__(256) fac_update(double* __restrict__ A, int d, int k) {
-    const int b = blockIdx.y;
-    int t = blockIdx.x, jj = 0;
-    const int m = d / NB - k - 1;  // trailing tiles per side
-    while (t >= m - jj) { t -= m - jj; ++jj; }   // column jj holds m - jj tiles (rows jj..m-1)
-    const int ib = k + 1 + jj + t, jb = k + 1 + jj;
-    double* Ab = A + (size_t)b * d * d;
-    extern __shared__ double dsm[];
-    Tile* As = reinterpret_cast<Tile*>(dsm);
-    Tile* Bs = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
-    load_tile_t(As, Ab + (size_t)(ib * NB) * d + k * NB, d);   // As[q][r] = A[ib][k][r][q]
-    load_tile_t(Bs, Ab + (size_t)(jb * NB) * d + k * NB, d);   // Bs[q][s] = A[jb][k][s][q]
-    __syncthreads();
-    double acc[4][4] = {};
-    mma_tile(As, Bs, acc);
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    double* out = Ab + (size_t)(ib * NB) * d + jb * NB;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) out[(size_t)(ty * 4 + i) * d + tx * 4 + j] -= acc[i][j];
-}
-
-// Copy the diagonal-tile inverses of all panels into X (they were produced panel by panel).
-__global__ void fac_inv_diag(const double* __restrict__ Dall, int d, double* __restrict__ X) {
-    const int b = blockIdx.y, kb = blockIdx.x;
-    const double* Db = Dall + ((size_t)b * (d / NB) + kb) * NB * NB;
-    double* Xb = X + (size_t)b * d * d;
-    for (int i = threadIdx.x; i < NB * NB; i += blockDim.x) {
-        const int r = i >> 6, c = i & 63;
-        Xb[(size_t)(kb * NB + r) * d + kb * NB + c] = Db[i];
+// Thread 0: wait until *p >= target. False when the graph was aborted or the wait ran out of time.
+__device__ bool wait_ge(const int* p, int target, const Dag& g, int b) {
+    if (ld_acquire(p) >= target) { __threadfence(); return true; }
+    const uint64_t t0 = gtimer();
+    unsigned ns = 32;
+    for (;;) {
+        __nanosleep(ns);
+        if (ns < 512) ns <<= 1;
+        if (ld_acquire(p) >= target) { __threadfence(); return true; }
+        if (*reinterpret_cast<volatile int*>(g.abort_flag)) return false;
+        if (gtimer() - t0 > WAIT_LIMIT_NS) {
+            atomicExch(g.abort_flag, 1);
+            clha_record_error(g.err, CLHA_ERR_TIMEOUT, b, 0, KID_FACTOR);
+            return false;
+        }
     }
 }
 
-// X[i][j] <- Linv_ii X[i][j] for the j < i tiles of block row i (in place).
-__global__ void __launch_bounds__(256) fac_inv_row(const double* __restrict__ Dall, int d, int i,
-                                                   double* __restrict__ X) {
-    const int b = blockIdx.y, jb = blockIdx.x;
-    double* Xt = X + (size_t)b * d * d + (size_t)(i * NB) * d + jb * NB;
-    extern __shared__ double dsm[];
-    Tile* As = reinterpret_cast<Tile*>(dsm);
-    Tile* Bs = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
-    load_tile_t(As, Dall + ((size_t)b * (d / NB) + i) * NB * NB, NB);   // As[q][r] = Linv_ii[r][q]
-    load_tile(Bs, Xt, d);                                              // Bs[q][s] = X[i][jb][q][s]
-    __syncthreads();
-    double acc[4][4] = {};
-    mma_tile(As, Bs, acc);
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) Xt[(size_t)(ty * 4 + a) * d + tx * 4 + c] = acc[a][c];
-}
-
-// X[r][j] -= L[r][i] X[i][j] for r > i, j <= i.
-__global__ void __launch_bounds__(256) fac_inv_upd(const double* __restrict__ L, int d, int i,
-                                                   double* __restrict__ X) {
-    const int b = blockIdx.y;
-    const int rb = i + 1 + blockIdx.x / (i + 1), jb = blockIdx.x % (i + 1);
-    const double* Lb = L + (size_t)b * d * d;
-    double* Xb = X + (size_t)b * d * d;
-    extern __shared__ double dsm[];
-    Tile* As = reinterpret_cast<Tile*>(dsm);
-    Tile* Bs = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
-    load_tile_t(As, Lb + (size_t)(rb * NB) * d + i * NB, d);     // As[q][r] = L[rb][i][r][q]
-    load_tile(Bs, Xb + (size_t)(i * NB) * d + jb * NB, d);       // Bs[q][s] = X[i][jb][q][s]
-    __syncthreads();
-    double acc[4][4] = {};
-    mma_tile(As, Bs, acc);
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    double* out = Xb + (size_t)(rb * NB) * d + jb * NB;
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) out[(size_t)(ty * 4 + a) * d + tx * 4 + c] -= acc[a][c];
-}
-
-__global__ void fac_store(const double* __restrict__ X, int d, float* __restrict__ U) {
-    const int b = blockIdx.y;
-    const size_t dd = (size_t)d * d;
-    for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < dd; idx += (size_t)gridDim.x * blockDim.x) {
-        size_t i = idx / d, j = idx % d;
-        U[b * dd + idx] = (j >= i) ? (float)X[b * dd + (size_t)(d - 1 - i) * d + (d - 1 - j)] : 0.f;
+// Tasks per problem in stage s, by class. Stage 0 holds P(0) and S(i,0); stage s >= 1 (m = s - 1)
+// holds the next panel's updates G(i,m+1,m), then P(m+1), the bulk of level m (F(j,m), Q(j,i,m),
+// the remaining G(i,j,m)) and last S(i,m+1): the Cholesky of panel m+1 overlaps level m's bulk
+// (lookahead of one panel) and the S tasks, which wait for it, come after that bulk.
+__device__ __forceinline__ void stage_counts(int nt, int s, long long (&n)[6]) {
+    if (s == 0) {
+        n[0] = 0; n[1] = 1; n[2] = 0; n[3] = 0; n[4] = 0; n[5] = nt - 1;
+        return;
     }
+    const int m = s - 1;
+    const long long R = nt - 1 - m;
+    n[0] = R;
+    n[1] = R >= 1 ? 1 : 0;
+    n[2] = m;
+    n[3] = (long long)(m + 1) * R;
+    n[4] = R >= 1 ? (R - 1) * R / 2 : 0;
+    n[5] = R >= 1 ? R - 1 : 0;
+}
+
+__global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
+    extern __shared__ double dsm[];
+    Tile* T0 = reinterpret_cast<Tile*>(dsm);
+    Tile* T1 = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
+    Tile* T2 = reinterpret_cast<Tile*>(dsm + 2 * TILE_DOUBLES);
+    double* dinv = dsm + 3 * TILE_DOUBLES;
+    unsigned long long* lvl = reinterpret_cast<unsigned long long*>(dinv + NB);   // [nt + 2] stage starts
+    __shared__ unsigned long long s_ticket;
+    __shared__ int s_ok;
+    const int nt = g.nt, batch = g.batch, tid = threadIdx.x;
+    if (tid == 0) {
+        unsigned long long acc = 0;
+        for (int s = 0; s <= nt; ++s) {
+            lvl[s] = acc;
+            long long n[6];
+            stage_counts(nt, s, n);
+            acc += (unsigned long long)(n[0] + n[1] + n[2] + n[3] + n[4] + n[5]) * batch;
+        }
+        lvl[nt + 1] = acc;
+    }
+    __syncthreads();
+
+    for (;;) {
+        if (tid == 0) s_ticket = *reinterpret_cast<volatile int*>(g.abort_flag) ? g.total : atomicAdd(g.ticket, 1ull);
+        __syncthreads();
+        const unsigned long long t = s_ticket;
+        if (t >= g.total) break;
+        // decode: stage, class, problem, task (q: 0 P, 1 S, 2/5 G, 3 F, 4 Q), level m, tiles i, j
+        int lo = 0, hi = nt;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (lvl[mid] <= t) lo = mid; else hi = mid - 1;
+        }
+        const int sg = lo;
+        unsigned long long r = t - lvl[sg];
+        long long n[6];
+        stage_counts(nt, sg, n);
+        int c = 0;
+#pragma unroll
+        for (int cq = 0; cq < 6; ++cq)   // (unrolled: n[] stays in registers)
+            if (c == cq && r >= (unsigned long long)n[cq] * batch) { r -= (unsigned long long)n[cq] * batch; ++c; }
+        const long long local = (long long)(r / batch);
+        const int b = (int)(r % batch);
+        int q, m = sg - 1, i = 0, j = 0;
+        if (c == 0) { q = 2; i = m + 1 + (int)local; j = m + 1; }
+        else if (c == 1) { q = 0; m = sg; }
+        else if (c == 2) { q = 3; j = (int)local; }
+        else if (c == 3) { q = 4; i = m + 1 + (int)(local / (m + 1)); j = (int)(local % (m + 1)); }
+        else if (c == 4) {
+            q = 5;
+            long long rem = local;
+            j = m + 2;
+            while (rem >= nt - j) { rem -= nt - j; ++j; }
+            i = j + (int)rem;
+        } else { q = 1; m = sg; i = m + 1 + (int)local; j = m; }
+
+        // wait for the inputs
+        if (tid == 0) {
+            bool ok = true;
+            switch (q) {
+                case 0: ok = wait_ge(st(g.stA, g, b, m, m), m, g, b); break;
+                case 1: ok = wait_ge(st(g.stA, g, b, i, m), m, g, b) && wait_ge(st(g.stA, g, b, m, m), m + 1, g, b); break;
+                case 2:
+                case 5:
+                    ok = wait_ge(st(g.stA, g, b, i, m), m + 1, g, b) && wait_ge(st(g.stA, g, b, j, m), m + 1, g, b) &&
+                         wait_ge(st(g.stA, g, b, i, j), m, g, b);
+                    break;
+                case 3: ok = wait_ge(st(g.stY, g, b, j, m), m - j, g, b) && wait_ge(st(g.stA, g, b, m, m), m + 1, g, b); break;
+                default:   // 4: R_ji += Y_jm L_im^T
+                    ok = wait_ge(st(g.stY, g, b, j, m), m - j + 1, g, b) && wait_ge(st(g.stA, g, b, i, m), m + 1, g, b) &&
+                         wait_ge(st(g.stY, g, b, j, i), m - j, g, b);
+                    break;
+            }
+            s_ok = ok;
+        }
+        __syncthreads();
+        if (!s_ok) break;
+
+        // run
+        int* out_state;
+        int out_value;
+        if (q == 0) {
+            tile_to_smem(T0, tile(g.A, g, b, m, m));
+            cp_async_wait_all();
+            __syncthreads();
+            tile_potrf_inv(T0, T1, T2, dinv, tile(g.A, g, b, m, m), g.D + ((size_t)b * nt + m) * TILE_ELEMS,
+                           tile(g.Y, g, b, m, m), g.err, b, NB * m, g.d);
+            __syncthreads();
+            if (tid == 0) {
+                __threadfence();
+                st_release(st(g.stY, g, b, m, m), 1);
+            }
+            out_state = st(g.stA, g, b, m, m);
+            out_value = m + 1;
+        } else {
+            const double *P, *Qm;
+            double* C;
+            bool load_c, negate;
+            if (q == 1) {            // L_im = A_im D_m^T
+                P = tile(g.A, g, b, i, m); Qm = g.D + ((size_t)b * nt + m) * TILE_ELEMS; C = tile(g.A, g, b, i, m);
+                load_c = false; negate = false;
+                out_state = st(g.stA, g, b, i, m); out_value = m + 1;
+            } else if (q == 2 || q == 5) {   // A_ij -= L_im L_jm^T
+                P = tile(g.A, g, b, i, m); Qm = tile(g.A, g, b, j, m); C = tile(g.A, g, b, i, j);
+                load_c = true; negate = true;
+                out_state = st(g.stA, g, b, i, j); out_value = m + 1;
+            } else if (q == 3) {     // Y_jm = -R_jm D_m^T
+                P = tile(g.Y, g, b, j, m); Qm = g.D + ((size_t)b * nt + m) * TILE_ELEMS; C = tile(g.Y, g, b, j, m);
+                load_c = false; negate = true;
+                out_state = st(g.stY, g, b, j, m); out_value = m - j + 1;
+            } else {                 // R_ji (+)= Y_jm L_im^T
+                P = tile(g.Y, g, b, j, m); Qm = tile(g.A, g, b, i, m); C = tile(g.Y, g, b, j, i);
+                load_c = (m != j); negate = false;
+                out_state = st(g.stY, g, b, j, i); out_value = m - j + 1;
+            }
+            tile_to_smem(T0, P);
+            tile_to_smem(T1, Qm);
+            cp_async_wait_all();
+            __syncthreads();
+            tile_gemm_nt(T0, T1, C, load_c, negate);
+        }
+        __syncthreads();   // every thread's stores issued; shared tiles free for the next task
+        if (tid == 0) {
+            __threadfence();
+            st_release(out_state, out_value);
+        }
+    }
+}
+
+constexpr size_t dag_smem_bytes(int nt) {
+    return (size_t)3 * TILE_DOUBLES * sizeof(double) + NB * sizeof(double) + (size_t)(nt + 2) * sizeof(unsigned long long);
 }
 
 }  // namespace
 
 size_t factor_workspace_bytes(int batch, int d) {
-    size_t dd = (size_t)d * d;
-    return clha_round_up((size_t)batch * dd * sizeof(double)) * 2 +
-           clha_round_up((size_t)batch * (d / NB) * NB * NB * sizeof(double));
+    const size_t nt = (size_t)d / NB;
+    const size_t tiles = (size_t)batch * nt * nt;
+    return 2 * clha_round_up(tiles * TILE_ELEMS * sizeof(double)) +
+           clha_round_up((size_t)batch * nt * TILE_ELEMS * sizeof(double)) +
+           clha_round_up(2 * tiles * sizeof(int) + 2 * sizeof(unsigned long long));
 }
 
-cudaError_t launch_factor(cudaStream_t s, const float* H_d, int batch, int d, float* U, void* ws, int* err) {
-    size_t dd = (size_t)d * d;
+cudaError_t launch_factor(cudaStream_t s, int num_sms, const float* H_d, int batch, int d, float* U, void* ws,
+                          int* err) {
+    const int nt = d / NB;
+    const size_t tiles = (size_t)batch * nt * nt;
     char* cur = (char*)ws;
-    double* A = (double*)clha_carve(cur, (size_t)batch * dd * sizeof(double));
-    double* X = (double*)clha_carve(cur, (size_t)batch * dd * sizeof(double));
-    double* Dall = (double*)clha_carve(cur, (size_t)batch * (d / NB) * NB * NB * sizeof(double));
-    const int nbk = d / NB;
-    const int smem = SMEM2;
-    cudaError_t e;
-    if ((e = cudaFuncSetAttribute(fac_potrf, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM3)) != cudaSuccess)
-        return e;
-    if ((e = cudaFuncSetAttribute(fac_trsm, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(fac_update, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(fac_inv_row, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
-        return e;
-    if ((e = cudaFuncSetAttribute(fac_inv_upd, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
-        return e;
-    unsigned eg = (unsigned)((dd + 255) / 256);
-    if (eg > 148 * 64) eg = 148 * 64;
-    fac_load<<<dim3(eg, batch), 256, 0, s>>>(H_d, d, A);
-    clha_note_launches(1);
-    e = cudaMemsetAsync(X, 0, (size_t)batch * dd * sizeof(double), s);
+    Dag g;
+    g.A = (double*)clha_carve(cur, tiles * TILE_ELEMS * sizeof(double));
+    g.Y = (double*)clha_carve(cur, tiles * TILE_ELEMS * sizeof(double));
+    g.D = (double*)clha_carve(cur, (size_t)batch * nt * TILE_ELEMS * sizeof(double));
+    const size_t state_bytes = 2 * tiles * sizeof(int) + 2 * sizeof(unsigned long long);
+    char* sts = (char*)clha_carve(cur, state_bytes);
+    g.ticket = (unsigned long long*)sts;
+    g.abort_flag = (int*)(sts + sizeof(unsigned long long));
+    g.stA = (int*)(sts + 2 * sizeof(unsigned long long));
+    g.stY = g.stA + tiles;
+    g.err = err;
+    g.nt = nt;
+    g.batch = batch;
+    g.d = d;
+    unsigned long long per = 0;
+    for (int m = 0; m < nt; ++m) {
+        const long long R = nt - 1 - m;
+        per += 1 + 2 * R + m + (m + 1) * R + (R >= 1 ? (R - 1) * R / 2 : 0);
+    }
+    g.total = per * (unsigned long long)batch;
+
+    const size_t smem = dag_smem_bytes(nt);
+    cudaError_t e = cudaFuncSetAttribute(fac_dag, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    for (int k = 0; k < nbk; ++k) {
-        fac_potrf<<<batch, 256, SMEM3, s>>>(A, d, k, Dall, err);
-        clha_note_launches(1);
-        const int rem = nbk - k - 1;
-        if (rem > 0) {
-            fac_trsm<<<dim3(rem, batch), 256, smem, s>>>(A, d, k, Dall);
-            clha_note_launches(1);
-            fac_update<<<dim3(rem * (rem + 1) / 2, batch), 256, smem, s>>>(A, d, k);
-            clha_note_launches(1);
-        }
-    }
-    fac_inv_diag<<<dim3(nbk, batch), 256, 0, s>>>(Dall, d, X);
+    if ((e = cudaMemsetAsync(sts, 0, state_bytes, s)) != cudaSuccess) return e;
+    fac_load<<<dim3((unsigned)(nt * (nt + 1) / 2), batch), 256, 0, s>>>(H_d, d, nt, g.A);
     clha_note_launches(1);
-    for (int i = 0; i < nbk; ++i) {
-        if (i > 0) {
-            fac_inv_row<<<dim3(i, batch), 256, smem, s>>>(Dall, d, i, X);
-            clha_note_launches(1);
-        }
-        if (i + 1 < nbk) {
-            fac_inv_upd<<<dim3((nbk - 1 - i) * (i + 1), batch), 256, smem, s>>>(A, d, i, X);
-            clha_note_launches(1);
-        }
-    }
-    fac_store<<<dim3(eg, batch), 256, 0, s>>>(X, d, U);
+    unsigned long long grid = 2ull * (unsigned long long)num_sms;
+    if (grid > g.total) grid = g.total;
+    fac_dag<<<(unsigned)grid, 256, smem, s>>>(g);
+    clha_note_launches(1);
+    fac_store<<<dim3((unsigned)(nt * nt), batch), 256, 0, s>>>(g.Y, d, nt, U);
     clha_note_launches(1);
     return cudaGetLastError();
 }

@@ -28,7 +28,10 @@
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int KCHUNK_BLOCKS = 64;  // KCHUNK = 4096 tokens per TMEM accumulation
+#ifndef CLHA_SYRK_KCHUNK_BLOCKS
+#define CLHA_SYRK_KCHUNK_BLOCKS 128
+#endif
+constexpr int KCHUNK_BLOCKS = CLHA_SYRK_KCHUNK_BLOCKS;  // 64-token blocks per TMEM accumulation
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
