@@ -120,8 +120,13 @@ __device__ __forceinline__ void tile_to_smem(Tile* dst, const double* __restrict
     }
 }
 
-// C (global tile, row-major 64x64) <- (load_c ? C : 0) + sign * P Q^T; P, Q already in shared memory.
-__device__ __forceinline__ void tile_gemm_nt(const Tile* Ps, const Tile* Qs, double* C, bool load_c, bool negate) {
+// C (global tile, row-major 64x64) <- (load_c ? C : 0) + sign * P Q^T. The operand copies into shared
+// memory and the loads of this thread's C fragments are all in flight together.
+__device__ __forceinline__ void tile_gemm_nt(const double* __restrict__ Pg, const double* __restrict__ Qg, Tile* Ps,
+                                             Tile* Qs, double* C, bool load_c, bool negate) {
+    tile_to_smem(Ps, Pg);
+    tile_to_smem(Qs, Qg);
+    asm volatile("cp.async.commit_group;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, tq = lane & 3;
     const int wm = warp >> 2, wn = warp & 3;   // warp block: rows 32 wm .., cols 16 wn ..
@@ -139,6 +144,8 @@ __device__ __forceinline__ void tile_gemm_nt(const Tile* Ps, const Tile* Qs, dou
                 c[mi][ni][0] = c[mi][ni][1] = 0.0;
             }
         }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
 #pragma unroll 4
     for (int k0 = 0; k0 < NB; k0 += 4) {
         double a[4], bq[2];
@@ -163,14 +170,15 @@ __device__ __forceinline__ void tile_gemm_nt(const Tile* Ps, const Tile* Qs, dou
 }
 
 // Cholesky of the 64x64 tile in T (lower, in place), its inverse X = L^-1; writes L to Lg, X to Dg,
-// X^T to Yg; W is scratch. Blocked by 16 columns: for each diagonal block, warp 0 factors it in
+// X^T to Yg. Blocked by 16 columns: for each diagonal block, warp 0 factors it in
 // registers (lane r holds row r; the pivot and the scaled column are broadcast by shuffles) and
 // inverts it by forward substitution (lane j solves column j); the CTA then forms the panel below
 // it, L_ib = A_ib L_bb^-T, and applies the rank-16 update to the trailing lower triangle. The full
 // inverse is assembled from the diagonal-block inverses by three bands
-// X[i][j] = -X[i][i] (sum_m L[i][m] X[m][j]).
-__device__ void tile_potrf_inv(Tile* T, Tile* W, Tile* X, double* dinv, double* Lg, double* Dg, double* Yg,
-                               int* err, int b, int col_base, int d) {
+// X[i][j] = -X[i][i] (sum_m L[i][m] X[m][j]), the partial sums parked in the unused strict upper
+// triangle of T (block (j, i) holds the sums of block (i, j)).
+__device__ void tile_potrf_inv(Tile* T, Tile* X, double* dinv, double* Lg, double* Dg, double* Yg, int* err, int b,
+                               int col_base, int d) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const double qnan = __longlong_as_double(0x7ff8000000000000ll);
     int bad = -1;   // first non-positive pivot (warp 0)
@@ -203,18 +211,15 @@ __device__ void tile_potrf_inv(Tile* T, Tile* W, Tile* X, double* dinv, double* 
                 for (int c = 0; c < 16; ++c) T[o + rr][o + c] = (c <= rr) ? a[c] : 0.0;
             }
             __syncwarp();
-            if (lane < 16) {   // column j = lane of the diagonal block's inverse
+            if (lane < 16) {   // column j = lane of the diagonal block's inverse (this lane's own X column)
                 const int j = lane;
-                double x[16];
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
                     double s = (r == j) ? 1.0 : 0.0;
 #pragma unroll
-                    for (int m = 0; m < r; ++m) s -= (m >= j) ? T[o + r][o + m] * x[m] : 0.0;
-                    x[r] = (r >= j) ? s * dinv[o + r] : 0.0;
+                    for (int m = 0; m < r; ++m) s -= (m >= j) ? T[o + r][o + m] * X[o + m][o + j] : 0.0;
+                    X[o + r][o + j] = (r >= j) ? s * dinv[o + r] : 0.0;
                 }
-#pragma unroll
-                for (int r = 0; r < 16; ++r) X[o + r][o + j] = x[r];
             }
         }
         __syncthreads();
@@ -257,20 +262,20 @@ __device__ void tile_potrf_inv(Tile* T, Tile* W, Tile* X, double* dinv, double* 
         if ((c >> 4) > (r >> 4)) X[r][c] = 0.0;
     }
     __syncthreads();
-    for (int delta = 1; delta < 4; ++delta) {       // bands; W holds the partial products
+    for (int delta = 1; delta < 4; ++delta) {       // bands; Tp[r][s] of block (i, j) sits at T[16j+r][16i+s]
         const int nblk = 4 - delta;
         for (int e = tid; e < nblk * 256; e += 256) {
             const int j = e >> 8, i = j + delta, r = (e >> 4) & 15, s = e & 15;
             double acc = 0.0;
             for (int m = 16 * j; m < 16 * i; ++m) acc = fma(T[16 * i + r][m], X[m][16 * j + s], acc);
-            W[16 * i + r][16 * j + s] = acc;
+            T[16 * j + r][16 * i + s] = acc;
         }
         __syncthreads();
         for (int e = tid; e < nblk * 256; e += 256) {
             const int j = e >> 8, i = j + delta, r = (e >> 4) & 15, s = e & 15;
             double acc = 0.0;
 #pragma unroll
-            for (int q = 0; q < 16; ++q) acc = fma(X[16 * i + r][16 * i + q], W[16 * i + q][16 * j + s], acc);
+            for (int q = 0; q < 16; ++q) acc = fma(X[16 * i + r][16 * i + q], T[16 * j + q][16 * i + s], acc);
             X[16 * i + r][16 * j + s] = -acc;
         }
         __syncthreads();
@@ -305,15 +310,15 @@ __device__ __forceinline__ int* st(int* base, const Dag& g, int b, int i, int j)
     return base + ((size_t)b * g.nt + i) * g.nt + j;
 }
 
-// Thread 0: wait until *p >= target. False when the graph was aborted or the wait ran out of time.
+// One thread: wait until *p >= target (acquire). False when the graph was aborted or the wait ran out of time.
 __device__ bool wait_ge(const int* p, int target, const Dag& g, int b) {
-    if (ld_acquire(p) >= target) { __threadfence(); return true; }
+    if (ld_acquire(p) >= target) return true;
     const uint64_t t0 = gtimer();
     unsigned ns = 32;
     for (;;) {
         __nanosleep(ns);
         if (ns < 512) ns <<= 1;
-        if (ld_acquire(p) >= target) { __threadfence(); return true; }
+        if (ld_acquire(p) >= target) return true;
         if (*reinterpret_cast<volatile int*>(g.abort_flag)) return false;
         if (gtimer() - t0 > WAIT_LIMIT_NS) {
             atomicExch(g.abort_flag, 1);
@@ -346,12 +351,11 @@ __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
     extern __shared__ double dsm[];
     Tile* T0 = reinterpret_cast<Tile*>(dsm);
     Tile* T1 = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
-    Tile* T2 = reinterpret_cast<Tile*>(dsm + 2 * TILE_DOUBLES);
-    double* dinv = dsm + 3 * TILE_DOUBLES;
+    double* dinv = dsm + 2 * TILE_DOUBLES;
     unsigned long long* lvl = reinterpret_cast<unsigned long long*>(dinv + NB);   // [nt + 2] stage starts
     __shared__ unsigned long long s_ticket;
     __shared__ int s_ok;
-    const int nt = g.nt, batch = g.batch, tid = threadIdx.x;
+    const int nt = g.nt, batch = g.batch, tid = threadIdx.x, lane = tid & 31;
     if (tid == 0) {
         unsigned long long acc = 0;
         for (int s = 0; s <= nt; ++s) {
@@ -362,13 +366,18 @@ __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
         }
         lvl[nt + 1] = acc;
     }
+    // Thread 0 holds the next number while the CTA runs the current task (taking numbers in order
+    // and running them in order keeps the schedule deadlock-free).
+    unsigned long long next = 0;
+    if (tid == 0) next = atomicAdd(g.ticket, 1ull);
     __syncthreads();
 
     for (;;) {
-        if (tid == 0) s_ticket = *reinterpret_cast<volatile int*>(g.abort_flag) ? g.total : atomicAdd(g.ticket, 1ull);
+        if (tid == 0) s_ticket = *reinterpret_cast<volatile int*>(g.abort_flag) ? g.total : next;
         __syncthreads();
         const unsigned long long t = s_ticket;
         if (t >= g.total) break;
+        if (tid == 0) next = atomicAdd(g.ticket, 1ull);
         // decode: stage, class, problem, task (q: 0 P, 1 S, 2/5 G, 3 F, 4 Q), level m, tiles i, j
         int lo = 0, hi = nt;
         while (lo < hi) {
@@ -398,81 +407,72 @@ __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
             i = j + (int)rem;
         } else { q = 1; m = sg; i = m + 1 + (int)local; j = m; }
 
-        // wait for the inputs
-        if (tid == 0) {
+        // operands, output and the states to wait for (lane k of warp 0 polls condition k)
+        const double *P = nullptr, *Qm = nullptr;
+        double* C = nullptr;
+        bool load_c = false, negate = false;
+        int* out_state;
+        int out_value;
+        const int* wp[3] = {nullptr, nullptr, nullptr};
+        int wt[3] = {0, 0, 0};
+        double* Dm = g.D + ((size_t)b * nt + m) * TILE_ELEMS;
+        if (q == 0) {            // P(m)
+            wp[0] = st(g.stA, g, b, m, m); wt[0] = m;
+            out_state = st(g.stA, g, b, m, m); out_value = m + 1;
+        } else if (q == 1) {     // L_im = A_im D_m^T
+            wp[0] = st(g.stA, g, b, i, m); wt[0] = m;
+            wp[1] = st(g.stA, g, b, m, m); wt[1] = m + 1;
+            P = tile(g.A, g, b, i, m); Qm = Dm; C = tile(g.A, g, b, i, m);
+            out_state = st(g.stA, g, b, i, m); out_value = m + 1;
+        } else if (q == 2 || q == 5) {   // A_ij -= L_im L_jm^T
+            wp[0] = st(g.stA, g, b, i, m); wt[0] = m + 1;
+            wp[1] = st(g.stA, g, b, j, m); wt[1] = m + 1;
+            wp[2] = st(g.stA, g, b, i, j); wt[2] = m;
+            P = tile(g.A, g, b, i, m); Qm = tile(g.A, g, b, j, m); C = tile(g.A, g, b, i, j);
+            load_c = true; negate = true;
+            out_state = st(g.stA, g, b, i, j); out_value = m + 1;
+        } else if (q == 3) {     // Y_jm = -R_jm D_m^T
+            wp[0] = st(g.stY, g, b, j, m); wt[0] = m - j;
+            wp[1] = st(g.stA, g, b, m, m); wt[1] = m + 1;
+            P = tile(g.Y, g, b, j, m); Qm = Dm; C = tile(g.Y, g, b, j, m);
+            negate = true;
+            out_state = st(g.stY, g, b, j, m); out_value = m - j + 1;
+        } else {                 // R_ji (+)= Y_jm L_im^T
+            wp[0] = st(g.stY, g, b, j, m); wt[0] = m - j + 1;
+            wp[1] = st(g.stA, g, b, i, m); wt[1] = m + 1;
+            wp[2] = st(g.stY, g, b, j, i); wt[2] = m - j;
+            P = tile(g.Y, g, b, j, m); Qm = tile(g.A, g, b, i, m); C = tile(g.Y, g, b, j, i);
+            load_c = (m != j);
+            out_state = st(g.stY, g, b, j, i); out_value = m - j + 1;
+        }
+        if (tid < 32) {
             bool ok = true;
-            switch (q) {
-                case 0: ok = wait_ge(st(g.stA, g, b, m, m), m, g, b); break;
-                case 1: ok = wait_ge(st(g.stA, g, b, i, m), m, g, b) && wait_ge(st(g.stA, g, b, m, m), m + 1, g, b); break;
-                case 2:
-                case 5:
-                    ok = wait_ge(st(g.stA, g, b, i, m), m + 1, g, b) && wait_ge(st(g.stA, g, b, j, m), m + 1, g, b) &&
-                         wait_ge(st(g.stA, g, b, i, j), m, g, b);
-                    break;
-                case 3: ok = wait_ge(st(g.stY, g, b, j, m), m - j, g, b) && wait_ge(st(g.stA, g, b, m, m), m + 1, g, b); break;
-                default:   // 4: R_ji += Y_jm L_im^T
-                    ok = wait_ge(st(g.stY, g, b, j, m), m - j + 1, g, b) && wait_ge(st(g.stA, g, b, i, m), m + 1, g, b) &&
-                         wait_ge(st(g.stY, g, b, j, i), m - j, g, b);
-                    break;
-            }
-            s_ok = ok;
+#pragma unroll
+            for (int k = 0; k < 3; ++k)
+                if (lane == k && wp[k]) ok = wait_ge(wp[k], wt[k], g, b);
+            ok = __all_sync(0xffffffffu, ok);
+            if (lane == 0) s_ok = ok;
         }
         __syncthreads();
         if (!s_ok) break;
 
-        // run
-        int* out_state;
-        int out_value;
         if (q == 0) {
             tile_to_smem(T0, tile(g.A, g, b, m, m));
             cp_async_wait_all();
             __syncthreads();
-            tile_potrf_inv(T0, T1, T2, dinv, tile(g.A, g, b, m, m), g.D + ((size_t)b * nt + m) * TILE_ELEMS,
-                           tile(g.Y, g, b, m, m), g.err, b, NB * m, g.d);
+            tile_potrf_inv(T0, T1, dinv, tile(g.A, g, b, m, m), Dm, tile(g.Y, g, b, m, m), g.err, b, NB * m, g.d);
             __syncthreads();
-            if (tid == 0) {
-                __threadfence();
-                st_release(st(g.stY, g, b, m, m), 1);
-            }
-            out_state = st(g.stA, g, b, m, m);
-            out_value = m + 1;
+            if (tid == 0) st_release(st(g.stY, g, b, m, m), 1);
         } else {
-            const double *P, *Qm;
-            double* C;
-            bool load_c, negate;
-            if (q == 1) {            // L_im = A_im D_m^T
-                P = tile(g.A, g, b, i, m); Qm = g.D + ((size_t)b * nt + m) * TILE_ELEMS; C = tile(g.A, g, b, i, m);
-                load_c = false; negate = false;
-                out_state = st(g.stA, g, b, i, m); out_value = m + 1;
-            } else if (q == 2 || q == 5) {   // A_ij -= L_im L_jm^T
-                P = tile(g.A, g, b, i, m); Qm = tile(g.A, g, b, j, m); C = tile(g.A, g, b, i, j);
-                load_c = true; negate = true;
-                out_state = st(g.stA, g, b, i, j); out_value = m + 1;
-            } else if (q == 3) {     // Y_jm = -R_jm D_m^T
-                P = tile(g.Y, g, b, j, m); Qm = g.D + ((size_t)b * nt + m) * TILE_ELEMS; C = tile(g.Y, g, b, j, m);
-                load_c = false; negate = true;
-                out_state = st(g.stY, g, b, j, m); out_value = m - j + 1;
-            } else {                 // R_ji (+)= Y_jm L_im^T
-                P = tile(g.Y, g, b, j, m); Qm = tile(g.A, g, b, i, m); C = tile(g.Y, g, b, j, i);
-                load_c = (m != j); negate = false;
-                out_state = st(g.stY, g, b, j, i); out_value = m - j + 1;
-            }
-            tile_to_smem(T0, P);
-            tile_to_smem(T1, Qm);
-            cp_async_wait_all();
-            __syncthreads();
-            tile_gemm_nt(T0, T1, C, load_c, negate);
+            tile_gemm_nt(P, Qm, T0, T1, C, load_c, negate);
         }
         __syncthreads();   // every thread's stores issued; shared tiles free for the next task
-        if (tid == 0) {
-            __threadfence();
-            st_release(out_state, out_value);
-        }
+        if (tid == 0) st_release(out_state, out_value);   // release: cumulative over the CTA's stores
     }
 }
 
 constexpr size_t dag_smem_bytes(int nt) {
-    return (size_t)3 * TILE_DOUBLES * sizeof(double) + NB * sizeof(double) + (size_t)(nt + 2) * sizeof(unsigned long long);
+    return (size_t)2 * TILE_DOUBLES * sizeof(double) + NB * sizeof(double) + (size_t)(nt + 2) * sizeof(unsigned long long);
 }
 
 }  // namespace
@@ -517,7 +517,7 @@ cudaError_t launch_factor(cudaStream_t s, int num_sms, const float* H_d, int bat
     if ((e = cudaMemsetAsync(sts, 0, state_bytes, s)) != cudaSuccess) return e;
     fac_load<<<dim3((unsigned)(nt * (nt + 1) / 2), batch), 256, 0, s>>>(H_d, d, nt, g.A);
     clha_note_launches(1);
-    unsigned long long grid = 2ull * (unsigned long long)num_sms;
+    unsigned long long grid = 2ull * (unsigned long long)num_sms;   // two resident CTAs per SM
     if (grid > g.total) grid = g.total;
     fac_dag<<<(unsigned)grid, 256, smem, s>>>(g);
     clha_note_launches(1);
