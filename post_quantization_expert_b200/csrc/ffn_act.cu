@@ -9,11 +9,16 @@
 // in fp64, which keeps the rounding of h to bf16 at the correctly rounded value far more often than
 // one long fp32 sum would (inputs with outlier channels cancel heavily); the SiLU product is
 // evaluated in fp64 and rounded once to bf16.
+// Data movement: 16-byte cp.async copies of the bf16 tiles into a double-buffered staging area
+// (rows past the segment's end are zero-filled), one conversion pass per 32-wide k-tile into
+// double-buffered fp32 tiles laid out k-major for the inner loop, one barrier per k-tile; the copy
+// of tile t+2 and the conversion of tile t+1 overlap the FMAs of tile t.
 #include "clha_internal.h"
 
 namespace {
 
 constexpr int TM = 64, TN = 64, TK = 32;
+constexpr int FLD = TM + 4;   // fp32 tile row (k-major): 16-byte aligned float4 reads
 
 __device__ __forceinline__ int find_segment(const int64_t* seg, int E, int64_t row) {
     int lo = 0, hi = E - 1;
@@ -24,11 +29,24 @@ __device__ __forceinline__ int find_segment(const int64_t* seg, int E, int64_t r
     return lo;
 }
 
-__global__ void __launch_bounds__(256) expert_act_simt(const __nv_bfloat16* __restrict__ X, int64_t rows, int dm,
-                                                       const int64_t* __restrict__ seg, int E,
-                                                       const __nv_bfloat16* __restrict__ Wg,
-                                                       const __nv_bfloat16* __restrict__ Wu, int dff,
-                                                       __nv_bfloat16* __restrict__ h) {
+__device__ __forceinline__ void cp_async16_zfill(void* smem_dst, const void* gsrc, bool valid) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+    const int n = valid ? 16 : 0;   // 0 source bytes: the 16 destination bytes are zero-filled
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gsrc), "r"(n) : "memory");
+}
+
+struct ActSmem {
+    __nv_bfloat16 stage[2][3][TM][TK];   // bf16 copies: X, Wg, Wu tiles (row-major, 64 B per row)
+    float f[2][3][TK][FLD];              // fp32, k-major
+};
+
+__global__ void __launch_bounds__(256, 2) expert_act_simt(const __nv_bfloat16* __restrict__ X, int64_t rows, int dm,
+                                                          const int64_t* __restrict__ seg, int E,
+                                                          const __nv_bfloat16* __restrict__ Wg,
+                                                          const __nv_bfloat16* __restrict__ Wu, int dff,
+                                                          __nv_bfloat16* __restrict__ h) {
+    extern __shared__ __align__(16) uint8_t act_smem[];
+    ActSmem& sm = *reinterpret_cast<ActSmem*>(act_smem);
     const int64_t m0 = (int64_t)blockIdx.x * TM;
     const int n0 = blockIdx.y * TN;
     int e = 0;
@@ -40,30 +58,58 @@ __global__ void __launch_bounds__(256) expert_act_simt(const __nv_bfloat16* __re
     }
     const __nv_bfloat16* wg = Wg + (size_t)e * dff * dm;
     const __nv_bfloat16* wu = Wu + (size_t)e * dff * dm;
-    __shared__ float As[TK][TM + 4];
-    __shared__ float Gs[TK][TN + 4];
-    __shared__ float Us[TK][TN + 4];
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    double ag[4][4] = {}, au[4][4] = {};
-    for (int k0 = 0; k0 < dm; k0 += TK) {
-        for (int i = threadIdx.x; i < TM * TK; i += 256) {
-            int m = i / TK, kk = i % TK;
-            int64_t row = m0 + m;
-            As[kk][m] = (row < valid_end) ? __bfloat162float(X[row * dm + k0 + kk]) : 0.f;
-            Gs[kk][m] = __bfloat162float(wg[(size_t)(n0 + m) * dm + k0 + kk]);
-            Us[kk][m] = __bfloat162float(wu[(size_t)(n0 + m) * dm + k0 + kk]);
+    const int tid = threadIdx.x;
+    const int lr = tid >> 2, lk = (tid & 3) * 8;   // this thread copies/converts row lr, k lk..lk+7
+    const bool row_ok = m0 + lr < valid_end;
+    const __nv_bfloat16* xsrc = X + (row_ok ? (m0 + lr) * dm : 0) + lk;
+    const __nv_bfloat16* gsrc = wg + (size_t)(n0 + lr) * dm + lk;
+    const __nv_bfloat16* usrc = wu + (size_t)(n0 + lr) * dm + lk;
+    const int nkt = dm / TK;
+
+    auto issue = [&](int kt) {
+        const int st = kt & 1, k0 = kt * TK;
+        cp_async16_zfill(&sm.stage[st][0][lr][lk], xsrc + k0, row_ok);
+        cp_async16_zfill(&sm.stage[st][1][lr][lk], gsrc + k0, true);
+        cp_async16_zfill(&sm.stage[st][2][lr][lk], usrc + k0, true);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    auto convert = [&](int kt) {
+        const int st = kt & 1;
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            const uint4 v = *reinterpret_cast<const uint4*>(&sm.stage[st][a][lr][lk]);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                sm.f[st][a][lk + 2 * q][lr] = __uint_as_float(w[q] << 16);
+                sm.f[st][a][lk + 2 * q + 1][lr] = __uint_as_float(w[q] & 0xffff0000u);
+            }
         }
+    };
+
+    const int tx = tid & 15, ty = tid >> 4;
+    double ag[4][4] = {}, au[4][4] = {};
+    issue(0);
+    if (nkt > 1) issue(1);
+    if (nkt > 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
+    else asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    convert(0);
+    for (int kt = 0; kt < nkt; ++kt) {
+        // tile kt+1 has landed (its copy was issued two steps ago); everyone is done with step kt-1
+        if (kt + 1 < nkt) asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncthreads();
+        if (kt + 1 < nkt) convert(kt + 1);
+        if (kt + 2 < nkt) issue(kt + 2);
+        const int st = kt & 1;
         float pg[4][4] = {}, pu[4][4] = {};
 #pragma unroll 8
         for (int kk = 0; kk < TK; ++kk) {
-            float a[4], g[4], u[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                a[i] = As[kk][ty * 4 + i];
-                g[i] = Gs[kk][tx * 4 + i];
-                u[i] = Us[kk][tx * 4 + i];
-            }
+            const float4 a4 = *reinterpret_cast<const float4*>(&sm.f[st][0][kk][ty * 4]);
+            const float4 g4 = *reinterpret_cast<const float4*>(&sm.f[st][1][kk][tx * 4]);
+            const float4 u4 = *reinterpret_cast<const float4*>(&sm.f[st][2][kk][tx * 4]);
+            const float a[4] = {a4.x, a4.y, a4.z, a4.w}, g[4] = {g4.x, g4.y, g4.z, g4.w},
+                        u[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -79,7 +125,6 @@ __global__ void __launch_bounds__(256) expert_act_simt(const __nv_bfloat16* __re
                 ag[i][j] += (double)pg[i][j];
                 au[i][j] += (double)pu[i][j];
             }
-        __syncthreads();
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -102,8 +147,15 @@ cudaError_t launch_expert_act(cudaStream_t s, int num_sms, const __nv_bfloat16* 
                               __nv_bfloat16* h, int* err) {
     (void)num_sms;
     (void)err;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(expert_act_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)sizeof(ActSmem));
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
     dim3 grid((unsigned)((rows + TM - 1) / TM), d_ff / TN);
-    expert_act_simt<<<grid, 256, 0, s>>>(X, rows, d_model, seg, E, Wg, Wu, d_ff, h);
+    expert_act_simt<<<grid, 256, sizeof(ActSmem), s>>>(X, rows, d_model, seg, E, Wg, Wu, d_ff, h);
     clha_note_launches(1);
     return cudaGetLastError();
 }
