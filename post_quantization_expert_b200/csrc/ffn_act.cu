@@ -12,7 +12,9 @@
 // Data movement: 16-byte cp.async copies of the bf16 tiles into a double-buffered staging area
 // (rows past the segment's end are zero-filled), one conversion pass per 32-wide k-tile into
 // double-buffered fp32 tiles laid out k-major for the inner loop, one barrier per k-tile; the copy
-// of tile t+2 and the conversion of tile t+1 overlap the FMAs of tile t.
+// of tile t+2 and the conversion of tile t+1 overlap the FMAs of tile t. The copy gives each row to
+// four lanes (coalesced); the conversion gives a warp 32 rows, so its transposing stores and its
+// reads of the padded staging rows are free of bank conflicts.
 #include "clha_internal.h"
 
 namespace {
@@ -35,9 +37,10 @@ __device__ __forceinline__ void cp_async16_zfill(void* smem_dst, const void* gsr
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gsrc), "r"(n) : "memory");
 }
 
+constexpr int SLD = TK + 8;   // bf16 staging row: 80 B, so 8 rows' 16-byte chunks hit distinct banks
 struct ActSmem {
-    __nv_bfloat16 stage[2][3][TM][TK];   // bf16 copies: X, Wg, Wu tiles (row-major, 64 B per row)
-    float f[2][3][TK][FLD];              // fp32, k-major
+    __nv_bfloat16 stage[2][3][TM][SLD];   // bf16 copies: X, Wg, Wu tiles (row-major)
+    float f[2][3][TK][FLD];               // fp32, k-major
 };
 
 __global__ void __launch_bounds__(256, 2) expert_act_simt(const __nv_bfloat16* __restrict__ X, int64_t rows, int dm,
@@ -59,7 +62,8 @@ __global__ void __launch_bounds__(256, 2) expert_act_simt(const __nv_bfloat16* _
     const __nv_bfloat16* wg = Wg + (size_t)e * dff * dm;
     const __nv_bfloat16* wu = Wu + (size_t)e * dff * dm;
     const int tid = threadIdx.x;
-    const int lr = tid >> 2, lk = (tid & 3) * 8;   // this thread copies/converts row lr, k lk..lk+7
+    const int lr = tid >> 2, lk = (tid & 3) * 8;       // this thread copies row lr, k lk..lk+7 (coalesced)
+    const int cr = tid & 63, ck = (tid >> 6) * 8;      // and converts row cr, k ck..ck+7 (a warp: 32 rows)
     const bool row_ok = m0 + lr < valid_end;
     const __nv_bfloat16* xsrc = X + (row_ok ? (m0 + lr) * dm : 0) + lk;
     const __nv_bfloat16* gsrc = wg + (size_t)(n0 + lr) * dm + lk;
@@ -77,12 +81,12 @@ __global__ void __launch_bounds__(256, 2) expert_act_simt(const __nv_bfloat16* _
         const int st = kt & 1;
 #pragma unroll
         for (int a = 0; a < 3; ++a) {
-            const uint4 v = *reinterpret_cast<const uint4*>(&sm.stage[st][a][lr][lk]);
+            const uint4 v = *reinterpret_cast<const uint4*>(&sm.stage[st][a][cr][ck]);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                sm.f[st][a][lk + 2 * q][lr] = __uint_as_float(w[q] << 16);
-                sm.f[st][a][lk + 2 * q + 1][lr] = __uint_as_float(w[q] & 0xffff0000u);
+                sm.f[st][a][ck + 2 * q][cr] = __uint_as_float(w[q] << 16);
+                sm.f[st][a][ck + 2 * q + 1][cr] = __uint_as_float(w[q] & 0xffff0000u);
             }
         }
     };
