@@ -9,6 +9,7 @@ Inputs are synthetic (seeded), resident in HBM; L2 is flushed (512 MB write) bef
   python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
 
 Kernel-level workloads (one JSON line per shape; used for the profiles and the roofline tables):
+  python bench.py --workload act --shape 18432x1024x512 ...   expert activation, dense bf16 X [n, d_model]
   python bench.py --workload hessian --shape 65536x4096 ...   Gram accumulation of dense bf16 X [n, d]
   python bench.py --workload gptq --shape 32x512x1024 ...     GPTQ of [batch, d_out, d_in] bf16 weights
   python bench.py --workload factor --shape 32x1024 ...       inverse-Cholesky factor of [batch, d, d]
@@ -143,8 +144,8 @@ def source_hash(phase: str) -> str:
 
 
 def measured_traffic(phase: str, workload: str):
-    """DRAM bytes per launch from profiles/dram_traffic.txt, only while the kernel source is the one
-    the counters were taken on (its hash is recorded beside the figure)."""
+    """DRAM bytes per step of a phase from profiles/dram_traffic.txt, only while the kernel source is
+    the one the counters were taken on (its hash is recorded beside the figure)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -333,19 +334,22 @@ def run_ours(args, world, rank, local):
     sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     kernels = {
         "hessian": ("tensor", hess_flops / 1e12, sustained, "TFLOP/s", "syrk_bf16_tc (tcgen05 kind::f16)"),
-        "gptq": ("alu", gptq_flops / 1e12, alu["fp32_tflops"], "TFLOP/s", "gptq_simt (fp32 FMA)"),
-        "factor": ("alu", factor_flops / 1e12, alu["fp64_tflops"], "TFLOP/s", "fac_* (fp64 FMA)"),
+        "gptq": ("alu", gptq_flops / 1e12, alu["fp32_tflops"], "TFLOP/s",
+                 "gptq_tc (per-column fp32 sweep; lazy updates on tcgen05 kind::tf32, 3xTF32)"),
+        "factor": ("alu", factor_flops / 1e12, alu["fp64_tflops"], "TFLOP/s",
+                   "fac_load + fac_dag + fac_store (fp64 tile-task graph, mma.sync m8n8k4 f64)"),
         "loss": ("alu", loss_flops / 1e12, alu["fp32_tflops"], "TFLOP/s", "loss_simt (fp32 FMA)"),
         "act": ("alu", act_flops / 1e12, alu["fp32_tflops"], "TFLOP/s", "expert_act_simt (fp32 FMA)"),
         "aggregate": ("hbm", agg_bytes / 1e9, peaks["hbm_gbs"], "GB/s", "agg_combine"),
     }
-    # the dominant single kernel: phases that are one kernel family per call (the factor is a chain
-    # of seven kernels per call and is reported in the phase table)
-    single = ("act", "gptq", "hessian", "aggregate")
+    # the dominant kernel: the phase that takes longest per step (each is one kernel per call, the
+    # factor one graph kernel between a load and a store); traffic is DRAM bytes per call
+    single = ("act", "gptq", "hessian", "aggregate", "factor")
     dom = max((k for k in phase_ms if k in single), key=lambda k: phase_ms[k])
     bound, work, peak, unit, kname = kernels[dom]
     achieved = work / (phase_ms[dom] / 1e3)
-    traffic = measured_traffic(dom, "moe-E16")
+    step_bytes = measured_traffic(dom, "moe-E16")   # per step; reported per timed call like `achieved`
+    traffic = step_bytes / phase_calls[dom] if step_bytes is not None and phase_calls.get(dom) else None
     phases = {k: {"ms": round(v, 4)} for k, v in sorted(phase_ms.items(), key=lambda kv: -kv[1])}
     for k, v in phases.items():
         if k in kernels:
@@ -378,7 +382,7 @@ def run_ours(args, world, rank, local):
             "hessian_frac_of_bf16_peak": hess_tflops / sustained,
             "roofline": {"kernel": kname, "phase": dom, "bound": bound, "achieved": achieved, "peak": peak,
                          "unit": unit, "frac": achieved / peak, "traffic": traffic,
-                         "launches_per_step": phase_calls.get(dom),
+                         "calls_per_step": phase_calls.get(dom),
                          "peak_source": src if bound in ("tensor", "hbm") else "derived (SM count x lanes x max clock)"},
             "phases_ms_per_step": phases,
             "e2e": {"value": world * cols_per_step / (e2e_ms / 1e3), "unit": "columns/s",
@@ -401,9 +405,19 @@ def run_kernel(args):
     alu = alu_peaks(peaks)
     g = torch.Generator(device="cuda")
     g.manual_seed(0)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     for shape in args.shape:
         dims = [int(v) for v in shape.split("x")]
-        if args.workload == "hessian":
+        if args.workload == "act":
+            n, dm, dff = dims
+            X = torch.randn((n, dm), device="cuda", generator=g).to(torch.bfloat16)
+            Wg = (0.03 * torch.randn((dff, dm), device="cuda", generator=g)).to(torch.bfloat16)
+            Wu = (0.03 * torch.randn((dff, dm), device="cuda", generator=g)).to(torch.bfloat16)
+            hbuf = torch.empty((n, dff), device="cuda", dtype=torch.bfloat16)
+            fn = lambda: L.clha_expert_act(ctx, X, n, dm, None, 1, Wg, Wu, dff, hbuf)
+            work, unit, bound, peak = 4 * n * dm * dff / 1e12, "TFLOP/s", "alu", alu["fp32_tflops"]
+            kname = "expert_act_simt"
+        elif args.workload == "hessian":
             n, d = dims
             X = torch.randn((n, d), device="cuda", generator=g).to(torch.bfloat16)
             acc = L.Accum(ctx, d, 1, 1)
@@ -422,7 +436,7 @@ def run_kernel(args):
             if args.workload == "factor":
                 fn = lambda: L.clha_factor(ctx, H, B, d, U)
                 work, unit, bound, peak = B * 2 * d ** 3 / 3 / 1e12, "TFLOP/s", "alu", alu["fp64_tflops"]
-                kname = "fac_* (fp64)"
+                kname = "fac_load + fac_dag + fac_store"
             else:
                 L.clha_factor(ctx, H, B, d, U)
                 W = (0.02 * torch.randn((B, d_out, d), device="cuda", generator=g)).to(torch.bfloat16)
@@ -436,18 +450,22 @@ def run_kernel(args):
         for _ in range(args.warmup):
             fn()
         torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(ctx.stream)
-        for _ in range(args.steps):
+        evs = []
+        for _ in range(args.steps):   # L2 flushed before every timed launch, each launch timed alone
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(ctx.stream)
             fn()
-        b.record(ctx.stream)
+            b.record(ctx.stream)
+            evs.append((a, b))
         torch.cuda.synchronize()
         L.clha_check(ctx)
-        ms = a.elapsed_time(b) / args.steps
+        ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
         achieved = work / (ms / 1e3)
         print(json.dumps({"workload": args.workload, "shape": shape, "kernel": kname, "ms": ms, "achieved": achieved,
                           "unit": unit, "bound": bound, "peak": peak, "frac": achieved / peak,
-                          "peak_source": src if bound == "tensor" else "derived (SM count x lanes x max clock)"}))
+                          "peak_source": src if bound == "tensor" else "derived (SM count x lanes x max clock)",
+                          "l2": "flushed (512 MB write) before every timed launch"}))
         torch.cuda.empty_cache()
     ctx.close()
     return 0
@@ -460,7 +478,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
-    ap.add_argument("--workload", choices=("moe", "hessian", "gptq", "factor"), default="moe",
+    ap.add_argument("--workload", choices=("moe", "act", "hessian", "gptq", "factor"), default="moe",
                     help="moe: the end-to-end calibration step (default); others: one kernel family")
     ap.add_argument("--shape", nargs="+", default=[], help="kernel workload shapes, e.g. 65536x4096")
     args = ap.parse_args()
