@@ -103,7 +103,10 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(mhz)}
 
 
-def dist_setup():
+def dist_setup(backend: str | None = None):
+    """One process per GPU under torchrun (RANK / LOCAL_RANK / WORLD_SIZE / MASTER_* from the env).
+    NCCL on GPUs; gloo when asked for (the CPU tests of this multi-rank logic). The process group
+    has a short timeout so ranks that wait for a missing peer end with an error."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -111,8 +114,12 @@ def dist_setup():
         import torch
         import torch.distributed as dist
         from datetime import timedelta
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+        backend = backend or "nccl"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timedelta(seconds=120))
     return world, rank, local
 
 
@@ -123,13 +130,26 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's figure (the job's time is set by it)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(units_per_step_per_rank: float, ms_max: float, world: int) -> float:
+    """Whole-job throughput under weak scaling: every rank processes its own units each step, and
+    the step takes as long as the slowest rank."""
+    return world * units_per_step_per_rank / (ms_max / 1e3)
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank calibrates its own independent layer pair: a distinct, reproducible input seed."""
+    return 1235 + 7919 * rank
 
 
 KERNEL_SOURCES = {"act": "ffn_act.cu", "gptq": "gptq.cu", "hessian": "hessian.cu", "aggregate": "aggregate.cu",
@@ -171,7 +191,7 @@ def blas_threads():
 # ------------------------------------------------------------------------------------------ workload
 def make_inputs(rank: int):
     from synth import workload
-    wl = workload(2, "cpu", seed=1235 + 7919 * rank)
+    wl = workload(2, "cpu", seed=rank_seed(rank))
     s = wl.spec
     X = [wl.x(l) for l in range(2)]
     lg = [wl.logits(l) for l in range(2)]
@@ -274,7 +294,7 @@ def run_ours(args, world, rank, local):
     step_ms = [a.elapsed_time(b) for a, b in ev]
     timer.collect()
     ms = max_over_ranks(statistics.mean(step_ms), world)
-    value = world * cols_per_step / (ms / 1e3)
+    value = job_value(cols_per_step, ms, world)
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
     pin = lambda t: t.pin_memory()
@@ -385,7 +405,7 @@ def run_ours(args, world, rank, local):
                          "calls_per_step": phase_calls.get(dom),
                          "peak_source": src if bound in ("tensor", "hbm") else "derived (SM count x lanes x max clock)"},
             "phases_ms_per_step": phases,
-            "e2e": {"value": world * cols_per_step / (e2e_ms / 1e3), "unit": "columns/s",
+            "e2e": {"value": job_value(cols_per_step, e2e_ms, world), "unit": "columns/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": int(launches),
             "clocks": clk,
