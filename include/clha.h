@@ -181,6 +181,22 @@ CLHA_API clha_status clha_aggregate(clha_ctx* ctx, const clha_accum* acc, int sl
  * CLHA_ERR_NOT_PD with the problem and column. */
 CLHA_API clha_status clha_factor(clha_ctx* ctx, const float* H_damped, int batch, int d, float* U);
 
+/* The same factor for up to CLHA_FACTOR_MAX_GROUPS groups of problems of different sizes in one
+ * launch of the task graph (e.g. the gate/up Hessians [E, d_model, d_model] and the down Hessians
+ * [E, d_ff, d_ff] of a layer group): each group is `batch` problems [batch, d, d] float32 on the
+ * device, H_damped read and U written as in clha_factor. The small groups' short dependency chains
+ * run alongside the large groups' bulk work. `groups` is a host array read during the call (the
+ * caller keeps ownership). Errors as in clha_factor; the problem index of a CLHA_ERR_NOT_PD report
+ * counts across the groups in order. */
+#define CLHA_FACTOR_MAX_GROUPS 4
+typedef struct clha_factor_group {
+    const float* H_damped;   /* device, [batch, d, d] */
+    float* U;                /* device, [batch, d, d] */
+    int batch;
+    int d;                   /* multiple of 128 */
+} clha_factor_group;
+CLHA_API clha_status clha_factor_groups(clha_ctx* ctx, int n_groups, const clha_factor_group* groups);
+
 /* GPTQ (CLHA page §2.2 (3)): column-sequential quantization of `batch` weights W [batch, d_out, d_in]
  * (bf16 or f32) in natural column order, with lazy updates over 128-column blocks. U holds n_u
  * factors [n_u, d_in, d_in] and problem b uses factor b % n_u (1 <= n_u <= batch; with gate and up

@@ -29,8 +29,13 @@ SYMBOLS = [
     "clha_route_topk", "clha_packed_rows", "clha_gather", "clha_gather_noalloc", "clha_expert_act",
     "clha_accum_create", "clha_accum_destroy", "clha_accum_zero", "clha_accum_buffers",
     "clha_accum_export", "clha_accum_import", "clha_collect",
-    "clha_aggregate", "clha_factor", "clha_quantize", "clha_loss",
+    "clha_aggregate", "clha_factor", "clha_factor_groups", "clha_quantize", "clha_loss",
 ]
+FACTOR_MAX_GROUPS = 4
+
+
+class FactorGroup(C.Structure):
+    _fields_ = [("H_damped", C.c_void_p), ("U", C.c_void_p), ("batch", C.c_int), ("d", C.c_int)]
 
 
 class QuantParams(C.Structure):
@@ -78,6 +83,7 @@ def load(path: str = LIB_PATH):
         "clha_collect": (i32, [vp, vp, i32, vp, i32, i64, i32, vp, i32, i32]),
         "clha_aggregate": (i32, [vp, vp, i32, i32, i32, vp, f64, vp, vp, vp, vp, vp]),
         "clha_factor": (i32, [vp, vp, i32, i32, vp]),
+        "clha_factor_groups": (i32, [vp, i32, vp]),
         "clha_quantize": (i32, [vp, vp, i32, vp, i32, i32, i32, i32, C.POINTER(QuantParams), vp, vp, vp, vp, vp,
                                 vp]),
         "clha_loss": (i32, [vp, vp, i32, vp, vp, i32, i32, i32, i32, vp]),
@@ -258,6 +264,12 @@ def clha_aggregate(ctx: Context, acc: Accum, slot0: int, n_slots: int, mode: int
 
 def clha_factor(ctx: Context, H_damped, batch: int, d: int, U):
     ctx._check(load().clha_factor(ctx.handle, _p(H_damped), batch, d, _p(U)))
+
+
+def clha_factor_groups(ctx: Context, groups):
+    """groups: sequence of (H_damped, batch, d, U), at most FACTOR_MAX_GROUPS; one graph launch."""
+    arr = (FactorGroup * len(groups))(*[FactorGroup(_p(H), _p(U), b, d) for H, b, d, U in groups])
+    ctx._check(load().clha_factor_groups(ctx.handle, len(groups), C.cast(arr, C.c_void_p)))
 
 
 def clha_quantize(ctx: Context, U, n_u: int, W, batch: int, d_out: int, d_in: int, bits: int, codes, scales,

@@ -386,18 +386,32 @@ extern "C" clha_status clha_aggregate(clha_ctx* ctx, const clha_accum* acc, int 
 }
 
 // ------------------------------------------------------------------------------ phase 3
-extern "C" clha_status clha_factor(clha_ctx* ctx, const float* H_damped, int batch, int d, float* U) {
+extern "C" clha_status clha_factor_groups(clha_ctx* ctx, int n_groups, const clha_factor_group* groups) {
     CHECK_CTX(ctx);
-    REQUIRE(H_damped && U, CLHA_ERR_INVALID_ARG, "clha_factor: null pointer");
-    REQUIRE(batch >= 1 && d > 0, CLHA_ERR_INVALID_ARG, "clha_factor: bad sizes");
-    REQUIRE(d % 128 == 0, CLHA_ERR_UNSUPPORTED_SHAPE, "clha_factor: d=%d is not a multiple of 128", d);
+    REQUIRE(groups, CLHA_ERR_INVALID_ARG, "clha_factor_groups: null groups");
+    REQUIRE(n_groups >= 1 && n_groups <= CLHA_FACTOR_MAX_GROUPS, CLHA_ERR_INVALID_ARG,
+            "clha_factor_groups: n_groups=%d outside 1..%d", n_groups, CLHA_FACTOR_MAX_GROUPS);
+    FactorGroup fg[CLHA_FACTOR_MAX_GROUPS];
+    for (int k = 0; k < n_groups; ++k) {
+        const clha_factor_group& g = groups[k];
+        REQUIRE(g.H_damped && g.U, CLHA_ERR_INVALID_ARG, "clha_factor: null pointer (group %d)", k);
+        REQUIRE(g.batch >= 1 && g.d > 0, CLHA_ERR_INVALID_ARG, "clha_factor: bad sizes (group %d)", k);
+        REQUIRE(g.d % 128 == 0, CLHA_ERR_UNSUPPORTED_SHAPE, "clha_factor: d=%d is not a multiple of 128 (group %d)",
+                g.d, k);
+        fg[k] = FactorGroup{g.H_damped, g.U, g.batch, g.d};
+    }
     SET_DEVICE(ctx);
     LaunchScope launch_scope(ctx);
     void* ws = nullptr;
-    clha_status st = clha_workspace(ctx, factor_workspace_bytes(batch, d), &ws);
+    clha_status st = clha_workspace(ctx, factor_workspace_bytes(fg, n_groups), &ws);
     if (st) return st;
-    CUDA_TRY(launch_factor(ctx->stream, ctx->num_sms, H_damped, batch, d, U, ws, ctx->d_err), "clha_factor");
+    CUDA_TRY(launch_factor(ctx->stream, ctx->num_sms, fg, n_groups, ws, ctx->d_err), "clha_factor");
     return CLHA_OK;
+}
+
+extern "C" clha_status clha_factor(clha_ctx* ctx, const float* H_damped, int batch, int d, float* U) {
+    clha_factor_group g{H_damped, U, batch, d};
+    return clha_factor_groups(ctx, 1, &g);
 }
 
 extern "C" clha_status clha_quantize(clha_ctx* ctx, const float* U, int n_u, const void* W, clha_dtype dtype,

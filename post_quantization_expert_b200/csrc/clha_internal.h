@@ -95,9 +95,13 @@ cudaError_t launch_aggregate(cudaStream_t s, const float* S, const int64_t* coun
                              int n_layers, int n_slots_total, int slot0, int n_slots,
                              clha_alpha_args a, double damp_frac, float* H_comb, float* H_d,
                              double* d_alpha, double* d_lambda, int* err);
-size_t factor_workspace_bytes(int batch, int d);
-cudaError_t launch_factor(cudaStream_t s, int num_sms, const float* H_d, int batch, int d, float* U, void* ws,
-                          int* err);
+struct FactorGroup {
+    const float* H;
+    float* U;
+    int batch, d;
+};
+size_t factor_workspace_bytes(const FactorGroup* groups, int n);
+cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups, int n, void* ws, int* err);
 size_t quantize_workspace_bytes(int batch, int d_out, int d_in);
 cudaError_t launch_quantize(cudaStream_t s, const float* U, int n_u, const void* W, int w_is_f32,
                             int batch, int d_out, int d_in, int bits, uint8_t* codes, float* scales,

@@ -5,11 +5,13 @@
 // is positive, so it is THE upper Cholesky factor of H_d^-1. This needs one Cholesky and one
 // triangular inverse (no explicit inverse of H_d, no second factorisation).
 //
-// Float64 throughout, on 64 x 64 tiles (nt = d / 64 per side), batched over problems. Three launches:
-//   fac_load    A = J H_d J, lower tiles, tile-major float64 (each tile 32 KB contiguous)
+// Float64 throughout, on 64 x 64 tiles (nt = d / 64 per side), batched over problems, in up to four
+// groups of different d that share one graph launch (the small groups' short critical paths then
+// overlap the large groups' bulk work):
+//   fac_load    A = J H_d J, lower tiles, tile-major float64 (each tile 32 KB contiguous); per group
 //   fac_dag     one persistent kernel that runs the whole blocked Cholesky and the blocked inverse
-//               as a graph of tile tasks (below)
-//   fac_store   U = J Y^T J as float32, strict lower triangle zero
+//               of every problem of every group as a graph of tile tasks (below)
+//   fac_store   U = J Y^T J as float32, strict lower triangle zero; per group
 //
 // Tile tasks. The inverse is kept transposed, Y = L^-T (upper), so that every product has the form
 // C <- alpha C + beta P Q^T with row-major tiles P and Q:
@@ -21,7 +23,8 @@
 // since L X = I with X = L^-1 = Y^T gives X_ij = -D_i sum_{m=j}^{i-1} L_im X_mj for i > j.
 //
 // Scheduling: tasks are numbered in a topological order (stages with a one-panel lookahead, see
-// stage_counts; problems interleaved inside each class) and CTAs take numbers from a global counter. Every tile has a monotone state counter: A_ij counts the
+// stage_counts; within a stage group after group, problems interleaved inside each class) and CTAs
+// take numbers from a global counter. Every tile has a monotone state counter: A_ij counts the
 // updates applied (j + 1 once L_ij is final); Y_ji counts the Q terms applied (i - j + 1 once final).
 // A task waits (thread 0, acquire loads, bounded by a time limit) until its inputs have reached the
 // states it needs, runs, and publishes its output tile's new state with a release store. Any task
@@ -290,28 +293,37 @@ __device__ void tile_potrf_inv(Tile* T, Tile* X, double* dinv, double* Lg, doubl
 }
 
 // ------------------------------------------------------------------------------ the task graph
-struct Dag {
+constexpr int MAX_GROUPS = 4;
+
+// One group: `batch` problems of the same size d (nt = d / 64 tiles per side), its own workspace.
+struct Grp {
     double* A;   // [batch][nt][nt] tiles, lower used: A, then L in place
     double* Y;   // [batch][nt][nt] tiles, upper used: R accumulators, then Y = L^-T
     double* D;   // [batch][nt] tiles: D_m = L_mm^-1
     int* stA;    // [batch][nt][nt]
     int* stY;    // [batch][nt][nt]
+    int nt, batch, d;
+    int pbase;   // index of the group's first problem across all groups (error reports)
+};
+
+struct Dag {
+    Grp grp[MAX_GROUPS];
+    int ng, max_nt;
     unsigned long long* ticket;
     int* abort_flag;
     int* err;
-    int nt, batch, d;
     unsigned long long total;
 };
 
-__device__ __forceinline__ double* tile(double* base, const Dag& g, int b, int i, int j) {
+__device__ __forceinline__ double* tile(double* base, const Grp& g, int b, int i, int j) {
     return base + (((size_t)b * g.nt + i) * g.nt + j) * TILE_ELEMS;
 }
-__device__ __forceinline__ int* st(int* base, const Dag& g, int b, int i, int j) {
+__device__ __forceinline__ int* st(int* base, const Grp& g, int b, int i, int j) {
     return base + ((size_t)b * g.nt + i) * g.nt + j;
 }
 
 // One thread: wait until *p >= target (acquire). False when the graph was aborted or the wait ran out of time.
-__device__ bool wait_ge(const int* p, int target, const Dag& g, int b) {
+__device__ bool wait_ge(const int* p, int target, const Dag& g, int problem) {
     if (ld_acquire(p) >= target) return true;
     const uint64_t t0 = gtimer();
     unsigned ns = 32;
@@ -322,7 +334,7 @@ __device__ bool wait_ge(const int* p, int target, const Dag& g, int b) {
         if (*reinterpret_cast<volatile int*>(g.abort_flag)) return false;
         if (gtimer() - t0 > WAIT_LIMIT_NS) {
             atomicExch(g.abort_flag, 1);
-            clha_record_error(g.err, CLHA_ERR_TIMEOUT, b, 0, KID_FACTOR);
+            clha_record_error(g.err, CLHA_ERR_TIMEOUT, problem, 0, KID_FACTOR);
             return false;
         }
     }
@@ -346,25 +358,29 @@ __device__ __forceinline__ void stage_counts(int nt, int s, long long (&n)[6]) {
     n[4] = R >= 1 ? (R - 1) * R / 2 : 0;
     n[5] = R >= 1 ? R - 1 : 0;
 }
+__device__ __forceinline__ unsigned long long stage_total(int nt, int s) {
+    if (s > nt) return 0;
+    long long n[6];
+    stage_counts(nt, s, n);
+    return (unsigned long long)(n[0] + n[1] + n[2] + n[3] + n[4] + n[5]);
+}
 
 __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
     extern __shared__ double dsm[];
     Tile* T0 = reinterpret_cast<Tile*>(dsm);
     Tile* T1 = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
     double* dinv = dsm + 2 * TILE_DOUBLES;
-    unsigned long long* lvl = reinterpret_cast<unsigned long long*>(dinv + NB);   // [nt + 2] stage starts
+    unsigned long long* lvl = reinterpret_cast<unsigned long long*>(dinv + NB);   // [max_nt + 2] stage starts
     __shared__ unsigned long long s_ticket;
     __shared__ int s_ok;
-    const int nt = g.nt, batch = g.batch, tid = threadIdx.x, lane = tid & 31;
-    if (tid == 0) {
+    const int S = g.max_nt, tid = threadIdx.x, lane = tid & 31;
+    if (tid == 0) {   // stage s holds, group after group, stage s of every group that has one
         unsigned long long acc = 0;
-        for (int s = 0; s <= nt; ++s) {
+        for (int s = 0; s <= S; ++s) {
             lvl[s] = acc;
-            long long n[6];
-            stage_counts(nt, s, n);
-            acc += (unsigned long long)(n[0] + n[1] + n[2] + n[3] + n[4] + n[5]) * batch;
+            for (int k = 0; k < g.ng; ++k) acc += stage_total(g.grp[k].nt, s) * g.grp[k].batch;
         }
-        lvl[nt + 1] = acc;
+        lvl[S + 1] = acc;
     }
     // Thread 0 holds the next number while the CTA runs the current task (taking numbers in order
     // and running them in order keeps the schedule deadlock-free).
@@ -378,14 +394,25 @@ __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
         const unsigned long long t = s_ticket;
         if (t >= g.total) break;
         if (tid == 0) next = atomicAdd(g.ticket, 1ull);
-        // decode: stage, class, problem, task (q: 0 P, 1 S, 2/5 G, 3 F, 4 Q), level m, tiles i, j
-        int lo = 0, hi = nt;
+        // decode: stage, group, class, problem, task (q: 0 P, 1 S, 2/5 G, 3 F, 4 Q), level m, tiles i, j
+        int lo = 0, hi = S;
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
             if (lvl[mid] <= t) lo = mid; else hi = mid - 1;
         }
         const int sg = lo;
         unsigned long long r = t - lvl[sg];
+        Grp G = g.grp[0];
+        bool found = false;
+#pragma unroll
+        for (int k = 0; k < MAX_GROUPS; ++k) {   // (unrolled: the group record stays in registers)
+            if (!found && k < g.ng) {
+                const unsigned long long c = stage_total(g.grp[k].nt, sg) * g.grp[k].batch;
+                if (r < c) { G = g.grp[k]; found = true; }
+                else r -= c;
+            }
+        }
+        const int nt = G.nt, batch = G.batch;
         long long n[6];
         stage_counts(nt, sg, n);
         int c = 0;
@@ -394,6 +421,7 @@ __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
             if (c == cq && r >= (unsigned long long)n[cq] * batch) { r -= (unsigned long long)n[cq] * batch; ++c; }
         const long long local = (long long)(r / batch);
         const int b = (int)(r % batch);
+        const int prob = G.pbase + b;
         int q, m = sg - 1, i = 0, j = 0;
         if (c == 0) { q = 2; i = m + 1 + (int)local; j = m + 1; }
         else if (c == 1) { q = 0; m = sg; }
@@ -415,41 +443,41 @@ __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
         int out_value;
         const int* wp[3] = {nullptr, nullptr, nullptr};
         int wt[3] = {0, 0, 0};
-        double* Dm = g.D + ((size_t)b * nt + m) * TILE_ELEMS;
+        double* Dm = G.D + ((size_t)b * nt + m) * TILE_ELEMS;
         if (q == 0) {            // P(m)
-            wp[0] = st(g.stA, g, b, m, m); wt[0] = m;
-            out_state = st(g.stA, g, b, m, m); out_value = m + 1;
+            wp[0] = st(G.stA, G, b, m, m); wt[0] = m;
+            out_state = st(G.stA, G, b, m, m); out_value = m + 1;
         } else if (q == 1) {     // L_im = A_im D_m^T
-            wp[0] = st(g.stA, g, b, i, m); wt[0] = m;
-            wp[1] = st(g.stA, g, b, m, m); wt[1] = m + 1;
-            P = tile(g.A, g, b, i, m); Qm = Dm; C = tile(g.A, g, b, i, m);
-            out_state = st(g.stA, g, b, i, m); out_value = m + 1;
+            wp[0] = st(G.stA, G, b, i, m); wt[0] = m;
+            wp[1] = st(G.stA, G, b, m, m); wt[1] = m + 1;
+            P = tile(G.A, G, b, i, m); Qm = Dm; C = tile(G.A, G, b, i, m);
+            out_state = st(G.stA, G, b, i, m); out_value = m + 1;
         } else if (q == 2 || q == 5) {   // A_ij -= L_im L_jm^T
-            wp[0] = st(g.stA, g, b, i, m); wt[0] = m + 1;
-            wp[1] = st(g.stA, g, b, j, m); wt[1] = m + 1;
-            wp[2] = st(g.stA, g, b, i, j); wt[2] = m;
-            P = tile(g.A, g, b, i, m); Qm = tile(g.A, g, b, j, m); C = tile(g.A, g, b, i, j);
+            wp[0] = st(G.stA, G, b, i, m); wt[0] = m + 1;
+            wp[1] = st(G.stA, G, b, j, m); wt[1] = m + 1;
+            wp[2] = st(G.stA, G, b, i, j); wt[2] = m;
+            P = tile(G.A, G, b, i, m); Qm = tile(G.A, G, b, j, m); C = tile(G.A, G, b, i, j);
             load_c = true; negate = true;
-            out_state = st(g.stA, g, b, i, j); out_value = m + 1;
+            out_state = st(G.stA, G, b, i, j); out_value = m + 1;
         } else if (q == 3) {     // Y_jm = -R_jm D_m^T
-            wp[0] = st(g.stY, g, b, j, m); wt[0] = m - j;
-            wp[1] = st(g.stA, g, b, m, m); wt[1] = m + 1;
-            P = tile(g.Y, g, b, j, m); Qm = Dm; C = tile(g.Y, g, b, j, m);
+            wp[0] = st(G.stY, G, b, j, m); wt[0] = m - j;
+            wp[1] = st(G.stA, G, b, m, m); wt[1] = m + 1;
+            P = tile(G.Y, G, b, j, m); Qm = Dm; C = tile(G.Y, G, b, j, m);
             negate = true;
-            out_state = st(g.stY, g, b, j, m); out_value = m - j + 1;
+            out_state = st(G.stY, G, b, j, m); out_value = m - j + 1;
         } else {                 // R_ji (+)= Y_jm L_im^T
-            wp[0] = st(g.stY, g, b, j, m); wt[0] = m - j + 1;
-            wp[1] = st(g.stA, g, b, i, m); wt[1] = m + 1;
-            wp[2] = st(g.stY, g, b, j, i); wt[2] = m - j;
-            P = tile(g.Y, g, b, j, m); Qm = tile(g.A, g, b, i, m); C = tile(g.Y, g, b, j, i);
+            wp[0] = st(G.stY, G, b, j, m); wt[0] = m - j + 1;
+            wp[1] = st(G.stA, G, b, i, m); wt[1] = m + 1;
+            wp[2] = st(G.stY, G, b, j, i); wt[2] = m - j;
+            P = tile(G.Y, G, b, j, m); Qm = tile(G.A, G, b, i, m); C = tile(G.Y, G, b, j, i);
             load_c = (m != j);
-            out_state = st(g.stY, g, b, j, i); out_value = m - j + 1;
+            out_state = st(G.stY, G, b, j, i); out_value = m - j + 1;
         }
         if (tid < 32) {
             bool ok = true;
 #pragma unroll
             for (int k = 0; k < 3; ++k)
-                if (lane == k && wp[k]) ok = wait_ge(wp[k], wt[k], g, b);
+                if (lane == k && wp[k]) ok = wait_ge(wp[k], wt[k], g, prob);
             ok = __all_sync(0xffffffffu, ok);
             if (lane == 0) s_ok = ok;
         }
@@ -457,12 +485,12 @@ __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
         if (!s_ok) break;
 
         if (q == 0) {
-            tile_to_smem(T0, tile(g.A, g, b, m, m));
+            tile_to_smem(T0, tile(G.A, G, b, m, m));
             cp_async_wait_all();
             __syncthreads();
-            tile_potrf_inv(T0, T1, dinv, tile(g.A, g, b, m, m), Dm, tile(g.Y, g, b, m, m), g.err, b, NB * m, g.d);
+            tile_potrf_inv(T0, T1, dinv, tile(G.A, G, b, m, m), Dm, tile(G.Y, G, b, m, m), g.err, prob, NB * m, G.d);
             __syncthreads();
-            if (tid == 0) st_release(st(g.stY, g, b, m, m), 1);
+            if (tid == 0) st_release(st(G.stY, G, b, m, m), 1);
         } else {
             tile_gemm_nt(P, Qm, T0, T1, C, load_c, negate);
         }
@@ -477,51 +505,88 @@ constexpr size_t dag_smem_bytes(int nt) {
 
 }  // namespace
 
-size_t factor_workspace_bytes(int batch, int d) {
-    const size_t nt = (size_t)d / NB;
-    const size_t tiles = (size_t)batch * nt * nt;
+namespace {
+size_t group_bytes(const FactorGroup& gr, size_t* states) {
+    const size_t nt = (size_t)gr.d / NB;
+    const size_t tiles = (size_t)gr.batch * nt * nt;
+    *states = 2 * tiles * sizeof(int);
     return 2 * clha_round_up(tiles * TILE_ELEMS * sizeof(double)) +
-           clha_round_up((size_t)batch * nt * TILE_ELEMS * sizeof(double)) +
-           clha_round_up(2 * tiles * sizeof(int) + 2 * sizeof(unsigned long long));
+           clha_round_up((size_t)gr.batch * nt * TILE_ELEMS * sizeof(double));
+}
+}  // namespace
+
+size_t factor_workspace_bytes(const FactorGroup* groups, int n) {
+    size_t total = 0, states = 2 * sizeof(unsigned long long);
+    for (int k = 0; k < n; ++k) {
+        size_t s;
+        total += group_bytes(groups[k], &s);
+        states += s;
+    }
+    return total + clha_round_up(states);
 }
 
-cudaError_t launch_factor(cudaStream_t s, int num_sms, const float* H_d, int batch, int d, float* U, void* ws,
-                          int* err) {
-    const int nt = d / NB;
-    const size_t tiles = (size_t)batch * nt * nt;
+cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups, int n, void* ws, int* err) {
+    if (n < 1 || n > MAX_GROUPS) return cudaErrorInvalidValue;
     char* cur = (char*)ws;
     Dag g;
-    g.A = (double*)clha_carve(cur, tiles * TILE_ELEMS * sizeof(double));
-    g.Y = (double*)clha_carve(cur, tiles * TILE_ELEMS * sizeof(double));
-    g.D = (double*)clha_carve(cur, (size_t)batch * nt * TILE_ELEMS * sizeof(double));
-    const size_t state_bytes = 2 * tiles * sizeof(int) + 2 * sizeof(unsigned long long);
-    char* sts = (char*)clha_carve(cur, state_bytes);
+    g.ng = n;
+    g.max_nt = 0;
+    g.err = err;
+    size_t state_bytes = 2 * sizeof(unsigned long long);
+    int pbase = 0;
+    for (int k = 0; k < n; ++k) {
+        const FactorGroup& gr = groups[k];
+        const int nt = gr.d / NB;
+        const size_t tiles = (size_t)gr.batch * nt * nt;
+        Grp& G = g.grp[k];
+        G.A = (double*)clha_carve(cur, tiles * TILE_ELEMS * sizeof(double));
+        G.Y = (double*)clha_carve(cur, tiles * TILE_ELEMS * sizeof(double));
+        G.D = (double*)clha_carve(cur, (size_t)gr.batch * nt * TILE_ELEMS * sizeof(double));
+        G.nt = nt;
+        G.batch = gr.batch;
+        G.d = gr.d;
+        G.pbase = pbase;
+        pbase += gr.batch;
+        state_bytes += 2 * tiles * sizeof(int);
+        if (nt > g.max_nt) g.max_nt = nt;
+    }
+    for (int k = n; k < MAX_GROUPS; ++k) g.grp[k] = g.grp[0];
+    char* sts = (char*)clha_carve(cur, state_bytes);   // task counter, abort flag, every group's states
     g.ticket = (unsigned long long*)sts;
     g.abort_flag = (int*)(sts + sizeof(unsigned long long));
-    g.stA = (int*)(sts + 2 * sizeof(unsigned long long));
-    g.stY = g.stA + tiles;
-    g.err = err;
-    g.nt = nt;
-    g.batch = batch;
-    g.d = d;
-    unsigned long long per = 0;
-    for (int m = 0; m < nt; ++m) {
-        const long long R = nt - 1 - m;
-        per += 1 + 2 * R + m + (m + 1) * R + (R >= 1 ? (R - 1) * R / 2 : 0);
+    int* st_cur = (int*)(sts + 2 * sizeof(unsigned long long));
+    g.total = 0;
+    for (int k = 0; k < n; ++k) {
+        Grp& G = g.grp[k];
+        const size_t tiles = (size_t)G.batch * G.nt * G.nt;
+        G.stA = st_cur;
+        G.stY = st_cur + tiles;
+        st_cur += 2 * tiles;
+        unsigned long long per = 0;
+        for (int m = 0; m < G.nt; ++m) {
+            const long long R = G.nt - 1 - m;
+            per += 1 + 2 * R + m + (m + 1) * R + (R >= 1 ? (R - 1) * R / 2 : 0);
+        }
+        g.total += per * (unsigned long long)G.batch;
     }
-    g.total = per * (unsigned long long)batch;
 
-    const size_t smem = dag_smem_bytes(nt);
+    const size_t smem = dag_smem_bytes(g.max_nt);
     cudaError_t e = cudaFuncSetAttribute(fac_dag, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(sts, 0, state_bytes, s)) != cudaSuccess) return e;
-    fac_load<<<dim3((unsigned)(nt * (nt + 1) / 2), batch), 256, 0, s>>>(H_d, d, nt, g.A);
-    clha_note_launches(1);
+    for (int k = 0; k < n; ++k) {
+        const Grp& G = g.grp[k];
+        fac_load<<<dim3((unsigned)(G.nt * (G.nt + 1) / 2), G.batch), 256, 0, s>>>(groups[k].H, G.d, G.nt, G.A);
+        clha_note_launches(1);
+    }
     unsigned long long grid = 2ull * (unsigned long long)num_sms;   // two resident CTAs per SM
     if (grid > g.total) grid = g.total;
     fac_dag<<<(unsigned)grid, 256, smem, s>>>(g);
     clha_note_launches(1);
-    fac_store<<<dim3((unsigned)(nt * nt), batch), 256, 0, s>>>(g.Y, d, nt, U);
-    clha_note_launches(1);
+    for (int k = 0; k < n; ++k) {
+        const Grp& G = g.grp[k];
+        fac_store<<<dim3((unsigned)(G.nt * G.nt), G.batch), 256, 0, s>>>(G.Y, G.d, G.nt, groups[k].U);
+        clha_note_launches(1);
+    }
     return cudaGetLastError();
 }

@@ -312,13 +312,14 @@ class MoECalibration:
         lo, hi = min(idx), max(idx) + 1
         contiguous = sorted(idx) == list(range(lo, hi))
         runs = [(lo, hi)] if contiguous else [(i, i + 1) for i in idx]
-        with t.span("factor"):
+        with t.span("factor"):   # one task-graph launch per run: routed in/down (+ shared in/down)
             for a, b in runs:
-                L.clha_factor(ctx, self.Hd_in[a * E:b * E], (b - a) * E, dm, self.U_in[a * E:b * E])
-                L.clha_factor(ctx, self.Hd_dn[a * E:b * E], (b - a) * E, dff, self.U_dn[a * E:b * E])
+                groups = [(self.Hd_in[a * E:b * E], (b - a) * E, dm, self.U_in[a * E:b * E]),
+                          (self.Hd_dn[a * E:b * E], (b - a) * E, dff, self.U_dn[a * E:b * E])]
                 if ns:
-                    L.clha_factor(ctx, self.Hd_sin[a:b], b - a, dm, self.U_sin[a:b])
-                    L.clha_factor(ctx, self.Hd_sdn[a * ns:b * ns], (b - a) * ns, sdff, self.U_sdn[a * ns:b * ns])
+                    groups += [(self.Hd_sin[a:b], b - a, dm, self.U_sin[a:b]),
+                               (self.Hd_sdn[a * ns:b * ns], (b - a) * ns, sdff, self.U_sdn[a * ns:b * ns])]
+                L.clha_factor_groups(ctx, groups)
         br, bs = self.bits_routed, self.bits_shared
         for i, m in zip(idx, modes):
             r = self.res[m]

@@ -254,6 +254,44 @@ def test_factor_matches_oracle(ctx, d, batch):
         assert rel_fro(got, want) < 1e-6
 
 
+def test_factor_groups_match_oracle_and_report_across_groups(ctx):
+    """Three groups of different sizes in one graph launch; each problem against the oracle. Then a
+    non-positive pivot in the last group's second problem: its index counts across the groups."""
+    specs = [(384, 3), (128, 2), (640, 2)]
+    groups, host = [], []
+    for gi, (d, batch) in enumerate(specs):
+        g = _gen(100 + gi)
+        Hs = []
+        for b in range(batch):
+            A = torch.randn((d, d // 4), generator=g).double()
+            Hs.append((A @ A.T / (d // 4) + 0.05 * torch.eye(d, dtype=torch.float64)).float())
+        Hd = torch.stack(Hs).to(DEV)
+        U = torch.full_like(Hd, float("nan"))
+        groups.append((Hd, batch, d, U))
+        host.append(Hs)
+    L.clha_factor_groups(ctx, groups)
+    L.clha_check(ctx)
+    for (Hd, batch, d, U), Hs in zip(groups, host):
+        for b in range(batch):
+            got = U[b].double().cpu().numpy()
+            assert np.all(np.tril(got, -1) == 0)
+            assert rel_fro(got, O.factor(Hs[b].double().numpy())) < 1e-6
+    # non-PD: problem 1 of group 2 = problem 3 + 2 + 1 = 6 across the groups, original column 70
+    Hd2 = groups[2][0]
+    Hd2[1] = torch.eye(640, device=DEV)
+    Hd2[1, 70, 70] = -1.0
+    L.clha_factor_groups(ctx, groups)
+    with pytest.raises(L.ClhaError) as ei:
+        L.clha_check(ctx)
+    assert ei.value.status == L.ERR_NOT_PD
+    assert "problem 6" in str(ei.value) and "index 70" in str(ei.value)
+    L.clha_check(ctx)
+    for b in range(3):   # the other problems are unaffected
+        assert torch.isfinite(groups[0][3][b]).all()
+    with pytest.raises(L.ClhaError):
+        L.clha_factor_groups(ctx, groups * 2)   # more than FACTOR_MAX_GROUPS
+
+
 def test_factor_non_pd_reports_column(ctx):
     d = 256
     H = torch.eye(d)
