@@ -2,21 +2,29 @@
 // aggregated Hessian's factor U (H_d^-1 = U^T U), restated from GPTQ (Frantar et al. 2022, Alg. 1).
 //
 // One CTA owns 128 rows of one weight and walks the columns in 128-column blocks (the lazy-update
-// block and the quantization group coincide). Warp roles:
-//   warps 0-3  one thread per row: a row's whole block lives in its registers, so the column-by-
-//              column error feedback inside a block needs no communication. Per block: take the lazy
-//              update from TMEM, w = W[:, blk] - acc; fix the group's grid from the current values;
-//              then for 128 columns q = clamp(round(w/s) + z), w_hat = s (q - z),
-//              e = (w - w_hat) / U_jj and w[:, c > j] -= e U[j, c] (U's diagonal block in shared
-//              memory). The block's errors go to global memory split into tf32 hi + lo parts.
-//   warp 4     TMA producer: for block b+1 it streams E[:, :cb] (hi, lo) and the U panel U[:cb, blk]
-//              (hi, lo, from a transposed copy so both operands are K-major) in 32-wide k steps;
-//              the last 128 k (the errors of the block being quantized) only after the row warps
-//              signal they are written.
-//   warp 5     MMA issuer: acc = E[:, :cb] U[:cb, blk] with tcgen05.mma kind::tf32, M=128 N=128 K=8,
-//              three products per step (hi*hi + hi*lo + lo*hi: float32-class accuracy from tf32
-//              inputs), into one of two TMEM accumulators, so block b+1's update overlaps block b's
-//              sequential columns.
+// block and the quantization group coincide), each block in four 32-column quarters. The column
+// recurrence w[:, c] -= e_j U[j, c] (c > j) is split three ways:
+//   * inside a quarter: fp32 FMAs in the row thread's registers (a row's 32 current values);
+//   * from a quarter to the later quarters of its block: one small tensor-core product
+//     acc[:, later] += E_q U[q, later], accumulated into the same TMEM columns that hold the block's
+//     lazy update (the row threads read each quarter's columns only after it);
+//   * from a block to all later blocks: the lazy update acc = E[:, :cb] U[:cb, blk], streamed while
+//     the previous block is being swept.
+// Products are tcgen05.mma kind::tf32 with operands split hi + lo and three products per step
+// (hi*hi + hi*lo + lo*hi: float32-class accuracy). Warp roles:
+//   warps 0-3  one thread per row: grid of the block from its current values, then per quarter: read
+//              the quarter's update from TMEM, q = clamp(round(w/s) + z), w_hat = s (q - z),
+//              e = (w - w_hat) / U_jj, in-quarter updates; write the quarter's errors as tf32 hi/lo
+//              into shared memory in the 128-byte-swizzled K-major layout, which is both the A operand
+//              of the quarter's product and the source of a TMA store of E to global memory (read
+//              by the later blocks' lazy updates).
+//   warp 4     TMA producer of the lazy update: E[:, :cb] (hi, lo) and the U panel U[:cb, blk] (hi,
+//              lo, from a transposed copy so both operands are K-major) in 32-wide k steps; the last
+//              128 k (the errors of the block being swept) only after they are stored.
+//   warp 5     MMA issuer: the quarter products as soon as they are requested (the next quarter's
+//              columns first, with their own completion signal, since they gate the row threads;
+//              then the rest), between them the next block's lazy update (one step in the tensor
+//              pipe at a time), into the other of two TMEM accumulators.
 // The grid and the code are decided with IEEE float32 operations (division and rounding to nearest
 // even), the same operations a float32 reference takes on the same current value.
 #include "clha_internal.h"
@@ -27,22 +35,33 @@ namespace {
 
 constexpr int R = 128;      // rows per CTA (one per row thread)
 constexpr int BLK = 128;    // columns per lazy block and per group
-constexpr int KS = 32;      // k per pipeline stage (one 128-byte row of fp32)
+constexpr int QW = 32;      // columns per quarter
+constexpr int KS = 32;      // k per lazy pipeline stage (one 128-byte row of fp32)
 constexpr int STAGES = 2;
 constexpr int A_BYTES = R * KS * 4;                       // 16 KB: E rows (hi or lo)
 constexpr int B_BYTES = KS * BLK * 4;                     // 16 KB: U panel (hi or lo), K-major
 constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;    // 64 KB
-constexpr int UD_OFF = STAGES * STAGE_BYTES;
-constexpr int UINV_OFF = UD_OFF + BLK * BLK * 4;
-constexpr int QROW = BLK + 4;                             // bytes per row of the code buffer (padded)
-constexpr int CODES_OFF = UINV_OFF + BLK * 4;            // block codes, [row][QROW] bytes
-constexpr int QE_OFF = CODES_OFF + R * QROW;             // one quarter's errors, [column][row] floats
-constexpr int QW = 32;                                    // columns per quarter of a block
-constexpr int BAR_OFF = QE_OFF + QW * R * 4;
-constexpr int SMEM_BYTES = BAR_OFF + 128 + 1024;
-constexpr int STG = 68;                                   // staging row (floats): 64 columns + pad
+constexpr int SA_OFF = STAGES * STAGE_BYTES;              // quarter errors hi, lo: [128 rows][32 k]
+constexpr int SA_BYTES = R * QW * 4;                      // 16 KB each
+// U rows of a quarter's product (K-major [n][32 k], hi then lo), two buffers used alternately:
+// quarters 0 and 2 (96 and 32 rows) in buffer 0, quarter 1 (64 rows) in buffer 1
+constexpr int SB0_OFF = SA_OFF + 2 * SA_BYTES;
+constexpr int SB0_HALF = 96 * QW * 4;                     // 12 KB
+constexpr int SB1_OFF = SB0_OFF + 2 * SB0_HALF;
+constexpr int SB1_HALF = 64 * QW * 4;                     // 8 KB
+constexpr int UQ_OFF = SB1_OFF + 2 * SB1_HALF;            // the block's four diagonal 32x32 U blocks
+constexpr int UINV_OFF = UQ_OFF + 4 * QW * QW * 4;
+constexpr int BAR_OFF = UINV_OFF + BLK * 4;
+constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;
 constexpr int kThreads = 192;
-constexpr uint32_t IDESC = tc::idesc_f32acc(2 /*tf32*/, 0 /*A K-major*/, 0 /*B K-major*/, R, BLK);
+constexpr uint32_t IDESC_LAZY = tc::idesc_f32acc(2 /*tf32*/, 0 /*A K-major*/, 0 /*B K-major*/, R, BLK);
+static_assert(SA_OFF % 1024 == 0 && SB0_OFF % 1024 == 0 && (SB0_OFF + SB0_HALF) % 1024 == 0 && SB1_OFF % 1024 == 0 &&
+                  (SB1_OFF + SB1_HALF) % 1024 == 0, "swizzle atoms");
+static_assert(SMEM_BYTES <= 232448, "shared memory");
+
+__host__ __device__ constexpr uint32_t idesc_spill(int n) {
+    return tc::idesc_f32acc(2, 0, 0, R, (uint32_t)n);
+}
 
 struct GptqParams {
     const float* U;        // [n_u, d_in, d_in] (for the diagonal blocks)
@@ -54,8 +73,6 @@ struct GptqParams {
     float* scales;
     uint8_t* zeros;
     float* W_hat;
-    float* Ehi;            // [batch, d_out, d_in]
-    float* Elo;
     const double* lambda;  // [n_u] damping of each factor, or null
     double* loss;          // [batch] |E|^2 - lambda |W_hat - W|^2, or null
     int* err;
@@ -69,80 +86,88 @@ __device__ __forceinline__ float to_tf32(float x) {
 
 __device__ __forceinline__ void row_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-// 16-byte asynchronous global -> shared copy (all of a thread's copies stay in flight together).
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(smem_dst)), "l"(gsrc) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
-__device__ __forceinline__ void fence_proxy_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Columns [32Q, 32Q+32) of the row's block, in order: quantize each, record its error and apply it
-// to the rest of the quarter (unrolled; every index is a compile-time constant).
-template <int Q>
-__device__ __forceinline__ void quarter_sweep(float (&w)[BLK], float s, float z, float maxq, const float* uinv,
-                                              const float (*Ud)[BLK], uint8_t (*qs)[QROW], float (*qe)[R], int t) {
+// This row's 32 current values of a quarter, in order: quantize each, keep its error in w[j] and
+// apply it to the quarter's later columns (unrolled; every index a compile-time constant). The codes
+// are packed four to a word.
+__device__ __forceinline__ void quarter_sweep(float (&w)[QW], float s, float z, float maxq, const float* uinv,
+                                              const float (*Uq)[QW], uint32_t (&codes)[QW / 4]) {
 #pragma unroll
-    for (int jj = 0; jj < QW; ++jj) {
-        const int j = Q * QW + jj;
+    for (int j = 0; j < QW; ++j) {
         float q = __fadd_rn(rintf(__fdiv_rn(w[j], s)), z);
         q = fminf(fmaxf(q, 0.f), maxq);
         const float wh = __fmul_rn(s, __fsub_rn(q, z));
         const float e = (w[j] - wh) * uinv[j];
-        w[j] = e;                                // a quantized column's register keeps its error
-        qs[t][j] = (uint8_t)q;
-        qe[jj][t] = e;
+        w[j] = e;
+        if ((j & 3) == 0) codes[j >> 2] = 0u;
+        codes[j >> 2] |= (uint32_t)q << (8 * (j & 3));
 #pragma unroll
-        for (int c = j + 1; c < (Q + 1) * QW; ++c) w[c] = fmaf(-e, Ud[j][c], w[c]);
+        for (int c = 1; c < QW; ++c)
+            if (c > j) w[c] = fmaf(-e, Uq[j][c], w[c]);
     }
 }
 
-// The quarter's 32 errors applied, column by column, to every later column of the block: a rolled
-// loop over the errors (read back from shared memory) keeps the code small.
-template <int Q>
-__device__ __forceinline__ void quarter_spill(float (&w)[BLK], const float (*Ud)[BLK], const float (*qe)[R], int t) {
-#pragma unroll 2
-    for (int jj = 0; jj < QW; ++jj) {
-        const float e = qe[jj][t];
-        const float4* u4 = reinterpret_cast<const float4*>(&Ud[Q * QW + jj][(Q + 1) * QW]);
+// W[row, c0 .. c0+31] as floats (bf16 or fp32 source).
+__device__ __forceinline__ void load_w32(const GptqParams& p, size_t off, float (&w)[QW]) {
+    if (p.w_f32) {
+        const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.W) + off);
 #pragma unroll
-        for (int c4 = 0; c4 < (BLK - (Q + 1) * QW) / 4; ++c4) {
-            const float4 u = u4[c4];
-            const int c = (Q + 1) * QW + 4 * c4;
-            w[c] = fmaf(-e, u.x, w[c]);
-            w[c + 1] = fmaf(-e, u.y, w[c + 1]);
-            w[c + 2] = fmaf(-e, u.z, w[c + 2]);
-            w[c + 3] = fmaf(-e, u.w, w[c + 3]);
+        for (int i = 0; i < QW / 4; ++i) {
+            const float4 v = src[i];
+            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        }
+    } else {
+        const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.W) + off);
+#pragma unroll
+        for (int i = 0; i < QW / 8; ++i) {
+            const uint4 v = src[i];
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __bfloat1622float2(h2[j]);
+                w[8 * i + 2 * j] = f.x;
+                w[8 * i + 2 * j + 1] = f.y;
+            }
         }
     }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUtensorMap tmElo,
-        const __grid_constant__ CUtensorMap tmUhi, const __grid_constant__ CUtensorMap tmUlo, GptqParams p) {
+        const __grid_constant__ CUtensorMap tmUhi, const __grid_constant__ CUtensorMap tmUlo,
+        const __grid_constant__ CUtensorMap tmQhi, const __grid_constant__ CUtensorMap tmQlo, GptqParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float (*Ud)[BLK] = reinterpret_cast<float (*)[BLK]>(smem + UD_OFF);
+    float (*Uq)[QW][QW] = reinterpret_cast<float (*)[QW][QW]>(smem + UQ_OFF);
     float* uinv = reinterpret_cast<float*>(smem + UINV_OFF);
-    uint8_t (*qs)[QROW] = reinterpret_cast<uint8_t (*)[QROW]>(smem + CODES_OFF);
-    float (*qe)[R] = reinterpret_cast<float (*)[R]>(smem + QE_OFF);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
     const uint32_t full0 = tc::smem_u32(bars);
     const uint32_t empty0 = full0 + 8 * STAGES;
-    const uint32_t tfull0 = empty0 + 8 * STAGES;
-    const uint32_t tempty0 = tfull0 + 16;
-    const uint32_t eready = tempty0 + 16;
-    const uint32_t drain = eready + 8;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + BAR_OFF + 8 * (2 * STAGES + 6));
+    const uint32_t tfull0 = empty0 + 8 * STAGES;   // lazy update of a block complete (per accumulator)
+    const uint32_t tempty0 = tfull0 + 16;          // row threads done with an accumulator
+    const uint32_t eready = tempty0 + 16;          // a block's errors are in global memory
+    const uint32_t sreq = eready + 8;              // a quarter's errors are in shared memory
+    const uint32_t sbfull = sreq + 8;              // the quarter product's U rows are in shared memory
+    const uint32_t sdone = sbfull + 8;             // the quarter product's next-quarter columns are done
+    const uint32_t sdone2 = sdone + 8;             // the whole quarter product is done (buffers free)
+    const uint32_t drain = sdone2 + 8;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + BAR_OFF + 8 * (2 * STAGES + 10));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const uint32_t sa_hi = tc::smem_u32(smem + SA_OFF), sa_lo = sa_hi + SA_BYTES;
+    const uint32_t sb0 = tc::smem_u32(smem + SB0_OFF), sb1 = tc::smem_u32(smem + SB1_OFF);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.y;
     const int r0 = blockIdx.x * R;
     const int u = b % p.n_u;
     const int nblk = p.d_in / BLK;
+    const int ey = b * p.d_out + r0;               // this CTA's rows in the [batch * d_out, d_in] E view
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             tc::mbar_init(full0 + 8 * s, 1);
@@ -152,7 +177,11 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
             tc::mbar_init(tfull0 + 8 * a, 1);
             tc::mbar_init(tempty0 + 8 * a, R);
         }
-        tc::mbar_init(eready, R);
+        tc::mbar_init(eready, 1);
+        tc::mbar_init(sreq, R);
+        tc::mbar_init(sbfull, 1);
+        tc::mbar_init(sdone, 1);
+        tc::mbar_init(sdone2, 1);
         tc::mbar_init(drain, 1);
         *abort_flag = 0;
         tc::fence_barrier_init();
@@ -164,7 +193,7 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 4) {
-        // ------------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------------ TMA producer (lazy update)
         if (lane == 0) {
             tc::prefetch_tmap(&tmEhi);
             tc::prefetch_tmap(&tmElo);
@@ -172,12 +201,11 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
             tc::prefetch_tmap(&tmUlo);
             int it = 0;
             bool ok = true;
-            const int ey = b * p.d_out + r0;
             for (int bb = 1; bb < nblk && ok; ++bb) {
                 const int cb = bb * BLK;
                 for (int ks = 0; ks < cb / KS; ++ks) {
                     const int k0 = ks * KS;
-                    if (k0 == cb - BLK) {   // errors of the previous block: wait until they are written
+                    if (k0 == cb - BLK) {   // errors of the previous block: wait until they are stored
                         if (!tc::mbar_wait_bounded(eready, (bb - 1) & 1, abort_flag)) { ok = false; break; }
                     }
                     const int s = it % STAGES;
@@ -202,37 +230,88 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
     } else if (warp == 5) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            int it = 0;
+            int it = 0, nq = 0;   // lazy k steps consumed; quarter products issued
             bool ok = true;
-            for (int bb = 1; bb < nblk && ok; ++bb) {
-                const int tcount = bb - 1;
-                const int acc = tcount & 1;
-                if (!tc::mbar_wait_bounded(tempty0 + 8 * acc, ((tcount >> 1) & 1) ^ 1, abort_flag)) break;
-                tc::fence_after_sync();
-                const uint32_t d_tmem = tmem + acc * BLK;
-                const int nks = bb * BLK / KS;
-                for (int ks = 0; ks < nks; ++ks, ++it) {
-                    const int s = it % STAGES;
-                    if (!tc::mbar_wait_bounded(full0 + 8 * s, (it / STAGES) & 1, abort_flag)) { ok = false; break; }
+            for (int bb = 0; bb < nblk && ok; ++bb) {
+                // block bb: its three quarter products (into acc bb & 1) and block bb+1's lazy update
+                const bool lazy = bb + 1 < nblk;
+                const int lacc = (bb + 1) & 1, pacc = bb & 1;
+                const int nks = lazy ? (bb + 1) * BLK / KS : 0;
+                int ks = 0, q = 0;
+                bool lazy_ready = !lazy;
+                if (lazy && bb >= 1) {   // the row threads are done with block bb-1's accumulator
+                    if (!tc::mbar_wait_bounded(tempty0 + 8 * lacc, ((bb - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
                     tc::fence_after_sync();
-                    const uint32_t ahi = tc::smem_u32(smem + s * STAGE_BYTES);
-                    const uint32_t alo = ahi + A_BYTES;
-                    const uint32_t bhi = ahi + 2 * A_BYTES;
-                    const uint32_t blo = bhi + B_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < KS / 8; ++kk) {
-                        const uint64_t dah = tc::sw128_desc(ahi + kk * 32, 16, 1024);
-                        const uint64_t dal = tc::sw128_desc(alo + kk * 32, 16, 1024);
-                        const uint64_t dbh = tc::sw128_desc(bhi + kk * 32, 16, 1024);
-                        const uint64_t dbl = tc::sw128_desc(blo + kk * 32, 16, 1024);
-                        tc::mma_tf32(d_tmem, dah, dbh, IDESC, (ks | kk) != 0);
-                        tc::mma_tf32(d_tmem, dah, dbl, IDESC, 1);
-                        tc::mma_tf32(d_tmem, dal, dbh, IDESC, 1);
-                    }
-                    tc::mma_commit(empty0 + 8 * s);
                 }
-                if (!ok) break;
-                tc::mma_commit(tfull0 + 8 * acc);
+                lazy_ready = true;
+                uint64_t t0 = tc::globaltimer_ns();
+                uint32_t spins = 0;
+                while (q < 3 || ks < nks) {
+                    bool progressed = false;
+                    if (q < 3 && tc::mbar_try_wait(sreq, nq & 1) && tc::mbar_try_wait(sbfull, nq & 1)) {
+                        tc::fence_after_sync();
+                        const uint32_t sbh = (q & 1) ? sb1 : sb0;
+                        const uint32_t sbl = sbh + ((q & 1) ? SB1_HALF : SB0_HALF);
+                        // part 1: the next quarter's 32 columns; part 2: the later ones
+                        for (int part = 0; part < 2; ++part) {
+                            const int n = part == 0 ? QW : BLK - QW * (q + 2);
+                            if (n > 0) {
+                                const uint32_t d_tmem = tmem + pacc * BLK + QW * (q + 1) + part * QW;
+                                const uint32_t id = idesc_spill(n);
+                                const uint32_t boff = part * 4096;   // 32 rows of 128 B
+#pragma unroll
+                                for (int kk = 0; kk < QW / 8; ++kk) {
+                                    const uint64_t dah = tc::sw128_desc(sa_hi + kk * 32, 16, 1024);
+                                    const uint64_t dal = tc::sw128_desc(sa_lo + kk * 32, 16, 1024);
+                                    const uint64_t dbh = tc::sw128_desc(sbh + boff + kk * 32, 16, 1024);
+                                    const uint64_t dbl = tc::sw128_desc(sbl + boff + kk * 32, 16, 1024);
+                                    tc::mma_tf32(d_tmem, dah, dbh, id, (bb > 0 || q > 0 || kk > 0) ? 1u : 0u);
+                                    tc::mma_tf32(d_tmem, dah, dbl, id, 1);
+                                    tc::mma_tf32(d_tmem, dal, dbh, id, 1);
+                                }
+                            }
+                            tc::mma_commit(part == 0 ? sdone : sdone2);
+                        }
+                        ++q;
+                        ++nq;
+                        progressed = true;
+                    }
+                    // a lazy step only once the previous one has left the tensor pipe, so that a
+                    // quarter product (which the row threads wait for) queues behind one step at most
+                    const bool pipe_clear = it == 0 || tc::mbar_try_wait(empty0 + 8 * ((it - 1) % STAGES), ((it - 1) / STAGES) & 1);
+                    if (lazy_ready && ks < nks && pipe_clear &&
+                        tc::mbar_try_wait(full0 + 8 * (it % STAGES), (it / STAGES) & 1)) {
+                        tc::fence_after_sync();
+                        const int s = it % STAGES;
+                        const uint32_t ahi = tc::smem_u32(smem + s * STAGE_BYTES);
+                        const uint32_t alo = ahi + A_BYTES;
+                        const uint32_t bhi = ahi + 2 * A_BYTES;
+                        const uint32_t blo = bhi + B_BYTES;
+                        const uint32_t d_tmem = tmem + lacc * BLK;
+#pragma unroll
+                        for (int kk = 0; kk < KS / 8; ++kk) {
+                            const uint64_t dah = tc::sw128_desc(ahi + kk * 32, 16, 1024);
+                            const uint64_t dal = tc::sw128_desc(alo + kk * 32, 16, 1024);
+                            const uint64_t dbh = tc::sw128_desc(bhi + kk * 32, 16, 1024);
+                            const uint64_t dbl = tc::sw128_desc(blo + kk * 32, 16, 1024);
+                            tc::mma_tf32(d_tmem, dah, dbh, IDESC_LAZY, (ks | kk) != 0);
+                            tc::mma_tf32(d_tmem, dah, dbl, IDESC_LAZY, 1);
+                            tc::mma_tf32(d_tmem, dal, dbh, IDESC_LAZY, 1);
+                        }
+                        tc::mma_commit(empty0 + 8 * s);
+                        ++ks;
+                        ++it;
+                        if (ks == nks) tc::mma_commit(tfull0 + 8 * lacc);
+                        progressed = true;
+                    }
+                    if (progressed) {
+                        t0 = tc::globaltimer_ns();
+                        spins = 0;
+                    } else if (((++spins) & 255u) == 0u) {
+                        if (*abort_flag) { ok = false; break; }
+                        if (tc::globaltimer_ns() - t0 > 2000000000ull) { *abort_flag = 1; ok = false; break; }
+                    }
+                }
             }
         }
         __syncwarp();
@@ -240,155 +319,164 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
         // ------------------------------------------------------------------ row threads
         const int t = threadIdx.x;
         const int row = r0 + t;
-        const size_t dd = (size_t)p.d_in * p.d_in;
-        const float* Ub = p.U + (size_t)u * dd;
+        const float* Ub = p.U + (size_t)u * p.d_in * p.d_in;
         const size_t wrow = ((size_t)b * p.d_out + row) * p.d_in;
         const float maxq = (float)((1 << p.bits) - 1);
         const int ngroups = p.d_in / BLK;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         bool ok = true;
+        int nq = 0;                  // quarter products requested so far
         double e2 = 0.0, d2 = 0.0;   // this row's |E|^2 and |W_hat - W|^2
+        auto load_sb = [&](int cb, int q) {   // the U rows of quarter q's product: n = later columns
+            const int nbox = 3 - q;
+            const uint32_t sbh = (q & 1) ? sb1 : sb0;
+            const uint32_t sbl = sbh + ((q & 1) ? SB1_HALF : SB0_HALF);
+            tc::mbar_arrive_expect_tx(sbfull, (uint32_t)(2 * nbox * 32 * QW * 4));
+            for (int bx = 0; bx < nbox; ++bx) {
+                const int n0 = u * p.d_in + cb + QW * (q + 1) + 32 * bx;
+                tc::tma_load_2d(sbh + bx * 4096, &tmQhi, sbfull, cb + QW * q, n0);
+                tc::tma_load_2d(sbl + bx * 4096, &tmQlo, sbfull, cb + QW * q, n0);
+            }
+        };
+        auto load_uq = [&](int cb) {          // the block's four diagonal 32x32 blocks of U
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int e = i * R + t;          // 0 .. 1023: (quarter, row, 16-byte piece)
+                const int qq = e >> 8, rr = (e >> 3) & 31, c4 = (e & 7) * 4;
+                cp_async16(&Uq[qq][rr][c4], Ub + (size_t)(cb + QW * qq + rr) * p.d_in + cb + QW * qq + c4);
+            }
+        };
+        // On a failed wait (abort) the row threads still run every step, so each reaches every named
+        // barrier; their later waits return at once.
+        load_uq(0);
         for (int bb = 0; bb < nblk; ++bb) {
             const int cb = bb * BLK;
-            row_bar();                                   // every row thread is done with the last Ud
-            // U's diagonal block: 128 rows x 512 B; thread t copies 16 B pieces (t % 32) of rows t/32 + 4i
-#pragma unroll 8
-            for (int i = 0; i < BLK / 4; ++i) {
-                const int r = (t >> 5) + 4 * i, c4 = (t & 31) * 4;
-                cp_async16(&Ud[r][c4], Ub + (size_t)(cb + r) * p.d_in + cb + c4);
-            }
-            cp_async_wait_all();
-            row_bar();
-            uinv[t] = 1.0f / Ud[t][t];
-            float w[BLK];
-            if (p.w_f32) {
-                const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.W) + wrow + cb);
-#pragma unroll
-                for (int i = 0; i < BLK / 4; ++i) {
-                    const float4 v = src[i];
-                    w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-                }
-            } else {
-                const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.W) + wrow + cb);
-#pragma unroll
-                for (int i = 0; i < BLK / 8; ++i) {
-                    const uint4 v = src[i];
-                    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float2 f = __bfloat1622float2(h2[j]);
-                        w[8 * i + 2 * j] = f.x;
-                        w[8 * i + 2 * j + 1] = f.y;
-                    }
-                }
-            }
-            if (bb > 0 && ok) {    // lazy update of this block from all earlier blocks' errors
-                const int tcount = bb - 1;
-                const int acc = tcount & 1;
-                if (!tc::mbar_wait_bounded(tfull0 + 8 * acc, (tcount >> 1) & 1, abort_flag)) ok = false;
+            const int acc = bb & 1;
+            const bool more = bb + 1 < nblk;
+            const size_t orow = ((size_t)b * p.d_out + row) * p.d_in + cb;   // this row's outputs
+            row_bar();                                   // the last block's readers of Uq are done
+            if (t == 0) load_sb(cb, 0);
+            cp_async_wait_all();                         // this block's Uq (issued during the last block)
+            uinv[t] = 1.0f / __ldg(Ub + (size_t)(cb + t) * p.d_in + cb + t);
+            if (bb > 0) {
+                if (!tc::mbar_wait_bounded(tfull0 + 8 * acc, (bb - 1) >> 1 & 1, abort_flag)) ok = false;
                 tc::fence_after_sync();
-                if (ok) {
-#pragma unroll
-                    for (int ch = 0; ch < BLK / 32; ++ch) {
-                        uint32_t v[32];
-                        tc::tmem_ld_32x32b_x32(tmem + lane_base + acc * BLK + ch * 32, v);
-                        tc::tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) w[ch * 32 + j] -= __uint_as_float(v[j]);
-                    }
-                }
-                tc::fence_before_sync();
-                tc::mbar_arrive(tempty0 + 8 * acc);
             }
-            row_bar();                                   // uinv complete
             // grid of the group from the current values (0 always on the grid; [-1, 1] if all zero)
             float xmin = 0.f, xmax = 0.f;
+            for (int ch = 0; ch < 4; ++ch) {
+                float w[QW];
+                load_w32(p, wrow + cb + QW * ch, w);
+                if (bb > 0) {
+                    uint32_t v[32];
+                    tc::tmem_ld_32x32b_x32(tmem + lane_base + acc * BLK + ch * QW, v);
+                    tc::tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < BLK; ++c) { xmin = fminf(xmin, w[c]); xmax = fmaxf(xmax, w[c]); }
+                    for (int j = 0; j < QW; ++j) w[j] -= __uint_as_float(v[j]);
+                }
+#pragma unroll
+                for (int j = 0; j < QW; ++j) { xmin = fminf(xmin, w[j]); xmax = fmaxf(xmax, w[j]); }
+            }
             if (xmin == 0.f && xmax == 0.f) { xmin = -1.f; xmax = 1.f; }
             const float s = __fdiv_rn(__fsub_rn(xmax, xmin), maxq);
             const float z = rintf(__fdiv_rn(-xmin, s));
-            const int g = cb / BLK;
-            p.scales[((size_t)b * p.d_out + row) * ngroups + g] = s;
-            p.zeros[((size_t)b * p.d_out + row) * ngroups + g] = (uint8_t)z;
-            // 128 columns in four quarters; each column still receives the errors of all earlier
-            // columns in column order, exactly as in a single column-by-column sweep
-            quarter_sweep<0>(w, s, z, maxq, uinv, Ud, qs, qe, t);
-            quarter_spill<0>(w, Ud, qe, t);
-            quarter_sweep<1>(w, s, z, maxq, uinv, Ud, qs, qe, t);
-            quarter_spill<1>(w, Ud, qe, t);
-            quarter_sweep<2>(w, s, z, maxq, uinv, Ud, qs, qe, t);
-            quarter_spill<2>(w, Ud, qe, t);
-            quarter_sweep<3>(w, s, z, maxq, uinv, Ud, qs, qe, t);
-            if (p.loss) {
-#pragma unroll
-                for (int c = 0; c < BLK; ++c) e2 = fma((double)w[c], (double)w[c], e2);
-            }
-            // Outputs go through shared memory so that each warp writes whole rows (coalesced).
-            // The U tile is no longer needed: its space stages the errors, 64 columns at a time.
-            qe[0][t] = s;                                // the quarter-error buffer is free too:
-            qe[1][t] = z;                                // it carries each row's grid to the writers
-            float* stg = reinterpret_cast<float*>(smem + UD_OFF);
-            const bool more = bb + 1 < nblk;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                row_bar();                               // Ud reads finished / previous half written out
-                if (more) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        *reinterpret_cast<float4*>(stg + t * STG + 4 * i) =
-                            make_float4(w[64 * h + 4 * i], w[64 * h + 4 * i + 1], w[64 * h + 4 * i + 2],
-                                        w[64 * h + 4 * i + 3]);
+            p.scales[((size_t)b * p.d_out + row) * ngroups + bb] = s;
+            p.zeros[((size_t)b * p.d_out + row) * ngroups + bb] = (uint8_t)z;
+            row_bar();                                   // Uq, uinv visible to every row thread
+            for (int q = 0; q < 4; ++q) {
+                float w[QW];
+                load_w32(p, wrow + cb + QW * q, w);
+                if (q > 0) {                             // the previous quarter's product reached this quarter
+                    if (!tc::mbar_wait_bounded(sdone, (nq - 1) & 1, abort_flag)) ok = false;
+                    tc::fence_after_sync();
+                    if (t == 0 && q < 3) load_sb(cb, q);
                 }
-                row_bar();
-                if (more) {    // errors for the later blocks' lazy updates, as tf32 hi + lo
-#pragma unroll 4
-                    for (int rr = 0; rr < 32; rr += 2) {
-                        const int r = warp * 32 + rr + (lane >> 4), c4 = (lane & 15) * 4;
-                        const float4 v = *reinterpret_cast<const float4*>(stg + r * STG + c4);
-                        const float hx = to_tf32(v.x), hy = to_tf32(v.y), hz = to_tf32(v.z), hw = to_tf32(v.w);
-                        const size_t o = ((size_t)b * p.d_out + r0 + r) * p.d_in + cb + 64 * h + c4;
-                        *reinterpret_cast<float4*>(p.Ehi + o) = make_float4(hx, hy, hz, hw);
-                        *reinterpret_cast<float4*>(p.Elo + o) =
-                            make_float4(to_tf32(v.x - hx), to_tf32(v.y - hy), to_tf32(v.z - hz), to_tf32(v.w - hw));
+                if (bb > 0 || q > 0) {
+                    uint32_t v[32];
+                    tc::tmem_ld_32x32b_x32(tmem + lane_base + acc * BLK + q * QW, v);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < QW; ++j) w[j] -= __uint_as_float(v[j]);
+                }
+                if (q == 3) {                            // last read of this accumulator
+                    tc::fence_before_sync();
+                    tc::mbar_arrive(tempty0 + 8 * acc);
+                }
+                uint32_t codes[QW / 4];
+                quarter_sweep(w, s, z, maxq, uinv + QW * q, Uq[q], codes);
+                // outputs of this quarter: codes (32 B) and w_hat (128 B) of this row
+                uint4* cdst = reinterpret_cast<uint4*>(p.codes + orow + QW * q);
+                cdst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                cdst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+                if (p.W_hat || p.loss) {
+                    float wo[QW];
+                    if (p.loss) load_w32(p, wrow + cb + QW * q, wo);
+#pragma unroll
+                    for (int c = 0; c < QW / 4; ++c) {
+                        float v[4];
+#pragma unroll
+                        for (int m = 0; m < 4; ++m)
+                            v[m] = __fmul_rn(s, __fsub_rn((float)((codes[c] >> (8 * m)) & 255u), z));
+                        if (p.W_hat)
+                            *reinterpret_cast<float4*>(p.W_hat + orow + QW * q + 4 * c) = make_float4(v[0], v[1], v[2], v[3]);
+                        if (p.loss) {
+#pragma unroll
+                            for (int m = 0; m < 4; ++m) {
+                                const double dv = (double)v[m] - (double)wo[4 * c + m];
+                                d2 = fma(dv, dv, d2);
+                            }
+                        }
                     }
                 }
-            }
-            if (more) {
-                fence_proxy_async_global();
-                tc::mbar_arrive(eready);
-            }
-            // codes, w_hat and |W_hat - W|^2 row by row: lane l owns columns 4l..4l+3
-#pragma unroll 2
-            for (int rr = 0; rr < 32; ++rr) {
-                const int r = warp * 32 + rr;
-                const size_t o = ((size_t)b * p.d_out + r0 + r) * p.d_in + cb + 4 * lane;
-                const uint32_t cw = *reinterpret_cast<const uint32_t*>(&qs[r][4 * lane]);
-                *reinterpret_cast<uint32_t*>(p.codes + o) = cw;
-                const float sr = qe[0][r], zr = qe[1][r];
-                float v[4];
-#pragma unroll
-                for (int m = 0; m < 4; ++m) v[m] = __fmul_rn(sr, __fsub_rn((float)((cw >> (8 * m)) & 255u), zr));
-                if (p.W_hat) *reinterpret_cast<float4*>(p.W_hat + o) = make_float4(v[0], v[1], v[2], v[3]);
                 if (p.loss) {
-                    float wv[4];
-                    if (p.w_f32) {
-                        const float4 f = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.W) + o);
-                        wv[0] = f.x; wv[1] = f.y; wv[2] = f.z; wv[3] = f.w;
-                    } else {
-                        const uint2 raw = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(p.W) + o);
-                        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
-                        const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
-                        wv[0] = f0.x; wv[1] = f0.y; wv[2] = f1.x; wv[3] = f1.y;
-                    }
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        const double dv = (double)v[m] - (double)wv[m];
-                        d2 = fma(dv, dv, d2);
+                    for (int j = 0; j < QW; ++j) e2 = fma((double)w[j], (double)w[j], e2);
+                }
+                if (q == 3 && !more) break;
+                // the quarter's errors as tf32 hi/lo, row t, 16-byte piece c at c ^ (t % 8); the buffer
+                // is free once the last quarter's whole product and its store have read it
+                if (q > 0 && !tc::mbar_wait_bounded(sdone2, (nq - 1) & 1, abort_flag)) ok = false;
+                if (t == 0) tc::bulk_wait_read<0>();
+                row_bar();
+                if (q == 3) load_uq(cb + BLK);           // every row is past its last use of Uq
+                uint8_t* sah = smem + SA_OFF + t * 128;
+                uint8_t* sal = sah + SA_BYTES;
+#pragma unroll
+                for (int c = 0; c < QW / 4; ++c) {
+                    const float h0 = to_tf32(w[4 * c]), h1 = to_tf32(w[4 * c + 1]), h2 = to_tf32(w[4 * c + 2]),
+                                h3 = to_tf32(w[4 * c + 3]);
+                    const int off = ((c ^ (t & 7)) << 4);
+                    *reinterpret_cast<float4*>(sah + off) = make_float4(h0, h1, h2, h3);
+                    *reinterpret_cast<float4*>(sal + off) =
+                        make_float4(to_tf32(w[4 * c] - h0), to_tf32(w[4 * c + 1] - h1), to_tf32(w[4 * c + 2] - h2),
+                                    to_tf32(w[4 * c + 3] - h3));
+                }
+                fence_proxy_async_smem();
+                if (q < 3) {
+                    tc::mbar_arrive(sreq);
+                    ++nq;
+                }
+                if (more) {
+                    row_bar();                           // every row's errors are in the buffer
+                    if (t == 0) {
+                        tc::tma_store_2d(&tmEhi, sa_hi, cb + QW * q, ey);
+                        tc::tma_store_2d(&tmElo, sa_lo, cb + QW * q, ey);
+                        tc::bulk_commit();
+                        if (q == 3) {
+                            tc::bulk_wait_all();
+                            fence_proxy_async_global();
+                            tc::mbar_arrive(eready);
+                        }
                     }
                 }
+            }
+            if (more) {   // this row's W for the next block into L1
+                const char* nxt = reinterpret_cast<const char*>(p.W) + (wrow + cb + BLK) * (p.w_f32 ? 4 : 2);
+                for (int o = 0; o < BLK * (p.w_f32 ? 4 : 2); o += 128)
+                    asm volatile("prefetch.global.L1 [%0];" ::"l"(nxt + o));
             }
         }
+        if (t == 0) tc::bulk_wait_all();
         if (p.loss) {
             double v = e2 - p.lambda[u] * d2;
 #pragma unroll
@@ -446,21 +534,21 @@ cudaError_t launch_quantize(cudaStream_t s, const float* U, int n_u, const void*
     float* Uhi = (float*)clha_carve(cur, (size_t)batch * d_in * d_in * sizeof(float));
     float* Ulo = (float*)clha_carve(cur, (size_t)batch * d_in * d_in * sizeof(float));
     cudaError_t e;
-    CUtensorMap tEhi, tElo, tUhi, tUlo;
+    CUtensorMap tEhi, tElo, tUhi, tUlo, tQhi, tQlo;
     if ((e = make_tmap_2d(&tEhi, Ehi, (uint64_t)batch * d_out, d_in, 4, R, KS)) != cudaSuccess) return e;
     if ((e = make_tmap_2d(&tElo, Elo, (uint64_t)batch * d_out, d_in, 4, R, KS)) != cudaSuccess) return e;
     if ((e = make_tmap_2d(&tUhi, Uhi, (uint64_t)n_u * d_in, d_in, 4, BLK, KS)) != cudaSuccess) return e;
     if ((e = make_tmap_2d(&tUlo, Ulo, (uint64_t)n_u * d_in, d_in, 4, BLK, KS)) != cudaSuccess) return e;
-    if (d_in > BLK) {
-        gptq_split_t<<<dim3(d_in / 32, d_in / 32, n_u), 256, 0, s>>>(U, d_in, Uhi, Ulo);
-        clha_note_launches(1);
-    }
+    if ((e = make_tmap_2d(&tQhi, Uhi, (uint64_t)n_u * d_in, d_in, 4, 32, QW)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d(&tQlo, Ulo, (uint64_t)n_u * d_in, d_in, 4, 32, QW)) != cudaSuccess) return e;
+    gptq_split_t<<<dim3(d_in / 32, d_in / 32, n_u), 256, 0, s>>>(U, d_in, Uhi, Ulo);
+    clha_note_launches(1);
     if ((e = cudaFuncSetAttribute(gptq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) != cudaSuccess)
         return e;
     if (loss && (e = cudaMemsetAsync(loss, 0, (size_t)batch * sizeof(double), s)) != cudaSuccess) return e;
-    GptqParams p{U, n_u, W, w_is_f32, d_out, d_in, bits, codes, scales, zeros, W_hat, Ehi, Elo, lambda, loss, err};
+    GptqParams p{U, n_u, W, w_is_f32, d_out, d_in, bits, codes, scales, zeros, W_hat, lambda, loss, err};
     dim3 grid(d_out / R, batch);
-    gptq_tc<<<grid, kThreads, SMEM_BYTES, s>>>(tEhi, tElo, tUhi, tUlo, p);
+    gptq_tc<<<grid, kThreads, SMEM_BYTES, s>>>(tEhi, tElo, tUhi, tUlo, tQhi, tQlo, p);
     clha_note_launches(1);
     return cudaGetLastError();
 }
