@@ -52,26 +52,36 @@ def alu_peaks(peaks):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+    """nvidia-smi clock / throttle-reason samples (every 20 ms, with timestamps); only those taken
+    inside the timed region's host-time window count."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
         self.path = None
+        self.window = None
 
     def start(self):
+        """Start sampling and wait (up to 5 s) until the first sample is written."""
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
+            t0 = time.time()
+            while time.time() - t0 < 5.0 and os.path.getsize(self.path) == 0:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
+
+    def mark(self, t_begin: float, t_end: float):
+        """Host-time window of the timed region."""
+        self.window = (t_begin, t_end)
 
     def stop(self):
         if self.proc is None:
@@ -82,25 +92,36 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.f.close()
-        mhz, mx, reasons = [], None, set()
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    mhz.append(float(parts[1]))
-                    mx = float(parts[2])
-                except ValueError:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                    rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+                except (ValueError, IndexError):
                     continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
         os.unlink(self.path)
-        if not mhz:
+        if not rows:
             return None
-        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(mhz)}
+        inside = rows
+        if self.window:
+            a, b = self.window
+            sel = [r for r in rows if a - 0.025 <= r[0] <= b + 0.025]
+            if sel:
+                inside = sel
+        reasons = set()
+        for r in inside:
+            for n, v in zip(names, r[3]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": inside[-1][2],
+                "reasons": sorted(reasons), "samples": len(inside),
+                "window": "timed region" if inside is not rows else "whole run (no sample inside the timed region)"}
 
 
 def dist_setup(backend: str | None = None):
@@ -281,6 +302,7 @@ def run_ours(args, world, rank, local):
     launches0 = L.clha_kernel_launches(ctx)
     ev = []
     stream = ctx.stream
+    t_begin = time.time()
     for _ in range(args.steps):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -289,6 +311,7 @@ def run_ours(args, world, rank, local):
         b.record(stream)
         ev.append((a, b))
     torch.cuda.synchronize()
+    clocks.mark(t_begin, time.time())
     launches = L.clha_kernel_launches(ctx) - launches0
     barrier(world)
     step_ms = [a.elapsed_time(b) for a, b in ev]
