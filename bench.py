@@ -6,7 +6,7 @@ the expert inputs -> expert activation -> Hessians of the down-projection inputs
 weightings (routing-frequency and equal) aggregate -> factor -> GPTQ of gate, up and down -> loss.
 Inputs are synthetic (seeded), resident in HBM; L2 is flushed (512 MB write) before every timed step.
 
-  python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+  python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference] [--parallel replicas|tokens]
 
 Kernel-level workloads (one JSON line per shape; used for the profiles and the roofline tables):
   python bench.py --workload act --shape 18432x1024x512 ...   expert activation, dense bf16 X [n, d_model]
@@ -15,7 +15,9 @@ Kernel-level workloads (one JSON line per shape; used for the profiles and the r
   python bench.py --workload factor --shape 32x1024 ...       inverse-Cholesky factor of [batch, d, d]
 
 With N > 1 (torchrun, one process per GPU) every rank calibrates its own independent layer pair:
-weak scaling, no data-path collective; the step time is the max over ranks.
+weak scaling, no data-path collective; the step time is the max over ranks. With --parallel tokens
+the ranks share one layer pair instead: each collects its share of the tokens, one NCCL all-reduce
+sums the Hessian accumulators, and each quantizes its own range of experts (strong scaling).
 """
 from __future__ import annotations
 
@@ -269,24 +271,46 @@ def run_ours(args, world, rank, local):
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    wl, X, lg, routed = make_inputs(rank)
+    sharded = args.parallel == "tokens"
+    # replicas: every rank calibrates its own pair; tokens: one pair, tokens and experts split over ranks
+    wl, X, lg, routed = make_inputs(0 if sharded else rank)
     s = wl.spec
     ctx = L.Context(local)
     timer = PhaseTimer(ctx.stream)
     w = stack_weights((routed, []), dev)
+    modes = s.alpha_modes
+    if sharded:
+        from post_quantization_expert_b200 import sharded as SH
+        t0, t1 = SH.token_range(s.tokens[0], rank, world)
+        X, lg = [x[t0:t1].contiguous() for x in X], [l[t0:t1].contiguous() for l in lg]
+        sh = SH.ShardedMoECalibration(ctx, rank, world, 2, t1 - t0, s.E, s.k, s.d_model, s.d_ff,
+                                      bits_routed=s.bits_routed, bits_shared=s.bits_shared, damp_frac=s.damp_frac,
+                                      timer=timer, modes=modes)
+        cal, qcal, wq = sh.collector, sh.quantizer, sh.local_weights(w)
+        cols_per_step = cal.columns() * len(modes) / world      # the pair's columns, per rank on average
+    else:
+        cal = qcal = MoECalibration(ctx, 2, max(s.tokens), s.E, s.k, s.d_model, s.d_ff, 0, 0, s.bits_routed,
+                                    s.bits_shared, s.damp_frac, timer=timer, modes=modes)
+        wq = w
+        cols_per_step = cal.columns() * len(modes)
     Xd = [x.to(dev) for x in X]
     Ld = [l.to(dev) for l in lg]
-    modes = s.alpha_modes
-    cal = MoECalibration(ctx, 2, max(s.tokens), s.E, s.k, s.d_model, s.d_ff, 0, 0, s.bits_routed, s.bits_shared,
-                         s.damp_frac, timer=timer, modes=modes)
-    cols_per_step = cal.columns() * len(modes)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
 
-    def step():
+    def calibrate():
         cal.reset()
         for l in range(2):
             cal.collect(l, Xd[l], Ld[l], w)
-        cal.quantize(w, modes)
+        if sharded:
+            if world > 1:
+                with timer.span("allreduce"):
+                    SH.dist_reduce(sh.reduce_tensors())
+            sh.quantize(wq, modes)
+        else:
+            cal.quantize(w, modes)
+
+    def step():
+        calibrate()
 
     timer.enabled = False
     for _ in range(args.warmup):
@@ -323,7 +347,7 @@ def run_ours(args, world, rank, local):
     pin = lambda t: t.pin_memory()
     hX, hL = [pin(x) for x in X], [pin(l) for l in lg]
     hW = [pin(w.Wgu.cpu()), pin(w.Wd.cpu())]
-    outs = {m: [cal.res[m].qgu, cal.res[m].qd] for m in modes}
+    outs = {m: [qcal.res[m].qgu, qcal.res[m].qd] for m in modes}
     hout = {m: [(pin(torch.empty_like(q.codes, device="cpu")), pin(torch.empty_like(q.scales, device="cpu")),
                  pin(torch.empty_like(q.zeros, device="cpu"))) for q in outs[m]] for m in modes}
     h2d = sum(t.numel() * t.element_size() for t in hX + hL + hW)
@@ -334,10 +358,10 @@ def run_ours(args, world, rank, local):
         with torch.cuda.stream(stream):
             for d_, h_ in zip(Xd + Ld + [w.Wgu, w.Wd], hX + hL + hW):
                 d_.copy_(h_, non_blocking=True)
-            cal.reset()
-            for l in range(2):
-                cal.collect(l, Xd[l], Ld[l], w)
-            cal.quantize(w, modes)
+            if sharded:
+                wq.Wgu.copy_(torch.cat([w.Wgu[sh.e0:sh.e1], w.Wgu[s.E + sh.e0:s.E + sh.e1]]))
+                wq.Wd.copy_(w.Wd[sh.e0:sh.e1])
+            calibrate()
             for m in modes:
                 for q, (hc, hs, hz) in zip(outs[m], hout[m]):
                     hc.copy_(q.codes, non_blocking=True)
@@ -366,12 +390,13 @@ def run_ours(args, world, rank, local):
     counts = [cal.counts[l].cpu().numpy().astype(np.int64) for l in range(2)]
     dm, dff, E = s.d_model, s.d_ff, s.E
     hess_flops = sum(int(c.sum()) * (dm * (dm + 1) + dff * (dff + 1)) for c in counts)
-    mats = [(dff, dm)] * (2 * E) + [(dm, dff)] * E          # gate, up, down per weighting
+    Eq = (sh.e1 - sh.e0) if sharded else E                  # experts this rank quantizes
+    mats = [(dff, dm)] * (2 * Eq) + [(dm, dff)] * Eq        # gate, up, down per weighting
     gptq_flops = len(modes) * sum(o * i * i for o, i in mats)
     loss_flops = len(modes) * sum(2 * o * i * i for o, i in mats)
-    factor_flops = len(modes) * E * (2 * dm ** 3 // 3 + 2 * dff ** 3 // 3)
+    factor_flops = len(modes) * Eq * (2 * dm ** 3 // 3 + 2 * dff ** 3 // 3)
     act_flops = sum(int(c.sum()) * 4 * dm * dff for c in counts)
-    agg_bytes = len(modes) * E * sum(2 * (d * (d + 32) // 2) * 4 + 2 * d * d * 4 for d in (dm, dff))
+    agg_bytes = len(modes) * Eq * sum(2 * (d * (d + 32) // 2) * 4 + 2 * d * d * 4 for d in (dm, dff))
     peaks, src = load_peaks()
     alu = alu_peaks(peaks)
     sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
@@ -414,12 +439,14 @@ def run_ours(args, world, rank, local):
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "columns/s", "n_gpus": world, "steps": K,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong" if sharded else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": s.name, "global_batch": world * sum(s.tokens), "tokens_per_layer": s.tokens[0],
                        "E": E, "top_k": s.k, "d_model": dm, "d_ff": dff, "bits": s.bits_routed,
                        "weightings": list(modes), "columns_per_step_per_gpu": cols_per_step,
-                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "parallelism": (f"tokens{world}+experts{world} (one NCCL all-reduce of S)" if sharded
+                                       else f"replicas{world}") if world > 1 else "single",
                        "l2": "flushed (512 MB write) before every timed step"},
             "hessian_tflops": hess_tflops,
             "hessian_frac_of_bf16_peak": hess_tflops / sustained,
@@ -520,6 +547,10 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--parallel", choices=("replicas", "tokens"), default="replicas",
+                    help="replicas (default): each rank calibrates its own layer pair (weak scaling); tokens: "
+                         "one pair, its tokens sharded over the ranks with one all-reduce of the Hessian sums, "
+                         "its experts quantized in parallel (strong scaling)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     ap.add_argument("--workload", choices=("moe", "act", "hessian", "gptq", "factor"), default="moe",
                     help="moe: the end-to-end calibration step (default); others: one kernel family")
