@@ -13,6 +13,7 @@ Kernel-level workloads (one JSON line per shape; used for the profiles and the r
   python bench.py --workload hessian --shape 65536x4096 ...   Gram accumulation of dense bf16 X [n, d]
   python bench.py --workload gptq --shape 32x512x1024 ...     GPTQ of [batch, d_out, d_in] bf16 weights
   python bench.py --workload factor --shape 32x1024 ...       inverse-Cholesky factor of [batch, d, d]
+  python bench.py --workload epmq --shape 8x4096x4096 ...     E-PMQ target W* = R H^-1 of K source experts
 
 With N > 1 (torchrun, one process per GPU) every rank calibrates its own independent layer pair:
 weak scaling, no data-path collective; the step time is the max over ranks. With --parallel tokens
@@ -487,6 +488,26 @@ def run_kernel(args):
             fn = lambda: L.clha_expert_act(ctx, X, n, dm, None, 1, Wg, Wu, dff, hbuf)
             work, unit, bound, peak = 4 * n * dm * dff / 1e12, "TFLOP/s", "alu", alu["fp32_tflops"]
             kname = "expert_act_simt"
+        elif args.workload == "epmq":
+            Ksrc, d_out, d = dims
+            Xs = torch.randn((Ksrc, 2 * d, d), device="cuda", generator=g).to(torch.bfloat16)
+            acc = L.Accum(ctx, d, Ksrc, 1)
+            for i in range(Ksrc):
+                L.clha_collect(ctx, acc, i, Xs[i], 2 * d, d)
+            del Xs
+            Hc = torch.empty((1, d, d), device="cuda")
+            Hd = torch.empty_like(Hc)
+            U = torch.empty_like(Hc)
+            lam = torch.empty(1, dtype=torch.float64, device="cuda")
+            L.clha_aggregate(ctx, acc, 0, 1, L.ALPHA_SUM, None, 0.01, Hc, Hd, lambda_dev=lam)
+            L.clha_factor(ctx, Hd, 1, d, U)
+            W_src = (0.02 * torch.randn((Ksrc, d_out, d), device="cuda", generator=g)).to(torch.bfloat16)
+            W_m = W_src.float().mean(0).to(torch.bfloat16)
+            Wt = torch.empty((d_out, d), device="cuda")
+            fn = lambda: L.clha_epmq_target(ctx, acc, 0, W_src, W_m, d_out, U, lam, Wt)
+            work = (2 * Ksrc * d_out * d * d + 2 * d ** 3 + 2 * d_out * d * d) / 1e12
+            unit, bound, peak = "TFLOP/s", "alu", alu["fp64_tflops"]
+            kname = "epmq_gemm x3 (fp64, mma.sync m8n8k4 f64)"
         elif args.workload == "hessian":
             n, d = dims
             X = torch.randn((n, d), device="cuda", generator=g).to(torch.bfloat16)
@@ -552,7 +573,7 @@ def main():
                          "one pair, its tokens sharded over the ranks with one all-reduce of the Hessian sums, "
                          "its experts quantized in parallel (strong scaling)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
-    ap.add_argument("--workload", choices=("moe", "act", "hessian", "gptq", "factor"), default="moe",
+    ap.add_argument("--workload", choices=("moe", "act", "hessian", "gptq", "factor", "epmq"), default="moe",
                     help="moe: the end-to-end calibration step (default); others: one kernel family")
     ap.add_argument("--shape", nargs="+", default=[], help="kernel workload shapes, e.g. 65536x4096")
     args = ap.parse_args()

@@ -59,7 +59,9 @@ typedef enum { CLHA_BF16 = 0, CLHA_F32 = 1 } clha_dtype;
 typedef enum {
     CLHA_ALPHA_ROUTING = 0,   /* alpha_i = n_i / sum_j n_j           (CLHA page §2.2 (2), "rt") */
     CLHA_ALPHA_EQUAL = 1,     /* alpha_i = 1 / n_layers              (CLHA page §2.2 (2), "eq") */
-    CLHA_ALPHA_EXPLICIT = 2   /* alpha from the caller; (1, 0) is per-layer calibration on layer 0 */
+    CLHA_ALPHA_EXPLICIT = 2,  /* alpha from the caller; (1, 0) is per-layer calibration on layer 0 */
+    CLHA_ALPHA_SUM = 3        /* alpha_i = n_i / 2, so H_comb = sum_i S_i: the unnormalised Gram sum
+                                 of the E-PMQ statistics (the E-PMQ page, section 2) */
 } clha_alpha_mode;
 
 /* GPTQ parameters: bits in 2..8, group = 128 (grid per 128 input columns), block = 128 (lazy-update
@@ -135,6 +137,9 @@ CLHA_API clha_status clha_expert_act(clha_ctx* ctx, const void* X, int64_t rows,
                             const int64_t* seg, int E, const void* Wg, const void* Wu, int d_ff,
                             void* h);
 
+/* Largest number of layers (or source experts) one accumulator holds. */
+#define CLHA_MAX_LAYERS 32
+
 /* Accumulator of per-(layer, slot) Gram matrices S = sum x x^T (float32 [d, d], upper triangle
  * authoritative, lower triangle may hold partial values) and token counts (int64). A slot is one
  * expert (or one dense weight). Layer-aware by construction (CLHA page §2.4): every collect names
@@ -196,6 +201,21 @@ typedef struct clha_factor_group {
     int d;                   /* multiple of 128 */
 } clha_factor_group;
 CLHA_API clha_status clha_factor_groups(clha_ctx* ctx, int n_groups, const clha_factor_group* groups);
+
+/* E-PMQ's quantization target (the E-PMQ page, section 2: expert-driven output targets, anchoring to
+ * the merged weights, and the solver's statistics H = sum_i H_i + lambda I, R = sum_i W_i H_i +
+ * lambda W_m). The K = n_layers "layers" of `acc` are the K source experts: S_i = acc's Gram of
+ * layer i in slot `slot` (H_i = S_i, upper triangle read). With U the clha_factor of the damped
+ * aggregate of that slot in mode CLHA_ALPHA_SUM (H_comb = sum_i S_i, H_damped = H) and lambda its
+ * damping (lambda_dev as written by clha_aggregate), computes in float64
+ *   W_target = (lambda W_m + sum_i W_i S_i) U^T U  =  R H^-1
+ * and writes it as float32 [d_out, d]; clha_quantize of W_target with U then runs E-PMQ's GPTQ step.
+ * W_src: device [K, d_out, d] (the source experts' weights), W_merged: device [d_out, d], both of
+ * `dtype`; U: device float32 [d, d]; lambda_dev: device double. d = acc's d; d_out a multiple of 64.
+ * Device pointers are the caller's. */
+CLHA_API clha_status clha_epmq_target(clha_ctx* ctx, const clha_accum* acc, int slot, const void* W_src,
+                                      const void* W_merged, clha_dtype dtype, int d_out, const float* U,
+                                      const double* lambda_dev, float* W_target);
 
 /* GPTQ (CLHA page §2.2 (3)): column-sequential quantization of `batch` weights W [batch, d_out, d_in]
  * (bf16 or f32) in natural column order, with lazy updates over 128-column blocks. U holds n_u

@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libclha.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_NOT_PD, ERR_NONFINITE, ERR_EMPTY, ERR_OOM, ERR_CUDA, ERR_TIMEOUT = range(9)
 STATUS_NAMES = ["OK", "INVALID_ARG", "UNSUPPORTED_SHAPE", "NOT_PD", "NONFINITE", "EMPTY", "OOM", "CUDA", "TIMEOUT"]
 BF16, F32 = 0, 1
-ALPHA_ROUTING, ALPHA_EQUAL, ALPHA_EXPLICIT = 0, 1, 2
+ALPHA_ROUTING, ALPHA_EQUAL, ALPHA_EXPLICIT, ALPHA_SUM = 0, 1, 2, 3
 
 # every symbol include/clha.h declares
 SYMBOLS = [
@@ -29,7 +29,7 @@ SYMBOLS = [
     "clha_route_topk", "clha_packed_rows", "clha_gather", "clha_gather_noalloc", "clha_expert_act",
     "clha_accum_create", "clha_accum_destroy", "clha_accum_zero", "clha_accum_buffers",
     "clha_accum_export", "clha_accum_import", "clha_collect",
-    "clha_aggregate", "clha_factor", "clha_factor_groups", "clha_quantize", "clha_loss",
+    "clha_aggregate", "clha_factor", "clha_factor_groups", "clha_epmq_target", "clha_quantize", "clha_loss",
 ]
 FACTOR_MAX_GROUPS = 4
 
@@ -84,6 +84,7 @@ def load(path: str = LIB_PATH):
         "clha_aggregate": (i32, [vp, vp, i32, i32, i32, vp, f64, vp, vp, vp, vp, vp]),
         "clha_factor": (i32, [vp, vp, i32, i32, vp]),
         "clha_factor_groups": (i32, [vp, i32, vp]),
+        "clha_epmq_target": (i32, [vp, vp, i32, vp, vp, i32, i32, vp, vp, vp]),
         "clha_quantize": (i32, [vp, vp, i32, vp, i32, i32, i32, i32, C.POINTER(QuantParams), vp, vp, vp, vp, vp,
                                 vp]),
         "clha_loss": (i32, [vp, vp, i32, vp, vp, i32, i32, i32, i32, vp]),
@@ -270,6 +271,12 @@ def clha_factor_groups(ctx: Context, groups):
     """groups: sequence of (H_damped, batch, d, U), at most FACTOR_MAX_GROUPS; one graph launch."""
     arr = (FactorGroup * len(groups))(*[FactorGroup(_p(H), _p(U), b, d) for H, b, d, U in groups])
     ctx._check(load().clha_factor_groups(ctx.handle, len(groups), C.cast(arr, C.c_void_p)))
+
+
+def clha_epmq_target(ctx: Context, acc: "Accum", slot: int, W_src, W_merged, d_out: int, U, lambda_dev, W_target):
+    """W_target = (lambda W_m + sum_i W_i S_i) U^T U for the accumulator's K source experts."""
+    ctx._check(load().clha_epmq_target(ctx.handle, acc.handle, slot, _p(W_src), _p(W_merged), _dtype(W_src), d_out,
+                                       _p(U), _p(lambda_dev), _p(W_target)))
 
 
 def clha_quantize(ctx: Context, U, n_u: int, W, batch: int, d_out: int, d_in: int, bits: int, codes, scales,

@@ -1,6 +1,7 @@
 // Phase 2 of CLHA (the CLHA page, §2.1 Proposition 1 and §2.2 (2)): H_comb = sum_i alpha_i H_i with
 // H_i = (2 / n_i) S_i, routing-frequency (alpha_i = n_i / sum n), equal (1/L) or explicit weights,
-// then GPTQ damping H_d = H_comb + lambda I, lambda = damp_frac * mean(diag H_comb).
+// or the plain Gram sum (alpha_i = n_i / 2, H_comb = sum S_i: the E-PMQ statistics), then GPTQ
+// damping H_d = H_comb + lambda I, lambda = damp_frac * mean(diag H_comb).
 //
 // Two kernels per call, both HBM-bound:
 //   agg_scalars  one block per slot: alpha (float64), lambda from the diagonals (float64 reduction),
@@ -22,8 +23,8 @@ __global__ void __launch_bounds__(256) agg_scalars(const float* __restrict__ S, 
                                                    double* __restrict__ d_lambda, int* err) {
     const int sl = blockIdx.x;
     const int slot = slot0 + sl;
-    __shared__ double alpha[16];
-    __shared__ int64_t cnt[16];
+    __shared__ double alpha[CLHA_MAX_LAYERS];
+    __shared__ int64_t cnt[CLHA_MAX_LAYERS];
     __shared__ double red[256];
     if (threadIdx.x == 0) {
         int64_t tot = 0;
@@ -35,6 +36,7 @@ __global__ void __launch_bounds__(256) agg_scalars(const float* __restrict__ S, 
             double al;
             if (a.mode == CLHA_ALPHA_ROUTING) al = tot > 0 ? (double)cnt[l] / (double)tot : 0.0;
             else if (a.mode == CLHA_ALPHA_EQUAL) al = 1.0 / L;
+            else if (a.mode == CLHA_ALPHA_SUM) al = (double)cnt[l] / 2.0;
             else al = a.alpha[l];
             alpha[l] = al;
             d_alpha[(size_t)sl * L + l] = al;
@@ -76,7 +78,7 @@ __global__ void __launch_bounds__(256) agg_combine(const float* __restrict__ S, 
     while (t >= nt - bi) { t -= nt - bi; ++bi; }
     const int bj = bi + t;  // bi <= bj
     __shared__ float tile[32][33];
-    __shared__ float coef[16];
+    __shared__ float coef[CLHA_MAX_LAYERS];
     if (threadIdx.x < L) {
         int64_t n = counts[(size_t)threadIdx.x * n_slots_total + slot];
         coef[threadIdx.x] = n > 0 ? (float)(d_alpha[(size_t)sl * L + threadIdx.x] * 2.0 / (double)n) : 0.f;

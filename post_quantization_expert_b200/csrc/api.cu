@@ -237,8 +237,8 @@ extern "C" clha_status clha_accum_create(clha_ctx* ctx, int d, int n_layers, int
     CHECK_CTX(ctx);
     REQUIRE(out, CLHA_ERR_INVALID_ARG, "clha_accum_create: null out");
     *out = nullptr;
-    REQUIRE(d > 0 && n_layers >= 1 && n_layers <= 16 && n_slots >= 1, CLHA_ERR_INVALID_ARG,
-            "clha_accum_create: need d > 0, 1 <= n_layers <= 16, n_slots >= 1");
+    REQUIRE(d > 0 && n_layers >= 1 && n_layers <= CLHA_MAX_LAYERS && n_slots >= 1, CLHA_ERR_INVALID_ARG,
+            "clha_accum_create: need d > 0, 1 <= n_layers <= %d, n_slots >= 1", CLHA_MAX_LAYERS);
     REQUIRE(d % 128 == 0, CLHA_ERR_UNSUPPORTED_SHAPE, "clha_accum_create: d=%d is not a multiple of 128", d);
     SET_DEVICE(ctx);
     clha_accum* acc = new (std::nothrow) clha_accum();
@@ -347,7 +347,8 @@ extern "C" clha_status clha_aggregate(clha_ctx* ctx, const clha_accum* acc, int 
     REQUIRE(acc && H_damped, CLHA_ERR_INVALID_ARG, "clha_aggregate: null pointer");
     REQUIRE(n_slots >= 1 && slot0 >= 0 && slot0 + n_slots <= acc->n_slots, CLHA_ERR_INVALID_ARG,
             "clha_aggregate: slots outside the accumulator");
-    REQUIRE(mode == CLHA_ALPHA_ROUTING || mode == CLHA_ALPHA_EQUAL || mode == CLHA_ALPHA_EXPLICIT,
+    REQUIRE(mode == CLHA_ALPHA_ROUTING || mode == CLHA_ALPHA_EQUAL || mode == CLHA_ALPHA_EXPLICIT ||
+                mode == CLHA_ALPHA_SUM,
             CLHA_ERR_INVALID_ARG, "clha_aggregate: unknown alpha mode");
     REQUIRE(mode != CLHA_ALPHA_EXPLICIT || alpha_in, CLHA_ERR_INVALID_ARG, "clha_aggregate: explicit alpha needs alpha_in");
     REQUIRE(damp_frac > 0.0 && damp_frac == damp_frac, CLHA_ERR_INVALID_ARG, "clha_aggregate: damp_frac must be > 0");
@@ -412,6 +413,30 @@ extern "C" clha_status clha_factor_groups(clha_ctx* ctx, int n_groups, const clh
 extern "C" clha_status clha_factor(clha_ctx* ctx, const float* H_damped, int batch, int d, float* U) {
     clha_factor_group g{H_damped, U, batch, d};
     return clha_factor_groups(ctx, 1, &g);
+}
+
+extern "C" clha_status clha_epmq_target(clha_ctx* ctx, const clha_accum* acc, int slot, const void* W_src,
+                                        const void* W_merged, clha_dtype dtype, int d_out, const float* U,
+                                        const double* lambda_dev, float* W_target) {
+    CHECK_CTX(ctx);
+    REQUIRE(acc && W_src && W_merged && U && lambda_dev && W_target, CLHA_ERR_INVALID_ARG,
+            "clha_epmq_target: null pointer");
+    REQUIRE(dtype == CLHA_BF16 || dtype == CLHA_F32, CLHA_ERR_INVALID_ARG, "clha_epmq_target: unknown dtype");
+    REQUIRE(slot >= 0 && slot < acc->n_slots, CLHA_ERR_INVALID_ARG, "clha_epmq_target: slot %d outside 0..%d", slot,
+            acc->n_slots - 1);
+    REQUIRE(d_out > 0 && d_out % 64 == 0, CLHA_ERR_UNSUPPORTED_SHAPE,
+            "clha_epmq_target: d_out=%d is not a positive multiple of 64", d_out);
+    SET_DEVICE(ctx);
+    LaunchScope launch_scope(ctx);
+    void* ws = nullptr;
+    const int d = acc->d;
+    clha_status st = clha_workspace(ctx, epmq_workspace_bytes(d_out, d), &ws);
+    if (st) return st;
+    const int64_t dd = (int64_t)d * d;
+    CUDA_TRY(launch_epmq_target(ctx->stream, acc->S + (size_t)slot * dd, (int64_t)acc->n_slots * dd, acc->n_layers,
+                                W_src, dtype == CLHA_BF16, W_merged, d_out, d, U, lambda_dev, W_target, ws),
+             "clha_epmq_target");
+    return CLHA_OK;
 }
 
 extern "C" clha_status clha_quantize(clha_ctx* ctx, const float* U, int n_u, const void* W, clha_dtype dtype,

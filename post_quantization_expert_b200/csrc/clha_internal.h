@@ -89,7 +89,7 @@ cudaError_t launch_collect_f32(cudaStream_t s, const float* X, int64_t rows, int
 struct clha_alpha_args {
     int mode;             // clha_alpha_mode
     int n_layers;
-    double alpha[16];     // explicit weights
+    double alpha[CLHA_MAX_LAYERS];   // explicit weights
 };
 cudaError_t launch_aggregate(cudaStream_t s, const float* S, const int64_t* counts, int d,
                              int n_layers, int n_slots_total, int slot0, int n_slots,
@@ -102,6 +102,10 @@ struct FactorGroup {
 };
 size_t factor_workspace_bytes(const FactorGroup* groups, int n);
 cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups, int n, void* ws, int* err);
+size_t epmq_workspace_bytes(int d_out, int d);
+cudaError_t launch_epmq_target(cudaStream_t s, const float* S_slot, int64_t layer_stride, int K, const void* W_src,
+                               int w_bf16, const void* W_m, int d_out, int d, const float* U, const double* lambda,
+                               float* W_target, void* ws);
 size_t quantize_workspace_bytes(int batch, int d_out, int d_in);
 cudaError_t launch_quantize(cudaStream_t s, const float* U, int n_u, const void* W, int w_is_f32,
                             int batch, int d_out, int d_in, int bits, uint8_t* codes, float* scales,

@@ -17,7 +17,7 @@ import torch
 
 from . import clha as L
 
-MODES = {"rt": L.ALPHA_ROUTING, "eq": L.ALPHA_EQUAL, "explicit": L.ALPHA_EXPLICIT}
+MODES = {"rt": L.ALPHA_ROUTING, "eq": L.ALPHA_EQUAL, "explicit": L.ALPHA_EXPLICIT, "sum": L.ALPHA_SUM}
 
 
 class PhaseTimer:
@@ -372,3 +372,38 @@ def stack_weights(wl, device) -> MoEWeights:
     if shared:
         return MoEWeights(gu(routed), dn(routed), gu(shared), dn(shared))
     return MoEWeights(gu(routed), dn(routed))
+
+
+class EPMQCalibration:
+    """E-PMQ of one merged linear layer (the E-PMQ page, section 2): the K source experts' calibration
+    activations are collected as the K layers of one accumulator slot; quantize() forms
+    H = sum_i S_i + lambda I (aggregation in the plain-sum weighting), factors it, computes the target
+    W* = (lambda W_m + sum_i W_i S_i) H^-1 and runs GPTQ of W* under H."""
+
+    def __init__(self, ctx: L.Context, K: int, d_out: int, d: int, bits: int, damp_frac: float = 0.01):
+        self.ctx, self.K, self.d_out, self.d, self.bits, self.damp = ctx, K, d_out, d, bits, damp_frac
+        dev = torch.device("cuda", ctx.device)
+        self.acc = L.Accum(ctx, d, K, 1)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.H = torch.empty((1, d, d), **f32)       # sum_i S_i (undamped)
+        self.H_d = torch.empty((1, d, d), **f32)     # + lambda I
+        self.U = torch.empty((1, d, d), **f32)
+        self.lam = torch.empty(1, dtype=torch.float64, device=dev)
+        self.W_target = torch.empty((d_out, d), **f32)
+        self.q = _quant_buffers(1, d_out, d, dev)
+
+    def collect(self, i: int, X_i: torch.Tensor):
+        """Activations of source expert i's calibration subset, [n_i, d] (bf16 or f32)."""
+        L.clha_collect(self.ctx, self.acc, i, X_i, X_i.shape[0], self.d)
+
+    def quantize(self, W_src: torch.Tensor, W_m: torch.Tensor):
+        """W_src [K, d_out, d], W_m [d_out, d] (same dtype). Results in self.q (codes, scales, zeros,
+        W_hat) and self.W_target."""
+        ctx = self.ctx
+        L.clha_aggregate(ctx, self.acc, 0, 1, L.ALPHA_SUM, None, self.damp, self.H, self.H_d, lambda_dev=self.lam)
+        L.clha_factor(ctx, self.H_d, 1, self.d, self.U)
+        L.clha_epmq_target(ctx, self.acc, 0, W_src, W_m, self.d_out, self.U, self.lam, self.W_target)
+        q = self.q
+        L.clha_quantize(ctx, self.U, 1, self.W_target, 1, self.d_out, self.d, self.bits, q.codes, q.scales, q.zeros,
+                        q.W_hat)
+        return q
