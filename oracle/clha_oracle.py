@@ -33,6 +33,8 @@ Readings where the pages are silent (each also listed in the design notes):
   * columns are quantized in natural order (no activation reordering).
   * a layer with no tokens contributes a zero Hessian; an expert with no tokens in any layer is an
     error (there is nothing to calibrate on).
+  * deployable codes are packed per row as one little-endian bit stream of 32-bit words, code j at
+    bits [b*j, b*j + b) (the pages give no layout); W_hat = s (q - z) per group in float32.
 """
 from __future__ import annotations
 
@@ -42,6 +44,7 @@ __all__ = [
     "route_topk", "expert_tokens", "gram", "hessian", "bf16_round", "silu", "ffn_act",
     "aggregate", "factor", "grid_fp32", "quantize_fp32", "gptq", "loss",
     "calibrate_dense", "calibrate_moe_group",
+    "pack_codes", "unpack_codes", "dequantize", "dequant_matmul",
 ]
 
 
@@ -277,3 +280,53 @@ def calibrate_moe_group(X_list, logits_list, k: int, routed, shared=(), experts=
         res["h"] = he
         out["experts"][key] = res
     return out
+
+
+# ------------------------------------------------------------------------------ deployable codes
+def pack_codes(codes, bits: int):
+    """Codes uint8 [rows, d_in] (values < 2^bits) -> uint32 [rows, d_in * bits / 32]: each row's codes
+    as one little-endian bit stream, code j at bits [bits*j, bits*j + bits) (a code may straddle two
+    words). The layout the deployable weights use; nothing in the pages fixes it."""
+    codes = np.asarray(codes, dtype=np.uint64)
+    rows, d_in = codes.shape
+    if (d_in * bits) % 32:
+        raise ValueError("d_in * bits must be a multiple of 32")
+    words = np.zeros((rows, d_in * bits // 32), dtype=np.uint64)
+    for j in range(d_in):
+        bit = bits * j
+        w, off = divmod(bit, 32)
+        words[:, w] |= (codes[:, j] << np.uint64(off)) & np.uint64(0xFFFFFFFF)
+        if off + bits > 32:
+            words[:, w + 1] |= codes[:, j] >> np.uint64(32 - off)
+    return words.astype(np.uint32)
+
+
+def unpack_codes(packed, bits: int, d_in: int):
+    """Inverse of pack_codes."""
+    packed = np.asarray(packed, dtype=np.uint64)
+    rows = packed.shape[0]
+    out = np.zeros((rows, d_in), dtype=np.uint8)
+    mask = np.uint64((1 << bits) - 1)
+    for j in range(d_in):
+        bit = bits * j
+        w, off = divmod(bit, 32)
+        v = packed[:, w] >> np.uint64(off)
+        if off + bits > 32:
+            v |= packed[:, w + 1] << np.uint64(32 - off)
+        out[:, j] = (v & mask).astype(np.uint8)
+    return out
+
+
+def dequantize(codes, scales, zeros, group: int = 128):
+    """W_hat = s (q - z) per group, in float32 (the same float32 operations GPTQ's W_hat uses)."""
+    codes = np.asarray(codes)
+    s = np.repeat(np.asarray(scales, np.float32), group, axis=1)
+    z = np.repeat(np.asarray(zeros, np.float32), group, axis=1)
+    return (s * (codes.astype(np.float32) - z)).astype(np.float32)
+
+
+def dequant_matmul(X, packed, scales, zeros, bits: int, group: int = 128):
+    """Y = X W_hat^T in float64 with W_hat decoded from the packed codes: the deployable layer's output."""
+    d_in = np.asarray(X).shape[1]
+    W_hat = dequantize(unpack_codes(packed, bits, d_in), scales, zeros, group)
+    return np.asarray(X, dtype=np.float64) @ W_hat.astype(np.float64).T

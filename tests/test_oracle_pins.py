@@ -360,3 +360,46 @@ def test_silu_and_ffn_act():
             want = g / (1 + np.exp(-g)) * u
             assert abs(h[t, f] - want) <= 2.0 ** -8 * abs(want) + 1e-300
             assert O.bf16_round(np.array([h[t, f]]))[0] == h[t, f]
+
+
+# ------------------------------------------------------------------------------ deployable codes
+def _golden_packed(golden_dir):
+    rows = []
+    with open(f"{golden_dir}/packed_codes_examples.txt") as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            b, codes, words = [p.strip() for p in line.split("|")]
+            rows.append((int(b), [int(c) for c in codes.split(",")], [int(w, 16) for w in words.split(",")]))
+    return rows
+
+
+def test_pack_codes_matches_hand_worked_words(golden_dir):
+    cases = _golden_packed(golden_dir)
+    assert len(cases) == 4
+    for bits, codes, words in cases:
+        got = O.pack_codes(np.array([codes], np.uint8), bits)
+        assert got.tolist() == [words], (bits, [hex(w) for w in got[0]])
+        np.testing.assert_array_equal(O.unpack_codes(got, bits, len(codes))[0], codes)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 7, 8])
+def test_pack_roundtrip(bits):
+    g = np.random.default_rng(bits)
+    codes = g.integers(0, 2 ** bits, size=(5, 256), dtype=np.uint8)
+    packed = O.pack_codes(codes, bits)
+    assert packed.shape == (5, 256 * bits // 32)
+    np.testing.assert_array_equal(O.unpack_codes(packed, bits, 256), codes)
+
+
+def test_dequantized_codes_are_gptq_w_hat_and_the_layer_output():
+    g = np.random.default_rng(3)
+    W = g.normal(0, 0.02, (8, 256))
+    A = g.normal(0, 1, (256, 300))
+    H = A @ A.T / 300 + 0.01 * np.eye(256)
+    codes, scales, zeros, W_hat = O.gptq(W, O.factor(H), 3, 128)
+    np.testing.assert_array_equal(O.dequantize(codes, scales, zeros, 128), W_hat)
+    X = g.normal(0, 1, (7, 256))
+    packed = O.pack_codes(codes, 3)
+    np.testing.assert_allclose(O.dequant_matmul(X, packed, scales, zeros, 3, 128), X @ W_hat.astype(np.float64).T,
+                               rtol=1e-15, atol=1e-15)
