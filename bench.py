@@ -14,6 +14,7 @@ Kernel-level workloads (one JSON line per shape; used for the profiles and the r
   python bench.py --workload gptq --shape 32x512x1024 ...     GPTQ of [batch, d_out, d_in] bf16 weights
   python bench.py --workload factor --shape 32x1024 ...       inverse-Cholesky factor of [batch, d, d]
   python bench.py --workload epmq --shape 8x4096x4096 ...     E-PMQ target W* = R H^-1 of K source experts
+  python bench.py --workload dequant --shape 8192x4096x4096   deployable layer from 3-bit packed codes
 
 With N > 1 (torchrun, one process per GPU) every rank calibrates its own independent layer pair:
 weak scaling, no data-path collective; the step time is the max over ranks. With --parallel tokens
@@ -488,6 +489,19 @@ def run_kernel(args):
             fn = lambda: L.clha_expert_act(ctx, X, n, dm, None, 1, Wg, Wu, dff, hbuf)
             work, unit, bound, peak = 4 * n * dm * dff / 1e12, "TFLOP/s", "alu", alu["fp32_tflops"]
             kname = "expert_act_simt"
+        elif args.workload == "dequant":
+            n, d_out, d_in = dims
+            bits = 3
+            X = torch.randn((n, d_in), device="cuda", generator=g).to(torch.bfloat16)
+            codes = torch.randint(0, 2 ** bits, (d_out, d_in), device="cuda", generator=g, dtype=torch.uint8)
+            packed = torch.empty((d_out, d_in * bits // 32), dtype=torch.int32, device="cuda")
+            L.clha_pack_codes(ctx, codes, d_out, d_in, bits, packed)
+            sc = 0.01 * torch.rand((d_out, d_in // 128), device="cuda", generator=g)
+            zs = torch.full((d_out, d_in // 128), 3, dtype=torch.uint8, device="cuda")
+            Y = torch.empty((n, d_out), device="cuda")
+            fn = lambda: L.clha_dequant_matmul(ctx, X, n, packed, sc, zs, d_out, d_in, bits, Y)
+            work, unit, bound, peak = 2 * n * d_out * d_in / 1e12, "TFLOP/s", "alu", alu["fp32_tflops"]
+            kname = "dequant_matmul_kernel (3-bit packed codes, fp32 FMA)"
         elif args.workload == "epmq":
             Ksrc, d_out, d = dims
             Xs = torch.randn((Ksrc, 2 * d, d), device="cuda", generator=g).to(torch.bfloat16)
@@ -573,7 +587,8 @@ def main():
                          "one pair, its tokens sharded over the ranks with one all-reduce of the Hessian sums, "
                          "its experts quantized in parallel (strong scaling)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
-    ap.add_argument("--workload", choices=("moe", "act", "hessian", "gptq", "factor", "epmq"), default="moe",
+    ap.add_argument("--workload", choices=("moe", "act", "hessian", "gptq", "factor", "epmq", "dequant"),
+                    default="moe",
                     help="moe: the end-to-end calibration step (default); others: one kernel family")
     ap.add_argument("--shape", nargs="+", default=[], help="kernel workload shapes, e.g. 65536x4096")
     args = ap.parse_args()

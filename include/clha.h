@@ -213,6 +213,25 @@ CLHA_API clha_status clha_factor_groups(clha_ctx* ctx, int n_groups, const clha_
  * W_src: device [K, d_out, d] (the source experts' weights), W_merged: device [d_out, d], both of
  * `dtype`; U: device float32 [d, d]; lambda_dev: device double. d = acc's d; d_out a multiple of 64.
  * Device pointers are the caller's. */
+/* ------------------------------------------------------------------------------ deployable codes */
+
+/* Packs GPTQ's codes (uint8 [rows, d_in], values < 2^bits) into uint32 [rows, d_in * bits / 32]:
+ * each row's codes as one little-endian bit stream, code j at bits [bits*j, bits*j + bits) (a code
+ * may straddle two words). bits in 2..8, d_in a multiple of 128. Device pointers are the caller's.
+ * The pages give no deployable layout; this one has no padding at any bit width. */
+CLHA_API clha_status clha_pack_codes(clha_ctx* ctx, const uint8_t* codes, int64_t rows, int d_in, int bits,
+                                     uint32_t* packed);
+/* W_hat = s (q - z) per 128-column group from packed codes (scales float32 and zeros uint8
+ * [rows, d_in / 128], as written by clha_quantize): float32 [rows, d_in], bit-identical to
+ * clha_quantize's W_hat. */
+CLHA_API clha_status clha_dequantize(clha_ctx* ctx, const uint32_t* packed, const float* scales, const uint8_t* zeros,
+                                     int64_t rows, int d_in, int bits, float* W_hat);
+/* The deployable layer: Y [n, d_out] float32 = X [n, d_in] W_hat^T, W_hat decoded from the packed
+ * codes inside the product (fp32 FMA). X bf16 or f32; d_out a multiple of 64. */
+CLHA_API clha_status clha_dequant_matmul(clha_ctx* ctx, const void* X, clha_dtype dtype, int64_t n,
+                                         const uint32_t* packed, const float* scales, const uint8_t* zeros, int d_out,
+                                         int d_in, int bits, float* Y);
+
 CLHA_API clha_status clha_epmq_target(clha_ctx* ctx, const clha_accum* acc, int slot, const void* W_src,
                                       const void* W_merged, clha_dtype dtype, int d_out, const float* U,
                                       const double* lambda_dev, float* W_target);

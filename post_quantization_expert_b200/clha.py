@@ -30,6 +30,7 @@ SYMBOLS = [
     "clha_accum_create", "clha_accum_destroy", "clha_accum_zero", "clha_accum_buffers",
     "clha_accum_export", "clha_accum_import", "clha_collect",
     "clha_aggregate", "clha_factor", "clha_factor_groups", "clha_epmq_target", "clha_quantize", "clha_loss",
+    "clha_pack_codes", "clha_dequantize", "clha_dequant_matmul",
 ]
 FACTOR_MAX_GROUPS = 4
 
@@ -85,6 +86,9 @@ def load(path: str = LIB_PATH):
         "clha_factor": (i32, [vp, vp, i32, i32, vp]),
         "clha_factor_groups": (i32, [vp, i32, vp]),
         "clha_epmq_target": (i32, [vp, vp, i32, vp, vp, i32, i32, vp, vp, vp]),
+        "clha_pack_codes": (i32, [vp, vp, i64, i32, i32, vp]),
+        "clha_dequantize": (i32, [vp, vp, vp, vp, i64, i32, i32, vp]),
+        "clha_dequant_matmul": (i32, [vp, vp, i32, i64, vp, vp, vp, i32, i32, i32, vp]),
         "clha_quantize": (i32, [vp, vp, i32, vp, i32, i32, i32, i32, C.POINTER(QuantParams), vp, vp, vp, vp, vp,
                                 vp]),
         "clha_loss": (i32, [vp, vp, i32, vp, vp, i32, i32, i32, i32, vp]),
@@ -277,6 +281,19 @@ def clha_epmq_target(ctx: Context, acc: "Accum", slot: int, W_src, W_merged, d_o
     """W_target = (lambda W_m + sum_i W_i S_i) U^T U for the accumulator's K source experts."""
     ctx._check(load().clha_epmq_target(ctx.handle, acc.handle, slot, _p(W_src), _p(W_merged), _dtype(W_src), d_out,
                                        _p(U), _p(lambda_dev), _p(W_target)))
+
+
+def clha_pack_codes(ctx: Context, codes, rows: int, d_in: int, bits: int, packed):
+    ctx._check(load().clha_pack_codes(ctx.handle, _p(codes), rows, d_in, bits, _p(packed)))
+
+
+def clha_dequantize(ctx: Context, packed, scales, zeros, rows: int, d_in: int, bits: int, W_hat):
+    ctx._check(load().clha_dequantize(ctx.handle, _p(packed), _p(scales), _p(zeros), rows, d_in, bits, _p(W_hat)))
+
+
+def clha_dequant_matmul(ctx: Context, X, n: int, packed, scales, zeros, d_out: int, d_in: int, bits: int, Y):
+    ctx._check(load().clha_dequant_matmul(ctx.handle, _p(X), _dtype(X), n, _p(packed), _p(scales), _p(zeros), d_out,
+                                          d_in, bits, _p(Y)))
 
 
 def clha_quantize(ctx: Context, U, n_u: int, W, batch: int, d_out: int, d_in: int, bits: int, codes, scales,

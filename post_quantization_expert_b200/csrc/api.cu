@@ -415,6 +415,49 @@ extern "C" clha_status clha_factor(clha_ctx* ctx, const float* H_damped, int bat
     return clha_factor_groups(ctx, 1, &g);
 }
 
+// ------------------------------------------------------------------------------ deployable codes
+extern "C" clha_status clha_pack_codes(clha_ctx* ctx, const uint8_t* codes, int64_t rows, int d_in, int bits,
+                                       uint32_t* packed) {
+    CHECK_CTX(ctx);
+    REQUIRE(rows >= 0 && bits >= 2 && bits <= 8, CLHA_ERR_INVALID_ARG, "clha_pack_codes: need rows >= 0, 2 <= bits <= 8");
+    REQUIRE(d_in > 0 && d_in % 128 == 0, CLHA_ERR_UNSUPPORTED_SHAPE, "clha_pack_codes: d_in=%d is not a multiple of 128",
+            d_in);
+    REQUIRE(rows == 0 || (codes && packed), CLHA_ERR_INVALID_ARG, "clha_pack_codes: null pointer");
+    SET_DEVICE(ctx);
+    LaunchScope launch_scope(ctx);
+    CUDA_TRY(launch_pack_codes(ctx->stream, codes, rows, d_in, bits, packed), "clha_pack_codes");
+    return CLHA_OK;
+}
+
+extern "C" clha_status clha_dequantize(clha_ctx* ctx, const uint32_t* packed, const float* scales,
+                                       const uint8_t* zeros, int64_t rows, int d_in, int bits, float* W_hat) {
+    CHECK_CTX(ctx);
+    REQUIRE(rows >= 0 && bits >= 2 && bits <= 8, CLHA_ERR_INVALID_ARG, "clha_dequantize: need rows >= 0, 2 <= bits <= 8");
+    REQUIRE(d_in > 0 && d_in % 128 == 0, CLHA_ERR_UNSUPPORTED_SHAPE, "clha_dequantize: d_in=%d is not a multiple of 128",
+            d_in);
+    REQUIRE(rows == 0 || (packed && scales && zeros && W_hat), CLHA_ERR_INVALID_ARG, "clha_dequantize: null pointer");
+    SET_DEVICE(ctx);
+    LaunchScope launch_scope(ctx);
+    CUDA_TRY(launch_dequantize(ctx->stream, packed, scales, zeros, rows, d_in, bits, W_hat), "clha_dequantize");
+    return CLHA_OK;
+}
+
+extern "C" clha_status clha_dequant_matmul(clha_ctx* ctx, const void* X, clha_dtype dtype, int64_t n,
+                                           const uint32_t* packed, const float* scales, const uint8_t* zeros,
+                                           int d_out, int d_in, int bits, float* Y) {
+    CHECK_CTX(ctx);
+    REQUIRE(dtype == CLHA_BF16 || dtype == CLHA_F32, CLHA_ERR_INVALID_ARG, "clha_dequant_matmul: unknown dtype");
+    REQUIRE(n >= 0 && bits >= 2 && bits <= 8, CLHA_ERR_INVALID_ARG, "clha_dequant_matmul: need n >= 0, 2 <= bits <= 8");
+    REQUIRE(d_in > 0 && d_in % 128 == 0 && d_out > 0 && d_out % 64 == 0, CLHA_ERR_UNSUPPORTED_SHAPE,
+            "clha_dequant_matmul: need d_in a multiple of 128 and d_out of 64 (got %d, %d)", d_in, d_out);
+    REQUIRE(n == 0 || (X && packed && scales && zeros && Y), CLHA_ERR_INVALID_ARG, "clha_dequant_matmul: null pointer");
+    SET_DEVICE(ctx);
+    LaunchScope launch_scope(ctx);
+    CUDA_TRY(launch_dequant_matmul(ctx->stream, X, dtype == CLHA_BF16, n, d_in, packed, scales, zeros, d_out, bits, Y),
+             "clha_dequant_matmul");
+    return CLHA_OK;
+}
+
 extern "C" clha_status clha_epmq_target(clha_ctx* ctx, const clha_accum* acc, int slot, const void* W_src,
                                         const void* W_merged, clha_dtype dtype, int d_out, const float* U,
                                         const double* lambda_dev, float* W_target) {

@@ -102,6 +102,13 @@ struct FactorGroup {
 };
 size_t factor_workspace_bytes(const FactorGroup* groups, int n);
 cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups, int n, void* ws, int* err);
+cudaError_t launch_pack_codes(cudaStream_t s, const uint8_t* codes, int64_t rows, int d_in, int bits,
+                              uint32_t* packed);
+cudaError_t launch_dequantize(cudaStream_t s, const uint32_t* packed, const float* scales, const uint8_t* zeros,
+                              int64_t rows, int d_in, int bits, float* W_hat);
+cudaError_t launch_dequant_matmul(cudaStream_t s, const void* X, int x_bf16, int64_t n, int d_in,
+                                  const uint32_t* packed, const float* scales, const uint8_t* zeros, int d_out, int bits,
+                                  float* Y);
 size_t epmq_workspace_bytes(int d_out, int d);
 cudaError_t launch_epmq_target(cudaStream_t s, const float* S_slot, int64_t layer_stride, int K, const void* W_src,
                                int w_bf16, const void* W_m, int d_out, int d, const float* U, const double* lambda,
