@@ -401,38 +401,45 @@ __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
             if (lvl[mid] <= t) lo = mid; else hi = mid - 1;
         }
         const int sg = lo;
-        unsigned long long r = t - lvl[sg];
+        // within a stage every count fits in 32 bits (a stage holds at most batch x ~nt^2 tasks):
+        // 32-bit arithmetic keeps the decode off the 64-bit division path
+        uint32_t r = (uint32_t)(t - lvl[sg]);
         Grp G = g.grp[0];
         bool found = false;
 #pragma unroll
         for (int k = 0; k < MAX_GROUPS; ++k) {   // (unrolled: the group record stays in registers)
             if (!found && k < g.ng) {
-                const unsigned long long c = stage_total(g.grp[k].nt, sg) * g.grp[k].batch;
+                const uint32_t c = (uint32_t)stage_total(g.grp[k].nt, sg) * (uint32_t)g.grp[k].batch;
                 if (r < c) { G = g.grp[k]; found = true; }
                 else r -= c;
             }
         }
-        const int nt = G.nt, batch = G.batch;
+        const int nt = G.nt;
+        const uint32_t batch = (uint32_t)G.batch;
         long long n[6];
         stage_counts(nt, sg, n);
         int c = 0;
 #pragma unroll
         for (int cq = 0; cq < 6; ++cq)   // (unrolled: n[] stays in registers)
-            if (c == cq && r >= (unsigned long long)n[cq] * batch) { r -= (unsigned long long)n[cq] * batch; ++c; }
-        const long long local = (long long)(r / batch);
-        const int b = (int)(r % batch);
+            if (c == cq && r >= (uint32_t)n[cq] * batch) { r -= (uint32_t)n[cq] * batch; ++c; }
+        const uint32_t local = r / batch;
+        const int b = (int)(r - local * batch);
         const int prob = G.pbase + b;
         int q, m = sg - 1, i = 0, j = 0;
         if (c == 0) { q = 2; i = m + 1 + (int)local; j = m + 1; }
         else if (c == 1) { q = 0; m = sg; }
         else if (c == 2) { q = 3; j = (int)local; }
-        else if (c == 3) { q = 4; i = m + 1 + (int)(local / (m + 1)); j = (int)(local % (m + 1)); }
-        else if (c == 4) {
+        else if (c == 3) {
+            q = 4;
+            const uint32_t ii = local / (uint32_t)(m + 1);
+            i = m + 1 + (int)ii;
+            j = (int)(local - ii * (uint32_t)(m + 1));
+        } else if (c == 4) {
             q = 5;
-            long long rem = local;
+            int rem = (int)local;
             j = m + 2;
             while (rem >= nt - j) { rem -= nt - j; ++j; }
-            i = j + (int)rem;
+            i = j + rem;
         } else { q = 1; m = sg; i = m + 1 + (int)local; j = m; }
 
         // operands, output and the states to wait for (lane k of warp 0 polls condition k)
@@ -570,6 +577,22 @@ cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups
         g.total += per * (unsigned long long)G.batch;
     }
 
+    // the kernel decodes a task's place inside its stage in 32-bit arithmetic
+    for (int st = 0; st <= g.max_nt; ++st) {
+        unsigned long long tasks = 0;
+        for (int k = 0; k < n; ++k) {
+            const int nt = g.grp[k].nt;
+            if (st > nt) continue;
+            unsigned long long per;
+            if (st == 0) per = (unsigned long long)nt;
+            else {
+                const long long m = st - 1, R = nt - 1 - m;
+                per = R + (R >= 1 ? 1 : 0) + m + (m + 1) * R + (R >= 1 ? (R - 1) * R / 2 + R - 1 : 0);
+            }
+            tasks += per * (unsigned long long)g.grp[k].batch;
+        }
+        if (tasks >= (1ull << 31)) return cudaErrorInvalidValue;
+    }
     const size_t smem = dag_smem_bytes(g.max_nt);
     cudaError_t e = cudaFuncSetAttribute(fac_dag, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
