@@ -192,7 +192,7 @@ class MoECalibration:
 
     def __init__(self, ctx: L.Context, n_layers: int, max_tokens: int, E: int, k: int, d_model: int, d_ff: int,
                  n_shared: int = 0, shared_dff: int = 0, bits_routed: int = 2, bits_shared: int = 3,
-                 damp_frac: float = 0.01, timer=NO_TIMER, modes=("rt",)):
+                 damp_frac: float = 0.01, timer=NO_TIMER, modes=("rt",), keep_hcomb: bool = False):
         self.ctx, self.n_layers, self.E, self.k = ctx, n_layers, E, k
         self.timer = timer
         self.d_model, self.d_ff, self.n_shared, self.shared_dff = d_model, d_ff, n_shared, shared_dff
@@ -213,20 +213,22 @@ class MoECalibration:
         self.modes = tuple(modes)
         nm = len(self.modes)
         f32 = dict(dtype=torch.float32, device=dev)
-        # [weighting][expert] Hessians and factors
-        self.Hc_in = torch.empty((nm * E, d_model, d_model), **f32)
-        self.Hd_in = torch.empty_like(self.Hc_in)
-        self.U_in = torch.empty_like(self.Hc_in)
-        self.Hc_dn = torch.empty((nm * E, d_ff, d_ff), **f32)
-        self.Hd_dn = torch.empty_like(self.Hc_dn)
-        self.U_dn = torch.empty_like(self.Hc_dn)
+        # [weighting][expert] Hessians and factors; the undamped aggregates only on request (GPTQ and
+        # its in-kernel loss need only the damped one and lambda)
+        hc = (lambda shape: torch.empty(shape, **f32)) if keep_hcomb else (lambda shape: None)
+        self.Hd_in = torch.empty((nm * E, d_model, d_model), **f32)
+        self.Hc_in = hc(self.Hd_in.shape)
+        self.U_in = torch.empty_like(self.Hd_in)
+        self.Hd_dn = torch.empty((nm * E, d_ff, d_ff), **f32)
+        self.Hc_dn = hc(self.Hd_dn.shape)
+        self.U_dn = torch.empty_like(self.Hd_dn)
         if n_shared:
-            self.Hc_sin = torch.empty((nm, d_model, d_model), **f32)
-            self.Hd_sin = torch.empty_like(self.Hc_sin)
-            self.U_sin = torch.empty_like(self.Hc_sin)
-            self.Hc_sdn = torch.empty((nm * n_shared, shared_dff, shared_dff), **f32)
-            self.Hd_sdn = torch.empty_like(self.Hc_sdn)
-            self.U_sdn = torch.empty_like(self.Hc_sdn)
+            self.Hd_sin = torch.empty((nm, d_model, d_model), **f32)
+            self.Hc_sin = hc(self.Hd_sin.shape)
+            self.U_sin = torch.empty_like(self.Hd_sin)
+            self.Hd_sdn = torch.empty((nm * n_shared, shared_dff, shared_dff), **f32)
+            self.Hc_sdn = hc(self.Hd_sdn.shape)
+            self.U_sdn = torch.empty_like(self.Hd_sdn)
         f64 = dict(dtype=torch.float64, device=dev)
         self.lam_in = torch.empty(nm * E, **f64)
         self.lam_dn = torch.empty(nm * E, **f64)
@@ -296,17 +298,19 @@ class MoECalibration:
         ctx, E, dm, dff, t = self.ctx, self.E, self.d_model, self.d_ff, self.timer
         ns, sdff = self.n_shared, self.shared_dff
         idx = [self.modes.index(m) for m in modes]
+        opt = lambda h, sl: None if h is None else h[sl]
         with t.span("aggregate"):
             for i, m in zip(idx, modes):
                 es, ss = slice(i * E, (i + 1) * E), slice(i * ns, (i + 1) * ns)
-                L.clha_aggregate(ctx, self.acc_in, 0, E, MODES[m], alpha, self.damp, self.Hc_in[es], self.Hd_in[es],
-                                 lambda_dev=self.lam_in[es])
-                L.clha_aggregate(ctx, self.acc_dn, 0, E, MODES[m], alpha, self.damp, self.Hc_dn[es], self.Hd_dn[es],
-                                 lambda_dev=self.lam_dn[es])
+                L.clha_aggregate(ctx, self.acc_in, 0, E, MODES[m], alpha, self.damp, opt(self.Hc_in, es),
+                                 self.Hd_in[es], lambda_dev=self.lam_in[es])
+                L.clha_aggregate(ctx, self.acc_dn, 0, E, MODES[m], alpha, self.damp, opt(self.Hc_dn, es),
+                                 self.Hd_dn[es], lambda_dev=self.lam_dn[es])
                 if ns:
-                    L.clha_aggregate(ctx, self.acc_in, E, 1, MODES[m], alpha, self.damp, self.Hc_sin[i:i + 1],
-                                     self.Hd_sin[i:i + 1], lambda_dev=self.lam_sin[i:i + 1])
-                    L.clha_aggregate(ctx, self.acc_sdn, 0, ns, MODES[m], alpha, self.damp, self.Hc_sdn[ss],
+                    L.clha_aggregate(ctx, self.acc_in, E, 1, MODES[m], alpha, self.damp,
+                                     opt(self.Hc_sin, slice(i, i + 1)), self.Hd_sin[i:i + 1],
+                                     lambda_dev=self.lam_sin[i:i + 1])
+                    L.clha_aggregate(ctx, self.acc_sdn, 0, ns, MODES[m], alpha, self.damp, opt(self.Hc_sdn, ss),
                                      self.Hd_sdn[ss], lambda_dev=self.lam_sdn[ss])
         # one batched factor per Hessian kind over every requested weighting (contiguous runs)
         lo, hi = min(idx), max(idx) + 1
