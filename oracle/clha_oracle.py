@@ -35,8 +35,16 @@ Readings where the pages are silent (each also listed in the design notes):
     error (there is nothing to calibrate on).
   * deployable codes are packed per row as one little-endian bit stream of 32-bit words, code j at
     bits [b*j, b*j + b) (the pages give no layout); W_hat = s (q - z) per group in float32.
+  * cross-layer routing divergence (CLHA page §4-5: the gains grow with it; no formula is given) is
+    the total-variation distance between two layers' expert frequencies p_l(e) = n_{l,e} / N_l.
+  * the Calibration Hessian Error (CLHA page §4) of a quantized weight is the loss of §2.1 under a
+    Hessian built from given tokens: on the calibration side the hook layer's own Hessian (the
+    distribution per-layer calibration fits), on the test side the aggregate of fresh tokens of
+    every layer sharing the weight (alpha by token share, the pooled distribution).
 """
 from __future__ import annotations
+
+from fractions import Fraction
 
 import numpy as np
 
@@ -45,6 +53,7 @@ __all__ = [
     "aggregate", "factor", "grid_fp32", "quantize_fp32", "gptq", "loss",
     "calibrate_dense", "calibrate_moe_group",
     "pack_codes", "unpack_codes", "dequantize", "dequant_matmul",
+    "routing_divergence", "hessian_error",
 ]
 
 
@@ -330,3 +339,27 @@ def dequant_matmul(X, packed, scales, zeros, bits: int, group: int = 128):
     d_in = np.asarray(X).shape[1]
     W_hat = dequantize(unpack_codes(packed, bits, d_in), scales, zeros, group)
     return np.asarray(X, dtype=np.float64) @ W_hat.astype(np.float64).T
+
+
+# ------------------------------------------------------------------- divergence and held-out error
+def routing_divergence(counts):
+    """Total-variation distance between the expert frequencies of every pair of layers:
+    TV[a][b] = 1/2 sum_e |n_{a,e}/N_a - n_{b,e}/N_b|, N_l = sum_e n_{l,e} (a reading: the CLHA page
+    names cross-layer routing divergence without defining it). counts: integer [L, E]. Evaluated as
+    an exact rational and rounded once to float64. A layer without tokens has no frequencies: error."""
+    c = [[int(v) for v in row] for row in np.asarray(counts)]
+    N = [sum(row) for row in c]
+    if any(n <= 0 for n in N):
+        raise ValueError("a layer without tokens has no expert frequencies")
+    L = len(c)
+    tv = np.zeros((L, L))
+    for a in range(L):
+        for b in range(L):
+            tv[a, b] = float(sum(abs(Fraction(x, N[a]) - Fraction(y, N[b])) for x, y in zip(c[a], c[b])) / 2)
+    return tv
+
+
+def hessian_error(W, W_hat, S_list, n_list, mode: str = "rt", alpha=None):
+    """The §2.1 loss of W_hat under the undamped aggregate of the given per-layer Gram sums: with
+    alpha = (1, 0, ...) the hook layer's own Hessian, with "rt" the pooled Hessian of all layers."""
+    return loss(W, W_hat, aggregate(S_list, n_list, mode, alpha)["H_comb"])

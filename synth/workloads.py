@@ -11,7 +11,13 @@ Input model (CLHA technical summary, section 2.1: each layer sees its own activa
   drift delta between layers sharing a weight: U_next = cos(pi*delta/2) U + sin(pi*delta/2) V,
   V an independent draw of U's distribution (delta = 0: same subspace, delta = 1: independent).
 Router logits are N(0, 1) per token and expert, plus log p_e for Zipf-skewed routing
-(p_e proportional to rank_e^-s over a seeded permutation of the experts).
+(p_e proportional to rank_e^-s over a seeded permutation of the experts), plus, for the routing
+sharpness sweep, beta * (-1)^j * v_e: a per-group expert preference v ~ N(0, I_E) that layer j of
+the group follows with alternating sign, so that raising beta concentrates each layer on its own
+experts and drives the layers' expert frequencies apart (a top-k choice is unchanged by a plain
+temperature on the logits, so sharpening acts on this preference).
+A split other than "cal" draws fresh tokens (X and logits) from the same per-layer laws and the
+same weights: the held-out data of the test-side reconstruction error.
 Outlier channels (a seeded 1% of channels) are multiplied by 20 before rounding to bf16.
 Weights are N(0, 0.02^2).
 """
@@ -52,6 +58,8 @@ class Spec:
     damp_frac: float = 0.01
     alpha_modes: tuple = ("rt",)
     chunk_tokens: int = 8192       # draw X in chunks of this many tokens (bounds temporaries)
+    split: str = "cal"             # "cal": calibration tokens; any other name: fresh tokens of the same law
+    sharpness: float = 0.0         # strength of the per-layer expert preference added to the logits
 
 
 def _spec_c1():
@@ -111,6 +119,7 @@ class Workload:
         self.device = torch.device(device)
         self._cov = {}
         self._x = {}
+        self._split = () if spec.split == "cal" else (spec.split,)   # calibration draws keep their tags
 
     # ------------------------------------------------------------------ generators
     def _gen(self, *tag) -> torch.Generator:
@@ -167,8 +176,8 @@ class Workload:
         out = torch.empty((n, s.d_model), dtype=s.dtype, device=self.device)
         for c0 in range(0, n, s.chunk_tokens):
             c1 = min(n, c0 + s.chunk_tokens)
-            z1 = self._randn((c1 - c0, s.d_model), "z1", layer, c0)
-            z2 = self._randn((c1 - c0, s.rank), "z2", layer, c0)
+            z1 = self._randn((c1 - c0, s.d_model), "z1", layer, c0, *self._split)
+            z2 = self._randn((c1 - c0, s.rank), "z2", layer, c0, *self._split)
             xc = z1.mul_(sqD).addmm_(z2, U.t())
             if s.outlier_frac > 0:
                 xc.mul_(scale)
@@ -185,7 +194,7 @@ class Workload:
         """Router logits [tokens, E] float32 for a MoE layer."""
         s = self.spec
         assert s.kind == "moe"
-        lg = self._randn((s.tokens[layer], s.E), "logits", layer)
+        lg = self._randn((s.tokens[layer], s.E), "logits", layer, *self._split)
         if s.zipf_s > 0:
             gi = self.group_index(layer)
             perm = torch.randperm(s.E, generator=self._gen("zipf", gi), device=self.device)
@@ -194,6 +203,11 @@ class Workload:
             logp = -s.zipf_s * torch.log(ranks)
             logp = logp - torch.logsumexp(logp, 0)
             lg = lg + logp[None, :]
+        if s.sharpness != 0.0:
+            gi = self.group_index(layer)
+            j = s.group_of_layers[gi].index(layer)
+            v = self._randn((s.E,), "pref", gi)
+            lg = lg + (s.sharpness * (-1.0) ** j) * v[None, :]
         return lg.contiguous()
 
     # ------------------------------------------------------------------ weights
