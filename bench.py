@@ -16,6 +16,11 @@ Kernel-level workloads (one JSON line per shape; used for the profiles and the r
   python bench.py --workload epmq --shape 8x4096x4096 ...     E-PMQ target W* = R H^-1 of K source experts
   python bench.py --workload dequant --shape 8192x4096x4096   deployable layer from 3-bit packed codes
 
+Routing-sharpness sweep (not a throughput line; one JSON line per sharpness):
+  python bench.py --workload sweep [--sharpness 0 0.1 ...]   the layer pair above at rising cross-layer
+      routing divergence: per-layer calibration (alpha = (1, 0)) against CLHA rt and eq, each scored on
+      the calibration hook layer and on fresh held-out tokens of both layers
+
 With N > 1 (torchrun, one process per GPU) every rank calibrates its own independent layer pair:
 weak scaling, no data-path collective; the step time is the max over ranks. With --parallel tokens
 the ranks share one layer pair instead: each collects its share of the tokens, one NCCL all-reduce
@@ -469,6 +474,62 @@ def run_ours(args, world, rank, local):
     return 0
 
 
+def run_sweep(args):
+    """Calibration- and test-side Hessian error of per-layer calibration (PLIC) and CLHA (rt, eq) as
+    the per-layer expert preference sharpens (the CLHA page, section 4). Synthetic tokens and weights:
+    the pages' numbers are perplexities of a trained model, which this does not reproduce."""
+    import numpy as np
+    import torch
+    from synth import workload
+    from post_quantization_expert_b200 import clha as L
+    from post_quantization_expert_b200.analysis import HessianError, mean_pairwise, routing_divergence
+    from post_quantization_expert_b200.pipeline import MoECalibration, stack_weights
+    ctx = L.Context(0)
+    rows = []
+    for beta in args.sharpness:
+        cal_wl = workload(2, "cpu", sharpness=beta)
+        test_wl = workload(2, "cpu", sharpness=beta, split="test")
+        s = cal_wl.spec
+        w = stack_weights(([cal_wl.expert_weights(0, e) for e in range(s.E)], []), "cuda")
+        mk = lambda modes: MoECalibration(ctx, 2, max(s.tokens), s.E, s.k, s.d_model, s.d_ff, 0, 0, s.bits_routed,
+                                          s.bits_shared, s.damp_frac, modes=modes)
+        cal, held = mk(("explicit", "rt", "eq")), mk(("rt",))
+        for col, wl in ((cal, cal_wl), (held, test_wl)):
+            for l in range(2):
+                col.collect(l, wl.x(l).to("cuda"), wl.logits(l).to("cuda"), w)
+        counts = cal.acc_in.buffers()[1][:, : s.E].cpu().numpy()
+        hook = (1.0, 0.0)
+        cal.quantize(w, alpha=hook)
+        he = HessianError(ctx, s.E, s.d_model, s.d_ff)
+        che_cal, che_test = {}, {}
+        for name, mode in (("plic", "explicit"), ("clha_rt", "rt"), ("clha_eq", "eq")):
+            r = cal.res[mode]
+            che_cal[name] = float(he(cal, w, r, "explicit", hook)["routed"].sum())
+            che_test[name] = float(he(held, w, r, "rt")["routed"].sum())
+        row = {"workload": "routing-sharpness sweep", "sharpness": beta,
+               "divergence_tv": mean_pairwise(routing_divergence(ctx, cal.acc_in, 0, s.E)),
+               "divergence_tv_test": mean_pairwise(routing_divergence(ctx, held.acc_in, 0, s.E)),
+               "min_expert_tokens_per_layer": [int(c) for c in counts.min(1)],
+               "che_cal": che_cal, "che_test": che_test,
+               "test_gain_rt_vs_plic": 1.0 - che_test["clha_rt"] / che_test["plic"],
+               "test_gain_eq_vs_plic": 1.0 - che_test["clha_eq"] / che_test["plic"],
+               "config": {"workload": s.name, "tokens_per_layer": s.tokens[0], "held_out_tokens_per_layer":
+                          test_wl.spec.tokens[0], "bits": s.bits_routed, "data": "synthetic"}}
+        rows.append(row)
+        print(json.dumps(row), flush=True)
+        del cal, held, he, w
+        torch.cuda.empty_cache()
+    if rows:
+        base = rows[0]["che_test"]
+        print(json.dumps({"workload": "routing-sharpness sweep summary",
+                          "sharpness": [r["sharpness"] for r in rows],
+                          "divergence_tv": [r["divergence_tv"] for r in rows],
+                          "test_error_vs_first": {k: [r["che_test"][k] / base[k] for r in rows] for k in base},
+                          "test_gain_rt_vs_plic": [r["test_gain_rt_vs_plic"] for r in rows]}), flush=True)
+    ctx.close()
+    return 0
+
+
 def run_kernel(args):
     """Kernel-level timing: CUDA events around `steps` launches after `warmup`, inputs resident."""
     import torch
@@ -588,13 +649,18 @@ def main():
                          "one pair, its tokens sharded over the ranks with one all-reduce of the Hessian sums, "
                          "its experts quantized in parallel (strong scaling)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
-    ap.add_argument("--workload", choices=("moe", "act", "hessian", "gptq", "factor", "epmq", "dequant"),
+    ap.add_argument("--workload", choices=("moe", "act", "hessian", "gptq", "factor", "epmq", "dequant", "sweep"),
                     default="moe",
-                    help="moe: the end-to-end calibration step (default); others: one kernel family")
+                    help="moe: the end-to-end calibration step (default); sweep: the routing-sharpness "
+                         "experiment; others: one kernel family")
+    ap.add_argument("--sharpness", type=float, nargs="+", default=[0.0, 0.1, 0.2, 0.3, 0.4, 0.5],
+                    help="sweep: strengths of the per-layer expert preference")
     ap.add_argument("--shape", nargs="+", default=[], help="kernel workload shapes, e.g. 65536x4096")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload == "sweep":
+        return run_sweep(args)
     if args.workload != "moe":
         if not args.shape:
             ap.error("--shape is required for kernel workloads")

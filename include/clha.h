@@ -226,6 +226,7 @@ CLHA_API clha_status clha_pack_codes(clha_ctx* ctx, const uint8_t* codes, int64_
  * clha_quantize's W_hat. */
 CLHA_API clha_status clha_dequantize(clha_ctx* ctx, const uint32_t* packed, const float* scales, const uint8_t* zeros,
                                      int64_t rows, int d_in, int bits, float* W_hat);
+
 /* The deployable layer: Y [n, d_out] float32 = X [n, d_in] W_hat^T, W_hat decoded from the packed
  * codes inside the product (fp32 FMA). X bf16 or f32; d_out a multiple of 64. */
 CLHA_API clha_status clha_dequant_matmul(clha_ctx* ctx, const void* X, clha_dtype dtype, int64_t n,
@@ -265,6 +266,25 @@ CLHA_API clha_status clha_quantize(clha_ctx* ctx, const float* U, int n_u, const
  * loss_out is a host double [batch] array (synchronises). */
 CLHA_API clha_status clha_loss(clha_ctx* ctx, const void* W, clha_dtype dtype, const float* W_hat,
                       const float* H, int n_h, int batch, int d_out, int d_in, double* loss_out);
+
+/* ------------------------------------------------------------------------------ analysis */
+
+#define CLHA_DIVERGENCE_MAX_LAYERS 1024
+
+/* Cross-layer routing divergence. The CLHA page (§4, the routing-sharpness experiment, and §5)
+ * relates CLHA's gains to the divergence of routing across the layers that share experts but gives
+ * no formula; it is read as the total-variation distance of two layers' expert frequencies:
+ *   tv[a * n_layers + b] = 1/2 sum_e |n_{a,e} / N_a - n_{b,e} / N_b|,  N_l = sum_e n_{l,e},
+ * over the experts e in [slot0, slot0 + E) of `counts`, a device int64 [n_layers, ld] array (an
+ * accumulator's counts from clha_accum_buffers, ld = its slot count). tv is a caller-owned device
+ * double [n_layers, n_layers] array, symmetric with a zero diagonal, values in [0, 1]. The sums are
+ * exact 64-bit integer arithmetic and the one division is float64: the correctly rounded value
+ * while 2 N_a N_b <= 2^53. Nothing synchronises. Errors, recorded on the device and returned by the
+ * next synchronising call or clha_check: a layer without tokens in the range gives CLHA_ERR_EMPTY, a
+ * count outside [0, 2^31) or N_l >= 2^31 gives CLHA_ERR_INVALID_ARG; the entries of such a layer's
+ * pairs are NaN. */
+CLHA_API clha_status clha_routing_divergence(clha_ctx* ctx, const int64_t* counts, int n_layers, int ld, int slot0,
+                                             int E, double* tv);
 
 #ifdef __cplusplus
 }

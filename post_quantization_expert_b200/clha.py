@@ -30,7 +30,7 @@ SYMBOLS = [
     "clha_accum_create", "clha_accum_destroy", "clha_accum_zero", "clha_accum_buffers",
     "clha_accum_export", "clha_accum_import", "clha_collect",
     "clha_aggregate", "clha_factor", "clha_factor_groups", "clha_epmq_target", "clha_quantize", "clha_loss",
-    "clha_pack_codes", "clha_dequantize", "clha_dequant_matmul",
+    "clha_pack_codes", "clha_dequantize", "clha_dequant_matmul", "clha_routing_divergence",
 ]
 FACTOR_MAX_GROUPS = 4
 
@@ -92,6 +92,7 @@ def load(path: str = LIB_PATH):
         "clha_quantize": (i32, [vp, vp, i32, vp, i32, i32, i32, i32, C.POINTER(QuantParams), vp, vp, vp, vp, vp,
                                 vp]),
         "clha_loss": (i32, [vp, vp, i32, vp, vp, i32, i32, i32, i32, vp]),
+        "clha_routing_divergence": (i32, [vp, vp, i32, i32, i32, i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -294,6 +295,12 @@ def clha_dequantize(ctx: Context, packed, scales, zeros, rows: int, d_in: int, b
 def clha_dequant_matmul(ctx: Context, X, n: int, packed, scales, zeros, d_out: int, d_in: int, bits: int, Y):
     ctx._check(load().clha_dequant_matmul(ctx.handle, _p(X), _dtype(X), n, _p(packed), _p(scales), _p(zeros), d_out,
                                           d_in, bits, _p(Y)))
+
+
+def clha_routing_divergence(ctx: Context, counts, n_layers: int, ld: int, slot0: int, E: int, tv):
+    """tv (float64 device [n_layers, n_layers]) = total-variation distance of the layers' expert
+    frequencies over experts [slot0, slot0 + E) of counts (int64 device [n_layers, ld])."""
+    ctx._check(load().clha_routing_divergence(ctx.handle, _p(counts), n_layers, ld, slot0, E, _p(tv)))
 
 
 def clha_quantize(ctx: Context, U, n_u: int, W, batch: int, d_out: int, d_in: int, bits: int, codes, scales,

@@ -97,6 +97,7 @@ static const char* kernel_name(int kid) {
         case KID_FACTOR: return "clha_factor";
         case KID_QUANTIZE: return "clha_quantize";
         case KID_LOSS: return "clha_loss";
+        case KID_DIVERGENCE: return "clha_routing_divergence";
         default: return "kernel";
     }
 }
@@ -455,6 +456,21 @@ extern "C" clha_status clha_dequant_matmul(clha_ctx* ctx, const void* X, clha_dt
     LaunchScope launch_scope(ctx);
     CUDA_TRY(launch_dequant_matmul(ctx->stream, X, dtype == CLHA_BF16, n, d_in, packed, scales, zeros, d_out, bits, Y),
              "clha_dequant_matmul");
+    return CLHA_OK;
+}
+
+extern "C" clha_status clha_routing_divergence(clha_ctx* ctx, const int64_t* counts, int n_layers, int ld,
+                                               int slot0, int E, double* tv) {
+    CHECK_CTX(ctx);
+    REQUIRE(counts && tv, CLHA_ERR_INVALID_ARG, "clha_routing_divergence: null pointer");
+    REQUIRE(n_layers >= 1 && n_layers <= CLHA_DIVERGENCE_MAX_LAYERS && E >= 1 && slot0 >= 0 && ld >= 1 &&
+                (int64_t)slot0 + E <= ld,
+            CLHA_ERR_INVALID_ARG, "clha_routing_divergence: need 1 <= n_layers <= %d, E >= 1, 0 <= slot0, slot0 + E <= ld",
+            CLHA_DIVERGENCE_MAX_LAYERS);
+    SET_DEVICE(ctx);
+    LaunchScope launch_scope(ctx);
+    CUDA_TRY(launch_routing_divergence(ctx->stream, counts, n_layers, ld, slot0, E, tv, ctx->d_err),
+             "clha_routing_divergence");
     return CLHA_OK;
 }
 

@@ -35,7 +35,7 @@ struct clha_accum {
 
 enum clha_kernel_id {
     KID_ROUTE = 1, KID_GATHER = 2, KID_ACT = 3, KID_COLLECT = 4, KID_AGGREGATE = 5,
-    KID_FACTOR = 6, KID_QUANTIZE = 7, KID_LOSS = 8
+    KID_FACTOR = 6, KID_QUANTIZE = 7, KID_LOSS = 8, KID_DIVERGENCE = 9
 };
 
 // ------------------------------------------------------------------------------ device helpers
@@ -109,6 +109,8 @@ cudaError_t launch_dequantize(cudaStream_t s, const uint32_t* packed, const floa
 cudaError_t launch_dequant_matmul(cudaStream_t s, const void* X, int x_bf16, int64_t n, int d_in,
                                   const uint32_t* packed, const float* scales, const uint8_t* zeros, int d_out, int bits,
                                   float* Y);
+cudaError_t launch_routing_divergence(cudaStream_t s, const int64_t* counts, int L, int ld, int slot0, int E,
+                                      double* tv, int* err);
 size_t epmq_workspace_bytes(int d_out, int d);
 cudaError_t launch_epmq_target(cudaStream_t s, const float* S_slot, int64_t layer_stride, int K, const void* W_src,
                                int w_bf16, const void* W_m, int d_out, int d, const float* U, const double* lambda,
