@@ -354,23 +354,29 @@ def run_ours(args, world, rank, local):
     pin = lambda t: t.pin_memory()
     hX, hL = [pin(x) for x in X], [pin(l) for l in lg]
     hW = [pin(w.Wgu.cpu()), pin(w.Wd.cpu())]
-    outs = {m: [qcal.res[m].qgu, qcal.res[m].qd] for m in modes}
-    hout = {m: [(pin(torch.empty_like(q.codes, device="cpu")), pin(torch.empty_like(q.scales, device="cpu")),
-                 pin(torch.empty_like(q.zeros, device="cpu"))) for q in outs[m]] for m in modes}
+    outs = {m: {"gu": qcal.res[m].qgu, "d": qcal.res[m].qd} for m in modes}
+    hout = {m: {k: (pin(torch.empty_like(q.codes, device="cpu")), pin(torch.empty_like(q.scales, device="cpu")),
+                    pin(torch.empty_like(q.zeros, device="cpu"))) for k, q in outs[m].items()} for m in modes}
     h2d = sum(t.numel() * t.element_size() for t in hX + hL + hW)
-    d2h = sum(t.numel() * t.element_size() for m in modes for trip in hout[m] for t in trip)
+    d2h = sum(t.numel() * t.element_size() for m in modes for trip in hout[m].values() for t in trip)
     timer.enabled = False
+    if not sharded:
+        from post_quantization_expert_b200.pipeline import HostStep, MoEWeights
+        host_step = HostStep(cal, [x.shape for x in X], [l.shape for l in lg], MoEWeights(*hW))
 
     def e2e_step():
+        if not sharded:     # copies on their own stream, overlapped with the compute
+            host_step.run(hX, hL, MoEWeights(*hW), hout, modes)
+            return
         with torch.cuda.stream(stream):
             for d_, h_ in zip(Xd + Ld + [w.Wgu, w.Wd], hX + hL + hW):
                 d_.copy_(h_, non_blocking=True)
-            if sharded:
-                wq.Wgu.copy_(torch.cat([w.Wgu[sh.e0:sh.e1], w.Wgu[s.E + sh.e0:s.E + sh.e1]]))
-                wq.Wd.copy_(w.Wd[sh.e0:sh.e1])
+            wq.Wgu.copy_(torch.cat([w.Wgu[sh.e0:sh.e1], w.Wgu[s.E + sh.e0:s.E + sh.e1]]))
+            wq.Wd.copy_(w.Wd[sh.e0:sh.e1])
             calibrate()
             for m in modes:
-                for q, (hc, hs, hz) in zip(outs[m], hout[m]):
+                for k, (hc, hs, hz) in hout[m].items():
+                    q = outs[m][k]
                     hc.copy_(q.codes, non_blocking=True)
                     hs.copy_(q.scales, non_blocking=True)
                     hz.copy_(q.zeros, non_blocking=True)

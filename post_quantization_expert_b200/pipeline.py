@@ -263,7 +263,10 @@ class MoECalibration:
             L.clha_accum_zero(self.ctx, a)
 
     # ------------------------------------------------------------------ phase 1
-    def collect(self, layer: int, X: torch.Tensor, logits: torch.Tensor, w: MoEWeights):
+    def collect(self, layer: int, X: torch.Tensor, logits: torch.Tensor, w: MoEWeights, before_act=None):
+        """Phase 1 for one layer's tokens. before_act (optional) is called once the steps that need only
+        X and the logits are queued, before the first that reads the weights (a caller copying the
+        weights in on another stream makes the compute stream wait there)."""
         ctx, E, k, n, t = self.ctx, self.E, self.k, X.shape[0], self.timer
         ids = self.ids[:n]
         seg = self.seg[layer]
@@ -273,13 +276,15 @@ class MoECalibration:
             L.clha_gather(ctx, X, n, self.d_model, ids, k, E, self.Xp, self.P, seg)
         with t.span("hessian"):
             L.clha_collect(ctx, self.acc_in, layer, self.Xp, self.P, self.d_model, seg, E, 0)
+            if self.n_shared:
+                L.clha_collect(ctx, self.acc_in, layer, X, n, self.d_model, None, 1, E)
+        if before_act is not None:
+            before_act()
         with t.span("act"):
             L.clha_expert_act(ctx, self.Xp, self.P, self.d_model, seg, E, w.Wg, w.Wu, self.d_ff, self.hp)
         with t.span("hessian"):
             L.clha_collect(ctx, self.acc_dn, layer, self.hp, self.P, self.d_ff, seg, E, 0)
         if self.n_shared:
-            with t.span("hessian"):
-                L.clha_collect(ctx, self.acc_in, layer, X, n, self.d_model, None, 1, E)
             hs = self.hs[:n]
             for i in range(self.n_shared):
                 with t.span("act"):
@@ -288,9 +293,12 @@ class MoECalibration:
                     L.clha_collect(ctx, self.acc_sdn, layer, hs, n, self.shared_dff, None, 1, i)
 
     # ------------------------------------------------------------------ phases 2 and 3
-    def quantize(self, w: MoEWeights, modes=None, alpha=None, with_loss: bool = True):
+    def quantize(self, w: MoEWeights, modes=None, alpha=None, with_loss: bool = True, on_output=None):
         """Aggregate, factor, GPTQ and score for each weighting in `modes` (a name or a tuple of the
-        weightings given at construction; default all of them)."""
+        weightings given at construction; default all of them). on_output(mode, part) (optional) is
+        called after each GPTQ call is queued, part one of "gu", "d", "sgu", "sd" (the QuantOut fields
+        of self.res[mode]), so that a caller can start copying those outputs while the next call runs."""
+        notify = on_output if on_output is not None else (lambda mode, part: None)
         if modes is None:
             modes = self.modes
         if isinstance(modes, str):
@@ -334,14 +342,18 @@ class MoECalibration:
                 q = r.qgu
                 L.clha_quantize(ctx, self.U_in[es], E, w.Wgu, 2 * E, dff, dm, br, q.codes, q.scales, q.zeros, q.W_hat,
                                 **opt(self.lam_in[es], lb[0:2 * E]))
+                notify(m, "gu")
                 L.clha_quantize(ctx, self.U_dn[es], E, w.Wd, E, dm, dff, br, r.qd.codes, r.qd.scales, r.qd.zeros,
                                 r.qd.W_hat, **opt(self.lam_dn[es], lb[2 * E:3 * E]))
+                notify(m, "d")
                 if ns:
                     q = r.sgu
                     L.clha_quantize(ctx, self.U_sin[i:i + 1], 1, w.Sgu, 2 * ns, sdff, dm, bs, q.codes, q.scales,
                                     q.zeros, q.W_hat, **opt(self.lam_sin[i:i + 1], lb[3 * E:3 * E + 2 * ns]))
+                    notify(m, "sgu")
                     L.clha_quantize(ctx, self.U_sdn[ss], ns, w.Sd, ns, dm, sdff, bs, r.sd.codes, r.sd.scales,
                                     r.sd.zeros, r.sd.W_hat, **opt(self.lam_sdn[ss], lb[3 * E + 2 * ns:]))
+                    notify(m, "sd")
             self._last = r
         if with_loss:      # one read of every weighting's losses
             host = self.loss_dev.cpu().numpy()
@@ -376,6 +388,82 @@ def stack_weights(wl, device) -> MoEWeights:
     if shared:
         return MoEWeights(gu(routed), dn(routed), gu(shared), dn(shared))
     return MoEWeights(gu(routed), dn(routed))
+
+
+PART_FIELDS = {"gu": "qgu", "d": "qd", "sgu": "sgu", "sd": "sd"}   # on_output part -> MoEResult field
+
+
+class HostStep:
+    """One MoE calibration step from pinned host memory to pinned host memory, the copies overlapped
+    with the compute. Host→device copies run on a copy stream in the order the compute needs them:
+    layer 0's tokens and logits, the gate/up weights (the first step that reads weights is layer 0's
+    expert activation), the other layers' tokens, then the down and always-active weights; the
+    compute stream (the context's) waits on an event before each first use. Each GPTQ call's codes,
+    scales and zeros go back on the copy stream as soon as that call is queued, while the next one
+    runs. Device copies of the inputs are owned here and reused by every step; the next step's input
+    copies wait until the previous step's compute has finished.
+    """
+
+    def __init__(self, cal: MoECalibration, x_shapes, logit_shapes, w_host: MoEWeights, x_dtype=torch.bfloat16):
+        self.cal = cal
+        dev = cal.dev
+        self.copy = torch.cuda.Stream(device=dev)
+        self.dX = [torch.empty(sh, dtype=x_dtype, device=dev) for sh in x_shapes]
+        self.dL = [torch.empty(sh, dtype=torch.float32, device=dev) for sh in logit_shapes]
+        like = lambda t: None if t is None else torch.empty(t.shape, dtype=t.dtype, device=dev)
+        self.w = MoEWeights(like(w_host.Wgu), like(w_host.Wd), like(w_host.Sgu), like(w_host.Sd))
+
+    def _ev(self):
+        return torch.cuda.Event()
+
+    def run(self, hX, hL, hW: MoEWeights, hout: dict, modes=None, alpha=None):
+        """hX, hL: per-layer pinned host tokens and logits; hW: pinned host weights; hout[mode][part]
+        = (codes, scales, zeros) pinned host tensors for the parts ("gu", "d", "sgu", "sd") to bring
+        back. Everything is queued; the caller synchronises with the context's stream."""
+        cal, cs, comp = self.cal, self.copy, self.cal.ctx.stream
+        start = self._ev()
+        start.record(comp)
+        cs.wait_event(start)           # the previous step no longer reads the device inputs
+        ev_in, ev_gu, ev_rest = [], self._ev(), self._ev()
+        with torch.cuda.stream(cs):
+            for l, (dx, dl, hx, hl) in enumerate(zip(self.dX, self.dL, hX, hL)):
+                dx.copy_(hx, non_blocking=True)
+                dl.copy_(hl, non_blocking=True)
+                ev_in.append(self._ev())
+                ev_in[-1].record(cs)
+                if l == 0:
+                    self.w.Wgu.copy_(hW.Wgu, non_blocking=True)
+                    if hW.Sgu is not None:
+                        self.w.Sgu.copy_(hW.Sgu, non_blocking=True)
+                    ev_gu.record(cs)
+            self.w.Wd.copy_(hW.Wd, non_blocking=True)
+            if hW.Sd is not None:
+                self.w.Sd.copy_(hW.Sd, non_blocking=True)
+            ev_rest.record(cs)
+        cal.reset()
+        for l in range(len(self.dX)):
+            comp.wait_event(ev_in[l])
+            n = hX[l].shape[0]
+            cal.collect(l, self.dX[l][:n], self.dL[l][:n], self.w,
+                        before_act=(lambda: comp.wait_event(ev_gu)) if l == 0 else None)
+        comp.wait_event(ev_rest)
+
+        def on_output(mode, part):
+            outs = hout.get(mode, {}).get(part)
+            if outs is None:
+                return
+            ready = self._ev()
+            ready.record(comp)
+            cs.wait_event(ready)
+            q = getattr(cal.res[mode], PART_FIELDS[part])
+            with torch.cuda.stream(cs):
+                for h, d in zip(outs, (q.codes, q.scales, q.zeros)):
+                    h.copy_(d, non_blocking=True)
+
+        cal.quantize(self.w, modes, alpha, on_output=on_output)
+        done = self._ev()
+        done.record(cs)
+        comp.wait_event(done)
 
 
 class EPMQCalibration:
