@@ -40,7 +40,8 @@
 namespace {
 
 constexpr int NB = 64;
-constexpr int LD = NB + 4;   // padded shared row (doubles): conflict-free m8n8k4 fragment loads
+constexpr int LD = NB + 8;   // padded shared row (doubles): the 16-byte fragment loads of two adjacent
+                             // rows fall in opposite halves of the banks (conflict-free)
 constexpr int TILE_DOUBLES = NB * LD;
 constexpr int TILE_ELEMS = NB * NB;
 constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;
@@ -124,7 +125,11 @@ __device__ __forceinline__ void tile_to_smem(Tile* dst, const double* __restrict
 }
 
 // C (global tile, row-major 64x64) <- (load_c ? C : 0) + sign * P Q^T. The operand copies into shared
-// memory and the loads of this thread's C fragments are all in flight together.
+// memory and the loads of this thread's C fragments are all in flight together. A negative sign is
+// applied to C on the way in and out (C - PQ^T = -(-C + PQ^T)), not to every operand fragment. Each
+// 16-byte shared load feeds two k-steps: in the k-block k0..k0+7 lane tq supplies k0+2tq to the
+// first m8n8k4 product and k0+2tq+1 to the second (the same k for its A and B fragments), so the
+// two products together cover the block.
 __device__ __forceinline__ void tile_gemm_nt(const double* __restrict__ Pg, const double* __restrict__ Qg, Tile* Ps,
                                              Tile* Qs, double* C, bool load_c, bool negate) {
     tile_to_smem(Ps, Pg);
@@ -141,35 +146,36 @@ __device__ __forceinline__ void tile_gemm_nt(const double* __restrict__ Pg, cons
             if (load_c) {
                 const double2 v = __ldcg(reinterpret_cast<const double2*>(
                     C + (32 * wm + 8 * mi + g) * NB + 16 * wn + 8 * ni + 2 * tq));
-                c[mi][ni][0] = v.x;
-                c[mi][ni][1] = v.y;
+                c[mi][ni][0] = negate ? -v.x : v.x;
+                c[mi][ni][1] = negate ? -v.y : v.y;
             } else {
                 c[mi][ni][0] = c[mi][ni][1] = 0.0;
             }
         }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
-#pragma unroll 4
-    for (int k0 = 0; k0 < NB; k0 += 4) {
-        double a[4], bq[2];
+#pragma unroll 2
+    for (int k0 = 0; k0 < NB; k0 += 8) {
+        double2 a[4], bq[2];
 #pragma unroll
-        for (int mi = 0; mi < 4; ++mi) {
-            a[mi] = Ps[32 * wm + 8 * mi + g][k0 + tq];
-            if (negate) a[mi] = -a[mi];
-        }
+        for (int mi = 0; mi < 4; ++mi) a[mi] = *reinterpret_cast<const double2*>(&Ps[32 * wm + 8 * mi + g][k0 + 2 * tq]);
 #pragma unroll
-        for (int ni = 0; ni < 2; ++ni) bq[ni] = Qs[16 * wn + 8 * ni + g][k0 + tq];
+        for (int ni = 0; ni < 2; ++ni) bq[ni] = *reinterpret_cast<const double2*>(&Qs[16 * wn + 8 * ni + g][k0 + 2 * tq]);
 #pragma unroll
         for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
-            for (int ni = 0; ni < 2; ++ni) dmma(c[mi][ni][0], c[mi][ni][1], a[mi], bq[ni]);
+            for (int ni = 0; ni < 2; ++ni) dmma(c[mi][ni][0], c[mi][ni][1], a[mi].x, bq[ni].x);
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+            for (int ni = 0; ni < 2; ++ni) dmma(c[mi][ni][0], c[mi][ni][1], a[mi].y, bq[ni].y);
     }
 #pragma unroll
     for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
         for (int ni = 0; ni < 2; ++ni)
             *reinterpret_cast<double2*>(C + (32 * wm + 8 * mi + g) * NB + 16 * wn + 8 * ni + 2 * tq) =
-                make_double2(c[mi][ni][0], c[mi][ni][1]);
+                negate ? make_double2(-c[mi][ni][0], -c[mi][ni][1]) : make_double2(c[mi][ni][0], c[mi][ni][1]);
 }
 
 // Cholesky of the 64x64 tile in T (lower, in place), its inverse X = L^-1; writes L to Lg, X to Dg,
@@ -371,7 +377,7 @@ __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
     Tile* T1 = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
     double* dinv = dsm + 2 * TILE_DOUBLES;
     unsigned long long* lvl = reinterpret_cast<unsigned long long*>(dinv + NB);   // [max_nt + 2] stage starts
-    __shared__ unsigned long long s_ticket;
+    __shared__ unsigned long long s_ticket, s_next;   // s_next: thread 0's prefetched number
     __shared__ int s_ok;
     const int S = g.max_nt, tid = threadIdx.x, lane = tid & 31;
     if (tid == 0) {   // stage s holds, group after group, stage s of every group that has one
@@ -384,16 +390,15 @@ __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
     }
     // Thread 0 holds the next number while the CTA runs the current task (taking numbers in order
     // and running them in order keeps the schedule deadlock-free).
-    unsigned long long next = 0;
-    if (tid == 0) next = atomicAdd(g.ticket, 1ull);
+    // The number of the next task is published in s_ticket before the barrier that ends the current
+    // one (every thread has read the current number before the dependency barrier).
+    if (tid == 0) s_ticket = atomicAdd(g.ticket, 1ull);
     __syncthreads();
 
     for (;;) {
-        if (tid == 0) s_ticket = *reinterpret_cast<volatile int*>(g.abort_flag) ? g.total : next;
-        __syncthreads();
         const unsigned long long t = s_ticket;
         if (t >= g.total) break;
-        if (tid == 0) next = atomicAdd(g.ticket, 1ull);
+        if (tid == 0) s_next = atomicAdd(g.ticket, 1ull);
         // decode: stage, group, class, problem, task (q: 0 P, 1 S, 2/5 G, 3 F, 4 Q), level m, tiles i, j
         int lo = 0, hi = S;
         while (lo < hi) {
@@ -501,6 +506,7 @@ __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
         } else {
             tile_gemm_nt(P, Qm, T0, T1, C, load_c, negate);
         }
+        if (tid == 0) s_ticket = *reinterpret_cast<volatile int*>(g.abort_flag) ? g.total : s_next;
         __syncthreads();   // every thread's stores issued; shared tiles free for the next task
         if (tid == 0) st_release(out_state, out_value);   // release: cumulative over the CTA's stores
     }
