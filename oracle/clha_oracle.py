@@ -32,7 +32,9 @@ Readings where the pages are silent (each also listed in the design notes):
     around those decisions stays float64.
   * columns are quantized in natural order (no activation reordering).
   * a layer with no tokens contributes a zero Hessian; an expert with no tokens in any layer is an
-    error (there is nothing to calibrate on).
+    error (there is nothing to calibrate on), or, on request, is quantized by round to nearest
+    (H_d = I), as is an expert whose weighted aggregate has no energy (per-layer calibration of an
+    expert that the hook layer never routes to).
   * deployable codes are packed per row as one little-endian bit stream of 32-bit words, code j at
     bits [b*j, b*j + b) (the pages give no layout); W_hat = s (q - z) per group in float32.
   * cross-layer routing divergence (CLHA page §4-5: the gains grow with it; no formula is given) is
@@ -126,20 +128,24 @@ def ffn_act(Xe, Wg, Wu):
 
 
 # ----------------------------------------------------------------------------------- phase 2
-def aggregate(S_list, n_list, mode: str = "rt", alpha=None, damp_frac: float = 0.01):
+def aggregate(S_list, n_list, mode: str = "rt", alpha=None, damp_frac: float = 0.01, empty: str = "error"):
     """Cross-layer aggregation (CLHA page §2.1 Proposition 1, §2.2 (2)) and damping.
 
     mode "rt": alpha_i = n_i / sum_j n_j; "eq": alpha_i = 1/L (0.5 for a pair);
     "explicit": alpha given (e.g. (1, 0) for per-layer calibration on the first layer only).
     Returns dict(alpha, H_comb, lam, H_d) with H_comb = sum_i alpha_i (2/n_i) S_i,
     lam = damp_frac * mean(diag H_comb), H_d = H_comb + lam I.
+    empty: what an aggregate without energy (no tokens at all, or none in the layers that carry
+    weight) becomes. "error" raises when no layer has tokens; "identity" gives H_comb = 0, lam = 1,
+    H_d = I, under which GPTQ is round to nearest (a reading: the harness quantizes an expert that
+    the calibration data never reach by RTN).
     """
     L = len(S_list)
     n = np.asarray(n_list, dtype=np.int64)
-    if n.sum() == 0:
+    if n.sum() == 0 and empty != "identity":
         raise ValueError("no tokens in any layer")
     if mode == "rt":
-        a = n / n.sum()
+        a = n / n.sum() if n.sum() > 0 else np.zeros(L)
     elif mode == "eq":
         a = np.full(L, 1.0 / L)
     elif mode == "explicit":
@@ -152,6 +158,8 @@ def aggregate(S_list, n_list, mode: str = "rt", alpha=None, damp_frac: float = 0
     for ai, Si, ni in zip(a, S_list, n):
         H_comb += ai * hessian(Si, int(ni))
     lam = damp_frac * float(np.mean(np.diag(H_comb)))
+    if empty == "identity" and np.trace(H_comb) == 0.0:
+        lam = 1.0
     H_d = H_comb + lam * np.eye(H_comb.shape[0])
     return {"alpha": a, "H_comb": H_comb, "lam": lam, "H_d": H_d}
 
@@ -251,7 +259,8 @@ def calibrate_dense(W, X_list, bits: int, group: int = 128, mode: str = "rt", al
 
 def calibrate_moe_group(X_list, logits_list, k: int, routed, shared=(), experts=None,
                         bits_routed: int = 2, bits_shared: int = 3, group: int = 128,
-                        mode: str = "rt", damp_frac: float = 0.01, shared_experts=None):
+                        mode: str = "rt", damp_frac: float = 0.01, shared_experts=None, alpha=None,
+                        empty: str = "error"):
     """CLHA on one group of layers sharing routed experts `routed` [(Wg, Wu, Wd)] and always-active
     experts `shared` (CLHA page §2.2 phases 1-3, §2.3 mixed precision, §2.4 per-layer accumulators).
 
@@ -278,7 +287,7 @@ def calibrate_moe_group(X_list, logits_list, k: int, routed, shared=(), experts=
         res = {"n": n}
         for kind, inputs, mats in (("H_in", Xe, (("gate", Wg), ("up", Wu))), ("H_down", he, (("down", Wd),))):
             S = [gram(x) for x in inputs]
-            agg = aggregate(S, n, mode, None, damp_frac)
+            agg = aggregate(S, n, mode, alpha, damp_frac, empty)
             U = factor(agg["H_d"])
             res[kind] = {"S": S, **agg, "U": U}
             for name, Wm in mats:

@@ -159,6 +159,29 @@ def test_aggregate_rejects_empty():
         O.aggregate([np.eye(2), np.eye(2)], [0, 0], "rt")
 
 
+def test_empty_aggregate_as_identity():
+    """No tokens at all, or none in the only weighted layer: H_comb = 0, lambda = 1, H_d = I, and GPTQ
+    under it gives the codes of GPTQ under any diagonal Hessian (round to nearest, pinned below)."""
+    d = 8
+    S = [np.zeros((d, d)), 3.0 * np.eye(d)]
+    for n, mode, alpha in (([0, 0], "rt", None), ([0, 0], "eq", None), ([0, 5], "explicit", (1.0, 0.0))):
+        agg = O.aggregate(S, n, mode, alpha, empty="identity")
+        np.testing.assert_array_equal(agg["H_comb"], 0.0)
+        assert agg["lam"] == 1.0
+        np.testing.assert_array_equal(agg["H_d"], np.eye(d))
+    W = 0.02 * RNG.standard_normal((4, 128))
+    S128 = [np.zeros((128, 128)), 3.0 * np.eye(128)]
+    U = O.factor(O.aggregate(S128, [0, 5], "explicit", (1.0, 0.0), empty="identity")["H_d"])
+    c_id = O.gptq(W, U, 3, 128)[0]
+    c_diag = O.gptq(W, O.factor(np.diag(RNG.uniform(0.5, 2.0, 128))), 3, 128)[0]
+    np.testing.assert_array_equal(c_id, c_diag)
+    # with energy the policy changes nothing
+    S2 = [_spd(d, seed=5), _spd(d, seed=6)]
+    a, b = O.aggregate(S2, [7, 9], "rt"), O.aggregate(S2, [7, 9], "rt", empty="identity")
+    np.testing.assert_array_equal(a["H_d"], b["H_d"])
+    assert a["lam"] == b["lam"]
+
+
 # ------------------------------------------------------------------------------------ factor
 @pytest.mark.parametrize("d", [1, 5, 64])
 def test_factor_inverse_cholesky(d):
