@@ -659,7 +659,7 @@ def main():
                     default="moe",
                     help="moe: the end-to-end calibration step (default); sweep: the routing-sharpness "
                          "experiment; others: one kernel family")
-    ap.add_argument("--sharpness", type=float, nargs="+", default=[0.0, 0.1, 0.2, 0.3, 0.4, 0.5],
+    ap.add_argument("--sharpness", type=float, nargs="+", default=[0.0, 0.1, 0.2, 0.3, 0.5, 0.75, 1.0],
                     help="sweep: strengths of the per-layer expert preference")
     ap.add_argument("--shape", nargs="+", default=[], help="kernel workload shapes, e.g. 65536x4096")
     args = ap.parse_args()

@@ -60,8 +60,14 @@ typedef enum {
     CLHA_ALPHA_ROUTING = 0,   /* alpha_i = n_i / sum_j n_j           (CLHA page §2.2 (2), "rt") */
     CLHA_ALPHA_EQUAL = 1,     /* alpha_i = 1 / n_layers              (CLHA page §2.2 (2), "eq") */
     CLHA_ALPHA_EXPLICIT = 2,  /* alpha from the caller; (1, 0) is per-layer calibration on layer 0 */
-    CLHA_ALPHA_SUM = 3        /* alpha_i = n_i / 2, so H_comb = sum_i S_i: the unnormalised Gram sum
+    CLHA_ALPHA_SUM = 3,       /* alpha_i = n_i / 2, so H_comb = sum_i S_i: the unnormalised Gram sum
                                  of the E-PMQ statistics (the E-PMQ page, section 2) */
+    /* Flag, or'ed into one of the modes above: a slot whose weighted aggregate has no energy
+     * (tr H_comb = 0: no tokens in any layer, or none in the layers with nonzero alpha) gets
+     * H_comb = 0, lambda = 1 and H_damped = I instead of CLHA_ERR_EMPTY (no tokens at all) or a zero
+     * H_damped that clha_factor rejects. GPTQ under H_damped = I is round to nearest: the calibration
+     * data say nothing about that expert. Its loss under H_comb is 0. */
+    CLHA_AGG_EMPTY_IDENTITY = 0x100
 } clha_alpha_mode;
 
 /* GPTQ parameters: bits in 2..8, group = 128 (grid per 128 input columns), block = 128 (lazy-update

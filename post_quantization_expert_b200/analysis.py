@@ -62,7 +62,8 @@ class HessianError:
         """{"routed": [E] gate + up + down losses, "shared": [n_shared] the same for the always-active
         experts} under the `mode` (alpha for "explicit") aggregate of cal's accumulators."""
         ctx, E, dm, dff = self.ctx, self.E, self.d_model, self.d_ff
-        m, dmp = MODES[mode], 0.01      # the damped aggregate is scratch: only H_comb is scored
+        # the damped aggregate is scratch (only H_comb is scored); an expert without tokens scores 0
+        m, dmp = MODES[mode] | L.AGG_EMPTY_IDENTITY, 0.01
         L.clha_aggregate(ctx, cal.acc_in, 0, E, m, alpha, dmp, self.Hc_in, self.Hd_in)
         L.clha_aggregate(ctx, cal.acc_dn, 0, E, m, alpha, dmp, self.Hc_dn, self.Hd_dn)
         gu = L.clha_loss(ctx, w.Wgu, r.qgu.W_hat, self.Hc_in, E, 2 * E, dff, dm)

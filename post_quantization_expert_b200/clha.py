@@ -22,6 +22,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_NOT_PD, ERR_NONFINITE, ERR_EMPTY
 STATUS_NAMES = ["OK", "INVALID_ARG", "UNSUPPORTED_SHAPE", "NOT_PD", "NONFINITE", "EMPTY", "OOM", "CUDA", "TIMEOUT"]
 BF16, F32 = 0, 1
 ALPHA_ROUTING, ALPHA_EQUAL, ALPHA_EXPLICIT, ALPHA_SUM = 0, 1, 2, 3
+AGG_EMPTY_IDENTITY = 0x100   # or'ed into an alpha mode: an aggregate without energy becomes H_d = I
 
 # every symbol include/clha.h declares
 SYMBOLS = [

@@ -1,7 +1,8 @@
 // Phase 2 of CLHA (the CLHA page, §2.1 Proposition 1 and §2.2 (2)): H_comb = sum_i alpha_i H_i with
 // H_i = (2 / n_i) S_i, routing-frequency (alpha_i = n_i / sum n), equal (1/L) or explicit weights,
 // or the plain Gram sum (alpha_i = n_i / 2, H_comb = sum S_i: the E-PMQ statistics), then GPTQ
-// damping H_d = H_comb + lambda I, lambda = damp_frac * mean(diag H_comb).
+// damping H_d = H_comb + lambda I, lambda = damp_frac * mean(diag H_comb); on request a slot without
+// energy (tr H_comb = 0) gets lambda = 1, so H_d = I and GPTQ under it is round to nearest.
 //
 // Two kernels per call, both HBM-bound:
 //   agg_scalars  one block per slot: alpha (float64), lambda from the diagonals (float64 reduction),
@@ -26,6 +27,8 @@ __global__ void __launch_bounds__(256) agg_scalars(const float* __restrict__ S, 
     __shared__ double alpha[CLHA_MAX_LAYERS];
     __shared__ int64_t cnt[CLHA_MAX_LAYERS];
     __shared__ double red[256];
+    const int amode = a.mode & 0xff;
+    const bool identity = (a.mode & CLHA_AGG_EMPTY_IDENTITY) != 0;
     if (threadIdx.x == 0) {
         int64_t tot = 0;
         for (int l = 0; l < L; ++l) {
@@ -34,14 +37,14 @@ __global__ void __launch_bounds__(256) agg_scalars(const float* __restrict__ S, 
         }
         for (int l = 0; l < L; ++l) {
             double al;
-            if (a.mode == CLHA_ALPHA_ROUTING) al = tot > 0 ? (double)cnt[l] / (double)tot : 0.0;
-            else if (a.mode == CLHA_ALPHA_EQUAL) al = 1.0 / L;
-            else if (a.mode == CLHA_ALPHA_SUM) al = (double)cnt[l] / 2.0;
+            if (amode == CLHA_ALPHA_ROUTING) al = tot > 0 ? (double)cnt[l] / (double)tot : 0.0;
+            else if (amode == CLHA_ALPHA_EQUAL) al = 1.0 / L;
+            else if (amode == CLHA_ALPHA_SUM) al = (double)cnt[l] / 2.0;
             else al = a.alpha[l];
             alpha[l] = al;
             d_alpha[(size_t)sl * L + l] = al;
         }
-        if (tot == 0) clha_record_error(err, CLHA_ERR_EMPTY, slot, 0, KID_AGGREGATE);
+        if (tot == 0 && !identity) clha_record_error(err, CLHA_ERR_EMPTY, slot, 0, KID_AGGREGATE);
     }
     __syncthreads();
     double acc = 0.0;
@@ -61,6 +64,7 @@ __global__ void __launch_bounds__(256) agg_scalars(const float* __restrict__ S, 
     }
     if (threadIdx.x == 0) {
         double lam = damp_frac * red[0] / d;
+        if (identity && red[0] == 0.0) lam = 1.0;   // no energy: H_d = I (round to nearest)
         d_lambda[sl] = lam;
         if (!isfinite(red[0])) clha_record_error(err, CLHA_ERR_NONFINITE, slot, -1, KID_AGGREGATE);
     }

@@ -348,18 +348,20 @@ extern "C" clha_status clha_aggregate(clha_ctx* ctx, const clha_accum* acc, int 
     REQUIRE(acc && H_damped, CLHA_ERR_INVALID_ARG, "clha_aggregate: null pointer");
     REQUIRE(n_slots >= 1 && slot0 >= 0 && slot0 + n_slots <= acc->n_slots, CLHA_ERR_INVALID_ARG,
             "clha_aggregate: slots outside the accumulator");
-    REQUIRE(mode == CLHA_ALPHA_ROUTING || mode == CLHA_ALPHA_EQUAL || mode == CLHA_ALPHA_EXPLICIT ||
-                mode == CLHA_ALPHA_SUM,
+    const int amode = (int)mode & 0xff;
+    REQUIRE(((int)mode & ~(0xff | CLHA_AGG_EMPTY_IDENTITY)) == 0 &&
+                (amode == CLHA_ALPHA_ROUTING || amode == CLHA_ALPHA_EQUAL || amode == CLHA_ALPHA_EXPLICIT ||
+                 amode == CLHA_ALPHA_SUM),
             CLHA_ERR_INVALID_ARG, "clha_aggregate: unknown alpha mode");
-    REQUIRE(mode != CLHA_ALPHA_EXPLICIT || alpha_in, CLHA_ERR_INVALID_ARG, "clha_aggregate: explicit alpha needs alpha_in");
+    REQUIRE(amode != CLHA_ALPHA_EXPLICIT || alpha_in, CLHA_ERR_INVALID_ARG, "clha_aggregate: explicit alpha needs alpha_in");
     REQUIRE(damp_frac > 0.0 && damp_frac == damp_frac, CLHA_ERR_INVALID_ARG, "clha_aggregate: damp_frac must be > 0");
     SET_DEVICE(ctx);
     LaunchScope launch_scope(ctx);
     clha_alpha_args a;
     memset(&a, 0, sizeof(a));
-    a.mode = mode;
+    a.mode = (int)mode;
     a.n_layers = acc->n_layers;
-    if (mode == CLHA_ALPHA_EXPLICIT)
+    if (amode == CLHA_ALPHA_EXPLICIT)
         for (int i = 0; i < acc->n_layers; ++i) a.alpha[i] = alpha_in[i];
     size_t need = clha_round_up((size_t)n_slots * acc->n_layers * sizeof(double)) +
                   clha_round_up((size_t)n_slots * sizeof(double));

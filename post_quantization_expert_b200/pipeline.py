@@ -192,8 +192,13 @@ class MoECalibration:
 
     def __init__(self, ctx: L.Context, n_layers: int, max_tokens: int, E: int, k: int, d_model: int, d_ff: int,
                  n_shared: int = 0, shared_dff: int = 0, bits_routed: int = 2, bits_shared: int = 3,
-                 damp_frac: float = 0.01, timer=NO_TIMER, modes=("rt",), keep_hcomb: bool = False):
+                 damp_frac: float = 0.01, timer=NO_TIMER, modes=("rt",), keep_hcomb: bool = False,
+                 unrouted_rtn: bool = True):
+        """unrouted_rtn: an expert whose weighted Hessian aggregate is empty (never routed, or, for
+        explicit alpha, never routed in the weighted layers) is quantized by round to nearest
+        (H_d = I, loss 0) instead of failing."""
         self.ctx, self.n_layers, self.E, self.k = ctx, n_layers, E, k
+        self.agg_flag = L.AGG_EMPTY_IDENTITY if unrouted_rtn else 0
         self.timer = timer
         self.d_model, self.d_ff, self.n_shared, self.shared_dff = d_model, d_ff, n_shared, shared_dff
         self.bits_routed, self.bits_shared, self.damp = bits_routed, bits_shared, damp_frac
@@ -310,15 +315,16 @@ class MoECalibration:
         with t.span("aggregate"):
             for i, m in zip(idx, modes):
                 es, ss = slice(i * E, (i + 1) * E), slice(i * ns, (i + 1) * ns)
-                L.clha_aggregate(ctx, self.acc_in, 0, E, MODES[m], alpha, self.damp, opt(self.Hc_in, es),
+                am = MODES[m] | self.agg_flag
+                L.clha_aggregate(ctx, self.acc_in, 0, E, am, alpha, self.damp, opt(self.Hc_in, es),
                                  self.Hd_in[es], lambda_dev=self.lam_in[es])
-                L.clha_aggregate(ctx, self.acc_dn, 0, E, MODES[m], alpha, self.damp, opt(self.Hc_dn, es),
+                L.clha_aggregate(ctx, self.acc_dn, 0, E, am, alpha, self.damp, opt(self.Hc_dn, es),
                                  self.Hd_dn[es], lambda_dev=self.lam_dn[es])
                 if ns:
-                    L.clha_aggregate(ctx, self.acc_in, E, 1, MODES[m], alpha, self.damp,
+                    L.clha_aggregate(ctx, self.acc_in, E, 1, am, alpha, self.damp,
                                      opt(self.Hc_sin, slice(i, i + 1)), self.Hd_sin[i:i + 1],
                                      lambda_dev=self.lam_sin[i:i + 1])
-                    L.clha_aggregate(ctx, self.acc_sdn, 0, ns, MODES[m], alpha, self.damp, opt(self.Hc_sdn, ss),
+                    L.clha_aggregate(ctx, self.acc_sdn, 0, ns, am, alpha, self.damp, opt(self.Hc_sdn, ss),
                                      self.Hd_sdn[ss], lambda_dev=self.lam_sdn[ss])
         # one batched factor per Hessian kind over every requested weighting (contiguous runs)
         lo, hi = min(idx), max(idx) + 1

@@ -112,3 +112,48 @@ def test_moe_pair_E64_top6_shared_reduced_tokens(ctx):
     """The E=64 top-6 shape with two always-active experts (CLHA-MP: routed 2-bit, shared 3-bit),
     Zipf-skewed routing and outlier channels, at 4096 tokens per layer."""
     _moe_pair(ctx, 3, [0, 63], ("rt",), shared_checked=[1], tokens=4096)
+
+
+def test_unrouted_experts_are_round_to_nearest(ctx):
+    """An expert the router never picks (expert 3) and, under per-layer calibration on layer 0, an
+    expert picked only in layer 1 (expert 5): their aggregates have no energy, so both sides quantize
+    them by round to nearest (H_d = I) with zero loss; a routed expert (0) alongside is unaffected."""
+    wl = workload(2, "cpu", tokens=1024)
+    s = wl.spec
+    Xs = [wl.x(l) for l in range(2)]
+    lgs = [wl.logits(l).clone() for l in range(2)]
+    for lg in lgs:
+        lg[:, 3] = -1.0e4
+    lgs[0][:, 5] = -1.0e4
+    routed = [wl.expert_weights(0, e) for e in range(s.E)]
+    w = stack_weights((routed, []), DEV)
+    modes = ("rt", "explicit")
+    cal = MoECalibration(ctx, 2, 1024, s.E, s.k, s.d_model, s.d_ff, 0, 0, s.bits_routed, s.bits_shared,
+                         s.damp_frac, modes=modes)
+    for l in range(2):
+        cal.collect(l, Xs[l].to(DEV), lgs[l].to(DEV), w)
+    cal.quantize(w, modes, alpha=(1.0, 0.0))
+    torch.cuda.synchronize()
+    cnt = cal.counts.cpu().numpy()
+    assert cnt[0, 3] == 0 and cnt[1, 3] == 0 and cnt[0, 5] == 0 and cnt[1, 5] > 0
+    X64 = [to64(X) for X in Xs]
+    W64 = [tuple(to64(t) for t in r) for r in routed]
+    # (expert 0 is checked under rt only: alone, layer 0 gives it ~128 tokens in 1024 dimensions, a
+    # Hessian so ill-conditioned that float32 GPTQ and the float64 oracle part ways on ~0.1 % of codes)
+    for mode, alpha, experts in (("rt", None, (3, 0)), ("explicit", (1.0, 0.0), (3, 5))):
+        ref = O.calibrate_moe_group(X64, [lg.numpy() for lg in lgs], s.k, W64, (), list(experts), s.bits_routed,
+                                    s.bits_shared, s.group, mode, s.damp_frac, alpha=alpha, empty="identity")
+        r = cal.res[mode]
+        for e in experts:
+            want = ref["experts"][("r", e)]
+            for name, q in (("gate", r.qg), ("up", r.qu), ("down", r.qd)):
+                assert code_agreement(q.codes[e].cpu().numpy(), want[name]["codes"]) >= 0.999, (mode, e, name)
+            got = r.expert_loss()[e]
+            if e == 0:
+                assert abs(got - want["loss"]) <= 1e-3 * want["loss"]
+            else:
+                # the in-kernel loss is |E|^2 - lambda |W_hat - W|^2 with E = W - W_hat here: zero up
+                # to the float32 rounding of the two sums
+                err2 = sum(float(((q.W_hat[e].double() - Wm.double().to(DEV)) ** 2).sum())
+                           for q, Wm in ((r.qg, routed[e][0]), (r.qu, routed[e][1]), (r.qd, routed[e][2])))
+                assert want["loss"] == 0.0 and abs(got) <= 1e-5 * err2, (mode, e, got, err2)
