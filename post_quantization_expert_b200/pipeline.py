@@ -298,11 +298,14 @@ class MoECalibration:
                     L.clha_collect(ctx, self.acc_sdn, layer, hs, n, self.shared_dff, None, 1, i)
 
     # ------------------------------------------------------------------ phases 2 and 3
-    def quantize(self, w: MoEWeights, modes=None, alpha=None, with_loss: bool = True, on_output=None):
+    def quantize(self, w: MoEWeights, modes=None, alpha=None, with_loss: bool = True, on_output=None,
+                 read_loss: bool = True):
         """Aggregate, factor, GPTQ and score for each weighting in `modes` (a name or a tuple of the
         weightings given at construction; default all of them). on_output(mode, part) (optional) is
         called after each GPTQ call is queued, part one of "gu", "d", "sgu", "sd" (the QuantOut fields
-        of self.res[mode]), so that a caller can start copying those outputs while the next call runs."""
+        of self.res[mode]), so that a caller can start copying those outputs while the next call runs.
+        read_loss=False leaves the losses in self.loss_dev (nothing synchronises) instead of reading
+        them into the results."""
         notify = on_output if on_output is not None else (lambda mode, part: None)
         if modes is None:
             modes = self.modes
@@ -361,7 +364,7 @@ class MoECalibration:
                                     r.sd.zeros, r.sd.W_hat, **opt(self.lam_sdn[ss], lb[3 * E + 2 * ns:]))
                     notify(m, "sd")
             self._last = r
-        if with_loss:      # one read of every weighting's losses
+        if with_loss and read_loss:      # one read of every weighting's losses
             host = self.loss_dev.cpu().numpy()
             for i, m in zip(idx, modes):
                 r, h = self.res[m], host[i]
@@ -400,76 +403,101 @@ PART_FIELDS = {"gu": "qgu", "d": "qd", "sgu": "sgu", "sd": "sd"}   # on_output p
 
 
 class HostStep:
-    """One MoE calibration step from pinned host memory to pinned host memory, the copies overlapped
-    with the compute. Host→device copies run on a copy stream in the order the compute needs them:
+    """MoE calibration steps from pinned host memory to pinned host memory, the copies overlapped with
+    the compute. Host→device copies run on an input stream in the order the compute needs them:
     layer 0's tokens and logits, the gate/up weights (the first step that reads weights is layer 0's
     expert activation), the other layers' tokens, then the down and always-active weights; the
     compute stream (the context's) waits on an event before each first use. Each GPTQ call's codes,
-    scales and zeros go back on the copy stream as soon as that call is queued, while the next one
-    runs. Device copies of the inputs are owned here and reused by every step; the next step's input
-    copies wait until the previous step's compute has finished.
+    scales and zeros, and at the end the losses, go back on an output stream as soon as the call is
+    queued, while the compute goes on. The device copies of the inputs come in `n_sets` sets used in
+    turn, so with two sets the next step's inputs are copied while the current step computes (a set
+    is refilled once the step that last used it has finished; outputs are rewritten only after the
+    previous step's copies of them are done). run() only queues work: nothing synchronises.
     """
 
-    def __init__(self, cal: MoECalibration, x_shapes, logit_shapes, w_host: MoEWeights, x_dtype=torch.bfloat16):
+    def __init__(self, cal: MoECalibration, x_shapes, logit_shapes, w_host: MoEWeights, x_dtype=torch.bfloat16,
+                 n_sets: int = 2):
         self.cal = cal
         dev = cal.dev
-        self.copy = torch.cuda.Stream(device=dev)
-        self.dX = [torch.empty(sh, dtype=x_dtype, device=dev) for sh in x_shapes]
-        self.dL = [torch.empty(sh, dtype=torch.float32, device=dev) for sh in logit_shapes]
+        self.inp = torch.cuda.Stream(device=dev)
+        self.out = torch.cuda.Stream(device=dev)
         like = lambda t: None if t is None else torch.empty(t.shape, dtype=t.dtype, device=dev)
-        self.w = MoEWeights(like(w_host.Wgu), like(w_host.Wd), like(w_host.Sgu), like(w_host.Sd))
+        self.sets = []
+        for _ in range(n_sets):
+            self.sets.append(dict(
+                X=[torch.empty(sh, dtype=x_dtype, device=dev) for sh in x_shapes],
+                L=[torch.empty(sh, dtype=torch.float32, device=dev) for sh in logit_shapes],
+                w=MoEWeights(like(w_host.Wgu), like(w_host.Wd), like(w_host.Sgu), like(w_host.Sd)),
+                free=None))                      # event: the last step that used this set has finished
+        self.step = 0
+        self.outputs_copied = None               # event: the previous step's outputs are on the host
 
-    def _ev(self):
-        return torch.cuda.Event()
-
-    def run(self, hX, hL, hW: MoEWeights, hout: dict, modes=None, alpha=None):
+    def run(self, hX, hL, hW: MoEWeights, hout: dict, modes=None, alpha=None, hloss=None):
         """hX, hL: per-layer pinned host tokens and logits; hW: pinned host weights; hout[mode][part]
         = (codes, scales, zeros) pinned host tensors for the parts ("gu", "d", "sgu", "sd") to bring
-        back. Everything is queued; the caller synchronises with the context's stream."""
-        cal, cs, comp = self.cal, self.copy, self.cal.ctx.stream
-        start = self._ev()
-        start.record(comp)
-        cs.wait_event(start)           # the previous step no longer reads the device inputs
-        ev_in, ev_gu, ev_rest = [], self._ev(), self._ev()
-        with torch.cuda.stream(cs):
-            for l, (dx, dl, hx, hl) in enumerate(zip(self.dX, self.dL, hX, hL)):
+        back; hloss (optional): pinned host float64 tensor shaped like the calibration's loss_dev.
+        Everything is queued; the caller synchronises with the context's stream."""
+        cal, comp = self.cal, self.cal.ctx.stream
+        st = self.sets[self.step % len(self.sets)]
+        self.step += 1
+        ev = torch.cuda.Event
+        if st["free"] is not None:
+            self.inp.wait_event(st["free"])      # the step that last read this set is done
+        ev_in, ev_gu, ev_rest = [], ev(), ev()
+        w = st["w"]
+        with torch.cuda.stream(self.inp):
+            for l, (dx, dl, hx, hl) in enumerate(zip(st["X"], st["L"], hX, hL)):
                 dx.copy_(hx, non_blocking=True)
                 dl.copy_(hl, non_blocking=True)
-                ev_in.append(self._ev())
-                ev_in[-1].record(cs)
+                ev_in.append(ev())
+                ev_in[-1].record(self.inp)
                 if l == 0:
-                    self.w.Wgu.copy_(hW.Wgu, non_blocking=True)
+                    w.Wgu.copy_(hW.Wgu, non_blocking=True)
                     if hW.Sgu is not None:
-                        self.w.Sgu.copy_(hW.Sgu, non_blocking=True)
-                    ev_gu.record(cs)
-            self.w.Wd.copy_(hW.Wd, non_blocking=True)
+                        w.Sgu.copy_(hW.Sgu, non_blocking=True)
+                    ev_gu.record(self.inp)
+            w.Wd.copy_(hW.Wd, non_blocking=True)
             if hW.Sd is not None:
-                self.w.Sd.copy_(hW.Sd, non_blocking=True)
-            ev_rest.record(cs)
+                w.Sd.copy_(hW.Sd, non_blocking=True)
+            ev_rest.record(self.inp)
         cal.reset()
-        for l in range(len(self.dX)):
+        for l in range(len(st["X"])):
             comp.wait_event(ev_in[l])
             n = hX[l].shape[0]
-            cal.collect(l, self.dX[l][:n], self.dL[l][:n], self.w,
+            cal.collect(l, st["X"][l][:n], st["L"][l][:n], w,
                         before_act=(lambda: comp.wait_event(ev_gu)) if l == 0 else None)
         comp.wait_event(ev_rest)
+        if self.outputs_copied is not None:
+            comp.wait_event(self.outputs_copied)   # the previous step's outputs have left the device
 
         def on_output(mode, part):
             outs = hout.get(mode, {}).get(part)
             if outs is None:
                 return
-            ready = self._ev()
+            ready = ev()
             ready.record(comp)
-            cs.wait_event(ready)
+            self.out.wait_event(ready)
             q = getattr(cal.res[mode], PART_FIELDS[part])
-            with torch.cuda.stream(cs):
+            with torch.cuda.stream(self.out):
                 for h, d in zip(outs, (q.codes, q.scales, q.zeros)):
                     h.copy_(d, non_blocking=True)
 
-        cal.quantize(self.w, modes, alpha, on_output=on_output)
-        done = self._ev()
-        done.record(cs)
-        comp.wait_event(done)
+        cal.quantize(w, modes, alpha, on_output=on_output, read_loss=hloss is None)
+        st["free"] = ev()
+        st["free"].record(comp)
+        if hloss is not None:
+            self.out.wait_event(st["free"])
+            with torch.cuda.stream(self.out):
+                hloss.copy_(cal.loss_dev, non_blocking=True)
+        done = ev()
+        done.record(self.out)
+        self.outputs_copied = done
+
+    def join(self):
+        """Make the context's stream wait for every copy queued so far (the outputs and losses of the
+        last step included), so that an event recorded on it after this covers them."""
+        if self.outputs_copied is not None:
+            self.cal.ctx.stream.wait_event(self.outputs_copied)
 
 
 class EPMQCalibration:

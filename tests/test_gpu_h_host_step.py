@@ -1,8 +1,8 @@
-"""The host-to-host calibration step (inputs copied in and outputs copied back on a side stream,
-overlapped with the compute) must give exactly what the same calls give on resident inputs: the
-copies only move bytes, and every kernel on this small pair is deterministic (each Gram tile takes
-one accumulation chunk, the factor applies its tile updates in a fixed order). Oracle parity of the
-calibration itself is covered by the end-to-end tests."""
+"""The host-to-host calibration step (inputs copied in and outputs copied back on their own streams,
+overlapped with the compute, inputs double-buffered) must give exactly what the same calls give on
+resident inputs: the copies only move bytes, and every kernel on this small pair is deterministic
+(each Gram tile takes one accumulation chunk, the factor applies its tile updates in a fixed order).
+Oracle parity of the calibration itself is covered by the end-to-end tests."""
 import pytest
 import torch
 
@@ -45,18 +45,25 @@ def test_host_step_matches_resident_path(ctx, n_shared):
                          for t in (out(m, p).codes, out(m, p).scales, out(m, p).zeros))
                 for p in parts} for m in modes}
     step = HostStep(cal, [x.shape for x in X], [l.shape for l in lg], hW)
-    for _ in range(2):
+    hloss = pin(torch.zeros(cal.loss_dev.shape, dtype=torch.float64))
+    ref_loss = ref.loss_dev.cpu()
+    for it in range(3):   # both input sets, then the first again; the losses read synchronously or not
         for m in modes:
             for trip in hout[m].values():
                 for t in trip:
                     t.zero_()
-        step.run(hX, hL, hW, hout, modes)
+        hloss.zero_()
+        step.run(hX, hL, hW, hout, modes, hloss=hloss if it != 1 else None)
+        step.join()
         torch.cuda.synchronize()
+        if it != 1:
+            assert (hloss - ref_loss).abs().max() <= 1e-12 * ref_loss.abs().max()
         for m in modes:
             for p in parts:
                 q = out(m, p)
                 for h, d in zip(hout[m][p], (q.codes, q.scales, q.zeros)):
                     assert torch.equal(h, d.cpu()), (m, p)
             # the in-kernel loss adds per-CTA float64 partial sums atomically: equal up to their order
-            for a, b in ((cal.res[m].qg.loss, ref.res[m].qg.loss), (cal.res[m].qd.loss, ref.res[m].qd.loss)):
-                assert abs(a - b).max() <= 1e-12 * abs(b).max()
+            if it == 1:
+                for a, b in ((cal.res[m].qg.loss, ref.res[m].qg.loss), (cal.res[m].qd.loss, ref.res[m].qd.loss)):
+                    assert abs(a - b).max() <= 1e-12 * abs(b).max()
