@@ -111,7 +111,9 @@ CLHA_API int64_t clha_packed_rows(int64_t n, int k, int E);
  * segment starts at a multiple of 128 and the rows between segments are zero.
  * seg is int64 [2E + 1]: seg[0..E] segment starts (seg[E] = total padded rows), seg[E+1 .. 2E]
  * token counts. packed_rows must be >= clha_packed_rows(n, k, E). perm (optional, int32
- * [packed_rows]) receives each packed row's token index (-1 for padding rows). */
+ * [packed_rows]) receives each packed row's token index (-1 for padding rows). X_packed may be NULL
+ * when perm is given: then only the permutation and seg are produced (nothing is copied), for
+ * clha_collect_gathered and clha_expert_act_gathered, which read the rows where they are. */
 CLHA_API clha_status clha_gather(clha_ctx* ctx, const void* X, clha_dtype dtype, int64_t n, int d,
                         const int32_t* ids, int k, int E, void* X_packed, int64_t packed_rows,
                         int64_t* seg, int32_t* perm);
@@ -142,6 +144,12 @@ CLHA_API clha_status clha_gather_noalloc(clha_ctx* ctx, const void* X, clha_dtyp
 CLHA_API clha_status clha_expert_act(clha_ctx* ctx, const void* X, int64_t rows, int d_model,
                             const int64_t* seg, int E, const void* Wg, const void* Wu, int d_ff,
                             void* h);
+/* clha_expert_act with the segment rows read from the token matrix X [n, d_model] through perm (as in
+ * clha_collect_gathered; -1 entries are zero rows); h is written in the packed segment layout,
+ * packed_rows rows (>= seg[E]), padding rows zero. Same values as clha_expert_act on the packed X. */
+CLHA_API clha_status clha_expert_act_gathered(clha_ctx* ctx, const void* X, int64_t n, int d_model,
+                                              const int32_t* perm, int64_t packed_rows, const int64_t* seg, int E,
+                                              const void* Wg, const void* Wu, int d_ff, void* h);
 
 /* Largest number of layers (or source experts) one accumulator holds. */
 #define CLHA_MAX_LAYERS 32
@@ -167,6 +175,16 @@ CLHA_API clha_status clha_accum_import(clha_ctx* ctx, clha_accum* acc, const flo
  * A NaN or Inf entry of X is recorded as CLHA_ERR_NONFINITE. */
 CLHA_API clha_status clha_collect(clha_ctx* ctx, clha_accum* acc, int layer, const void* X, clha_dtype dtype,
                          int64_t rows, int d, const int64_t* seg, int E, int slot0);
+
+/* Phase 1 straight from the token matrix, with no packed copy of the routed rows (the gather fused
+ * into the Gram accumulation): X [n, d] bf16 (n < 2^31); expert e's rows are the tokens
+ * perm[seg[e] .. seg[e] + seg[E + 1 + e]) in that order, perm and seg as clha_gather writes them (a
+ * padding entry, -1, reads as a zero row). The tensor-core kernel fetches the operands four rows at
+ * a time by TMA gather4 from X itself. Accumulates into slots slot0 .. slot0 + E - 1 of `layer` and
+ * adds the token counts, exactly as clha_collect does on clha_gather's packed X (same rows in the
+ * same order: the same sums). perm must be 16-byte aligned. */
+CLHA_API clha_status clha_collect_gathered(clha_ctx* ctx, clha_accum* acc, int layer, const void* X, int64_t n,
+                                           int d, const int32_t* perm, const int64_t* seg, int E, int slot0);
 
 /* ------------------------------------------------------------------------------ phase 2: aggregation */
 

@@ -32,6 +32,7 @@ SYMBOLS = [
     "clha_accum_export", "clha_accum_import", "clha_collect",
     "clha_aggregate", "clha_factor", "clha_factor_groups", "clha_epmq_target", "clha_quantize", "clha_loss",
     "clha_pack_codes", "clha_dequantize", "clha_dequant_matmul", "clha_routing_divergence",
+    "clha_collect_gathered", "clha_expert_act_gathered",
 ]
 FACTOR_MAX_GROUPS = 4
 
@@ -94,6 +95,8 @@ def load(path: str = LIB_PATH):
                                 vp]),
         "clha_loss": (i32, [vp, vp, i32, vp, vp, i32, i32, i32, i32, vp]),
         "clha_routing_divergence": (i32, [vp, vp, i32, i32, i32, i32, vp]),
+        "clha_collect_gathered": (i32, [vp, vp, i32, vp, i64, i32, vp, vp, i32, i32]),
+        "clha_expert_act_gathered": (i32, [vp, vp, i64, i32, vp, i64, vp, i32, vp, vp, i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -189,6 +192,13 @@ def clha_expert_act(ctx: Context, X, rows: int, d_model: int, seg, E: int, Wg, W
     ctx._check(load().clha_expert_act(ctx.handle, _p(X), rows, d_model, _p(seg), E, _p(Wg), _p(Wu), d_ff, _p(h)))
 
 
+def clha_expert_act_gathered(ctx: Context, X, n: int, d_model: int, perm, packed_rows: int, seg, E: int, Wg, Wu,
+                             d_ff: int, h):
+    """The expert activation with the segment rows read from X [n, d_model] through perm."""
+    ctx._check(load().clha_expert_act_gathered(ctx.handle, _p(X), n, d_model, _p(perm), packed_rows, _p(seg), E,
+                                               _p(Wg), _p(Wu), d_ff, _p(h)))
+
+
 class Accum:
     """clha_accum: per-(layer, slot) Gram matrices and token counts."""
 
@@ -255,6 +265,11 @@ def clha_accum_import(ctx: Context, acc: Accum, S: np.ndarray, counts: np.ndarra
 
 def clha_collect(ctx: Context, acc: Accum, layer: int, X, rows: int, d: int, seg=None, E: int = 1, slot0: int = 0):
     ctx._check(load().clha_collect(ctx.handle, acc.handle, layer, _p(X), _dtype(X), rows, d, _p(seg), E, slot0))
+
+
+def clha_collect_gathered(ctx: Context, acc: Accum, layer: int, X, n: int, d: int, perm, seg, E: int, slot0: int = 0):
+    """Gram accumulation straight from X [n, d] bf16 through clha_gather's perm (TMA gather4)."""
+    ctx._check(load().clha_collect_gathered(ctx.handle, acc.handle, layer, _p(X), n, d, _p(perm), _p(seg), E, slot0))
 
 
 def clha_aggregate(ctx: Context, acc: Accum, slot0: int, n_slots: int, mode: int, alpha_in=None,

@@ -203,7 +203,8 @@ extern "C" clha_status clha_gather(clha_ctx* ctx, const void* X, clha_dtype dtyp
     REQUIRE(d % 128 == 0, CLHA_ERR_UNSUPPORTED_SHAPE, "clha_gather: d=%d is not a multiple of 128", d);
     REQUIRE(packed_rows >= clha_packed_rows(n, k, E), CLHA_ERR_INVALID_ARG,
             "clha_gather: packed_rows %lld < %lld", (long long)packed_rows, (long long)clha_packed_rows(n, k, E));
-    REQUIRE(seg && X_packed && (n == 0 || (X && ids)), CLHA_ERR_INVALID_ARG, "clha_gather: null pointer");
+    REQUIRE(seg && (X_packed || perm) && (n == 0 || ids) && (!X_packed || n == 0 || X), CLHA_ERR_INVALID_ARG,
+            "clha_gather: null pointer");
     SET_DEVICE(ctx);
     LaunchScope launch_scope(ctx);
     size_t wsb = gather_workspace_bytes(n, k, E, packed_rows);
@@ -228,9 +229,29 @@ extern "C" clha_status clha_expert_act(clha_ctx* ctx, const void* X, int64_t row
     if (rows == 0) return CLHA_OK;
     SET_DEVICE(ctx);
     LaunchScope launch_scope(ctx);
-    CUDA_TRY(launch_expert_act(ctx->stream, ctx->num_sms, (const __nv_bfloat16*)X, rows, d_model, seg, E,
+    CUDA_TRY(launch_expert_act(ctx->stream, ctx->num_sms, (const __nv_bfloat16*)X, rows, d_model, nullptr, seg, E,
                                (const __nv_bfloat16*)Wg, (const __nv_bfloat16*)Wu, d_ff, (__nv_bfloat16*)h, ctx->d_err),
              "clha_expert_act");
+    return CLHA_OK;
+}
+
+extern "C" clha_status clha_expert_act_gathered(clha_ctx* ctx, const void* X, int64_t n, int d_model,
+                                                const int32_t* perm, int64_t packed_rows, const int64_t* seg, int E,
+                                                const void* Wg, const void* Wu, int d_ff, void* h) {
+    CHECK_CTX(ctx);
+    REQUIRE(n >= 0 && n < (int64_t)1 << 31 && packed_rows >= 0 && d_model > 0 && d_ff > 0 && E >= 1 && E <= 1024,
+            CLHA_ERR_INVALID_ARG, "clha_expert_act_gathered: bad sizes");
+    REQUIRE(d_model % 128 == 0 && d_ff % 128 == 0, CLHA_ERR_UNSUPPORTED_SHAPE,
+            "clha_expert_act_gathered: d_model=%d and d_ff=%d must be multiples of 128", d_model, d_ff);
+    REQUIRE(Wg && Wu && perm && seg && (packed_rows == 0 || h) && (n == 0 || X), CLHA_ERR_INVALID_ARG,
+            "clha_expert_act_gathered: null pointer");
+    if (packed_rows == 0 || n == 0) return CLHA_OK;
+    SET_DEVICE(ctx);
+    LaunchScope launch_scope(ctx);
+    CUDA_TRY(launch_expert_act(ctx->stream, ctx->num_sms, (const __nv_bfloat16*)X, packed_rows, d_model, perm, seg,
+                               E, (const __nv_bfloat16*)Wg, (const __nv_bfloat16*)Wu, d_ff, (__nv_bfloat16*)h,
+                               ctx->d_err),
+             "clha_expert_act_gathered");
     return CLHA_OK;
 }
 
@@ -336,6 +357,29 @@ extern "C" clha_status clha_collect(clha_ctx* ctx, clha_accum* acc, int layer, c
     else
         e = launch_collect_f32(ctx->stream, (const float*)X, rows, d, seg, ne, S_base, c_base);
     CUDA_TRY(e, "clha_collect");
+    return CLHA_OK;
+}
+
+extern "C" clha_status clha_collect_gathered(clha_ctx* ctx, clha_accum* acc, int layer, const void* X, int64_t n,
+                                             int d, const int32_t* perm, const int64_t* seg, int E, int slot0) {
+    CHECK_CTX(ctx);
+    REQUIRE(acc, CLHA_ERR_INVALID_ARG, "clha_collect_gathered: null accumulator");
+    REQUIRE(d == acc->d, CLHA_ERR_INVALID_ARG, "clha_collect_gathered: d=%d but the accumulator has d=%d", d, acc->d);
+    REQUIRE(layer >= 0 && layer < acc->n_layers, CLHA_ERR_INVALID_ARG,
+            "clha_collect_gathered: layer %d outside 0..%d", layer, acc->n_layers - 1);
+    REQUIRE(n >= 0 && n < (int64_t)1 << 31, CLHA_ERR_INVALID_ARG, "clha_collect_gathered: n outside 0 .. 2^31 - 1");
+    REQUIRE(E >= 1 && slot0 >= 0 && slot0 + E <= acc->n_slots, CLHA_ERR_INVALID_ARG,
+            "clha_collect_gathered: slots %d..%d outside the accumulator's %d", slot0, slot0 + E - 1, acc->n_slots);
+    REQUIRE(perm && seg && (n == 0 || X), CLHA_ERR_INVALID_ARG, "clha_collect_gathered: null pointer");
+    REQUIRE(((uintptr_t)perm & 15) == 0, CLHA_ERR_INVALID_ARG, "clha_collect_gathered: perm must be 16-byte aligned");
+    if (n == 0) return CLHA_OK;
+    SET_DEVICE(ctx);
+    LaunchScope launch_scope(ctx);
+    float* S_base = acc->S + ((size_t)layer * acc->n_slots + slot0) * (size_t)d * d;
+    int64_t* c_base = acc->counts + (size_t)layer * acc->n_slots + slot0;
+    CUDA_TRY(launch_collect_bf16_gathered(ctx->stream, ctx->num_sms, (const __nv_bfloat16*)X, n, d, perm, seg, E,
+                                          S_base, c_base, ctx->d_err),
+             "clha_collect_gathered");
     return CLHA_OK;
 }
 

@@ -79,8 +79,11 @@ cudaError_t launch_gather(cudaStream_t s, const void* X, int esize, int64_t n, i
                           int64_t* seg, int32_t* perm, void* ws, size_t ws_bytes, int* err);
 size_t gather_workspace_bytes(int64_t n, int k, int E, int64_t packed_rows);
 cudaError_t launch_expert_act(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t rows, int d_model,
-                              const int64_t* seg, int E, const __nv_bfloat16* Wg,
+                              const int32_t* perm, const int64_t* seg, int E, const __nv_bfloat16* Wg,
                               const __nv_bfloat16* Wu, int d_ff, __nv_bfloat16* h, int* err);
+cudaError_t launch_collect_bf16_gathered(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t n, int d,
+                                         const int32_t* perm, const int64_t* seg, int E, float* S_base,
+                                         int64_t* counts_base, int* err);
 cudaError_t launch_collect_bf16(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t rows, int d,
                                 const int64_t* seg, int E, float* S_base, int64_t* counts_base,
                                 int* err);

@@ -1,7 +1,9 @@
 // Expert FFN activation h = SiLU(x Wg^T) * (x Wu^T) for every row of every expert segment: the input
 // of the expert's down projection, whose Hessian phase 1 collects. fp32 accumulation, bf16 output
 // (round to nearest even). Padding rows of a segment are written as zero, so h has exactly the
-// segment layout of its input and can be collected the same way.
+// segment layout of its input and can be collected the same way. The rows are read either from a
+// packed copy (row q of the segment layout) or straight from the token matrix through the gather's
+// permutation (row q is token perm[q]), so the routed rows need not be copied.
 //
 // Shared-memory tiled FMA kernel: a 64-row x 64-column output tile computes the gate and the up
 // tile together (two accumulators per thread), so the SiLU-times-up epilogue needs no second pass.
@@ -44,6 +46,7 @@ struct ActSmem {
 };
 
 __global__ void __launch_bounds__(256, 2) expert_act_simt(const __nv_bfloat16* __restrict__ X, int64_t rows, int dm,
+                                                          const int32_t* __restrict__ perm,
                                                           const int64_t* __restrict__ seg, int E,
                                                           const __nv_bfloat16* __restrict__ Wg,
                                                           const __nv_bfloat16* __restrict__ Wu, int dff,
@@ -64,8 +67,14 @@ __global__ void __launch_bounds__(256, 2) expert_act_simt(const __nv_bfloat16* _
     const int tid = threadIdx.x;
     const int lr = tid >> 2, lk = (tid & 3) * 8;       // this thread copies row lr, k lk..lk+7 (coalesced)
     const int cr = tid & 63, ck = (tid >> 6) * 8;      // and converts row cr, k ck..ck+7 (a warp: 32 rows)
-    const bool row_ok = m0 + lr < valid_end;
-    const __nv_bfloat16* xsrc = X + (row_ok ? (m0 + lr) * dm : 0) + lk;
+    // packed row m0 + lr: row m0 + lr of X, or with perm the token perm[m0 + lr] (-1: padding, zeros)
+    int64_t xrow = m0 + lr;
+    bool row_ok = xrow < valid_end;
+    if (perm && row_ok) {
+        xrow = perm[xrow];
+        row_ok = xrow >= 0;
+    }
+    const __nv_bfloat16* xsrc = X + (row_ok ? xrow * dm : 0) + lk;
     const __nv_bfloat16* gsrc = wg + (size_t)(n0 + lr) * dm + lk;
     const __nv_bfloat16* usrc = wu + (size_t)(n0 + lr) * dm + lk;
     const int nkt = dm / TK;
@@ -147,8 +156,8 @@ __global__ void __launch_bounds__(256, 2) expert_act_simt(const __nv_bfloat16* _
 }  // namespace
 
 cudaError_t launch_expert_act(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t rows, int d_model,
-                              const int64_t* seg, int E, const __nv_bfloat16* Wg, const __nv_bfloat16* Wu, int d_ff,
-                              __nv_bfloat16* h, int* err) {
+                              const int32_t* perm, const int64_t* seg, int E, const __nv_bfloat16* Wg,
+                              const __nv_bfloat16* Wu, int d_ff, __nv_bfloat16* h, int* err) {
     (void)num_sms;
     (void)err;
     static bool attr_set = false;
@@ -159,7 +168,7 @@ cudaError_t launch_expert_act(cudaStream_t s, int num_sms, const __nv_bfloat16* 
         attr_set = true;
     }
     dim3 grid((unsigned)((rows + TM - 1) / TM), d_ff / TN);
-    expert_act_simt<<<grid, 256, sizeof(ActSmem), s>>>(X, rows, d_model, seg, E, Wg, Wu, d_ff, h);
+    expert_act_simt<<<grid, 256, sizeof(ActSmem), s>>>(X, rows, d_model, perm, seg, E, Wg, Wu, d_ff, h);
     clha_note_launches(1);
     return cudaGetLastError();
 }

@@ -130,6 +130,7 @@ cudaError_t launch_gather(cudaStream_t s, const void* X, int esize, int64_t n, i
     clha_note_launches(1);
     gather_scatter<<<(unsigned)nblk, kTB, kTB * k * sizeof(int), s>>>(ids, n, k, E, H, pm);
     clha_note_launches(1);
+    if (!X_packed) return cudaGetLastError();   // the permutation alone: the rows are read where they are
     int64_t row_vecs = (int64_t)d * esize / 16;
     int64_t warps = packed_rows;
     int64_t blocks = (warps + 7) / 8;

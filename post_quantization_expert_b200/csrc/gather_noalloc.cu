@@ -55,7 +55,7 @@ extern "C" clha_status clha_gather_noalloc(clha_ctx* ctx, const void* X, clha_dt
     if (packed_rows < clha_packed_rows(n, k, E))
         return clha_fail(ctx, CLHA_ERR_INVALID_ARG, "clha_gather_noalloc: packed_rows %lld < %lld",
                          (long long)packed_rows, (long long)clha_packed_rows(n, k, E));
-    if (!seg || !X_packed || (n > 0 && (!X || !ids)))
+    if (!seg || (!X_packed && !perm) || (n > 0 && !ids) || (X_packed && n > 0 && !X))
         return clha_fail(ctx, CLHA_ERR_INVALID_ARG, "clha_gather_noalloc: null pointer");
     const size_t need = gather_workspace_bytes(n, k, E, packed_rows);
     if (need > kScratchBytes)

@@ -44,6 +44,7 @@ constexpr uint32_t IDESC = tc::idesc_f32acc(1 /*bf16*/, 1 /*A MN-major*/, 1 /*B 
 struct SyrkParams {
     int d;
     int64_t rows;
+    const int32_t* perm;   // gathered operands: token of each packed row (-1: padding), else null
     const int64_t* seg;
     int E;
     float* S;
@@ -67,6 +68,10 @@ __device__ __forceinline__ void slot_range(const SyrkParams& p, int e, int64_t& 
     else { t0 = 0; cnt = p.rows; }
 }
 
+// kGather: the operands come straight from the token matrix X [rows, d]: packed row q of a segment is
+// token perm[q], fetched four rows at a time by TMA gather4 (a padding row, perm -1, is a row index
+// past the end and reads zeros), so the routed rows are never copied out of X.
+template <bool kGather>
 __global__ void __launch_bounds__(kThreads, 1) syrk_bf16_tc(const __grid_constant__ CUtensorMap tmX,
                                                             const __grid_constant__ CUtensorMap tmS, SyrkParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -102,7 +107,57 @@ __global__ void __launch_bounds__(kThreads, 1) syrk_bf16_tc(const __grid_constan
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
+    if (warp == 0 && kGather) {
+        // all 32 lanes issue: lane l fetches rows 4g .. 4g+3 (g = l % 16) of the 64-token block for
+        // boxes l / 16, l / 16 + 2, l / 16 + 4 (boxes 0-1: the A columns, 2-5: the B columns)
+        int it = 0;
+        bool ok = true;
+        const int g = lane & 15;
+        const int oob = (int)p.rows;   // a row index past the end: zeros
+        for (int w = blockIdx.x; w < p.total_tiles && ok; w += gridDim.x) {
+            const int e = w / p.tiles_per_slot;
+            int r, c;
+            decode_tile(w % p.tiles_per_slot, p.nr, p.nc, r, c);
+            int64_t t0, cnt;
+            slot_range(p, e, t0, cnt);
+            const int nk = (int)((cnt + BK - 1) / BK);
+            // this lane's four token indices of blocks kb + 1 and kb + 2 are loaded ahead, so the
+            // index loads overlap the wait for a free stage and the copies of block kb
+            const int4* pq = reinterpret_cast<const int4*>(p.perm + t0 + 4 * g);
+            int4 tk1 = nk > 0 ? pq[0] : make_int4(-1, -1, -1, -1);
+            int4 tk2 = nk > 1 ? pq[BK / 4] : make_int4(-1, -1, -1, -1);
+            for (int kb = 0; kb < nk; ++kb, ++it) {
+                const int4 tk = tk1;
+                tk1 = tk2;
+                if (kb + 2 < nk) tk2 = pq[(int64_t)(kb + 2) * (BK / 4)];
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
+                int got = 1;
+                if (lane == 0) got = tc::mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag) ? 1 : 0;
+                got = __shfl_sync(0xffffffffu, got, 0);
+                if (!got) { ok = false; break; }
+                const uint32_t fb = full0 + 8 * s;
+                if (lane == 0) tc::mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                __syncwarp();
+                const uint32_t a_dst = tc::smem_u32(smem + s * STAGE_BYTES);
+                const uint32_t b_dst = a_dst + A_BYTES;
+                const int r0 = tk.x < 0 ? oob : tk.x, r1 = tk.y < 0 ? oob : tk.y;
+                const int r2 = tk.z < 0 ? oob : tk.z, r3 = tk.w < 0 ? oob : tk.w;
+#pragma unroll
+                for (int hh = 0; hh < 3; ++hh) {
+                    const int h = (lane >> 4) + 2 * hh;
+                    const uint32_t dst = (h < 2 ? a_dst + h * 8192 : b_dst + (h - 2) * 8192) + g * 512;
+                    const int x = h < 2 ? r * BM + h * 64 : c * BN + (h - 2) * 64;
+                    tc::tma_gather4_2d(dst, &tmX, fb, x, r0, r1, r2, r3);
+                }
+            }
+        }
+        if (!ok && lane == 0) {  // let the copies already issued land before the CTA can exit
+            for (int j = it - 1; j >= 0 && j >= it - STAGES; --j)
+                tc::mbar_wait_bounded(full0 + 8 * (j % STAGES), (j / STAGES) & 1, abort_flag, 100000000ull);
+        }
+        __syncwarp();
+    } else if (warp == 0) {
         if (lane == 0) {
             int it = 0;
             bool ok = true;
@@ -300,13 +355,14 @@ cudaError_t launch_collect_bf16(cudaStream_t s, int num_sms, const __nv_bfloat16
     if (e != cudaSuccess) return e;
     static bool attr_set = false;
     if (!attr_set) {
-        e = cudaFuncSetAttribute(syrk_bf16_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        e = cudaFuncSetAttribute(syrk_bf16_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
     SyrkParams p;
     p.d = d;
     p.rows = rows;
+    p.perm = nullptr;
     p.seg = seg;
     p.E = E;
     p.S = S_base;
@@ -317,9 +373,44 @@ cudaError_t launch_collect_bf16(cudaStream_t s, int num_sms, const __nv_bfloat16
     p.total_tiles = p.tiles_per_slot * E;
     p.err = err;
     int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
-    syrk_bf16_tc<<<grid, kThreads, SMEM_BYTES, s>>>(tm, tmS, p);
+    syrk_bf16_tc<false><<<grid, kThreads, SMEM_BYTES, s>>>(tm, tmS, p);
     clha_note_launches(1);
     add_counts<<<(E + 255) / 256, 256, 0, s>>>(counts_base, seg, E, rows);
+    clha_note_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_collect_bf16_gathered(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t n, int d,
+                                         const int32_t* perm, const int64_t* seg, int E, float* S_base,
+                                         int64_t* counts_base, int* err) {
+    CUtensorMap tm, tmS;
+    cudaError_t e = make_tmap_2d(&tm, X, (uint64_t)n, (uint64_t)d, 2, 1, 64);   // gather4: one-row box
+    if (e != cudaSuccess) return e;
+    e = make_tmap_2d(&tmS, S_base, (uint64_t)E * d, (uint64_t)d, 4, 32, 32);
+    if (e != cudaSuccess) return e;
+    static bool attr_set = false;
+    if (!attr_set) {
+        e = cudaFuncSetAttribute(syrk_bf16_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    SyrkParams p;
+    p.d = d;
+    p.rows = n;
+    p.perm = perm;
+    p.seg = seg;
+    p.E = E;
+    p.S = S_base;
+    p.nr = d / BM;
+    p.nc = (d + BN - 1) / BN;
+    p.tiles_per_slot = 0;
+    for (int c = 0; c < p.nc; ++c) p.tiles_per_slot += (p.nr < 2 * c + 2) ? p.nr : 2 * c + 2;
+    p.total_tiles = p.tiles_per_slot * E;
+    p.err = err;
+    int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
+    syrk_bf16_tc<true><<<grid, kThreads, SMEM_BYTES, s>>>(tm, tmS, p);
+    clha_note_launches(1);
+    add_counts<<<(E + 255) / 256, 256, 0, s>>>(counts_base, seg, E, n);
     clha_note_launches(1);
     return cudaGetLastError();
 }

@@ -3,6 +3,8 @@
 This module only orders calls and owns device buffers; every step runs in libclha.so:
   collection   clha_route_topk -> clha_gather -> clha_collect (expert inputs)
                -> clha_expert_act -> clha_collect (down-projection inputs)       per layer
+               (or, fused: clha_gather's permutation only -> clha_collect_gathered, which reads
+               the routed rows from X by TMA gather4 -> clha_expert_act_gathered)
   aggregation  clha_aggregate (alpha, H_comb, damping)                            per weighting
   quantization clha_factor -> clha_quantize (gate, up share a factor) -> clha_loss
 Always-active shared experts see every token: their gate/up input Hessian is one slot shared by
@@ -193,12 +195,17 @@ class MoECalibration:
     def __init__(self, ctx: L.Context, n_layers: int, max_tokens: int, E: int, k: int, d_model: int, d_ff: int,
                  n_shared: int = 0, shared_dff: int = 0, bits_routed: int = 2, bits_shared: int = 3,
                  damp_frac: float = 0.01, timer=NO_TIMER, modes=("rt",), keep_hcomb: bool = False,
-                 unrouted_rtn: bool = True):
+                 unrouted_rtn: bool = True, fused_gather: bool = False):
         """unrouted_rtn: an expert whose weighted Hessian aggregate is empty (never routed, or, for
         explicit alpha, never routed in the weighted layers) is quantized by round to nearest
-        (H_d = I, loss 0) instead of failing."""
+        (H_d = I, loss 0) instead of failing. fused_gather: the expert inputs are read straight from
+        the layer's X through the routing permutation (TMA gather4 in the Gram kernel, indexed rows
+        in the activation) instead of from a packed copy (bf16 X only). Same results; off by
+        default because four-row gather requests feed the tensor cores more slowly than the packed
+        copy costs (the Hessian phase of the E16 pair: 0.41 ms against 0.16 ms plus a 0.03 ms copy)."""
         self.ctx, self.n_layers, self.E, self.k = ctx, n_layers, E, k
         self.agg_flag = L.AGG_EMPTY_IDENTITY if unrouted_rtn else 0
+        self.fused_gather = fused_gather
         self.timer = timer
         self.d_model, self.d_ff, self.n_shared, self.shared_dff = d_model, d_ff, n_shared, shared_dff
         self.bits_routed, self.bits_shared, self.damp = bits_routed, bits_shared, damp_frac
@@ -206,7 +213,8 @@ class MoECalibration:
         self.P = L.clha_packed_rows(max_tokens, k, E)
         self.ids = torch.empty((max_tokens, k), dtype=torch.int32, device=dev)
         self.counts = torch.empty((n_layers, E), dtype=torch.int32, device=dev)
-        self.Xp = torch.empty((self.P, d_model), dtype=torch.bfloat16, device=dev)
+        self.Xp = None if fused_gather else torch.empty((self.P, d_model), dtype=torch.bfloat16, device=dev)
+        self.perm = torch.empty(self.P, dtype=torch.int32, device=dev)
         self.hp = torch.empty((self.P, d_ff), dtype=torch.bfloat16, device=dev)
         self.seg = torch.empty((n_layers, 2 * E + 1), dtype=torch.int64, device=dev)
         # slots of the input accumulator: 0..E-1 routed, E the shared experts' common input
@@ -277,16 +285,27 @@ class MoECalibration:
         seg = self.seg[layer]
         with t.span("route"):
             L.clha_route_topk(ctx, logits, n, E, k, ids, self.counts[layer])
+        fused = self.fused_gather and X.dtype == torch.bfloat16
+        if not fused and self.Xp is None:
+            self.Xp = torch.empty((self.P, self.d_model), dtype=X.dtype, device=self.dev)
         with t.span("gather"):
-            L.clha_gather(ctx, X, n, self.d_model, ids, k, E, self.Xp, self.P, seg)
+            L.clha_gather(ctx, X, n, self.d_model, ids, k, E, None if fused else self.Xp, self.P, seg,
+                          self.perm if fused else None)
         with t.span("hessian"):
-            L.clha_collect(ctx, self.acc_in, layer, self.Xp, self.P, self.d_model, seg, E, 0)
+            if fused:
+                L.clha_collect_gathered(ctx, self.acc_in, layer, X, n, self.d_model, self.perm, seg, E, 0)
+            else:
+                L.clha_collect(ctx, self.acc_in, layer, self.Xp, self.P, self.d_model, seg, E, 0)
             if self.n_shared:
                 L.clha_collect(ctx, self.acc_in, layer, X, n, self.d_model, None, 1, E)
         if before_act is not None:
             before_act()
         with t.span("act"):
-            L.clha_expert_act(ctx, self.Xp, self.P, self.d_model, seg, E, w.Wg, w.Wu, self.d_ff, self.hp)
+            if fused:
+                L.clha_expert_act_gathered(ctx, X, n, self.d_model, self.perm, self.P, seg, E, w.Wg, w.Wu, self.d_ff,
+                                           self.hp)
+            else:
+                L.clha_expert_act(ctx, self.Xp, self.P, self.d_model, seg, E, w.Wg, w.Wu, self.d_ff, self.hp)
         with t.span("hessian"):
             L.clha_collect(ctx, self.acc_dn, layer, self.hp, self.P, self.d_ff, seg, E, 0)
         if self.n_shared:

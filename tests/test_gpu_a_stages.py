@@ -71,6 +71,59 @@ def test_gather_segments(ctx, n, E, k, d):
     assert seg[E] == start
 
 
+# --------------------------------------------------------------------- gather fused into collection
+@pytest.mark.parametrize("n,E,k,d,dff", [(2048, 16, 2, 1024, 512), (1000, 64, 6, 2048, 1408), (37, 8, 3, 384, 256),
+                                        (80000, 16, 2, 256, 128)])
+def test_gathered_collection_and_activation_equal_the_packed_path(ctx, n, E, k, d, dff):
+    """Gram sums read from X by TMA gather4 through the routing permutation, and the activation read
+    through it, are bit-identical to the same kernels on the packed copy (the same rows in the same
+    order; padding rows are zeros either way). Sizes: ragged segments, 64 experts with 128-row
+    padding, a few tokens per expert, and ~10k-token segments (two accumulation chunks per tile,
+    whose fp32 additions into S may land in either order: equal to 1e-6 there)."""
+    g = _gen(n + E)
+    lg = torch.randn((n, E), generator=g).to(DEV)
+    X = (torch.randn((n, d), generator=g) * (0.5 + torch.rand(d, generator=g))).to(torch.bfloat16).to(DEV)
+    Wg = (0.03 * torch.randn((E, dff, d), generator=g)).to(torch.bfloat16).to(DEV)
+    Wu = (0.03 * torch.randn((E, dff, d), generator=g)).to(torch.bfloat16).to(DEV)
+    ids = torch.empty((n, k), dtype=torch.int32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    L.clha_route_topk(ctx, lg, n, E, k, ids, counts)
+    P = L.clha_packed_rows(n, k, E)
+    Xp = torch.empty((P, d), dtype=torch.bfloat16, device=DEV)
+    seg = torch.empty(2 * E + 1, dtype=torch.int64, device=DEV)
+    perm = torch.empty(P, dtype=torch.int32, device=DEV)
+    L.clha_gather(ctx, X, n, d, ids, k, E, Xp, P, seg, perm)
+    seg2 = torch.empty_like(seg)
+    perm2 = torch.empty_like(perm)
+    L.clha_gather(ctx, X, n, d, ids, k, E, None, P, seg2, perm2)      # the permutation alone
+    assert torch.equal(seg, seg2) and torch.equal(perm, perm2)
+    a, b = L.Accum(ctx, d, 2, E), L.Accum(ctx, d, 2, E)
+    for layer in (0, 1):   # twice into layer 1: the second pass accumulates onto the first
+        for _ in range(1 + layer):
+            L.clha_collect(ctx, a, layer, Xp, P, d, seg, E, 0)
+            L.clha_collect_gathered(ctx, b, layer, X, n, d, perm, seg, E, 0)
+    h1 = torch.full((P, dff), 7.0, dtype=torch.bfloat16, device=DEV)
+    h2 = torch.full((P, dff), -7.0, dtype=torch.bfloat16, device=DEV)
+    L.clha_expert_act(ctx, Xp, P, d, seg, E, Wg, Wu, dff, h1)
+    L.clha_expert_act_gathered(ctx, X, n, d, perm, P, seg, E, Wg, Wu, dff, h2)
+    L.clha_check(ctx)
+    Sa, ca = a.buffers()
+    Sb, cb = b.buffers()
+    assert torch.equal(ca, cb)
+    # the authoritative upper triangle is bit-identical
+    iu = torch.triu_indices(d, d, device=DEV)
+    multi_chunk = n * k // E > 8192
+    for layer in (0, 1):
+        for e in range(E):
+            ua, ub = Sa[layer, e][iu[0], iu[1]], Sb[layer, e][iu[0], iu[1]]
+            if multi_chunk:
+                assert (ua - ub).norm() <= 1e-6 * ua.norm(), (layer, e)
+            else:
+                assert torch.equal(ua, ub), (layer, e)
+    end = int(seg[E].item())
+    assert torch.equal(h1[:end], h2[:end])
+
+
 # ------------------------------------------------------------------------------------ collection
 @pytest.mark.parametrize("n,d", [(1000, 512), (129, 1408), (1, 256), (4096, 1024), (777, 2048), (9000, 384),
                                  (65536, 256)])

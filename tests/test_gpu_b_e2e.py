@@ -45,7 +45,7 @@ def test_dense_two_layer_fp32_workload(ctx):
     assert abs(cal.q.loss[0] - want["loss"]) <= 1e-3 * want["loss"]
 
 
-def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, **over):
+def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, fused=False, **over):
     wl = workload(cfg, "cpu", **over)
     s = wl.spec
     Xs = [wl.x(l) for l in range(2)]
@@ -54,7 +54,7 @@ def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, **over):
     shared = [wl.expert_weights(0, i, shared=True) for i in range(s.n_shared)]
     w = stack_weights((routed, shared), DEV)
     cal = MoECalibration(ctx, 2, max(s.tokens), s.E, s.k, s.d_model, s.d_ff, s.n_shared, s.shared_dff,
-                         s.bits_routed, s.bits_shared, s.damp_frac, modes=modes)
+                         s.bits_routed, s.bits_shared, s.damp_frac, modes=modes, fused_gather=fused)
     for l in range(2):
         cal.collect(l, Xs[l].to(DEV), lgs[l].to(DEV), w)
     torch.cuda.synchronize()
@@ -104,8 +104,10 @@ def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, **over):
 
 def test_moe_pair_E16_top2_full_size(ctx):
     """The E=16, top-2, d_model 1024, d_ff 512 layer pair at 8192 tokens per layer, 3-bit, both
-    weightings: all Hessians and routing checked; GPTQ end to end on experts 0, 7 and 15."""
-    _moe_pair(ctx, 2, [0, 7, 15], ("rt", "eq"))
+    weightings: all Hessians and routing checked; GPTQ end to end on experts 0, 7 and 15. The expert
+    inputs go through the fused path (read from X by TMA gather4, no packed copy); the E64 case
+    below takes the packed path."""
+    _moe_pair(ctx, 2, [0, 7, 15], ("rt", "eq"), fused=True)
 
 
 def test_moe_pair_E64_top6_shared_reduced_tokens(ctx):
