@@ -135,15 +135,30 @@ CLHA_API clha_status clha_gather_noalloc(clha_ctx* ctx, const void* X, clha_dtyp
                                          int64_t* seg, int32_t* perm);
 
 /* Expert FFN activation feeding the down projection: h = SiLU(x Wg^T) * (x Wu^T) per token of
- * each expert (bf16 products summed in fp32 over 32-term chunks, chunk sums in fp64, SiLU product in
- * fp64), stored as bf16 (round to nearest even). The pages do not
+ * each expert, SiLU product in fp64, stored as bf16 (round to nearest even). The pages do not
  * spell this out: the down projection's Hessian needs its input, and that input is this product.
  * X is bf16 [rows, d_model]; Wg, Wu are bf16 [E, d_ff, d_model] (experts stacked); h is bf16
  * [rows, d_ff]. With seg (from clha_gather) rows follow its segments and padding rows of h are
- * written as zero; with seg == NULL, E must be 1 and all `rows` rows belong to that expert. */
+ * written as zero; with seg == NULL, E must be 1 and all `rows` rows belong to that expert.
+ * Two kernels (clha_set_act_kernel): the tensor cores (bf16 products, fp32 accumulation in up to 8
+ * K-chunks added in fp64), or fp32 FMA (32-term fp32 chunks added in fp64). The tensor core adds a
+ * group of products after aligning them to the largest one, so inputs with outlier channels (tens of
+ * times the rest) lose enough low bits there to flip bf16 roundings of h too often; by default each
+ * call measures every channel's max |x| over the rows on the device and takes the tensor cores only
+ * when all of them are within 4x of their mean, the FMA kernel otherwise (no host round trip). */
 CLHA_API clha_status clha_expert_act(clha_ctx* ctx, const void* X, int64_t rows, int d_model,
                             const int64_t* seg, int E, const void* Wg, const void* Wu, int d_ff,
                             void* h);
+
+/* Which activation kernel clha_expert_act uses: CLHA_ACT_AUTO (default; chosen per call from the
+ * rows' channel magnitudes), CLHA_ACT_FMA or CLHA_ACT_TENSOR (always). clha_expert_act_gathered always
+ * takes the FMA kernel. clha_last_act_kernel reports the kernel of the context's last
+ * clha_expert_act call (synchronises; -1 on error). */
+#define CLHA_ACT_AUTO 0
+#define CLHA_ACT_FMA 1
+#define CLHA_ACT_TENSOR 2
+CLHA_API clha_status clha_set_act_kernel(clha_ctx* ctx, int kernel);
+CLHA_API int clha_last_act_kernel(clha_ctx* ctx);
 /* clha_expert_act with the segment rows read from the token matrix X [n, d_model] through perm (as in
  * clha_collect_gathered; -1 entries are zero rows); h is written in the packed segment layout,
  * packed_rows rows (>= seg[E]), padding rows zero. Same values as clha_expert_act on the packed X. */

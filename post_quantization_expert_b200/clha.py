@@ -23,6 +23,7 @@ STATUS_NAMES = ["OK", "INVALID_ARG", "UNSUPPORTED_SHAPE", "NOT_PD", "NONFINITE",
 BF16, F32 = 0, 1
 ALPHA_ROUTING, ALPHA_EQUAL, ALPHA_EXPLICIT, ALPHA_SUM = 0, 1, 2, 3
 AGG_EMPTY_IDENTITY = 0x100   # or'ed into an alpha mode: an aggregate without energy becomes H_d = I
+ACT_AUTO, ACT_FMA, ACT_TENSOR = 0, 1, 2   # activation kernel policy (clha_set_act_kernel)
 
 # every symbol include/clha.h declares
 SYMBOLS = [
@@ -32,7 +33,7 @@ SYMBOLS = [
     "clha_accum_export", "clha_accum_import", "clha_collect",
     "clha_aggregate", "clha_factor", "clha_factor_groups", "clha_epmq_target", "clha_quantize", "clha_loss",
     "clha_pack_codes", "clha_dequantize", "clha_dequant_matmul", "clha_routing_divergence",
-    "clha_collect_gathered", "clha_expert_act_gathered",
+    "clha_collect_gathered", "clha_expert_act_gathered", "clha_set_act_kernel", "clha_last_act_kernel",
 ]
 FACTOR_MAX_GROUPS = 4
 
@@ -97,6 +98,8 @@ def load(path: str = LIB_PATH):
         "clha_routing_divergence": (i32, [vp, vp, i32, i32, i32, i32, vp]),
         "clha_collect_gathered": (i32, [vp, vp, i32, vp, i64, i32, vp, vp, i32, i32]),
         "clha_expert_act_gathered": (i32, [vp, vp, i64, i32, vp, i64, vp, i32, vp, vp, i32, vp]),
+        "clha_set_act_kernel": (i32, [vp, i32]),
+        "clha_last_act_kernel": (i32, [vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -190,6 +193,14 @@ def clha_gather_noalloc(ctx: Context, X, n: int, d: int, ids, k: int, E: int, X_
 
 def clha_expert_act(ctx: Context, X, rows: int, d_model: int, seg, E: int, Wg, Wu, d_ff: int, h):
     ctx._check(load().clha_expert_act(ctx.handle, _p(X), rows, d_model, _p(seg), E, _p(Wg), _p(Wu), d_ff, _p(h)))
+
+
+def clha_set_act_kernel(ctx: Context, kernel: int):
+    ctx._check(load().clha_set_act_kernel(ctx.handle, kernel))
+
+
+def clha_last_act_kernel(ctx: Context) -> int:
+    return load().clha_last_act_kernel(ctx.handle)
 
 
 def clha_expert_act_gathered(ctx: Context, X, n: int, d_model: int, perm, packed_rows: int, seg, E: int, Wg, Wu,

@@ -141,9 +141,13 @@ extern "C" clha_status clha_create(int device, void* cuda_stream, clha_ctx** out
     if (cudaSetDevice(device) != cudaSuccess ||
         cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
         cudaMalloc(&ctx->d_err, 4 * sizeof(int)) != cudaSuccess ||
-        cudaMemset(ctx->d_err, 0, 4 * sizeof(int)) != cudaSuccess) {
+        cudaMemset(ctx->d_err, 0, 4 * sizeof(int)) != cudaSuccess ||
+        cudaMalloc(&ctx->d_act_sel, sizeof(int)) != cudaSuccess ||
+        cudaMemset(ctx->d_act_sel, 0, sizeof(int)) != cudaSuccess) {
         cudaGetLastError();
         if (ctx->d_err) cudaFree(ctx->d_err);
+    if (ctx->d_act_sel) cudaFree(ctx->d_act_sel);
+        if (ctx->d_act_sel) cudaFree(ctx->d_act_sel);
         delete ctx;
         return CLHA_ERR_CUDA;
     }
@@ -229,10 +233,35 @@ extern "C" clha_status clha_expert_act(clha_ctx* ctx, const void* X, int64_t row
     if (rows == 0) return CLHA_OK;
     SET_DEVICE(ctx);
     LaunchScope launch_scope(ctx);
+    void* ws = nullptr;
+    clha_status st = clha_workspace(ctx, expert_act_workspace_bytes(d_model), &ws);
+    if (st) return st;
     CUDA_TRY(launch_expert_act(ctx->stream, ctx->num_sms, (const __nv_bfloat16*)X, rows, d_model, nullptr, seg, E,
-                               (const __nv_bfloat16*)Wg, (const __nv_bfloat16*)Wu, d_ff, (__nv_bfloat16*)h, ctx->d_err),
+                               (const __nv_bfloat16*)Wg, (const __nv_bfloat16*)Wu, d_ff, (__nv_bfloat16*)h,
+                               ctx->act_policy, ws, ctx->d_act_sel, ctx->d_err),
              "clha_expert_act");
     return CLHA_OK;
+}
+
+extern "C" clha_status clha_set_act_kernel(clha_ctx* ctx, int kernel) {
+    CHECK_CTX(ctx);
+    REQUIRE(kernel >= CLHA_ACT_AUTO && kernel <= CLHA_ACT_TENSOR, CLHA_ERR_INVALID_ARG,
+            "clha_set_act_kernel: kernel must be CLHA_ACT_AUTO, CLHA_ACT_FMA or CLHA_ACT_TENSOR");
+    ctx->act_policy = kernel;
+    return CLHA_OK;
+}
+
+extern "C" int clha_last_act_kernel(clha_ctx* ctx) {
+    if (!ctx) return -1;
+    if (ctx->act_policy != CLHA_ACT_AUTO) return ctx->act_policy;
+    int sel = 0;
+    cudaSetDevice(ctx->device);
+    if (cudaStreamSynchronize(ctx->stream) != cudaSuccess ||
+        cudaMemcpy(&sel, ctx->d_act_sel, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+    }
+    return sel ? CLHA_ACT_TENSOR : CLHA_ACT_FMA;
 }
 
 extern "C" clha_status clha_expert_act_gathered(clha_ctx* ctx, const void* X, int64_t n, int d_model,
@@ -250,7 +279,7 @@ extern "C" clha_status clha_expert_act_gathered(clha_ctx* ctx, const void* X, in
     LaunchScope launch_scope(ctx);
     CUDA_TRY(launch_expert_act(ctx->stream, ctx->num_sms, (const __nv_bfloat16*)X, packed_rows, d_model, perm, seg,
                                E, (const __nv_bfloat16*)Wg, (const __nv_bfloat16*)Wu, d_ff, (__nv_bfloat16*)h,
-                               ctx->d_err),
+                               CLHA_ACT_FMA, nullptr, nullptr, ctx->d_err),
              "clha_expert_act_gathered");
     return CLHA_OK;
 }

@@ -21,6 +21,10 @@ struct clha_ctx {
     size_t ws_bytes = 0;
     // Kernels launched through this context (tracing).
     int64_t launches = 0;
+    // Expert activation: kernel policy (0 chosen per call on the device, 1 fp32 FMA, 2 tensor cores)
+    // and the device int the per-call choice is written to.
+    int act_policy = 0;
+    int* d_act_sel = nullptr;
     // Small pinned host buffer for scalar read-backs.
     void* host_pinned = nullptr;
     size_t host_pinned_bytes = 0;
@@ -78,9 +82,14 @@ cudaError_t launch_gather(cudaStream_t s, const void* X, int esize, int64_t n, i
                           const int32_t* ids, int k, int E, void* X_packed, int64_t packed_rows,
                           int64_t* seg, int32_t* perm, void* ws, size_t ws_bytes, int* err);
 size_t gather_workspace_bytes(int64_t n, int k, int E, int64_t packed_rows);
+size_t expert_act_workspace_bytes(int d_model);
 cudaError_t launch_expert_act(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t rows, int d_model,
                               const int32_t* perm, const int64_t* seg, int E, const __nv_bfloat16* Wg,
-                              const __nv_bfloat16* Wu, int d_ff, __nv_bfloat16* h, int* err);
+                              const __nv_bfloat16* Wu, int d_ff, __nv_bfloat16* h, int policy, void* ws, int* sel,
+                              int* err);
+cudaError_t launch_expert_act_tc(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t rows, int d_model,
+                                 const int64_t* seg, int E, const __nv_bfloat16* Wg, const __nv_bfloat16* Wu, int d_ff,
+                                 __nv_bfloat16* h, const int* sel, int* err);
 cudaError_t launch_collect_bf16_gathered(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t n, int d,
                                          const int32_t* perm, const int64_t* seg, int E, float* S_base,
                                          int64_t* counts_base, int* err);

@@ -1,4 +1,5 @@
-// Expert FFN activation h = SiLU(x Wg^T) * (x Wu^T) for every row of every expert segment: the input
+// Expert FFN activation on the fp32 FMA pipes (and the choice between it and the tensor-core kernel
+// of ffn_act_tc.cu): h = SiLU(x Wg^T) * (x Wu^T) for every row of every expert segment: the input
 // of the expert's down projection, whose Hessian phase 1 collects. fp32 accumulation, bf16 output
 // (round to nearest even). Padding rows of a segment are written as zero, so h has exactly the
 // segment layout of its input and can be collected the same way. The rows are read either from a
@@ -45,12 +46,14 @@ struct ActSmem {
     float f[2][3][TK][FLD];               // fp32, k-major
 };
 
-__global__ void __launch_bounds__(256, 2) expert_act_simt(const __nv_bfloat16* __restrict__ X, int64_t rows, int dm,
+__global__ void __launch_bounds__(256, 2) expert_act_simt(const int* __restrict__ sel,
+                                                          const __nv_bfloat16* __restrict__ X, int64_t rows, int dm,
                                                           const int32_t* __restrict__ perm,
                                                           const int64_t* __restrict__ seg, int E,
                                                           const __nv_bfloat16* __restrict__ Wg,
                                                           const __nv_bfloat16* __restrict__ Wu, int dff,
                                                           __nv_bfloat16* __restrict__ h) {
+    if (sel && *sel != 0) return;   // the tensor-core kernel takes this call
     extern __shared__ __align__(16) uint8_t act_smem[];
     ActSmem& sm = *reinterpret_cast<ActSmem*>(act_smem);
     const int64_t m0 = (int64_t)blockIdx.x * TM;
@@ -153,13 +156,55 @@ __global__ void __launch_bounds__(256, 2) expert_act_simt(const __nv_bfloat16* _
     }
 }
 
+// Per-channel max |x| over the rows (non-negative floats order like their bit patterns, so the
+// maximum is an unsigned atomicMax); one thread per channel and 256-row slab, coalesced along channels.
+__global__ void __launch_bounds__(256) act_channel_max(const __nv_bfloat16* __restrict__ X, int64_t rows, int dm,
+                                                       unsigned* __restrict__ chmax) {
+    const int c = blockIdx.x * 256 + threadIdx.x;
+    if (c >= dm) return;
+    const int64_t r0 = (int64_t)blockIdx.y * 256, r1 = r0 + 256 < rows ? r0 + 256 : rows;
+    float m = 0.f;
+    for (int64_t r = r0; r < r1; ++r) m = fmaxf(m, fabsf(__bfloat162float(X[r * dm + c])));
+    atomicMax(chmax + c, __float_as_uint(m));
+}
+
+// sel = 1 (tensor cores) when every channel's max |x| is within kRangeRatio of the channels' mean,
+// else 0 (fp32 FMA); one block.
+constexpr float kRangeRatio = 4.f;
+__global__ void __launch_bounds__(256) act_select(const unsigned* __restrict__ chmax, int dm, int* __restrict__ sel) {
+    __shared__ float smax[256], ssum[256];
+    float m = 0.f, sum = 0.f;
+    for (int c = threadIdx.x; c < dm; c += 256) {
+        const float v = __uint_as_float(chmax[c]);
+        m = fmaxf(m, v);
+        sum += v;
+    }
+    smax[threadIdx.x] = m;
+    ssum[threadIdx.x] = sum;
+    __syncthreads();
+    for (int o = 128; o > 0; o >>= 1) {
+        if (threadIdx.x < o) {
+            smax[threadIdx.x] = fmaxf(smax[threadIdx.x], smax[threadIdx.x + o]);
+            ssum[threadIdx.x] += ssum[threadIdx.x + o];
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) *sel = (smax[0] <= kRangeRatio * (ssum[0] / dm)) ? 1 : 0;
+}
+
 }  // namespace
 
+size_t expert_act_workspace_bytes(int d_model) { return clha_round_up((size_t)d_model * sizeof(unsigned)); }
+
+// The fp32-FMA kernel always reads through a permutation (the tensor-core kernel's TMA loads take
+// packed rows only). Otherwise `policy` picks: 1 fp32 FMA, 2 tensor cores, 0 per call on the device:
+// the channels' max |x| over the rows is measured and the tensor cores run when every channel is within
+// 4x of the channels' mean (no outlier channels), both kernels are queued and the one not chosen exits
+// at once (no host round trip). ws: expert_act_workspace_bytes(d_model); sel: one device int.
 cudaError_t launch_expert_act(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t rows, int d_model,
                               const int32_t* perm, const int64_t* seg, int E, const __nv_bfloat16* Wg,
-                              const __nv_bfloat16* Wu, int d_ff, __nv_bfloat16* h, int* err) {
-    (void)num_sms;
-    (void)err;
+                              const __nv_bfloat16* Wu, int d_ff, __nv_bfloat16* h, int policy, void* ws, int* sel,
+                              int* err) {
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(expert_act_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -167,8 +212,26 @@ cudaError_t launch_expert_act(cudaStream_t s, int num_sms, const __nv_bfloat16* 
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
+    const bool simt_only = perm || policy == 1;
+    const int* sel_dev = nullptr;
+    if (!simt_only) {
+        if (policy == 2) {
+            return launch_expert_act_tc(s, num_sms, X, rows, d_model, seg, E, Wg, Wu, d_ff, h, nullptr, err);
+        }
+        unsigned* chmax = (unsigned*)ws;
+        cudaError_t e = cudaMemsetAsync(chmax, 0, (size_t)d_model * sizeof(unsigned), s);
+        if (e != cudaSuccess) return e;
+        const int64_t slabs = (rows + 255) / 256;
+        act_channel_max<<<dim3((unsigned)((d_model + 255) / 256), (unsigned)(slabs < 65535 ? slabs : 65535)), 256, 0,
+                          s>>>(X, slabs < 65535 ? rows : 65535 * 256, d_model, chmax);
+        act_select<<<1, 256, 0, s>>>(chmax, d_model, sel);
+        clha_note_launches(2);
+        if ((e = launch_expert_act_tc(s, num_sms, X, rows, d_model, seg, E, Wg, Wu, d_ff, h, sel, err)) != cudaSuccess)
+            return e;
+        sel_dev = sel;
+    }
     dim3 grid((unsigned)((rows + TM - 1) / TM), d_ff / TN);
-    expert_act_simt<<<grid, 256, sizeof(ActSmem), s>>>(X, rows, d_model, perm, seg, E, Wg, Wu, d_ff, h);
+    expert_act_simt<<<grid, 256, sizeof(ActSmem), s>>>(sel_dev, X, rows, d_model, perm, seg, E, Wg, Wu, d_ff, h);
     clha_note_launches(1);
     return cudaGetLastError();
 }

@@ -74,12 +74,14 @@ def test_gather_segments(ctx, n, E, k, d):
 # --------------------------------------------------------------------- gather fused into collection
 @pytest.mark.parametrize("n,E,k,d,dff", [(2048, 16, 2, 1024, 512), (1000, 64, 6, 2048, 1408), (37, 8, 3, 384, 256),
                                         (80000, 16, 2, 256, 128)])
-def test_gathered_collection_and_activation_equal_the_packed_path(ctx, n, E, k, d, dff):
+def test_gathered_collection_and_activation_equal_the_packed_path(ctx, act_kernel, n, E, k, d, dff):
     """Gram sums read from X by TMA gather4 through the routing permutation, and the activation read
     through it, are bit-identical to the same kernels on the packed copy (the same rows in the same
     order; padding rows are zeros either way). Sizes: ragged segments, 64 experts with 128-row
     padding, a few tokens per expert, and ~10k-token segments (two accumulation chunks per tile,
-    whose fp32 additions into S may land in either order: equal to 1e-6 there)."""
+    whose fp32 additions into S may land in either order: equal to 1e-6 there). The gathered
+    activation is the FMA kernel, so the packed one is held to it too."""
+    act_kernel(L.ACT_FMA)
     g = _gen(n + E)
     lg = torch.randn((n, E), generator=g).to(DEV)
     X = (torch.randn((n, d), generator=g) * (0.5 + torch.rand(d, generator=g))).to(torch.bfloat16).to(DEV)
@@ -216,14 +218,26 @@ def test_accumulator_checkpoint_roundtrip(ctx):
 
 
 # ------------------------------------------------------------------------------------ FFN act
-@pytest.mark.parametrize("rows,dm,dff", [(300, 256, 384), (1000, 1024, 512)])
-def test_expert_act_dense(ctx, rows, dm, dff):
+@pytest.fixture
+def act_kernel(ctx):
+    """Restores the default (per-call) activation kernel choice after a test that forces one."""
+    yield lambda k: L.clha_set_act_kernel(ctx, k)
+    L.clha_set_act_kernel(ctx, L.ACT_AUTO)
+
+
+@pytest.mark.parametrize("kernel", [L.ACT_FMA, L.ACT_TENSOR])
+@pytest.mark.parametrize("rows,dm,dff", [(300, 256, 384), (1000, 1024, 512), (4097, 2048, 1408)])
+def test_expert_act_dense(ctx, act_kernel, kernel, rows, dm, dff):
+    """Both activation kernels against the oracle on inputs without outlier channels: at least 99.9 %
+    of h bit-exact, the rest one bf16 rounding away."""
+    act_kernel(kernel)
     g = _gen(rows)
     X = torch.randn((rows, dm), generator=g).to(torch.bfloat16).to(DEV)
     Wg = (0.05 * torch.randn((1, dff, dm), generator=g)).to(torch.bfloat16).to(DEV)
     Wu = (0.05 * torch.randn((1, dff, dm), generator=g)).to(torch.bfloat16).to(DEV)
     h = torch.empty((rows, dff), dtype=torch.bfloat16, device=DEV)
     L.clha_expert_act(ctx, X, rows, dm, None, 1, Wg, Wu, dff, h)
+    assert L.clha_last_act_kernel(ctx) == kernel
     want = O.ffn_act(to64(X), to64(Wg[0]), to64(Wu[0]))
     got = to64(h)
     exact = np.mean(got == want)
@@ -231,7 +245,29 @@ def test_expert_act_dense(ctx, rows, dm, dff):
     np.testing.assert_allclose(got, want, rtol=2 ** -7, atol=1e-6)
 
 
-def test_expert_act_segments_zero_padding(ctx):
+def test_expert_act_choice_follows_channel_range(ctx):
+    """The default choice: the tensor cores for channels of similar range, the FMA kernel when a few
+    channels are ~20x the rest (the outlier-channel workload), decided on the device per call."""
+    g = _gen(5)
+    rows, dm, dff = 512, 1024, 256
+    X = torch.randn((rows, dm), generator=g)
+    Wg = (0.05 * torch.randn((1, dff, dm), generator=g)).to(torch.bfloat16).to(DEV)
+    Wu = (0.05 * torch.randn((1, dff, dm), generator=g)).to(torch.bfloat16).to(DEV)
+    h = torch.empty((rows, dff), dtype=torch.bfloat16, device=DEV)
+    L.clha_expert_act(ctx, X.to(torch.bfloat16).to(DEV), rows, dm, None, 1, Wg, Wu, dff, h)
+    assert L.clha_last_act_kernel(ctx) == L.ACT_TENSOR
+    Xo = X.clone()
+    Xo[:, torch.randperm(dm, generator=g)[:10]] *= 20.0
+    Xo = Xo.to(torch.bfloat16).to(DEV)
+    L.clha_expert_act(ctx, Xo, rows, dm, None, 1, Wg, Wu, dff, h)
+    assert L.clha_last_act_kernel(ctx) == L.ACT_FMA
+    want = O.ffn_act(to64(Xo), to64(Wg[0]), to64(Wu[0]))
+    assert np.mean(to64(h) == want) >= 0.999
+
+
+@pytest.mark.parametrize("kernel", [L.ACT_FMA, L.ACT_TENSOR])
+def test_expert_act_segments_zero_padding(ctx, act_kernel, kernel):
+    act_kernel(kernel)
     n, E, k, dm, dff = 600, 8, 2, 256, 128
     g = _gen(9)
     lg = torch.randn((n, E), generator=g).to(DEV)

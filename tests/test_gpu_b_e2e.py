@@ -45,7 +45,7 @@ def test_dense_two_layer_fp32_workload(ctx):
     assert abs(cal.q.loss[0] - want["loss"]) <= 1e-3 * want["loss"]
 
 
-def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, fused=False, **over):
+def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, fused=False, act=None, **over):
     wl = workload(cfg, "cpu", **over)
     s = wl.spec
     Xs = [wl.x(l) for l in range(2)]
@@ -57,6 +57,8 @@ def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, fused=False
                          s.bits_routed, s.bits_shared, s.damp_frac, modes=modes, fused_gather=fused)
     for l in range(2):
         cal.collect(l, Xs[l].to(DEV), lgs[l].to(DEV), w)
+        if act is not None:   # the kernel the default per-call choice took (last activation call)
+            assert L.clha_last_act_kernel(ctx) == act
     torch.cuda.synchronize()
     X64 = [to64(X) for X in Xs]
     # routing counts: bit-exact
@@ -104,16 +106,17 @@ def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, fused=False
 
 def test_moe_pair_E16_top2_full_size(ctx):
     """The E=16, top-2, d_model 1024, d_ff 512 layer pair at 8192 tokens per layer, 3-bit, both
-    weightings: all Hessians and routing checked; GPTQ end to end on experts 0, 7 and 15. The expert
-    inputs go through the fused path (read from X by TMA gather4, no packed copy); the E64 case
-    below takes the packed path."""
-    _moe_pair(ctx, 2, [0, 7, 15], ("rt", "eq"), fused=True)
+    weightings: all Hessians and routing checked; GPTQ end to end on experts 0, 7 and 15. The packed
+    path, where the activation runs on the tensor cores (no outlier channels here)."""
+    _moe_pair(ctx, 2, [0, 7, 15], ("rt", "eq"), act=L.ACT_TENSOR)
 
 
 def test_moe_pair_E64_top6_shared_reduced_tokens(ctx):
     """The E=64 top-6 shape with two always-active experts (CLHA-MP: routed 2-bit, shared 3-bit),
-    Zipf-skewed routing and outlier channels, at 4096 tokens per layer."""
-    _moe_pair(ctx, 3, [0, 63], ("rt",), shared_checked=[1], tokens=4096)
+    Zipf-skewed routing and outlier channels, at 4096 tokens per layer. The fused path (the expert
+    inputs read from X by TMA gather4, no packed copy); the activation runs on the FMA kernel, which
+    the outlier channels call for."""
+    _moe_pair(ctx, 3, [0, 63], ("rt",), shared_checked=[1], fused=True, act=L.ACT_FMA, tokens=4096)
 
 
 def test_unrouted_experts_are_round_to_nearest(ctx):
