@@ -182,15 +182,18 @@ def rank_seed(rank: int) -> int:
     return 1235 + 7919 * rank
 
 
-KERNEL_SOURCES = {"act": "ffn_act.cu", "gptq": "gptq.cu", "hessian": "hessian.cu", "aggregate": "aggregate.cu",
-                  "factor": "factor.cu"}
+KERNEL_SOURCES = {"act": ("ffn_act.cu", "ffn_act_tc.cu"), "gptq": ("gptq.cu",), "hessian": ("hessian.cu",),
+                  "aggregate": ("aggregate.cu",), "factor": ("factor.cu",)}
 
 
 def source_hash(phase: str) -> str:
+    """sha1 prefix of the phase's kernel source file(s), concatenated in order."""
     import hashlib
-    path = os.path.join(ROOT, "post_quantization_expert_b200", "csrc", KERNEL_SOURCES[phase])
-    with open(path, "rb") as f:
-        return hashlib.sha1(f.read()).hexdigest()[:12]
+    h = hashlib.sha1()
+    for name in KERNEL_SOURCES[phase]:
+        with open(os.path.join(ROOT, "post_quantization_expert_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
 
 
 def measured_traffic(phase: str, workload: str):
@@ -420,6 +423,7 @@ def run_ours(args, world, rank, local):
     peaks, src = load_peaks()
     alu = alu_peaks(peaks)
     sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    act_tc = L.clha_last_act_kernel(ctx) == L.ACT_TENSOR   # the activation kernel the steps took
     kernels = {
         "hessian": ("tensor", hess_flops / 1e12, sustained, "TFLOP/s", "syrk_bf16_tc (tcgen05 kind::f16)"),
         "gptq": ("alu", gptq_flops / 1e12, alu["fp32_tflops"], "TFLOP/s",
@@ -427,7 +431,8 @@ def run_ours(args, world, rank, local):
         "factor": ("alu", factor_flops / 1e12, alu["fp64_tflops"], "TFLOP/s",
                    "fac_load + fac_dag + fac_store (fp64 tile-task graph, mma.sync m8n8k4 f64)"),
         "loss": ("alu", loss_flops / 1e12, alu["fp32_tflops"], "TFLOP/s", "loss_simt (fp32 FMA)"),
-        "act": ("alu", act_flops / 1e12, alu["fp32_tflops"], "TFLOP/s", "expert_act_simt (fp32 FMA)"),
+        "act": (("tensor", act_flops / 1e12, sustained, "TFLOP/s", "expert_act_tc (tcgen05 kind::f16)") if act_tc else
+                ("alu", act_flops / 1e12, alu["fp32_tflops"], "TFLOP/s", "expert_act_simt (fp32 FMA)")),
         "aggregate": ("hbm", agg_bytes / 1e9, peaks["hbm_gbs"], "GB/s", "agg_combine"),
     }
     # the dominant kernel: the phase that takes longest per step (each is one kernel per call, the
@@ -562,7 +567,7 @@ def run_kernel(args):
             hbuf = torch.empty((n, dff), device="cuda", dtype=torch.bfloat16)
             fn = lambda: L.clha_expert_act(ctx, X, n, dm, None, 1, Wg, Wu, dff, hbuf)
             work, unit, bound, peak = 4 * n * dm * dff / 1e12, "TFLOP/s", "alu", alu["fp32_tflops"]
-            kname = "expert_act_simt"
+            kname = "expert_act_simt (fp32 FMA)"
         elif args.workload == "dequant":
             n, d_out, d_in = dims
             bits = 3
@@ -639,6 +644,8 @@ def run_kernel(args):
             evs.append((a, b))
         torch.cuda.synchronize()
         L.clha_check(ctx)
+        if args.workload == "act" and L.clha_last_act_kernel(ctx) == L.ACT_TENSOR:   # the kernel that ran
+            bound, peak, kname = "tensor", peaks["bf16_tflops"], "expert_act_tc (tcgen05 kind::f16)"
         ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
         achieved = work / (ms / 1e3)
         print(json.dumps({"workload": args.workload, "shape": shape, "kernel": kname, "ms": ms, "achieved": achieved,
