@@ -7,8 +7,9 @@
 // Two kernels per call, both HBM-bound:
 //   agg_scalars  one block per slot: alpha (float64), lambda from the diagonals (float64 reduction),
 //                empty-slot and non-finite checks;
-//   agg_combine  one block per 32x32 upper tile pair: reads each layer's upper tile of S once and
-//                writes both the tile and its mirror image (through shared memory, coalesced).
+//   agg_combine  one block per 64x64 upper tile pair: reads each layer's upper tile of S once (16-byte
+//                loads) and writes both the tile and its mirror image (through shared memory, coalesced
+//                16-byte stores).
 #include "clha_internal.h"
 
 namespace {
@@ -70,18 +71,23 @@ __global__ void __launch_bounds__(256) agg_scalars(const float* __restrict__ S, 
     }
 }
 
+// One block per 64x64 upper tile pair (bi <= bj) of one slot: each thread combines 4 rows x 4 columns
+// of the upper tile from 16-byte loads of every layer's S (v = sum_l coef_l S_l, fused multiply-adds in
+// layer order), writes them with 16-byte stores, and the mirror tile (and, in a diagonal tile, the
+// lower half) comes transposed through shared memory.
 __global__ void __launch_bounds__(256) agg_combine(const float* __restrict__ S, const int64_t* __restrict__ counts,
                                                    int d, int L, int n_slots_total, int slot0,
                                                    const double* __restrict__ d_alpha,
                                                    const double* __restrict__ d_lambda, float* __restrict__ H_comb,
                                                    float* __restrict__ H_d, int* err) {
+    constexpr int T = 64;
     const int sl = blockIdx.y;
     const int slot = slot0 + sl;
-    const int nt = d / 32;
+    const int nt = d / T;
     int t = blockIdx.x, bi = 0;
     while (t >= nt - bi) { t -= nt - bi; ++bi; }
     const int bj = bi + t;  // bi <= bj
-    __shared__ float tile[32][33];
+    __shared__ float tile[T][T + 1];
     __shared__ float coef[CLHA_MAX_LAYERS];
     if (threadIdx.x < L) {
         int64_t n = counts[(size_t)threadIdx.x * n_slots_total + slot];
@@ -89,33 +95,55 @@ __global__ void __launch_bounds__(256) agg_combine(const float* __restrict__ S, 
     }
     __syncthreads();
     const float lam = (float)d_lambda[sl];
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+    const int c4 = (threadIdx.x & 15) * 4, r0 = threadIdx.x >> 4;   // rows r0, r0 + 16, r0 + 32, r0 + 48
+    float v[4][4];
     bool bad = false;
-    for (int r = ty; r < 32; r += 8) {
-        const int i = bi * 32 + r, j = bj * 32 + tx;
-        float v = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int r = r0 + 16 * k;
+        const size_t off = (size_t)(bi * T + r) * d + bj * T + c4;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[k][q] = 0.f;
         for (int l = 0; l < L; ++l) {
-            float c = coef[l];
-            if (c != 0.f) v = fmaf(c, S[(((size_t)l * n_slots_total + slot) * d + i) * d + j], v);
+            const float c = coef[l];
+            if (c != 0.f) {
+                const float4 sv = *reinterpret_cast<const float4*>(S + ((size_t)l * n_slots_total + slot) * d * d + off);
+                v[k][0] = fmaf(c, sv.x, v[k][0]);
+                v[k][1] = fmaf(c, sv.y, v[k][1]);
+                v[k][2] = fmaf(c, sv.z, v[k][2]);
+                v[k][3] = fmaf(c, sv.w, v[k][3]);
+            }
         }
-        if (!isfinite(v)) bad = true;
-        tile[r][tx] = v;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (!isfinite(v[k][q])) bad = true;
+            tile[r][c4 + q] = v[k][q];
+        }
     }
-    if (bad) clha_record_error(err, CLHA_ERR_NONFINITE, slot, bi * 32, KID_AGGREGATE);
+    if (bad) clha_record_error(err, CLHA_ERR_NONFINITE, slot, bi * T, KID_AGGREGATE);
     __syncthreads();
     float* Hc = H_comb ? H_comb + (size_t)sl * d * d : nullptr;
     float* Hd = H_d + (size_t)sl * d * d;
-    for (int r = ty; r < 32; r += 8) {
-        // upper tile (bi, bj): entry (r, tx); inside a diagonal tile take the upper value for r > tx
-        const int i = bi * 32 + r, j = bj * 32 + tx;
-        float v = (bi == bj && r > tx) ? tile[tx][r] : tile[r][tx];
-        if (Hc) Hc[(size_t)i * d + j] = v;
-        Hd[(size_t)i * d + j] = v + (i == j ? lam : 0.f);
-        if (bi != bj) {  // mirror tile (bj, bi): entry (r, tx) = upper (tx, r)
-            const int i2 = bj * 32 + r, j2 = bi * 32 + tx;
-            float m = tile[tx][r];
-            if (Hc) Hc[(size_t)i2 * d + j2] = m;
-            Hd[(size_t)i2 * d + j2] = m;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int r = r0 + 16 * k;
+        // upper tile (bi, bj); inside a diagonal tile entries below the diagonal take the upper value
+        float4 o;
+        float* op = reinterpret_cast<float*>(&o);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) op[q] = (bi == bj && r > c4 + q) ? tile[c4 + q][r] : v[k][q];
+        const size_t up = (size_t)(bi * T + r) * d + bj * T + c4;
+        if (Hc) *reinterpret_cast<float4*>(Hc + up) = o;
+        if (bi == bj && r >= c4 && r < c4 + 4) op[r - c4] += lam;
+        *reinterpret_cast<float4*>(Hd + up) = o;
+        if (bi != bj) {   // mirror tile (bj, bi): entry (r, c) = upper (c, r)
+            float4 m;
+            float* mp = reinterpret_cast<float*>(&m);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) mp[q] = tile[c4 + q][r];
+            const size_t lo = (size_t)(bj * T + r) * d + bi * T + c4;
+            if (Hc) *reinterpret_cast<float4*>(Hc + lo) = m;
+            *reinterpret_cast<float4*>(Hd + lo) = m;
         }
     }
 }
@@ -128,7 +156,7 @@ cudaError_t launch_aggregate(cudaStream_t s, const float* S, const int64_t* coun
     agg_scalars<<<n_slots, 256, 0, s>>>(S, counts, d, n_layers, n_slots_total, slot0, a, damp_frac, d_alpha, d_lambda,
                                         err);
     clha_note_launches(1);
-    int nt = d / 32;
+    int nt = d / 64;
     dim3 grid(nt * (nt + 1) / 2, n_slots);
     agg_combine<<<grid, 256, 0, s>>>(S, counts, d, n_layers, n_slots_total, slot0, d_alpha, d_lambda, H_comb, H_d,
                                      err);
