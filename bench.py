@@ -418,8 +418,8 @@ def run_ours(args, world, rank, local):
     loss_flops = len(modes) * sum(2 * o * i * i for o, i in mats)
     factor_flops = len(modes) * Eq * (2 * dm ** 3 // 3 + 2 * dff ** 3 // 3)
     act_flops = sum(int(c.sum()) * 4 * dm * dff for c in counts)
-    # per slot and weighting: both layers' upper tiles of S read, the damped aggregate written (full)
-    agg_bytes = len(modes) * Eq * sum(2 * (d * (d + 32) // 2) * 4 + d * d * 4 for d in (dm, dff))
+    # per slot and weighting: both layers' upper triangles of S read, the damped aggregate written (full)
+    agg_bytes = len(modes) * Eq * sum(2 * (d * (d + 1) // 2) * 4 + d * d * 4 for d in (dm, dff))
     peaks, src = load_peaks()
     alu = alu_peaks(peaks)
     sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
