@@ -157,15 +157,37 @@ __global__ void __launch_bounds__(256, 2) expert_act_simt(const int* __restrict_
 }
 
 // Per-channel max |x| over the rows (non-negative floats order like their bit patterns, so the
-// maximum is an unsigned atomicMax); one thread per channel and 256-row slab, coalesced along channels.
+// maximum is an unsigned atomicMax). A block covers 256 channels and a 256-row slab: lane l of every
+// warp reads channels 8l .. 8l+7 of a row with one 16-byte load, warp w takes the slab's rows w, w+8,
+// .., and the eight warps' maxima meet in shared memory.
 __global__ void __launch_bounds__(256) act_channel_max(const __nv_bfloat16* __restrict__ X, int64_t rows, int dm,
                                                        unsigned* __restrict__ chmax) {
-    const int c = blockIdx.x * 256 + threadIdx.x;
-    if (c >= dm) return;
+    __shared__ float part[8][256];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int c0 = blockIdx.x * 256 + lane * 8;            // dm is a multiple of 128; c0 + 7 < dm or c0 >= dm
     const int64_t r0 = (int64_t)blockIdx.y * 256, r1 = r0 + 256 < rows ? r0 + 256 : rows;
-    float m = 0.f;
-    for (int64_t r = r0; r < r1; ++r) m = fmaxf(m, fabsf(__bfloat162float(X[r * dm + c])));
-    atomicMax(chmax + c, __float_as_uint(m));
+    float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (c0 < dm) {
+        for (int64_t r = r0 + warp; r < r1; r += 8) {
+            const uint4 v = *reinterpret_cast<const uint4*>(X + r * dm + c0);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                m[2 * q] = fmaxf(m[2 * q], fabsf(__uint_as_float(w[q] << 16)));
+                m[2 * q + 1] = fmaxf(m[2 * q + 1], fabsf(__uint_as_float(w[q] & 0xffff0000u)));
+            }
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) part[warp][lane * 8 + q] = m[q];
+    __syncthreads();
+    const int c = blockIdx.x * 256 + threadIdx.x;
+    if (c < dm) {
+        float v = part[0][threadIdx.x];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) v = fmaxf(v, part[w][threadIdx.x]);
+        atomicMax(chmax + c, __float_as_uint(v));
+    }
 }
 
 // sel = 1 (tensor cores) when every channel's max |x| is within kRangeRatio of the channels' mean,
