@@ -178,123 +178,122 @@ __device__ __forceinline__ void tile_gemm_nt(const double* __restrict__ Pg, cons
                 negate ? make_double2(-c[mi][ni][0], -c[mi][ni][1]) : make_double2(c[mi][ni][0], c[mi][ni][1]);
 }
 
-// Cholesky of the 64x64 tile in T (lower, in place), its inverse X = L^-1; writes L to Lg, X to Dg,
-// X^T to Yg. Blocked by 16 columns: for each diagonal block, warp 0 factors it in
-// registers (lane r holds row r; the pivot and the scaled column are broadcast by shuffles) and
-// inverts it by forward substitution (lane j solves column j); the CTA then forms the panel below
-// it, L_ib = A_ib L_bb^-T, and applies the rank-16 update to the trailing lower triangle. The full
-// inverse is assembled from the diagonal-block inverses by three bands
-// X[i][j] = -X[i][i] (sum_m L[i][m] X[m][j]), the partial sums parked in the unused strict upper
-// triangle of T (block (j, i) holds the sums of block (i, j)).
-__device__ void tile_potrf_inv(Tile* T, Tile* X, double* dinv, double* Lg, double* Dg, double* Yg, int* err, int b,
+// Cholesky of the 64x64 tile in T (lower, in place) and its inverse X = L^-1 (lower, in Xs with
+// row pitch XLD); writes L to Lg, X to Dg, X^T to Yg. Right-looking by blocks of 8 columns (o = 8 kb),
+// three CTA barriers per block:
+//   1. warp 0 factors the 8x8 diagonal block in registers, every lane the whole block (no shuffles
+//      on the pivot chain), and lane j < 8 solves column j of its inverse X_bb. Meanwhile warps 1-7
+//      form S = L_b,<o X_<o,<o, the sums that the block row of the inverse needs: with L X = I,
+//      L_bb X_bj + S_bj = 0, so X_bj = -X_bb S_bj.
+//   2. the panel below, L_ib = A_ib X_bb^T (kept transposed in PT), and X_bj = -X_bb S_bj.
+//   3. the rank-8 update of the trailing lower triangle, A_ij -= L_ib L_jb^T, and L_ib into T.
+// Every shared access walks a row of T, Xs, S or PT across the lanes, or is a broadcast: the column
+// reads of the inverse use Xs's odd pitch (65 doubles), so they are conflict-free too.
+constexpr int XLD = NB + 1;
+constexpr int P_SCRATCH = 2 * 8 * NB;   // S [8][64] and PT [8][64]
+
+__device__ __forceinline__ constexpr int pk(int r, int c) { return r * (r + 1) / 2 + c; }   // packed lower 8x8
+
+__device__ void tile_potrf_inv(Tile* T, double* Xs, double* scr, double* Lg, double* Dg, double* Yg, int* err, int b,
                                int col_base, int d) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const double qnan = __longlong_as_double(0x7ff8000000000000ll);
+    double* S = scr;             // S[r][j]  = sum_{m < o} L[o+r][m] X[m][j],   j < o
+    double* PT = scr + 8 * NB;   // PT[c][i] = L[i][o+c],                      i >= o + 8
     int bad = -1;   // first non-positive pivot (warp 0)
-    for (int kb = 0; kb < 4; ++kb) {
-        const int o = 16 * kb;
+    for (int kb = 0; kb < 8; ++kb) {
+        const int o = 8 * kb;
         if (warp == 0) {
-            const int rr = lane & 15;   // lanes 16..31 shadow lanes 0..15 and write nothing
-            double a[16];
+            double a[36];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) a[c] = T[o + rr][o + c];
+            for (int r = 0; r < 8; ++r)
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const double p = __shfl_sync(0xffffffffu, a[c], c);
+                for (int c = 0; c <= r; ++c) a[pk(r, c)] = T[o + r][o + c];
+            double inv[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const double p = a[pk(c, c)];
                 const bool ok = (p > 0.0) && isfinite(p);
                 if (!ok && bad < 0) bad = o + c;
-                const double inv = ok ? rsqrt(p) : qnan;
-                const double l = (rr == c) ? p * inv : a[c] * inv;
-                a[c] = l;
+                inv[c] = ok ? rsqrt(p) : qnan;
+                a[pk(c, c)] = p * inv[c];
 #pragma unroll
-                for (int cc = 1; cc < 16; ++cc) {   // constant trip count keeps a[] in registers
-                    if (cc > c) {
-                        const double lcc = __shfl_sync(0xffffffffu, l, cc);
-                        if (rr >= cc) a[cc] = fma(-l, lcc, a[cc]);
-                    }
-                }
-                if (lane == c) dinv[o + c] = inv;
-            }
-            if (lane < 16) {
+                for (int r = c + 1; r < 8; ++r) a[pk(r, c)] *= inv[c];
 #pragma unroll
-                for (int c = 0; c < 16; ++c) T[o + rr][o + c] = (c <= rr) ? a[c] : 0.0;
+                for (int r = c + 1; r < 8; ++r)
+#pragma unroll
+                    for (int k = c + 1; k <= r; ++k) a[pk(r, k)] = fma(-a[pk(r, c)], a[pk(k, c)], a[pk(r, k)]);
             }
-            __syncwarp();
-            if (lane < 16) {   // column j = lane of the diagonal block's inverse (this lane's own X column)
+            if (lane == 0) {
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+#pragma unroll
+                    for (int c = 0; c <= r; ++c) T[o + r][o + c] = a[pk(r, c)];
+            }
+            if (lane < 8) {   // column j of X_bb: L_bb x = e_j, 1 / L_rr = inv[r]
                 const int j = lane;
+                double x[8];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    double s = (r == j) ? 1.0 : 0.0;
+                for (int r = 0; r < 8; ++r) {
+                    double sum = (r == j) ? 1.0 : 0.0;
 #pragma unroll
-                    for (int m = 0; m < r; ++m) s -= (m >= j) ? T[o + r][o + m] * X[o + m][o + j] : 0.0;
-                    X[o + r][o + j] = (r >= j) ? s * dinv[o + r] : 0.0;
+                    for (int m = 0; m < r; ++m) sum = (m >= j) ? fma(-a[pk(r, m)], x[m], sum) : sum;
+                    x[r] = (r >= j) ? sum * inv[r] : 0.0;
+                    Xs[(o + r) * XLD + o + j] = x[r];
                 }
+            }
+        } else {
+            for (int e = tid - 32; e < 8 * o; e += 224) {
+                const int r = e / o, j = e - r * o;
+                double s0 = 0.0, s1 = 0.0;
+                int m = j;
+                for (; m + 1 < o; m += 2) {
+                    s0 = fma(T[o + r][m], Xs[m * XLD + j], s0);
+                    s1 = fma(T[o + r][m + 1], Xs[(m + 1) * XLD + j], s1);
+                }
+                if (m < o) s0 = fma(T[o + r][m], Xs[m * XLD + j], s0);
+                S[r * NB + j] = s0 + s1;
             }
         }
         __syncthreads();
-        const int rows = 48 - o;   // rows below the diagonal block
-        if (rows > 0) {
-            double v[3];
-#pragma unroll
-            for (int it = 0; it < 3; ++it) {   // L[i][o+c] = sum_{k<=c} A[i][o+k] Xbb[c][k]
-                const int e = it * 256 + tid;
+        const int npanel = (56 - o) * 8;   // panel entries; with the 8 o entries of X_b,<o always 448
+        for (int e = tid; e < 448; e += 256) {
+            if (e < npanel) {
+                const int i = o + 8 + (e >> 3), c = e & 7;
                 double acc = 0.0;
-                if (e < rows * 16) {
-                    const int i = o + 16 + (e >> 4), c = e & 15;
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) acc = (k <= c) ? fma(T[i][o + k], X[o + c][o + k], acc) : acc;
-                }
-                v[it] = acc;
-            }
-            __syncthreads();
+                for (int k = 0; k < 8; ++k) acc = (k <= c) ? fma(T[i][o + k], Xs[(o + c) * XLD + o + k], acc) : acc;
+                PT[c * NB + i] = acc;
+            } else {
+                const int f = e - npanel, r = f / o, j = f - r * o;
+                double acc = 0.0;
 #pragma unroll
-            for (int it = 0; it < 3; ++it) {
-                const int e = it * 256 + tid;
-                if (e < rows * 16) T[o + 16 + (e >> 4)][o + (e & 15)] = v[it];
+                for (int q = 0; q < 8; ++q) acc = (q <= r) ? fma(Xs[(o + r) * XLD + o + q], S[q * NB + j], acc) : acc;
+                Xs[(o + r) * XLD + j] = -acc;
             }
-            __syncthreads();
-            for (int e = tid; e < rows * rows; e += 256) {   // trailing lower triangle, rank 16
-                const int i = o + 16 + e / rows, j = o + 16 + e % rows;
-                if (j <= i) {
-                    double acc = T[i][j];
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) acc = fma(-T[i][o + k], T[j][o + k], acc);
-                    T[i][j] = acc;
-                }
-            }
-            __syncthreads();
         }
+        __syncthreads();
+        for (int i = o + 8 + warp; i < NB; i += 8) {
+            double li[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) li[c] = PT[c * NB + i];
+            for (int j = o + 8 + lane; j <= i; j += 32) {
+                double acc = T[i][j];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc = fma(-li[c], PT[c * NB + j], acc);
+                T[i][j] = acc;
+            }
+            if (lane < 8) T[i][o + lane] = PT[lane * NB + i];
+        }
+        __syncthreads();
     }
     if (tid == 0 && bad >= 0) clha_record_error(err, CLHA_ERR_NOT_PD, b, d - 1 - (col_base + bad), KID_FACTOR);
-    for (int i = tid; i < TILE_ELEMS; i += 256) {   // strict upper blocks of X are zero
-        const int r = i >> 6, c = i & 63;
-        if ((c >> 4) > (r >> 4)) X[r][c] = 0.0;
-    }
-    __syncthreads();
-    for (int delta = 1; delta < 4; ++delta) {       // bands; Tp[r][s] of block (i, j) sits at T[16j+r][16i+s]
-        const int nblk = 4 - delta;
-        for (int e = tid; e < nblk * 256; e += 256) {
-            const int j = e >> 8, i = j + delta, r = (e >> 4) & 15, s = e & 15;
-            double acc = 0.0;
-            for (int m = 16 * j; m < 16 * i; ++m) acc = fma(T[16 * i + r][m], X[m][16 * j + s], acc);
-            T[16 * j + r][16 * i + s] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < nblk * 256; e += 256) {
-            const int j = e >> 8, i = j + delta, r = (e >> 4) & 15, s = e & 15;
-            double acc = 0.0;
-#pragma unroll
-            for (int q = 0; q < 16; ++q) acc = fma(X[16 * i + r][16 * i + q], T[16 * j + q][16 * i + s], acc);
-            X[16 * i + r][16 * j + s] = -acc;
-        }
-        __syncthreads();
-    }
 #pragma unroll 4
     for (int e = tid; e < TILE_ELEMS; e += 256) {
         const int r = e >> 6, c = e & 63;
         Lg[e] = (c <= r) ? T[r][c] : 0.0;
-        Dg[e] = X[r][c];
-        Yg[e] = X[c][r];
+        Dg[e] = (c <= r) ? Xs[r * XLD + c] : 0.0;
+        Yg[e] = (r <= c) ? Xs[c * XLD + r] : 0.0;
     }
 }
 
@@ -375,8 +374,8 @@ __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
     extern __shared__ double dsm[];
     Tile* T0 = reinterpret_cast<Tile*>(dsm);
     Tile* T1 = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
-    double* dinv = dsm + 2 * TILE_DOUBLES;
-    unsigned long long* lvl = reinterpret_cast<unsigned long long*>(dinv + NB);   // [max_nt + 2] stage starts
+    double* scr = dsm + 2 * TILE_DOUBLES;   // the diagonal task's S and PT
+    unsigned long long* lvl = reinterpret_cast<unsigned long long*>(scr + P_SCRATCH);   // [max_nt + 2] stage starts
     __shared__ unsigned long long s_ticket, s_next;   // s_next: thread 0's prefetched number
     __shared__ int s_ok;
     const int S = g.max_nt, tid = threadIdx.x, lane = tid & 31;
@@ -500,7 +499,7 @@ __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
             tile_to_smem(T0, tile(G.A, G, b, m, m));
             cp_async_wait_all();
             __syncthreads();
-            tile_potrf_inv(T0, T1, dinv, tile(G.A, G, b, m, m), Dm, tile(G.Y, G, b, m, m), g.err, prob, NB * m, G.d);
+            tile_potrf_inv(T0, reinterpret_cast<double*>(T1), scr, tile(G.A, G, b, m, m), Dm, tile(G.Y, G, b, m, m), g.err, prob, NB * m, G.d);
             __syncthreads();
             if (tid == 0) st_release(st(G.stY, G, b, m, m), 1);
         } else {
@@ -513,7 +512,7 @@ __global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
 }
 
 constexpr size_t dag_smem_bytes(int nt) {
-    return (size_t)2 * TILE_DOUBLES * sizeof(double) + NB * sizeof(double) + (size_t)(nt + 2) * sizeof(unsigned long long);
+    return (size_t)(2 * TILE_DOUBLES + P_SCRATCH) * sizeof(double) + (size_t)(nt + 2) * sizeof(unsigned long long);
 }
 
 }  // namespace

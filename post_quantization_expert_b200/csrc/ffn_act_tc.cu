@@ -10,7 +10,7 @@
 //              MMA produces the gate and the up pre-activations side by side. K is cut into up to 8
 //              chunks, each accumulated into its own 64 TMEM columns and handed over as soon as it is
 //              done, so the epilogue reads chunk c while chunk c+1 runs.
-//   warps 2-9  epilogue, two warps per TMEM lane quadrant, each half of the tile's columns: the chunk
+//   warps 2-17 epilogue, four warps per TMEM lane quadrant, each a quarter of the tile's columns: the chunk
 //              sums are added in fp64, h = SiLU(g) * u is evaluated in fp64 and rounded once to bf16
 //              (as the fp32-FMA kernel does).
 // Products of bf16 values are exact, but the tensor core adds a group's products after aligning them
@@ -31,8 +31,8 @@ constexpr int B_BYTES = 2 * BNH * BK * 2;       // 8 KB (gate rows then up rows)
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * NCH + 1) + 16;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + BAR_BYTES;
-constexpr int kThreads = 320;                   // producer, MMA issuer, 8 epilogue warps
-constexpr int EPI = 256;                         // epilogue threads
+constexpr int kThreads = 576;                   // producer, MMA issuer, 16 epilogue warps
+constexpr int EPI = 512;                         // epilogue threads
 constexpr uint32_t IDESC = tc::idesc_f32acc(1 /*bf16*/, 0 /*K-major*/, 0 /*K-major*/, BM, 2 * BNH);
 
 struct ActParams {
@@ -172,17 +172,17 @@ expert_act_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         }
         __syncwarp();
     } else {
-        // warps 2-9: warp w reads TMEM lanes 32 (w % 4) .. (its quadrant) and half (w - 2) / 4 of the
-        // tile's 32 h-columns (16 gate and 16 up values per row and chunk)
-        const int q = warp & 3, half = (warp - 2) >> 2;
-        constexpr int HW = BNH / 2;
+        // warps 2-17: warp w reads TMEM lanes 32 (w % 4) .. (its quadrant) and quarter (w - 2) / 4 of
+        // the tile's 32 h-columns (8 gate and 8 up values per row and chunk)
+        const int q = warp & 3, quarter = (warp - 2) >> 2;
+        constexpr int HW = BNH / 4;
         int tcount = 0;
         int64_t m0, vend;
         int n0, e;
         bool ok = true;
         for (int64_t w = blockIdx.x; ok && decode(p, m_tiles, w, m0, n0, e, vend); w += gridDim.x) {
             const int64_t row = m0 + q * 32 + lane;
-            const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + half * HW;
+            const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + quarter * HW;
             double g[HW], u[HW];
 #pragma unroll
             for (int j = 0; j < HW; ++j) { g[j] = 0.0; u[j] = 0.0; }
@@ -190,8 +190,8 @@ expert_act_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 if (!tc::mbar_wait_bounded(cfull0 + 8 * c, tcount & 1, abort_flag)) { ok = false; break; }
                 tc::fence_after_sync();
                 uint32_t vg[HW], vu[HW];
-                tc::tmem_ld_32x32b_x16(tb + c * (2 * BNH), vg);          // gate pre-activation, chunk c
-                tc::tmem_ld_32x32b_x16(tb + c * (2 * BNH) + BNH, vu);    // up pre-activation, chunk c
+                tc::tmem_ld_32x32b_x8(tb + c * (2 * BNH), vg);           // gate pre-activation, chunk c
+                tc::tmem_ld_32x32b_x8(tb + c * (2 * BNH) + BNH, vu);     // up pre-activation, chunk c
                 tc::tmem_wait_ld();
                 tc::fence_before_sync();
                 tc::mbar_arrive(cempty0 + 8 * c);
@@ -212,9 +212,8 @@ expert_act_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     out[j / 2] = (uint32_t)__bfloat16_as_ushort(__double2bfloat16(h0)) |
                                  ((uint32_t)__bfloat16_as_ushort(__double2bfloat16(h1)) << 16);
                 }
-                uint4* dst = reinterpret_cast<uint4*>(p.h + row * p.dff + n0 + half * HW);
+                uint4* dst = reinterpret_cast<uint4*>(p.h + row * p.dff + n0 + quarter * HW);
                 dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-                dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
             }
             ++tcount;
         }
