@@ -48,6 +48,9 @@ constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;
 
 typedef double Tile[LD];
 
+// Barrier of the graph kernel's 256 compute threads (the scheduler warp does not take part).
+__device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t gtimer() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -153,7 +156,7 @@ __device__ __forceinline__ void tile_gemm_nt(const double* __restrict__ Pg, cons
             }
         }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
-    __syncthreads();
+    cbar();
 #pragma unroll 2
     for (int k0 = 0; k0 < NB; k0 += 8) {
         double2 a[4], bq[2];
@@ -255,7 +258,7 @@ __device__ void tile_potrf_inv(Tile* T, double* Xs, double* scr, double* Lg, dou
                 S[r * NB + j] = s0 + s1;
             }
         }
-        __syncthreads();
+        cbar();
         const int npanel = (56 - o) * 8;   // panel entries; with the 8 o entries of X_b,<o always 448
         for (int e = tid; e < 448; e += 256) {
             if (e < npanel) {
@@ -272,7 +275,7 @@ __device__ void tile_potrf_inv(Tile* T, double* Xs, double* scr, double* Lg, dou
                 Xs[(o + r) * XLD + j] = -acc;
             }
         }
-        __syncthreads();
+        cbar();
         for (int i = o + 8 + warp; i < NB; i += 8) {
             double li[8];
 #pragma unroll
@@ -285,7 +288,7 @@ __device__ void tile_potrf_inv(Tile* T, double* Xs, double* scr, double* Lg, dou
             }
             if (lane < 8) T[i][o + lane] = PT[lane * NB + i];
         }
-        __syncthreads();
+        cbar();
     }
     if (tid == 0 && bad >= 0) clha_record_error(err, CLHA_ERR_NOT_PD, b, d - 1 - (col_base + bad), KID_FACTOR);
 #pragma unroll 4
@@ -299,6 +302,8 @@ __device__ void tile_potrf_inv(Tile* T, double* Xs, double* scr, double* Lg, dou
 
 // ------------------------------------------------------------------------------ the task graph
 constexpr int MAX_GROUPS = 4;
+constexpr int CW = 256;                 // compute threads (8 warps)
+constexpr int DAG_THREADS = CW + 32;    // + the scheduler warp
 
 // One group: `batch` problems of the same size d (nt = d / 64 tiles per side), its own workspace.
 struct Grp {
@@ -370,144 +375,205 @@ __device__ __forceinline__ unsigned long long stage_total(int nt, int s) {
     return (unsigned long long)(n[0] + n[1] + n[2] + n[3] + n[4] + n[5]);
 }
 
-__global__ void __launch_bounds__(256, 2) fac_dag(Dag g) {
+// A decoded task: class q (0 P, 1 S, 2/5 G, 3 F, 4 Q), group k, problem b of the group, level m,
+// tiles i, j; its inputs' states to wait for; its outputs' states once done.
+struct Task {
+    int q, k, b, m, i, j;
+    int status;                   // READY, WAIT (its inputs were not all ready yet), STOP
+};
+constexpr int READY = 0, WAIT = 1, STOP = 2;
+struct Deps {
+    const int* wp[3];
+    int wt[3];
+    int* out;                     // output state and its new value
+    int out_value;
+    int* out2;                    // P(m) also completes Y_mm (state 1)
+};
+
+__device__ __forceinline__ void decode_task(const Dag& g, const unsigned long long* lvl, unsigned long long t, Task& d,
+                                            Deps& dp) {
+    const int S = g.max_nt;
+    int lo = 0, hi = S;   // stage: last s with lvl[s] <= t
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (lvl[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    const int sg = lo;
+    // within a stage every count fits in 32 bits (a stage holds at most batch x ~nt^2 tasks):
+    // 32-bit arithmetic keeps the decode off the 64-bit division path
+    uint32_t r = (uint32_t)(t - lvl[sg]);
+    int k = 0;
+    bool found = false;
+#pragma unroll
+    for (int kk = 0; kk < MAX_GROUPS; ++kk) {
+        if (!found && kk < g.ng) {
+            const uint32_t c = (uint32_t)stage_total(g.grp[kk].nt, sg) * (uint32_t)g.grp[kk].batch;
+            if (r < c) { k = kk; found = true; }
+            else r -= c;
+        }
+    }
+    const Grp& G = g.grp[k];
+    const int nt = G.nt;
+    const uint32_t batch = (uint32_t)G.batch;
+    long long n[6];
+    stage_counts(nt, sg, n);
+    int c = 0;
+#pragma unroll
+    for (int cq = 0; cq < 6; ++cq)
+        if (c == cq && r >= (uint32_t)n[cq] * batch) { r -= (uint32_t)n[cq] * batch; ++c; }
+    const uint32_t local = r / batch;
+    const int b = (int)(r - local * batch);
+    int q, m = sg - 1, i = 0, j = 0;
+    if (c == 0) { q = 2; i = m + 1 + (int)local; j = m + 1; }
+    else if (c == 1) { q = 0; m = sg; }
+    else if (c == 2) { q = 3; j = (int)local; }
+    else if (c == 3) {
+        q = 4;
+        const uint32_t ii = local / (uint32_t)(m + 1);
+        i = m + 1 + (int)ii;
+        j = (int)(local - ii * (uint32_t)(m + 1));
+    } else if (c == 4) {
+        q = 5;
+        int rem = (int)local;
+        j = m + 2;
+        while (rem >= nt - j) { rem -= nt - j; ++j; }
+        i = j + rem;
+    } else { q = 1; m = sg; i = m + 1 + (int)local; j = m; }
+    d.q = q; d.k = k; d.b = b; d.m = m; d.i = i; d.j = j;
+    dp.wp[0] = dp.wp[1] = dp.wp[2] = nullptr;
+    dp.wt[0] = dp.wt[1] = dp.wt[2] = 0;
+    dp.out2 = nullptr;
+    if (q == 0) {            // P(m)
+        dp.wp[0] = st(G.stA, G, b, m, m); dp.wt[0] = m;
+        dp.out = st(G.stA, G, b, m, m); dp.out_value = m + 1;
+        dp.out2 = st(G.stY, G, b, m, m);
+    } else if (q == 1) {     // L_im = A_im D_m^T
+        dp.wp[0] = st(G.stA, G, b, i, m); dp.wt[0] = m;
+        dp.wp[1] = st(G.stA, G, b, m, m); dp.wt[1] = m + 1;
+        dp.out = st(G.stA, G, b, i, m); dp.out_value = m + 1;
+    } else if (q == 2 || q == 5) {   // A_ij -= L_im L_jm^T
+        dp.wp[0] = st(G.stA, G, b, i, m); dp.wt[0] = m + 1;
+        dp.wp[1] = st(G.stA, G, b, j, m); dp.wt[1] = m + 1;
+        dp.wp[2] = st(G.stA, G, b, i, j); dp.wt[2] = m;
+        dp.out = st(G.stA, G, b, i, j); dp.out_value = m + 1;
+    } else if (q == 3) {     // Y_jm = -R_jm D_m^T
+        dp.wp[0] = st(G.stY, G, b, j, m); dp.wt[0] = m - j;
+        dp.wp[1] = st(G.stA, G, b, m, m); dp.wt[1] = m + 1;
+        dp.out = st(G.stY, G, b, j, m); dp.out_value = m - j + 1;
+    } else {                 // R_ji (+)= Y_jm L_im^T
+        dp.wp[0] = st(G.stY, G, b, j, m); dp.wt[0] = m - j + 1;
+        dp.wp[1] = st(G.stA, G, b, i, m); dp.wt[1] = m + 1;
+        dp.wp[2] = st(G.stY, G, b, j, i); dp.wt[2] = m - j;
+        dp.out = st(G.stY, G, b, j, i); dp.out_value = m - j + 1;
+    }
+}
+
+// Warps 0-7 run tasks; warp 8 schedules them. While the compute warps run task n - 1, the scheduler
+// takes the next number, decodes it into task n and checks its inputs' states once, then meets the
+// compute warps at the CTA barrier that ends task n - 1 (the task descriptors are double-buffered),
+// and after it releases task n - 1's outputs (cumulative over the compute warps' stores, which the
+// barrier orders before it). When an input was not ready, the descriptor says WAIT: the scheduler
+// releases the finished task first, then waits for the inputs and meets the compute warps at a second
+// barrier (READY or STOP). Releasing every finished task before any blocking wait keeps the schedule
+// deadlock-free: tasks are taken in number order, every task waited on has a smaller number, and the
+// smallest unfinished number is always either running or waiting only on finished, released tasks.
+__global__ void __launch_bounds__(DAG_THREADS, 2) fac_dag(Dag g) {
     extern __shared__ double dsm[];
     Tile* T0 = reinterpret_cast<Tile*>(dsm);
     Tile* T1 = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
     double* scr = dsm + 2 * TILE_DOUBLES;   // the diagonal task's S and PT
     unsigned long long* lvl = reinterpret_cast<unsigned long long*>(scr + P_SCRATCH);   // [max_nt + 2] stage starts
-    __shared__ unsigned long long s_ticket, s_next;   // s_next: thread 0's prefetched number
-    __shared__ int s_ok;
-    const int S = g.max_nt, tid = threadIdx.x, lane = tid & 31;
-    if (tid == 0) {   // stage s holds, group after group, stage s of every group that has one
-        unsigned long long acc = 0;
-        for (int s = 0; s <= S; ++s) {
-            lvl[s] = acc;
-            for (int k = 0; k < g.ng; ++k) acc += stage_total(g.grp[k].nt, s) * g.grp[k].batch;
-        }
-        lvl[S + 1] = acc;
-    }
-    // Thread 0 holds the next number while the CTA runs the current task (taking numbers in order
-    // and running them in order keeps the schedule deadlock-free).
-    // The number of the next task is published in s_ticket before the barrier that ends the current
-    // one (every thread has read the current number before the dependency barrier).
-    if (tid == 0) s_ticket = atomicAdd(g.ticket, 1ull);
-    __syncthreads();
+    __shared__ Task s_task[2];
+    __shared__ int s_final[2];   // a WAIT task's final status (READY or STOP), read after the second barrier
+    const int tid = threadIdx.x, lane = tid & 31;
 
-    for (;;) {
-        const unsigned long long t = s_ticket;
-        if (t >= g.total) break;
-        if (tid == 0) s_next = atomicAdd(g.ticket, 1ull);
-        // decode: stage, group, class, problem, task (q: 0 P, 1 S, 2/5 G, 3 F, 4 Q), level m, tiles i, j
-        int lo = 0, hi = S;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (lvl[mid] <= t) lo = mid; else hi = mid - 1;
-        }
-        const int sg = lo;
-        // within a stage every count fits in 32 bits (a stage holds at most batch x ~nt^2 tasks):
-        // 32-bit arithmetic keeps the decode off the 64-bit division path
-        uint32_t r = (uint32_t)(t - lvl[sg]);
-        Grp G = g.grp[0];
-        bool found = false;
-#pragma unroll
-        for (int k = 0; k < MAX_GROUPS; ++k) {   // (unrolled: the group record stays in registers)
-            if (!found && k < g.ng) {
-                const uint32_t c = (uint32_t)stage_total(g.grp[k].nt, sg) * (uint32_t)g.grp[k].batch;
-                if (r < c) { G = g.grp[k]; found = true; }
-                else r -= c;
+    if (tid >= CW) {
+        // ---------------------------------------------------------------- scheduler (warp 8)
+        const int S = g.max_nt;
+        if (lane == 0) {   // stage s holds, group after group, stage s of every group that has one
+            unsigned long long acc = 0;
+            for (int s = 0; s <= S; ++s) {
+                lvl[s] = acc;
+                for (int k = 0; k < g.ng; ++k) acc += stage_total(g.grp[k].nt, s) * g.grp[k].batch;
             }
+            lvl[S + 1] = acc;
         }
-        const int nt = G.nt;
-        const uint32_t batch = (uint32_t)G.batch;
-        long long n[6];
-        stage_counts(nt, sg, n);
-        int c = 0;
-#pragma unroll
-        for (int cq = 0; cq < 6; ++cq)   // (unrolled: n[] stays in registers)
-            if (c == cq && r >= (uint32_t)n[cq] * batch) { r -= (uint32_t)n[cq] * batch; ++c; }
-        const uint32_t local = r / batch;
-        const int b = (int)(r - local * batch);
-        const int prob = G.pbase + b;
-        int q, m = sg - 1, i = 0, j = 0;
-        if (c == 0) { q = 2; i = m + 1 + (int)local; j = m + 1; }
-        else if (c == 1) { q = 0; m = sg; }
-        else if (c == 2) { q = 3; j = (int)local; }
-        else if (c == 3) {
-            q = 4;
-            const uint32_t ii = local / (uint32_t)(m + 1);
-            i = m + 1 + (int)ii;
-            j = (int)(local - ii * (uint32_t)(m + 1));
-        } else if (c == 4) {
-            q = 5;
-            int rem = (int)local;
-            j = m + 2;
-            while (rem >= nt - j) { rem -= nt - j; ++j; }
-            i = j + rem;
-        } else { q = 1; m = sg; i = m + 1 + (int)local; j = m; }
+        __syncwarp();
+        int* run_out = nullptr;   // outputs of the task the compute warps are running
+        int* run_out2 = nullptr;
+        int run_value = 0;
+        int slot = 0;
+        for (;;) {
+            unsigned long long t = 0;
+            if (lane == 0) t = atomicAdd(g.ticket, 1ull);
+            t = __shfl_sync(0xffffffffu, t, 0);
+            Task d;
+            Deps dp;
+            d.status = STOP;
+            const int* wpl = nullptr;   // lane k < 3 checks input k
+            int wtl = 0;
+            if (t < g.total && !*reinterpret_cast<volatile int*>(g.abort_flag)) {
+                decode_task(g, lvl, t, d, dp);
+                if (lane < 3) { wpl = dp.wp[lane]; wtl = dp.wt[lane]; }
+                const bool ready = !wpl || ld_acquire(wpl) >= wtl;
+                d.status = __all_sync(0xffffffffu, ready) ? READY : WAIT;
+            }
+            if (lane == 0) s_task[slot] = d;
+            __syncwarp();
+            __syncthreads();   // end of the running task; the compute warps read s_task[slot]
+            if (lane == 0 && run_out) {
+                if (run_out2) st_release(run_out2, 1);
+                st_release(run_out, run_value);
+            }
+            if (d.status == WAIT) {
+                bool ok = !wpl || wait_ge(wpl, wtl, g, g.grp[d.k].pbase + d.b);
+                ok = __all_sync(0xffffffffu, ok);
+                if (lane == 0) s_final[slot] = ok ? READY : STOP;
+                __syncwarp();
+                __syncthreads();   // the compute warps read the final status
+                if (!ok) break;
+            } else if (d.status == STOP) {
+                break;
+            }
+            run_out = dp.out;
+            run_out2 = dp.out2;
+            run_value = dp.out_value;
+            slot ^= 1;
+        }
+        return;
+    }
 
-        // operands, output and the states to wait for (lane k of warp 0 polls condition k)
-        const double *P = nullptr, *Qm = nullptr;
-        double* C = nullptr;
-        bool load_c = false, negate = false;
-        int* out_state;
-        int out_value;
-        const int* wp[3] = {nullptr, nullptr, nullptr};
-        int wt[3] = {0, 0, 0};
-        double* Dm = G.D + ((size_t)b * nt + m) * TILE_ELEMS;
+    // -------------------------------------------------------------------- compute (warps 0-7)
+    int slot = 0;
+    for (;;) {
+        __syncthreads();   // the scheduler has published the next task
+        Task d = s_task[slot];
+        if (d.status == WAIT) {
+            __syncthreads();
+            d.status = s_final[slot];
+        }
+        if (d.status != READY) break;
+        slot ^= 1;
+        const Grp& G = g.grp[d.k];
+        const int q = d.q, b = d.b, m = d.m, i = d.i, j = d.j;
+        double* Dm = G.D + ((size_t)b * G.nt + m) * TILE_ELEMS;
         if (q == 0) {            // P(m)
-            wp[0] = st(G.stA, G, b, m, m); wt[0] = m;
-            out_state = st(G.stA, G, b, m, m); out_value = m + 1;
-        } else if (q == 1) {     // L_im = A_im D_m^T
-            wp[0] = st(G.stA, G, b, i, m); wt[0] = m;
-            wp[1] = st(G.stA, G, b, m, m); wt[1] = m + 1;
-            P = tile(G.A, G, b, i, m); Qm = Dm; C = tile(G.A, G, b, i, m);
-            out_state = st(G.stA, G, b, i, m); out_value = m + 1;
-        } else if (q == 2 || q == 5) {   // A_ij -= L_im L_jm^T
-            wp[0] = st(G.stA, G, b, i, m); wt[0] = m + 1;
-            wp[1] = st(G.stA, G, b, j, m); wt[1] = m + 1;
-            wp[2] = st(G.stA, G, b, i, j); wt[2] = m;
-            P = tile(G.A, G, b, i, m); Qm = tile(G.A, G, b, j, m); C = tile(G.A, G, b, i, j);
-            load_c = true; negate = true;
-            out_state = st(G.stA, G, b, i, j); out_value = m + 1;
-        } else if (q == 3) {     // Y_jm = -R_jm D_m^T
-            wp[0] = st(G.stY, G, b, j, m); wt[0] = m - j;
-            wp[1] = st(G.stA, G, b, m, m); wt[1] = m + 1;
-            P = tile(G.Y, G, b, j, m); Qm = Dm; C = tile(G.Y, G, b, j, m);
-            negate = true;
-            out_state = st(G.stY, G, b, j, m); out_value = m - j + 1;
-        } else {                 // R_ji (+)= Y_jm L_im^T
-            wp[0] = st(G.stY, G, b, j, m); wt[0] = m - j + 1;
-            wp[1] = st(G.stA, G, b, i, m); wt[1] = m + 1;
-            wp[2] = st(G.stY, G, b, j, i); wt[2] = m - j;
-            P = tile(G.Y, G, b, j, m); Qm = tile(G.A, G, b, i, m); C = tile(G.Y, G, b, j, i);
-            load_c = (m != j);
-            out_state = st(G.stY, G, b, j, i); out_value = m - j + 1;
-        }
-        if (tid < 32) {
-            bool ok = true;
-#pragma unroll
-            for (int k = 0; k < 3; ++k)
-                if (lane == k && wp[k]) ok = wait_ge(wp[k], wt[k], g, prob);
-            ok = __all_sync(0xffffffffu, ok);
-            if (lane == 0) s_ok = ok;
-        }
-        __syncthreads();
-        if (!s_ok) break;
-
-        if (q == 0) {
             tile_to_smem(T0, tile(G.A, G, b, m, m));
             cp_async_wait_all();
-            __syncthreads();
-            tile_potrf_inv(T0, reinterpret_cast<double*>(T1), scr, tile(G.A, G, b, m, m), Dm, tile(G.Y, G, b, m, m), g.err, prob, NB * m, G.d);
-            __syncthreads();
-            if (tid == 0) st_release(st(G.stY, G, b, m, m), 1);
-        } else {
-            tile_gemm_nt(P, Qm, T0, T1, C, load_c, negate);
+            cbar();
+            tile_potrf_inv(T0, reinterpret_cast<double*>(T1), scr, tile(G.A, G, b, m, m), Dm, tile(G.Y, G, b, m, m),
+                           g.err, G.pbase + b, NB * m, G.d);
+        } else if (q == 1) {     // L_im = A_im D_m^T
+            tile_gemm_nt(tile(G.A, G, b, i, m), Dm, T0, T1, tile(G.A, G, b, i, m), false, false);
+        } else if (q == 2 || q == 5) {   // A_ij -= L_im L_jm^T
+            tile_gemm_nt(tile(G.A, G, b, i, m), tile(G.A, G, b, j, m), T0, T1, tile(G.A, G, b, i, j), true, true);
+        } else if (q == 3) {     // Y_jm = -R_jm D_m^T
+            tile_gemm_nt(tile(G.Y, G, b, j, m), Dm, T0, T1, tile(G.Y, G, b, j, m), false, true);
+        } else {                 // R_ji (+)= Y_jm L_im^T
+            tile_gemm_nt(tile(G.Y, G, b, j, m), tile(G.A, G, b, i, m), T0, T1, tile(G.Y, G, b, j, i), m != j, false);
         }
-        if (tid == 0) s_ticket = *reinterpret_cast<volatile int*>(g.abort_flag) ? g.total : s_next;
-        __syncthreads();   // every thread's stores issued; shared tiles free for the next task
-        if (tid == 0) st_release(out_state, out_value);   // release: cumulative over the CTA's stores
+        // the barrier at the top of the loop ends the task: every compute thread's stores are issued
+        // before the scheduler's release, and the shared tiles are free for the next task's copies
     }
 }
 
@@ -609,7 +675,7 @@ cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups
     }
     unsigned long long grid = 2ull * (unsigned long long)num_sms;   // two resident CTAs per SM
     if (grid > g.total) grid = g.total;
-    fac_dag<<<(unsigned)grid, 256, smem, s>>>(g);
+    fac_dag<<<(unsigned)grid, DAG_THREADS, smem, s>>>(g);
     clha_note_launches(1);
     for (int k = 0; k < n; ++k) {
         const Grp& G = g.grp[k];
