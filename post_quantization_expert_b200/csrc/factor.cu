@@ -185,108 +185,171 @@ __device__ __forceinline__ void tile_gemm_nt(const double* __restrict__ Pg, cons
 // row pitch XLD); writes L to Lg, X to Dg, X^T to Yg. Right-looking by blocks of 8 columns (o = 8 kb),
 // three CTA barriers per block:
 //   1. warp 0 factors the 8x8 diagonal block in registers, every lane the whole block (no shuffles
-//      on the pivot chain), and lane j < 8 solves column j of its inverse X_bb. Meanwhile warps 1-7
+//      on the pivot chain; two 4-column stages keep the live values few), and lane j < 8 solves
+//      column j of its inverse X_bb. Meanwhile warps 1-7
 //      form S = L_b,<o X_<o,<o, the sums that the block row of the inverse needs: with L X = I,
 //      L_bb X_bj + S_bj = 0, so X_bj = -X_bb S_bj.
 //   2. the panel below, L_ib = A_ib X_bb^T (kept transposed in PT), and X_bj = -X_bb S_bj.
 //   3. the rank-8 update of the trailing lower triangle, A_ij -= L_ib L_jb^T, and L_ib into T.
-// Every shared access walks a row of T, Xs, S or PT across the lanes, or is a broadcast: the column
-// reads of the inverse use Xs's odd pitch (65 doubles), so they are conflict-free too.
+// The products of steps 1-3 are 8x8 blocks on the FP64 tensor path (m8n8k4, k = 8 in two steps), one
+// block per warp at a time; only the pivot chain of step 1 runs as scalar fp64 arithmetic.
+// The inverse's column reads use Xs's odd pitch (65 doubles), so they are conflict-free.
 constexpr int XLD = NB + 1;
-constexpr int P_SCRATCH = 2 * 8 * NB;   // S [8][64] and PT [8][64]
+constexpr int PLD = NB + 8;             // row pitch of S and PT (the fragment loads of rows k and k+1
+                                        // fall in opposite halves of the banks)
+constexpr int P_SCRATCH = 2 * 8 * PLD;  // S [8][PLD] and PT [8][PLD]
 
-__device__ __forceinline__ constexpr int pk(int r, int c) { return r * (r + 1) / 2 + c; }   // packed lower 8x8
+__device__ __forceinline__ constexpr int pk(int r, int c) { return r * (r + 1) / 2 + c; }   // packed lower
+
+// In-register Cholesky of a 4x4 block (packed lower, in place) with the reciprocals of its diagonal;
+// the first non-positive pivot's column (col0 + c) goes to `bad`, and the factor turns NaN from there.
+__device__ __forceinline__ void chol4(double (&a)[10], double (&inv)[4], int& bad, int col0, double qnan) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const double p = a[pk(c, c)];
+        const bool ok = (p > 0.0) && isfinite(p);
+        if (!ok && bad < 0) bad = col0 + c;
+        inv[c] = ok ? rsqrt(p) : qnan;
+        a[pk(c, c)] = p * inv[c];
+#pragma unroll
+        for (int r = c + 1; r < 4; ++r) a[pk(r, c)] *= inv[c];
+#pragma unroll
+        for (int r = c + 1; r < 4; ++r)
+#pragma unroll
+            for (int k = c + 1; k <= r; ++k) a[pk(r, k)] = fma(-a[pk(r, c)], a[pk(k, c)], a[pk(r, k)]);
+    }
+}
 
 __device__ void tile_potrf_inv(Tile* T, double* Xs, double* scr, double* Lg, double* Dg, double* Yg, int* err, int b,
                                int col_base, int d) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const double qnan = __longlong_as_double(0x7ff8000000000000ll);
-    double* S = scr;             // S[r][j]  = sum_{m < o} L[o+r][m] X[m][j],   j < o
-    double* PT = scr + 8 * NB;   // PT[c][i] = L[i][o+c],                      i >= o + 8
+    double* S = scr;              // S[r][j]  = sum_{m < o} L[o+r][m] X[m][j],   j < o
+    double* PT = scr + 8 * PLD;   // PT[c][i] = L[i][o+c],                      i >= o + 8
+    const int g = lane >> 2, tq = lane & 3;   // m8n8k4 fragment coordinates
     int bad = -1;   // first non-positive pivot (warp 0)
     for (int kb = 0; kb < 8; ++kb) {
         const int o = 8 * kb;
         if (warp == 0) {
-            double a[36];
+            // two 4-column stages, so that at most ~30 of the block's values are live at once:
+            // L11 = chol(A11); L21 = A21 L11^-T; A22 -= L21 L21^T; L22 = chol(A22)
+            double* dinv = PT;   // 1 / L_cc of this block (PT is free until step 2)
+            double a11[10], inv[4];
 #pragma unroll
-            for (int r = 0; r < 8; ++r)
+            for (int r = 0; r < 4; ++r)
 #pragma unroll
-                for (int c = 0; c <= r; ++c) a[pk(r, c)] = T[o + r][o + c];
-            double inv[8];
+                for (int c = 0; c <= r; ++c) a11[pk(r, c)] = T[o + r][o + c];
+            chol4(a11, inv, bad, o, qnan);
+            double l21[4][4];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const double p = a[pk(c, c)];
-                const bool ok = (p > 0.0) && isfinite(p);
-                if (!ok && bad < 0) bad = o + c;
-                inv[c] = ok ? rsqrt(p) : qnan;
-                a[pk(c, c)] = p * inv[c];
+            for (int r = 0; r < 4; ++r)
 #pragma unroll
-                for (int r = c + 1; r < 8; ++r) a[pk(r, c)] *= inv[c];
+                for (int c = 0; c < 4; ++c) {
+                    double v = T[o + 4 + r][o + c];
 #pragma unroll
-                for (int r = c + 1; r < 8; ++r)
-#pragma unroll
-                    for (int k = c + 1; k <= r; ++k) a[pk(r, k)] = fma(-a[pk(r, c)], a[pk(k, c)], a[pk(r, k)]);
-            }
+                    for (int k = 0; k < c; ++k) v = fma(-l21[r][k], a11[pk(c, k)], v);
+                    l21[r][c] = v * inv[c];
+                }
             if (lane == 0) {
 #pragma unroll
-                for (int r = 0; r < 8; ++r)
+                for (int r = 0; r < 4; ++r) {
+                    dinv[r] = inv[r];
 #pragma unroll
-                    for (int c = 0; c <= r; ++c) T[o + r][o + c] = a[pk(r, c)];
+                    for (int c = 0; c <= r; ++c) T[o + r][o + c] = a11[pk(r, c)];
+                }
             }
-            if (lane < 8) {   // column j of X_bb: L_bb x = e_j, 1 / L_rr = inv[r]
+            double a22[10];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int c = 0; c <= r; ++c) {
+                    double v = T[o + 4 + r][o + 4 + c];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) v = fma(-l21[r][k], l21[c][k], v);
+                    a22[pk(r, c)] = v;
+                }
+            if (lane == 0) {
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) T[o + 4 + r][o + c] = l21[r][c];
+            }
+            chol4(a22, inv, bad, o + 4, qnan);
+            if (lane == 0) {
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    dinv[4 + r] = inv[r];
+#pragma unroll
+                    for (int c = 0; c <= r; ++c) T[o + 4 + r][o + 4 + c] = a22[pk(r, c)];
+                }
+            }
+            __syncwarp();
+            if (lane < 8) {   // column j of X_bb: L_bb x = e_j, L_bb read back from T (broadcasts)
                 const int j = lane;
                 double x[8];
 #pragma unroll
                 for (int r = 0; r < 8; ++r) {
                     double sum = (r == j) ? 1.0 : 0.0;
 #pragma unroll
-                    for (int m = 0; m < r; ++m) sum = (m >= j) ? fma(-a[pk(r, m)], x[m], sum) : sum;
-                    x[r] = (r >= j) ? sum * inv[r] : 0.0;
+                    for (int m = 0; m < r; ++m) sum = (m >= j) ? fma(-T[o + r][o + m], x[m], sum) : sum;
+                    x[r] = (r >= j) ? sum * dinv[r] : 0.0;
                     Xs[(o + r) * XLD + o + j] = x[r];
                 }
             }
-        } else {
-            for (int e = tid - 32; e < 8 * o; e += 224) {
-                const int r = e / o, j = e - r * o;
-                double s0 = 0.0, s1 = 0.0;
-                int m = j;
-                for (; m + 1 < o; m += 2) {
-                    s0 = fma(T[o + r][m], Xs[m * XLD + j], s0);
-                    s1 = fma(T[o + r][m + 1], Xs[(m + 1) * XLD + j], s1);
-                }
-                if (m < o) s0 = fma(T[o + r][m], Xs[m * XLD + j], s0);
-                S[r * NB + j] = s0 + s1;
+        } else if (warp - 1 < kb) {
+            // block jb = warp - 1 of S: the sum over the blocks mb = jb .. kb-1 of L_{b,mb} X_{mb,jb}
+            // (the diagonal block X_{jb,jb} holds zeros above its diagonal)
+            const int jb = warp - 1;
+            double c0 = 0.0, c1 = 0.0;
+            for (int mb = jb; mb < kb; ++mb) {
+#pragma unroll
+                for (int s4 = 0; s4 < 8; s4 += 4)
+                    dmma(c0, c1, T[o + g][8 * mb + s4 + tq], Xs[(8 * mb + s4 + tq) * XLD + 8 * jb + g]);
             }
+            S[g * PLD + 8 * jb + 2 * tq] = c0;
+            S[g * PLD + 8 * jb + 2 * tq + 1] = c1;
         }
         cbar();
-        const int npanel = (56 - o) * 8;   // panel entries; with the 8 o entries of X_b,<o always 448
-        for (int e = tid; e < 448; e += 256) {
-            if (e < npanel) {
+        // warps 0 .. 6-kb: panel block row bi = kb+1+warp, L_{bi,b} = A_{bi,b} X_bb^T, kept transposed;
+        // the next kb warps: block jb of the block row of the inverse, X_{b,jb} = -X_bb S_{b,jb}
+        if (warp < 7 - kb) {
+            const int bi = kb + 1 + warp;
+            double c0 = 0.0, c1 = 0.0;
+#pragma unroll
+            for (int s4 = 0; s4 < 8; s4 += 4)
+                dmma(c0, c1, T[8 * bi + g][o + s4 + tq], Xs[(o + g) * XLD + o + s4 + tq]);
+            PT[(2 * tq) * PLD + 8 * bi + g] = c0;
+            PT[(2 * tq + 1) * PLD + 8 * bi + g] = c1;
+        } else if (warp < 7) {
+            const int jb = warp - (7 - kb);
+            double c0 = 0.0, c1 = 0.0;
+#pragma unroll
+            for (int s4 = 0; s4 < 8; s4 += 4)
+                dmma(c0, c1, Xs[(o + g) * XLD + o + s4 + tq], S[(s4 + tq) * PLD + 8 * jb + g]);
+            Xs[(o + g) * XLD + 8 * jb + 2 * tq] = -c0;
+            Xs[(o + g) * XLD + 8 * jb + 2 * tq + 1] = -c1;
+        }
+        cbar();
+        {   // trailing blocks (bi, bj), kb < bj <= bi: A_{bi,bj} -= L_{bi,b} L_{bj,b}^T (whole 8x8 blocks;
+            // above the diagonal of a diagonal block nothing is read), as -(-A + L L^T)
+            const int nb = 7 - kb;
+            for (int e = warp; e < nb * (nb + 1) / 2; e += 8) {
+                int bi = 0, bj = e;
+                while (bj > bi) { bj -= bi + 1; ++bi; }
+                bi += kb + 1;
+                bj += kb + 1;
+                double2* cp = reinterpret_cast<double2*>(&T[8 * bi + g][8 * bj + 2 * tq]);
+                const double2 cv = *cp;
+                double c0 = -cv.x, c1 = -cv.y;
+#pragma unroll
+                for (int s4 = 0; s4 < 8; s4 += 4)
+                    dmma(c0, c1, PT[(s4 + tq) * PLD + 8 * bi + g], PT[(s4 + tq) * PLD + 8 * bj + g]);
+                *cp = make_double2(-c0, -c1);
+            }
+            for (int e = tid; e < (56 - o) * 8; e += 256) {   // the panel into T
                 const int i = o + 8 + (e >> 3), c = e & 7;
-                double acc = 0.0;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) acc = (k <= c) ? fma(T[i][o + k], Xs[(o + c) * XLD + o + k], acc) : acc;
-                PT[c * NB + i] = acc;
-            } else {
-                const int f = e - npanel, r = f / o, j = f - r * o;
-                double acc = 0.0;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) acc = (q <= r) ? fma(Xs[(o + r) * XLD + o + q], S[q * NB + j], acc) : acc;
-                Xs[(o + r) * XLD + j] = -acc;
+                T[i][o + c] = PT[c * PLD + i];
             }
-        }
-        cbar();
-        for (int i = o + 8 + warp; i < NB; i += 8) {
-            double li[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) li[c] = PT[c * NB + i];
-            for (int j = o + 8 + lane; j <= i; j += 32) {
-                double acc = T[i][j];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) acc = fma(-li[c], PT[c * NB + j], acc);
-                T[i][j] = acc;
-            }
-            if (lane < 8) T[i][o + lane] = PT[lane * NB + i];
         }
         cbar();
     }
@@ -514,7 +577,10 @@ __global__ void __launch_bounds__(DAG_THREADS, 2) fac_dag(Dag g) {
             int wtl = 0;
             if (t < g.total && !*reinterpret_cast<volatile int*>(g.abort_flag)) {
                 decode_task(g, lvl, t, d, dp);
-                if (lane < 3) { wpl = dp.wp[lane]; wtl = dp.wt[lane]; }
+                if (lane < 3) {   // (selects, not an indexed local array)
+                    wpl = lane == 0 ? dp.wp[0] : lane == 1 ? dp.wp[1] : dp.wp[2];
+                    wtl = lane == 0 ? dp.wt[0] : lane == 1 ? dp.wt[1] : dp.wt[2];
+                }
                 const bool ready = !wpl || ld_acquire(wpl) >= wtl;
                 d.status = __all_sync(0xffffffffu, ready) ? READY : WAIT;
             }
