@@ -68,6 +68,10 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
     const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
 }
+// Bring a contiguous, 16-byte aligned range (a multiple of 16 bytes) into L2 (no completion to wait for).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
@@ -284,16 +288,19 @@ __device__ void tile_potrf_inv(Tile* T, double* Xs, double* scr, double* Lg, dou
                 }
             }
             __syncwarp();
-            if (lane < 8) {   // column j of X_bb: L_bb x = e_j, L_bb read back from T (broadcasts)
+            if (lane < 8) {   // column j of X_bb: L_bb x = e_j, L_bb read back from T (broadcasts);
+                              // right-looking, so that the dependent chain is one multiply and one
+                              // fma per row
                 const int j = lane;
-                double x[8];
+                double acc[8];
 #pragma unroll
-                for (int r = 0; r < 8; ++r) {
-                    double sum = (r == j) ? 1.0 : 0.0;
+                for (int r = 0; r < 8; ++r) acc[r] = (r == j) ? 1.0 : 0.0;
 #pragma unroll
-                    for (int m = 0; m < r; ++m) sum = (m >= j) ? fma(-T[o + r][o + m], x[m], sum) : sum;
-                    x[r] = (r >= j) ? sum * dinv[r] : 0.0;
-                    Xs[(o + r) * XLD + o + j] = x[r];
+                for (int m = 0; m < 8; ++m) {
+                    const double x = (m >= j) ? acc[m] * dinv[m] : 0.0;
+                    Xs[(o + m) * XLD + o + j] = x;
+#pragma unroll
+                    for (int r = m + 1; r < 8; ++r) acc[r] = fma(-T[o + r][o + m], x, acc[r]);
                 }
             }
         } else if (warp - 1 < kb) {
@@ -577,6 +584,19 @@ __global__ void __launch_bounds__(DAG_THREADS, 2) fac_dag(Dag g) {
             int wtl = 0;
             if (t < g.total && !*reinterpret_cast<volatile int*>(g.abort_flag)) {
                 decode_task(g, lvl, t, d, dp);
+                if (lane < 3) {   // the task's tiles into L2 while the compute warps run the current one
+                    const Grp& G = g.grp[d.k];
+                    const double* Dm = G.D + ((size_t)d.b * G.nt + d.m) * TILE_ELEMS;
+                    const double* pt = nullptr;
+                    if (d.q == 0) pt = lane == 0 ? tile(G.A, G, d.b, d.m, d.m) : nullptr;
+                    else if (d.q == 1) pt = lane == 0 ? tile(G.A, G, d.b, d.i, d.m) : lane == 1 ? Dm : nullptr;
+                    else if (d.q == 2 || d.q == 5)
+                        pt = tile(G.A, G, d.b, lane == 2 ? d.i : lane == 1 ? d.j : d.i, lane == 2 ? d.j : d.m);
+                    else if (d.q == 3) pt = lane == 0 ? tile(G.Y, G, d.b, d.j, d.m) : lane == 1 ? Dm : nullptr;
+                    else pt = lane == 0 ? tile(G.Y, G, d.b, d.j, d.m) : lane == 1 ? tile(G.A, G, d.b, d.i, d.m)
+                                                                     : tile(G.Y, G, d.b, d.j, d.i);
+                    if (pt) prefetch_l2(pt, TILE_ELEMS * sizeof(double));
+                }
                 if (lane < 3) {   // (selects, not an indexed local array)
                     wpl = lane == 0 ? dp.wp[0] : lane == 1 ? dp.wp[1] : dp.wp[2];
                     wtl = lane == 0 ? dp.wt[0] : lane == 1 ? dp.wt[1] : dp.wt[2];
