@@ -26,14 +26,17 @@
 // stage_counts; within a stage group after group, problems interleaved inside each class) and CTAs
 // take numbers from a global counter. Every tile has a monotone state counter: A_ij counts the
 // updates applied (j + 1 once L_ij is final); Y_ji counts the Q terms applied (i - j + 1 once final).
-// A task waits (thread 0, acquire loads, bounded by a time limit) until its inputs have reached the
-// states it needs, runs, and publishes its output tile's new state with a release store. Any task
-// waited on has a smaller number and so is held by a CTA that is already running: the schedule
-// cannot deadlock however many CTAs are resident. Tile data moves through L2 only (cp.async.cg and
-// ld.global.cg), never through a stale L1 line.
+// Each CTA has 8 compute warps and a scheduler warp: the scheduler takes the next number, decodes
+// it, prefetches its tiles into L2 and checks (acquire loads, bounded by a time limit) that its
+// inputs have reached the states it needs while the compute warps run the current task; after the
+// barrier that ends a task it publishes the output tile's new state with a release store. Any task
+// waited on has a smaller number and is running or finished (a finished task is released before the
+// scheduler waits on anything): the schedule cannot deadlock however many CTAs are resident. Tile
+// data moves through L2 only (cp.async.cg and ld.global.cg), never through a stale L1 line.
 //
 // Products run on the FP64 tensor-core path (mma.sync m8n8k4 f64): 8 warps, each a 32 x 16 block
-// of the 64 x 64 output, operands in padded shared memory.
+// of the 64 x 64 output, operands in padded shared memory; the diagonal task's inner products are
+// 8 x 8 blocks on the same path.
 // A non-positive pivot is recorded (problem, original column) and the problem's factor is NaN.
 #include "clha_internal.h"
 
