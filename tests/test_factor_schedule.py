@@ -1,0 +1,132 @@
+"""The factor graph's task numbering, on the CPU.
+
+The factor kernel (csrc/factor.cu) runs the blocked Cholesky and the blocked inverse of every problem as
+64x64 tile tasks that CTAs take from one global counter, in number order, and each task waits until
+its inputs' tiles have reached the states it needs. That schedule is deadlock-free only if the
+numbering is topological: every task a task waits on has a smaller number. This test restates the
+numbering (the stage layout and class counts of stage_counts and the class decode of decode_task)
+and checks:
+  * run in number order, every task finds its inputs in the states it waits for, each tile update
+    is applied exactly once and in order, and every tile ends final (L_ij: state j + 1, Y_ji:
+    i - j + 1);
+  * the count per problem equals the launcher's closed form;
+  * a model of the in-order ticket protocol (W CTAs, each holding a running task and the next
+    number it has taken, a finished task released at once) always drains, for several W.
+"""
+import random
+
+import pytest
+
+
+def stage_counts(nt, s):
+    """Tasks per problem in stage s by class: next panel's updates G(i,m+1,m), P(m+1), F(j,m),
+    Q(j,i,m), the remaining G(i,j,m), S(i,m+1) (stage 0: P(0), S(i,0))."""
+    if s == 0:
+        return [0, 1, 0, 0, 0, nt - 1]
+    m = s - 1
+    R = nt - 1 - m
+    return [R, 1 if R >= 1 else 0, m, (m + 1) * R, (R - 1) * R // 2 if R >= 1 else 0, R - 1 if R >= 1 else 0]
+
+
+def decode(nt, s, c, local):
+    m = s - 1
+    if c == 0:
+        return ("G", m, m + 1 + local, m + 1)
+    if c == 1:
+        return ("P", s, 0, 0)
+    if c == 2:
+        return ("F", m, 0, local)
+    if c == 3:
+        ii = local // (m + 1)
+        return ("Q", m, m + 1 + ii, local - ii * (m + 1))
+    if c == 4:
+        rem, j = local, m + 2
+        while rem >= nt - j:
+            rem -= nt - j
+            j += 1
+        return ("G", m, j + rem, j)
+    return ("S", s, s + 1 + local, s)
+
+
+def tasks(nt):
+    out = []
+    for s in range(nt + 1):
+        for c, cnt in enumerate(stage_counts(nt, s)):
+            out += [decode(nt, s, c, local) for local in range(cnt)]
+    return out
+
+
+def deps(task):
+    """(tile kind, i, j, state needed) of the inputs, and (tile kind, i, j, new state) of the outputs."""
+    kind, m, i, j = task
+    if kind == "P":
+        return [("A", m, m, m)], [("A", m, m, m + 1), ("Y", m, m, 1)]
+    if kind == "S":
+        return [("A", i, m, m), ("A", m, m, m + 1)], [("A", i, m, m + 1)]
+    if kind == "G":
+        return [("A", i, m, m + 1), ("A", j, m, m + 1), ("A", i, j, m)], [("A", i, j, m + 1)]
+    if kind == "F":
+        return [("Y", j, m, m - j), ("A", m, m, m + 1)], [("Y", j, m, m - j + 1)]
+    return [("Y", j, m, m - j + 1), ("A", i, m, m + 1), ("Y", j, i, m - j)], [("Y", j, i, m - j + 1)]
+
+
+@pytest.mark.parametrize("nt", list(range(1, 34)))
+def test_numbering_is_topological_and_complete(nt):
+    state = {}
+    for t in tasks(nt):
+        ins, outs = deps(t)
+        for key in ins:
+            assert state.get(key[:3], 0) >= key[3], (t, key, state.get(key[:3], 0))
+        for key in outs:
+            assert state.get(key[:3], 0) == key[3] - 1, (t, key)   # each update once, in order
+            state[key[:3]] = key[3]
+    for i in range(nt):
+        for j in range(i + 1):
+            assert state[("A", i, j)] == j + 1
+            assert state[("Y", j, i)] == i - j + 1
+
+
+@pytest.mark.parametrize("nt", [1, 2, 5, 16, 128])
+def test_count_matches_launcher_closed_form(nt):
+    closed = sum(1 + 2 * R + m + (m + 1) * R + ((R - 1) * R // 2 if R >= 1 else 0)
+                 for m in range(nt) for R in [nt - 1 - m])
+    assert len(tasks(nt)) == closed
+
+
+@pytest.mark.parametrize("n_cta", [1, 2, 7, 64])
+def test_in_order_ticket_protocol_drains(n_cta):
+    """Several problems of two sizes interleaved (stage by stage, as the kernel numbers them); CTAs
+    take numbers in order, each holds at most its running task and its next number, and a task
+    starts only when its inputs are final. Random completion order; it must never stall."""
+    groups = [(6, 3), (3, 2)]   # (nt, batch)
+    numbered = []
+    for s in range(max(nt for nt, _ in groups) + 1):
+        for gi, (nt, batch) in enumerate(groups):
+            if s > nt:
+                continue
+            for c, cnt in enumerate(stage_counts(nt, s)):
+                for local in range(cnt):
+                    for b in range(batch):
+                        numbered.append((gi, b, decode(nt, s, c, local)))
+    rng = random.Random(n_cta)
+    state, nxt = {}, 0
+    held = [[] for _ in range(n_cta)]   # per CTA: [running or waiting task, next number]
+    done = 0
+    while done < len(numbered):
+        for h in held:                   # take numbers in order
+            while len(h) < 2 and nxt < len(numbered):
+                h.append(nxt)
+                nxt += 1
+        ready = []
+        for ci, h in enumerate(held):
+            if h:
+                gi, b, t = numbered[h[0]]
+                ins, _ = deps(t)
+                if all(state.get((gi, b) + k[:3], 0) >= k[3] for k in ins):
+                    ready.append(ci)
+        assert ready, "stalled"
+        ci = rng.choice(ready)
+        gi, b, t = numbered[held[ci].pop(0)]
+        for k in deps(t)[1]:
+            state[(gi, b) + k[:3]] = k[3]
+        done += 1
