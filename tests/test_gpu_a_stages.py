@@ -324,8 +324,10 @@ def test_aggregate_matches_oracle(ctx, mode):
 
 
 # ------------------------------------------------------------------------------------ factor
-@pytest.mark.parametrize("d,batch", [(128, 1), (512, 3), (1408, 1)])
+@pytest.mark.parametrize("d,batch", [(128, 1), (128, 5), (512, 3), (896, 2), (1408, 1)])
 def test_factor_matches_oracle(ctx, d, batch):
+    """Two tiles per side (one with an odd batch), 8, 14 and 22 tiles; every problem against the
+    oracle's float64 inverse Cholesky."""
     g = _gen(d)
     Hs = []
     for b in range(batch):
