@@ -25,6 +25,8 @@ struct clha_ctx {
     // and the device int the per-call choice is written to.
     int act_policy = 0;
     int* d_act_sel = nullptr;
+    // Time limit of each dependency wait inside the factor graph (clha_set_factor_wait_limit).
+    uint64_t factor_wait_ns = 4000000000ull;
     // Small pinned host buffer for scalar read-backs.
     void* host_pinned = nullptr;
     size_t host_pinned_bytes = 0;
@@ -82,6 +84,7 @@ cudaError_t launch_gather(cudaStream_t s, const void* X, int esize, int64_t n, i
                           const int32_t* ids, int k, int E, void* X_packed, int64_t packed_rows,
                           int64_t* seg, int32_t* perm, void* ws, size_t ws_bytes, int* err);
 size_t gather_workspace_bytes(int64_t n, int k, int E, int64_t packed_rows);
+constexpr int kGatherBlockTokens = 256;   // tokens per block of the histogram and scatter passes
 size_t expert_act_workspace_bytes(int d_model);
 cudaError_t launch_expert_act(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t rows, int d_model,
                               const int32_t* perm, const int64_t* seg, int E, const __nv_bfloat16* Wg,
@@ -113,7 +116,8 @@ struct FactorGroup {
     int batch, d;
 };
 size_t factor_workspace_bytes(const FactorGroup* groups, int n);
-cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups, int n, void* ws, int* err);
+cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups, int n, void* ws, int* err,
+                          uint64_t wait_ns);
 cudaError_t launch_pack_codes(cudaStream_t s, const uint8_t* codes, int64_t rows, int d_in, int bits,
                               uint32_t* packed);
 cudaError_t launch_dequantize(cudaStream_t s, const uint32_t* packed, const float* scales, const uint8_t* zeros,

@@ -14,7 +14,7 @@
 
 namespace {
 
-constexpr int kTB = 256;  // tokens per block in passes 1 and 3
+constexpr int kTB = kGatherBlockTokens;  // tokens per block in passes 1 and 3
 
 __global__ void gather_hist(const int32_t* __restrict__ ids, int64_t n, int k, int E, int* __restrict__ H,
                             int* err) {

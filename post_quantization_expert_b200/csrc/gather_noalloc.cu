@@ -9,12 +9,15 @@
 //
 // The array is a file-scope __device__ object, so every GPU that loads libclha.so holds it until
 // the process exits. In host code its name only stands for the symbol; its device address comes
-// from cudaGetSymbolAddress, taken once per device (with that device current) on the first call
-// there and cached. All calls share the array and it keeps the last call's contents: the gather
-// rewrites every histogram entry it reads and resets the permutation to -1 before scattering, and
-// calls that overlap on the GPU (different streams, different contexts) race on it.
-#include <mutex>
-
+// from cudaGetSymbolAddress, looked up on every call with the call's device current (a cheap
+// lookup, and one that stays right if the context is reset and the module loaded again at another
+// address). All calls share the array and it keeps the last call's contents: the gather rewrites
+// every histogram entry it reads and resets a permutation kept in the array to -1 before
+// scattering, and calls that overlap on the GPU (different streams, different contexts) race on it.
+//
+// Scratch per call: the per-block expert histograms, ceil(n/256)*E int32 entries (256 tokens per block), and, only when
+// the caller passes no perm array, the token permutation, packed_rows int32 entries (each part
+// rounded up to 256 bytes).
 #include "clha_internal.h"
 
 namespace {
@@ -22,21 +25,13 @@ namespace {
 constexpr size_t kScratchBytes = size_t(4) << 20;  // 4 MiB
 static __device__ __align__(256) unsigned char g_gather_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 128;
-void* g_scratch_addr[kMaxDevices] = {};
-std::mutex g_scratch_mutex;
-
-// Device address of the scratch array on `device` (which must be current).
-cudaError_t scratch_address(int device, void** out) {
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_addr[device]) {
-        void* p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_gather_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[device] = p;
-    }
-    *out = g_scratch_addr[device];
-    return cudaSuccess;
+// Bytes of the fixed array this gather uses: what launch_gather carves out of it.
+size_t noalloc_scratch_bytes(int64_t n, int E, int64_t packed_rows, bool perm_given) {
+    int64_t nblk = (n + kGatherBlockTokens - 1) / kGatherBlockTokens;
+    if (nblk < 1) nblk = 1;
+    size_t b = clha_round_up((size_t)nblk * E * sizeof(int));
+    if (!perm_given) b += clha_round_up((size_t)packed_rows * sizeof(int32_t));
+    return b;
 }
 
 }  // namespace
@@ -57,18 +52,16 @@ extern "C" clha_status clha_gather_noalloc(clha_ctx* ctx, const void* X, clha_dt
                          (long long)packed_rows, (long long)clha_packed_rows(n, k, E));
     if (!seg || (!X_packed && !perm) || (n > 0 && !ids) || (X_packed && n > 0 && !X))
         return clha_fail(ctx, CLHA_ERR_INVALID_ARG, "clha_gather_noalloc: null pointer");
-    const size_t need = gather_workspace_bytes(n, k, E, packed_rows);
+    const size_t need = noalloc_scratch_bytes(n, E, packed_rows, perm != nullptr);
     if (need > kScratchBytes)
         return clha_fail(ctx, CLHA_ERR_INVALID_ARG,
                          "clha_gather_noalloc: this gather needs %zu bytes of scratch but the fixed array holds %zu "
-                         "(4 MiB); use clha_gather, or fewer tokens / experts per call",
+                         "(4 MiB); use clha_gather, pass a perm array, or fewer tokens / experts per call",
                          need, kScratchBytes);
-    if (ctx->device < 0 || ctx->device >= kMaxDevices)
-        return clha_fail(ctx, CLHA_ERR_INVALID_ARG, "clha_gather_noalloc: device %d out of range", ctx->device);
     cudaError_t e = cudaSetDevice(ctx->device);
     if (e != cudaSuccess) return clha_cuda_check(ctx, e, "clha_gather_noalloc: cudaSetDevice");
     void* scratch = nullptr;
-    e = scratch_address(ctx->device, &scratch);
+    e = cudaGetSymbolAddress(&scratch, g_gather_scratch);
     if (e != cudaSuccess) return clha_cuda_check(ctx, e, "clha_gather_noalloc: cudaGetSymbolAddress");
     const int64_t l0 = clha_total_launches();
     e = launch_gather(ctx->stream, X, es, n, d, ids, k, E, X_packed, packed_rows, seg, perm, scratch, kScratchBytes,
