@@ -51,7 +51,8 @@ typedef enum {
     CLHA_ERR_EMPTY = 5,             /* aggregation over slots with no tokens in any layer */
     CLHA_ERR_OOM = 6,               /* workspace allocation failed */
     CLHA_ERR_CUDA = 7,              /* a CUDA runtime call failed (message in last_error) */
-    CLHA_ERR_TIMEOUT = 8            /* reserved: a bounded device-side wait ran out */
+    CLHA_ERR_TIMEOUT = 8            /* a bounded device-side wait ran out (factor graph, GPTQ, Gram,
+                                       activation); the kernel returned and the context stays usable */
 } clha_status;
 
 typedef enum { CLHA_BF16 = 0, CLHA_F32 = 1 } clha_dtype;
@@ -123,13 +124,16 @@ CLHA_API clha_status clha_gather(clha_ctx* ctx, const void* X, clha_dtype dtype,
  * callers that must not see the library allocate device memory: processes whose memory is handed
  * out by their own allocator (a framework's caching allocator, a fixed arena), where a cudaMalloc
  * can fail once the arena holds the memory and a cudaFree synchronises the whole device.
- * Its scratch (block histograms and the token permutation, clha_gather's workspace) is a fixed
- * 4 MiB array in the library's device image, which every GPU that loads the library holds until
- * the process exits. A gather whose scratch exceeds it (roughly n*k + 128*E above ~1M rows) is
- * rejected with CLHA_ERR_INVALID_ARG before anything is queued. The first call on a device looks up
- * the array's device address (cudaGetSymbolAddress) with that device current, and caches it; make
- * that first call before any stream capture. All calls share the array and it keeps the last
- * call's contents (each call rewrites what it reads); calls that overlap on the GPU race on it. */
+ * Its scratch (clha_gather's workspace) is a fixed 4 MiB array in the library's device image,
+ * which every GPU that loads the library holds until the process exits. A call needs
+ * ceil(n/256)*E*4 bytes there for the block histograms, plus packed_rows*4 bytes for the token
+ * permutation only when perm is NULL (each part rounded up to 256 bytes). So with perm given the
+ * limit is ceil(n/256)*E <= ~1M (e.g. n = 8M tokens at E = 32); with perm NULL, roughly
+ * n*k + 128*E <= ~1M packed rows. A larger gather is rejected with CLHA_ERR_INVALID_ARG before
+ * anything is queued. Every call looks up the array's device address (cudaGetSymbolAddress) with
+ * the context's device current; the first call on a device may load the module, so make it before
+ * any stream capture. All calls share the array and it keeps the last call's contents (each call
+ * rewrites what it reads); calls that overlap on the GPU race on it. */
 CLHA_API clha_status clha_gather_noalloc(clha_ctx* ctx, const void* X, clha_dtype dtype, int64_t n, int d,
                                          const int32_t* ids, int k, int E, void* X_packed, int64_t packed_rows,
                                          int64_t* seg, int32_t* perm);
@@ -241,17 +245,15 @@ typedef struct clha_factor_group {
 } clha_factor_group;
 CLHA_API clha_status clha_factor_groups(clha_ctx* ctx, int n_groups, const clha_factor_group* groups);
 
-/* E-PMQ's quantization target (the E-PMQ page, section 2: expert-driven output targets, anchoring to
- * the merged weights, and the solver's statistics H = sum_i H_i + lambda I, R = sum_i W_i H_i +
- * lambda W_m). The K = n_layers "layers" of `acc` are the K source experts: S_i = acc's Gram of
- * layer i in slot `slot` (H_i = S_i, upper triangle read). With U the clha_factor of the damped
- * aggregate of that slot in mode CLHA_ALPHA_SUM (H_comb = sum_i S_i, H_damped = H) and lambda its
- * damping (lambda_dev as written by clha_aggregate), computes in float64
- *   W_target = (lambda W_m + sum_i W_i S_i) U^T U  =  R H^-1
- * and writes it as float32 [d_out, d]; clha_quantize of W_target with U then runs E-PMQ's GPTQ step.
- * W_src: device [K, d_out, d] (the source experts' weights), W_merged: device [d_out, d], both of
- * `dtype`; U: device float32 [d, d]; lambda_dev: device double. d = acc's d; d_out a multiple of 64.
- * Device pointers are the caller's. */
+/* Time limit, in nanoseconds, of each dependency wait inside clha_factor's task graph (a CTA waiting
+ * for a tile that another CTA is still producing); 0 restores the default of 4 s. A wait that runs
+ * out sets the graph's abort flag: every CTA stops taking tasks and returns, the call's U is
+ * undefined, and the next synchronising call (clha_check) reports CLHA_ERR_TIMEOUT. The context stays
+ * usable, and the next clha_factor starts a fresh graph. Nothing in the method needs another limit;
+ * it exists so that a stalled graph ends with an error instead of holding the GPU, and so that this
+ * path can be exercised (a limit of a microsecond or so runs out on the first real dependency). */
+CLHA_API clha_status clha_set_factor_wait_limit(clha_ctx* ctx, uint64_t ns);
+
 /* ------------------------------------------------------------------------------ deployable codes */
 
 /* Packs GPTQ's codes (uint8 [rows, d_in], values < 2^bits) into uint32 [rows, d_in * bits / 32]:
@@ -272,6 +274,17 @@ CLHA_API clha_status clha_dequant_matmul(clha_ctx* ctx, const void* X, clha_dtyp
                                          const uint32_t* packed, const float* scales, const uint8_t* zeros, int d_out,
                                          int d_in, int bits, float* Y);
 
+/* E-PMQ's quantization target (the E-PMQ page, section 2: expert-driven output targets, anchoring to
+ * the merged weights, and the solver's statistics H = sum_i H_i + lambda I, R = sum_i W_i H_i +
+ * lambda W_m). The K = n_layers "layers" of `acc` are the K source experts: S_i = acc's Gram of
+ * layer i in slot `slot` (H_i = S_i, upper triangle read). With U the clha_factor of the damped
+ * aggregate of that slot in mode CLHA_ALPHA_SUM (H_comb = sum_i S_i, H_damped = H) and lambda its
+ * damping (lambda_dev as written by clha_aggregate), computes in float64
+ *   W_target = (lambda W_m + sum_i W_i S_i) U^T U  =  R H^-1
+ * and writes it as float32 [d_out, d]; clha_quantize of W_target with U then runs E-PMQ's GPTQ step.
+ * W_src: device [K, d_out, d] (the source experts' weights), W_merged: device [d_out, d], both of
+ * `dtype`; U: device float32 [d, d]; lambda_dev: device double. d = acc's d; d_out a multiple of 64.
+ * Device pointers are the caller's. */
 CLHA_API clha_status clha_epmq_target(clha_ctx* ctx, const clha_accum* acc, int slot, const void* W_src,
                                       const void* W_merged, clha_dtype dtype, int d_out, const float* U,
                                       const double* lambda_dev, float* W_target);

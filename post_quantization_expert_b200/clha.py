@@ -34,6 +34,7 @@ SYMBOLS = [
     "clha_aggregate", "clha_factor", "clha_factor_groups", "clha_epmq_target", "clha_quantize", "clha_loss",
     "clha_pack_codes", "clha_dequantize", "clha_dequant_matmul", "clha_routing_divergence",
     "clha_collect_gathered", "clha_expert_act_gathered", "clha_set_act_kernel", "clha_last_act_kernel",
+    "clha_set_factor_wait_limit",
 ]
 FACTOR_MAX_GROUPS = 4
 
@@ -100,6 +101,7 @@ def load(path: str = LIB_PATH):
         "clha_expert_act_gathered": (i32, [vp, vp, i64, i32, vp, i64, vp, i32, vp, vp, i32, vp]),
         "clha_set_act_kernel": (i32, [vp, i32]),
         "clha_last_act_kernel": (i32, [vp]),
+        "clha_set_factor_wait_limit": (i32, [vp, C.c_uint64]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -297,6 +299,11 @@ def clha_aggregate(ctx: Context, acc: Accum, slot0: int, n_slots: int, mode: int
 
 def clha_factor(ctx: Context, H_damped, batch: int, d: int, U):
     ctx._check(load().clha_factor(ctx.handle, _p(H_damped), batch, d, _p(U)))
+
+
+def clha_set_factor_wait_limit(ctx: Context, ns: int):
+    """Limit of each dependency wait in the factor graph, in ns (0: the default, 4 s)."""
+    ctx._check(load().clha_set_factor_wait_limit(ctx.handle, ns))
 
 
 def clha_factor_groups(ctx: Context, groups):

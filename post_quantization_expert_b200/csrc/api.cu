@@ -146,7 +146,6 @@ extern "C" clha_status clha_create(int device, void* cuda_stream, clha_ctx** out
         cudaMemset(ctx->d_act_sel, 0, sizeof(int)) != cudaSuccess) {
         cudaGetLastError();
         if (ctx->d_err) cudaFree(ctx->d_err);
-    if (ctx->d_act_sel) cudaFree(ctx->d_act_sel);
         if (ctx->d_act_sel) cudaFree(ctx->d_act_sel);
         delete ctx;
         return CLHA_ERR_CUDA;
@@ -161,6 +160,7 @@ extern "C" void clha_destroy(clha_ctx* ctx) {
     cudaStreamSynchronize(ctx->stream);
     if (ctx->ws) cudaFree(ctx->ws);
     if (ctx->d_err) cudaFree(ctx->d_err);
+    if (ctx->d_act_sel) cudaFree(ctx->d_act_sel);
     if (ctx->host_pinned) cudaFreeHost(ctx->host_pinned);
     delete ctx;
 }
@@ -482,7 +482,14 @@ extern "C" clha_status clha_factor_groups(clha_ctx* ctx, int n_groups, const clh
     void* ws = nullptr;
     clha_status st = clha_workspace(ctx, factor_workspace_bytes(fg, n_groups), &ws);
     if (st) return st;
-    CUDA_TRY(launch_factor(ctx->stream, ctx->num_sms, fg, n_groups, ws, ctx->d_err), "clha_factor");
+    CUDA_TRY(launch_factor(ctx->stream, ctx->num_sms, fg, n_groups, ws, ctx->d_err, ctx->factor_wait_ns),
+             "clha_factor");
+    return CLHA_OK;
+}
+
+extern "C" clha_status clha_set_factor_wait_limit(clha_ctx* ctx, uint64_t ns) {
+    CHECK_CTX(ctx);
+    ctx->factor_wait_ns = ns ? ns : 4000000000ull;
     return CLHA_OK;
 }
 

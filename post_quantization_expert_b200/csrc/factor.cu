@@ -28,7 +28,9 @@
 // updates applied (j + 1 once L_ij is final); Y_ji counts the Q terms applied (i - j + 1 once final).
 // Each CTA has 8 compute warps and a scheduler warp: the scheduler takes the next number, decodes
 // it, prefetches its tiles into L2 and checks (acquire loads, bounded by a time limit) that its
-// inputs have reached the states it needs while the compute warps run the current task; after the
+// inputs have reached the states it needs while the compute warps run the current task (each wait
+// bounded by the context's limit, 4 s by default; one that runs out aborts the whole graph and
+// records CLHA_ERR_TIMEOUT); after the
 // barrier that ends a task it publishes the output tile's new state with a release store. Any task
 // waited on has a smaller number and is running or finished (a finished task is released before the
 // scheduler waits on anything): the schedule cannot deadlock however many CTAs are resident. Tile
@@ -47,7 +49,6 @@ constexpr int LD = NB + 8;   // padded shared row (doubles): the 16-byte fragmen
                              // rows fall in opposite halves of the banks (conflict-free)
 constexpr int TILE_DOUBLES = NB * LD;
 constexpr int TILE_ELEMS = NB * NB;
-constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;
 
 typedef double Tile[LD];
 
@@ -396,6 +397,7 @@ struct Dag {
     int* abort_flag;
     int* err;
     unsigned long long total;
+    uint64_t wait_ns;   // time limit of one dependency wait
 };
 
 __device__ __forceinline__ double* tile(double* base, const Grp& g, int b, int i, int j) {
@@ -415,7 +417,7 @@ __device__ bool wait_ge(const int* p, int target, const Dag& g, int problem) {
         if (ns < 512) ns <<= 1;
         if (ld_acquire(p) >= target) return true;
         if (*reinterpret_cast<volatile int*>(g.abort_flag)) return false;
-        if (gtimer() - t0 > WAIT_LIMIT_NS) {
+        if (gtimer() - t0 > g.wait_ns) {
             atomicExch(g.abort_flag, 1);
             clha_record_error(g.err, CLHA_ERR_TIMEOUT, problem, 0, KID_FACTOR);
             return false;
@@ -692,13 +694,15 @@ size_t factor_workspace_bytes(const FactorGroup* groups, int n) {
     return total + clha_round_up(states);
 }
 
-cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups, int n, void* ws, int* err) {
+cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups, int n, void* ws, int* err,
+                          uint64_t wait_ns) {
     if (n < 1 || n > MAX_GROUPS) return cudaErrorInvalidValue;
     char* cur = (char*)ws;
     Dag g;
     g.ng = n;
     g.max_nt = 0;
     g.err = err;
+    g.wait_ns = wait_ns;
     size_t state_bytes = 2 * sizeof(unsigned long long);
     int pbase = 0;
     for (int k = 0; k < n; ++k) {

@@ -397,6 +397,39 @@ def test_factor_non_pd_reports_column(ctx):
     L.clha_check(ctx)   # the error is cleared
 
 
+def test_factor_wait_limit_runs_out_and_context_recovers(ctx):
+    """A bounded device wait that runs out (failure detection without a GPU fault): with a 1 us limit
+    on the factor graph's dependency waits, the CTAs that wait for a diagonal task (about 30 us of
+    work) give up, the graph aborts and returns, and the next synchronising call reports
+    CLHA_ERR_TIMEOUT. With the default limit restored, the same context factors the same inputs
+    correctly."""
+    d, batch = 1024, 4
+    g = _gen(7)
+    Hs = []
+    for b in range(batch):
+        A = torch.randn((d, d // 4), generator=g).double()
+        Hs.append((A @ A.T / (d // 4) + 0.05 * torch.eye(d, dtype=torch.float64)).float())
+    Hd = torch.stack(Hs).to(DEV)
+    U = torch.full_like(Hd, float("nan"))
+    try:
+        L.clha_set_factor_wait_limit(ctx, 1000)
+        L.clha_factor(ctx, Hd, batch, d, U)
+        with pytest.raises(L.ClhaError) as ei:
+            L.clha_check(ctx)
+        assert ei.value.status == L.ERR_TIMEOUT
+        assert "clha_factor" in str(ei.value)
+    finally:
+        L.clha_set_factor_wait_limit(ctx, 0)
+    L.clha_check(ctx)                      # the record was cleared
+    U.fill_(float("nan"))
+    L.clha_factor(ctx, Hd, batch, d, U)
+    L.clha_check(ctx)
+    for b in range(batch):
+        got = U[b].double().cpu().numpy()
+        assert np.all(np.tril(got, -1) == 0)
+        assert rel_fro(got, O.factor(Hs[b].double().numpy())) < 1e-6
+
+
 # ------------------------------------------------------------------------------------ GPTQ
 def _H(d, seed, rank=None, damp=0.01):
     g = _gen(seed)
