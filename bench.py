@@ -1,12 +1,19 @@
-"""Throughput of CLHA calibration on B200: expert weight columns quantized per second, end to end.
+"""Throughput of CLHA calibration on B200: weight columns quantized per second, end to end.
 
-One step = the whole hot path on one weight-sharing MoE layer pair (E=16 routed experts, top-2,
-d_model 1024, d_ff 512, 8192 tokens per layer, 3-bit): for both layers route -> gather -> Hessians of
-the expert inputs -> expert activation -> Hessians of the down-projection inputs; then for both
-weightings (routing-frequency and equal) aggregate -> factor -> GPTQ of gate, up and down -> loss.
-Inputs are synthetic (seeded), resident in HBM; L2 is flushed (512 MB write) before every timed step.
+Default workload (the largest one that fits one GPU): one weight W [8192, 28672] bf16 shared by 4
+layers, 65536 calibration tokens per layer (d_in 28672, rank-64 covariance plus diagonal, drift 0.3
+between consecutive layers), routing-frequency alpha, 4-bit, group 128. One step = the whole hot
+path: zero the accumulators, Gram of each layer's tokens (4 x 53.9 TFLOP), aggregate and damp,
+inverse-Cholesky factor (15.7 TFLOP in float64), GPTQ of W (28672 columns) with its in-kernel loss.
+Inputs are synthetic (seeded), resident in HBM (15 GB of X per step, far larger than L2; a 512 MB
+flush write before every timed step as well).
 
-  python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference] [--parallel replicas|tokens]
+  python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+
+The MoE layer pair (E=16 routed experts, top-2, d_model 1024, d_ff 512, 8192 tokens per layer,
+3-bit; route -> gather -> Hessians -> expert activation -> down-projection Hessians per layer, then
+for both weightings aggregate -> factor -> GPTQ of gate, up and down -> loss):
+  python bench.py --workload moe-e16 [--parallel replicas|tokens]
 
 Kernel-level workloads (one JSON line per shape; used for the profiles and the roofline tables):
   python bench.py --workload act --shape 18432x1024x512 ...   expert activation, dense bf16 X [n, d_model]
@@ -21,10 +28,11 @@ Routing-sharpness sweep (not a throughput line; one JSON line per sharpness):
       routing divergence: per-layer calibration (alpha = (1, 0)) against CLHA rt and eq, each scored on
       the calibration hook layer and on fresh held-out tokens of both layers
 
-With N > 1 (torchrun, one process per GPU) every rank calibrates its own independent layer pair:
-weak scaling, no data-path collective; the step time is the max over ranks. With --parallel tokens
-the ranks share one layer pair instead: each collects its share of the tokens, one NCCL all-reduce
-sums the Hessian accumulators, and each quantizes its own range of experts (strong scaling).
+With N > 1 (torchrun, one process per GPU) every rank calibrates its own independent weight (or
+layer pair): weak scaling, no data-path collective; the step time is the max over ranks. With
+--workload moe-e16 --parallel tokens the ranks share one layer pair instead: each collects its share
+of the tokens, one NCCL all-reduce sums the Hessian accumulators, and each quantizes its own range of
+experts (strong scaling).
 """
 from __future__ import annotations
 
@@ -43,6 +51,7 @@ sys.path.insert(0, ROOT)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 N_SMS = 148
 METRIC = "expert weight columns quantized/sec (CLHA-GPTQ end to end)"
+DENSE_CPU_CHANNELS = 768      # the oracle's bounded sample of the dense workload: this principal block
 
 
 def load_peaks():
@@ -177,9 +186,10 @@ def job_value(units_per_step_per_rank: float, ms_max: float, world: int) -> floa
     return world * units_per_step_per_rank / (ms_max / 1e3)
 
 
-def rank_seed(rank: int) -> int:
-    """Each rank calibrates its own independent layer pair: a distinct, reproducible input seed."""
-    return 1235 + 7919 * rank
+def rank_seed(rank: int, base: int = 1235) -> int:
+    """Each rank calibrates its own independent problem: a distinct, reproducible input seed (rank 0
+    keeps the workload's own seed)."""
+    return base + 7919 * rank
 
 
 KERNEL_SOURCES = {"act": ("ffn_act.cu", "ffn_act_tc.cu"), "gptq": ("gptq.cu",), "hessian": ("hessian.cu",),
@@ -491,6 +501,227 @@ def run_ours(args, world, rank, local):
     return 0
 
 
+# ------------------------------------------------------------------------------ dense stress workload
+def dense_oracle_sample(Xs, W, spec, channels: int = DENSE_CPU_CHANNELS):
+    """The float64 oracle on a bounded sample of the dense workload: the same calibration restricted to
+    the first `channels` input channels (each layer's Gram over all its tokens on that principal block,
+    routing-frequency aggregate and damping, factor, GPTQ of every row of W on those columns, loss).
+    Returns the columns quantized."""
+    import numpy as np
+    import oracle as O
+    X64 = [np.ascontiguousarray(x[:, :channels].double().cpu().numpy()) for x in Xs]
+    W64 = W[:, :channels].double().cpu().numpy()
+    O.calibrate_dense(W64, X64, spec.bits_routed, spec.group, "rt", None, spec.damp_frac)
+    return channels
+
+
+def dense_inputs(rank: int, device):
+    from synth import workload
+    wl = workload(5, device)
+    wl = workload(5, device, seed=rank_seed(rank, wl.spec.seed))
+    return wl
+
+
+def run_reference_dense(args, world, rank):
+    """The oracle arm: each step the float64 oracle on the bounded sample of the dense workload."""
+    if rank != 0:
+        return 0
+    import torch
+    dev = "cuda" if torch.cuda.is_available() else "cpu"   # inputs drawn where the GPU arm draws them
+    wl = dense_inputs(0, dev)
+    s = wl.spec
+    C = DENSE_CPU_CHANNELS
+    Xs = [wl.x(l, cache=False)[:, :C].cpu() for l in range(s.n_layers)]
+    W = wl.dense_weight().cpu()
+    for _ in range(args.warmup):
+        dense_oracle_sample(Xs, W, s)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        cols = dense_oracle_sample(Xs, W, s)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * statistics.mean(times)
+    value = cols / (ms / 1e3)
+    sample = (f"the calibration restricted to the first {C} of {s.d_model} input channels: Gram of all "
+              f"{s.n_layers} x {s.tokens[0]} tokens on that block, aggregate, factor, GPTQ of all {s.d_out} rows "
+              f"on those {C} columns, loss")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "columns/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": s.name, "columns_per_step": cols, "l2": "n/a (host)"},
+            "cpu_baseline": {"value": value, "unit": "columns/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "columns/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def run_dense(args, world, rank, local):
+    """One weight shared by 4 layers (the largest single-GPU workload): every rank calibrates its own."""
+    import torch
+    from post_quantization_expert_b200 import clha as L
+    from post_quantization_expert_b200.pipeline import DenseCalibration, DenseHostStep, PhaseTimer
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = dense_inputs(rank, dev)
+    s = wl.spec
+    nl, n, d, d_out = s.n_layers, s.tokens[0], s.d_model, s.d_out
+    ctx = L.Context(local)
+    timer = PhaseTimer(ctx.stream)
+    cal = DenseCalibration(ctx, d_out, d, nl, s.bits_routed, s.damp_frac, timer=timer, keep_hcomb=False)
+    W = wl.dense_weight()
+    Xd = [wl.x(l, cache=False) for l in range(nl)]
+    torch.cuda.synchronize()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    cols_per_step = d
+
+    def step():
+        cal.reset()
+        for l in range(nl):
+            cal.collect(l, Xd[l])
+        cal.quantize(W, "rt", read_loss=False)
+
+    timer.enabled = False
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    L.clha_check(ctx)
+    timer.enabled = True
+    timer.reset()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    launches0 = L.clha_kernel_launches(ctx)
+    ev = []
+    stream = ctx.stream
+    t_begin = time.time()
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    t_end = time.time()
+    launches = L.clha_kernel_launches(ctx) - launches0
+    L.clha_check(ctx)
+    barrier(world)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    timer.collect()
+    ms = max_over_ranks(statistics.mean(step_ms), world)
+    value = job_value(cols_per_step, ms, world)
+    loss_dev = float(cal.loss_dev[0].item())
+
+    # ---- end to end through the public API: pinned host X and W in, codes / scales / zeros / loss out
+    timer.enabled = False
+    hX = [x.cpu().pin_memory() for x in Xd]
+    hW = W.cpu().pin_memory()
+    del Xd
+    torch.cuda.empty_cache()
+    q = cal.q
+    hout = tuple(torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (q.codes, q.scales, q.zeros))
+    hloss = torch.empty(1, dtype=torch.float64).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in hX) + hW.numel() * hW.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in hout) + 8
+    hs = DenseHostStep(cal, [x.shape for x in hX], hX[0].dtype, hW.shape, hW.dtype)
+    for _ in range(2):
+        hs.run(hX, hW, hout, hloss)
+    hs.join()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks.mark(t_begin, t_end)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        flush.zero_()
+        hs.run(hX, hW, hout, hloss)
+    hs.join()
+    b.record(stream)
+    torch.cuda.synchronize()
+    L.clha_check(ctx)
+    clk = clocks.stop()
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / args.steps, world)
+    assert abs(float(hloss[0]) - loss_dev) <= 1e-9 * abs(loss_dev), (float(hloss[0]), loss_dev)   # same inputs
+
+    # ---- per-phase rates and the roofline of the dominant kernel
+    K = args.steps
+    phase_ms = {k: v / K for k, v in timer.totals.items()}
+    phase_calls = {k: v // K for k, v in timer.counts.items()}
+    peaks, src = load_peaks()
+    alu = alu_peaks(peaks)
+    sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    hess_flops = nl * n * d * (d + 1)
+    factor_flops = 2 * d ** 3 // 3
+    gptq_flops = d_out * d * d
+    agg_bytes = nl * (d * (d + 1) // 2) * 4 + d * d * 4     # every layer's upper triangle read, H_d written
+    kernels = {
+        "hessian": ("tensor", hess_flops / 1e12, sustained, "TFLOP/s", "syrk_bf16_tc (tcgen05 kind::f16)"),
+        "factor": ("alu", factor_flops / 1e12, alu["fp64_tflops"], "TFLOP/s",
+                   "fac_load + fac_dag + fac_store (fp64 tile-task graph, mma.sync m8n8k4 f64)"),
+        "gptq": ("alu", gptq_flops / 1e12, alu["fp32_tflops"], "TFLOP/s",
+                 "gptq_tc (per-column fp32 sweep; lazy updates on tcgen05 kind::tf32, 3xTF32)"),
+        "aggregate": ("hbm", agg_bytes / 1e9, peaks["hbm_gbs"], "GB/s", "agg_combine"),
+    }
+    dom = max((k for k in phase_ms if k in kernels), key=lambda k: phase_ms[k])
+    bound, work, peak, unit, kname = kernels[dom]
+    achieved = work / (phase_ms[dom] / 1e3)
+    step_bytes = measured_traffic(dom, "dense-stress")
+    traffic = step_bytes / phase_calls[dom] if step_bytes is not None and phase_calls.get(dom) else None
+    phases = {k: {"ms": round(v, 3)} for k, v in sorted(phase_ms.items(), key=lambda kv: -kv[1])}
+    for k, v in phases.items():
+        if k in kernels:
+            _, wk, pk, un, _ = kernels[k]
+            v["achieved"] = round(wk / (phase_ms[k] / 1e3), 3)
+            v["unit"] = un
+            v["frac"] = round(v["achieved"] / pk, 4)
+    hess_tflops = hess_flops / 1e12 / (phase_ms["hessian"] / 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        C = DENSE_CPU_CHANNELS
+        Xs = [wl.x(l, cache=False)[:, :C].cpu() for l in range(nl)]
+        t0 = time.perf_counter()
+        c = dense_oracle_sample(Xs, W.cpu(), s)
+        dt = time.perf_counter() - t0
+        cpu = {"value": c / dt, "unit": "columns/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"the calibration restricted to the first {C} of {d} input channels (Gram of all "
+                         f"{nl} x {n} tokens on that block, aggregate, factor, GPTQ of all {d_out} rows on "
+                         f"those columns, loss): {c} columns in {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "columns/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": s.name, "global_batch": world * nl * n, "tokens_per_layer": n,
+                       "layers": nl, "d_out": d_out, "d_in": d, "bits": s.bits_routed, "group": s.group,
+                       "weighting": "rt", "columns_per_step_per_gpu": cols_per_step,
+                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (15 GB of X read per step) and a 512 MB flush write "
+                             "before every timed step"},
+            "hessian_tflops": hess_tflops,
+            "hessian_frac_of_bf16_peak": hess_tflops / sustained,
+            "hessian_peak": "bf16 sustained (the step lasts about a second)",
+            "roofline": {"kernel": kname, "phase": dom, "bound": bound, "achieved": achieved, "peak": peak,
+                         "unit": unit, "frac": achieved / peak, "traffic": traffic,
+                         "calls_per_step": phase_calls.get(dom),
+                         "peak_source": src if bound in ("tensor", "hbm") else "derived (SM count x lanes x max clock)"},
+            "phases_ms_per_step": phases,
+            "e2e": {"value": job_value(cols_per_step, e2e_ms, world), "unit": "columns/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line))
+    ctx.close()
+    return 0
+
+
 def run_sweep(args):
     """Calibration- and test-side Hessian error of per-layer calibration (PLIC) and CLHA (rt, eq) as
     the per-layer expert preference sharpens (the CLHA page, section 4). Synthetic tokens and weights:
@@ -660,7 +891,7 @@ def run_kernel(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--parallel", choices=("replicas", "tokens"), default="replicas",
@@ -668,9 +899,11 @@ def main():
                          "one pair, its tokens sharded over the ranks with one all-reduce of the Hessian sums, "
                          "its experts quantized in parallel (strong scaling)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
-    ap.add_argument("--workload", choices=("moe", "act", "hessian", "gptq", "factor", "epmq", "dequant", "sweep"),
-                    default="moe",
-                    help="moe: the end-to-end calibration step (default); sweep: the routing-sharpness "
+    ap.add_argument("--workload", choices=("dense", "moe-e16", "act", "hessian", "gptq", "factor", "epmq", "dequant",
+                                           "sweep"),
+                    default="dense",
+                    help="dense: the end-to-end calibration step of the 8192x28672 weight shared by 4 layers "
+                         "(default); moe-e16: the E16 MoE layer pair; sweep: the routing-sharpness "
                          "experiment; others: one kernel family")
     ap.add_argument("--sharpness", type=float, nargs="+", default=[0.0, 0.1, 0.2, 0.3, 0.5, 0.75, 1.0],
                     help="sweep: strengths of the per-layer expert preference")
@@ -680,12 +913,18 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.workload == "sweep":
         return run_sweep(args)
-    if args.workload != "moe":
+    if args.workload not in ("dense", "moe-e16"):
         if not args.shape:
             ap.error("--shape is required for kernel workloads")
         return run_kernel(args)
+    if args.parallel == "tokens" and args.workload != "moe-e16":
+        ap.error("--parallel tokens applies to --workload moe-e16")
     world, rank, local = dist_setup()
     try:
+        if args.workload == "dense":
+            if args.impl == "reference":
+                return run_reference_dense(args, world, rank)
+            return run_dense(args, world, rank, local)
         if args.impl == "reference":
             return run_reference(args, world, rank)
         return run_ours(args, world, rank, local)

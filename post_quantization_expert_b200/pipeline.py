@@ -103,14 +103,16 @@ class DenseCalibration:
     """One weight W [d_out, d_in] shared by n_layers layers (no routing)."""
 
     def __init__(self, ctx: L.Context, d_out: int, d_in: int, n_layers: int, bits: int, damp_frac: float = 0.01,
-                 timer=NO_TIMER):
+                 timer=NO_TIMER, keep_hcomb: bool = True):
+        """keep_hcomb=False: the undamped aggregate is not written (GPTQ and its in-kernel loss need only
+        the damped one and lambda)."""
         self.ctx, self.d_out, self.d_in, self.n_layers, self.bits, self.damp = ctx, d_out, d_in, n_layers, bits, damp_frac
         self.timer = timer
-        dev = torch.device("cuda", ctx.device)
+        self.dev = dev = torch.device("cuda", ctx.device)
         self.acc = L.Accum(ctx, d_in, n_layers, 1)
-        self.H_comb = torch.empty((1, d_in, d_in), dtype=torch.float32, device=dev)
-        self.H_d = torch.empty_like(self.H_comb)
-        self.U = torch.empty_like(self.H_comb)
+        self.H_d = torch.empty((1, d_in, d_in), dtype=torch.float32, device=dev)
+        self.H_comb = torch.empty_like(self.H_d) if keep_hcomb else None
+        self.U = torch.empty_like(self.H_d)
         self.q = _quant_buffers(1, d_out, d_in, dev)
         self.lam = torch.empty(1, dtype=torch.float64, device=dev)
         self.loss_dev = torch.empty(1, dtype=torch.float64, device=dev)
@@ -122,7 +124,10 @@ class DenseCalibration:
         with self.timer.span("hessian"):
             L.clha_collect(self.ctx, self.acc, layer, X, X.shape[0], self.d_in, None, 1, 0)
 
-    def quantize(self, W: torch.Tensor, mode: str = "rt", alpha=None, with_loss: bool = True, want_host=False):
+    def quantize(self, W: torch.Tensor, mode: str = "rt", alpha=None, with_loss: bool = True, want_host=False,
+                 read_loss: bool = True):
+        """Aggregate, factor and GPTQ (with the in-kernel loss). read_loss=False leaves the loss in
+        self.loss_dev (nothing synchronises)."""
         t = self.timer
         with t.span("aggregate"):
             host = L.clha_aggregate(self.ctx, self.acc, 0, 1, MODES[mode], alpha, self.damp, self.H_comb, self.H_d,
@@ -133,7 +138,7 @@ class DenseCalibration:
             L.clha_quantize(self.ctx, self.U, 1, W, 1, self.d_out, self.d_in, self.bits, self.q.codes, self.q.scales,
                             self.q.zeros, self.q.W_hat, lam=self.lam if with_loss else None,
                             loss=self.loss_dev if with_loss else None)
-        if with_loss:
+        if with_loss and read_loss:
             self.q.loss = self.loss_dev.cpu().numpy()
         return host
 
@@ -515,6 +520,68 @@ class HostStep:
     def join(self):
         """Make the context's stream wait for every copy queued so far (the outputs and losses of the
         last step included), so that an event recorded on it after this covers them."""
+        if self.outputs_copied is not None:
+            self.cal.ctx.stream.wait_event(self.outputs_copied)
+
+
+class DenseHostStep:
+    """Dense calibration steps (one weight shared by several layers) from pinned host memory to pinned
+    host memory. Each layer's tokens, then the weight, go to the device on an input stream; the
+    compute stream (the context's) collects a layer as soon as its tokens have arrived, so the
+    copies of later layers overlap the Gram work of earlier ones. The device copies of the inputs
+    come in `n_sets` sets used in turn: with two, the next step's inputs cross PCIe while this step
+    aggregates, factors and quantizes. Codes, scales, zeros and the loss go back on an output stream.
+    run() only queues work: nothing synchronises."""
+
+    def __init__(self, cal: DenseCalibration, x_shapes, x_dtype, w_shape, w_dtype, n_sets: int = 2):
+        self.cal = cal
+        dev = cal.dev
+        self.inp = torch.cuda.Stream(device=dev)
+        self.out = torch.cuda.Stream(device=dev)
+        self.sets = [dict(X=[torch.empty(sh, dtype=x_dtype, device=dev) for sh in x_shapes],
+                          W=torch.empty(w_shape, dtype=w_dtype, device=dev), free=None) for _ in range(n_sets)]
+        self.step = 0
+        self.outputs_copied = None
+
+    def run(self, hX, hW, hout, hloss=None, mode: str = "rt"):
+        """hX: per-layer pinned host tokens; hW: pinned host weight; hout = (codes, scales, zeros)
+        pinned host tensors shaped like cal.q's; hloss (optional): pinned float64 [1]."""
+        cal, comp = self.cal, self.cal.ctx.stream
+        st = self.sets[self.step % len(self.sets)]
+        self.step += 1
+        ev = torch.cuda.Event
+        if st["free"] is not None:
+            self.inp.wait_event(st["free"])
+        ev_x, ev_w = [], ev()
+        with torch.cuda.stream(self.inp):
+            for dx, hx in zip(st["X"], hX):
+                dx.copy_(hx, non_blocking=True)
+                ev_x.append(ev())
+                ev_x[-1].record(self.inp)
+            st["W"].copy_(hW, non_blocking=True)
+            ev_w.record(self.inp)
+        cal.reset()
+        for l, dx in enumerate(st["X"]):
+            comp.wait_event(ev_x[l])
+            cal.collect(l, dx)
+        comp.wait_event(ev_w)
+        if self.outputs_copied is not None:
+            comp.wait_event(self.outputs_copied)
+        cal.quantize(st["W"], mode, read_loss=hloss is None)
+        st["free"] = ev()
+        st["free"].record(comp)
+        self.out.wait_event(st["free"])
+        with torch.cuda.stream(self.out):
+            for h, d in zip(hout, (cal.q.codes, cal.q.scales, cal.q.zeros)):
+                h.copy_(d, non_blocking=True)
+            if hloss is not None:
+                hloss.copy_(cal.loss_dev, non_blocking=True)
+        done = ev()
+        done.record(self.out)
+        self.outputs_copied = done
+
+    def join(self):
+        """Make the context's stream wait for every copy queued so far."""
         if self.outputs_copied is not None:
             self.cal.ctx.stream.wait_event(self.outputs_copied)
 
