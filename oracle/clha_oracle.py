@@ -52,7 +52,7 @@ import numpy as np
 
 __all__ = [
     "route_topk", "expert_tokens", "gram", "hessian", "bf16_round", "silu", "ffn_act",
-    "aggregate", "factor", "grid_fp32", "quantize_fp32", "gptq", "loss",
+    "aggregate", "factor", "boundary_distance", "grid_fp32", "quantize_fp32", "gptq", "loss",
     "calibrate_dense", "calibrate_moe_group",
     "pack_codes", "unpack_codes", "dequantize", "dequant_matmul",
     "routing_divergence", "hessian_error",
@@ -176,12 +176,21 @@ def factor(H_d):
     return np.linalg.cholesky(Hinv).T
 
 
-def grid_fp32(wgrp, bits: int):
+def boundary_distance(v):
+    """Distance of each value to the nearest rounding boundary of round-to-nearest-integer (the
+    half-integers): 0.5 for an integer, 0 exactly on a boundary. A diagnostic of how close a rounding
+    decision was, not part of the method."""
+    v = np.asarray(v, dtype=np.float64)
+    return np.abs(np.abs(v - np.rint(v)) - 0.5)
+
+
+def grid_fp32(wgrp, bits: int, return_margin: bool = False):
     """Asymmetric min-max grid of each row of a group, decided in binary32.
 
     wgrp: [rows, g] current values. Returns (s, z) float32 [rows]: step s = (xmax - xmin)/(2^b - 1)
     and integer zero point z = round(-xmin / s), with xmin <= 0 <= xmax (0 always on the grid) and
-    [-1, 1] for an all-zero group.
+    [-1, 1] for an all-zero group. return_margin: also the boundary distance of -xmin / s, the value
+    the zero point rounds.
     """
     w = np.asarray(wgrp, dtype=np.float64).astype(np.float32)
     maxq = np.float32(2 ** bits - 1)
@@ -191,7 +200,10 @@ def grid_fp32(wgrp, bits: int):
     xmin = np.where(dead, np.float32(-1), xmin).astype(np.float32)
     xmax = np.where(dead, np.float32(1), xmax).astype(np.float32)
     s = ((xmax - xmin).astype(np.float32) / maxq).astype(np.float32)
-    z = np.rint((-xmin).astype(np.float32) / s).astype(np.float32)
+    zv = ((-xmin).astype(np.float32) / s).astype(np.float32)
+    z = np.rint(zv).astype(np.float32)
+    if return_margin:
+        return s, z, boundary_distance(zv)
     return s, z
 
 
@@ -204,36 +216,56 @@ def quantize_fp32(w, s, z, bits: int):
     return q, wq
 
 
-def gptq(W, U, bits: int, group: int):
+def gptq(W, U, bits: int, group: int, block: int | None = None, margins: bool = False):
     """GPTQ column-sequential quantization of W [d_out, d_in] with U = chol_upper(H_d^-1).
 
-    Unblocked form (lazy blocks change only the order of the same float64 updates). For each column
-    j in natural order: at a group start, fix each row's grid from the current values of that group;
-    quantize the current value; e = (w_j - what_j) / U_jj; subtract e * U[j, k] from every later
-    column k of the row. Rows are independent and are processed together.
+    For each column j in natural order: at a group start, fix each row's grid from the current
+    values of that group; quantize the current value; e = (w_j - what_j) / U_jj; subtract e * U[j, k]
+    from every later column k of the row. Rows are independent and are processed together.
+    block=None applies every update at once (unblocked). block=B is GPTQ's lazy-batch form
+    (Algorithm 1): inside a block of B columns the updates reach the block's own later columns column
+    by column, and the later blocks receive the block's errors in one product E U[block, later] at
+    its end: the same float64 updates in another order.
     Returns codes uint8 [d_out, d_in], scales float32 and zeros uint8 [d_out, d_in/group],
-    W_hat float32 [d_out, d_in].
+    W_hat float32 [d_out, d_in]; with margins=True also a dict of rounding margins, the boundary
+    distance of each code's value w/s ("code", [d_out, d_in]) and of each zero point's -xmin/s
+    ("zero", [d_out, d_in/group]): how far each integer decision was from flipping.
     """
     Wc = np.array(W, dtype=np.float64, copy=True)
     U = np.asarray(U, dtype=np.float64)
     d_out, d_in = Wc.shape
     if d_in % group:
         raise ValueError("d_in must be a multiple of the group size")
+    B = d_in if block is None else int(block)
     codes = np.zeros((d_out, d_in), np.uint8)
     scales = np.zeros((d_out, d_in // group), np.float32)
     zeros = np.zeros((d_out, d_in // group), np.uint8)
     W_hat = np.zeros((d_out, d_in), np.float32)
+    mc = np.zeros((d_out, d_in)) if margins else None
+    mz = np.zeros((d_out, d_in // group)) if margins else None
     s = z = None
-    for j in range(d_in):
-        if j % group == 0:
-            s, z = grid_fp32(Wc[:, j:j + group], bits)
-            scales[:, j // group] = s
-            zeros[:, j // group] = z.astype(np.uint8)
-        q, wq = quantize_fp32(Wc[:, j], s, z, bits)
-        codes[:, j] = q.astype(np.uint8)
-        W_hat[:, j] = wq
-        err = (Wc[:, j] - wq.astype(np.float64)) / U[j, j]
-        Wc[:, j + 1:] -= np.outer(err, U[j, j + 1:])
+    for b0 in range(0, d_in, B):
+        b1 = min(d_in, b0 + B)
+        Err = np.zeros((d_out, b1 - b0))
+        for j in range(b0, b1):
+            if j % group == 0:
+                s, z, zm = grid_fp32(Wc[:, j:j + group], bits, return_margin=True)
+                scales[:, j // group] = s
+                zeros[:, j // group] = z.astype(np.uint8)
+                if margins:
+                    mz[:, j // group] = zm
+            q, wq = quantize_fp32(Wc[:, j], s, z, bits)
+            if margins:
+                mc[:, j] = boundary_distance((Wc[:, j].astype(np.float32) / s).astype(np.float32))
+            codes[:, j] = q.astype(np.uint8)
+            W_hat[:, j] = wq
+            err = (Wc[:, j] - wq.astype(np.float64)) / U[j, j]
+            Err[:, j - b0] = err
+            Wc[:, j + 1:b1] -= np.outer(err, U[j, j + 1:b1])
+        if b1 < d_in:
+            Wc[:, b1:] -= Err @ U[b0:b1, b1:]
+    if margins:
+        return codes, scales, zeros, W_hat, {"code": mc, "zero": mz}
     return codes, scales, zeros, W_hat
 
 
@@ -245,29 +277,32 @@ def loss(W, W_hat, H):
 
 # ----------------------------------------------------------------------------------- pipelines
 def calibrate_dense(W, X_list, bits: int, group: int = 128, mode: str = "rt", alpha=None,
-                    damp_frac: float = 0.01):
-    """CLHA for one weight W [d_out, d_in] shared by the layers whose inputs are X_list."""
+                    damp_frac: float = 0.01, block: int | None = 128):
+    """CLHA for one weight W [d_out, d_in] shared by the layers whose inputs are X_list (GPTQ in its
+    lazy-batch form with `block` columns per batch; None: unblocked). "margin" holds GPTQ's rounding
+    margins."""
     S = [gram(X) for X in X_list]
     n = [int(np.asarray(X).shape[0]) for X in X_list]
     agg = aggregate(S, n, mode, alpha, damp_frac)
     U = factor(agg["H_d"])
-    codes, scales, zeros, W_hat = gptq(W, U, bits, group)
+    codes, scales, zeros, W_hat, margin = gptq(W, U, bits, group, block, margins=True)
     return {"S": S, "n": n, **agg, "U": U, "codes": codes, "scales": scales, "zeros": zeros,
-            "W_hat": W_hat, "loss": loss(W, W_hat, agg["H_comb"]),
+            "W_hat": W_hat, "margin": margin, "loss": loss(W, W_hat, agg["H_comb"]),
             "layer_loss": [loss(W, W_hat, hessian(Si, ni)) for Si, ni in zip(S, n)]}
 
 
 def calibrate_moe_group(X_list, logits_list, k: int, routed, shared=(), experts=None,
                         bits_routed: int = 2, bits_shared: int = 3, group: int = 128,
                         mode: str = "rt", damp_frac: float = 0.01, shared_experts=None, alpha=None,
-                        empty: str = "error"):
+                        empty: str = "error", block: int | None = 128):
     """CLHA on one group of layers sharing routed experts `routed` [(Wg, Wu, Wd)] and always-active
     experts `shared` (CLHA page §2.2 phases 1-3, §2.3 mixed precision, §2.4 per-layer accumulators).
 
     experts / shared_experts: which routed / always-active experts to calibrate (default: all).
     Returns per-layer routing and, per expert key ("r", e) / ("s", e): token counts "n", the Hessian
     data "H_in" (gate/up inputs x) and "H_down" (down-projection inputs h), and the GPTQ results
-    "gate", "up", "down".
+    "gate", "up", "down" (with their rounding margins under "margin"). GPTQ runs in its lazy-batch
+    form with `block` columns per batch (None: unblocked).
     """
     E = len(routed)
     if experts is None:
@@ -291,8 +326,8 @@ def calibrate_moe_group(X_list, logits_list, k: int, routed, shared=(), experts=
             U = factor(agg["H_d"])
             res[kind] = {"S": S, **agg, "U": U}
             for name, Wm in mats:
-                codes, scales, zeros, W_hat = gptq(Wm, U, bits, group)
-                res[name] = {"codes": codes, "scales": scales, "zeros": zeros, "W_hat": W_hat,
+                codes, scales, zeros, W_hat, margin = gptq(Wm, U, bits, group, block, margins=True)
+                res[name] = {"codes": codes, "scales": scales, "zeros": zeros, "W_hat": W_hat, "margin": margin,
                              "loss": loss(Wm, W_hat, agg["H_comb"])}
         res["loss"] = res["gate"]["loss"] + res["up"]["loss"] + res["down"]["loss"]
         res["h"] = he

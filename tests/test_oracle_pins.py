@@ -276,35 +276,37 @@ def test_gptq_two_columns_closed_form():
     np.testing.assert_array_equal(W_hat[:, 1], wq1)
 
 
-def _blocked_gptq(W, U, bits, group, block):
-    """Lazy-block form: updates inside a block are applied column by column, the accumulated errors
-    reach later blocks in one product at the end of each block."""
-    Wc = np.array(W, dtype=np.float64)
-    d_out, d_in = Wc.shape
-    codes = np.zeros((d_out, d_in), np.uint8)
-    for b0 in range(0, d_in, block):
-        b1 = min(d_in, b0 + block)
-        Err = np.zeros((d_out, b1 - b0))
-        for j in range(b0, b1):
-            if j % group == 0:
-                s, z = O.grid_fp32(Wc[:, j:j + group], bits)
-            q, wq = O.quantize_fp32(Wc[:, j], s, z, bits)
-            codes[:, j] = q
-            e = (Wc[:, j] - wq.astype(np.float64)) / U[j, j]
-            Err[:, j - b0] = e
-            Wc[:, j + 1:b1] -= np.outer(e, U[j, j + 1:b1])
-        Wc[:, b1:] -= Err @ U[b0:b1, b1:]
-    return codes
-
-
 @pytest.mark.parametrize("block", [1, 8, 32, 128])
 def test_gptq_blocking_does_not_change_codes(block):
     d = 256
     H = _spd(d, rank=64, seed=3, damp=0.02)
     U = O.factor(H)
     W = 0.02 * RNG.standard_normal((8, d))
-    codes, *_ = O.gptq(W, U, 3, 128)
-    np.testing.assert_array_equal(_blocked_gptq(W, U, 3, 128, block), codes)
+    codes, scales, zeros, W_hat = O.gptq(W, U, 3, 128)
+    cb, sb, zb, wb, mb = O.gptq(W, U, 3, 128, block=block, margins=True)
+    np.testing.assert_array_equal(cb, codes)
+    np.testing.assert_array_equal(sb, scales)
+    np.testing.assert_array_equal(zb, zeros)
+    np.testing.assert_array_equal(wb, W_hat)
+    assert mb["code"].shape == codes.shape and np.all((mb["code"] >= 0) & (mb["code"] <= 0.5))
+
+
+def test_gptq_margins_are_distances_to_the_rounding_boundary():
+    """With H = I (round to nearest) the code margin of w is |(|w/s - rint(w/s)|) - 1/2|, worked by
+    hand on values placed at known offsets from the grid: a value on a grid point has margin 1/2, one
+    a quarter step past a boundary has margin 1/4; the zero point's margin is that of -xmin/s."""
+    # one row, one group of 128: xmin = -0.3 and xmax = 0.4 fix s = 0.7/7 = 0.1 (3 bits) and z = 3
+    w = np.zeros(128)
+    w[0], w[1] = -0.3, 0.4
+    w[2] = 0.15 + 0.025          # a quarter step past the boundary 1.5 s: code 3 + 2 = 5
+    w[3] = 0.2                   # on the grid point 2 s: code 5
+    w[4] = -0.05 - 0.0125        # an eighth of a step past the boundary -0.5 s: code 3 - 1 = 2
+    codes, scales, zeros, _, m = O.gptq(w[None], np.eye(128), 3, 128, margins=True)
+    assert scales[0, 0] == np.float32(np.float32(np.float32(0.4) - np.float32(-0.3)) / np.float32(7)) and zeros[0, 0] == 3
+    np.testing.assert_allclose(m["code"][0, :5], [0.5, 0.5, 0.25, 0.5, 0.125], atol=1e-5)
+    assert list(codes[0, :5]) == [0, 7, 5, 5, 2]
+    np.testing.assert_allclose(m["zero"][0, 0], 0.5, atol=1e-5)     # -xmin/s = 3
+    np.testing.assert_allclose(O.boundary_distance([0.5, 1.0, 2.25, -0.75]), [0.0, 0.5, 0.25, 0.25])
 
 
 def test_brute_force_lower_bounds_gptq():
