@@ -299,7 +299,10 @@ CLHA_API clha_status clha_epmq_target(clha_ctx* ctx, const clha_accum* acc, int 
  * and its error (w - w_hat)/U_jj is subtracted along row j of U from the later columns. The grid and
  * the code are decided in IEEE float32 (round to nearest even); the updates inside a block accumulate
  * in float32 and the lazy block updates run on the tensor cores in three tf32 products (hi*hi +
- * hi*lo + lo*hi), float32-class accuracy.
+ * hi*lo + lo*hi), float32-class accuracy. The columns are taken in chunks of 512: a lazy update sums
+ * at most one chunk's errors in the tensor core's accumulator, and each finished chunk's errors are
+ * folded into float32 running weights of the later columns with round-to-nearest adds (workspace:
+ * one more float32 copy of W when d_in > 512).
  * Outputs: codes uint8 [batch, d_out, d_in], scales float32 and zeros uint8 [batch, d_out, d_in/128],
  * W_hat float32 [batch, d_out, d_in] (may be NULL).
  * Optional loss (device double [batch], overwritten), given lambda (device double [n_u], the damping of
@@ -337,6 +340,23 @@ CLHA_API clha_status clha_loss(clha_ctx* ctx, const void* W, clha_dtype dtype, c
  * pairs are NaN. */
 CLHA_API clha_status clha_routing_divergence(clha_ctx* ctx, const int64_t* counts, int n_layers, int ld, int slot0,
                                              int E, double* tv);
+
+/* ----------------------------------------------------------------------- multi-GPU exchange */
+
+/* Packed upper triangles of a batch of Gram sums, for the token-sharded collection's exchange
+ * between GPUs (the CLHA page, §2.2 (1): the Hessians are sums over tokens, so GPUs that collect
+ * disjoint token shares add their partial sums; S is symmetric and only its upper triangle is read,
+ * so only d(d+1)/2 floats per matrix need to cross). The matrices are S + (o * outer_stride + i) * d * d
+ * for o < n_outer, i < n_inner (outer_stride >= n_inner, in matrices; e.g. the slots [e0, e0 + n) of
+ * every layer of an accumulator: S = the accumulator's S at slot e0, n_outer = its layers,
+ * outer_stride = its slot count, n_inner = n). packed holds them in (o, i) order, each as rows
+ * i = 0 .. d-1 of entries (i, i .. d-1): d(d+1)/2 floats per matrix. clha_unpack_upper writes the
+ * upper triangles back and leaves the strict lower triangles as they were. Device pointers, the
+ * caller's; nothing synchronises. */
+CLHA_API clha_status clha_pack_upper(clha_ctx* ctx, const float* S, int64_t n_outer, int64_t outer_stride,
+                                     int64_t n_inner, int d, float* packed);
+CLHA_API clha_status clha_unpack_upper(clha_ctx* ctx, const float* packed, int64_t n_outer, int64_t outer_stride,
+                                       int64_t n_inner, int d, float* S);
 
 #ifdef __cplusplus
 }

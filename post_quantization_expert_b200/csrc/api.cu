@@ -601,7 +601,7 @@ extern "C" clha_status clha_quantize(clha_ctx* ctx, const float* U, int n_u, con
     void* ws = nullptr;
     clha_status st = clha_workspace(ctx, quantize_workspace_bytes(batch, d_out, d_in), &ws);
     if (st) return st;
-    CUDA_TRY(launch_quantize(ctx->stream, U, n_u, W, dtype == CLHA_F32, batch, d_out, d_in, p->bits, codes,
+    CUDA_TRY(launch_quantize(ctx->stream, ctx->num_sms, U, n_u, W, dtype == CLHA_F32, batch, d_out, d_in, p->bits, codes,
                              scales, zeros, W_hat, lambda, loss, ws, ctx->d_err), "clha_quantize");
     return CLHA_OK;
 }
@@ -628,3 +628,28 @@ extern "C" clha_status clha_loss(clha_ctx* ctx, const void* W, clha_dtype dtype,
     return clha_sync_and_check(ctx, "clha_loss");
 }
 
+
+// ------------------------------------------------------------------------------ multi-GPU exchange
+extern "C" clha_status clha_pack_upper(clha_ctx* ctx, const float* S, int64_t n_outer, int64_t outer_stride,
+                                       int64_t n_inner, int d, float* packed) {
+    CHECK_CTX(ctx);
+    REQUIRE(n_outer >= 0 && n_inner >= 0 && d > 0 && outer_stride >= n_inner, CLHA_ERR_INVALID_ARG,
+            "clha_pack_upper: bad sizes (need n_outer, n_inner >= 0, d > 0, outer_stride >= n_inner)");
+    REQUIRE((S && packed) || n_outer * n_inner == 0, CLHA_ERR_INVALID_ARG, "clha_pack_upper: null pointer");
+    SET_DEVICE(ctx);
+    LaunchScope launch_scope(ctx);
+    CUDA_TRY(launch_pack_upper(ctx->stream, S, n_outer, outer_stride, n_inner, d, packed), "clha_pack_upper");
+    return CLHA_OK;
+}
+
+extern "C" clha_status clha_unpack_upper(clha_ctx* ctx, const float* packed, int64_t n_outer, int64_t outer_stride,
+                                         int64_t n_inner, int d, float* S) {
+    CHECK_CTX(ctx);
+    REQUIRE(n_outer >= 0 && n_inner >= 0 && d > 0 && outer_stride >= n_inner, CLHA_ERR_INVALID_ARG,
+            "clha_unpack_upper: bad sizes (need n_outer, n_inner >= 0, d > 0, outer_stride >= n_inner)");
+    REQUIRE((S && packed) || n_outer * n_inner == 0, CLHA_ERR_INVALID_ARG, "clha_unpack_upper: null pointer");
+    SET_DEVICE(ctx);
+    LaunchScope launch_scope(ctx);
+    CUDA_TRY(launch_unpack_upper(ctx->stream, packed, n_outer, outer_stride, n_inner, d, S), "clha_unpack_upper");
+    return CLHA_OK;
+}

@@ -131,8 +131,12 @@ size_t epmq_workspace_bytes(int d_out, int d);
 cudaError_t launch_epmq_target(cudaStream_t s, const float* S_slot, int64_t layer_stride, int K, const void* W_src,
                                int w_bf16, const void* W_m, int d_out, int d, const float* U, const double* lambda,
                                float* W_target, void* ws);
+cudaError_t launch_pack_upper(cudaStream_t s, const float* S, int64_t n_outer, int64_t outer_stride, int64_t n_inner,
+                              int d, float* P);
+cudaError_t launch_unpack_upper(cudaStream_t s, const float* P, int64_t n_outer, int64_t outer_stride,
+                                int64_t n_inner, int d, float* S);
 size_t quantize_workspace_bytes(int batch, int d_out, int d_in);
-cudaError_t launch_quantize(cudaStream_t s, const float* U, int n_u, const void* W, int w_is_f32,
+cudaError_t launch_quantize(cudaStream_t s, int num_sms, const float* U, int n_u, const void* W, int w_is_f32,
                             int batch, int d_out, int d_in, int bits, uint8_t* codes, float* scales,
                             uint8_t* zeros, float* W_hat, const double* lambda, double* loss, void* ws,
                             int* err);

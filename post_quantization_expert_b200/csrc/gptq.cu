@@ -27,6 +27,14 @@
 //              pipe at a time), into the other of two TMEM accumulators.
 // The grid and the code are decided with IEEE float32 operations (division and rounding to nearest
 // even), the same operations a float32 reference takes on the same current value.
+//
+// Column chunks. The tensor core's fp32 accumulator does not round each addition to nearest, so a
+// lazy update that sums the errors of many thousands of columns in TMEM drifts away from the exact
+// sum (enough, on long rows, to flip rounding decisions that float32 arithmetic rounding to nearest
+// would not). A launch therefore quantizes one chunk of at most CHUNK = 512 columns, its lazy updates
+// summing only that chunk's errors, and gptq_trail then folds the chunk's errors into float32 running
+// weights of every later column (a tcgen05 product over the chunk, subtracted by TMA reduce-add: fp32
+// adds rounded to nearest). A weight with at most CHUNK columns takes one launch and no running copy.
 #include "clha_internal.h"
 #include "tc_ptx.h"
 #include "tmap.h"
@@ -66,8 +74,10 @@ __host__ __device__ constexpr uint32_t idesc_spill(int n) {
 struct GptqParams {
     const float* U;        // [n_u, d_in, d_in] (for the diagonal blocks)
     int n_u;               // problem b uses factor b % n_u
-    const void* W;
+    const void* W;         // the original weights (the loss compares W_hat with them)
     int w_f32;
+    const float* Wc;       // float32 running weights (W minus the earlier chunks' updates), or null: W
+    int c0, c1;            // the column chunk this launch quantizes
     int d_out, d_in, bits;
     uint8_t* codes;
     float* scales;
@@ -113,10 +123,10 @@ __device__ __forceinline__ void quarter_sweep(float (&w)[QW], float s, float z, 
     }
 }
 
-// W[row, c0 .. c0+31] as floats (bf16 or fp32 source).
-__device__ __forceinline__ void load_w32(const GptqParams& p, size_t off, float (&w)[QW]) {
-    if (p.w_f32) {
-        const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.W) + off);
+// W[row, c0 .. c0+31] as floats (bf16 or fp32 source); cur: the running weights when they exist.
+__device__ __forceinline__ void load_w32(const GptqParams& p, size_t off, float (&w)[QW], bool cur = false) {
+    if (p.w_f32 || (cur && p.Wc)) {
+        const float4* src = reinterpret_cast<const float4*>((cur && p.Wc ? p.Wc : reinterpret_cast<const float*>(p.W)) + off);
 #pragma unroll
         for (int i = 0; i < QW / 4; ++i) {
             const float4 v = src[i];
@@ -167,6 +177,7 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
     const int r0 = blockIdx.x * R;
     const int u = b % p.n_u;
     const int nblk = p.d_in / BLK;
+    const int b_lo = p.c0 / BLK, b_hi = p.c1 / BLK;   // this launch's blocks; local index lb = bb - b_lo
     const int ey = b * p.d_out + r0;               // this CTA's rows in the [batch * d_out, d_in] E view
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -201,12 +212,12 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
             tc::prefetch_tmap(&tmUlo);
             int it = 0;
             bool ok = true;
-            for (int bb = 1; bb < nblk && ok; ++bb) {
+            for (int bb = b_lo + 1; bb < b_hi && ok; ++bb) {
                 const int cb = bb * BLK;
-                for (int ks = 0; ks < cb / KS; ++ks) {
+                for (int ks = p.c0 / KS; ks < cb / KS; ++ks) {   // the chunk's earlier errors only
                     const int k0 = ks * KS;
                     if (k0 == cb - BLK) {   // errors of the previous block: wait until they are stored
-                        if (!tc::mbar_wait_bounded(eready, (bb - 1) & 1, abort_flag)) { ok = false; break; }
+                        if (!tc::mbar_wait_bounded(eready, (bb - 1 - b_lo) & 1, abort_flag)) { ok = false; break; }
                     }
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
@@ -232,15 +243,16 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
         if (lane == 0) {
             int it = 0, nq = 0;   // lazy k steps consumed; quarter products issued
             bool ok = true;
-            for (int bb = 0; bb < nblk && ok; ++bb) {
-                // block bb: its three quarter products (into acc bb & 1) and block bb+1's lazy update
-                const bool lazy = bb + 1 < nblk;
-                const int lacc = (bb + 1) & 1, pacc = bb & 1;
-                const int nks = lazy ? (bb + 1) * BLK / KS : 0;
+            for (int bb = b_lo; bb < b_hi && ok; ++bb) {
+                // block bb: its three quarter products (into acc lb & 1) and block bb+1's lazy update
+                const int lb = bb - b_lo;
+                const bool lazy = bb + 1 < b_hi;
+                const int lacc = (lb + 1) & 1, pacc = lb & 1;
+                const int nks = lazy ? ((bb + 1) * BLK - p.c0) / KS : 0;
                 int ks = 0, q = 0;
                 bool lazy_ready = !lazy;
-                if (lazy && bb >= 1) {   // the row threads are done with block bb-1's accumulator
-                    if (!tc::mbar_wait_bounded(tempty0 + 8 * lacc, ((bb - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+                if (lazy && lb >= 1) {   // the row threads are done with block bb-1's accumulator
+                    if (!tc::mbar_wait_bounded(tempty0 + 8 * lacc, ((lb - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
                     tc::fence_after_sync();
                 }
                 lazy_ready = true;
@@ -265,7 +277,7 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                                     const uint64_t dal = tc::sw128_desc(sa_lo + kk * 32, 16, 1024);
                                     const uint64_t dbh = tc::sw128_desc(sbh + boff + kk * 32, 16, 1024);
                                     const uint64_t dbl = tc::sw128_desc(sbl + boff + kk * 32, 16, 1024);
-                                    tc::mma_tf32(d_tmem, dah, dbh, id, (bb > 0 || q > 0 || kk > 0) ? 1u : 0u);
+                                    tc::mma_tf32(d_tmem, dah, dbh, id, (lb > 0 || q > 0 || kk > 0) ? 1u : 0u);
                                     tc::mma_tf32(d_tmem, dah, dbl, id, 1);
                                     tc::mma_tf32(d_tmem, dal, dbh, id, 1);
                                 }
@@ -348,26 +360,28 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
         };
         // On a failed wait (abort) the row threads still run every step, so each reaches every named
         // barrier; their later waits return at once.
-        load_uq(0);
-        for (int bb = 0; bb < nblk; ++bb) {
+        load_uq(p.c0);
+        for (int bb = b_lo; bb < b_hi; ++bb) {
             const int cb = bb * BLK;
-            const int acc = bb & 1;
-            const bool more = bb + 1 < nblk;
+            const int lb = bb - b_lo;
+            const int acc = lb & 1;
+            const bool more = bb + 1 < nblk;             // later blocks (of this chunk or later ones) need E
+            const bool next_here = bb + 1 < b_hi;        // the next block is this launch's
             const size_t orow = ((size_t)b * p.d_out + row) * p.d_in + cb;   // this row's outputs
             row_bar();                                   // the last block's readers of Uq are done
             if (t == 0) load_sb(cb, 0);
             cp_async_wait_all();                         // this block's Uq (issued during the last block)
             uinv[t] = 1.0f / __ldg(Ub + (size_t)(cb + t) * p.d_in + cb + t);
-            if (bb > 0) {
-                if (!tc::mbar_wait_bounded(tfull0 + 8 * acc, (bb - 1) >> 1 & 1, abort_flag)) ok = false;
+            if (lb > 0) {
+                if (!tc::mbar_wait_bounded(tfull0 + 8 * acc, (lb - 1) >> 1 & 1, abort_flag)) ok = false;
                 tc::fence_after_sync();
             }
             // grid of the group from the current values (0 always on the grid; [-1, 1] if all zero)
             float xmin = 0.f, xmax = 0.f;
             for (int ch = 0; ch < 4; ++ch) {
                 float w[QW];
-                load_w32(p, wrow + cb + QW * ch, w);
-                if (bb > 0) {
+                load_w32(p, wrow + cb + QW * ch, w, true);
+                if (lb > 0) {
                     uint32_t v[32];
                     tc::tmem_ld_32x32b_x32(tmem + lane_base + acc * BLK + ch * QW, v);
                     tc::tmem_wait_ld();
@@ -385,13 +399,13 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
             row_bar();                                   // Uq, uinv visible to every row thread
             for (int q = 0; q < 4; ++q) {
                 float w[QW];
-                load_w32(p, wrow + cb + QW * q, w);
+                load_w32(p, wrow + cb + QW * q, w, true);
                 if (q > 0) {                             // the previous quarter's product reached this quarter
                     if (!tc::mbar_wait_bounded(sdone, (nq - 1) & 1, abort_flag)) ok = false;
                     tc::fence_after_sync();
                     if (t == 0 && q < 3) load_sb(cb, q);
                 }
-                if (bb > 0 || q > 0) {
+                if (lb > 0 || q > 0) {
                     uint32_t v[32];
                     tc::tmem_ld_32x32b_x32(tmem + lane_base + acc * BLK + q * QW, v);
                     tc::tmem_wait_ld();
@@ -438,7 +452,7 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                 if (q > 0 && !tc::mbar_wait_bounded(sdone2, (nq - 1) & 1, abort_flag)) ok = false;
                 if (t == 0) tc::bulk_wait_read<0>();
                 row_bar();
-                if (q == 3) load_uq(cb + BLK);           // every row is past its last use of Uq
+                if (q == 3 && next_here) load_uq(cb + BLK);   // every row is past its last use of Uq
                 uint8_t* sah = smem + SA_OFF + t * 128;
                 uint8_t* sal = sah + SA_BYTES;
 #pragma unroll
@@ -470,9 +484,10 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                     }
                 }
             }
-            if (more) {   // this row's W for the next block into L1
-                const char* nxt = reinterpret_cast<const char*>(p.W) + (wrow + cb + BLK) * (p.w_f32 ? 4 : 2);
-                for (int o = 0; o < BLK * (p.w_f32 ? 4 : 2); o += 128)
+            if (next_here) {   // this row's weights for the next block into L1
+                const int es = (p.w_f32 || p.Wc) ? 4 : 2;
+                const char* nxt = reinterpret_cast<const char*>(p.Wc ? (const void*)p.Wc : p.W) + (wrow + cb + BLK) * es;
+                for (int o = 0; o < BLK * es; o += 128)
                     asm volatile("prefetch.global.L1 [%0];" ::"l"(nxt + o));
             }
         }
@@ -496,6 +511,193 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
         tc::tmem_dealloc(tmem, 256);
     }
     if (threadIdx.x == 0 && *abort_flag) clha_record_error(p.err, CLHA_ERR_TIMEOUT, b, r0, KID_QUANTIZE);
+}
+
+// ------------------------------------------------------------------------------ trailing update
+// The tensor core adds a product into its fp32 accumulator without rounding to nearest, so a long
+// chain of accumulations drifts (for a lazy update over tens of thousands of columns, far enough to
+// move GPTQ's rounding decisions). GPTQ therefore runs in column chunks of CHUNK columns: inside a
+// chunk the lazy updates accumulate at most CHUNK columns of errors in TMEM, and at the end of a chunk
+// this kernel folds the chunk's errors into the running weights of all later columns,
+//   Wc[rows, n] -= sum_{k in chunk} E[rows, k] U[k, n],   n >= chunk end,
+// as a 3xTF32 tcgen05 product (K = the chunk) whose fp32 result is subtracted by a TMA reduce-add (the
+// L2's fp32 adds round to nearest). Persistent: tiles of 128 rows x 128 columns; warp 0 is the TMA
+// producer, warp 1 the MMA issuer (two TMEM accumulators, so a tile's epilogue overlaps the next
+// tile's products), warps 2-5 the epilogue (one TMEM lane quadrant each).
+constexpr int CHUNK = 512;
+constexpr int T_STAGES = 2;
+constexpr int T_STG_OFF = T_STAGES * STAGE_BYTES;           // 128 KB of operand stages
+constexpr int T_BAR_OFF = T_STG_OFF + 4 * 2 * 4096;          // + two 4 KB staging boxes per epilogue warp
+constexpr int T_SMEM_BYTES = T_BAR_OFF + 256 + 1024;
+static_assert(T_SMEM_BYTES <= 232448, "shared memory");
+
+struct TrailParams {
+    int d_out, d_in, n_u;
+    int c0, c1;          // the chunk whose errors are folded; columns >= c1 are updated
+    int n_rt, n_ct;      // row tiles (batch * d_out / 128) and column tiles ((d_in - c1) / 128)
+    int* err;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+gptq_trail(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUtensorMap tmElo,
+           const __grid_constant__ CUtensorMap tmUhi, const __grid_constant__ CUtensorMap tmUlo,
+           const __grid_constant__ CUtensorMap tmWc, TrailParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T_BAR_OFF);
+    const uint32_t full0 = tc::smem_u32(bars);
+    const uint32_t empty0 = full0 + 8 * T_STAGES;
+    const uint32_t tfull0 = empty0 + 8 * T_STAGES;
+    const uint32_t tempty0 = tfull0 + 16;
+    const uint32_t drain = tempty0 + 16;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * T_STAGES + 5);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int total = p.n_rt * p.n_ct;
+    const int nk = (p.c1 - p.c0) / KS;
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < T_STAGES; ++st) {
+            tc::mbar_init(full0 + 8 * st, 1);
+            tc::mbar_init(empty0 + 8 * st, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            tc::mbar_init(tfull0 + 8 * a, 1);
+            tc::mbar_init(tempty0 + 8 * a, 128);
+        }
+        tc::mbar_init(drain, 1);
+        *abort_flag = 0;
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) tc::tmem_alloc(tc::smem_u32(tmem_slot), 256);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tc::prefetch_tmap(&tmEhi);
+            tc::prefetch_tmap(&tmElo);
+            tc::prefetch_tmap(&tmUhi);
+            tc::prefetch_tmap(&tmUlo);
+            int it = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+                const int rt = w % p.n_rt, ct = w / p.n_rt;
+                const int row0 = rt * R;
+                const int u = (row0 / p.d_out) % p.n_u;
+                const int ny = u * p.d_in + p.c1 + ct * BLK;   // rows n of the transposed factor
+                for (int ks = 0; ks < nk; ++ks, ++it) {
+                    const int st = it % T_STAGES;
+                    const uint32_t ph = (it / T_STAGES) & 1;
+                    if (!tc::mbar_wait_bounded(empty0 + 8 * st, ph ^ 1, abort_flag)) { ok = false; break; }
+                    const uint32_t fb = full0 + 8 * st;
+                    tc::mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    const uint32_t sa = tc::smem_u32(smem + st * STAGE_BYTES);
+                    const int k0 = p.c0 + ks * KS;
+                    tc::tma_load_2d(sa, &tmEhi, fb, k0, row0);
+                    tc::tma_load_2d(sa + A_BYTES, &tmElo, fb, k0, row0);
+                    tc::tma_load_2d(sa + 2 * A_BYTES, &tmUhi, fb, k0, ny);
+                    tc::tma_load_2d(sa + 2 * A_BYTES + B_BYTES, &tmUlo, fb, k0, ny);
+                }
+            }
+            if (!ok) {   // let the copies already issued land before the CTA can exit
+                for (int j = it - 1; j >= 0 && j >= it - T_STAGES; --j)
+                    tc::mbar_wait_bounded(full0 + 8 * (j % T_STAGES), (j / T_STAGES) & 1, abort_flag, 100000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int it = 0, tcount = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++tcount) {
+                const int acc = tcount & 1;
+                if (!tc::mbar_wait_bounded(tempty0 + 8 * acc, ((tcount >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                tc::fence_after_sync();
+                const uint32_t d_tmem = tmem + acc * BLK;
+                for (int ks = 0; ks < nk; ++ks, ++it) {
+                    const int st = it % T_STAGES;
+                    if (!tc::mbar_wait_bounded(full0 + 8 * st, (it / T_STAGES) & 1, abort_flag)) { ok = false; break; }
+                    tc::fence_after_sync();
+                    const uint32_t ahi = tc::smem_u32(smem + st * STAGE_BYTES);
+                    const uint32_t alo = ahi + A_BYTES, bhi = ahi + 2 * A_BYTES, blo = bhi + B_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < KS / 8; ++kk) {
+                        const uint64_t dah = tc::sw128_desc(ahi + kk * 32, 16, 1024);
+                        const uint64_t dal = tc::sw128_desc(alo + kk * 32, 16, 1024);
+                        const uint64_t dbh = tc::sw128_desc(bhi + kk * 32, 16, 1024);
+                        const uint64_t dbl = tc::sw128_desc(blo + kk * 32, 16, 1024);
+                        tc::mma_tf32(d_tmem, dah, dbh, IDESC_LAZY, (ks | kk) != 0);
+                        tc::mma_tf32(d_tmem, dah, dbl, IDESC_LAZY, 1);
+                        tc::mma_tf32(d_tmem, dal, dbh, IDESC_LAZY, 1);
+                    }
+                    tc::mma_commit(empty0 + 8 * st);
+                }
+                if (!ok) break;
+                tc::mma_commit(tfull0 + 8 * acc);
+            }
+        }
+        __syncwarp();
+    } else {
+        // epilogue: each warp's 32 rows, 32 columns at a time, negated, 128-byte-swizzled into a staging
+        // box and added into Wc by TMA reduce-add
+        const int q = warp & 3;
+        const uint32_t stg = tc::smem_u32(smem + T_STG_OFF) + q * 8192;
+        int sb = 0, tcount = 0;
+        for (int w = blockIdx.x; w < total; w += gridDim.x, ++tcount) {
+            const int rt = w % p.n_rt, ct = w / p.n_rt;
+            const int wrow = rt * R + q * 32;
+            const int n0 = p.c1 + ct * BLK;
+            const int acc = tcount & 1;
+            if (!tc::mbar_wait_bounded(tfull0 + 8 * acc, (tcount >> 1) & 1, abort_flag)) break;
+            tc::fence_after_sync();
+#pragma unroll 1
+            for (int ch = 0; ch < BLK / 32; ++ch) {
+                uint32_t v[32];
+                tc::tmem_ld_32x32b_x32(tmem + acc * BLK + ch * 32 + ((uint32_t)(q * 32) << 16), v);
+                tc::tmem_wait_ld();
+                const uint32_t buf = stg + sb * 4096;
+                if (lane == 0) tc::bulk_wait_read<1>();   // the reduce that last used buf has read it
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                 ::"r"(buf + lane * 128 + ((j ^ (lane & 7)) << 4)), "r"(v[4 * j] ^ 0x80000000u),
+                                 "r"(v[4 * j + 1] ^ 0x80000000u), "r"(v[4 * j + 2] ^ 0x80000000u),
+                                 "r"(v[4 * j + 3] ^ 0x80000000u) : "memory");
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tc::tma_reduce_add_2d(&tmWc, buf, n0 + ch * 32, wrow);
+                    tc::bulk_commit();
+                }
+                sb ^= 1;
+            }
+            tc::fence_before_sync();
+            tc::mbar_arrive(tempty0 + 8 * acc);
+        }
+        if (lane == 0) tc::bulk_wait_all();
+        __syncwarp();
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        if (lane == 0) {
+            tc::mma_commit(drain);
+            tc::mbar_wait_bounded(drain, 0, abort_flag, 100000000ull);
+        }
+        __syncwarp();
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 256);
+    }
+    if (threadIdx.x == 0 && *abort_flag) clha_record_error(p.err, CLHA_ERR_TIMEOUT, blockIdx.x, 0, KID_QUANTIZE);
+}
+
+// The running weights start as the weights themselves (float32).
+__global__ void gptq_init_wc(const void* __restrict__ W, int w_f32, size_t n, float* __restrict__ Wc) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        Wc[i] = w_f32 ? reinterpret_cast<const float*>(W)[i]
+                      : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(W)[i]);
 }
 
 // U -> transposed (hi, lo) tf32 parts: hi_t[j][i] + lo_t[j][i] ~ U[i][j], so the lazy-update
@@ -522,33 +724,55 @@ __global__ void __launch_bounds__(256) gptq_split_t(const float* __restrict__ U,
 size_t quantize_workspace_bytes(int batch, int d_out, int d_in) {
     const size_t e = clha_round_up((size_t)batch * d_out * d_in * sizeof(float));
     const size_t uu = clha_round_up((size_t)batch * d_in * d_in * sizeof(float));
-    return 2 * e + 2 * uu;
+    return 2 * e + 2 * uu + (d_in > CHUNK ? e : 0);   // E hi/lo, U^T hi/lo, the running weights
 }
 
-cudaError_t launch_quantize(cudaStream_t s, const float* U, int n_u, const void* W, int w_is_f32, int batch,
-                            int d_out, int d_in, int bits, uint8_t* codes, float* scales, uint8_t* zeros,
+cudaError_t launch_quantize(cudaStream_t s, int num_sms, const float* U, int n_u, const void* W, int w_is_f32,
+                            int batch, int d_out, int d_in, int bits, uint8_t* codes, float* scales, uint8_t* zeros,
                             float* W_hat, const double* lambda, double* loss, void* ws, int* err) {
     char* cur = (char*)ws;
-    float* Ehi = (float*)clha_carve(cur, (size_t)batch * d_out * d_in * sizeof(float));
-    float* Elo = (float*)clha_carve(cur, (size_t)batch * d_out * d_in * sizeof(float));
+    const size_t wsz = (size_t)batch * d_out * d_in;
+    float* Ehi = (float*)clha_carve(cur, wsz * sizeof(float));
+    float* Elo = (float*)clha_carve(cur, wsz * sizeof(float));
     float* Uhi = (float*)clha_carve(cur, (size_t)batch * d_in * d_in * sizeof(float));
     float* Ulo = (float*)clha_carve(cur, (size_t)batch * d_in * d_in * sizeof(float));
+    const bool chunked = d_in > CHUNK;
+    float* Wc = chunked ? (float*)clha_carve(cur, wsz * sizeof(float)) : nullptr;
     cudaError_t e;
-    CUtensorMap tEhi, tElo, tUhi, tUlo, tQhi, tQlo;
+    CUtensorMap tEhi, tElo, tUhi, tUlo, tQhi, tQlo, tWc;
     if ((e = make_tmap_2d(&tEhi, Ehi, (uint64_t)batch * d_out, d_in, 4, R, KS)) != cudaSuccess) return e;
     if ((e = make_tmap_2d(&tElo, Elo, (uint64_t)batch * d_out, d_in, 4, R, KS)) != cudaSuccess) return e;
     if ((e = make_tmap_2d(&tUhi, Uhi, (uint64_t)n_u * d_in, d_in, 4, BLK, KS)) != cudaSuccess) return e;
     if ((e = make_tmap_2d(&tUlo, Ulo, (uint64_t)n_u * d_in, d_in, 4, BLK, KS)) != cudaSuccess) return e;
     if ((e = make_tmap_2d(&tQhi, Uhi, (uint64_t)n_u * d_in, d_in, 4, 32, QW)) != cudaSuccess) return e;
     if ((e = make_tmap_2d(&tQlo, Ulo, (uint64_t)n_u * d_in, d_in, 4, 32, QW)) != cudaSuccess) return e;
+    if (chunked && (e = make_tmap_2d(&tWc, Wc, (uint64_t)batch * d_out, d_in, 4, 32, 32)) != cudaSuccess) return e;
     gptq_split_t<<<dim3(d_in / 32, d_in / 32, n_u), 256, 0, s>>>(U, d_in, Uhi, Ulo);
     clha_note_launches(1);
     if ((e = cudaFuncSetAttribute(gptq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) != cudaSuccess)
         return e;
+    if (chunked &&
+        (e = cudaFuncSetAttribute(gptq_trail, cudaFuncAttributeMaxDynamicSharedMemorySize, T_SMEM_BYTES)) != cudaSuccess)
+        return e;
     if (loss && (e = cudaMemsetAsync(loss, 0, (size_t)batch * sizeof(double), s)) != cudaSuccess) return e;
-    GptqParams p{U, n_u, W, w_is_f32, d_out, d_in, bits, codes, scales, zeros, W_hat, lambda, loss, err};
-    dim3 grid(d_out / R, batch);
-    gptq_tc<<<grid, kThreads, SMEM_BYTES, s>>>(tEhi, tElo, tUhi, tUlo, tQhi, tQlo, p);
-    clha_note_launches(1);
+    if (chunked) {
+        gptq_init_wc<<<4 * num_sms, 256, 0, s>>>(W, w_is_f32, wsz, Wc);
+        clha_note_launches(1);
+    }
+    const int n_rt = (int)((size_t)batch * d_out / R);
+    for (int c0 = 0; c0 < d_in; c0 += CHUNK) {
+        const int c1 = c0 + CHUNK < d_in ? c0 + CHUNK : d_in;
+        GptqParams p{U, n_u, W, w_is_f32, Wc, c0, c1, d_out, d_in, bits, codes, scales, zeros, W_hat, lambda, loss,
+                     err};
+        gptq_tc<<<dim3(d_out / R, batch), kThreads, SMEM_BYTES, s>>>(tEhi, tElo, tUhi, tUlo, tQhi, tQlo, p);
+        clha_note_launches(1);
+        if (c1 < d_in) {   // fold this chunk's errors into the running weights of every later column
+            TrailParams tp{d_out, d_in, n_u, c0, c1, n_rt, (d_in - c1) / BLK, err};
+            const int tiles = tp.n_rt * tp.n_ct;
+            gptq_trail<<<tiles < num_sms ? tiles : num_sms, kThreads, T_SMEM_BYTES, s>>>(tEhi, tElo, tUhi, tUlo, tWc,
+                                                                                       tp);
+            clha_note_launches(1);
+        }
+    }
     return cudaGetLastError();
 }
