@@ -67,11 +67,11 @@ def objective(Q, W_src, H_src, W_m, lam):
 def epmq(W_src, H_src, W_m, bits: int, group: int = 128, damp_frac: float = 0.01):
     """E-PMQ of one merged layer: statistics, target W* = R H^-1, GPTQ of W* under H (U = the upper
     Cholesky factor of H^-1). Returns the statistics, the target, the GPTQ outputs and the objective
-    of the quantized weight."""
+    of the quantized weight (GPTQ in its lazy-batch form, with its rounding margins)."""
     H, R, lam = statistics(W_src, H_src, W_m, damp_frac)
     W_star = target(H, R)
     U = _clha.factor(H)
-    codes, scales, zeros, W_hat = _clha.gptq(W_star, U, bits, group)
+    codes, scales, zeros, W_hat, margin = _clha.gptq(W_star, U, bits, group, 128, margins=True)
     return {"H": H, "R": R, "lam": lam, "W_star": W_star, "U": U, "codes": codes, "scales": scales,
-            "zeros": zeros, "W_hat": W_hat,
+            "zeros": zeros, "W_hat": W_hat, "margin": margin,
             "objective": objective(W_hat.astype(np.float64), W_src, H_src, W_m, lam)}

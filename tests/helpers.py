@@ -21,3 +21,42 @@ def rel_fro(a, b):
 def code_agreement(a, b):
     a, b = np.asarray(a), np.asarray(b)
     return float(np.mean(a == b))
+
+
+# A code mismatch is certified as a rounding-boundary flip when, at the first place its row parts
+# ways with the oracle (the first mismatching code, or an earlier group whose zero point differs),
+# the oracle's own value was within FLIP_TOL of a step from the rounding boundary. Before that place
+# both sides made every decision alike, so their current values differ only by rounding order; a
+# value that far from a boundary cannot flip. Later mismatches in the row follow from the first (the
+# two runs then propagate different errors) and are not certified one by one.
+FLIP_TOL = 1e-3
+
+
+def certify_codes(got_codes, got_zeros, want, group=128, tol=FLIP_TOL):
+    """Agreement of one matrix's codes with the oracle's (want: a GPTQ result with "codes", "zeros"
+    and "margin") and the certification of every row that differs. Returns a dict: agree (fraction
+    of equal codes), rows (rows that differ), certified (of those, rows whose first difference is a
+    boundary flip), worst (largest margin, in steps, at a first difference)."""
+    gc, wc = np.asarray(got_codes), np.asarray(want["codes"])
+    gz, wz = np.asarray(got_zeros), np.asarray(want["zeros"])
+    mism, zmism = gc != wc, gz != wz
+    rows = np.nonzero(mism.any(1) | zmism.any(1))[0]
+    worst, certified = 0.0, 0
+    for r in rows:
+        jc = int(np.argmax(mism[r])) if mism[r].any() else None
+        jz = int(np.argmax(zmism[r])) if zmism[r].any() else None
+        if jz is not None and (jc is None or jz * group <= jc):
+            m = float(want["margin"]["zero"][r, jz])
+        else:
+            m = float(want["margin"]["code"][r, jc])
+        worst = max(worst, m)
+        certified += m <= tol
+    return {"agree": 1.0 - float(mism.mean()), "rows": len(rows), "certified": int(certified), "worst": worst}
+
+
+def assert_codes(got_codes, got_zeros, want, what, bar=0.999):
+    """The code bar: at least `bar` of the codes equal the oracle's, and every row that differs
+    starts with a certified rounding-boundary flip."""
+    c = certify_codes(got_codes, got_zeros, want)
+    assert c["agree"] >= bar and c["certified"] == c["rows"], (what, c)
+    return c
