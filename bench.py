@@ -31,8 +31,9 @@ Routing-sharpness sweep (not a throughput line; one JSON line per sharpness):
 With N > 1 (torchrun, one process per GPU) every rank calibrates its own independent weight (or
 layer pair): weak scaling, no data-path collective; the step time is the max over ranks. With
 --workload moe-e16 --parallel tokens the ranks share one layer pair instead: each collects its share
-of the tokens, one NCCL all-reduce sums the Hessian accumulators, and each quantizes its own range of
-experts (strong scaling).
+of the tokens, one NCCL reduce-scatter sums the packed upper triangles of the Hessian accumulators
+onto the rank that quantizes each expert, and each quantizes its own range of experts (strong
+scaling).
 """
 from __future__ import annotations
 
@@ -322,9 +323,9 @@ def run_ours(args, world, rank, local):
         for l in range(2):
             cal.collect(l, Xd[l], Ld[l], w)
         if sharded:
-            if world > 1:
-                with timer.span("allreduce"):
-                    SH.dist_reduce(sh.reduce_tensors())
+            if world > 1:   # packed upper triangles reduce-scattered to their owners, counts all-reduced
+                with timer.span("exchange"):
+                    SH.exchange([sh], SH.dist_reduce_scatter, SH.dist_reduce)
             sh.quantize(wq, modes)
         else:
             cal.quantize(w, modes)
@@ -480,7 +481,7 @@ def run_ours(args, world, rank, local):
             "config": {"workload": s.name, "global_batch": world * sum(s.tokens), "tokens_per_layer": s.tokens[0],
                        "E": E, "top_k": s.k, "d_model": dm, "d_ff": dff, "bits": s.bits_routed,
                        "weightings": list(modes), "columns_per_step_per_gpu": cols_per_step,
-                       "parallelism": (f"tokens{world}+experts{world} (one NCCL all-reduce of S)" if sharded
+                       "parallelism": (f"tokens{world}+experts{world} (NCCL reduce-scatter of packed S triangles to owners)" if sharded
                                        else f"replicas{world}") if world > 1 else "single",
                        "l2": "flushed (512 MB write) before every timed step"},
             "hessian_tflops": hess_tflops,
@@ -896,7 +897,7 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--parallel", choices=("replicas", "tokens"), default="replicas",
                     help="replicas (default): each rank calibrates its own layer pair (weak scaling); tokens: "
-                         "one pair, its tokens sharded over the ranks with one all-reduce of the Hessian sums, "
+                         "one pair, its tokens sharded over the ranks with one reduce-scatter of the packed Hessian sums to their owners, "
                          "its experts quantized in parallel (strong scaling)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     ap.add_argument("--workload", choices=("dense", "moe-e16", "act", "hessian", "gptq", "factor", "epmq", "dequant",

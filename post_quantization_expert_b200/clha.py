@@ -34,7 +34,7 @@ SYMBOLS = [
     "clha_aggregate", "clha_factor", "clha_factor_groups", "clha_epmq_target", "clha_quantize", "clha_loss",
     "clha_pack_codes", "clha_dequantize", "clha_dequant_matmul", "clha_routing_divergence",
     "clha_collect_gathered", "clha_expert_act_gathered", "clha_set_act_kernel", "clha_last_act_kernel",
-    "clha_set_factor_wait_limit",
+    "clha_set_factor_wait_limit", "clha_pack_upper", "clha_unpack_upper",
 ]
 FACTOR_MAX_GROUPS = 4
 
@@ -102,6 +102,8 @@ def load(path: str = LIB_PATH):
         "clha_set_act_kernel": (i32, [vp, i32]),
         "clha_last_act_kernel": (i32, [vp]),
         "clha_set_factor_wait_limit": (i32, [vp, C.c_uint64]),
+        "clha_pack_upper": (i32, [vp, vp, i64, i64, i64, i32, vp]),
+        "clha_unpack_upper": (i32, [vp, vp, i64, i64, i64, i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -349,3 +351,13 @@ def clha_loss(ctx: Context, W, W_hat, H, n_h: int, batch: int, d_out: int, d_in:
     out = np.empty(batch, np.float64)
     ctx._check(load().clha_loss(ctx.handle, _p(W), _dtype(W), _p(W_hat), _p(H), n_h, batch, d_out, d_in, _p(out)))
     return out
+
+
+def clha_pack_upper(ctx: Context, S, n_outer: int, outer_stride: int, n_inner: int, d: int, packed):
+    """Upper triangles of matrices S[(o * outer_stride + i)] (o < n_outer, i < n_inner) into packed."""
+    ctx._check(load().clha_pack_upper(ctx.handle, _p(S), n_outer, outer_stride, n_inner, d, _p(packed)))
+
+
+def clha_unpack_upper(ctx: Context, packed, n_outer: int, outer_stride: int, n_inner: int, d: int, S):
+    """The inverse of clha_pack_upper on the upper triangles (the strict lower ones are left alone)."""
+    ctx._check(load().clha_unpack_upper(ctx.handle, _p(packed), n_outer, outer_stride, n_inner, d, _p(S)))

@@ -8,9 +8,15 @@ aggregates, factors and quantizes its own contiguous range of experts (the alway
 rank 0), and the results are gathered at the end. The all-reduce is the only exchange on the data
 path; the kernels are the single-GPU ones.
 
-The reduction is left to the caller (`dist_reduce` or `simulated_reduce` on `reduce_tensors()`), so the
-same code runs with torch.distributed (NCCL between GPUs, gloo on CPU) or with the ranks simulated
-one after another in one process.
+The reduction is left to the caller, so the same code runs with torch.distributed (NCCL between
+GPUs, gloo on CPU) or with the ranks simulated one after another in one process. Two forms:
+  * all-reduce (`dist_reduce` or `simulated_reduce` on `reduce_tensors()`): every rank receives every
+    slot's full d x d sums;
+  * owner exchange (`exchange()` with `dist_reduce_scatter` or `simulated_reduce_scatter`): each rank
+    packs the upper triangles of its partial sums into one buffer laid out by owner (`ExchangeLayout`),
+    one reduce-scatter delivers to each rank the summed triangles of only the slots it quantizes, and
+    the token counts (a few integers) are all-reduced. Against the all-reduce of full matrices that
+    moves a quarter of the bytes: half for the triangles, half for reduce-scatter against all-reduce.
 """
 from __future__ import annotations
 
@@ -58,6 +64,56 @@ def simulated_reduce(per_rank: Sequence[Sequence[torch.Tensor]]):
             t.copy_(total)
 
 
+def packed_floats(d: int) -> int:
+    """Floats of one packed upper triangle (d(d+1)/2)."""
+    return d * (d + 1) // 2
+
+
+class ExchangeLayout:
+    """Which accumulator slots each rank owns, and where their packed triangles sit in the exchange
+    buffer. Rank r owns the routed experts [e0, e1) of expert_range (their input slots in `in` and
+    their down-projection slots in `dn`); rank 0 also owns the always-active experts (input slot E
+    of `in`, every slot of `sdn`). Its chunk holds, part after part, each part's matrices in (layer,
+    slot) order; every chunk is padded to the longest one, so the buffer is world * chunk floats."""
+
+    def __init__(self, E: int, world: int, n_layers: int, d_model: int, d_ff: int, n_shared: int = 0,
+                 shared_dff: int = 0):
+        self.world, self.E = world, E
+        dims = {"in": d_model, "dn": d_ff, "sdn": shared_dff}
+        self.parts = []            # per rank: [(acc, slot0, nslots, d, offset in the chunk)]
+        lens = []
+        for r in range(world):
+            e0, e1 = expert_range(E, r, world)
+            spec = [("in", e0, e1 - e0), ("dn", e0, e1 - e0)]
+            if r == 0 and n_shared:
+                spec += [("in", E, 1), ("sdn", 0, n_shared)]
+            off, parts = 0, []
+            for acc, s0, ns in spec:
+                parts.append((acc, s0, ns, dims[acc], off))
+                off += n_layers * ns * packed_floats(dims[acc])
+            self.parts.append(parts)
+            lens.append(off)
+        self.n_layers = n_layers
+        self.chunk = max(lens)
+        self.used = lens
+
+
+def dist_reduce_scatter(out: torch.Tensor, inp: torch.Tensor, group=None):
+    """Sum `inp` [world * chunk] over the ranks; this rank's chunk of the sum lands in `out`."""
+    import torch.distributed as dist
+    dist.reduce_scatter_tensor(out, inp, op=dist.ReduceOp.SUM, group=group)
+
+
+def simulated_reduce_scatter(outs: Sequence[torch.Tensor], inps: Sequence[torch.Tensor]):
+    """The same for ranks simulated in one process: out_r = sum over ranks (in rank order) of chunk r."""
+    chunk = outs[0].numel()
+    for r, out in enumerate(outs):
+        total = inps[0][r * chunk:(r + 1) * chunk].clone()
+        for inp in inps[1:]:
+            total += inp[r * chunk:(r + 1) * chunk]
+        out.copy_(total)
+
+
 class ShardedMoECalibration:
     """One rank's part of a token-sharded, expert-parallel calibration of one weight-sharing group.
 
@@ -80,9 +136,12 @@ class ShardedMoECalibration:
         self.quantizer = MoECalibration(ctx, n_layers, 1, self.e1 - self.e0, k, d_model, d_ff,
                                         self.local_shared, shared_dff, bits_routed, bits_shared, damp_frac,
                                         timer=timer, modes=modes)
+        self.exchanged = False
+        self.layout = ExchangeLayout(E, world, n_layers, d_model, d_ff, n_shared, shared_dff)
 
     def reset(self):
         self.collector.reset()
+        self.exchanged = False
 
     def collect(self, layer: int, X_shard: torch.Tensor, logits_shard: torch.Tensor, w: MoEWeights):
         self.collector.collect(layer, X_shard, logits_shard, w)
@@ -91,6 +150,48 @@ class ShardedMoECalibration:
         c = self.collector
         accs = [c.acc_in, c.acc_dn] + ([c.acc_sdn] if c.n_shared else [])
         return [t for a in accs for t in accum_tensors(a)]
+
+    def _accs(self, holder):
+        accs = {"in": holder.acc_in, "dn": holder.acc_dn}
+        if holder.n_shared:
+            accs["sdn"] = holder.acc_sdn
+        return accs
+
+    def exchange_send(self, layout: ExchangeLayout) -> torch.Tensor:
+        """This rank's send buffer [world * chunk]: for every owner rank, the packed upper triangles of
+        this rank's partial sums of the slots that rank owns (padding zero)."""
+        c = self.collector
+        accs = self._accs(c)
+        send = torch.zeros(layout.world * layout.chunk, dtype=torch.float32, device=c.dev)
+        for r, parts in enumerate(layout.parts):
+            for acc, s0, ns, d, off in parts:
+                S, _ = accs[acc].buffers()
+                if ns:
+                    base = r * layout.chunk + off
+                    L.clha_pack_upper(self.ctx, S[:, s0], S.shape[0], S.shape[1], ns, d,
+                                      send[base: base + S.shape[0] * ns * packed_floats(d)])
+        return send
+
+    def exchange_receive(self, layout: ExchangeLayout, recv: torch.Tensor):
+        """Unpack this rank's summed chunk into its quantizer's accumulators (the slots it owns, in the
+        quantizer's own slot order) and take the token counts of those slots from the collector's
+        (already summed) counts."""
+        c, q = self.collector, self.quantizer
+        qaccs, caccs = self._accs(q), self._accs(c)
+        for acc, s0, ns, d, off in layout.parts[self.rank]:
+            if not ns:
+                continue
+            Sq, cq = qaccs[acc].buffers()
+            _, cc = caccs[acc].buffers()
+            q0 = s0 - self.e0 if acc in ("in", "dn") and s0 < self.E else (Sq.shape[1] - 1 if acc == "in" else 0)
+            L.clha_unpack_upper(self.ctx, recv[off: off + Sq.shape[0] * ns * packed_floats(d)], Sq.shape[0],
+                                Sq.shape[1], ns, d, Sq[:, q0])
+            cq[:, q0:q0 + ns].copy_(cc[:, s0:s0 + ns])
+        self.exchanged = True
+
+    def count_tensors(self) -> list[torch.Tensor]:
+        """The token counts of every accumulator (all-reduced alongside the exchange: a few integers)."""
+        return [a.buffers()[1] for a in self._accs(self.collector).values()]
 
     def local_weights(self, w: MoEWeights) -> MoEWeights:
         """This rank's experts' weights, stacked (gate of e0..e1-1, then up, then down)."""
@@ -102,9 +203,14 @@ class ShardedMoECalibration:
         return out
 
     def quantize(self, w_local: MoEWeights, modes=None):
-        """After the reduction: copy this rank's summed Hessians into its own accumulators, then
-        aggregate, factor, GPTQ and score them (results in self.quantizer.res[mode])."""
+        """After the reduction: copy this rank's summed Hessians into its own accumulators (unless the
+        owner exchange already put them there), then aggregate, factor, GPTQ and score them (results
+        in self.quantizer.res[mode])."""
         c, q, e0, e1 = self.collector, self.quantizer, self.e0, self.e1
+        if self.exchanged:
+            self.exchanged = False
+            q.quantize(w_local, modes)
+            return q.res
         S, cnt = c.acc_in.buffers()
         Sq, cq = q.acc_in.buffers()
         Sq[:, : e1 - e0].copy_(S[:, e0:e1])
@@ -144,3 +250,20 @@ def gather_expert_rows(local: torch.Tensor, E_local: int, E: int, world: int, gr
         e0, e1 = expert_range(E, r, world)
         rows.append(parts[r][: e1 - e0])
     return torch.cat(rows)
+
+
+def exchange(ranks, reduce_scatter=None, all_reduce=None):
+    """The owner exchange for the given rank objects (one per process under torch.distributed, or all
+    of them when the ranks are simulated in one process): pack, reduce-scatter the triangles, all-reduce
+    the counts, unpack into each rank's quantizer."""
+    layout = ranks[0].layout
+    sends = [rk.exchange_send(layout) for rk in ranks]
+    recvs = [torch.empty(layout.chunk, dtype=torch.float32, device=s.device) for s in sends]
+    if len(ranks) == 1 and reduce_scatter is not None:
+        reduce_scatter(recvs[0], sends[0])
+        all_reduce(ranks[0].count_tensors())
+    else:
+        simulated_reduce_scatter(recvs, sends)
+        simulated_reduce([rk.count_tensors() for rk in ranks])
+    for rk, recv in zip(ranks, recvs):
+        rk.exchange_receive(layout, recv)
