@@ -353,11 +353,26 @@ def clha_loss(ctx: Context, W, W_hat, H, n_h: int, batch: int, d_out: int, d_in:
     return out
 
 
-def clha_pack_upper(ctx: Context, S, n_outer: int, outer_stride: int, n_inner: int, d: int, packed):
-    """Upper triangles of matrices S[(o * outer_stride + i)] (o < n_outer, i < n_inner) into packed."""
-    ctx._check(load().clha_pack_upper(ctx.handle, _p(S), n_outer, outer_stride, n_inner, d, _p(packed)))
+def _mat_ptr(S, first: int, n_outer: int, outer_stride: int, n_inner: int, d: int):
+    """Address of matrix `first` of a contiguous stack of d x d float32 matrices, after checking that the
+    strided batch (o * outer_stride + i, o < n_outer, i < n_inner, from `first`) stays inside it."""
+    ptr = _p(S)
+    if S.dtype != torch.float32 or S.numel() % (d * d):
+        raise ValueError("expected a stack of d x d float32 matrices")
+    last = first + (n_outer - 1) * outer_stride + n_inner if n_outer * n_inner else first
+    if first < 0 or last * d * d > S.numel():
+        raise ValueError("matrix batch outside the tensor")
+    return ptr + first * d * d * 4 if ptr else ptr
 
 
-def clha_unpack_upper(ctx: Context, packed, n_outer: int, outer_stride: int, n_inner: int, d: int, S):
+def clha_pack_upper(ctx: Context, S, n_outer: int, outer_stride: int, n_inner: int, d: int, packed, first: int = 0):
+    """Upper triangles of matrices first + o * outer_stride + i (o < n_outer, i < n_inner) of the
+    contiguous stack S (e.g. an accumulator's S viewed as [layers * slots, d, d]) into packed."""
+    ctx._check(load().clha_pack_upper(ctx.handle, _mat_ptr(S, first, n_outer, outer_stride, n_inner, d), n_outer,
+                                      outer_stride, n_inner, d, _p(packed)))
+
+
+def clha_unpack_upper(ctx: Context, packed, n_outer: int, outer_stride: int, n_inner: int, d: int, S, first: int = 0):
     """The inverse of clha_pack_upper on the upper triangles (the strict lower ones are left alone)."""
-    ctx._check(load().clha_unpack_upper(ctx.handle, _p(packed), n_outer, outer_stride, n_inner, d, _p(S)))
+    ctx._check(load().clha_unpack_upper(ctx.handle, _p(packed), n_outer, outer_stride, n_inner, d,
+                                        _mat_ptr(S, first, n_outer, outer_stride, n_inner, d)))

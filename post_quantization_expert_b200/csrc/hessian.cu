@@ -7,14 +7,14 @@
 //              (128-byte swizzle; both operands are "M/N-major": one token row = 64 contiguous
 //              channels, which is how X is laid out, so no transpose is ever materialised).
 //   warp 1     MMA issuer: tcgen05.mma kind::f16 M=128 N=256 K=16, four per 64-token block,
-//              accumulating in TMEM one chunk of at most KCHUNK tokens at a time; two accumulators
+//              accumulating in TMEM one chunk of at most 2048 (d < 8192) or 8192 tokens at a time; two accumulators
 //              (512 TMEM columns) so the epilogue of one chunk overlaps the MMAs of the next.
 //   warps 2-5  epilogue: tcgen05.ld of the fp32 chunk sum, one 32x32 sub-tile per warp at a time
 //              written to a swizzled shared-memory buffer (two per warp) and added into S by a TMA
 //              bulk reduce (the L2 performs the fp32 adds), so the epilogue never reads S.
 // Why chunks: the tensor core's fp32 accumulation does not round to nearest, and over tens of
 // thousands of tokens the Gram diagonal (a sum of positive terms) drifts low by a few 1e-4
-// relative. Summing at most KCHUNK tokens per accumulator and adding the chunk sums into S with
+// relative. Summing at most one chunk of tokens per accumulator and adding the chunk sums into S with
 // round-to-nearest fp32 adds bounds that drift by the chunk length instead of the token count.
 // Only tiles that touch the upper triangle are computed (rows tile r <= 2c+1 for column tile c);
 // entries below the diagonal inside those tiles are correct values but the upper triangle is the
@@ -28,10 +28,14 @@
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-#ifndef CLHA_SYRK_KCHUNK_BLOCKS
-#define CLHA_SYRK_KCHUNK_BLOCKS 128
-#endif
-constexpr int KCHUNK_BLOCKS = CLHA_SYRK_KCHUNK_BLOCKS;  // 64-token blocks per TMEM accumulation
+// 64-token blocks per TMEM accumulation. The tensor core's fp32 accumulator does not round each add
+// to nearest, so a long sum drifts (linearly in its length); chunk sums are added into S by TMA
+// reduce-add, which rounds to nearest. Short chunks where the Hessian is small (an expert's d_model or
+// d_ff: cheap extra epilogues, and the experts' Hessians feed GPTQ on rank-deficient, ill-conditioned
+// problems), long ones for large d (each chunk's epilogue moves a whole 128x256 fp32 tile).
+constexpr int KCHUNK_BLOCKS_SMALL_D = 32;     // 2048 tokens, d < 8192
+constexpr int KCHUNK_BLOCKS_LARGE_D = 128;    // 8192 tokens, d >= 8192
+__host__ __device__ constexpr int kchunk_blocks(int d) { return d < 8192 ? KCHUNK_BLOCKS_SMALL_D : KCHUNK_BLOCKS_LARGE_D; }
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -197,8 +201,8 @@ __global__ void __launch_bounds__(kThreads, 1) syrk_bf16_tc(const __grid_constan
                 int64_t t0, cnt;
                 slot_range(p, e, t0, cnt);
                 const int nk = (int)((cnt + BK - 1) / BK);
-                for (int kc = 0; kc < nk && ok; kc += KCHUNK_BLOCKS) {
-                    const int kend = min(nk, kc + KCHUNK_BLOCKS);
+                for (int kc = 0; kc < nk && ok; kc += kchunk_blocks(p.d)) {
+                    const int kend = min(nk, kc + kchunk_blocks(p.d));
                     const int acc = tcount & 1;
                     const uint32_t aph = (tcount >> 1) & 1;
                     if (!tc::mbar_wait_bounded(tempty0 + 8 * acc, aph ^ 1, abort_flag)) { ok = false; break; }
@@ -241,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1) syrk_bf16_tc(const __grid_constan
             const int warp_row_min = r * BM + q * 32;
             const int srow = e * p.d + warp_row_min;  // row of this warp's sub-tiles in the [E*d, d] view
             bool ok = true;
-            for (int kc = 0; kc < nk; kc += KCHUNK_BLOCKS) {
+            for (int kc = 0; kc < nk; kc += kchunk_blocks(p.d)) {
                 const int acc = tcount & 1;
                 const uint32_t aph = (tcount >> 1) & 1;
                 if (!tc::mbar_wait_bounded(tfull0 + 8 * acc, aph, abort_flag)) { ok = false; break; }

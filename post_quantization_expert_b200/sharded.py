@@ -168,8 +168,8 @@ class ShardedMoECalibration:
                 S, _ = accs[acc].buffers()
                 if ns:
                     base = r * layout.chunk + off
-                    L.clha_pack_upper(self.ctx, S[:, s0], S.shape[0], S.shape[1], ns, d,
-                                      send[base: base + S.shape[0] * ns * packed_floats(d)])
+                    L.clha_pack_upper(self.ctx, S, S.shape[0], S.shape[1], ns, d,
+                                      send[base: base + S.shape[0] * ns * packed_floats(d)], first=s0)
         return send
 
     def exchange_receive(self, layout: ExchangeLayout, recv: torch.Tensor):
@@ -183,9 +183,14 @@ class ShardedMoECalibration:
                 continue
             Sq, cq = qaccs[acc].buffers()
             _, cc = caccs[acc].buffers()
-            q0 = s0 - self.e0 if acc in ("in", "dn") and s0 < self.E else (Sq.shape[1] - 1 if acc == "in" else 0)
+            if acc == "sdn":
+                q0 = 0                       # the always-active experts' down-projection slots
+            elif s0 == self.E:
+                q0 = Sq.shape[1] - 1         # the always-active experts' shared input slot (last)
+            else:
+                q0 = s0 - self.e0            # this rank's routed experts, from its slot 0
             L.clha_unpack_upper(self.ctx, recv[off: off + Sq.shape[0] * ns * packed_floats(d)], Sq.shape[0],
-                                Sq.shape[1], ns, d, Sq[:, q0])
+                                Sq.shape[1], ns, d, Sq, first=q0)
             cq[:, q0:q0 + ns].copy_(cc[:, s0:s0 + ns])
         self.exchanged = True
 

@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import oracle as O
-from helpers import assert_codes, rel_fro, sym_from_upper, to64
+from helpers import CONFIG_BAR, assert_codes, rel_fro, sym_from_upper, to64
 from post_quantization_expert_b200 import clha as L
 
 pytestmark = pytest.mark.gpu
@@ -456,7 +456,7 @@ def test_quantize_matches_oracle_on_same_factor(ctx, d_out, d_in, bits, wdt):
     L.clha_quantize(ctx, Ud, 1, Wd, 1, d_out, d_in, bits, codes, scales, zeros, W_hat, lam=lam, loss=loss)
     wc, ws, wz, wh, wm = O.gptq(to64(W), U32.astype(np.float64), bits, 128, margins=True)
     assert_codes(codes[0].cpu().numpy(), zeros[0].cpu().numpy(), dict(codes=wc, zeros=wz, margin=wm),
-                 (d_out, d_in, bits))
+                 (d_out, d_in, bits), bar=CONFIG_BAR)
     # first group of every row: identical inputs, so the grid is bit-identical
     np.testing.assert_array_equal(scales[0, :, 0].cpu().numpy(), ws[:, 0])
     np.testing.assert_array_equal(zeros[0, :, 0].cpu().numpy(), wz[:, 0])
@@ -500,7 +500,8 @@ def test_quantize_batched_shared_factor(ctx):
     L.clha_quantize(ctx, Ud, 2, W.to(DEV), 4, d_out, d_in, bits, codes, scales, zeros, None)
     for b in range(4):
         wc, _, wz, _, wm = O.gptq(to64(W[b]), Us[b % 2].astype(np.float64), bits, 128, margins=True)
-        assert_codes(codes[b].cpu().numpy(), zeros[b].cpu().numpy(), dict(codes=wc, zeros=wz, margin=wm), b)
+        assert_codes(codes[b].cpu().numpy(), zeros[b].cpu().numpy(), dict(codes=wc, zeros=wz, margin=wm), b,
+                     bar=CONFIG_BAR)
 
 
 # ------------------------------------------------------------------------------------ loss

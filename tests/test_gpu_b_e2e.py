@@ -1,13 +1,14 @@
 """End-to-end parity of the GPU calibration path with the float64 oracle on the seeded workloads:
 routing counts bit-exact, Hessians within 1e-4 relative Frobenius error, codes agreeing on >= 99.9%
-of entries, per-expert reconstruction loss within 1e-3 relative. Where the oracle cannot afford a
-whole workload, it checks every Hessian and a sample of experts' GPTQ end to end."""
+of entries with every differing row starting at a certified rounding-boundary flip, per-expert
+reconstruction loss within 1e-3 relative. Where the oracle cannot afford a whole workload, it checks
+every Hessian and a sample of experts' GPTQ end to end."""
 import numpy as np
 import pytest
 import torch
 
 import oracle as O
-from helpers import code_agreement, rel_fro, sym_from_upper, to64
+from helpers import CONFIG_BAR, CodeTally, assert_codes, rel_fro, sym_from_upper, to64
 from post_quantization_expert_b200 import clha as L
 from post_quantization_expert_b200.pipeline import DenseCalibration, MoECalibration, stack_weights
 from synth import workload
@@ -41,7 +42,8 @@ def test_dense_two_layer_fp32_workload(ctx):
     np.testing.assert_allclose(lam[0], want["lam"], rtol=1e-5)
     assert rel_fro(cal.H_comb[0].double().cpu().numpy(), want["H_comb"]) < 1e-4
     assert rel_fro(cal.U[0].double().cpu().numpy(), want["U"]) < 1e-4
-    assert code_agreement(cal.q.codes[0].cpu().numpy(), want["codes"]) >= 0.999
+    print("dense c1 codes", assert_codes(cal.q.codes[0].cpu().numpy(), cal.q.zeros[0].cpu().numpy(), want, "dense",
+                                         bar=CONFIG_BAR))
     assert abs(cal.q.loss[0] - want["loss"]) <= 1e-3 * want["loss"]
 
 
@@ -79,6 +81,7 @@ def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, fused=False
             assert rel_fro(sym_from_upper(S_in[l, s.E].double().cpu().numpy()), O.gram(X64[l])) < 1e-4
     # sampled experts: down-projection Hessians and the whole GPTQ path, per weighting
     ref = {}
+    tally = CodeTally((cfg, over.get("tokens")))
     cal.quantize(w, modes)           # every weighting in one pass (batched factorisation)
     torch.cuda.synchronize()
     for mode in modes:
@@ -96,11 +99,11 @@ def _moe_pair(ctx, cfg, experts_checked, modes, shared_checked=None, fused=False
             else:
                 qs = {"gate": out.sg, "up": out.su, "down": out.sd}
             for name, q in qs.items():
-                agree = code_agreement(q.codes[e].cpu().numpy(), r[name]["codes"])
-                assert agree >= 0.999, (mode, key, name, agree)
+                tally.add(q.codes[e].cpu().numpy(), q.zeros[e].cpu().numpy(), r[name], (mode, key, name))
             got_loss = sum(qs[n].loss[e] for n in ("gate", "up", "down"))
             assert abs(got_loss - r["loss"]) <= 1e-3 * r["loss"], (mode, key, got_loss, r["loss"])
         ref[mode] = res
+    tally.check()
     return cal, ref
 
 
@@ -143,16 +146,17 @@ def test_unrouted_experts_are_round_to_nearest(ctx):
     assert cnt[0, 3] == 0 and cnt[1, 3] == 0 and cnt[0, 5] == 0 and cnt[1, 5] > 0
     X64 = [to64(X) for X in Xs]
     W64 = [tuple(to64(t) for t in r) for r in routed]
-    # (expert 0 is checked under rt only: alone, layer 0 gives it ~128 tokens in 1024 dimensions, a
-    # Hessian so ill-conditioned that float32 GPTQ and the float64 oracle part ways on ~0.1 % of codes)
-    for mode, alpha, experts in (("rt", None, (3, 0)), ("explicit", (1.0, 0.0), (3, 5))):
+    # expert 0 under alpha = (1, 0) sees only layer 0's ~128 tokens in 1024 dimensions: a Hessian
+    # that is rank-deficient up to the damping, the hardest case for the code bar
+    tally = CodeTally("unrouted")
+    for mode, alpha, experts in (("rt", None, (3, 0)), ("explicit", (1.0, 0.0), (3, 5, 0))):
         ref = O.calibrate_moe_group(X64, [lg.numpy() for lg in lgs], s.k, W64, (), list(experts), s.bits_routed,
                                     s.bits_shared, s.group, mode, s.damp_frac, alpha=alpha, empty="identity")
         r = cal.res[mode]
         for e in experts:
             want = ref["experts"][("r", e)]
             for name, q in (("gate", r.qg), ("up", r.qu), ("down", r.qd)):
-                assert code_agreement(q.codes[e].cpu().numpy(), want[name]["codes"]) >= 0.999, (mode, e, name)
+                tally.add(q.codes[e].cpu().numpy(), q.zeros[e].cpu().numpy(), want[name], (mode, e, name))
             got = r.expert_loss()[e]
             if e == 0:
                 assert abs(got - want["loss"]) <= 1e-3 * want["loss"]
@@ -162,3 +166,4 @@ def test_unrouted_experts_are_round_to_nearest(ctx):
                 err2 = sum(float(((q.W_hat[e].double() - Wm.double().to(DEV)) ** 2).sum())
                            for q, Wm in ((r.qg, routed[e][0]), (r.qu, routed[e][1]), (r.qd, routed[e][2])))
                 assert want["loss"] == 0.0 and abs(got) <= 1e-5 * err2, (mode, e, got, err2)
+    tally.check()

@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_codes, rel_fro, to64
+from helpers import CONFIG_BAR, assert_codes, rel_fro, to64
 from oracle import epmq_oracle as EP
 from post_quantization_expert_b200 import clha as L
 from post_quantization_expert_b200.pipeline import EPMQCalibration
@@ -41,7 +41,7 @@ def test_sum_aggregate_and_target_match_oracle(ctx, K, d_out, d, wdt):
     # float64 products of float32 factor entries: the rounding of U (2^-24) grows with cond(H)
     assert rel_fro(cal.W_target.double().cpu().numpy(), W_star) < 1e-5
     o = EP.epmq([to64(w) for w in W_src], S64, to64(W_m), bits=3)
-    assert_codes(cal.q.codes[0].cpu().numpy(), cal.q.zeros[0].cpu().numpy(), o, "epmq from Grams")
+    assert_codes(cal.q.codes[0].cpu().numpy(), cal.q.zeros[0].cpu().numpy(), o, "epmq from Grams", bar=CONFIG_BAR)
 
 
 def test_epmq_end_to_end_from_activations(ctx):
@@ -55,7 +55,7 @@ def test_epmq_end_to_end_from_activations(ctx):
     H_src = [to64(x).T @ to64(x) for x in X]
     o = EP.epmq([to64(w) for w in W_src], H_src, to64(W_m), bits=3)
     assert rel_fro(cal.W_target.double().cpu().numpy(), o["W_star"]) < 1e-4   # phase-1 Grams within 1e-4
-    assert_codes(q.codes[0].cpu().numpy(), q.zeros[0].cpu().numpy(), o, "epmq from activations")
+    assert_codes(q.codes[0].cpu().numpy(), q.zeros[0].cpu().numpy(), o, "epmq from activations", bar=CONFIG_BAR)
     got = EP.objective(q.W_hat[0].double().cpu().numpy(), [to64(w) for w in W_src], H_src, to64(W_m), o["lam"])
     assert abs(got - o["objective"]) <= 1e-3 * o["objective"]
     # and the quantized weight is closer to the experts' outputs than GPTQ of the merged weight alone
