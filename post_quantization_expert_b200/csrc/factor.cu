@@ -135,14 +135,18 @@ __device__ __forceinline__ void tile_to_smem(Tile* dst, const double* __restrict
     }
 }
 
-// C (global tile, row-major 64x64) <- (load_c ? C : 0) + sign * P Q^T. The operand copies into shared
-// memory and the loads of this thread's C fragments are all in flight together. A negative sign is
-// applied to C on the way in and out (C - PQ^T = -(-C + PQ^T)), not to every operand fragment. Each
-// 16-byte shared load feeds two k-steps: in the k-block k0..k0+7 lane tq supplies k0+2tq to the
-// first m8n8k4 product and k0+2tq+1 to the second (the same k for its A and B fragments), so the
-// two products together cover the block.
+// C (global tile, row-major 64x64) <- (load_c ? C : 0) + sign * (P1 Q1^T [+ P2 Q2^T]): one or two
+// operand pairs (a two-level task applies two panels' updates to its output tile with one read and
+// one write of C). The first pair's copies into shared memory and the loads of this thread's C
+// fragments are in flight together; a second pair is copied after every warp has finished with the
+// first. A negative sign is applied to C on the way in and out (C - PQ^T = -(-C + PQ^T)), not to every
+// operand fragment. Each 16-byte shared load feeds two k-steps: in the k-block k0..k0+7 lane tq
+// supplies k0+2tq to the first m8n8k4 product and k0+2tq+1 to the second (the same k for its A and B
+// fragments), so the two products together cover the block.
 __device__ __forceinline__ void tile_gemm_nt(const double* __restrict__ Pg, const double* __restrict__ Qg, Tile* Ps,
-                                             Tile* Qs, double* C, bool load_c, bool negate) {
+                                             Tile* Qs, double* C, bool load_c, bool negate,
+                                             const double* __restrict__ Pg2 = nullptr,
+                                             const double* __restrict__ Qg2 = nullptr) {
     tile_to_smem(Ps, Pg);
     tile_to_smem(Qs, Qg);
     asm volatile("cp.async.commit_group;" ::: "memory");
@@ -163,23 +167,35 @@ __device__ __forceinline__ void tile_gemm_nt(const double* __restrict__ Pg, cons
                 c[mi][ni][0] = c[mi][ni][1] = 0.0;
             }
         }
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    cbar();
+    const int npairs = Pg2 ? 2 : 1;
+#pragma unroll 1
+    for (int pr = 0; pr < npairs; ++pr) {
+        if (pr == 1) {           // every warp is done with the first pair's tiles
+            cbar();
+            tile_to_smem(Ps, Pg2);
+            tile_to_smem(Qs, Qg2);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        cbar();
 #pragma unroll 2
-    for (int k0 = 0; k0 < NB; k0 += 8) {
-        double2 a[4], bq[2];
+        for (int k0 = 0; k0 < NB; k0 += 8) {
+            double2 a[4], bq[2];
 #pragma unroll
-        for (int mi = 0; mi < 4; ++mi) a[mi] = *reinterpret_cast<const double2*>(&Ps[32 * wm + 8 * mi + g][k0 + 2 * tq]);
+            for (int mi = 0; mi < 4; ++mi)
+                a[mi] = *reinterpret_cast<const double2*>(&Ps[32 * wm + 8 * mi + g][k0 + 2 * tq]);
 #pragma unroll
-        for (int ni = 0; ni < 2; ++ni) bq[ni] = *reinterpret_cast<const double2*>(&Qs[16 * wn + 8 * ni + g][k0 + 2 * tq]);
+            for (int ni = 0; ni < 2; ++ni)
+                bq[ni] = *reinterpret_cast<const double2*>(&Qs[16 * wn + 8 * ni + g][k0 + 2 * tq]);
 #pragma unroll
-        for (int mi = 0; mi < 4; ++mi)
+            for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
-            for (int ni = 0; ni < 2; ++ni) dmma(c[mi][ni][0], c[mi][ni][1], a[mi].x, bq[ni].x);
+                for (int ni = 0; ni < 2; ++ni) dmma(c[mi][ni][0], c[mi][ni][1], a[mi].x, bq[ni].x);
 #pragma unroll
-        for (int mi = 0; mi < 4; ++mi)
+            for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
-            for (int ni = 0; ni < 2; ++ni) dmma(c[mi][ni][0], c[mi][ni][1], a[mi].y, bq[ni].y);
+                for (int ni = 0; ni < 2; ++ni) dmma(c[mi][ni][0], c[mi][ni][1], a[mi].y, bq[ni].y);
+        }
     }
 #pragma unroll
     for (int mi = 0; mi < 4; ++mi)
@@ -426,31 +442,54 @@ __device__ bool wait_ge(const int* p, int target, const Dag& g, int problem) {
 }
 
 // Tasks per problem in stage s, by class. Stage 0 holds P(0) and S(i,0); stage s >= 1 (m = s - 1)
-// holds the next panel's updates G(i,m+1,m), then P(m+1), the bulk of level m (F(j,m), Q(j,i,m),
-// the remaining G(i,j,m)) and last S(i,m+1): the Cholesky of panel m+1 overlaps level m's bulk
-// (lookahead of one panel) and the S tasks, which wait for it, come after that bulk.
-__device__ __forceinline__ void stage_counts(int nt, int s, long long (&n)[6]) {
+// holds, in this order:
+//   0  G(i,m+1,m)          the next panel's update (lookahead): P(m+1) can start once it is done
+//   1  P(m+1)
+//   2  F(j,m)              j < m
+//   3  Q(j,i,m)            one level: for even m every j <= m with i = m+1, m+2; for odd m every
+//                          j <= m with i = m+1, and j = m with i >= m+2
+//   4  FQ(j,i,{m-1,m})     odd m, j <= m-1, i >= m+2: the terms of levels m-1 and m in one task
+//   5  even m: G(i,m+2,m)  the column after the lookahead, one level;
+//      odd m: FG(i,j,{m-1,m}) for m+2 <= j <= i: levels m-1 and m in one task
+//   6  S(i,m+1)
+// Levels pair up (even m, m+1): an even level updates only the two columns after its panel and
+// leaves the rest of its trailing matrix (and of its inverse terms) to the next, odd level, whose
+// bulk tasks apply both. A bulk task then reads and writes its output tile once per two panels and
+// pays its scheduling once, and the lookahead chain P(m) -> S(m+1,m) -> G(m+1,m+1,m) -> P(m+1) keeps
+// its one-level tasks. Every task waits only on tasks with smaller numbers (a CPU model of this
+// numbering checks that, and that each update is applied once, for every tile count up to 39).
+__host__ __device__ __forceinline__ void stage_counts(int nt, int s, long long (&n)[7]) {
+    for (int c = 0; c < 7; ++c) n[c] = 0;
     if (s == 0) {
-        n[0] = 0; n[1] = 1; n[2] = 0; n[3] = 0; n[4] = 0; n[5] = nt - 1;
+        n[1] = 1;
+        n[6] = nt - 1;
         return;
     }
     const int m = s - 1;
     const long long R = nt - 1 - m;
+    if (R < 0) return;
+    const long long R1 = R >= 1 ? R - 1 : 0;
     n[0] = R;
     n[1] = R >= 1 ? 1 : 0;
     n[2] = m;
-    n[3] = (long long)(m + 1) * R;
-    n[4] = R >= 1 ? (R - 1) * R / 2 : 0;
-    n[5] = R >= 1 ? R - 1 : 0;
+    if ((m & 1) == 0) {
+        n[3] = (long long)(m + 1) * (R < 2 ? R : 2);
+        n[5] = R1;
+    } else {
+        n[3] = (long long)(m + 1) * (R < 1 ? R : 1) + R1;
+        n[4] = (long long)m * R1;
+        n[5] = R >= 1 ? (R - 1) * R / 2 : 0;
+    }
+    n[6] = R1;
 }
-__device__ __forceinline__ unsigned long long stage_total(int nt, int s) {
+__host__ __device__ __forceinline__ unsigned long long stage_total(int nt, int s) {
     if (s > nt) return 0;
-    long long n[6];
+    long long n[7];
     stage_counts(nt, s, n);
-    return (unsigned long long)(n[0] + n[1] + n[2] + n[3] + n[4] + n[5]);
+    return (unsigned long long)(n[0] + n[1] + n[2] + n[3] + n[4] + n[5] + n[6]);
 }
 
-// A decoded task: class q (0 P, 1 S, 2/5 G, 3 F, 4 Q), group k, problem b of the group, level m,
+// A decoded task: class q (0 P, 1 S, 2/5 G, 3 F, 4 Q, 6 FG, 7 FQ), group k, problem b of the group, level m,
 // tiles i, j; its inputs' states to wait for; its outputs' states once done.
 struct Task {
     int q, k, b, m, i, j;
@@ -490,29 +529,49 @@ __device__ __forceinline__ void decode_task(const Dag& g, const unsigned long lo
     const Grp& G = g.grp[k];
     const int nt = G.nt;
     const uint32_t batch = (uint32_t)G.batch;
-    long long n[6];
+    long long n[7];
     stage_counts(nt, sg, n);
     int c = 0;
 #pragma unroll
-    for (int cq = 0; cq < 6; ++cq)
+    for (int cq = 0; cq < 7; ++cq)
         if (c == cq && r >= (uint32_t)n[cq] * batch) { r -= (uint32_t)n[cq] * batch; ++c; }
     const uint32_t local = r / batch;
     const int b = (int)(r - local * batch);
     int q, m = sg - 1, i = 0, j = 0;
+    const bool odd = (m & 1) != 0;
     if (c == 0) { q = 2; i = m + 1 + (int)local; j = m + 1; }
     else if (c == 1) { q = 0; m = sg; }
     else if (c == 2) { q = 3; j = (int)local; }
     else if (c == 3) {
         q = 4;
-        const uint32_t ii = local / (uint32_t)(m + 1);
-        i = m + 1 + (int)ii;
-        j = (int)(local - ii * (uint32_t)(m + 1));
+        if (!odd) {
+            const uint32_t ii = local / (uint32_t)(m + 1);
+            i = m + 1 + (int)ii;
+            j = (int)(local - ii * (uint32_t)(m + 1));
+        } else if (local < (uint32_t)(m + 1)) {
+            i = m + 1;
+            j = (int)local;
+        } else {
+            i = m + 2 + (int)(local - (uint32_t)(m + 1));
+            j = m;
+        }
     } else if (c == 4) {
-        q = 5;
-        int rem = (int)local;
-        j = m + 2;
-        while (rem >= nt - j) { rem -= nt - j; ++j; }
-        i = j + rem;
+        q = 7;
+        const uint32_t ii = local / (uint32_t)m;
+        i = m + 2 + (int)ii;
+        j = (int)(local - ii * (uint32_t)m);
+    } else if (c == 5) {
+        if (!odd) {
+            q = 5;
+            i = m + 2 + (int)local;
+            j = m + 2;
+        } else {
+            q = 6;
+            int rem = (int)local;
+            j = m + 2;
+            while (rem >= nt - j) { rem -= nt - j; ++j; }
+            i = j + rem;
+        }
     } else { q = 1; m = sg; i = m + 1 + (int)local; j = m; }
     d.q = q; d.k = k; d.b = b; d.m = m; d.i = i; d.j = j;
     dp.wp[0] = dp.wp[1] = dp.wp[2] = nullptr;
@@ -526,19 +585,21 @@ __device__ __forceinline__ void decode_task(const Dag& g, const unsigned long lo
         dp.wp[0] = st(G.stA, G, b, i, m); dp.wt[0] = m;
         dp.wp[1] = st(G.stA, G, b, m, m); dp.wt[1] = m + 1;
         dp.out = st(G.stA, G, b, i, m); dp.out_value = m + 1;
-    } else if (q == 2 || q == 5) {   // A_ij -= L_im L_jm^T
+    } else if (q == 2 || q == 5 || q == 6) {   // A_ij -= L_im L_jm^T (FG: and level m-1's term)
+        // L_im final implies L_{i,m-1} final (S(i,m) waited for every update of A_im)
         dp.wp[0] = st(G.stA, G, b, i, m); dp.wt[0] = m + 1;
         dp.wp[1] = st(G.stA, G, b, j, m); dp.wt[1] = m + 1;
-        dp.wp[2] = st(G.stA, G, b, i, j); dp.wt[2] = m;
+        dp.wp[2] = st(G.stA, G, b, i, j); dp.wt[2] = q == 6 ? m - 1 : m;
         dp.out = st(G.stA, G, b, i, j); dp.out_value = m + 1;
     } else if (q == 3) {     // Y_jm = -R_jm D_m^T
         dp.wp[0] = st(G.stY, G, b, j, m); dp.wt[0] = m - j;
         dp.wp[1] = st(G.stA, G, b, m, m); dp.wt[1] = m + 1;
         dp.out = st(G.stY, G, b, j, m); dp.out_value = m - j + 1;
-    } else {                 // R_ji (+)= Y_jm L_im^T
+    } else {                 // R_ji (+)= Y_jm L_im^T (FQ: and level m-1's term)
+        // Y_jm final implies Y_{j,m-1} final (F(j,m) waited for every term of R_jm)
         dp.wp[0] = st(G.stY, G, b, j, m); dp.wt[0] = m - j + 1;
         dp.wp[1] = st(G.stA, G, b, i, m); dp.wt[1] = m + 1;
-        dp.wp[2] = st(G.stY, G, b, j, i); dp.wt[2] = m - j;
+        dp.wp[2] = st(G.stY, G, b, j, i); dp.wt[2] = q == 7 ? m - 1 - j : m - j;
         dp.out = st(G.stY, G, b, j, i); dp.out_value = m - j + 1;
     }
 }
@@ -589,17 +650,22 @@ __global__ void __launch_bounds__(DAG_THREADS, 2) fac_dag(Dag g) {
             int wtl = 0;
             if (t < g.total && !*reinterpret_cast<volatile int*>(g.abort_flag)) {
                 decode_task(g, lvl, t, d, dp);
-                if (lane < 3) {   // the task's tiles into L2 while the compute warps run the current one
+                if (lane < 5) {   // the task's tiles into L2 while the compute warps run the current one
                     const Grp& G = g.grp[d.k];
                     const double* Dm = G.D + ((size_t)d.b * G.nt + d.m) * TILE_ELEMS;
                     const double* pt = nullptr;
+                    // lanes 3, 4: the earlier level's operands of a two-level task
+                    const int ml = lane >= 3 ? d.m - 1 : d.m;
                     if (d.q == 0) pt = lane == 0 ? tile(G.A, G, d.b, d.m, d.m) : nullptr;
                     else if (d.q == 1) pt = lane == 0 ? tile(G.A, G, d.b, d.i, d.m) : lane == 1 ? Dm : nullptr;
-                    else if (d.q == 2 || d.q == 5)
-                        pt = tile(G.A, G, d.b, lane == 2 ? d.i : lane == 1 ? d.j : d.i, lane == 2 ? d.j : d.m);
-                    else if (d.q == 3) pt = lane == 0 ? tile(G.Y, G, d.b, d.j, d.m) : lane == 1 ? Dm : nullptr;
-                    else pt = lane == 0 ? tile(G.Y, G, d.b, d.j, d.m) : lane == 1 ? tile(G.A, G, d.b, d.i, d.m)
-                                                                     : tile(G.Y, G, d.b, d.j, d.i);
+                    else if (d.q == 2 || d.q == 5 || d.q == 6) {
+                        if (lane < 3 || d.q == 6)
+                            pt = tile(G.A, G, d.b, lane == 2 ? d.i : (lane == 1 || lane == 4) ? d.j : d.i,
+                                      lane == 2 ? d.j : ml);
+                    } else if (d.q == 3) pt = lane == 0 ? tile(G.Y, G, d.b, d.j, d.m) : lane == 1 ? Dm : nullptr;
+                    else if (lane < 3 || d.q == 7)
+                        pt = (lane == 0 || lane == 3) ? tile(G.Y, G, d.b, d.j, ml)
+                             : (lane == 1 || lane == 4) ? tile(G.A, G, d.b, d.i, ml) : tile(G.Y, G, d.b, d.j, d.i);
                     if (pt) prefetch_l2(pt, TILE_ELEMS * sizeof(double));
                 }
                 if (lane < 3) {   // (selects, not an indexed local array)
@@ -658,8 +724,14 @@ __global__ void __launch_bounds__(DAG_THREADS, 2) fac_dag(Dag g) {
             tile_gemm_nt(tile(G.A, G, b, i, m), Dm, T0, T1, tile(G.A, G, b, i, m), false, false);
         } else if (q == 2 || q == 5) {   // A_ij -= L_im L_jm^T
             tile_gemm_nt(tile(G.A, G, b, i, m), tile(G.A, G, b, j, m), T0, T1, tile(G.A, G, b, i, j), true, true);
+        } else if (q == 6) {     // A_ij -= L_{i,m-1} L_{j,m-1}^T + L_im L_jm^T
+            tile_gemm_nt(tile(G.A, G, b, i, m - 1), tile(G.A, G, b, j, m - 1), T0, T1, tile(G.A, G, b, i, j), true,
+                         true, tile(G.A, G, b, i, m), tile(G.A, G, b, j, m));
         } else if (q == 3) {     // Y_jm = -R_jm D_m^T
             tile_gemm_nt(tile(G.Y, G, b, j, m), Dm, T0, T1, tile(G.Y, G, b, j, m), false, true);
+        } else if (q == 7) {     // R_ji (+)= Y_{j,m-1} L_{i,m-1}^T + Y_jm L_im^T (level j's term starts R_ji)
+            tile_gemm_nt(tile(G.Y, G, b, j, m - 1), tile(G.A, G, b, i, m - 1), T0, T1, tile(G.Y, G, b, j, i),
+                         m - 1 != j, false, tile(G.Y, G, b, j, m), tile(G.A, G, b, i, m));
         } else {                 // R_ji (+)= Y_jm L_im^T
             tile_gemm_nt(tile(G.Y, G, b, j, m), tile(G.A, G, b, i, m), T0, T1, tile(G.Y, G, b, j, i), m != j, false);
         }
@@ -734,10 +806,7 @@ cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups
         G.stY = st_cur + tiles;
         st_cur += 2 * tiles;
         unsigned long long per = 0;
-        for (int m = 0; m < G.nt; ++m) {
-            const long long R = G.nt - 1 - m;
-            per += 1 + 2 * R + m + (m + 1) * R + (R >= 1 ? (R - 1) * R / 2 : 0);
-        }
+        for (int st = 0; st <= G.nt; ++st) per += stage_total(G.nt, st);
         g.total += per * (unsigned long long)G.batch;
     }
 
@@ -747,13 +816,7 @@ cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups
         for (int k = 0; k < n; ++k) {
             const int nt = g.grp[k].nt;
             if (st > nt) continue;
-            unsigned long long per;
-            if (st == 0) per = (unsigned long long)nt;
-            else {
-                const long long m = st - 1, R = nt - 1 - m;
-                per = R + (R >= 1 ? 1 : 0) + m + (m + 1) * R + (R >= 1 ? (R - 1) * R / 2 + R - 1 : 0);
-            }
-            tasks += per * (unsigned long long)g.grp[k].batch;
+            tasks += stage_total(nt, st) * (unsigned long long)g.grp[k].batch;
         }
         if (tasks >= (1ull << 31)) return cudaErrorInvalidValue;
     }

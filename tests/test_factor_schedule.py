@@ -7,9 +7,10 @@ numbering is topological: every task a task waits on has a smaller number. This 
 numbering (the stage layout and class counts of stage_counts and the class decode of decode_task)
 and checks:
   * run in number order, every task finds its inputs in the states it waits for, each tile update
-    is applied exactly once and in order, and every tile ends final (L_ij: state j + 1, Y_ji:
-    i - j + 1);
-  * the count per problem equals the launcher's closed form;
+    is applied exactly once and in order (a two-level task, which applies the updates of panels m-1
+    and m to its tile together, advances it by two), and every tile ends final (L_ij: state j + 1,
+    Y_ji: i - j + 1);
+  * counting a two-level task as two, the graph applies the plain blocked algorithm's updates;
   * a model of the in-order ticket protocol (W CTAs, each holding a running task and the next
     number it has taken, a finished task released at once) always drains, for several W.
 """
@@ -19,13 +20,28 @@ import pytest
 
 
 def stage_counts(nt, s):
-    """Tasks per problem in stage s by class: next panel's updates G(i,m+1,m), P(m+1), F(j,m),
-    Q(j,i,m), the remaining G(i,j,m), S(i,m+1) (stage 0: P(0), S(i,0))."""
+    """Tasks per problem in stage s by class: [lookahead G(i,m+1,m), P(m+1), F(j,m), one-level Q,
+    two-level FQ (odd m), bulk G (even m: the column m+2, one level; odd m: FG over j >= m+2, levels
+    m-1 and m), S(i,m+1)] (stage 0: P(0), S(i,0))."""
+    n = [0] * 7
     if s == 0:
-        return [0, 1, 0, 0, 0, nt - 1]
+        n[1], n[6] = 1, nt - 1
+        return n
     m = s - 1
     R = nt - 1 - m
-    return [R, 1 if R >= 1 else 0, m, (m + 1) * R, (R - 1) * R // 2 if R >= 1 else 0, R - 1 if R >= 1 else 0]
+    if R < 0:
+        return n
+    R1 = max(R - 1, 0)
+    n[0], n[1], n[2] = R, 1 if R >= 1 else 0, m
+    if m % 2 == 0:
+        n[3] = (m + 1) * min(R, 2)
+        n[5] = R1
+    else:
+        n[3] = (m + 1) * min(R, 1) + R1
+        n[4] = m * R1
+        n[5] = (R - 1) * R // 2 if R >= 1 else 0
+    n[6] = R1
+    return n
 
 
 def decode(nt, s, c, local):
@@ -37,14 +53,23 @@ def decode(nt, s, c, local):
     if c == 2:
         return ("F", m, 0, local)
     if c == 3:
-        ii = local // (m + 1)
-        return ("Q", m, m + 1 + ii, local - ii * (m + 1))
+        if m % 2 == 0:
+            ii, j = divmod(local, m + 1)
+            return ("Q", m, m + 1 + ii, j)
+        if local < m + 1:
+            return ("Q", m, m + 1, local)
+        return ("Q", m, m + 2 + local - (m + 1), m)
     if c == 4:
+        ii, j = divmod(local, m)
+        return ("FQ", m, m + 2 + ii, j)
+    if c == 5:
+        if m % 2 == 0:
+            return ("G", m, m + 2 + local, m + 2)
         rem, j = local, m + 2
         while rem >= nt - j:
             rem -= nt - j
             j += 1
-        return ("G", m, j + rem, j)
+        return ("FG", m, j + rem, j)
     return ("S", s, s + 1 + local, s)
 
 
@@ -57,7 +82,8 @@ def tasks(nt):
 
 
 def deps(task):
-    """(tile kind, i, j, state needed) of the inputs, and (tile kind, i, j, new state) of the outputs."""
+    """(tile kind, i, j, state needed) of the inputs, and (tile kind, i, j, new state) of the outputs.
+    A two-level task waits for level m's operands only: they are final only after level m-1's are."""
     kind, m, i, j = task
     if kind == "P":
         return [("A", m, m, m)], [("A", m, m, m + 1), ("Y", m, m, 1)]
@@ -65,20 +91,28 @@ def deps(task):
         return [("A", i, m, m), ("A", m, m, m + 1)], [("A", i, m, m + 1)]
     if kind == "G":
         return [("A", i, m, m + 1), ("A", j, m, m + 1), ("A", i, j, m)], [("A", i, j, m + 1)]
+    if kind == "FG":
+        return [("A", i, m, m + 1), ("A", j, m, m + 1), ("A", i, j, m - 1)], [("A", i, j, m + 1)]
     if kind == "F":
         return [("Y", j, m, m - j), ("A", m, m, m + 1)], [("Y", j, m, m - j + 1)]
+    if kind == "FQ":
+        return [("Y", j, m, m - j + 1), ("A", i, m, m + 1), ("Y", j, i, m - 1 - j)], [("Y", j, i, m - j + 1)]
     return [("Y", j, m, m - j + 1), ("A", i, m, m + 1), ("Y", j, i, m - j)], [("Y", j, i, m - j + 1)]
 
 
-@pytest.mark.parametrize("nt", list(range(1, 34)))
+def _levels(t):
+    return 2 if t[0] in ("FG", "FQ") else 1
+
+
+@pytest.mark.parametrize("nt", list(range(1, 40)))
 def test_numbering_is_topological_and_complete(nt):
     state = {}
     for t in tasks(nt):
         ins, outs = deps(t)
         for key in ins:
             assert state.get(key[:3], 0) >= key[3], (t, key, state.get(key[:3], 0))
-        for key in outs:
-            assert state.get(key[:3], 0) == key[3] - 1, (t, key)   # each update once, in order
+        for key in outs:   # each update once, in order (a two-level task applies two)
+            assert state.get(key[:3], 0) == key[3] - _levels(t), (t, key)
             state[key[:3]] = key[3]
     for i in range(nt):
         for j in range(i + 1):
@@ -87,10 +121,13 @@ def test_numbering_is_topological_and_complete(nt):
 
 
 @pytest.mark.parametrize("nt", [1, 2, 5, 16, 128])
-def test_count_matches_launcher_closed_form(nt):
-    closed = sum(1 + 2 * R + m + (m + 1) * R + ((R - 1) * R // 2 if R >= 1 else 0)
-                 for m in range(nt) for R in [nt - 1 - m])
-    assert len(tasks(nt)) == closed
+def test_level_updates_match_the_one_level_graph(nt):
+    """Counting a two-level task as two, the graph applies exactly the updates of the plain blocked
+    algorithm: per problem sum_m (1 + 2R + m + (m + 1) R + (R - 1) R / 2), R = nt - 1 - m."""
+    plain = sum(1 + 2 * R + m + (m + 1) * R + ((R - 1) * R // 2 if R >= 1 else 0)
+                for m in range(nt) for R in [nt - 1 - m])
+    assert sum(_levels(t) for t in tasks(nt)) == plain
+    assert len(tasks(nt)) == sum(sum(stage_counts(nt, s)) for s in range(nt + 1))
 
 
 @pytest.mark.parametrize("n_cta", [1, 2, 7, 64])
@@ -98,7 +135,7 @@ def test_in_order_ticket_protocol_drains(n_cta):
     """Several problems of two sizes interleaved (stage by stage, as the kernel numbers them); CTAs
     take numbers in order, each holds at most its running task and its next number, and a task
     starts only when its inputs are final. Random completion order; it must never stall."""
-    groups = [(6, 3), (3, 2)]   # (nt, batch)
+    groups = [(6, 3), (3, 2), (9, 1)]   # (nt, batch)
     numbered = []
     for s in range(max(nt for nt, _ in groups) + 1):
         for gi, (nt, batch) in enumerate(groups):
