@@ -234,7 +234,9 @@ extern "C" clha_status clha_expert_act(clha_ctx* ctx, const void* X, int64_t row
     SET_DEVICE(ctx);
     LaunchScope launch_scope(ctx);
     void* ws = nullptr;
-    clha_status st = clha_workspace(ctx, expert_act_workspace_bytes(d_model), &ws);
+    // the tensor-core path with outlier channels needs masked weight copies: only the automatic choice
+    const size_t wsb = ctx->act_policy == CLHA_ACT_AUTO ? expert_act_workspace_bytes(d_model, E, d_ff, rows) : 256;
+    clha_status st = clha_workspace(ctx, wsb, &ws);
     if (st) return st;
     CUDA_TRY(launch_expert_act(ctx->stream, ctx->num_sms, (const __nv_bfloat16*)X, rows, d_model, nullptr, seg, E,
                                (const __nv_bfloat16*)Wg, (const __nv_bfloat16*)Wu, d_ff, (__nv_bfloat16*)h,

@@ -85,14 +85,18 @@ cudaError_t launch_gather(cudaStream_t s, const void* X, int esize, int64_t n, i
                           int64_t* seg, int32_t* perm, void* ws, size_t ws_bytes, int* err);
 size_t gather_workspace_bytes(int64_t n, int k, int E, int64_t packed_rows);
 constexpr int kGatherBlockTokens = 256;   // tokens per block of the histogram and scatter passes
-size_t expert_act_workspace_bytes(int d_model);
+// Outlier channels (max |x| above 4x the channels' mean) the tensor-core activation takes out of its
+// tensor-core sums and adds exactly in its epilogue; more than this and the fp32-FMA kernel runs.
+constexpr int kMaxOutliers = 64;
+size_t expert_act_workspace_bytes(int d_model, int E, int d_ff, int64_t rows);
 cudaError_t launch_expert_act(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t rows, int d_model,
                               const int32_t* perm, const int64_t* seg, int E, const __nv_bfloat16* Wg,
                               const __nv_bfloat16* Wu, int d_ff, __nv_bfloat16* h, int policy, void* ws, int* sel,
                               int* err);
 cudaError_t launch_expert_act_tc(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t rows, int d_model,
                                  const int64_t* seg, int E, const __nv_bfloat16* Wg, const __nv_bfloat16* Wu, int d_ff,
-                                 __nv_bfloat16* h, const int* sel, int* err);
+                                 __nv_bfloat16* h, const int* sel, const __nv_bfloat16* Wgm, const __nv_bfloat16* Wum,
+                                 const int* out_n, const float* xo, const float* wo, int* err);
 cudaError_t launch_collect_bf16_gathered(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t n, int d,
                                          const int32_t* perm, const int64_t* seg, int E, float* S_base,
                                          int64_t* counts_base, int* err);

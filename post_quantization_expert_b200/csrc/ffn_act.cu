@@ -190,11 +190,16 @@ __global__ void __launch_bounds__(256) act_channel_max(const __nv_bfloat16* __re
     }
 }
 
-// sel = 1 (tensor cores) when every channel's max |x| is within kRangeRatio of the channels' mean,
-// else 0 (fp32 FMA); one block.
+// The choice, on the device, from the channels' max |x| over the rows: a channel is an outlier when
+// its max is above kRangeRatio times the channels' mean. sel = 1 (tensor cores) when there is none;
+// sel = 2 (tensor cores with the outlier channels taken out of the tensor-core sums and added in the
+// epilogue) when there are at most kMaxOutliers, listed in ascending order in out_idx[0 .. *out_n);
+// else sel = 0 (fp32 FMA). One block of 256 threads.
 constexpr float kRangeRatio = 4.f;
-__global__ void __launch_bounds__(256) act_select(const unsigned* __restrict__ chmax, int dm, int* __restrict__ sel) {
+__global__ void __launch_bounds__(256) act_select(const unsigned* __restrict__ chmax, int dm, int* __restrict__ sel,
+                                                  int* __restrict__ out_n, int* __restrict__ out_idx) {
     __shared__ float smax[256], ssum[256];
+    __shared__ int scount[257];
     float m = 0.f, sum = 0.f;
     for (int c = threadIdx.x; c < dm; c += 256) {
         const float v = __uint_as_float(chmax[c]);
@@ -211,18 +216,91 @@ __global__ void __launch_bounds__(256) act_select(const unsigned* __restrict__ c
         }
         __syncthreads();
     }
-    if (threadIdx.x == 0) *sel = (smax[0] <= kRangeRatio * (ssum[0] / dm)) ? 1 : 0;
+    const float limit = kRangeRatio * (ssum[0] / dm);
+    if (smax[0] <= limit) {
+        if (threadIdx.x == 0) { *sel = 1; *out_n = 0; }
+        return;
+    }
+    // the outliers of each thread's contiguous channel range, then their places by a prefix sum
+    const int per = (dm + 255) / 256, c0 = threadIdx.x * per, c1 = c0 + per < dm ? c0 + per : dm;
+    int cnt = 0;
+    for (int c = c0; c < c1; ++c) cnt += __uint_as_float(chmax[c]) > limit;
+    scount[threadIdx.x + 1] = cnt;
+    if (threadIdx.x == 0) scount[0] = 0;
+    __syncthreads();
+    if (threadIdx.x == 0)
+        for (int t = 1; t <= 256; ++t) scount[t] += scount[t - 1];
+    __syncthreads();
+    const int total = scount[256];
+    if (total > kMaxOutliers) {
+        if (threadIdx.x == 0) { *sel = 0; *out_n = 0; }
+        return;
+    }
+    int pos = scount[threadIdx.x];
+    for (int c = c0; c < c1; ++c)
+        if (__uint_as_float(chmax[c]) > limit) out_idx[pos++] = c;
+    if (threadIdx.x == 0) { *sel = 2; *out_n = total; }
+}
+
+// sel == 2: the weights with the outlier channels zeroed (Wgm, Wum: what the tensor cores multiply),
+// and the outlier channels' weights as float32, wo[e][0 gate | 1 up][o][f] (what the epilogue adds).
+// One warp per weight row.
+__global__ void __launch_bounds__(256) act_prep_weights(const int* __restrict__ sel, const int* __restrict__ out_n,
+                                                        const int* __restrict__ out_idx,
+                                                        const __nv_bfloat16* __restrict__ Wg,
+                                                        const __nv_bfloat16* __restrict__ Wu, int E, int dff, int dm,
+                                                        __nv_bfloat16* __restrict__ Wgm, __nv_bfloat16* __restrict__ Wum,
+                                                        float* __restrict__ wo) {
+    if (*sel != 2) return;
+    const int n = *out_n;
+    const int lane = threadIdx.x & 31;
+    const int64_t nrows = 2LL * E * dff;
+    for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < nrows;
+         r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+        const int gu = r >= (int64_t)E * dff;
+        const int64_t er = gu ? r - (int64_t)E * dff : r;
+        const __nv_bfloat16* src = (gu ? Wu : Wg) + er * dm;
+        __nv_bfloat16* dst = (gu ? Wum : Wgm) + er * dm;
+        for (int c = lane * 8; c < dm; c += 256)
+            *reinterpret_cast<uint4*>(dst + c) = __ldg(reinterpret_cast<const uint4*>(src + c));
+        __syncwarp();
+        const int e = (int)(er / dff), f = (int)(er - (int64_t)e * dff);
+        for (int o = lane; o < n; o += 32) {
+            const int c = out_idx[o];
+            wo[((size_t)(2 * e + gu) * kMaxOutliers + o) * dff + f] = __bfloat162float(src[c]);
+            dst[c] = __float2bfloat16(0.f);
+        }
+    }
+}
+
+// sel == 2: the outlier channels of every row as float32, xo[row][o].
+__global__ void __launch_bounds__(256) act_prep_rows(const int* __restrict__ sel, const int* __restrict__ out_n,
+                                                     const int* __restrict__ out_idx,
+                                                     const __nv_bfloat16* __restrict__ X, int64_t rows, int dm,
+                                                     float* __restrict__ xo) {
+    if (*sel != 2) return;
+    const int n = *out_n;
+    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < rows; r += (int64_t)gridDim.x * blockDim.x)
+        for (int o = 0; o < n; ++o) xo[r * kMaxOutliers + o] = __bfloat162float(X[r * dm + out_idx[o]]);
 }
 
 }  // namespace
 
-size_t expert_act_workspace_bytes(int d_model) { return clha_round_up((size_t)d_model * sizeof(unsigned)); }
+// Workspace: the channel maxima, the outlier list, and for the tensor-core path with outliers the
+// masked weight copies, the outlier weights and the rows' outlier channels.
+size_t expert_act_workspace_bytes(int d_model, int E, int d_ff, int64_t rows) {
+    return clha_round_up((size_t)d_model * sizeof(unsigned)) + clha_round_up((kMaxOutliers + 1) * sizeof(int)) +
+           2 * clha_round_up((size_t)E * d_ff * d_model * sizeof(__nv_bfloat16)) +
+           clha_round_up((size_t)2 * E * kMaxOutliers * d_ff * sizeof(float)) +
+           clha_round_up((size_t)rows * kMaxOutliers * sizeof(float));
+}
 
 // The fp32-FMA kernel always reads through a permutation (the tensor-core kernel's TMA loads take
-// packed rows only). Otherwise `policy` picks: 1 fp32 FMA, 2 tensor cores, 0 per call on the device:
-// the channels' max |x| over the rows is measured and the tensor cores run when every channel is within
-// 4x of the channels' mean (no outlier channels), both kernels are queued and the one not chosen exits
-// at once (no host round trip). ws: expert_act_workspace_bytes(d_model); sel: one device int.
+// packed rows only). Otherwise `policy` picks: 1 fp32 FMA, 2 tensor cores, 0 per call on the device
+// (act_select): the tensor cores when at most kMaxOutliers channels are outliers (their products then
+// leave the tensor-core sums and are added in the epilogue), else the FMA kernel; every kernel is
+// queued and the ones not chosen exit at once (no host round trip). ws: expert_act_workspace_bytes;
+// sel: one device int.
 cudaError_t launch_expert_act(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t rows, int d_model,
                               const int32_t* perm, const int64_t* seg, int E, const __nv_bfloat16* Wg,
                               const __nv_bfloat16* Wu, int d_ff, __nv_bfloat16* h, int policy, void* ws, int* sel,
@@ -238,17 +316,28 @@ cudaError_t launch_expert_act(cudaStream_t s, int num_sms, const __nv_bfloat16* 
     const int* sel_dev = nullptr;
     if (!simt_only) {
         if (policy == 2) {
-            return launch_expert_act_tc(s, num_sms, X, rows, d_model, seg, E, Wg, Wu, d_ff, h, nullptr, err);
+            return launch_expert_act_tc(s, num_sms, X, rows, d_model, seg, E, Wg, Wu, d_ff, h, nullptr, nullptr,
+                                        nullptr, nullptr, nullptr, nullptr, err);
         }
-        unsigned* chmax = (unsigned*)ws;
+        char* cur = (char*)ws;
+        unsigned* chmax = (unsigned*)clha_carve(cur, (size_t)d_model * sizeof(unsigned));
+        int* out_n = (int*)clha_carve(cur, (kMaxOutliers + 1) * sizeof(int));
+        int* out_idx = out_n + 1;
+        __nv_bfloat16* Wgm = (__nv_bfloat16*)clha_carve(cur, (size_t)E * d_ff * d_model * sizeof(__nv_bfloat16));
+        __nv_bfloat16* Wum = (__nv_bfloat16*)clha_carve(cur, (size_t)E * d_ff * d_model * sizeof(__nv_bfloat16));
+        float* wo = (float*)clha_carve(cur, (size_t)2 * E * kMaxOutliers * d_ff * sizeof(float));
+        float* xo = (float*)clha_carve(cur, (size_t)rows * kMaxOutliers * sizeof(float));
         cudaError_t e = cudaMemsetAsync(chmax, 0, (size_t)d_model * sizeof(unsigned), s);
         if (e != cudaSuccess) return e;
         const int64_t slabs = (rows + 255) / 256;
         act_channel_max<<<dim3((unsigned)((d_model + 255) / 256), (unsigned)(slabs < 65535 ? slabs : 65535)), 256, 0,
                           s>>>(X, slabs < 65535 ? rows : 65535 * 256, d_model, chmax);
-        act_select<<<1, 256, 0, s>>>(chmax, d_model, sel);
-        clha_note_launches(2);
-        if ((e = launch_expert_act_tc(s, num_sms, X, rows, d_model, seg, E, Wg, Wu, d_ff, h, sel, err)) != cudaSuccess)
+        act_select<<<1, 256, 0, s>>>(chmax, d_model, sel, out_n, out_idx);
+        act_prep_weights<<<4 * num_sms, 256, 0, s>>>(sel, out_n, out_idx, Wg, Wu, E, d_ff, d_model, Wgm, Wum, wo);
+        act_prep_rows<<<2 * num_sms, 256, 0, s>>>(sel, out_n, out_idx, X, rows, d_model, xo);
+        clha_note_launches(4);
+        if ((e = launch_expert_act_tc(s, num_sms, X, rows, d_model, seg, E, Wg, Wu, d_ff, h, sel, Wgm, Wum, out_n, xo,
+                                      wo, err)) != cudaSuccess)
             return e;
         sel_dev = sel;
     }

@@ -36,13 +36,17 @@ constexpr int EPI = 512;                         // epilogue threads
 constexpr uint32_t IDESC = tc::idesc_f32acc(1 /*bf16*/, 0 /*K-major*/, 0 /*K-major*/, BM, 2 * BNH);
 
 struct ActParams {
-    const int* sel;        // null: run; else run only when *sel == 1 (the tensor-core kernel was chosen)
+    const int* sel;        // null: run (no outlier channels taken out); else run when *sel is 1 or 2, and
+                           // with *sel == 2 multiply the masked weights and add the outlier channels' terms
     int64_t rows;          // rows of X and h
     int dm, dff;
     const int64_t* seg;    // null: one expert, all rows valid
     int E;
     __nv_bfloat16* h;
     int n_tiles_n;         // dff / 32
+    const int* out_n;      // outlier channels (sel == 2)
+    const float* xo;       // [rows][kMaxOutliers] the rows' outlier channels
+    const float* wo;       // [E][2][kMaxOutliers][dff] their gate and up weights
     int* err;
 };
 
@@ -73,8 +77,11 @@ __device__ __forceinline__ bool decode(const ActParams& p, int64_t m_tiles, int6
 
 __global__ void __launch_bounds__(kThreads, 1)
 expert_act_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmWg,
-       const __grid_constant__ CUtensorMap tmWu, ActParams p) {
-    if (p.sel && *p.sel != 1) return;   // the fp32-FMA kernel takes this call (uniform: before any setup)
+       const __grid_constant__ CUtensorMap tmWu, const __grid_constant__ CUtensorMap tmWgm,
+       const __grid_constant__ CUtensorMap tmWum, ActParams p) {
+    const int selv = p.sel ? *p.sel : 1;
+    if (selv == 0) return;              // the fp32-FMA kernel takes this call (uniform: before any setup)
+    const bool masked = selv == 2;      // outlier channels: zeroed in the weights the tensor cores read
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
@@ -114,9 +121,11 @@ expert_act_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 
     if (warp == 0) {
         if (lane == 0) {
+            const CUtensorMap* mg = masked ? &tmWgm : &tmWg;
+            const CUtensorMap* mu = masked ? &tmWum : &tmWu;
             tc::prefetch_tmap(&tmX);
-            tc::prefetch_tmap(&tmWg);
-            tc::prefetch_tmap(&tmWu);
+            tc::prefetch_tmap(mg);
+            tc::prefetch_tmap(mu);
             int it = 0;
             bool ok = true;
             int64_t m0, vend;
@@ -130,8 +139,8 @@ expert_act_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     tc::mbar_arrive_expect_tx(fb, STAGE_BYTES);
                     const uint32_t a_dst = tc::smem_u32(smem + s * STAGE_BYTES);
                     tc::tma_load_2d(a_dst, &tmX, fb, kb * BK, (int)m0);
-                    tc::tma_load_2d(a_dst + A_BYTES, &tmWg, fb, kb * BK, wy);
-                    tc::tma_load_2d(a_dst + A_BYTES + B_BYTES / 2, &tmWu, fb, kb * BK, wy);
+                    tc::tma_load_2d(a_dst + A_BYTES, mg, fb, kb * BK, wy);
+                    tc::tma_load_2d(a_dst + A_BYTES + B_BYTES / 2, mu, fb, kb * BK, wy);
                 }
             }
             if (!ok) {
@@ -176,6 +185,7 @@ expert_act_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         // the tile's 32 h-columns (8 gate and 8 up values per row and chunk)
         const int q = warp & 3, quarter = (warp - 2) >> 2;
         constexpr int HW = BNH / 4;
+        static_assert(HW == 8, "the outlier terms below are written out for 8 columns");
         int tcount = 0;
         int64_t m0, vend;
         int n0, e;
@@ -202,6 +212,25 @@ expert_act_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 }
             }
             if (!ok) break;
+            if (masked && row < vend) {   // the outlier channels' terms: bf16 products (exact in fp32) summed in fp64
+                const int no = *p.out_n;
+                const float* xr = p.xo + row * kMaxOutliers;
+                const float* wg = p.wo + (size_t)(2 * e) * kMaxOutliers * p.dff + n0 + quarter * HW;
+                const float* wu = wg + (size_t)kMaxOutliers * p.dff;
+                for (int o = 0; o < no; ++o) {
+                    const float x = __ldg(xr + o);
+                    const float4 g0 = __ldg(reinterpret_cast<const float4*>(wg + (size_t)o * p.dff));
+                    const float4 g1 = __ldg(reinterpret_cast<const float4*>(wg + (size_t)o * p.dff + 4));
+                    const float4 u0 = __ldg(reinterpret_cast<const float4*>(wu + (size_t)o * p.dff));
+                    const float4 u1 = __ldg(reinterpret_cast<const float4*>(wu + (size_t)o * p.dff + 4));
+                    g[0] += (double)(x * g0.x); g[1] += (double)(x * g0.y); g[2] += (double)(x * g0.z);
+                    g[3] += (double)(x * g0.w); g[4] += (double)(x * g1.x); g[5] += (double)(x * g1.y);
+                    g[6] += (double)(x * g1.z); g[7] += (double)(x * g1.w);
+                    u[0] += (double)(x * u0.x); u[1] += (double)(x * u0.y); u[2] += (double)(x * u0.z);
+                    u[3] += (double)(x * u0.w); u[4] += (double)(x * u1.x); u[5] += (double)(x * u1.y);
+                    u[6] += (double)(x * u1.z); u[7] += (double)(x * u1.w);
+                }
+            }
             if (row < p.rows) {
                 const bool valid = row < vend;
                 uint32_t out[HW / 2];
@@ -236,12 +265,18 @@ expert_act_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 
 cudaError_t launch_expert_act_tc(cudaStream_t s, int num_sms, const __nv_bfloat16* X, int64_t rows, int d_model,
                                  const int64_t* seg, int E, const __nv_bfloat16* Wg, const __nv_bfloat16* Wu, int d_ff,
-                                 __nv_bfloat16* h, const int* sel, int* err) {
-    CUtensorMap tX, tG, tU;
+                                 __nv_bfloat16* h, const int* sel, const __nv_bfloat16* Wgm, const __nv_bfloat16* Wum,
+                                 const int* out_n, const float* xo, const float* wo, int* err) {
+    CUtensorMap tX, tG, tU, tGm, tUm;
     cudaError_t e;
     if ((e = make_tmap_2d(&tX, X, (uint64_t)rows, (uint64_t)d_model, 2, BM, BK)) != cudaSuccess) return e;
     if ((e = make_tmap_2d(&tG, Wg, (uint64_t)E * d_ff, (uint64_t)d_model, 2, BNH, BK)) != cudaSuccess) return e;
     if ((e = make_tmap_2d(&tU, Wu, (uint64_t)E * d_ff, (uint64_t)d_model, 2, BNH, BK)) != cudaSuccess) return e;
+    // the masked copies (outlier channels zeroed); without them the unmasked weights stand in (unused)
+    if ((e = make_tmap_2d(&tGm, Wgm ? Wgm : Wg, (uint64_t)E * d_ff, (uint64_t)d_model, 2, BNH, BK)) != cudaSuccess)
+        return e;
+    if ((e = make_tmap_2d(&tUm, Wum ? Wum : Wu, (uint64_t)E * d_ff, (uint64_t)d_model, 2, BNH, BK)) != cudaSuccess)
+        return e;
     static bool attr_set = false;
     if (!attr_set) {
         if ((e = cudaFuncSetAttribute(expert_act_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
@@ -249,8 +284,8 @@ cudaError_t launch_expert_act_tc(cudaStream_t s, int num_sms, const __nv_bfloat1
             return e;
         attr_set = true;
     }
-    ActParams p{sel, rows, d_model, d_ff, seg, E, h, d_ff / BNH, err};
-    expert_act_tc<<<num_sms, kThreads, SMEM_BYTES, s>>>(tX, tG, tU, p);
+    ActParams p{sel, rows, d_model, d_ff, seg, E, h, d_ff / BNH, out_n, xo, wo, err};
+    expert_act_tc<<<num_sms, kThreads, SMEM_BYTES, s>>>(tX, tG, tU, tGm, tUm, p);
     clha_note_launches(1);
     return cudaGetLastError();
 }

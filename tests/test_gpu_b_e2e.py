@@ -117,9 +117,10 @@ def test_moe_pair_E16_top2_full_size(ctx):
 def test_moe_pair_E64_top6_shared_reduced_tokens(ctx):
     """The E=64 top-6 shape with two always-active experts (CLHA-MP: routed 2-bit, shared 3-bit),
     Zipf-skewed routing and outlier channels, at 4096 tokens per layer. The fused path (the expert
-    inputs read from X by TMA gather4, no packed copy); the activation runs on the FMA kernel, which
-    the outlier channels call for."""
-    _moe_pair(ctx, 3, [0, 63], ("rt",), shared_checked=[1], fused=True, act=L.ACT_FMA, tokens=4096)
+    inputs read from X by TMA gather4, no packed copy; the routed experts' activation reads its rows
+    through the permutation on the FMA kernel); the always-active experts' activation, the last of a
+    collect, runs on the tensor cores with the outlier channels taken out of the tensor-core sums."""
+    _moe_pair(ctx, 3, [0, 63], ("rt",), shared_checked=[1], fused=True, act=L.ACT_TENSOR, tokens=4096)
 
 
 def test_unrouted_experts_are_round_to_nearest(ctx):
