@@ -51,7 +51,7 @@ from fractions import Fraction
 import numpy as np
 
 __all__ = [
-    "route_topk", "expert_tokens", "gram", "hessian", "bf16_round", "silu", "ffn_act",
+    "route_topk", "expert_tokens", "gram", "hessian", "bf16_round", "bf16_margin", "silu", "ffn_act",
     "aggregate", "factor", "boundary_distance", "grid_fp32", "quantize_fp32", "gptq", "loss",
     "calibrate_dense", "calibrate_moe_group",
     "pack_codes", "unpack_codes", "dequantize", "dequant_matmul",
@@ -119,12 +119,25 @@ def silu(a):
     return out
 
 
-def ffn_act(Xe, Wg, Wu):
-    """Input of an expert's down projection, h = SiLU(x Wg^T) * (x Wu^T), rounded to bfloat16."""
+def bf16_margin(v):
+    """Distance of each value to the nearest rounding boundary of bf16_round (the midpoints between
+    neighbouring bfloat16 values), in units of the bfloat16 step at the value: 0.5 for a value that
+    is a bfloat16 number, 0 on a midpoint. A diagnostic of how close a rounding decision was."""
+    v = np.asarray(v, dtype=np.float64)
+    _, ex = np.frexp(v)
+    return boundary_distance(np.ldexp(v, -np.maximum(ex - 8, -133)))
+
+
+def ffn_act(Xe, Wg, Wu, return_margin: bool = False):
+    """Input of an expert's down projection, h = SiLU(x Wg^T) * (x Wu^T), rounded to bfloat16;
+    with return_margin also bf16_margin of the unrounded values."""
     Xe = np.asarray(Xe, dtype=np.float64)
     a = Xe @ np.asarray(Wg, dtype=np.float64).T
     b = Xe @ np.asarray(Wu, dtype=np.float64).T
-    return bf16_round(silu(a) * b)
+    v = silu(a) * b
+    if return_margin:
+        return bf16_round(v), bf16_margin(v)
+    return bf16_round(v)
 
 
 # ----------------------------------------------------------------------------------- phase 2
@@ -301,7 +314,8 @@ def calibrate_moe_group(X_list, logits_list, k: int, routed, shared=(), experts=
     experts / shared_experts: which routed / always-active experts to calibrate (default: all).
     Returns per-layer routing and, per expert key ("r", e) / ("s", e): token counts "n", the Hessian
     data "H_in" (gate/up inputs x) and "H_down" (down-projection inputs h), and the GPTQ results
-    "gate", "up", "down" (with their rounding margins under "margin"). GPTQ runs in its lazy-batch
+    "gate", "up", "down" (with their rounding margins under "margin"), and the down projection's
+    inputs "h" per layer with their bf16 rounding margins "h_margin". GPTQ runs in its lazy-batch
     form with `block` columns per batch (None: unblocked).
     """
     E = len(routed)
@@ -317,7 +331,8 @@ def calibrate_moe_group(X_list, logits_list, k: int, routed, shared=(), experts=
              for i in shared_experts]
     for key, (Wg, Wu, Wd), tok_l, bits in jobs:
         Xe = [np.asarray(X, dtype=np.float64)[t] for X, t in zip(X_list, tok_l)]
-        he = [ffn_act(x, Wg, Wu) for x in Xe]
+        hm = [ffn_act(x, Wg, Wu, return_margin=True) for x in Xe]
+        he = [h for h, _ in hm]
         n = [len(t) for t in tok_l]
         res = {"n": n}
         for kind, inputs, mats in (("H_in", Xe, (("gate", Wg), ("up", Wu))), ("H_down", he, (("down", Wd),))):
@@ -331,6 +346,7 @@ def calibrate_moe_group(X_list, logits_list, k: int, routed, shared=(), experts=
                              "loss": loss(Wm, W_hat, agg["H_comb"])}
         res["loss"] = res["gate"]["loss"] + res["up"]["loss"] + res["down"]["loss"]
         res["h"] = he
+        res["h_margin"] = [m for _, m in hm]
         out["experts"][key] = res
     return out
 

@@ -93,3 +93,28 @@ class CodeTally:
         print("codes total", self.what, f"{agree:.6f} over {len(self.matrices)} matrices, {self.total} codes")
         assert agree >= CONFIG_BAR, (self.what, agree)
         return agree
+
+
+# h differences: the GPU and the oracle round h to bfloat16 from values that differ by float32-level
+# errors in the pre-activations (the exact sums are float64 on the oracle's side). An element can
+# then land on the other bfloat16 neighbour: near a rounding midpoint, or anywhere for a tiny h whose
+# terms cancel. Such differences are one bfloat16 step each and rare (a wrong token, weight or
+# expert would move most elements by far more); in an expert with ~100 tokens a single one on a large
+# h moves the Gram of h by ~1e-4 relative.
+H_DIFF_MAX = 1e-3
+
+
+def certify_h(got_h, want_h, margin, what):
+    """Every element of h that differs from the oracle's is one bfloat16 step away, and at most
+    H_DIFF_MAX of the elements differ. Returns (fraction that differs, largest rounding margin of a
+    differing element, in steps; near 0 for a flip at a midpoint)."""
+    got_h, want_h, margin = np.asarray(got_h), np.asarray(want_h), np.asarray(margin)
+    diff = got_h != want_h
+    if not diff.any():
+        return 0.0, 0.0
+    _, ex = np.frexp(want_h[diff])
+    step = np.ldexp(1.0, np.maximum(ex - 8, -133))
+    assert np.all(np.abs(got_h[diff] - want_h[diff]) <= step * (1 + 1e-12)), what
+    frac = float(diff.mean())
+    assert frac <= H_DIFF_MAX, (what, frac)
+    return frac, float(margin[diff].max())

@@ -428,3 +428,14 @@ def test_dequantized_codes_are_gptq_w_hat_and_the_layer_output():
     packed = O.pack_codes(codes, 3)
     np.testing.assert_allclose(O.dequant_matmul(X, packed, scales, zeros, 3, 128), X @ W_hat.astype(np.float64).T,
                                rtol=1e-15, atol=1e-15)
+
+
+def test_bf16_margin_hand_worked():
+    """bfloat16 has 8 significant bits: in [1, 2) the step is 2^-7. 1 is on the grid (margin 1/2),
+    1 + 2^-8 is a midpoint (0), 1 + 3 * 2^-10 lies 3/8 of a step above 1, 1/8 below the midpoint 1 + 2^-8
+    (margin 1/8); in [4, 8) the step is 2^-5, so 4 + 2^-7 is a quarter step past 4 (margin 1/4)."""
+    got = O.bf16_margin([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -10, 4.0 + 2 ** -7, -(1.0 + 2 ** -8)])
+    np.testing.assert_allclose(got, [0.5, 0.0, 0.125, 0.25, 0.0], atol=1e-12)
+    # a value rounds to its neighbour exactly when the margin sign flips: nudging a midpoint
+    v = 1.0 + 2 ** -8
+    assert O.bf16_round(v - 1e-9) == 1.0 and O.bf16_round(v + 1e-9) == 1.0 + 2 ** -7
