@@ -65,9 +65,13 @@ def load_peaks():
 
 
 def alu_peaks(peaks):
-    """Nominal SIMT peaks at the maximum SM clock: 128 FP32 and 64 FP64 FMA lanes per SM."""
+    """Nominal SIMT peaks at the maximum SM clock (128 FP32 and 64 FP64 FMA lanes per SM), and the
+    3xTF32 product rate: the tf32 tensor peak (the measured bf16 peak times the nominal tf32/bf16
+    ratio, 1.1 / 2.25 PFLOP/s) divided by the three tf32 products of each float32-class product."""
     mhz = peaks.get("sm_max_mhz", 1965.0)
-    return {"fp32_tflops": N_SMS * 128 * 2 * mhz * 1e6 / 1e12, "fp64_tflops": N_SMS * 64 * 2 * mhz * 1e6 / 1e12}
+    tf32 = peaks["bf16_tflops"] * 1.1 / 2.25
+    return {"fp32_tflops": N_SMS * 128 * 2 * mhz * 1e6 / 1e12, "fp64_tflops": N_SMS * 64 * 2 * mhz * 1e6 / 1e12,
+            "tf32x3_tflops": tf32 / 3}
 
 
 class ClockSampler:
@@ -437,8 +441,9 @@ def run_ours(args, world, rank, local):
     act_tc = L.clha_last_act_kernel(ctx) == L.ACT_TENSOR   # the activation kernel the steps took
     kernels = {
         "hessian": ("tensor", hess_flops / 1e12, sustained, "TFLOP/s", "syrk_bf16_tc (tcgen05 kind::f16)"),
-        "gptq": ("alu", gptq_flops / 1e12, alu["fp32_tflops"], "TFLOP/s",
-                 "gptq_tc (per-column fp32 sweep; lazy updates on tcgen05 kind::tf32, 3xTF32)"),
+        "gptq": ("tensor", gptq_flops / 1e12, alu["tf32x3_tflops"], "TFLOP/s",
+                 "gptq_tc + gptq_trail (column sweep in fp32; lazy and trailing updates on tcgen05 kind::tf32, "
+                 "3xTF32; peak: tf32 / 3)"),
         "factor": ("alu", factor_flops / 1e12, alu["fp64_tflops"], "TFLOP/s",
                    "fac_load + fac_dag + fac_store (fp64 tile-task graph, mma.sync m8n8k4 f64)"),
         "loss": ("alu", loss_flops / 1e12, alu["fp32_tflops"], "TFLOP/s", "loss_simt (fp32 FMA)"),
@@ -663,8 +668,9 @@ def run_dense(args, world, rank, local):
         "hessian": ("tensor", hess_flops / 1e12, sustained, "TFLOP/s", "syrk_bf16_tc (tcgen05 kind::f16)"),
         "factor": ("alu", factor_flops / 1e12, alu["fp64_tflops"], "TFLOP/s",
                    "fac_load + fac_dag + fac_store (fp64 tile-task graph, mma.sync m8n8k4 f64)"),
-        "gptq": ("alu", gptq_flops / 1e12, alu["fp32_tflops"], "TFLOP/s",
-                 "gptq_tc (per-column fp32 sweep; lazy updates on tcgen05 kind::tf32, 3xTF32)"),
+        "gptq": ("tensor", gptq_flops / 1e12, alu["tf32x3_tflops"], "TFLOP/s",
+                 "gptq_tc + gptq_trail (column sweep in fp32; lazy and trailing updates on tcgen05 kind::tf32, "
+                 "3xTF32; peak: tf32 / 3)"),
         "aggregate": ("hbm", agg_bytes / 1e9, peaks["hbm_gbs"], "GB/s", "agg_combine"),
     }
     dom = max((k for k in phase_ms if k in kernels), key=lambda k: phase_ms[k])
@@ -861,8 +867,8 @@ def run_kernel(args):
                 zs = torch.empty((B, d_out, d // 128), dtype=torch.uint8, device="cuda")
                 Wh = torch.empty((B, d_out, d), device="cuda")
                 fn = lambda: L.clha_quantize(ctx, U, B, W, B, d_out, d, 3, codes, sc, zs, Wh)
-                work, unit, bound, peak = B * d_out * d * d / 1e12, "TFLOP/s", "alu", alu["fp32_tflops"]
-                kname = "gptq_tc"
+                work, unit, bound, peak = B * d_out * d * d / 1e12, "TFLOP/s", "tensor", alu["tf32x3_tflops"]
+                kname = "gptq_tc + gptq_trail (3xTF32; peak: tf32 / 3)"
         for _ in range(args.warmup):
             fn()
         torch.cuda.synchronize()
@@ -882,7 +888,9 @@ def run_kernel(args):
         achieved = work / (ms / 1e3)
         print(json.dumps({"workload": args.workload, "shape": shape, "kernel": kname, "ms": ms, "achieved": achieved,
                           "unit": unit, "bound": bound, "peak": peak, "frac": achieved / peak,
-                          "peak_source": src if bound == "tensor" else "derived (SM count x lanes x max clock)",
+                          "peak_source": (src if bound == "tensor" and args.workload != "gptq" else
+                                          "derived (measured bf16 x nominal tf32/bf16, / 3)" if bound == "tensor" else
+                                          "derived (SM count x lanes x max clock)"),
                           "l2": "flushed (512 MB write) before every timed launch"}))
         torch.cuda.empty_cache()
     ctx.close()

@@ -143,6 +143,26 @@ def test_collect_dense_bf16(ctx, n, d):
     assert torch.all(S[0] == 0)
 
 
+@pytest.mark.parametrize("n,d", [(1100, 8192), (700, 8320)])
+def test_collect_large_d(ctx, n, d):
+    """Channel counts of 8192 and up, where the chunk sums run over longer token ranges: a ragged token
+    count, and d = 8320 (an odd number of 128-channel tiles, so the last tile column holds one
+    diagonal tile only). The Gram equals the float64 one; a second call into another layer of the
+    same accumulator, over a token range that starts mid-block, accumulates there and leaves the first
+    layer alone."""
+    g = _gen(n + d)
+    X = (torch.randn((n, d), generator=g) * (1 + torch.rand(d, generator=g))).to(torch.bfloat16).to(DEV)
+    acc = L.Accum(ctx, d, 2, 1)
+    L.clha_collect(ctx, acc, 0, X, n, d)
+    L.clha_collect(ctx, acc, 1, X[37:].contiguous(), n - 37, d)
+    S, cnt = acc.buffers()
+    torch.cuda.synchronize()
+    X64 = to64(X)
+    assert rel_fro(sym_from_upper(S[0, 0].double().cpu().numpy()), O.gram(X64)) < 1e-4
+    assert rel_fro(sym_from_upper(S[1, 0].double().cpu().numpy()), O.gram(X64[37:])) < 1e-4
+    assert cnt[0, 0].item() == n and cnt[1, 0].item() == n - 37
+
+
 def test_collect_routed_bf16_and_accumulates(ctx):
     n, E, k, d = 3000, 16, 2, 1024
     g = _gen(7)

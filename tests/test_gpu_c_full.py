@@ -23,7 +23,8 @@ import pytest
 import torch
 
 import oracle as O
-from helpers import CONFIG_BAR, CodeTally, assert_codes, rel_fro, sym_from_upper, to64
+from helpers import (CONFIG_BAR, H_INPUT_BAR, MATRIX_BAR, CodeTally, assert_codes, certify_h, rel_fro,
+                     sym_from_upper, to64)
 from post_quantization_expert_b200.pipeline import DenseCalibration, MoECalibration, stack_weights
 from synth import workload
 
@@ -31,20 +32,37 @@ pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 DEV = "cuda:0"
 
 
-def _check_experts(ref, out, S_accs, E, what, tally):
+def _check_experts(ref, out, S_accs, E, what, tally, h_gpu=None):
     """Hessians, certified codes and losses of every expert in an oracle result against the GPU's.
-    S_accs: (S_in, S_dn, S_sdn) accumulator buffers; the always-active experts share input slot E."""
+    S_accs: (S_in, S_dn, S_sdn) accumulator buffers; the always-active experts share input slot E.
+    A down-projection Hessian more than 1e-4 from the oracle's is accepted only when h_gpu (the GPU's
+    h of that routed expert and layer) shows why: its Gram equals the GPU's Hessian to 1e-4, every h
+    element that differs from the oracle's is one bf16 step away and at most 0.1 % differ, and the
+    difference stays under 1e-3 (a sparse expert, where one such difference on a large h moves the
+    Gram by ~1e-4). The codes of such a down projection are held to H_INPUT_BAR."""
     S_in, S_dn, S_sdn = S_accs
     for (kind, e), r in ref["experts"].items():
+        h_moved = False
         for j in range(len(r["n"])):
             s_in = S_in[j, e] if kind == "r" else S_in[j, E]
             s_dn = S_dn[j, e] if kind == "r" else S_sdn[j, e]
             assert rel_fro(sym_from_upper(s_in.double().cpu().numpy()), r["H_in"]["S"][j]) < 1e-4, (what, kind, e, j)
-            assert rel_fro(sym_from_upper(s_dn.double().cpu().numpy()), r["H_down"]["S"][j]) < 1e-4, (what, kind, e, j)
+            got_dn = sym_from_upper(s_dn.double().cpu().numpy())
+            rel_dn = rel_fro(got_dn, r["H_down"]["S"][j])
+            if rel_dn >= 1e-4:
+                assert h_gpu is not None and (kind, e, j) in h_gpu, (what, kind, e, j, rel_dn)
+                hg = h_gpu[(kind, e, j)]
+                assert rel_fro(got_dn, O.gram(hg)) < 1e-4, (what, kind, e, j)
+                frac, worst = certify_h(hg, r["h"][j], r["h_margin"][j], (what, kind, e, j))
+                assert rel_dn < 1e-3, (what, kind, e, j, rel_dn)
+                h_moved = True
+                print("H_down", what, kind, e, j, f"{rel_dn:.3g} from one-step h differences "
+                      f"({frac:.2e} of h, largest rounding margin {worst:.3g})")
         qs = ({"gate": out.qg, "up": out.qu, "down": out.qd} if kind == "r" else
               {"gate": out.sg, "up": out.su, "down": out.sd})
         for name, q in qs.items():
-            tally.add(q.codes[e].cpu().numpy(), q.zeros[e].cpu().numpy(), r[name], (what, kind, e, name, r["n"]))
+            bar = H_INPUT_BAR if name == "down" and h_moved else MATRIX_BAR
+            tally.add(q.codes[e].cpu().numpy(), q.zeros[e].cpu().numpy(), r[name], (what, kind, e, name, r["n"]), bar)
         got = sum(qs[n].loss[e] for n in qs)
         assert abs(got - r["loss"]) <= 1e-3 * r["loss"], (what, kind, e, got, r["loss"])
 
@@ -98,7 +116,9 @@ def test_moe_E64_top6_shared_full_size(ctx):
     the 8 least-routed and the 8 most-routed routed experts and both always-active experts end to end
     against the oracle (Hessians, codes with flip certification, loss). Many of the least-routed
     experts see fewer tokens than d_model in a layer: their Hessians are rank-deficient up to the
-    damping, the hardest case for the code bar."""
+    damping, the hardest case for the code bar, and their down-projection Hessians are sums of ~70
+    outer products, where a single certified bf16 rounding flip of h counts. The activation runs on
+    the tensor cores with the x20 channels taken out of the tensor-core sums."""
     from post_quantization_expert_b200 import clha as L
     wl = workload(3, "cpu")
     s = wl.spec
@@ -109,17 +129,21 @@ def test_moe_E64_top6_shared_full_size(ctx):
                          s.bits_routed, s.bits_shared, s.damp_frac, modes=("rt",))
     Xs = [wl.x(l) for l in range(2)]
     lgs = [wl.logits(l) for l in range(2)]
-    for l in range(2):
-        cal.collect(l, Xs[l].to(DEV), lgs[l].to(DEV), w)
-        print("E64 activation kernel", L.clha_last_act_kernel(ctx))
-    cal.quantize(w, ("rt",))
-    torch.cuda.synchronize()
     routes = [O.route_topk(lg.numpy(), s.k) for lg in lgs]
-    for l in range(2):
-        np.testing.assert_array_equal(cal.counts[l].cpu().numpy(), routes[l][1])
     total = routes[0][1] + routes[1][1]
     order = [int(e) for e in np.argsort(total, kind="stable")]
     checked = sorted(set(order[:8] + order[-8:]))
+    h_gpu = {}
+    for l in range(2):
+        cal.collect(l, Xs[l].to(DEV), lgs[l].to(DEV), w)
+        assert L.clha_last_act_kernel(ctx) == L.ACT_TENSOR     # outlier channels taken out of the sums
+        seg = cal.seg[l].cpu().numpy()
+        for e in checked:                                      # this layer's h of the checked experts
+            h_gpu[("r", e, l)] = cal.hp[seg[e]:seg[e] + routes[l][1][e]].double().cpu().numpy()
+    cal.quantize(w, ("rt",))
+    torch.cuda.synchronize()
+    for l in range(2):
+        np.testing.assert_array_equal(cal.counts[l].cpu().numpy(), routes[l][1])
     least = np.minimum(routes[0][1], routes[1][1])
     assert (least[order[:8]] < s.d_model).sum() >= 4          # rank-deficient per-layer Hessians included
     X64 = [to64(X) for X in Xs]
@@ -130,7 +154,7 @@ def test_moe_E64_top6_shared_full_size(ctx):
     assert len(ref["experts"]) == 16 + s.n_shared
     S_accs = (cal.acc_in.buffers()[0], cal.acc_dn.buffers()[0], cal.acc_sdn.buffers()[0])
     tally = CodeTally("E64")
-    _check_experts(ref, cal.res["rt"], S_accs, s.E, "E64", tally)
+    _check_experts(ref, cal.res["rt"], S_accs, s.E, "E64", tally, h_gpu)
     tally.check()
 
 
