@@ -64,6 +64,23 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+FORMS = {"inv": 0, "block": 1}   # clha_factor_form: CLHA_FACTOR_INV_CHOL, CLHA_FACTOR_BLOCK_CHOL
+
+
+def factor_work(d: int, form: int) -> int:
+    """Algorithmic flops of one factor: U takes the Cholesky and the triangular inverse (2d^3/3); F the
+    Cholesky (d^3/3) and the block scaling, F_ab = R_ab U_bb above the diagonal blocks: per 64 rows of a
+    128-column block three 64^3 tile products (L_ip D_p + L_i,p+1 X and L_i,p+1 D_p+1), 192 flops per
+    element of the upper triangle, 96 d^2."""
+    return 2 * d ** 3 // 3 if form == FORMS["inv"] else d ** 3 // 3 + 96 * d * d
+
+
+def factor_kernels(form: int) -> str:
+    if form == FORMS["inv"]:
+        return "fac_load + fac_dag + fac_store (fp64 tile-task graph, mma.sync m8n8k4 f64)"
+    return "fac_load + fac_dag (Cholesky only) + fac_pair + fac_store_f (fp64, mma.sync m8n8k4 f64)"
+
+
 def alu_peaks(peaks):
     """Nominal SIMT peaks at the maximum SM clock (128 FP32 and 64 FP64 FMA lanes per SM), and the
     3xTF32 product rate: the tf32 tensor peak (the measured bf16 peak times the nominal tf32/bf16
@@ -431,7 +448,7 @@ def run_ours(args, world, rank, local):
     mats = [(dff, dm)] * (2 * Eq) + [(dm, dff)] * Eq        # gate, up, down per weighting
     gptq_flops = len(modes) * sum(o * i * i for o, i in mats)
     loss_flops = len(modes) * sum(2 * o * i * i for o, i in mats)
-    factor_flops = len(modes) * Eq * (2 * dm ** 3 // 3 + 2 * dff ** 3 // 3)
+    factor_flops = len(modes) * Eq * (factor_work(dm, cal.form) + factor_work(dff, cal.form))
     act_flops = sum(int(c.sum()) * 4 * dm * dff for c in counts)
     # per slot and weighting: both layers' upper triangles of S read, the damped aggregate written (full)
     agg_bytes = len(modes) * Eq * sum(2 * (d * (d + 1) // 2) * 4 + d * d * 4 for d in (dm, dff))
@@ -444,8 +461,7 @@ def run_ours(args, world, rank, local):
         "gptq": ("tensor", gptq_flops / 1e12, alu["tf32x3_tflops"], "TFLOP/s",
                  "gptq_tc + gptq_trail (column sweep in fp32; lazy and trailing updates on tcgen05 kind::tf32, "
                  "3xTF32; peak: tf32 / 3)"),
-        "factor": ("alu", factor_flops / 1e12, alu["fp64_tflops"], "TFLOP/s",
-                   "fac_load + fac_dag + fac_store (fp64 tile-task graph, mma.sync m8n8k4 f64)"),
+        "factor": ("alu", factor_flops / 1e12, alu["fp64_tflops"], "TFLOP/s", factor_kernels(cal.form)),
         "loss": ("alu", loss_flops / 1e12, alu["fp32_tflops"], "TFLOP/s", "loss_simt (fp32 FMA)"),
         "act": (("tensor", act_flops / 1e12, sustained, "TFLOP/s", "expert_act_tc (tcgen05 kind::f16)") if act_tc else
                 ("alu", act_flops / 1e12, alu["fp32_tflops"], "TFLOP/s", "expert_act_simt (fp32 FMA)")),
@@ -661,13 +677,12 @@ def run_dense(args, world, rank, local):
     alu = alu_peaks(peaks)
     sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     hess_flops = nl * n * d * (d + 1)
-    factor_flops = 2 * d ** 3 // 3
+    factor_flops = factor_work(d, cal.form)
     gptq_flops = d_out * d * d
     agg_bytes = nl * (d * (d + 1) // 2) * 4 + d * d * 4     # every layer's upper triangle read, H_d written
     kernels = {
         "hessian": ("tensor", hess_flops / 1e12, sustained, "TFLOP/s", "syrk_bf16_tc (tcgen05 kind::f16)"),
-        "factor": ("alu", factor_flops / 1e12, alu["fp64_tflops"], "TFLOP/s",
-                   "fac_load + fac_dag + fac_store (fp64 tile-task graph, mma.sync m8n8k4 f64)"),
+        "factor": ("alu", factor_flops / 1e12, alu["fp64_tflops"], "TFLOP/s", factor_kernels(cal.form)),
         "gptq": ("tensor", gptq_flops / 1e12, alu["tf32x3_tflops"], "TFLOP/s",
                  "gptq_tc + gptq_trail (column sweep in fp32; lazy and trailing updates on tcgen05 kind::tf32, "
                  "3xTF32; peak: tf32 / 3)"),
@@ -855,18 +870,19 @@ def run_kernel(args):
             H = (A @ A.transpose(1, 2) / (d // 2) + 0.05 * torch.eye(d, device="cuda")).contiguous()
             del A
             U = torch.empty_like(H)
+            form = FORMS[args.factor_form]
             if args.workload == "factor":
-                fn = lambda: L.clha_factor(ctx, H, B, d, U)
-                work, unit, bound, peak = B * 2 * d ** 3 / 3 / 1e12, "TFLOP/s", "alu", alu["fp64_tflops"]
-                kname = "fac_load + fac_dag + fac_store"
+                fn = lambda: L.clha_factor_as(ctx, form, H, B, d, U)
+                work, unit, bound, peak = B * factor_work(d, form) / 1e12, "TFLOP/s", "alu", alu["fp64_tflops"]
+                kname = factor_kernels(form)
             else:
-                L.clha_factor(ctx, H, B, d, U)
+                L.clha_factor_as(ctx, form, H, B, d, U)
                 W = (0.02 * torch.randn((B, d_out, d), device="cuda", generator=g)).to(torch.bfloat16)
                 codes = torch.empty((B, d_out, d), dtype=torch.uint8, device="cuda")
                 sc = torch.empty((B, d_out, d // 128), device="cuda")
                 zs = torch.empty((B, d_out, d // 128), dtype=torch.uint8, device="cuda")
                 Wh = torch.empty((B, d_out, d), device="cuda")
-                fn = lambda: L.clha_quantize(ctx, U, B, W, B, d_out, d, 3, codes, sc, zs, Wh)
+                fn = lambda: L.clha_quantize(ctx, U, B, W, B, d_out, d, 3, codes, sc, zs, Wh, form=form)
                 work, unit, bound, peak = B * d_out * d * d / 1e12, "TFLOP/s", "tensor", alu["tf32x3_tflops"]
                 kname = "gptq_tc + gptq_trail (3xTF32; peak: tf32 / 3)"
         for _ in range(args.warmup):
@@ -917,6 +933,8 @@ def main():
     ap.add_argument("--sharpness", type=float, nargs="+", default=[0.0, 0.1, 0.2, 0.3, 0.5, 0.75, 1.0],
                     help="sweep: strengths of the per-layer expert preference")
     ap.add_argument("--shape", nargs="+", default=[], help="kernel workload shapes, e.g. 65536x4096")
+    ap.add_argument("--factor-form", choices=tuple(FORMS), default="block",
+                    help="factor and gptq kernel workloads: U (inv) or the block-scaled Cholesky factor (block)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -245,6 +245,20 @@ typedef struct clha_factor_group {
 } clha_factor_group;
 CLHA_API clha_status clha_factor_groups(clha_ctx* ctx, int n_groups, const clha_factor_group* groups);
 
+/* The factor in either of two forms, each written as float32 [batch, d, d], zero below the diagonal:
+ *   CLHA_FACTOR_INV_CHOL    U, as clha_factor writes it (H_damped^-1 = U^T U);
+ *   CLHA_FACTOR_BLOCK_CHOL  F, the Cholesky factor of H_damped scaled per 128-column block: with R
+ *                           upper and H_damped = R R^T, and U = R^-1 (U_bb = R_bb^-1 on the diagonal
+ *                           blocks), F_bb = U_bb and F_ab = R_ab U_bb for a < b.
+ * F takes one Cholesky and no triangular inverse (half the flops of U). GPTQ with F
+ * (clha_quantize_as) makes the same decisions as GPTQ with U, up to rounding: every step inside a
+ * block uses U_bb, and the lazy update of block b from the earlier columns a, W_b - E_a U_ab with
+ * GPTQ's scaled errors E (W - W_hat = E U), equals W_b + (W_a - W_hat_a) F_ab. F serves GPTQ only:
+ * E-PMQ's target needs U. Groups, errors and limits as clha_factor_groups. */
+typedef enum clha_factor_form { CLHA_FACTOR_INV_CHOL = 0, CLHA_FACTOR_BLOCK_CHOL = 1 } clha_factor_form;
+CLHA_API clha_status clha_factor_groups_as(clha_ctx* ctx, clha_factor_form form, int n_groups,
+                                           const clha_factor_group* groups);
+
 /* Time limit, in nanoseconds, of each dependency wait inside clha_factor's task graph (a CTA waiting
  * for a tile that another CTA is still producing); 0 restores the default of 4 s. A wait that runs
  * out sets the graph's abort flag: every CTA stops taking tasks and returns, the call's U is
@@ -314,6 +328,15 @@ CLHA_API clha_status clha_quantize(clha_ctx* ctx, const float* U, int n_u, const
                           int batch, int d_out, int d_in, const clha_quant_params* params,
                           uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
                           const double* lambda, double* loss);
+/* clha_quantize with the factor in the given form (CLHA_FACTOR_BLOCK_CHOL: F from
+ * clha_factor_groups_as). Under F the lazy and trailing updates take W_hat - W of the earlier columns
+ * in place of their scaled errors; the grid, the codes, W_hat and the loss are defined exactly as in
+ * clha_quantize. Arguments, outputs and errors as clha_quantize; an unknown form is
+ * CLHA_ERR_INVALID_ARG. */
+CLHA_API clha_status clha_quantize_as(clha_ctx* ctx, clha_factor_form form, const float* F, int n_u, const void* W,
+                                      clha_dtype dtype, int batch, int d_out, int d_in,
+                                      const clha_quant_params* params, uint8_t* codes, float* scales, uint8_t* zeros,
+                                      float* W_hat, const double* lambda, double* loss);
 
 /* Loss of the CLHA page §2.1, one term: loss_out[b] = tr[(W_hat - W) H (W_hat - W)^T] for `batch`
  * problems; H holds n_h matrices and problem b uses H[b % n_h] (1 <= n_h <= batch). Tile sums are

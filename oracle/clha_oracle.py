@@ -52,7 +52,7 @@ import numpy as np
 
 __all__ = [
     "route_topk", "expert_tokens", "gram", "hessian", "bf16_round", "bf16_margin", "silu", "ffn_act",
-    "aggregate", "factor", "boundary_distance", "grid_fp32", "quantize_fp32", "gptq", "loss",
+    "aggregate", "factor", "factor_block_scaled", "boundary_distance", "grid_fp32", "quantize_fp32", "gptq", "loss",
     "calibrate_dense", "calibrate_moe_group",
     "pack_codes", "unpack_codes", "dequantize", "dequant_matmul",
     "routing_divergence", "hessian_error",
@@ -187,6 +187,29 @@ def factor(H_d):
     Hinv = Linv.T @ Linv
     Hinv = 0.5 * (Hinv + Hinv.T)
     return np.linalg.cholesky(Hinv).T
+
+
+def factor_block_scaled(H_d, block: int = 128):
+    """F: the Cholesky factor of H_d scaled per column block, which GPTQ can use in place of U (a
+    reformulation of GPTQ's lazy update, not a step of the pages).
+
+    R is upper with H_d = R R^T (the Cholesky factorisation taken in reversed index order), and
+    U = R^-1 is the same U as factor(H_d). A triangular matrix's inverse has the inverses of its
+    diagonal blocks on its diagonal, so U_bb = R_bb^-1. F holds U_bb on each diagonal block b and
+    R_ab U_bb on the blocks a < b above it, zeros below. With D = W - W_hat and GPTQ's scaled errors E
+    (W - W_hat = E U, so E = D R and E_a U_aa = D_a), and U_ab = -U_aa R_ab U_bb, the lazy update
+    W_b - E_a U_ab equals W_b + D_a F_ab. block = d gives F = U."""
+    H_d = np.asarray(H_d, dtype=np.float64)
+    d = H_d.shape[0]
+    rev = np.arange(d)[::-1]
+    R = np.linalg.cholesky(H_d[np.ix_(rev, rev)])[np.ix_(rev, rev)]   # upper, H_d = R R^T
+    F = np.zeros_like(H_d)
+    for b0 in range(0, d, block):
+        b1 = min(d, b0 + block)
+        Ubb = np.linalg.inv(R[b0:b1, b0:b1])
+        F[b0:b1, b0:b1] = np.triu(Ubb)
+        F[:b0, b0:b1] = R[:b0, b0:b1] @ Ubb
+    return F
 
 
 def boundary_distance(v):

@@ -34,9 +34,12 @@ SYMBOLS = [
     "clha_aggregate", "clha_factor", "clha_factor_groups", "clha_epmq_target", "clha_quantize", "clha_loss",
     "clha_pack_codes", "clha_dequantize", "clha_dequant_matmul", "clha_routing_divergence",
     "clha_collect_gathered", "clha_expert_act_gathered", "clha_set_act_kernel", "clha_last_act_kernel",
-    "clha_set_factor_wait_limit", "clha_pack_upper", "clha_unpack_upper",
+    "clha_set_factor_wait_limit", "clha_pack_upper", "clha_unpack_upper", "clha_factor_groups_as",
+    "clha_quantize_as",
 ]
 FACTOR_MAX_GROUPS = 4
+# clha_factor_form: U with H_d^-1 = U^T U, or F, the block-scaled Cholesky factor of H_d (GPTQ only)
+FACTOR_INV_CHOL, FACTOR_BLOCK_CHOL = 0, 1
 
 
 class FactorGroup(C.Structure):
@@ -89,12 +92,15 @@ def load(path: str = LIB_PATH):
         "clha_aggregate": (i32, [vp, vp, i32, i32, i32, vp, f64, vp, vp, vp, vp, vp]),
         "clha_factor": (i32, [vp, vp, i32, i32, vp]),
         "clha_factor_groups": (i32, [vp, i32, vp]),
+        "clha_factor_groups_as": (i32, [vp, i32, i32, vp]),
         "clha_epmq_target": (i32, [vp, vp, i32, vp, vp, i32, i32, vp, vp, vp]),
         "clha_pack_codes": (i32, [vp, vp, i64, i32, i32, vp]),
         "clha_dequantize": (i32, [vp, vp, vp, vp, i64, i32, i32, vp]),
         "clha_dequant_matmul": (i32, [vp, vp, i32, i64, vp, vp, vp, i32, i32, i32, vp]),
         "clha_quantize": (i32, [vp, vp, i32, vp, i32, i32, i32, i32, C.POINTER(QuantParams), vp, vp, vp, vp, vp,
                                 vp]),
+        "clha_quantize_as": (i32, [vp, i32, vp, i32, vp, i32, i32, i32, i32, C.POINTER(QuantParams), vp, vp, vp, vp,
+                                   vp, vp]),
         "clha_loss": (i32, [vp, vp, i32, vp, vp, i32, i32, i32, i32, vp]),
         "clha_routing_divergence": (i32, [vp, vp, i32, i32, i32, i32, vp]),
         "clha_collect_gathered": (i32, [vp, vp, i32, vp, i64, i32, vp, vp, i32, i32]),
@@ -308,10 +314,19 @@ def clha_set_factor_wait_limit(ctx: Context, ns: int):
     ctx._check(load().clha_set_factor_wait_limit(ctx.handle, ns))
 
 
-def clha_factor_groups(ctx: Context, groups):
-    """groups: sequence of (H_damped, batch, d, U), at most FACTOR_MAX_GROUPS; one graph launch."""
+def clha_factor_groups(ctx: Context, groups, form: int = FACTOR_INV_CHOL):
+    """groups: sequence of (H_damped, batch, d, U), at most FACTOR_MAX_GROUPS; one graph launch.
+    form FACTOR_BLOCK_CHOL writes F (for clha_quantize with the same form) in place of U."""
     arr = (FactorGroup * len(groups))(*[FactorGroup(_p(H), _p(U), b, d) for H, b, d, U in groups])
-    ctx._check(load().clha_factor_groups(ctx.handle, len(groups), C.cast(arr, C.c_void_p)))
+    if form == FACTOR_INV_CHOL:
+        ctx._check(load().clha_factor_groups(ctx.handle, len(groups), C.cast(arr, C.c_void_p)))
+    else:
+        ctx._check(load().clha_factor_groups_as(ctx.handle, form, len(groups), C.cast(arr, C.c_void_p)))
+
+
+def clha_factor_as(ctx: Context, form: int, H_damped, batch: int, d: int, F):
+    """One group of clha_factor_groups in the given form."""
+    clha_factor_groups(ctx, [(H_damped, batch, d, F)], form)
 
 
 def clha_epmq_target(ctx: Context, acc: "Accum", slot: int, W_src, W_merged, d_out: int, U, lambda_dev, W_target):
@@ -340,11 +355,18 @@ def clha_routing_divergence(ctx: Context, counts, n_layers: int, ld: int, slot0:
 
 
 def clha_quantize(ctx: Context, U, n_u: int, W, batch: int, d_out: int, d_in: int, bits: int, codes, scales,
-                  zeros, W_hat=None, group: int = 128, block: int = 128, damp_frac: float = 0.01, lam=None, loss=None):
-    """lam (float64 device [n_u]) and loss (float64 device [batch]) request the in-kernel loss."""
+                  zeros, W_hat=None, group: int = 128, block: int = 128, damp_frac: float = 0.01, lam=None, loss=None,
+                  form: int = FACTOR_INV_CHOL):
+    """lam (float64 device [n_u]) and loss (float64 device [batch]) request the in-kernel loss; form: what
+    U holds (FACTOR_BLOCK_CHOL: F from clha_factor_groups with that form)."""
     qp = QuantParams(bits, group, block, damp_frac)
-    ctx._check(load().clha_quantize(ctx.handle, _p(U), n_u, _p(W), _dtype(W), batch, d_out, d_in, C.byref(qp),
-                                    _p(codes), _p(scales), _p(zeros), _p(W_hat), _p(lam), _p(loss)))
+    if form == FACTOR_INV_CHOL:
+        ctx._check(load().clha_quantize(ctx.handle, _p(U), n_u, _p(W), _dtype(W), batch, d_out, d_in, C.byref(qp),
+                                        _p(codes), _p(scales), _p(zeros), _p(W_hat), _p(lam), _p(loss)))
+    else:
+        ctx._check(load().clha_quantize_as(ctx.handle, form, _p(U), n_u, _p(W), _dtype(W), batch, d_out, d_in,
+                                           C.byref(qp), _p(codes), _p(scales), _p(zeros), _p(W_hat), _p(lam),
+                                           _p(loss)))
 
 
 def clha_loss(ctx: Context, W, W_hat, H, n_h: int, batch: int, d_out: int, d_in: int) -> np.ndarray:

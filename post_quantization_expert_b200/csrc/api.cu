@@ -465,8 +465,11 @@ extern "C" clha_status clha_aggregate(clha_ctx* ctx, const clha_accum* acc, int 
 }
 
 // ------------------------------------------------------------------------------ phase 3
-extern "C" clha_status clha_factor_groups(clha_ctx* ctx, int n_groups, const clha_factor_group* groups) {
+extern "C" clha_status clha_factor_groups_as(clha_ctx* ctx, clha_factor_form form, int n_groups,
+                                             const clha_factor_group* groups) {
     CHECK_CTX(ctx);
+    REQUIRE(form == CLHA_FACTOR_INV_CHOL || form == CLHA_FACTOR_BLOCK_CHOL, CLHA_ERR_INVALID_ARG,
+            "clha_factor: unknown form %d", (int)form);
     REQUIRE(groups, CLHA_ERR_INVALID_ARG, "clha_factor_groups: null groups");
     REQUIRE(n_groups >= 1 && n_groups <= CLHA_FACTOR_MAX_GROUPS, CLHA_ERR_INVALID_ARG,
             "clha_factor_groups: n_groups=%d outside 1..%d", n_groups, CLHA_FACTOR_MAX_GROUPS);
@@ -484,9 +487,13 @@ extern "C" clha_status clha_factor_groups(clha_ctx* ctx, int n_groups, const clh
     void* ws = nullptr;
     clha_status st = clha_workspace(ctx, factor_workspace_bytes(fg, n_groups), &ws);
     if (st) return st;
-    CUDA_TRY(launch_factor(ctx->stream, ctx->num_sms, fg, n_groups, ws, ctx->d_err, ctx->factor_wait_ns),
+    CUDA_TRY(launch_factor(ctx->stream, ctx->num_sms, fg, n_groups, ws, ctx->d_err, ctx->factor_wait_ns, (int)form),
              "clha_factor");
     return CLHA_OK;
+}
+
+extern "C" clha_status clha_factor_groups(clha_ctx* ctx, int n_groups, const clha_factor_group* groups) {
+    return clha_factor_groups_as(ctx, CLHA_FACTOR_INV_CHOL, n_groups, groups);
 }
 
 extern "C" clha_status clha_set_factor_wait_limit(clha_ctx* ctx, uint64_t ns) {
@@ -582,11 +589,13 @@ extern "C" clha_status clha_epmq_target(clha_ctx* ctx, const clha_accum* acc, in
     return CLHA_OK;
 }
 
-extern "C" clha_status clha_quantize(clha_ctx* ctx, const float* U, int n_u, const void* W, clha_dtype dtype,
-                                     int batch, int d_out, int d_in, const clha_quant_params* p,
-                                     uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
-                                     const double* lambda, double* loss) {
+extern "C" clha_status clha_quantize_as(clha_ctx* ctx, clha_factor_form form, const float* U, int n_u, const void* W,
+                                        clha_dtype dtype, int batch, int d_out, int d_in, const clha_quant_params* p,
+                                        uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
+                                        const double* lambda, double* loss) {
     CHECK_CTX(ctx);
+    REQUIRE(form == CLHA_FACTOR_INV_CHOL || form == CLHA_FACTOR_BLOCK_CHOL, CLHA_ERR_INVALID_ARG,
+            "clha_quantize: unknown factor form %d", (int)form);
     REQUIRE(U && W && p && codes && scales && zeros, CLHA_ERR_INVALID_ARG, "clha_quantize: null pointer");
     REQUIRE(dtype == CLHA_BF16 || dtype == CLHA_F32, CLHA_ERR_INVALID_ARG, "clha_quantize: unknown dtype");
     REQUIRE(batch >= 1 && d_out > 0 && d_in > 0 && n_u >= 1 && n_u <= batch, CLHA_ERR_INVALID_ARG,
@@ -604,8 +613,16 @@ extern "C" clha_status clha_quantize(clha_ctx* ctx, const float* U, int n_u, con
     clha_status st = clha_workspace(ctx, quantize_workspace_bytes(batch, d_out, d_in), &ws);
     if (st) return st;
     CUDA_TRY(launch_quantize(ctx->stream, ctx->num_sms, U, n_u, W, dtype == CLHA_F32, batch, d_out, d_in, p->bits, codes,
-                             scales, zeros, W_hat, lambda, loss, ws, ctx->d_err), "clha_quantize");
+                             scales, zeros, W_hat, lambda, loss, ws, ctx->d_err, (int)form), "clha_quantize");
     return CLHA_OK;
+}
+
+extern "C" clha_status clha_quantize(clha_ctx* ctx, const float* U, int n_u, const void* W, clha_dtype dtype,
+                                     int batch, int d_out, int d_in, const clha_quant_params* p,
+                                     uint8_t* codes, float* scales, uint8_t* zeros, float* W_hat,
+                                     const double* lambda, double* loss) {
+    return clha_quantize_as(ctx, CLHA_FACTOR_INV_CHOL, U, n_u, W, dtype, batch, d_out, d_in, p, codes, scales, zeros,
+                            W_hat, lambda, loss);
 }
 
 extern "C" clha_status clha_loss(clha_ctx* ctx, const void* W, clha_dtype dtype, const float* W_hat, const float* H,

@@ -120,8 +120,9 @@ struct FactorGroup {
     int batch, d;
 };
 size_t factor_workspace_bytes(const FactorGroup* groups, int n);
+// form 0: U (H_d^-1 = U^T U); form 1: F, the block-scaled Cholesky factor of H_d (factor.cu)
 cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups, int n, void* ws, int* err,
-                          uint64_t wait_ns);
+                          uint64_t wait_ns, int form);
 cudaError_t launch_pack_codes(cudaStream_t s, const uint8_t* codes, int64_t rows, int d_in, int bits,
                               uint32_t* packed);
 cudaError_t launch_dequantize(cudaStream_t s, const uint32_t* packed, const float* scales, const uint8_t* zeros,
@@ -143,6 +144,6 @@ size_t quantize_workspace_bytes(int batch, int d_out, int d_in);
 cudaError_t launch_quantize(cudaStream_t s, int num_sms, const float* U, int n_u, const void* W, int w_is_f32,
                             int batch, int d_out, int d_in, int bits, uint8_t* codes, float* scales,
                             uint8_t* zeros, float* W_hat, const double* lambda, double* loss, void* ws,
-                            int* err);
+                            int* err, int form);   // form as launch_factor's: the factor U holds
 cudaError_t launch_loss(cudaStream_t s, const void* W, int w_is_f32, const float* W_hat, const float* H,
                         int n_h, int batch, int d_out, int d_in, double* d_loss);

@@ -1,9 +1,22 @@
-// GPTQ's factor of the damped Hessian: U upper triangular with H_d^-1 = U^T U.
+// GPTQ's factor of the damped Hessian, in one of two forms:
+//   U (CLHA_FACTOR_INV_CHOL)    upper triangular with H_d^-1 = U^T U;
+//   F (CLHA_FACTOR_BLOCK_CHOL)  the Cholesky factor of H_d itself, scaled per 128-column block.
 //
 // With J the index reversal, let L be the lower Cholesky factor of J H_d J. Then R = J L J is upper
 // with H_d = R R^T, and U = R^-1 = J L^-1 J is upper with U^T U = (R R^T)^-1 = H_d^-1; its diagonal
-// is positive, so it is THE upper Cholesky factor of H_d^-1. This needs one Cholesky and one
-// triangular inverse (no explicit inverse of H_d, no second factorisation).
+// is positive, so it is THE upper Cholesky factor of H_d^-1. U needs one Cholesky and one triangular
+// inverse (no explicit inverse of H_d, no second factorisation).
+//
+// F needs the Cholesky only. U's diagonal blocks are the inverses of R's (U_bb = R_bb^-1), and
+// U_ab = -U_aa R_ab U_bb above them. F holds U_bb on the diagonal blocks and F_ab = R_ab U_bb (a < b)
+// above them. GPTQ's lazy update of block b, W_b - E_a U_ab with E = (W - W_hat) R the scaled errors
+// of the earlier columns a, then equals W_b + (W_a - W_hat_a) F_ab, since E_a U_aa = W_a - W_hat_a.
+// So F serves GPTQ in place of U at half the factor's flops: the inverse terms (F and Q tasks below)
+// drop out, and the block scaling is one small product per tile, done by the store. In J order a
+// 128-block b of F is the pair of 64-tiles (p, p+1), p even, of L, and J F J = L blockdiag(L_bb^-1):
+//   L_bb^-1 = [[D_p, 0], [X, D_{p+1}]],   X = -D_{p+1} L_{p+1,p} D_p,
+// so the tiles of J F J are D_p, X, D_{p+1} on the diagonal block, L_ip D_p + L_{i,p+1} X and
+// L_{i,p+1} D_{p+1} below it (i >= p + 2).
 //
 // Float64 throughout, on 64 x 64 tiles (nt = d / 64 per side), batched over problems, in up to four
 // groups of different d that share one graph launch (the small groups' short critical paths then
@@ -12,6 +25,9 @@
 //   fac_dag     one persistent kernel that runs the whole blocked Cholesky and the blocked inverse
 //               of every problem of every group as a graph of tile tasks (below)
 //   fac_store   U = J Y^T J as float32, strict lower triangle zero; per group
+// and for F, the graph without its inverse tasks, then
+//   fac_pair    X^T of every 128-block (two tile products, kept in the otherwise unused tile Y_{p,p+1})
+//   fac_store_f F = J (L blockdiag(L_bb^-1)) J as float32, the products on the FP64 tensor path
 //
 // Tile tasks. The inverse is kept transposed, Y = L^-T (upper), so that every product has the form
 // C <- alpha C + beta P Q^T with row-major tiles P and Q:
@@ -135,7 +151,8 @@ __device__ __forceinline__ void tile_to_smem(Tile* dst, const double* __restrict
     }
 }
 
-// C (global tile, row-major 64x64) <- (load_c ? C : 0) + sign * (P1 Q1^T [+ P2 Q2^T]): one or two
+// C (row-major 64x64, row pitch ldc; global, or shared when !load_c) <- (load_c ? C : 0) +
+// sign * (P1 Q1^T [+ P2 Q2^T]): one or two
 // operand pairs (a two-level task applies two panels' updates to its output tile with one read and
 // one write of C). The first pair's copies into shared memory and the loads of this thread's C
 // fragments are in flight together; a second pair is copied after every warp has finished with the
@@ -146,7 +163,7 @@ __device__ __forceinline__ void tile_to_smem(Tile* dst, const double* __restrict
 __device__ __forceinline__ void tile_gemm_nt(const double* __restrict__ Pg, const double* __restrict__ Qg, Tile* Ps,
                                              Tile* Qs, double* C, bool load_c, bool negate,
                                              const double* __restrict__ Pg2 = nullptr,
-                                             const double* __restrict__ Qg2 = nullptr) {
+                                             const double* __restrict__ Qg2 = nullptr, int ldc = NB) {
     tile_to_smem(Ps, Pg);
     tile_to_smem(Qs, Qg);
     asm volatile("cp.async.commit_group;" ::: "memory");
@@ -201,7 +218,7 @@ __device__ __forceinline__ void tile_gemm_nt(const double* __restrict__ Pg, cons
     for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
         for (int ni = 0; ni < 2; ++ni)
-            *reinterpret_cast<double2*>(C + (32 * wm + 8 * mi + g) * NB + 16 * wn + 8 * ni + 2 * tq) =
+            *reinterpret_cast<double2*>(C + (32 * wm + 8 * mi + g) * ldc + 16 * wn + 8 * ni + 2 * tq) =
                 negate ? make_double2(-c[mi][ni][0], -c[mi][ni][1]) : make_double2(c[mi][ni][0], c[mi][ni][1]);
 }
 
@@ -414,6 +431,7 @@ struct Dag {
     int* err;
     unsigned long long total;
     uint64_t wait_ns;   // time limit of one dependency wait
+    int inv;            // 1: Cholesky and inverse (U); 0: Cholesky only (F)
 };
 
 __device__ __forceinline__ double* tile(double* base, const Grp& g, int b, int i, int j) {
@@ -458,7 +476,9 @@ __device__ bool wait_ge(const int* p, int target, const Dag& g, int problem) {
 // pays its scheduling once, and the lookahead chain P(m) -> S(m+1,m) -> G(m+1,m+1,m) -> P(m+1) keeps
 // its one-level tasks. Every task waits only on tasks with smaller numbers (a CPU model of this
 // numbering checks that, and that each update is applied once, for every tile count up to 39).
-__host__ __device__ __forceinline__ void stage_counts(int nt, int s, long long (&n)[7]) {
+// Without the inverse (the F form) classes 2, 3 and 4 are empty and the rest keep their numbers'
+// order and dependencies, which never involve Y.
+__host__ __device__ __forceinline__ void stage_counts(int nt, int s, long long (&n)[7], bool inv = true) {
     for (int c = 0; c < 7; ++c) n[c] = 0;
     if (s == 0) {
         n[1] = 1;
@@ -481,11 +501,12 @@ __host__ __device__ __forceinline__ void stage_counts(int nt, int s, long long (
         n[5] = R >= 1 ? (R - 1) * R / 2 : 0;
     }
     n[6] = R1;
+    if (!inv) n[2] = n[3] = n[4] = 0;
 }
-__host__ __device__ __forceinline__ unsigned long long stage_total(int nt, int s) {
+__host__ __device__ __forceinline__ unsigned long long stage_total(int nt, int s, bool inv = true) {
     if (s > nt) return 0;
     long long n[7];
-    stage_counts(nt, s, n);
+    stage_counts(nt, s, n, inv);
     return (unsigned long long)(n[0] + n[1] + n[2] + n[3] + n[4] + n[5] + n[6]);
 }
 
@@ -521,7 +542,7 @@ __device__ __forceinline__ void decode_task(const Dag& g, const unsigned long lo
 #pragma unroll
     for (int kk = 0; kk < MAX_GROUPS; ++kk) {
         if (!found && kk < g.ng) {
-            const uint32_t c = (uint32_t)stage_total(g.grp[kk].nt, sg) * (uint32_t)g.grp[kk].batch;
+            const uint32_t c = (uint32_t)stage_total(g.grp[kk].nt, sg, g.inv) * (uint32_t)g.grp[kk].batch;
             if (r < c) { k = kk; found = true; }
             else r -= c;
         }
@@ -530,7 +551,7 @@ __device__ __forceinline__ void decode_task(const Dag& g, const unsigned long lo
     const int nt = G.nt;
     const uint32_t batch = (uint32_t)G.batch;
     long long n[7];
-    stage_counts(nt, sg, n);
+    stage_counts(nt, sg, n, g.inv);
     int c = 0;
 #pragma unroll
     for (int cq = 0; cq < 7; ++cq)
@@ -630,7 +651,7 @@ __global__ void __launch_bounds__(DAG_THREADS, 2) fac_dag(Dag g) {
             unsigned long long acc = 0;
             for (int s = 0; s <= S; ++s) {
                 lvl[s] = acc;
-                for (int k = 0; k < g.ng; ++k) acc += stage_total(g.grp[k].nt, s) * g.grp[k].batch;
+                for (int k = 0; k < g.ng; ++k) acc += stage_total(g.grp[k].nt, s, g.inv) * g.grp[k].batch;
             }
             lvl[S + 1] = acc;
         }
@@ -744,6 +765,62 @@ constexpr size_t dag_smem_bytes(int nt) {
     return (size_t)(2 * TILE_DOUBLES + P_SCRATCH) * sizeof(double) + (size_t)(nt + 2) * sizeof(unsigned long long);
 }
 
+// ------------------------------------------------------------------------------ the F form
+// X^T of the 128-block (p, p+1), p = 2 blockIdx.x, into the tile Y_{p,p+1} (unused without the
+// inverse): T = Y_pp L_{p+1,p}^T = (L_{p+1,p} D_p)^T, then Y_{p,p+1} = -T D_{p+1}^T = X^T.
+constexpr size_t PAIR_SMEM = 2 * TILE_DOUBLES * sizeof(double);
+__global__ void __launch_bounds__(256) fac_pair(Grp G) {
+    extern __shared__ double dsm[];
+    Tile* Ps = reinterpret_cast<Tile*>(dsm);
+    Tile* Qs = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
+    const int b = blockIdx.y, p = 2 * blockIdx.x;
+    double* Yx = tile(G.Y, G, b, p, p + 1);
+    tile_gemm_nt(tile(G.Y, G, b, p, p), tile(G.A, G, b, p + 1, p), Ps, Qs, Yx, false, false);
+    __threadfence();   // T reaches L2, where the next product's copies read it
+    cbar();
+    tile_gemm_nt(Yx, G.D + ((size_t)b * G.nt + p + 1) * TILE_ELEMS, Ps, Qs, Yx, false, true);
+}
+
+// F tile (ta, tc), ta <= tc, is the 180-degree rotation of the tile (it, jt) = (nt-1-ta, nt-1-tc) of
+// J F J = L blockdiag(L_bb^-1): D_jt on the diagonal; for even jt, X at it = jt + 1 and
+// L_{it,jt} D_jt + L_{it,jt+1} X below; for odd jt, L_{it,jt} D_jt below. The tile is formed in shared
+// memory (products on the FP64 tensor path) and written as float32; tiles below the diagonal are zero.
+constexpr size_t STORE_F_SMEM = 3 * TILE_DOUBLES * sizeof(double);
+__global__ void __launch_bounds__(256) fac_store_f(Grp G, float* __restrict__ F) {
+    extern __shared__ double dsm[];
+    Tile* Ps = reinterpret_cast<Tile*>(dsm);
+    Tile* Qs = reinterpret_cast<Tile*>(dsm + TILE_DOUBLES);
+    Tile* Os = reinterpret_cast<Tile*>(dsm + 2 * TILE_DOUBLES);
+    const int b = blockIdx.y, nt = G.nt, d = G.d;
+    const int ta = blockIdx.x / nt, tc = blockIdx.x % nt;
+    float* Fb = F + (size_t)b * d * d;
+    if (ta > tc) {
+        for (int e = threadIdx.x; e < TILE_ELEMS; e += 256)
+            Fb[(size_t)(NB * ta + (e >> 6)) * d + NB * tc + (e & 63)] = 0.f;
+        return;
+    }
+    const int it = nt - 1 - ta, jt = nt - 1 - tc;
+    const double* Yjj = tile(G.Y, G, b, jt, jt);   // D_jt^T
+    if (it == jt) {
+        const double* Dj = G.D + ((size_t)b * nt + jt) * TILE_ELEMS;
+        for (int e = threadIdx.x; e < TILE_ELEMS; e += 256) Os[e >> 6][e & 63] = __ldcg(Dj + e);
+    } else if ((jt & 1) == 0 && it == jt + 1) {
+        const double* Yx = tile(G.Y, G, b, jt, jt + 1);
+        for (int e = threadIdx.x; e < TILE_ELEMS; e += 256) Os[e & 63][e >> 6] = __ldcg(Yx + e);
+    } else if ((jt & 1) == 0) {
+        tile_gemm_nt(tile(G.A, G, b, it, jt), Yjj, Ps, Qs, &Os[0][0], false, false, tile(G.A, G, b, it, jt + 1),
+                     tile(G.Y, G, b, jt, jt + 1), LD);
+    } else {
+        tile_gemm_nt(tile(G.A, G, b, it, jt), Yjj, Ps, Qs, &Os[0][0], false, false, nullptr, nullptr, LD);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < TILE_ELEMS; e += 256) {
+        const int ra = e >> 6, rc = e & 63;
+        const float v = (ta == tc && ra > rc) ? 0.f : (float)Os[63 - ra][63 - rc];
+        Fb[(size_t)(NB * ta + ra) * d + NB * tc + rc] = v;
+    }
+}
+
 }  // namespace
 
 namespace {
@@ -767,14 +844,15 @@ size_t factor_workspace_bytes(const FactorGroup* groups, int n) {
 }
 
 cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups, int n, void* ws, int* err,
-                          uint64_t wait_ns) {
-    if (n < 1 || n > MAX_GROUPS) return cudaErrorInvalidValue;
+                          uint64_t wait_ns, int form) {
+    if (n < 1 || n > MAX_GROUPS || (form != 0 && form != 1)) return cudaErrorInvalidValue;
     char* cur = (char*)ws;
     Dag g;
     g.ng = n;
     g.max_nt = 0;
     g.err = err;
     g.wait_ns = wait_ns;
+    g.inv = form == 0;
     size_t state_bytes = 2 * sizeof(unsigned long long);
     int pbase = 0;
     for (int k = 0; k < n; ++k) {
@@ -806,7 +884,7 @@ cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups
         G.stY = st_cur + tiles;
         st_cur += 2 * tiles;
         unsigned long long per = 0;
-        for (int st = 0; st <= G.nt; ++st) per += stage_total(G.nt, st);
+        for (int st = 0; st <= G.nt; ++st) per += stage_total(G.nt, st, g.inv);
         g.total += per * (unsigned long long)G.batch;
     }
 
@@ -816,7 +894,7 @@ cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups
         for (int k = 0; k < n; ++k) {
             const int nt = g.grp[k].nt;
             if (st > nt) continue;
-            tasks += stage_total(nt, st) * (unsigned long long)g.grp[k].batch;
+            tasks += stage_total(nt, st, g.inv) * (unsigned long long)g.grp[k].batch;
         }
         if (tasks >= (1ull << 31)) return cudaErrorInvalidValue;
     }
@@ -833,10 +911,24 @@ cudaError_t launch_factor(cudaStream_t s, int num_sms, const FactorGroup* groups
     if (grid > g.total) grid = g.total;
     fac_dag<<<(unsigned)grid, DAG_THREADS, smem, s>>>(g);
     clha_note_launches(1);
-    for (int k = 0; k < n; ++k) {
+    if (form == 0) {
+        for (int k = 0; k < n; ++k) {
+            const Grp& G = g.grp[k];
+            fac_store<<<dim3((unsigned)(G.nt * G.nt), G.batch), 256, 0, s>>>(G.Y, G.d, G.nt, groups[k].U);
+            clha_note_launches(1);
+        }
+        return cudaGetLastError();
+    }
+    if ((e = cudaFuncSetAttribute(fac_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PAIR_SMEM)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(fac_store_f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STORE_F_SMEM)) !=
+        cudaSuccess)
+        return e;
+    for (int k = 0; k < n; ++k) {   // d is a multiple of 128: nt is even
         const Grp& G = g.grp[k];
-        fac_store<<<dim3((unsigned)(G.nt * G.nt), G.batch), 256, 0, s>>>(G.Y, G.d, G.nt, groups[k].U);
-        clha_note_launches(1);
+        fac_pair<<<dim3((unsigned)(G.nt / 2), G.batch), 256, PAIR_SMEM, s>>>(G);
+        fac_store_f<<<dim3((unsigned)(G.nt * G.nt), G.batch), 256, STORE_F_SMEM, s>>>(G, groups[k].U);
+        clha_note_launches(2);
     }
     return cudaGetLastError();
 }

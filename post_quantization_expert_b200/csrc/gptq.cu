@@ -28,6 +28,11 @@
 // The grid and the code are decided with IEEE float32 operations (division and rounding to nearest
 // even), the same operations a float32 reference takes on the same current value.
 //
+// The factor may also be F, the block-scaled Cholesky factor of H_d (factor.cu): its diagonal blocks
+// are U's, so everything inside a block is unchanged, and the later blocks' lazy updates (and the
+// trailing updates) take W_hat - W of the earlier columns in place of their scaled errors e; the row
+// threads write it over e in the same shared buffer once the quarter product has read e.
+//
 // Column chunks. The tensor core's fp32 accumulator does not round each addition to nearest, so a
 // lazy update that sums the errors of many thousands of columns in TMEM drifts away from the exact
 // sum (enough, on long rows, to flip rounding decisions that float32 arithmetic rounding to nearest
@@ -86,6 +91,7 @@ struct GptqParams {
     const double* lambda;  // [n_u] damping of each factor, or null
     double* loss;          // [batch] |E|^2 - lambda |W_hat - W|^2, or null
     int* err;
+    int blk;               // U holds F, the block-scaled Cholesky factor of H_d (lazy operand W_hat - W)
 };
 
 __device__ __forceinline__ float to_tf32(float x) {
@@ -455,20 +461,39 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                 if (q == 3 && next_here) load_uq(cb + BLK);   // every row is past its last use of Uq
                 uint8_t* sah = smem + SA_OFF + t * 128;
                 uint8_t* sal = sah + SA_BYTES;
+                auto put_row = [&](const float (&v)[QW]) {
 #pragma unroll
-                for (int c = 0; c < QW / 4; ++c) {
-                    const float h0 = to_tf32(w[4 * c]), h1 = to_tf32(w[4 * c + 1]), h2 = to_tf32(w[4 * c + 2]),
-                                h3 = to_tf32(w[4 * c + 3]);
-                    const int off = ((c ^ (t & 7)) << 4);
-                    *reinterpret_cast<float4*>(sah + off) = make_float4(h0, h1, h2, h3);
-                    *reinterpret_cast<float4*>(sal + off) =
-                        make_float4(to_tf32(w[4 * c] - h0), to_tf32(w[4 * c + 1] - h1), to_tf32(w[4 * c + 2] - h2),
-                                    to_tf32(w[4 * c + 3] - h3));
+                    for (int c = 0; c < QW / 4; ++c) {
+                        const float h0 = to_tf32(v[4 * c]), h1 = to_tf32(v[4 * c + 1]), h2 = to_tf32(v[4 * c + 2]),
+                                    h3 = to_tf32(v[4 * c + 3]);
+                        const int off = ((c ^ (t & 7)) << 4);
+                        *reinterpret_cast<float4*>(sah + off) = make_float4(h0, h1, h2, h3);
+                        *reinterpret_cast<float4*>(sal + off) =
+                            make_float4(to_tf32(v[4 * c] - h0), to_tf32(v[4 * c + 1] - h1),
+                                        to_tf32(v[4 * c + 2] - h2), to_tf32(v[4 * c + 3] - h3));
+                    }
+                    fence_proxy_async_smem();
+                };
+                if (!p.blk || q < 3) {                   // e: the quarter product's operand
+                    put_row(w);
+                    if (q < 3) {
+                        tc::mbar_arrive(sreq);
+                        ++nq;
+                    }
                 }
-                fence_proxy_async_smem();
-                if (q < 3) {
-                    tc::mbar_arrive(sreq);
-                    ++nq;
+                if (more && p.blk) {
+                    // the later blocks' lazy operand under F: W_hat - W of the quarter (original W), written
+                    // over e once the quarter product has read it
+                    float wo[QW];
+                    load_w32(p, wrow + cb + QW * q, wo);
+#pragma unroll
+                    for (int c = 0; c < QW / 4; ++c)
+#pragma unroll
+                        for (int m = 0; m < 4; ++m)
+                            w[4 * c + m] = __fsub_rn(__fmul_rn(s, __fsub_rn((float)((codes[c] >> (8 * m)) & 255u), z)),
+                                                     wo[4 * c + m]);
+                    if (q < 3 && !tc::mbar_wait_bounded(sdone2, (nq - 1) & 1, abort_flag)) ok = false;
+                    put_row(w);
                 }
                 if (more) {
                     row_bar();                           // every row's errors are in the buffer
@@ -729,7 +754,8 @@ size_t quantize_workspace_bytes(int batch, int d_out, int d_in) {
 
 cudaError_t launch_quantize(cudaStream_t s, int num_sms, const float* U, int n_u, const void* W, int w_is_f32,
                             int batch, int d_out, int d_in, int bits, uint8_t* codes, float* scales, uint8_t* zeros,
-                            float* W_hat, const double* lambda, double* loss, void* ws, int* err) {
+                            float* W_hat, const double* lambda, double* loss, void* ws, int* err, int form) {
+    if (form != 0 && form != 1) return cudaErrorInvalidValue;
     char* cur = (char*)ws;
     const size_t wsz = (size_t)batch * d_out * d_in;
     float* Ehi = (float*)clha_carve(cur, wsz * sizeof(float));
@@ -763,7 +789,7 @@ cudaError_t launch_quantize(cudaStream_t s, int num_sms, const float* U, int n_u
     for (int c0 = 0; c0 < d_in; c0 += CHUNK) {
         const int c1 = c0 + CHUNK < d_in ? c0 + CHUNK : d_in;
         GptqParams p{U, n_u, W, w_is_f32, Wc, c0, c1, d_out, d_in, bits, codes, scales, zeros, W_hat, lambda, loss,
-                     err};
+                     err, form};
         gptq_tc<<<dim3(d_out / R, batch), kThreads, SMEM_BYTES, s>>>(tEhi, tElo, tUhi, tUlo, tQhi, tQlo, p);
         clha_note_launches(1);
         if (c1 < d_in) {   // fold this chunk's errors into the running weights of every later column

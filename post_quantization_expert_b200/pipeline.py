@@ -103,10 +103,12 @@ class DenseCalibration:
     """One weight W [d_out, d_in] shared by n_layers layers (no routing)."""
 
     def __init__(self, ctx: L.Context, d_out: int, d_in: int, n_layers: int, bits: int, damp_frac: float = 0.01,
-                 timer=NO_TIMER, keep_hcomb: bool = True):
+                 timer=NO_TIMER, keep_hcomb: bool = True, factor_form: int = L.FACTOR_BLOCK_CHOL):
         """keep_hcomb=False: the undamped aggregate is not written (GPTQ and its in-kernel loss need only
-        the damped one and lambda)."""
+        the damped one and lambda). factor_form: what self.U holds, F (the block-scaled Cholesky factor
+        of H_d, the default: half the factor's work) or U (H_d^-1 = U^T U)."""
         self.ctx, self.d_out, self.d_in, self.n_layers, self.bits, self.damp = ctx, d_out, d_in, n_layers, bits, damp_frac
+        self.form = factor_form
         self.timer = timer
         self.dev = dev = torch.device("cuda", ctx.device)
         self.acc = L.Accum(ctx, d_in, n_layers, 1)
@@ -133,11 +135,11 @@ class DenseCalibration:
             host = L.clha_aggregate(self.ctx, self.acc, 0, 1, MODES[mode], alpha, self.damp, self.H_comb, self.H_d,
                                     want_host=want_host, lambda_dev=self.lam)
         with t.span("factor"):
-            L.clha_factor(self.ctx, self.H_d, 1, self.d_in, self.U)
+            L.clha_factor_as(self.ctx, self.form, self.H_d, 1, self.d_in, self.U)
         with t.span("gptq"):
             L.clha_quantize(self.ctx, self.U, 1, W, 1, self.d_out, self.d_in, self.bits, self.q.codes, self.q.scales,
                             self.q.zeros, self.q.W_hat, lam=self.lam if with_loss else None,
-                            loss=self.loss_dev if with_loss else None)
+                            loss=self.loss_dev if with_loss else None, form=self.form)
         if with_loss and read_loss:
             self.q.loss = self.loss_dev.cpu().numpy()
         return host
@@ -200,15 +202,18 @@ class MoECalibration:
     def __init__(self, ctx: L.Context, n_layers: int, max_tokens: int, E: int, k: int, d_model: int, d_ff: int,
                  n_shared: int = 0, shared_dff: int = 0, bits_routed: int = 2, bits_shared: int = 3,
                  damp_frac: float = 0.01, timer=NO_TIMER, modes=("rt",), keep_hcomb: bool = False,
-                 unrouted_rtn: bool = True, fused_gather: bool = False):
+                 unrouted_rtn: bool = True, fused_gather: bool = False, factor_form: int = L.FACTOR_BLOCK_CHOL):
         """unrouted_rtn: an expert whose weighted Hessian aggregate is empty (never routed, or, for
         explicit alpha, never routed in the weighted layers) is quantized by round to nearest
         (H_d = I, loss 0) instead of failing. fused_gather: the expert inputs are read straight from
         the layer's X through the routing permutation (TMA gather4 in the Gram kernel, indexed rows
         in the activation) instead of from a packed copy (bf16 X only). Same results; off by
         default because four-row gather requests feed the tensor cores more slowly than the packed
-        copy costs (the Hessian phase of the E16 pair: 0.41 ms against 0.16 ms plus a 0.03 ms copy)."""
+        copy costs (the Hessian phase of the E16 pair: 0.41 ms against 0.16 ms plus a 0.03 ms copy).
+        factor_form: what the U_* buffers hold, F (the block-scaled Cholesky factor of each H_d, the
+        default) or U (H_d^-1 = U^T U)."""
         self.ctx, self.n_layers, self.E, self.k = ctx, n_layers, E, k
+        self.form = factor_form
         self.agg_flag = L.AGG_EMPTY_IDENTITY if unrouted_rtn else 0
         self.fused_gather = fused_gather
         self.timer = timer
@@ -364,13 +369,14 @@ class MoECalibration:
                 if ns:
                     groups += [(self.Hd_sin[a:b], b - a, dm, self.U_sin[a:b]),
                                (self.Hd_sdn[a * ns:b * ns], (b - a) * ns, sdff, self.U_sdn[a * ns:b * ns])]
-                L.clha_factor_groups(ctx, groups)
+                L.clha_factor_groups(ctx, groups, self.form)
         br, bs = self.bits_routed, self.bits_shared
         for i, m in zip(idx, modes):
             r = self.res[m]
             es, ss = slice(i * E, (i + 1) * E), slice(i * ns, (i + 1) * ns)
             lb = self.loss_dev[i]
-            opt = (lambda lam, lo: dict(lam=lam, loss=lo)) if with_loss else (lambda lam, lo: {})
+            opt = ((lambda lam, lo: dict(lam=lam, loss=lo, form=self.form)) if with_loss else
+                   (lambda lam, lo: dict(form=self.form)))
             with t.span("gptq"):
                 q = r.qgu
                 L.clha_quantize(ctx, self.U_in[es], E, w.Wgu, 2 * E, dff, dm, br, q.codes, q.scales, q.zeros, q.W_hat,

@@ -13,16 +13,18 @@ and checks:
   * counting a two-level task as two, the graph applies the plain blocked algorithm's updates;
   * a model of the in-order ticket protocol (W CTAs, each holding a running task and the next
     number it has taken, a finished task released at once) always drains, for several W.
+The same checks run on the Cholesky-only graph of the block-scaled factor F (classes F, Q and FQ
+empty): L final, no Y tile beyond the diagonal tasks' touched.
 """
 import random
 
 import pytest
 
 
-def stage_counts(nt, s):
+def stage_counts(nt, s, inv=True):
     """Tasks per problem in stage s by class: [lookahead G(i,m+1,m), P(m+1), F(j,m), one-level Q,
     two-level FQ (odd m), bulk G (even m: the column m+2, one level; odd m: FG over j >= m+2, levels
-    m-1 and m), S(i,m+1)] (stage 0: P(0), S(i,0))."""
+    m-1 and m), S(i,m+1)] (stage 0: P(0), S(i,0)). inv=False: the Cholesky only (F, Q, FQ empty)."""
     n = [0] * 7
     if s == 0:
         n[1], n[6] = 1, nt - 1
@@ -41,6 +43,8 @@ def stage_counts(nt, s):
         n[4] = m * R1
         n[5] = (R - 1) * R // 2 if R >= 1 else 0
     n[6] = R1
+    if not inv:
+        n[2] = n[3] = n[4] = 0
     return n
 
 
@@ -73,10 +77,10 @@ def decode(nt, s, c, local):
     return ("S", s, s + 1 + local, s)
 
 
-def tasks(nt):
+def tasks(nt, inv=True):
     out = []
     for s in range(nt + 1):
-        for c, cnt in enumerate(stage_counts(nt, s)):
+        for c, cnt in enumerate(stage_counts(nt, s, inv)):
             out += [decode(nt, s, c, local) for local in range(cnt)]
     return out
 
@@ -104,10 +108,11 @@ def _levels(t):
     return 2 if t[0] in ("FG", "FQ") else 1
 
 
+@pytest.mark.parametrize("inv", [True, False])
 @pytest.mark.parametrize("nt", list(range(1, 40)))
-def test_numbering_is_topological_and_complete(nt):
+def test_numbering_is_topological_and_complete(nt, inv):
     state = {}
-    for t in tasks(nt):
+    for t in tasks(nt, inv):
         ins, outs = deps(t)
         for key in ins:
             assert state.get(key[:3], 0) >= key[3], (t, key, state.get(key[:3], 0))
@@ -117,7 +122,10 @@ def test_numbering_is_topological_and_complete(nt):
     for i in range(nt):
         for j in range(i + 1):
             assert state[("A", i, j)] == j + 1
-            assert state[("Y", j, i)] == i - j + 1
+            if inv:
+                assert state[("Y", j, i)] == i - j + 1
+            else:
+                assert state.get(("Y", j, i), 0) == (1 if i == j else 0)
 
 
 @pytest.mark.parametrize("nt", [1, 2, 5, 16, 128])
@@ -128,10 +136,14 @@ def test_level_updates_match_the_one_level_graph(nt):
                 for m in range(nt) for R in [nt - 1 - m])
     assert sum(_levels(t) for t in tasks(nt)) == plain
     assert len(tasks(nt)) == sum(sum(stage_counts(nt, s)) for s in range(nt + 1))
+    # the Cholesky alone: sum_m (1 + 2R + (R - 1) R / 2 + R) one-level tile updates (P, S, G)
+    chol = sum(1 + 2 * R + ((R - 1) * R // 2 if R >= 1 else 0) for m in range(nt) for R in [nt - 1 - m])
+    assert sum(_levels(t) for t in tasks(nt, False)) == chol
 
 
+@pytest.mark.parametrize("inv", [True, False])
 @pytest.mark.parametrize("n_cta", [1, 2, 7, 64])
-def test_in_order_ticket_protocol_drains(n_cta):
+def test_in_order_ticket_protocol_drains(n_cta, inv):
     """Several problems of two sizes interleaved (stage by stage, as the kernel numbers them); CTAs
     take numbers in order, each holds at most its running task and its next number, and a task
     starts only when its inputs are final. Random completion order; it must never stall."""
@@ -141,7 +153,7 @@ def test_in_order_ticket_protocol_drains(n_cta):
         for gi, (nt, batch) in enumerate(groups):
             if s > nt:
                 continue
-            for c, cnt in enumerate(stage_counts(nt, s)):
+            for c, cnt in enumerate(stage_counts(nt, s, inv)):
                 for local in range(cnt):
                     for b in range(batch):
                         numbered.append((gi, b, decode(nt, s, c, local)))

@@ -411,6 +411,47 @@ def test_factor_matches_oracle(ctx, d, batch):
         assert rel_fro(got, want) < 1e-6
 
 
+@pytest.mark.parametrize("d,batch", [(128, 1), (256, 5), (512, 3), (896, 2), (1408, 1)])
+def test_factor_block_form_matches_oracle(ctx, d, batch):
+    """F, the block-scaled Cholesky factor: one 128-block (its X tile only), an odd batch, and 4, 7 and
+    11 blocks; every problem against the oracle's float64 F (whose own pin is the OBS recurrence)."""
+    g = _gen(d + 1)
+    Hs = []
+    for b in range(batch):
+        A = torch.randn((d, d // 4), generator=g).double()
+        Hs.append((A @ A.T / (d // 4) + 0.05 * torch.eye(d, dtype=torch.float64)).float())
+    Hd = torch.stack(Hs).to(DEV)
+    F = torch.full_like(Hd, float("nan"))
+    L.clha_factor_as(ctx, L.FACTOR_BLOCK_CHOL, Hd, batch, d, F)
+    L.clha_check(ctx)
+    for b in range(batch):
+        got = F[b].double().cpu().numpy()
+        assert np.all(np.tril(got, -1) == 0)
+        assert rel_fro(got, O.factor_block_scaled(Hs[b].double().numpy())) < 1e-6
+
+
+def test_factor_block_form_groups(ctx):
+    """Three groups of different sizes in one Cholesky-only graph launch, each problem against the
+    oracle's F; an unknown form is rejected."""
+    specs = [(384, 3), (128, 2), (640, 2)]
+    groups, host = [], []
+    for gi, (d, batch) in enumerate(specs):
+        g = _gen(200 + gi)
+        Hs = []
+        for b in range(batch):
+            A = torch.randn((d, d // 4), generator=g).double()
+            Hs.append((A @ A.T / (d // 4) + 0.05 * torch.eye(d, dtype=torch.float64)).float())
+        groups.append((torch.stack(Hs).to(DEV), batch, d, torch.full((batch, d, d), float("nan"), device=DEV)))
+        host.append(Hs)
+    L.clha_factor_groups(ctx, groups, L.FACTOR_BLOCK_CHOL)
+    L.clha_check(ctx)
+    for (Hd, batch, d, F), Hs in zip(groups, host):
+        for b in range(batch):
+            assert rel_fro(F[b].double().cpu().numpy(), O.factor_block_scaled(Hs[b].double().numpy())) < 1e-6
+    with pytest.raises(L.ClhaError):
+        L.clha_factor_groups(ctx, groups, 2)
+
+
 def test_factor_groups_match_oracle_and_report_across_groups(ctx):
     """Three groups of different sizes in one graph launch; each problem against the oracle. Then a
     non-positive pivot in the last group's second problem: its index counts across the groups."""
@@ -504,14 +545,25 @@ def _H(d, seed, rank=None, damp=0.01):
     return H.numpy()
 
 
+@pytest.mark.parametrize("form", ["inv", "block"])
 @pytest.mark.parametrize("d_out,d_in,bits,wdt", [(256, 512, 2, torch.float32), (384, 1024, 3, torch.bfloat16),
-                                                   (128, 128, 4, torch.bfloat16), (256, 256, 8, torch.float32)])
-def test_quantize_matches_oracle_on_same_factor(ctx, d_out, d_in, bits, wdt):
+                                                   (128, 128, 4, torch.bfloat16), (256, 256, 8, torch.float32),
+                                                   (256, 1152, 4, torch.bfloat16)])
+def test_quantize_matches_oracle_on_same_factor(ctx, d_out, d_in, bits, wdt, form):
+    """GPTQ against the oracle's (the pages' recurrence with U). inv: both sides take the same float32 U.
+    block: the kernel takes float32 F and runs the lazy and trailing updates on W_hat - W, the oracle
+    the exact U. d_in = 1152: two full chunks of 512 columns and a ragged one of 128."""
     H = _H(d_in, d_in + bits)
     agg = O.aggregate([H], [2], "rt")
     U32 = np.ascontiguousarray(O.factor(agg["H_d"]), np.float32)
     W = (0.02 * torch.randn((d_out, d_in), generator=_gen(bits))).to(wdt)
-    Ud = torch.from_numpy(U32)[None].to(DEV)
+    if form == "block":
+        Ud = torch.from_numpy(np.ascontiguousarray(O.factor_block_scaled(agg["H_d"]), np.float32))[None].to(DEV)
+        U_or = O.factor(agg["H_d"])
+    else:
+        Ud = torch.from_numpy(U32)[None].to(DEV)
+        U_or = U32.astype(np.float64)
+    fcode = L.FACTOR_BLOCK_CHOL if form == "block" else L.FACTOR_INV_CHOL
     Wd = W[None].to(DEV).contiguous()
     codes = torch.empty((1, d_out, d_in), dtype=torch.uint8, device=DEV)
     scales = torch.empty((1, d_out, d_in // 128), device=DEV)
@@ -519,10 +571,11 @@ def test_quantize_matches_oracle_on_same_factor(ctx, d_out, d_in, bits, wdt):
     W_hat = torch.empty((1, d_out, d_in), device=DEV)
     lam = torch.tensor([agg["lam"]], dtype=torch.float64, device=DEV)
     loss = torch.full((1,), float("nan"), dtype=torch.float64, device=DEV)
-    L.clha_quantize(ctx, Ud, 1, Wd, 1, d_out, d_in, bits, codes, scales, zeros, W_hat, lam=lam, loss=loss)
-    wc, ws, wz, wh, wm = O.gptq(to64(W), U32.astype(np.float64), bits, 128, margins=True)
-    assert_codes(codes[0].cpu().numpy(), zeros[0].cpu().numpy(), dict(codes=wc, zeros=wz, margin=wm),
-                 (d_out, d_in, bits), bar=CONFIG_BAR)
+    L.clha_quantize(ctx, Ud, 1, Wd, 1, d_out, d_in, bits, codes, scales, zeros, W_hat, lam=lam, loss=loss,
+                    form=fcode)
+    wc, ws, wz, wh, wm = O.gptq(to64(W), U_or, bits, 128, margins=True)
+    print("codes", form, assert_codes(codes[0].cpu().numpy(), zeros[0].cpu().numpy(),
+                                      dict(codes=wc, zeros=wz, margin=wm), (d_out, d_in, bits, form), bar=CONFIG_BAR))
     # first group of every row: identical inputs, so the grid is bit-identical
     np.testing.assert_array_equal(scales[0, :, 0].cpu().numpy(), ws[:, 0])
     np.testing.assert_array_equal(zeros[0, :, 0].cpu().numpy(), wz[:, 0])
@@ -538,34 +591,48 @@ def test_quantize_matches_oracle_on_same_factor(ctx, d_out, d_in, bits, wdt):
     assert torch.equal(W_hat[0], s * (q - z))
 
 
-def test_quantize_diagonal_hessian_is_rtn_bit_exact(ctx):
-    d_out, d_in = 256, 384
+@pytest.mark.parametrize("form", ["inv", "block"])
+def test_quantize_diagonal_hessian_is_rtn_bit_exact(ctx, form):
+    """A diagonal H makes U and F the same diagonal matrix: no column moves another, GPTQ is round to
+    nearest in either form (d_in = 640: two chunks, so the trailing update adds exact zeros)."""
+    d_out, d_in = 256, 640
     W = (0.02 * torch.randn((d_out, d_in), generator=_gen(3))).to(torch.bfloat16)
     H = np.diag(np.linspace(0.5, 2.0, d_in))
-    U = O.factor(O.aggregate([H], [2], "rt")["H_d"])
+    Hd = O.aggregate([H], [2], "rt")["H_d"]
+    U = O.factor(Hd)
+    np.testing.assert_allclose(O.factor_block_scaled(Hd), U, rtol=1e-14)
     Ud = torch.from_numpy(np.ascontiguousarray(U, np.float32))[None].to(DEV)
     codes = torch.empty((1, d_out, d_in), dtype=torch.uint8, device=DEV)
     scales = torch.empty((1, d_out, d_in // 128), device=DEV)
     zeros = torch.empty((1, d_out, d_in // 128), dtype=torch.uint8, device=DEV)
-    L.clha_quantize(ctx, Ud, 1, W[None].to(DEV).contiguous(), 1, d_out, d_in, 3, codes, scales, zeros, None)
+    L.clha_quantize(ctx, Ud, 1, W[None].to(DEV).contiguous(), 1, d_out, d_in, 3, codes, scales, zeros, None,
+                    form=L.FACTOR_BLOCK_CHOL if form == "block" else L.FACTOR_INV_CHOL)
     wc, ws, wz, _ = O.gptq(to64(W), U.astype(np.float32).astype(np.float64), 3, 128)
     np.testing.assert_array_equal(codes[0].cpu().numpy(), wc)
     np.testing.assert_array_equal(scales[0].cpu().numpy(), ws)
     np.testing.assert_array_equal(zeros[0].cpu().numpy(), wz)
 
 
-def test_quantize_batched_shared_factor(ctx):
+@pytest.mark.parametrize("form", ["inv", "block"])
+def test_quantize_batched_shared_factor(ctx, form):
     """n_u = 2: problems 0, 2 use factor 0 and problems 1, 3 factor 1 (gate and up stacked share one)."""
-    d_out, d_in, bits = 128, 256, 3
-    Us = [np.ascontiguousarray(O.factor(O.aggregate([_H(d_in, s)], [2], "rt")["H_d"]), np.float32) for s in (1, 2)]
+    d_out, d_in, bits = 128, 768, 3
+    Hds = [O.aggregate([_H(d_in, s)], [2], "rt")["H_d"] for s in (1, 2)]
+    Us = [np.ascontiguousarray(O.factor(h), np.float32) for h in Hds]
     W = (0.02 * torch.randn((4, d_out, d_in), generator=_gen(4))).to(torch.bfloat16)
-    Ud = torch.from_numpy(np.stack(Us)).to(DEV)
+    if form == "block":
+        Ud = torch.from_numpy(np.stack([np.ascontiguousarray(O.factor_block_scaled(h), np.float32) for h in Hds]))
+        Uor = [O.factor(h) for h in Hds]
+    else:
+        Ud = torch.from_numpy(np.stack(Us))
+        Uor = [u.astype(np.float64) for u in Us]
     codes = torch.empty((4, d_out, d_in), dtype=torch.uint8, device=DEV)
     scales = torch.empty((4, d_out, d_in // 128), device=DEV)
     zeros = torch.empty((4, d_out, d_in // 128), dtype=torch.uint8, device=DEV)
-    L.clha_quantize(ctx, Ud, 2, W.to(DEV), 4, d_out, d_in, bits, codes, scales, zeros, None)
+    L.clha_quantize(ctx, Ud.to(DEV), 2, W.to(DEV), 4, d_out, d_in, bits, codes, scales, zeros, None,
+                    form=L.FACTOR_BLOCK_CHOL if form == "block" else L.FACTOR_INV_CHOL)
     for b in range(4):
-        wc, _, wz, _, wm = O.gptq(to64(W[b]), Us[b % 2].astype(np.float64), bits, 128, margins=True)
+        wc, _, wz, _, wm = O.gptq(to64(W[b]), Uor[b % 2], bits, 128, margins=True)
         assert_codes(codes[b].cpu().numpy(), zeros[b].cpu().numpy(), dict(codes=wc, zeros=wz, margin=wm), b,
                      bar=CONFIG_BAR)
 

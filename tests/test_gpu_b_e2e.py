@@ -17,12 +17,12 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def _dense_case(ctx, cfg, **over):
+def _dense_case(ctx, cfg, form=L.FACTOR_BLOCK_CHOL, **over):
     wl = workload(cfg, "cpu", **over)
     s = wl.spec
     W = wl.dense_weight()
     Xs = [wl.x(l) for l in range(s.n_layers)]
-    cal = DenseCalibration(ctx, s.d_out, s.d_model, s.n_layers, s.bits_routed, s.damp_frac)
+    cal = DenseCalibration(ctx, s.d_out, s.d_model, s.n_layers, s.bits_routed, s.damp_frac, factor_form=form)
     for l, X in enumerate(Xs):
         cal.collect(l, X.to(DEV))
     alpha, lam = cal.quantize(W.to(DEV), "rt", want_host=True)
@@ -31,9 +31,12 @@ def _dense_case(ctx, cfg, **over):
     return cal, want, alpha, lam, W
 
 
-def test_dense_two_layer_fp32_workload(ctx):
-    """The dense fp32 workload: W 256x512 shared by two layers of 1000 and 1024 tokens, 2-bit."""
-    cal, want, alpha, lam, W = _dense_case(ctx, 1)
+@pytest.mark.parametrize("form", ["block", "inv"])
+def test_dense_two_layer_fp32_workload(ctx, form):
+    """The dense fp32 workload: W 256x512 shared by two layers of 1000 and 1024 tokens, 2-bit; GPTQ with
+    either factor form against the oracle's (the pages' recurrence with U)."""
+    block = form == "block"
+    cal, want, alpha, lam, W = _dense_case(ctx, 1, L.FACTOR_BLOCK_CHOL if block else L.FACTOR_INV_CHOL)
     S, cnt = cal.acc.buffers()
     assert cnt[:, 0].tolist() == [1000, 1024]
     for l in range(2):
@@ -41,7 +44,8 @@ def test_dense_two_layer_fp32_workload(ctx):
     np.testing.assert_allclose(alpha[0], [1000 / 2024, 1024 / 2024], rtol=1e-15)
     np.testing.assert_allclose(lam[0], want["lam"], rtol=1e-5)
     assert rel_fro(cal.H_comb[0].double().cpu().numpy(), want["H_comb"]) < 1e-4
-    assert rel_fro(cal.U[0].double().cpu().numpy(), want["U"]) < 1e-4
+    want_factor = O.factor_block_scaled(want["H_d"]) if block else want["U"]
+    assert rel_fro(cal.U[0].double().cpu().numpy(), want_factor) < 1e-4
     print("dense c1 codes", assert_codes(cal.q.codes[0].cpu().numpy(), cal.q.zeros[0].cpu().numpy(), want, "dense",
                                          bar=CONFIG_BAR))
     assert abs(cal.q.loss[0] - want["loss"]) <= 1e-3 * want["loss"]

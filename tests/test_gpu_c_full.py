@@ -23,8 +23,9 @@ import pytest
 import torch
 
 import oracle as O
-from helpers import (CONFIG_BAR, H_INPUT_BAR, MATRIX_BAR, CodeTally, assert_codes, certify_h, rel_fro,
-                     sym_from_upper, to64)
+from helpers import (CONFIG_BAR, H_INPUT_BAR, MATRIX_BAR, CodeTally, assert_codes, certify_h, check_loss,
+                     rel_fro, sym_from_upper, to64)
+from post_quantization_expert_b200.clha import FACTOR_BLOCK_CHOL
 from post_quantization_expert_b200.pipeline import DenseCalibration, MoECalibration, stack_weights
 from synth import workload
 
@@ -32,9 +33,10 @@ pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 DEV = "cuda:0"
 
 
-def _check_experts(ref, out, S_accs, E, what, tally, h_gpu=None):
+def _check_experts(ref, out, S_accs, E, what, tally, weights, h_gpu=None):
     """Hessians, certified codes and losses of every expert in an oracle result against the GPU's.
     S_accs: (S_in, S_dn, S_sdn) accumulator buffers; the always-active experts share input slot E.
+    weights: (kind, e) -> (Wg, Wu, Wd) as float64 arrays, for the loss bar (check_loss).
     A down-projection Hessian more than 1e-4 from the oracle's is accepted only when h_gpu (the GPU's
     h of that routed expert and layer) shows why: its Gram equals the GPU's Hessian to 1e-4, every h
     element that differs from the oracle's is one bf16 step away and at most 0.1 % differ, and the
@@ -60,11 +62,13 @@ def _check_experts(ref, out, S_accs, E, what, tally, h_gpu=None):
                       f"({frac:.2e} of h, largest rounding margin {worst:.3g})")
         qs = ({"gate": out.qg, "up": out.qu, "down": out.qd} if kind == "r" else
               {"gate": out.sg, "up": out.su, "down": out.sd})
-        for name, q in qs.items():
+        for wi, (name, q) in enumerate(qs.items()):
             bar = H_INPUT_BAR if name == "down" and h_moved else MATRIX_BAR
-            tally.add(q.codes[e].cpu().numpy(), q.zeros[e].cpu().numpy(), r[name], (what, kind, e, name, r["n"]), bar)
-        got = sum(qs[n].loss[e] for n in qs)
-        assert abs(got - r["loss"]) <= 1e-3 * r["loss"], (what, kind, e, got, r["loss"])
+            codes, zeros = q.codes[e].cpu().numpy(), q.zeros[e].cpu().numpy()
+            tally.add(codes, zeros, r[name], (what, kind, e, name, r["n"]), bar)
+            H = r["H_down" if name == "down" else "H_in"]["H_comb"]
+            check_loss(q.loss[e], weights[(kind, e)][wi], to64(q.W_hat[e]), codes, zeros, r[name], H,
+                       (what, kind, e, name))
 
 
 def test_stack_of_12_pairs_full_size(ctx):
@@ -104,7 +108,9 @@ def test_stack_of_12_pairs_full_size(ctx):
                                          for e, r in enumerate(routed)],
                                         [tuple(to64(t) for t in sh) for sh in shared], experts,
                                         s.bits_routed, s.bits_shared, s.group, mode, s.damp_frac)
-            _check_experts(ref, cal.res[mode], S_accs, s.E, (gi, s.drifts[gi], mode), tally)
+            wts = {("r", e): tuple(to64(t) for t in routed[e]) for e in experts}
+            wts.update({("s", i): tuple(to64(t) for t in sh) for i, sh in enumerate(shared)})
+            _check_experts(ref, cal.res[mode], S_accs, s.E, (gi, s.drifts[gi], mode), tally, wts)
         del cal, w
         torch.cuda.empty_cache()
     tally.check()
@@ -154,7 +160,9 @@ def test_moe_E64_top6_shared_full_size(ctx):
     assert len(ref["experts"]) == 16 + s.n_shared
     S_accs = (cal.acc_in.buffers()[0], cal.acc_dn.buffers()[0], cal.acc_sdn.buffers()[0])
     tally = CodeTally("E64")
-    _check_experts(ref, cal.res["rt"], S_accs, s.E, "E64", tally, h_gpu)
+    wts = {("r", e): routed64[e] for e in checked}
+    wts.update({("s", i): tuple(to64(t) for t in sh) for i, sh in enumerate(shared)})
+    _check_experts(ref, cal.res["rt"], S_accs, s.E, "E64", tally, wts, h_gpu)
     tally.check()
 
 
@@ -190,6 +198,21 @@ def _gptq_consistency(W, W_hat, codes, scales, zeros, U, rows, bits):
     return agree / total, grid_ok / groups
 
 
+def _r_from_f(F, block=128):
+    """R (upper, H_d = R R^T) from the block-scaled factor F, in float64 on the device: the diagonal
+    blocks of F are U's, U_bb = R_bb^-1, and F_ab = R_ab U_bb above them."""
+    F = F.double()
+    d = F.shape[0]
+    R = torch.zeros_like(F)
+    eye = torch.eye(block, dtype=torch.float64, device=F.device)
+    for b0 in range(0, d, block):
+        b1 = b0 + block
+        Rbb = torch.linalg.solve_triangular(F[b0:b1, b0:b1], eye, upper=True)
+        R[b0:b1, b0:b1] = Rbb
+        R[:b0, b0:b1] = F[:b0, b0:b1] @ Rbb
+    return R
+
+
 def test_dense_stress_shape_full_size(ctx):
     wl = workload(5, DEV)
     s = wl.spec
@@ -217,28 +240,36 @@ def test_dense_stress_shape_full_size(ctx):
         assert rel_fro(full_blk, sub_ref[l]) < 1e-4, l
     agg_ref = O.aggregate(sub_ref, [n] * L, "rt")
     assert rel_fro(cal.H_comb[0][Jt][:, Jt].double().cpu().numpy(), agg_ref["H_comb"]) < 1e-4
-    # factor, trailing block: U[t:, t:] = R22^-1 depends only on H_d[t:, t:] (H_d = R R^T, R upper)
+    # factor (the block-scaled Cholesky factor F), trailing block: F[t:, t:] depends only on H_d[t:, t:]
+    # (H_d = R R^T, R upper, so R[t:, t:] is the factor of H_d[t:, t:]; t a multiple of 128)
+    assert cal.form == FACTOR_BLOCK_CHOL
     t = d - 2048
     Hd_tail = cal.H_d[0][t:, t:].double().cpu().numpy()
-    assert rel_fro(cal.U[0][t:, t:].double().cpu().numpy(), O.factor(Hd_tail)) < 1e-6
-    # factor: U^T U H_d v = v on random vectors (float64 products of the float32 outputs)
-    U = cal.U[0].double()
+    assert rel_fro(cal.U[0][t:, t:].double().cpu().numpy(), O.factor_block_scaled(Hd_tail)) < 1e-6
+    assert torch.count_nonzero(torch.tril(cal.U[0], -1)) == 0
+    # R from F (float64 on the device): R_bb = F_bb^-1, R_ab = F_ab R_bb; then R R^T v = H_d v
+    R = _r_from_f(cal.U[0])
     Hd = cal.H_d[0].double()
     v = torch.randn((d, 4), dtype=torch.float64, device=DEV, generator=torch.Generator(DEV).manual_seed(1))
+    assert (torch.linalg.norm(R @ (R.T @ v) - Hd @ v) / torch.linalg.norm(Hd @ v)).item() < 1e-5
+    # U = R^-1; U^T U H_d v = v (float32-rounded F, cond(H_d) ~ 1e4)
+    U = torch.linalg.solve_triangular(R, torch.eye(d, dtype=torch.float64, device=DEV), upper=True)
+    del R
     res = U.T @ (U @ (Hd @ v)) - v
-    assert (torch.linalg.norm(res) / torch.linalg.norm(v)).item() < 1e-2   # fp32-rounded U, cond(H_d) ~ 1e4
-    assert torch.all(torch.diagonal(U) > 0) and torch.count_nonzero(torch.tril(cal.U[0], -1)) == 0
+    assert (torch.linalg.norm(res) / torch.linalg.norm(v)).item() < 1e-2
+    assert torch.all(torch.diagonal(U) > 0)
     # GPTQ: sampled rows consistent with the recurrence
     rows = g.choice(s.d_out, 6, replace=False)
     agree, grid_ok = _gptq_consistency(W, cal.q.W_hat[0], cal.q.codes[0], cal.q.scales[0], cal.q.zeros[0], U, rows,
                                        s.bits_routed)
     assert agree >= 0.999 and grid_ok >= 0.99, (agree, grid_ok)
+    U64 = U.cpu().numpy()
     del U, Hd
     torch.cuda.empty_cache()
-    # GPTQ stage-wise: the oracle's GPTQ of 16 sampled rows under the GPU's factor (rows are independent)
+    # GPTQ stage-wise: the oracle's GPTQ of 16 sampled rows under the GPU's factor (as U, rebuilt from F
+    # in float64; rows are independent)
     rows = np.sort(g.choice(s.d_out, 16, replace=False))
     rt = torch.from_numpy(rows).to(DEV)
-    U64 = cal.U[0].cpu().numpy().astype(np.float64)
     wc, ws, wz, wh, wm = O.gptq(to64(W[rt]), U64, s.bits_routed, s.group, 128, margins=True)
     del U64
     c = assert_codes(cal.q.codes[0][rt].cpu().numpy(), cal.q.zeros[0][rt].cpu().numpy(),

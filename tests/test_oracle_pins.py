@@ -198,6 +198,37 @@ def test_factor_inverse_cholesky(d):
     np.testing.assert_allclose(U, np.linalg.inv(R), rtol=1e-9, atol=1e-12)
 
 
+@pytest.mark.parametrize("d,block", [(64, 16), (96, 32), (130, 64), (128, 128)])
+def test_factor_block_scaled_gives_the_obs_lazy_update(d, block):
+    """F against the textbook OBS recurrence, which holds no factor at all: quantize column j (any
+    rounding rule will do), then move the remaining columns by -(w_j - w_hat_j) / [H_F^-1]_00 times the
+    first row of H_F^-1, F the columns not yet quantized. At the start of every block the recurrence's
+    current values equal W_b + (W - W_hat)_a F_ab, the earlier columns a < b entering only through
+    F; inside a block F is U. A transposed F, a wrong sign, a block of R left unscaled or a diagonal
+    block of R instead of U fails it."""
+    H = _spd(d, rank=d // 2, seed=d + 7, damp=0.05)
+    W = 0.02 * RNG.standard_normal((5, d))
+    F = O.factor_block_scaled(H, block)
+    assert np.allclose(np.tril(F, -1), 0)
+    cur, W_hat = np.zeros_like(W), np.zeros_like(W)
+    for r in range(W.shape[0]):
+        w = W[r].copy()
+        for j in range(d):
+            if j % block == 0:
+                cur[r, j:j + block] = w[j:j + block]
+            W_hat[r, j] = np.round(w[j] * 64) / 64
+            rest = np.arange(j, d)
+            Hinv = np.linalg.inv(H[np.ix_(rest, rest)])
+            w[j:] -= (w[j] - W_hat[r, j]) / Hinv[0, 0] * Hinv[0, :]
+    D = W - W_hat
+    U = O.factor(H)
+    for b0 in range(0, d, block):
+        b1 = min(d, b0 + block)
+        np.testing.assert_allclose(W[:, b0:b1] + D[:, :b0] @ F[:b0, b0:b1], cur[:, b0:b1], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(F[b0:b1, b0:b1], U[b0:b1, b0:b1], rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(O.factor_block_scaled(H, d), U, rtol=1e-9, atol=1e-12)   # one block: F = U
+
+
 # ------------------------------------------------------------------------------------ grid + GPTQ
 def test_grid_golden(golden_dir):
     for line in _golden_lines(os.path.join(golden_dir, "grid_minmax_examples.txt")):
