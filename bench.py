@@ -332,7 +332,8 @@ def run_ours(args, world, rank, local):
         cols_per_step = cal.columns() * len(modes) / world      # the pair's columns, per rank on average
     else:
         cal = qcal = MoECalibration(ctx, 2, max(s.tokens), s.E, s.k, s.d_model, s.d_ff, 0, 0, s.bits_routed,
-                                    s.bits_shared, s.damp_frac, timer=timer, modes=modes)
+                                    s.bits_shared, s.damp_frac, timer=timer, modes=modes,
+                                    factor_form=FORMS[args.factor_form])
         wq = w
         cols_per_step = cal.columns() * len(modes)
     Xd = [x.to(dev) for x in X]
@@ -591,7 +592,8 @@ def run_dense(args, world, rank, local):
     nl, n, d, d_out = s.n_layers, s.tokens[0], s.d_model, s.d_out
     ctx = L.Context(local)
     timer = PhaseTimer(ctx.stream)
-    cal = DenseCalibration(ctx, d_out, d, nl, s.bits_routed, s.damp_frac, timer=timer, keep_hcomb=False)
+    cal = DenseCalibration(ctx, d_out, d, nl, s.bits_routed, s.damp_frac, timer=timer, keep_hcomb=False,
+                           factor_form=FORMS[args.factor_form])
     W = wl.dense_weight()
     Xd = [wl.x(l, cache=False) for l in range(nl)]
     torch.cuda.synchronize()
@@ -934,7 +936,7 @@ def main():
                     help="sweep: strengths of the per-layer expert preference")
     ap.add_argument("--shape", nargs="+", default=[], help="kernel workload shapes, e.g. 65536x4096")
     ap.add_argument("--factor-form", choices=tuple(FORMS), default="block",
-                    help="factor and gptq kernel workloads: U (inv) or the block-scaled Cholesky factor (block)")
+                    help="GPTQ's factor: U (inv) or the block-scaled Cholesky factor of H (block, the default)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

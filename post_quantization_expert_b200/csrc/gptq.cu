@@ -31,7 +31,8 @@
 // The factor may also be F, the block-scaled Cholesky factor of H_d (factor.cu): its diagonal blocks
 // are U's, so everything inside a block is unchanged, and the later blocks' lazy updates (and the
 // trailing updates) take W_hat - W of the earlier columns in place of their scaled errors e; the row
-// threads write it over e in the same shared buffer once the quarter product has read e.
+// threads write it over e in the same shared buffer once the quarter product has read e, and the TMA
+// store takes it from there.
 //
 // Column chunks. The tensor core's fp32 accumulator does not round each addition to nearest, so a
 // lazy update that sums the errors of many thousands of columns in TMEM drifts away from the exact
@@ -483,7 +484,8 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                 }
                 if (more && p.blk) {
                     // the later blocks' lazy operand under F: W_hat - W of the quarter (original W), written
-                    // over e once the quarter product has read it
+                    // over e once the quarter product has read it (a second buffer does not fit in shared
+                    // memory; stores straight from registers to global memory measured slower)
                     float wo[QW];
                     load_w32(p, wrow + cb + QW * q, wo);
 #pragma unroll
