@@ -75,6 +75,13 @@ def factor_work(d: int, form: int) -> int:
     return 2 * d ** 3 // 3 if form == FORMS["inv"] else d ** 3 // 3 + 96 * d * d
 
 
+def gram_kernel(d: int) -> str:
+    """The kernel of one dense Gram: pairs of SMs from d = 4096 (the library's threshold)."""
+    if d >= 4096:
+        return "syrk_bf16_pair (tcgen05 kind::f16, cta_group::2: 256x256 tiles on SM pairs)"
+    return "syrk_bf16_tc (tcgen05 kind::f16)"
+
+
 def factor_kernels(form: int) -> str:
     if form == FORMS["inv"]:
         return "fac_load + fac_dag + fac_store (fp64 tile-task graph, mma.sync m8n8k4 f64)"
@@ -683,7 +690,7 @@ def run_dense(args, world, rank, local):
     gptq_flops = d_out * d * d
     agg_bytes = nl * (d * (d + 1) // 2) * 4 + d * d * 4     # every layer's upper triangle read, H_d written
     kernels = {
-        "hessian": ("tensor", hess_flops / 1e12, sustained, "TFLOP/s", "syrk_bf16_tc (tcgen05 kind::f16)"),
+        "hessian": ("tensor", hess_flops / 1e12, sustained, "TFLOP/s", gram_kernel(d)),
         "factor": ("alu", factor_flops / 1e12, alu["fp64_tflops"], "TFLOP/s", factor_kernels(cal.form)),
         "gptq": ("tensor", gptq_flops / 1e12, alu["tf32x3_tflops"], "TFLOP/s",
                  "gptq_tc + gptq_trail (column sweep in fp32; lazy and trailing updates on tcgen05 kind::tf32, "
@@ -862,7 +869,7 @@ def run_kernel(args):
             acc = L.Accum(ctx, d, 1, 1)
             fn = lambda: L.clha_collect(ctx, acc, 0, X, n, d)
             work, unit, bound, peak = n * d * (d + 1) / 1e12, "TFLOP/s", "tensor", peaks["bf16_tflops"]
-            kname = "syrk_bf16_tc"
+            kname = gram_kernel(d)
         else:
             if args.workload == "gptq":
                 B, d_out, d = dims

@@ -28,6 +28,7 @@
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int kPairMinD = 4096;   // one dense Gram with d at least this runs on pairs of SMs (syrk_bf16_pair)
 // 64-token blocks per TMEM accumulation. The tensor core's fp32 accumulator does not round each add
 // to nearest, so a long sum drifts (linearly in its length); chunk sums are added into S by TMA
 // reduce-add, which rounds to nearest. Short chunks where the Hessian is small (an expert's d_model or
@@ -298,6 +299,218 @@ __global__ void __launch_bounds__(kThreads, 1) syrk_bf16_tc(const __grid_constan
     if (threadIdx.x == 0 && *abort_flag) clha_record_error(p.err, CLHA_ERR_TIMEOUT, blockIdx.x, 0, KID_COLLECT);
 }
 
+// ------------------------------------------------------------------------------ pairs of SMs
+// The dense Gram at large d on CTA pairs (a cluster of two CTAs sharing each tcgen05.mma,
+// cta_group::2): output tiles of 256 x 256, CTA k of a pair holding rows 128k .. 128k+127 of the tile
+// (its half of A) and columns 128k .. 128k+127 (its half of B) in its shared memory, and its 128 rows
+// of each accumulator in its TMEM. For the same tensor-core work a stage then carries 32 KB per SM
+// instead of 48 KB, so six stages fit against four, and each SM's TMA traffic per flop falls by a
+// third. Roles as in syrk_bf16_tc, on both CTAs, except that only the leader (rank 0) issues MMAs
+// (M = 256, N = 256) and waits on the operand barriers, which count both CTAs' copies; its commits
+// reach both CTAs' stage and accumulator barriers (multicast), and both CTAs' epilogue warps arrive
+// on the leader's accumulator-empty barrier. Tile rows at or past d (the second half of the last row
+// tile when d is not a multiple of 256) are computed on zero-filled operands and never written.
+constexpr int P_STAGES = 6;
+constexpr int P_HALF = 128;                      // rows of A and columns of B per CTA
+constexpr int P_A_BYTES = P_HALF * BK * 2;       // 16 KB
+constexpr int P_STAGE_BYTES = 2 * P_A_BYTES;     // A half + B half
+constexpr int P_BAR_OFF = P_STAGES * P_STAGE_BYTES;
+constexpr int P_STG_OFF = P_BAR_OFF + 1024;
+constexpr int P_SMEM_BYTES = P_STG_OFF + STG_BYTES + 1024;
+constexpr int P_TILE = 256;
+constexpr uint32_t IDESC_PAIR = tc::idesc_f32acc(1 /*bf16*/, 1 /*A MN-major*/, 1 /*B MN-major*/, 256, 256);
+static_assert(P_SMEM_BYTES <= 232448, "shared memory");
+
+// Pair tiles in bands of 8 tile columns, row-major inside a band: the pairs working at one time share
+// about sqrt(pairs) row blocks and 8 column blocks of X, so a block is read from DRAM once for several
+// tiles (on 65536 x 28672, 163 GB of DRAM reads per call against 232 GB column after column).
+__device__ __forceinline__ void decode_pair_tile(int t, int& R, int& C, int nC) {
+    constexpr int WB = 8;
+    int cmin = 0, cmax = 0;
+    for (;;) {
+        cmax = min(nC, cmin + WB) - 1;
+        const int nb = (cmax + 1) * (cmax + 2) / 2 - cmin * (cmin + 1) / 2;
+        if (t < nb) break;
+        t -= nb;
+        cmin += WB;
+    }
+    for (R = 0;; ++R) {
+        const int c0 = max(R, cmin);
+        const int cnt = cmax - c0 + 1;
+        if (t < cnt) { C = c0 + t; return; }
+        t -= cnt;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) syrk_bf16_pair(const __grid_constant__ CUtensorMap tmX,
+                                                              const __grid_constant__ CUtensorMap tmS, SyrkParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P_BAR_OFF);
+    const uint32_t full0 = tc::smem_u32(bars);            // [P_STAGES] leader: both CTAs' copies of a stage
+    const uint32_t empty0 = full0 + 8 * P_STAGES;         // [P_STAGES] each CTA: its stage may be refilled
+    const uint32_t tfull0 = empty0 + 8 * P_STAGES;        // [2] each CTA: an accumulator holds a finished chunk
+    const uint32_t tempty0 = tfull0 + 16;                 // [2] leader: both CTAs' epilogues are done with it
+    const uint32_t drain = tempty0 + 16;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P_STAGES + 5);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const uint32_t rank = tc::cluster_ctarank();
+    const bool leader = rank == 0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int nk = (int)((p.rows + BK - 1) / BK);
+    const int kcb = kchunk_blocks(p.d);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < P_STAGES; ++s) {
+            tc::mbar_init(full0 + 8 * s, 1);
+            tc::mbar_init(empty0 + 8 * s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            tc::mbar_init(tfull0 + 8 * a, 1);
+            tc::mbar_init(tempty0 + 8 * a, 8);   // one arrival per epilogue warp of either CTA
+        }
+        tc::mbar_init(drain, 1);
+        *abort_flag = 0;
+        tc::fence_barrier_init();
+        tc::prefetch_tmap(&tmX);
+        tc::prefetch_tmap(&tmS);
+    }
+    if (warp == 1) tc::tmem_alloc_pair(tc::smem_u32(tmem_slot), 512);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::cluster_sync();   // both CTAs' barriers exist before any copy or arrival reaches them
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint32_t full_leader = tc::mapa_shared(full0, 0);
+            int it = 0;
+            bool ok = true;
+            for (int w = pair; w < p.total_tiles && ok; w += npairs) {
+                int R, C;
+                decode_pair_tile(w, R, C, p.nc);
+                const int ra = R * P_TILE + (int)rank * P_HALF, cb = C * P_TILE + (int)rank * P_HALF;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % P_STAGES;
+                    const uint32_t ph = (it / P_STAGES) & 1;
+                    if (!tc::mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort_flag)) { ok = false; break; }
+                    if (leader) tc::mbar_arrive_expect_tx(full0 + 8 * s, 2 * P_STAGE_BYTES);
+                    const uint32_t fb = full_leader + 8 * s;
+                    const uint32_t a_dst = tc::smem_u32(smem + s * P_STAGE_BYTES);
+                    const uint32_t b_dst = a_dst + P_A_BYTES;
+                    const int y = kb * BK;
+#pragma unroll
+                    for (int h = 0; h < P_HALF / 64; ++h) tc::tma_load_2d_pair(a_dst + h * 8192, &tmX, fb, ra + h * 64, y);
+#pragma unroll
+                    for (int h = 0; h < P_HALF / 64; ++h) tc::tma_load_2d_pair(b_dst + h * 8192, &tmX, fb, cb + h * 64, y);
+                }
+            }
+            if (!ok && leader) {  // the copies already issued (both CTAs') land before either CTA can exit
+                for (int j = it - 1; j >= 0 && j >= it - P_STAGES; --j)
+                    tc::mbar_wait_bounded(full0 + 8 * (j % P_STAGES), (j / P_STAGES) & 1, abort_flag, 100000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            int it = 0, tcount = 0;
+            bool ok = true;
+            for (int w = pair; w < p.total_tiles && ok; w += npairs) {
+                for (int kc = 0; kc < nk && ok; kc += kcb) {
+                    const int kend = min(nk, kc + kcb);
+                    const int acc = tcount & 1;
+                    const uint32_t aph = (tcount >> 1) & 1;
+                    if (!tc::mbar_wait_bounded(tempty0 + 8 * acc, aph ^ 1, abort_flag)) { ok = false; break; }
+                    tc::fence_after_sync();
+                    const uint32_t d_tmem = tmem + acc * P_TILE;
+                    for (int kb = kc; kb < kend; ++kb, ++it) {
+                        const int s = it % P_STAGES;
+                        const uint32_t ph = (it / P_STAGES) & 1;
+                        if (!tc::mbar_wait_bounded(full0 + 8 * s, ph, abort_flag)) { ok = false; break; }
+                        tc::fence_after_sync();
+                        const uint32_t a_base = tc::smem_u32(smem + s * P_STAGE_BYTES);
+                        const uint32_t b_base = a_base + P_A_BYTES;
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint64_t ad = tc::sw128_desc(a_base + kk * 2048, 8192, 1024);
+                            const uint64_t bd = tc::sw128_desc(b_base + kk * 2048, 8192, 1024);
+                            tc::mma_f16_pair(d_tmem, ad, bd, IDESC_PAIR, ((kb - kc) | kk) != 0);
+                        }
+                        tc::mma_commit_pair(empty0 + 8 * s, 0x3);
+                    }
+                    if (!ok) break;
+                    tc::mma_commit_pair(tfull0 + 8 * acc, 0x3);
+                    ++tcount;
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        const uint32_t stg = tc::smem_u32(smem + P_STG_OFF) + q * 8192;
+        const uint32_t tempty_leader = tc::mapa_shared(tempty0, 0);
+        int sb = 0;
+        int tcount = 0;
+        for (int w = pair; w < p.total_tiles; w += npairs) {
+            int R, C;
+            decode_pair_tile(w, R, C, p.nc);
+            const int warp_row_min = R * P_TILE + (int)rank * P_HALF + q * 32;
+            bool ok = true;
+            for (int kc = 0; kc < nk; kc += kcb) {
+                const int acc = tcount & 1;
+                const uint32_t aph = (tcount >> 1) & 1;
+                if (!tc::mbar_wait_bounded(tfull0 + 8 * acc, aph, abort_flag)) { ok = false; break; }
+                tc::fence_after_sync();
+#pragma unroll 1
+                for (int ch = 0; ch < P_TILE / 32 && warp_row_min < p.d; ++ch) {
+                    const int col0 = C * P_TILE + ch * 32;
+                    if (col0 >= p.d) break;
+                    if (col0 + 31 < warp_row_min) continue;  // whole sub-tile strictly below the diagonal
+                    uint32_t v[32];
+                    tc::tmem_ld_32x32b_x32(tmem + acc * P_TILE + ch * 32 + ((uint32_t)(q * 32) << 16), v);
+                    tc::tmem_wait_ld();
+                    const uint32_t buf = stg + sb * 4096;
+                    if (lane == 0) tc::bulk_wait_read<1>();  // the reduce that last used buf has read it
+                    __syncwarp();
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                     ::"r"(buf + lane * 128 + ((j ^ (lane & 7)) << 4)), "r"(v[4 * j]),
+                                     "r"(v[4 * j + 1]), "r"(v[4 * j + 2]), "r"(v[4 * j + 3]) : "memory");
+                    tc::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tc::tma_reduce_add_2d(&tmS, buf, col0, warp_row_min);
+                        tc::bulk_commit();
+                    }
+                    sb ^= 1;
+                }
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive_cluster(tempty_leader + 8 * acc);
+                ++tcount;
+            }
+            if (!ok) break;
+        }
+        if (lane == 0) tc::bulk_wait_all();
+        __syncwarp();
+    }
+
+    __syncthreads();
+    if (warp == 1 && leader) {
+        if (lane == 0) {
+            tc::mma_commit_pair(drain, 0x1);
+            tc::mbar_wait_bounded(drain, 0, abort_flag, 100000000ull);
+        }
+        __syncwarp();
+    }
+    tc::fence_before_sync();
+    tc::cluster_sync();   // the leader's last products (which read both CTAs' shared memory) are done
+    tc::fence_after_sync();
+    if (warp == 1) tc::tmem_dealloc_pair(tmem, 512);
+    if (threadIdx.x == 0 && *abort_flag) clha_record_error(p.err, CLHA_ERR_TIMEOUT, blockIdx.x, 0, KID_COLLECT);
+}
+
 __global__ void add_counts(int64_t* counts, const int64_t* seg, int E, int64_t rows) {
     int e = blockIdx.x * blockDim.x + threadIdx.x;
     if (e < E) counts[e] += seg ? seg[E + 1 + e] : rows;
@@ -370,15 +583,50 @@ cudaError_t launch_collect_bf16(cudaStream_t s, int num_sms, const __nv_bfloat16
     p.seg = seg;
     p.E = E;
     p.S = S_base;
-    p.nr = d / BM;
-    p.nc = (d + BN - 1) / BN;
-    p.tiles_per_slot = 0;
-    for (int c = 0; c < p.nc; ++c) p.tiles_per_slot += (p.nr < 2 * c + 2) ? p.nr : 2 * c + 2;
-    p.total_tiles = p.tiles_per_slot * E;
     p.err = err;
-    int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
-    syrk_bf16_tc<false><<<grid, kThreads, SMEM_BYTES, s>>>(tm, tmS, p);
-    clha_note_launches(1);
+    if (!seg && E == 1 && d >= kPairMinD) {   // one dense Gram at large d: pairs of SMs
+        static bool pair_attr_set = false;
+        if (!pair_attr_set) {
+            e = cudaFuncSetAttribute(syrk_bf16_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+            pair_attr_set = true;
+        }
+        const int nC = (d + P_TILE - 1) / P_TILE;
+        p.nr = p.nc = nC;
+        p.tiles_per_slot = p.total_tiles = nC * (nC + 1) / 2;
+        int npairs = num_sms / 2;
+        if (npairs > p.total_tiles) npairs = p.total_tiles;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(2 * npairs));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = P_SMEM_BYTES;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int max_clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&max_clusters, syrk_bf16_pair, &cfg) == cudaSuccess && max_clusters > 0 &&
+            max_clusters < npairs) {
+            npairs = max_clusters;
+            cfg.gridDim = dim3((unsigned)(2 * npairs));
+        }
+        e = cudaLaunchKernelEx(&cfg, syrk_bf16_pair, tm, tmS, p);
+        if (e != cudaSuccess) return e;
+        clha_note_launches(1);
+    } else {
+        p.nr = d / BM;
+        p.nc = (d + BN - 1) / BN;
+        p.tiles_per_slot = 0;
+        for (int c = 0; c < p.nc; ++c) p.tiles_per_slot += (p.nr < 2 * c + 2) ? p.nr : 2 * c + 2;
+        p.total_tiles = p.tiles_per_slot * E;
+        int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
+        syrk_bf16_tc<false><<<grid, kThreads, SMEM_BYTES, s>>>(tm, tmS, p);
+        clha_note_launches(1);
+    }
     add_counts<<<(E + 255) / 256, 256, 0, s>>>(counts_base, seg, E, rows);
     clha_note_launches(1);
     return cudaGetLastError();

@@ -143,12 +143,14 @@ def test_collect_dense_bf16(ctx, n, d):
     assert torch.all(S[0] == 0)
 
 
-@pytest.mark.parametrize("n,d", [(1100, 8192), (700, 8320)])
+@pytest.mark.parametrize("n,d", [(1100, 8192), (700, 8320), (5000, 4096), (6000, 4224)])
 def test_collect_large_d(ctx, n, d):
-    """Channel counts of 8192 and up, where the chunk sums run over longer token ranges: a ragged token
-    count, and d = 8320 (an odd number of 128-channel tiles, so the last tile column holds one
-    diagonal tile only). The Gram equals the float64 one; a second call into another layer of the
-    same accumulator, over a token range that starts mid-block, accumulates there and leaves the first
+    """One dense Gram at d >= 4096 runs on pairs of SMs (256 x 256 tiles, one tcgen05.mma over both
+    CTAs' shared memory). Ragged token counts; 2048-token chunks below d = 8192 (5000 tokens: three
+    chunks per tile) and 8192-token ones above; d = 8320 and 4224 are not multiples of 256, so the
+    last tile's second row half lies past the matrix (computed on zero-filled operands, never
+    written). The Gram equals the float64 one; a second call into another layer of the same
+    accumulator, over a token range that starts mid-block, accumulates there and leaves the first
     layer alone."""
     g = _gen(n + d)
     X = (torch.randn((n, d), generator=g) * (1 + torch.rand(d, generator=g))).to(torch.bfloat16).to(DEV)
