@@ -897,7 +897,10 @@ def run_kernel(args):
         for _ in range(args.warmup):
             fn()
         torch.cuda.synchronize()
+        clocks = ClockSampler(0)
+        clocks.start()
         evs = []
+        t_begin = time.time()
         for _ in range(args.steps):   # L2 flushed before every timed launch, each launch timed alone
             flush.zero_()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -906,6 +909,8 @@ def run_kernel(args):
             b.record(ctx.stream)
             evs.append((a, b))
         torch.cuda.synchronize()
+        clocks.mark(t_begin, time.time())
+        clk = clocks.stop()
         L.clha_check(ctx)
         if args.workload == "act" and L.clha_last_act_kernel(ctx) == L.ACT_TENSOR:   # the kernel that ran
             bound, peak, kname = "tensor", peaks["bf16_tflops"], "expert_act_tc (tcgen05 kind::f16)"
@@ -916,7 +921,7 @@ def run_kernel(args):
                           "peak_source": (src if bound == "tensor" and args.workload != "gptq" else
                                           "derived (measured bf16 x nominal tf32/bf16, / 3)" if bound == "tensor" else
                                           "derived (SM count x lanes x max clock)"),
-                          "l2": "flushed (512 MB write) before every timed launch"}))
+                          "l2": "flushed (512 MB write) before every timed launch", "clocks": clk}))
         torch.cuda.empty_cache()
     ctx.close()
     return 0
