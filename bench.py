@@ -513,6 +513,7 @@ def run_ours(args, world, rank, local):
                        "parallelism": (f"tokens{world}+experts{world} (NCCL reduce-scatter of packed S triangles to owners)" if sharded
                                        else f"replicas{world}") if world > 1 else "single",
                        "l2": "flushed (512 MB write) before every timed step"},
+            "weights_per_s": value * 3 * E / cal.columns(),   # matrices (gate, up, down: 3E per cal.columns())
             "hessian_tflops": hess_tflops,
             "hessian_frac_of_bf16_peak": hess_tflops / sustained,
             "roofline": {"kernel": kname, "phase": dom, "bound": bound, "achieved": achieved, "peak": peak,
@@ -734,6 +735,7 @@ def run_dense(args, world, rank, local):
                        "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (15 GB of X read per step) and a 512 MB flush write "
                              "before every timed step"},
+            "weights_per_s": value / d,   # one weight [d_out, d] per step per GPU
             "hessian_tflops": hess_tflops,
             "hessian_frac_of_bf16_peak": hess_tflops / sustained,
             "hessian_peak": "bf16 sustained (the step lasts about a second)",
