@@ -261,14 +261,18 @@ def blas_threads():
 
 
 # ------------------------------------------------------------------------------------------ workload
-def make_inputs(rank: int):
+MOE_CONFIGS = {"moe-e16": 2, "moe-e64": 3}   # the E16 top-2 pair; the E64 top-6 pair with 2 always-active experts
+
+
+def make_inputs(rank: int, cfg: int = 2):
     from synth import workload
-    wl = workload(2, "cpu", seed=rank_seed(rank))
+    wl = workload(cfg, "cpu", seed=rank_seed(rank))
     s = wl.spec
     X = [wl.x(l) for l in range(2)]
     lg = [wl.logits(l) for l in range(2)]
     routed = [wl.expert_weights(0, e) for e in range(s.E)]
-    return wl, X, lg, routed
+    shared = [wl.expert_weights(0, i, shared=True) for i in range(s.n_shared)]
+    return wl, X, lg, routed, shared
 
 
 def oracle_sample(X, lg, routed, spec, expert: int):
@@ -279,7 +283,7 @@ def oracle_sample(X, lg, routed, spec, expert: int):
     L64 = [l.numpy() for l in lg]
     W64 = [tuple(t.double().numpy() for t in routed[expert])]
     cols = 0
-    for mode in ("rt", "eq"):
+    for mode in spec.alpha_modes:
         O.calibrate_moe_group(X64, L64, spec.k, [W64[0] if e == expert else None for e in range(spec.E)], (),
                               [expert], spec.bits_routed, spec.bits_shared, spec.group, mode, spec.damp_frac)
         cols += 2 * spec.d_model + spec.d_ff
@@ -289,7 +293,7 @@ def oracle_sample(X, lg, routed, spec, expert: int):
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
-    wl, X, lg, routed = make_inputs(0)
+    wl, X, lg, routed, _ = make_inputs(0, MOE_CONFIGS[args.workload])
     s = wl.spec
     for i in range(args.warmup):
         oracle_sample(X, lg, routed, s, i % s.E)
@@ -300,7 +304,8 @@ def run_reference(args, world, rank):
         times.append(time.perf_counter() - t0)
     ms = 1e3 * statistics.mean(times)
     value = cols / (ms / 1e3)
-    sample = "one routed expert per step (gate, up, down) through route, gather, Hessians, aggregate, factor, GPTQ and loss, both weightings"
+    sample = (f"one routed expert per step (gate, up, down) through route, gather, Hessians, aggregate, factor, "
+              f"GPTQ and loss, weightings {'/'.join(s.alpha_modes)}")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "columns/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -322,11 +327,12 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     sharded = args.parallel == "tokens"
     # replicas: every rank calibrates its own pair; tokens: one pair, tokens and experts split over ranks
-    wl, X, lg, routed = make_inputs(0 if sharded else rank)
+    wl, X, lg, routed, shared = make_inputs(0 if sharded else rank, MOE_CONFIGS[args.workload])
     s = wl.spec
+    ns, sdff = s.n_shared, s.shared_dff
     ctx = L.Context(local)
     timer = PhaseTimer(ctx.stream)
-    w = stack_weights((routed, []), dev)
+    w = stack_weights((routed, shared), dev)
     modes = s.alpha_modes
     if sharded:
         from post_quantization_expert_b200 import sharded as SH
@@ -338,7 +344,7 @@ def run_ours(args, world, rank, local):
         cal, qcal, wq = sh.collector, sh.quantizer, sh.local_weights(w)
         cols_per_step = cal.columns() * len(modes) / world      # the pair's columns, per rank on average
     else:
-        cal = qcal = MoECalibration(ctx, 2, max(s.tokens), s.E, s.k, s.d_model, s.d_ff, 0, 0, s.bits_routed,
+        cal = qcal = MoECalibration(ctx, 2, max(s.tokens), s.E, s.k, s.d_model, s.d_ff, ns, sdff, s.bits_routed,
                                     s.bits_shared, s.damp_frac, timer=timer, modes=modes,
                                     factor_form=FORMS[args.factor_form])
         wq = w
@@ -396,8 +402,11 @@ def run_ours(args, world, rank, local):
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
     pin = lambda t: t.pin_memory()
     hX, hL = [pin(x) for x in X], [pin(l) for l in lg]
-    hW = [pin(w.Wgu.cpu()), pin(w.Wd.cpu())]
+    hW = [pin(w.Wgu.cpu()), pin(w.Wd.cpu())] + ([pin(w.Sgu.cpu()), pin(w.Sd.cpu())] if ns else [])
     outs = {m: {"gu": qcal.res[m].qgu, "d": qcal.res[m].qd} for m in modes}
+    if ns:
+        for m in modes:
+            outs[m].update({"sgu": qcal.res[m].sgu, "sd": qcal.res[m].sd})
     hout = {m: {k: (pin(torch.empty_like(q.codes, device="cpu")), pin(torch.empty_like(q.scales, device="cpu")),
                     pin(torch.empty_like(q.zeros, device="cpu"))) for k, q in outs[m].items()} for m in modes}
     h2d = sum(t.numel() * t.element_size() for t in hX + hL + hW)
@@ -452,14 +461,22 @@ def run_ours(args, world, rank, local):
     counts = [cal.counts[l].cpu().numpy().astype(np.int64) for l in range(2)]
     dm, dff, E = s.d_model, s.d_ff, s.E
     hess_flops = sum(int(c.sum()) * (dm * (dm + 1) + dff * (dff + 1)) for c in counts)
+    act_flops = sum(int(c.sum()) * 4 * dm * dff for c in counts)
     Eq = (sh.e1 - sh.e0) if sharded else E                  # experts this rank quantizes
     mats = [(dff, dm)] * (2 * Eq) + [(dm, dff)] * Eq        # gate, up, down per weighting
+    factor_flops = len(modes) * Eq * (factor_work(dm, cal.form) + factor_work(dff, cal.form))
+    # per slot and weighting: both layers' upper triangles of S read, the damped aggregate written (full)
+    agg = lambda d: 2 * (d * (d + 1) // 2) * 4 + d * d * 4
+    agg_bytes = len(modes) * Eq * (agg(dm) + agg(dff))
+    if ns:   # always-active experts: every token, one shared input Gram, one down Gram each
+        for n_l in s.tokens[:2]:
+            hess_flops += n_l * (dm * (dm + 1) + ns * sdff * (sdff + 1))
+            act_flops += n_l * ns * 4 * dm * sdff
+        mats += [(sdff, dm)] * (2 * ns) + [(dm, sdff)] * ns
+        factor_flops += len(modes) * (factor_work(dm, cal.form) + ns * factor_work(sdff, cal.form))
+        agg_bytes += len(modes) * (agg(dm) + ns * agg(sdff))
     gptq_flops = len(modes) * sum(o * i * i for o, i in mats)
     loss_flops = len(modes) * sum(2 * o * i * i for o, i in mats)
-    factor_flops = len(modes) * Eq * (factor_work(dm, cal.form) + factor_work(dff, cal.form))
-    act_flops = sum(int(c.sum()) * 4 * dm * dff for c in counts)
-    # per slot and weighting: both layers' upper triangles of S read, the damped aggregate written (full)
-    agg_bytes = len(modes) * Eq * sum(2 * (d * (d + 1) // 2) * 4 + d * d * 4 for d in (dm, dff))
     peaks, src = load_peaks()
     alu = alu_peaks(peaks)
     sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
@@ -481,7 +498,7 @@ def run_ours(args, world, rank, local):
     dom = max((k for k in phase_ms if k in single), key=lambda k: phase_ms[k])
     bound, work, peak, unit, kname = kernels[dom]
     achieved = work / (phase_ms[dom] / 1e3)
-    step_bytes = measured_traffic(dom, "moe-E16")   # per step; reported per timed call like `achieved`
+    step_bytes = measured_traffic(dom, "moe-E16" if s.E == 16 else s.name)   # per step; per timed call
     traffic = step_bytes / phase_calls[dom] if step_bytes is not None and phase_calls.get(dom) else None
     phases = {k: {"ms": round(v, 4)} for k, v in sorted(phase_ms.items(), key=lambda kv: -kv[1])}
     for k, v in phases.items():
@@ -499,7 +516,8 @@ def run_ours(args, world, rank, local):
         c = oracle_sample(X, lg, routed, s, 0)
         dt = time.perf_counter() - t0
         cpu = {"value": c / dt, "unit": "columns/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"expert 0 of layer pair (gate, up, down; both weightings; {c} columns) in {dt:.1f} s"}
+               "sample": f"routed expert 0 of the layer pair (gate, up, down; weightings {'/'.join(modes)}; "
+                         f"{c} columns) in {dt:.1f} s"}
 
     if rank == 0:
         line = {
@@ -509,11 +527,12 @@ def run_ours(args, world, rank, local):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": s.name, "global_batch": world * sum(s.tokens), "tokens_per_layer": s.tokens[0],
                        "E": E, "top_k": s.k, "d_model": dm, "d_ff": dff, "bits": s.bits_routed,
+                       "always_active": ns, "always_active_d_ff": sdff, "always_active_bits": s.bits_shared if ns else None,
                        "weightings": list(modes), "columns_per_step_per_gpu": cols_per_step,
                        "parallelism": (f"tokens{world}+experts{world} (NCCL reduce-scatter of packed S triangles to owners)" if sharded
                                        else f"replicas{world}") if world > 1 else "single",
                        "l2": "flushed (512 MB write) before every timed step"},
-            "weights_per_s": value * 3 * E / cal.columns(),   # matrices (gate, up, down: 3E per cal.columns())
+            "weights_per_s": value * 3 * (E + ns) / cal.columns(),   # matrices: gate, up, down of every expert
             "hessian_tflops": hess_tflops,
             "hessian_frac_of_bf16_peak": hess_tflops / sustained,
             "roofline": {"kernel": kname, "phase": dom, "bound": bound, "achieved": achieved, "peak": peak,
@@ -940,7 +959,7 @@ def main():
                          "one pair, its tokens sharded over the ranks with one reduce-scatter of the packed Hessian sums to their owners, "
                          "its experts quantized in parallel (strong scaling)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
-    ap.add_argument("--workload", choices=("dense", "moe-e16", "act", "hessian", "gptq", "factor", "epmq", "dequant",
+    ap.add_argument("--workload", choices=("dense", "moe-e16", "moe-e64", "act", "hessian", "gptq", "factor", "epmq", "dequant",
                                            "sweep"),
                     default="dense",
                     help="dense: the end-to-end calibration step of the 8192x28672 weight shared by 4 layers "
@@ -956,7 +975,7 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.workload == "sweep":
         return run_sweep(args)
-    if args.workload not in ("dense", "moe-e16"):
+    if args.workload not in ("dense", "moe-e16", "moe-e64"):
         if not args.shape:
             ap.error("--shape is required for kernel workloads")
         return run_kernel(args)
