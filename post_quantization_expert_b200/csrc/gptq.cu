@@ -267,7 +267,7 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                 uint32_t spins = 0;
                 while (q < 3 || ks < nks) {
                     bool progressed = false;
-                    if (q < 3 && tc::mbar_try_wait(sreq, nq & 1) && tc::mbar_try_wait(sbfull, nq & 1)) {
+                    if (q < 3 && tc::mbar_test_wait(sreq, nq & 1) && tc::mbar_test_wait(sbfull, nq & 1)) {
                         tc::fence_after_sync();
                         const uint32_t sbh = (q & 1) ? sb1 : sb0;
                         const uint32_t sbl = sbh + ((q & 1) ? SB1_HALF : SB0_HALF);
@@ -297,9 +297,9 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                     }
                     // a lazy step only once the previous one has left the tensor pipe, so that a
                     // quarter product (which the row threads wait for) queues behind one step at most
-                    const bool pipe_clear = it == 0 || tc::mbar_try_wait(empty0 + 8 * ((it - 1) % STAGES), ((it - 1) / STAGES) & 1);
+                    const bool pipe_clear = it == 0 || tc::mbar_test_wait(empty0 + 8 * ((it - 1) % STAGES), ((it - 1) / STAGES) & 1);
                     if (lazy_ready && ks < nks && pipe_clear &&
-                        tc::mbar_try_wait(full0 + 8 * (it % STAGES), (it / STAGES) & 1)) {
+                        tc::mbar_test_wait(full0 + 8 * (it % STAGES), (it / STAGES) & 1)) {
                         tc::fence_after_sync();
                         const int s = it % STAGES;
                         const uint32_t ahi = tc::smem_u32(smem + s * STAGE_BYTES);
@@ -425,44 +425,9 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                 }
                 uint32_t codes[QW / 4];
                 quarter_sweep(w, s, z, maxq, uinv + QW * q, Uq[q], codes);
-                // outputs of this quarter: codes (32 B) and w_hat (128 B) of this row
-                uint4* cdst = reinterpret_cast<uint4*>(p.codes + orow + QW * q);
-                cdst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-                cdst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-                if (p.W_hat || p.loss) {
-                    float wo[QW];
-                    if (p.loss) load_w32(p, wrow + cb + QW * q, wo);
-#pragma unroll
-                    for (int c = 0; c < QW / 4; ++c) {
-                        float v[4];
-#pragma unroll
-                        for (int m = 0; m < 4; ++m)
-                            v[m] = __fmul_rn(s, __fsub_rn((float)((codes[c] >> (8 * m)) & 255u), z));
-                        if (p.W_hat)
-                            *reinterpret_cast<float4*>(p.W_hat + orow + QW * q + 4 * c) = make_float4(v[0], v[1], v[2], v[3]);
-                        if (p.loss) {
-#pragma unroll
-                            for (int m = 0; m < 4; ++m) {
-                                const double dv = (double)v[m] - (double)wo[4 * c + m];
-                                d2 = fma(dv, dv, d2);
-                            }
-                        }
-                    }
-                }
-                if (p.loss) {
-#pragma unroll
-                    for (int j = 0; j < QW; ++j) e2 = fma((double)w[j], (double)w[j], e2);
-                }
-                if (q == 3 && !more) break;
-                // the quarter's errors as tf32 hi/lo, row t, 16-byte piece c at c ^ (t % 8); the buffer
-                // is free once the last quarter's whole product and its store have read it
-                if (q > 0 && !tc::mbar_wait_bounded(sdone2, (nq - 1) & 1, abort_flag)) ok = false;
-                if (t == 0) tc::bulk_wait_read<0>();
-                row_bar();
-                if (q == 3 && next_here) load_uq(cb + BLK);   // every row is past its last use of Uq
                 uint8_t* sah = smem + SA_OFF + t * 128;
                 uint8_t* sal = sah + SA_BYTES;
-                auto put_row = [&](const float (&v)[QW]) {
+                auto put_row = [&](const float (&v)[QW]) {   // row t, 16-byte piece c at c ^ (t % 8)
 #pragma unroll
                     for (int c = 0; c < QW / 4; ++c) {
                         const float h0 = to_tf32(v[4 * c]), h1 = to_tf32(v[4 * c + 1]), h2 = to_tf32(v[4 * c + 2]),
@@ -475,19 +440,58 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                     }
                     fence_proxy_async_smem();
                 };
-                if (!p.blk || q < 3) {                   // e: the quarter product's operand
-                    put_row(w);
-                    if (q < 3) {
-                        tc::mbar_arrive(sreq);
-                        ++nq;
+                float wo[QW];                                // the original weights of the quarter (issued
+                if (p.loss || (p.blk && more)) load_w32(p, wrow + cb + QW * q, wo);   // before the handoff)
+                // first the quarter's errors as tf32 hi/lo into the shared buffer and the request for the
+                // quarter product, which gates the next quarter; the outputs below overlap that product.
+                // The buffer is free once the last quarter's whole product and its store have read it.
+                if (!(q == 3 && !more)) {
+                    if (q > 0 && !tc::mbar_wait_bounded(sdone2, (nq - 1) & 1, abort_flag)) ok = false;
+                    if (t == 0) tc::bulk_wait_read<0>();
+                    row_bar();
+                    if (q == 3 && next_here) load_uq(cb + BLK);   // every row is past its last use of Uq
+                    if (!p.blk || q < 3) {                   // e: the quarter product's operand
+                        put_row(w);
+                        if (q < 3) {
+                            tc::mbar_arrive(sreq);
+                            ++nq;
+                        }
                     }
+                }
+                // outputs of this quarter: codes (32 B) and w_hat (128 B) of this row, the loss terms
+                uint4* cdst = reinterpret_cast<uint4*>(p.codes + orow + QW * q);
+                cdst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                cdst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+                if (p.W_hat || p.loss) {
+                    double dq[4] = {0.0, 0.0, 0.0, 0.0};     // four independent chains: the fp64 FMA
+#pragma unroll                                              // latency, not its rate, bounds one chain
+                    for (int c = 0; c < QW / 4; ++c) {
+                        float v[4];
+#pragma unroll
+                        for (int m = 0; m < 4; ++m)
+                            v[m] = __fmul_rn(s, __fsub_rn((float)((codes[c] >> (8 * m)) & 255u), z));
+                        if (p.W_hat)
+                            *reinterpret_cast<float4*>(p.W_hat + orow + QW * q + 4 * c) = make_float4(v[0], v[1], v[2], v[3]);
+                        if (p.loss) {
+#pragma unroll
+                            for (int m = 0; m < 4; ++m) {
+                                const double dv = (double)v[m] - (double)wo[4 * c + m];
+                                dq[m] = fma(dv, dv, dq[m]);
+                            }
+                        }
+                    }
+                    d2 += (dq[0] + dq[1]) + (dq[2] + dq[3]);
+                }
+                if (p.loss) {
+                    double eq[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+                    for (int j = 0; j < QW; ++j) eq[j & 3] = fma((double)w[j], (double)w[j], eq[j & 3]);
+                    e2 += (eq[0] + eq[1]) + (eq[2] + eq[3]);
                 }
                 if (more && p.blk) {
                     // the later blocks' lazy operand under F: W_hat - W of the quarter (original W), written
                     // over e once the quarter product has read it (a second buffer does not fit in shared
                     // memory; stores straight from registers to global memory measured slower)
-                    float wo[QW];
-                    load_w32(p, wrow + cb + QW * q, wo);
 #pragma unroll
                     for (int c = 0; c < QW / 4; ++c)
 #pragma unroll
