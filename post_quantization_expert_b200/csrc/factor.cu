@@ -587,11 +587,17 @@ __device__ __forceinline__ void decode_task(const Dag& g, const unsigned long lo
             i = m + 2 + (int)local;
             j = m + 2;
         } else {
+            // FG(i, j) for m+2 <= j <= i < nt, column after column (nt - j tasks in column j): the
+            // column k = j - (m+2) is the largest with cum(k) = k R2 - k(k-1)/2 <= local, R2 = nt - m - 2,
+            // the smaller root of a quadratic, then a unit step either way for the rounding of the root
             q = 6;
-            int rem = (int)local;
-            j = m + 2;
-            while (rem >= nt - j) { rem -= nt - j; ++j; }
-            i = j + rem;
+            const long long R2 = nt - m - 2, B = 2 * R2 + 1, lc = (long long)local;
+            long long k = (long long)((double)B - sqrt((double)(B * B - 8 * lc))) / 2;
+            auto cum = [&](long long kk) { return kk * R2 - kk * (kk - 1) / 2; };
+            while (k > 0 && cum(k) > lc) --k;
+            while (cum(k + 1) <= lc) ++k;
+            j = m + 2 + (int)k;
+            i = j + (int)(lc - cum(k));
         }
     } else { q = 1; m = sg; i = m + 1 + (int)local; j = m; }
     d.q = q; d.k = k; d.b = b; d.m = m; d.i = i; d.j = j;

@@ -16,6 +16,7 @@ and checks:
 The same checks run on the Cholesky-only graph of the block-scaled factor F (classes F, Q and FQ
 empty): L final, no Y tile beyond the diagonal tasks' touched.
 """
+import math
 import random
 
 import pytest
@@ -69,11 +70,17 @@ def decode(nt, s, c, local):
     if c == 5:
         if m % 2 == 0:
             return ("G", m, m + 2 + local, m + 2)
-        rem, j = local, m + 2
-        while rem >= nt - j:
-            rem -= nt - j
-            j += 1
-        return ("FG", m, j + rem, j)
+        # the kernel's closed form: column k = j - (m+2), the smaller root of the triangular count
+        R2 = nt - m - 2
+        B = 2 * R2 + 1
+        k = int((B - math.sqrt(float(B * B - 8 * local))) // 2)
+        cum = lambda kk: kk * R2 - kk * (kk - 1) // 2
+        while k > 0 and cum(k) > local:
+            k -= 1
+        while cum(k + 1) <= local:
+            k += 1
+        j = m + 2 + k
+        return ("FG", m, j + local - cum(k), j)
     return ("S", s, s + 1 + local, s)
 
 
@@ -126,6 +133,28 @@ def test_numbering_is_topological_and_complete(nt, inv):
                 assert state[("Y", j, i)] == i - j + 1
             else:
                 assert state.get(("Y", j, i), 0) == (1 if i == j else 0)
+
+
+def _fg_by_walk(nt, m, local):
+    """The bulk task's tiles by walking the columns (the plain definition of the numbering)."""
+    rem, j = local, m + 2
+    while rem >= nt - j:
+        rem -= nt - j
+        j += 1
+    return j + rem, j
+
+
+@pytest.mark.parametrize("nt", [3, 4, 17, 64, 224, 448, 1000])
+def test_bulk_task_closed_form_decode(nt):
+    """The closed-form decode of a two-level bulk task (a quadratic's root and a unit correction) gives
+    the tiles that walking the columns gives, for every task of small graphs and a sample of large ones."""
+    for m in range(1, nt, 2):
+        R = nt - 1 - m
+        n = (R - 1) * R // 2 if R >= 1 else 0
+        step = max(1, n // 2000)
+        for local in list(range(0, n, step)) + ([n - 1] if n else []):
+            _, _, i, j = decode(nt, m + 1, 5, local)
+            assert (i, j) == _fg_by_walk(nt, m, local), (nt, m, local)
 
 
 @pytest.mark.parametrize("nt", [1, 2, 5, 16, 128])
