@@ -52,7 +52,7 @@ sys.path.insert(0, ROOT)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 N_SMS = 148
 METRIC = "expert weight columns quantized/sec (CLHA-GPTQ end to end)"
-DENSE_CPU_CHANNELS = 2048     # the oracle's bounded sample of the dense workload: this principal block
+DENSE_CPU_CHANNELS = 2560     # the oracle's bounded sample of the dense workload: this principal block
 
 
 def load_peaks():
