@@ -8,8 +8,10 @@
  *   (1) collection  — per layer and per active expert, a Hessian and a token count
  *                     (clha_route_topk, clha_gather, clha_expert_act, clha_collect);
  *   (2) aggregation — H_comb = sum_i alpha_i H_i with routing-frequency or equal weights (clha_aggregate);
- *   (3) quantization — standard GPTQ column-sequential updates with H_comb (clha_factor, clha_quantize),
- *                     scored by the loss of section 2.1 (clha_loss).
+ *   (3) quantization — standard GPTQ column-sequential updates with H_comb (clha_factor_groups_as,
+ *                     clha_quantize_as; GPTQ's factor either U with H^-1 = U^T U, as the paper states
+ *                     it, or the block-scaled Cholesky factor of H itself, which gives the same
+ *                     updates at half the factor's work), scored by the loss of section 2.1 (clha_loss).
  * GPTQ is the algorithm of Frantar et al. (2022), "GPTQ: Accurate Post-Training Quantization for
  * Generative Pre-trained Transformers", Algorithm 1.
  *
