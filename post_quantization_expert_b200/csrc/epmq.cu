@@ -119,12 +119,9 @@ __global__ void __launch_bounds__(256) epmq_gemm(GemmArgs g) {
 constexpr int SMEM = 2 * TILE_DOUBLES * sizeof(double);
 
 cudaError_t run(cudaStream_t s, const GemmArgs& g, int M, int N) {
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(epmq_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    // per call: the attribute belongs to the current device's context (a process may drive several)
+    cudaError_t e = cudaFuncSetAttribute(epmq_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    if (e != cudaSuccess) return e;
     epmq_gemm<<<dim3(N / NB, M / NB), 256, SMEM, s>>>(g);
     clha_note_launches(1);
     return cudaGetLastError();

@@ -305,12 +305,10 @@ cudaError_t launch_expert_act(cudaStream_t s, int num_sms, const __nv_bfloat16* 
                               const int32_t* perm, const int64_t* seg, int E, const __nv_bfloat16* Wg,
                               const __nv_bfloat16* Wu, int d_ff, __nv_bfloat16* h, int policy, void* ws, int* sel,
                               int* err) {
-    static bool attr_set = false;
-    if (!attr_set) {
+    {   // per call: the attribute belongs to the current device's context (a process may drive several)
         cudaError_t e = cudaFuncSetAttribute(expert_act_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)sizeof(ActSmem));
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     const bool simt_only = perm || policy == 1;
     const int* sel_dev = nullptr;

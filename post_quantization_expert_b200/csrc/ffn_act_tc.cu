@@ -277,13 +277,10 @@ cudaError_t launch_expert_act_tc(cudaStream_t s, int num_sms, const __nv_bfloat1
         return e;
     if ((e = make_tmap_2d(&tUm, Wum ? Wum : Wu, (uint64_t)E * d_ff, (uint64_t)d_model, 2, BNH, BK)) != cudaSuccess)
         return e;
-    static bool attr_set = false;
-    if (!attr_set) {
-        if ((e = cudaFuncSetAttribute(expert_act_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
-            cudaSuccess)
-            return e;
-        attr_set = true;
-    }
+    // per call: the attribute belongs to the current device's context (a process may drive several)
+    if ((e = cudaFuncSetAttribute(expert_act_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
+        cudaSuccess)
+        return e;
     ActParams p{sel, rows, d_model, d_ff, seg, E, h, d_ff / BNH, out_n, xo, wo, err};
     expert_act_tc<<<num_sms, kThreads, SMEM_BYTES, s>>>(tX, tG, tU, tGm, tUm, p);
     clha_note_launches(1);

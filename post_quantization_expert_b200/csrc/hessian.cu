@@ -570,12 +570,9 @@ cudaError_t launch_collect_bf16(cudaStream_t s, int num_sms, const __nv_bfloat16
     if (e != cudaSuccess) return e;
     e = make_tmap_2d(&tmS, S_base, (uint64_t)E * d, (uint64_t)d, 4, 32, 32);
     if (e != cudaSuccess) return e;
-    static bool attr_set = false;
-    if (!attr_set) {
-        e = cudaFuncSetAttribute(syrk_bf16_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    // per call: the attribute belongs to the current device's context (a process may drive several)
+    e = cudaFuncSetAttribute(syrk_bf16_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
     SyrkParams p;
     p.d = d;
     p.rows = rows;
@@ -585,12 +582,8 @@ cudaError_t launch_collect_bf16(cudaStream_t s, int num_sms, const __nv_bfloat16
     p.S = S_base;
     p.err = err;
     if (!seg && E == 1 && d >= kPairMinD) {   // one dense Gram at large d: pairs of SMs
-        static bool pair_attr_set = false;
-        if (!pair_attr_set) {
-            e = cudaFuncSetAttribute(syrk_bf16_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
-            if (e != cudaSuccess) return e;
-            pair_attr_set = true;
-        }
+        e = cudaFuncSetAttribute(syrk_bf16_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
+        if (e != cudaSuccess) return e;
         const int nC = (d + P_TILE - 1) / P_TILE;
         p.nr = p.nc = nC;
         p.tiles_per_slot = p.total_tiles = nC * (nC + 1) / 2;
@@ -640,12 +633,8 @@ cudaError_t launch_collect_bf16_gathered(cudaStream_t s, int num_sms, const __nv
     if (e != cudaSuccess) return e;
     e = make_tmap_2d(&tmS, S_base, (uint64_t)E * d, (uint64_t)d, 4, 32, 32);
     if (e != cudaSuccess) return e;
-    static bool attr_set = false;
-    if (!attr_set) {
-        e = cudaFuncSetAttribute(syrk_bf16_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    e = cudaFuncSetAttribute(syrk_bf16_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
     SyrkParams p;
     p.d = d;
     p.rows = n;
