@@ -19,8 +19,9 @@
 //              of the quarter's product and the source of a TMA store of E to global memory (read
 //              by the later blocks' lazy updates).
 //   warp 4     TMA producer of the lazy update: E[:, :cb] (hi, lo) and the U panel U[:cb, blk] (hi,
-//              lo, from a transposed copy so both operands are K-major) in 32-wide k steps; the last
-//              128 k (the errors of the block being swept) only after they are stored.
+//              lo, from a transposed copy so both operands are K-major) in 32-wide k steps; each of
+//              the last four (the quarters of the block being swept) once that quarter is stored, so
+//              that only the last quarter's step is left when the block ends.
 //   warp 5     MMA issuer: the quarter products as soon as they are requested (the next quarter's
 //              columns first, with their own completion signal, since they gate the row threads;
 //              then the rest), between them the next block's lazy update (one step in the tensor
@@ -168,13 +169,13 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
     const uint32_t empty0 = full0 + 8 * STAGES;
     const uint32_t tfull0 = empty0 + 8 * STAGES;   // lazy update of a block complete (per accumulator)
     const uint32_t tempty0 = tfull0 + 16;          // row threads done with an accumulator
-    const uint32_t eready = tempty0 + 16;          // a block's errors are in global memory
-    const uint32_t sreq = eready + 8;              // a quarter's errors are in shared memory
+    const uint32_t qready0 = tempty0 + 16;         // [4] quarter q of a block: its errors are in global memory
+    const uint32_t sreq = qready0 + 32;            // a quarter's errors are in shared memory
     const uint32_t sbfull = sreq + 8;              // the quarter product's U rows are in shared memory
     const uint32_t sdone = sbfull + 8;             // the quarter product's next-quarter columns are done
     const uint32_t sdone2 = sdone + 8;             // the whole quarter product is done (buffers free)
     const uint32_t drain = sdone2 + 8;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + BAR_OFF + 8 * (2 * STAGES + 10));
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + BAR_OFF + 8 * (2 * STAGES + 13));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     const uint32_t sa_hi = tc::smem_u32(smem + SA_OFF), sa_lo = sa_hi + SA_BYTES;
     const uint32_t sb0 = tc::smem_u32(smem + SB0_OFF), sb1 = tc::smem_u32(smem + SB1_OFF);
@@ -195,7 +196,7 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
             tc::mbar_init(tfull0 + 8 * a, 1);
             tc::mbar_init(tempty0 + 8 * a, R);
         }
-        tc::mbar_init(eready, 1);
+        for (int qq = 0; qq < 4; ++qq) tc::mbar_init(qready0 + 8 * qq, 1);
         tc::mbar_init(sreq, R);
         tc::mbar_init(sbfull, 1);
         tc::mbar_init(sdone, 1);
@@ -223,8 +224,10 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                 const int cb = bb * BLK;
                 for (int ks = p.c0 / KS; ks < cb / KS; ++ks) {   // the chunk's earlier errors only
                     const int k0 = ks * KS;
-                    if (k0 == cb - BLK) {   // errors of the previous block: wait until they are stored
-                        if (!tc::mbar_wait_bounded(eready, (bb - 1 - b_lo) & 1, abort_flag)) { ok = false; break; }
+                    if (k0 >= cb - BLK) {   // the previous block's errors: each quarter once it is stored, so
+                                            // that only the last quarter's step remains at the block's end
+                        const int qi = (k0 - (cb - BLK)) / KS;
+                        if (!tc::mbar_wait_bounded(qready0 + 8 * qi, (bb - 1 - b_lo) & 1, abort_flag)) { ok = false; break; }
                     }
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
@@ -447,7 +450,15 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                 // The buffer is free once the last quarter's whole product and its store have read it.
                 if (!(q == 3 && !more)) {
                     if (q > 0 && !tc::mbar_wait_bounded(sdone2, (nq - 1) & 1, abort_flag)) ok = false;
-                    if (t == 0) tc::bulk_wait_read<0>();
+                    if (t == 0) {
+                        if (q > 0 && more) {                 // the previous quarter's store is complete: its
+                            tc::bulk_wait_all();             // errors may feed the next block's lazy update
+                            fence_proxy_async_global();
+                            tc::mbar_arrive(qready0 + 8 * (q - 1));
+                        } else {
+                            tc::bulk_wait_read<0>();
+                        }
+                    }
                     row_bar();
                     if (q == 3 && next_here) load_uq(cb + BLK);   // every row is past its last use of Uq
                     if (!p.blk || q < 3) {                   // e: the quarter product's operand
@@ -510,7 +521,7 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                         if (q == 3) {
                             tc::bulk_wait_all();
                             fence_proxy_async_global();
-                            tc::mbar_arrive(eready);
+                            tc::mbar_arrive(qready0 + 24);
                         }
                     }
                 }
