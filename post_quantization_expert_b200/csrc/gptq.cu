@@ -171,11 +171,12 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
     const uint32_t tempty0 = tfull0 + 16;          // row threads done with an accumulator
     const uint32_t qready0 = tempty0 + 16;         // [4] quarter q of a block: its errors are in global memory
     const uint32_t sreq = qready0 + 32;            // a quarter's errors are in shared memory
-    const uint32_t sbfull = sreq + 8;              // the quarter product's U rows are in shared memory
-    const uint32_t sdone = sbfull + 8;             // the quarter product's next-quarter columns are done
+    const uint32_t sbfull0 = sreq + 8;             // U rows of quarter 0 or 2's product in buffer 0 (twice a block)
+    const uint32_t sbfull1 = sbfull0 + 8;          // U rows of quarter 1's product in buffer 1 (once a block)
+    const uint32_t sdone = sbfull1 + 8;            // the quarter product's next-quarter columns are done
     const uint32_t sdone2 = sdone + 8;             // the whole quarter product is done (buffers free)
     const uint32_t drain = sdone2 + 8;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + BAR_OFF + 8 * (2 * STAGES + 13));
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + BAR_OFF + 8 * (2 * STAGES + 14));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     const uint32_t sa_hi = tc::smem_u32(smem + SA_OFF), sa_lo = sa_hi + SA_BYTES;
     const uint32_t sb0 = tc::smem_u32(smem + SB0_OFF), sb1 = tc::smem_u32(smem + SB1_OFF);
@@ -198,7 +199,8 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
         }
         for (int qq = 0; qq < 4; ++qq) tc::mbar_init(qready0 + 8 * qq, 1);
         tc::mbar_init(sreq, R);
-        tc::mbar_init(sbfull, 1);
+        tc::mbar_init(sbfull0, 1);
+        tc::mbar_init(sbfull1, 1);
         tc::mbar_init(sdone, 1);
         tc::mbar_init(sdone2, 1);
         tc::mbar_init(drain, 1);
@@ -270,7 +272,9 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                 uint32_t spins = 0;
                 while (q < 3 || ks < nks) {
                     bool progressed = false;
-                    if (q < 3 && tc::mbar_test_wait(sreq, nq & 1) && tc::mbar_test_wait(sbfull, nq & 1)) {
+                    const uint32_t sbf = (q & 1) ? sbfull1 : sbfull0;   // phases: 2 per block for buffer 0
+                    const uint32_t sbp = (q & 1) ? (uint32_t)(lb & 1) : (uint32_t)((q >> 1) & 1);
+                    if (q < 3 && tc::mbar_test_wait(sreq, nq & 1) && tc::mbar_test_wait(sbf, sbp)) {
                         tc::fence_after_sync();
                         const uint32_t sbh = (q & 1) ? sb1 : sb0;
                         const uint32_t sbl = sbh + ((q & 1) ? SB1_HALF : SB0_HALF);
@@ -353,11 +357,12 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
             const int nbox = 3 - q;
             const uint32_t sbh = (q & 1) ? sb1 : sb0;
             const uint32_t sbl = sbh + ((q & 1) ? SB1_HALF : SB0_HALF);
-            tc::mbar_arrive_expect_tx(sbfull, (uint32_t)(2 * nbox * 32 * QW * 4));
+            const uint32_t sbf = (q & 1) ? sbfull1 : sbfull0;
+            tc::mbar_arrive_expect_tx(sbf, (uint32_t)(2 * nbox * 32 * QW * 4));
             for (int bx = 0; bx < nbox; ++bx) {
                 const int n0 = u * p.d_in + cb + QW * (q + 1) + 32 * bx;
-                tc::tma_load_2d(sbh + bx * 4096, &tmQhi, sbfull, cb + QW * q, n0);
-                tc::tma_load_2d(sbl + bx * 4096, &tmQlo, sbfull, cb + QW * q, n0);
+                tc::tma_load_2d(sbh + bx * 4096, &tmQhi, sbf, cb + QW * q, n0);
+                tc::tma_load_2d(sbl + bx * 4096, &tmQlo, sbf, cb + QW * q, n0);
             }
         };
         auto load_uq = [&](int cb) {          // the block's four diagonal 32x32 blocks of U
@@ -379,7 +384,11 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
             const bool next_here = bb + 1 < b_hi;        // the next block is this launch's
             const size_t orow = ((size_t)b * p.d_out + row) * p.d_in + cb;   // this row's outputs
             row_bar();                                   // the last block's readers of Uq are done
-            if (t == 0) load_sb(cb, 0);
+            bool sb2_sent = false;                       // quarter 2's U rows (buffer 0, after quarter 0's product)
+            if (t == 0) {                                // both buffers are free: the last block's products are done
+                load_sb(cb, 0);
+                load_sb(cb, 1);
+            }
             cp_async_wait_all();                         // this block's Uq (issued during the last block)
             uinv[t] = 1.0f / __ldg(Ub + (size_t)(cb + t) * p.d_in + cb + t);
             if (lb > 0) {
@@ -413,7 +422,6 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                 if (q > 0) {                             // the previous quarter's product reached this quarter
                     if (!tc::mbar_wait_bounded(sdone, (nq - 1) & 1, abort_flag)) ok = false;
                     tc::fence_after_sync();
-                    if (t == 0 && q < 3) load_sb(cb, q);
                 }
                 if (lb > 0 || q > 0) {
                     uint32_t v[32];
@@ -450,6 +458,10 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                 // The buffer is free once the last quarter's whole product and its store have read it.
                 if (!(q == 3 && !more)) {
                     if (q > 0 && !tc::mbar_wait_bounded(sdone2, (nq - 1) & 1, abort_flag)) ok = false;
+                    if (q == 1 && t == 0 && !sb2_sent) {     // quarter 0's product is done with buffer 0
+                        load_sb(cb, 2);
+                        sb2_sent = true;
+                    }
                     if (t == 0) {
                         if (q > 0 && more) {                 // the previous quarter's store is complete: its
                             tc::bulk_wait_all();             // errors may feed the next block's lazy update
@@ -510,6 +522,10 @@ gptq_tc(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUten
                             w[4 * c + m] = __fsub_rn(__fmul_rn(s, __fsub_rn((float)((codes[c] >> (8 * m)) & 255u), z)),
                                                      wo[4 * c + m]);
                     if (q < 3 && !tc::mbar_wait_bounded(sdone2, (nq - 1) & 1, abort_flag)) ok = false;
+                    if (q == 0 && t == 0) {                  // quarter 0's product is done with buffer 0
+                        load_sb(cb, 2);
+                        sb2_sent = true;
+                    }
                     put_row(w);
                 }
                 if (more) {
